@@ -1,0 +1,350 @@
+#!/usr/bin/env python3
+"""Benchmark of the MXFP4 routed-expert MoE layer on B200.
+
+One step = one k3moe_layer call over one batch of the workload's tokens (the
+whole hot path: router, softmax, top-k, dispatch, routed gate/up + SwiGLU,
+down projections, shared expert, combine).  Default workload: the K3-shape
+decode layer (d=7168, ff=1536, 896 experts, top-16, bf16 shared expert
+ff=1536, T=1 token), all 896 experts resident in HBM (15.7 GB).
+
+Timing: W warm-up steps, then K timed steps; before every step a 256 MiB
+buffer is written so L2 (126 MB) holds none of the weights; each step is
+bracketed by CUDA events on the launching stream (the flush stays outside),
+and the per-kernel durations come from events the library records between
+its kernels (k3moe_layer_timed).  Multi-GPU: replicas only (each rank runs
+its own layer instance on its own GPU, no collective in the data path);
+value = tokens of all ranks / max-over-ranks time.
+
+--impl reference times the fp64 CPU oracle on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import k3gen  # noqa: E402
+
+METRIC = "MoE-layer tokens/s"
+UNIT = "tokens/s"
+
+
+def workload_desc(cfg):
+    return (f"{cfg.name}: d={cfg.d}, ff={cfg.ff}, E={cfg.E}, top-{cfg.k}, shared ff={cfg.ff_shared},"
+            f" T={cfg.T}, bias={cfg.bias or 'none'}")
+
+
+def alg_bytes(cfg, U):
+    """Algorithmic HBM bytes of one layer call: router weights, shared expert,
+    each distinct selected expert once, activations in and out."""
+    router = cfg.E * cfg.d * 4
+    shared = 3 * cfg.d * cfg.ff_shared * 2
+    experts = U * cfg.blob_bytes
+    act = cfg.T * cfg.d * 2 * 2
+    return router + shared + experts + act
+
+
+def gu_bytes(cfg, U, pairs):
+    """Algorithmic bytes of one routed gate/up launch: W_g and W_u of each
+    distinct expert (nibbles + scales), x in, SwiGLU activations out."""
+    return U * 2 * cfg.d * cfg.ff * 17 // 32 + cfg.T * cfg.d * 2 + pairs * cfg.ff * 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_time(cfg, seconds=10.0):
+    """Time the fp64 oracle (as it stands) on whole tokens of the workload
+    until ~`seconds` of work; -> (tokens/s, threads, n_tokens)."""
+    import oracle
+    orc = oracle.oracle()
+    x = k3gen.hidden(cfg)
+    w = k3gen.router(cfg)
+    b = k3gen.bias(cfg)
+    sh = k3gen.shared(cfg) if cfg.ff_shared else None
+    cache = {}
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    done = 0
+    t_total = 0.0
+    while t_total < seconds and done < cfg.T:
+        xs = x[done:done + 1]
+        # blob generation is input preparation, kept outside the timed region
+        _, _, idx, _ = orc.route(xs, w, b, cfg.k)
+        for e in idx[0]:
+            if int(e) not in cache:
+                cache[int(e)] = k3gen.expert_blob(cfg, int(e))
+        t0 = time.perf_counter()
+        _, _, idx, wt = orc.route(xs, w, b, cfg.k)
+        orc.combine(xs, wt, [cache[int(e)] for e in idx[0]], sh, cfg.d, cfg.ff)
+        t_total += time.perf_counter() - t0
+        done += 1
+    return done / t_total, threads, done, t_total
+
+
+def run_reference(args, cfg, rank):
+    if rank != 0:
+        return
+    tok_s, threads, n, t = cpu_oracle_time(cfg, seconds=max(5.0, 2.0 * args.steps))
+    ms = 1000.0 * t / n
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": n, "warmup": 0, "ms_per_step": ms * cfg.T, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(cfg)},
+        "cpu_baseline": {"value": tok_s, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{n} token(s) of the workload, fp64 scalar C oracle"},
+        "e2e": {"value": tok_s, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="k3_decode", choices=list(k3gen.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quick", action="store_true", help="profiling mode: no e2e/cpu legs")
+    args = ap.parse_args()
+    if args.warmup < 3 and not args.quick:
+        args.warmup = 3
+    cfg = k3gen.CONFIGS[args.config]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import mxfp4_routed_expert_softmax_b200 as k3
+    from k3gen import device as kdev
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    W = kdev.weights(cfg)
+    inp = kdev.DeviceInputs(cfg)
+    T = inp.T
+    dims = k3.make_dims(cfg.d, cfg.ff, cfg.E, cfg.k, cfg.ff_shared,
+                        k3.K3MOE_OUT_FP32 if cfg.out_fp32 else 0)
+    ws = k3.new_workspace(dims, T, host_staging=True)
+    ybytes = 4 if cfg.out_fp32 else 2
+    y = torch.empty((T, cfg.d), dtype=torch.float32 if cfg.out_fp32 else torch.int16, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    sg, su, sd = W.shared
+
+    def step_plain():
+        k3.check(k3.k3moe_layer(inp.x, T, W.w_router, inp.bias, W.blob_ptrs, sg, su, sd, dims, y,
+                                None, None, ws), "k3moe_layer")
+
+    single_pass = T <= 8
+    nev = 5
+    # warm-up
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step_plain()
+    torch.cuda.synchronize()
+    k3.check(k3.k3moe_device_status(ws), "device status")
+
+    # distinct experts of the batch (for the algorithmic byte count)
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
+    k3.check(k3.k3moe_route(inp.x, T, W.w_router, inp.bias, dims, idx, wts, ws), "route")
+    idx_np = idx.cpu().numpy()
+    U = len(np.unique(idx_np))
+    pairs = T * cfg.k
+
+    # timed region
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    kern_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)]
+               for _ in range(args.steps)] if single_pass else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 255)
+        if single_pass:
+            ev = kern_ev[i]
+            step_ev[i][0].record(stream)
+            st, nk = k3.k3moe_layer_timed(inp.x, T, W.w_router, inp.bias, W.blob_ptrs, sg, su, sd,
+                                          dims, y, ws, ev)
+            k3.check(st, "k3moe_layer_timed")
+            step_ev[i][1].record(stream)
+        else:
+            step_ev[i][0].record(stream)
+            step_plain()
+            step_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    k3.check(k3.k3moe_device_status(ws), "device status")
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * T * args.steps / (total_ms / 1000.0)
+
+    # per-kernel durations (events recorded between the library's kernels)
+    kernels = ["route_shared", "expert_gu", "expert_down", "combine"]
+    per_kernel = {}
+    if single_pass:
+        for j, name in enumerate(kernels):
+            per_kernel[name] = statistics.mean(kern_ev[i][j].elapsed_time(kern_ev[i][j + 1])
+                                               for i in range(args.steps))
+    peak, peak_kind = load_peaks()
+    gu_ms = per_kernel.get("expert_gu")
+    gb = gu_bytes(cfg, U, pairs)
+    roofline = None
+    if gu_ms:
+        ach = gb / (gu_ms / 1000.0) / 1e9
+        roofline = {"bound": "hbm", "kernel": "expert_gu", "achieved": round(ach, 1),
+                    "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 4),
+                    "peak_kind": f"{peak_kind} (burst copy, MEASURED_PEAKS.json hbm_gbs)"
+                    if peak_kind == "measured" else "fallback 6.65 TB/s",
+                    "traffic": None, "alg_bytes_per_launch": gb}
+    layer_gbs = alg_bytes(cfg, U) / (ms_per_step / 1000.0) / 1e9
+
+    # end to end: host activations in and out through the C ABI, copies timed
+    e2e = None
+    if not args.quick:
+        import torch as _t
+        xh = _t.from_numpy(inp.x_host.view(np.int16)).pin_memory()
+        yh = _t.empty((T, cfg.d), dtype=_t.float32 if cfg.out_fp32 else _t.int16).pin_memory()
+        e_ms = 0.0
+        for i in range(args.warmup + args.steps):
+            flush.fill_(i & 255)
+            a, b = _t.cuda.Event(enable_timing=True), _t.cuda.Event(enable_timing=True)
+            a.record(stream)
+            k3.check(k3.k3moe_layer_from_host(xh, T, W.w_router, inp.bias, W.blob_ptrs, sg, su, sd,
+                                              dims, yh, ws), "from_host")
+            b.record(stream)
+            b.synchronize()  # the result is on the host here
+            if i >= args.warmup:
+                e_ms += a.elapsed_time(b)
+        if world > 1:
+            t = _t.tensor([e_ms], dtype=_t.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * T * args.steps / (e_ms / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * ybytes}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
+        tok_s, threads, n, t = cpu_oracle_time(cfg, seconds=10.0)
+        cpu = {"value": tok_s, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{n} token(s) of the workload ({t:.1f} s), fp64 scalar C oracle, "
+                         f"OpenMP over output rows"}
+
+    chunks = (T + 7) // 8
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16/bf16 mma, f32 accumulate",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(cfg), "global_batch": world * T, "seq_len": 1,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "256 MiB buffer written before every step, outside the timed events",
+                   "distinct_experts": U},
+        "layer_hbm_gbs": round(layer_gbs, 1),
+        "layer_hbm_frac": round(layer_gbs / peak, 4),
+        "per_kernel_ms": {k: round(v, 5) for k, v in per_kernel.items()},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 4 * chunks * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,203 @@
+/*
+ * k3moe -- one Kimi-K3-shape mixture-of-experts FFN layer computed directly on
+ * packed MXFP4 expert weights, for NVIDIA B200 (sm_100a).
+ *
+ * The layer (per token x, hidden size d):
+ *   l   = W_r x + b                              router logits over E experts
+ *   p   = softmax(l)                              over all E experts
+ *   idx = the k experts with the largest l, ties to the lower index, listed in
+ *         descending order; w_j = p_idx_j (not renormalised over the k)
+ *   o_e = W_d,e (silu(W_g,e x) * W_u,e x)         SwiGLU expert, MXFP4 weights
+ *   S   = W_d,s (silu(W_g,s x) * W_u,s x)         shared expert, bf16 weights
+ *   y   = S + sum_j w_j o_idx_j
+ * Sources: "Kimi K3 纯 C 语言 CPU 推理实战" (chenxutan.com), section 1.2 (the
+ * routing formula, K = 16 of 896 experts plus an always-on shared expert) and
+ * section 2.4 (router GEMV, stable softmax over all experts, top-k, weighted
+ * combine; the MoELayer/moe_forward interface); the kimi-k3-in-c project card
+ * ("P053"), core features (experts multiplied directly on the packed nibbles,
+ * never dequantised; MXFP4 = 4-bit E2M1 nibble + shared E8M0 scale, 0.53125
+ * bytes per weight) and architecture notes (the config reader refuses
+ * defaults: every argument here is explicit and validated).
+ *
+ * ---------------------------------------------------------------------------
+ * Data formats (all device memory, little-endian, row-major):
+ *   x          bf16 [T][d]
+ *   w_router   fp32 [E][d]
+ *   bias       fp32 [E], or NULL for no bias (added to the logits before the
+ *              softmax, so it moves both the selection and the weights)
+ *   expert blob, one per routed expert, 3*d*ff*17/32 bytes, 16-byte aligned:
+ *     [W_g nibbles | W_g scales | W_u nibbles | W_u scales | W_d nibbles | W_d scales]
+ *     W_g, W_u: ff rows x d columns; W_d: d rows x ff columns.
+ *     A nibble plane holds rows*cols/2 bytes: element (r, c) is the low nibble
+ *     (bits 0-3) of byte r*cols/2 + c/2 when c is even, the high nibble when c
+ *     is odd.  A scale plane holds rows*cols/32 E8M0 bytes: byte r*cols/32 + c/32
+ *     scales the 32 consecutive elements of row r that contain column c.
+ *     E2M1 code: sign bit 3, 2 exponent bits (bias 1), 1 mantissa bit ->
+ *     {0, 0.5, 1, 1.5, 2, 3, 4, 6}; E8M0 byte e -> 2^(e-127), 255 = NaN
+ *     (OCP Microscaling Formats v1.0).
+ *   shared expert: W_g,s, W_u,s bf16 [ff_shared][d], W_d,s bf16 [d][ff_shared]
+ *   y          [T][d], bf16 (round to nearest even, once, from the fp32 sum) or
+ *              fp32 with K3MOE_OUT_FP32
+ *   idx        int32 [T][k], weight fp32 [T][k]
+ *
+ * Precision: routed-expert weights are decoded exactly (E2M1 x 2^(e-127) is
+ * exact); products are formed exactly and summed in fp32.  Router logits are
+ * summed in fp32 from the exact fp32 weights and bf16 inputs.
+ *
+ * Ownership and ordering: the caller owns every buffer and the stream.  Calls
+ * allocate nothing, never synchronise, and are ordered on `stream`; results
+ * are valid once the stream reaches them, and inputs must stay unmodified
+ * until then.  `ws` is caller-owned device scratch of at least
+ * k3moe_workspace_size() bytes, 256-byte aligned and zero-filled before its
+ * first use (each call leaves it ready for the next); one workspace must not
+ * be used by two calls that may run at the same time.
+ *
+ * Errors: every call validates all arguments before launching anything and
+ * returns a status; on failure nothing is launched.  Launch failures return
+ * K3MOE_ERR_CUDA (the CUDA error text is kept for k3moe_last_error()).
+ * Conditions only the device can see (a blob pointer that is not 16-byte
+ * aligned, a bounded wait that ran out) are recorded in the workspace status
+ * word and read with k3moe_device_status().
+ * ---------------------------------------------------------------------------
+ */
+#ifndef K3MOE_H
+#define K3MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define K3MOE_ABI_VERSION 1
+
+typedef enum {
+    K3MOE_OK = 0,
+    K3MOE_ERR_INVALID_ARGUMENT = 1,   /* null/misaligned pointer, bad count */
+    K3MOE_ERR_UNSUPPORTED_SHAPE = 2,  /* dimension outside the supported set */
+    K3MOE_ERR_WORKSPACE_TOO_SMALL = 3,
+    K3MOE_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
+    K3MOE_ERR_DEVICE_TIMEOUT = 5,     /* a bounded device wait ran out */
+    K3MOE_ERR_DEVICE_CHECK = 6        /* a device-side argument check failed */
+} k3moe_status;
+
+/* flags */
+#define K3MOE_OUT_FP32 1u  /* y (and expert_ffn's out) in fp32 instead of bf16 */
+#define K3MOE_NO_SHARED 2u /* skip the shared expert (its pointers may be NULL) */
+
+/*
+ * Layer dimensions.  d and ff: multiples of 64, 64 <= d <= 8192,
+ * 64 <= ff <= 8192; 1 <= n_experts <= 1024; 1 <= top_k <= min(n_experts, 32);
+ * ff_shared: 0 (no shared expert) or a multiple of 64 up to 8192.  Shapes
+ * whose staging tiles do not fit in one SM's shared memory (large ff or
+ * ff_shared) return K3MOE_ERR_UNSUPPORTED_SHAPE.  Unknown flag bits are
+ * rejected.
+ */
+typedef struct {
+    int32_t d;
+    int32_t ff;
+    int32_t n_experts;
+    int32_t top_k;
+    int32_t ff_shared;
+    uint32_t flags;
+} k3moe_dims;
+
+/* ABI version of the loaded library (K3MOE_ABI_VERSION when it matches). */
+int k3moe_abi_version(void);
+
+/* Bytes of one routed expert's blob: 3*d*ff*17/32; 0 if dims are invalid. */
+size_t k3moe_blob_bytes(const k3moe_dims *dims);
+
+/* Scratch bytes a call with up to T_max tokens needs; 0 if dims are invalid. */
+size_t k3moe_workspace_size(const k3moe_dims *dims, int32_t T_max);
+
+/*
+ * Router, softmax over all experts, top-k (tutorial page, section 2.4):
+ *   idx[t][j] = j-th selected expert of token t (descending logit, ties to the
+ *               lower index), weight[t][j] = its softmax probability.
+ * x: bf16 [T][d]; w_router: fp32 [E][d]; bias: fp32 [E] or NULL;
+ * idx: int32 [T][k]; weight: fp32 [T][k].  All pointers 16-byte aligned
+ * except bias, idx and weight (4-byte aligned).
+ */
+k3moe_status k3moe_route(const void *x, int32_t T, const float *w_router, const float *bias,
+                         const k3moe_dims *dims, int32_t *idx, float *weight, void *ws,
+                         size_t ws_bytes, void *stream);
+
+/*
+ * One routed expert applied to T tokens, unweighted (the per-expert step of
+ * the tutorial page's section 2.4 loop, on the packed nibbles per the project
+ * card): out[t] = W_d (silu(W_g x_t) * W_u x_t).
+ * blob: one expert blob as above (16-byte aligned); out: [T][d] bf16, or fp32
+ * with K3MOE_OUT_FP32.  n_experts/top_k/ff_shared in dims are not used but
+ * must still be valid.
+ */
+k3moe_status k3moe_expert_ffn(const void *x, int32_t T, const uint8_t *blob,
+                              const k3moe_dims *dims, void *out, void *ws, size_t ws_bytes,
+                              void *stream);
+
+/*
+ * The whole layer (tutorial page, sections 1.2 and 2.4):
+ *   y[t] = S(x_t) + sum_j w[t][j] o_idx[t][j](x_t)
+ * expert_blobs: DEVICE array of E device pointers, expert e's blob at
+ *   expert_blobs[e] (each 16-byte aligned; checked on the device);
+ * shared_wg/wu/wd: bf16 shared-expert matrices, or NULL with ff_shared == 0
+ *   or K3MOE_NO_SHARED;
+ * y: [T][d] bf16 or fp32 (K3MOE_OUT_FP32);
+ * idx_out / w_out: optional copies of the routing ([T][k]), may be NULL.
+ */
+k3moe_status k3moe_layer(const void *x, int32_t T, const float *w_router, const float *bias,
+                         const uint8_t *const *expert_blobs, const void *shared_wg,
+                         const void *shared_wu, const void *shared_wd, const k3moe_dims *dims,
+                         void *y, int32_t *idx_out, float *w_out, void *ws, size_t ws_bytes,
+                         void *stream);
+
+/*
+ * k3moe_layer with the activations in HOST memory: copies x_host ([T][d]
+ * bf16) into the workspace, runs the layer, and copies y back to y_host
+ * ([T][d], bf16 or fp32 per flags), all ordered on `stream` (the copies are
+ * asynchronous when the host buffers are page-locked).  Weights stay in
+ * device memory as for k3moe_layer.  The host buffers must stay valid until
+ * the stream reaches the end of the call.  Needs
+ * k3moe_workspace_size(dims, T) + k3moe_host_staging_bytes(dims, T) bytes.
+ */
+size_t k3moe_host_staging_bytes(const k3moe_dims *dims, int32_t T);
+k3moe_status k3moe_layer_from_host(const void *x_host, int32_t T, const float *w_router,
+                                   const float *bias, const uint8_t *const *expert_blobs,
+                                   const void *shared_wg, const void *shared_wu,
+                                   const void *shared_wd, const k3moe_dims *dims, void *y_host,
+                                   void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * k3moe_layer for per-kernel timing (device input and output, up to 8 tokens,
+ * i.e. one pass of the kernels): `events` are n_events cudaEvent_t handles
+ * created by the caller; events[0] is recorded on `stream` before the first
+ * kernel and events[i] after the i-th kernel, for i up to the number of
+ * kernels the call launches, which is written to *n_kernels (4: router and
+ * shared gate/up with top-k, routed gate/up, down projections, combine).
+ * The computation and its result are those of k3moe_layer.
+ */
+k3moe_status k3moe_layer_timed(const void *x, int32_t T, const float *w_router, const float *bias,
+                               const uint8_t *const *expert_blobs, const void *shared_wg,
+                               const void *shared_wu, const void *shared_wd,
+                               const k3moe_dims *dims, void *y, void *ws, size_t ws_bytes,
+                               void *stream, void *const *events, int32_t n_events,
+                               int32_t *n_kernels);
+
+/*
+ * Synchronises `stream`, then reads and clears the workspace status word:
+ * K3MOE_OK, K3MOE_ERR_DEVICE_CHECK or K3MOE_ERR_DEVICE_TIMEOUT.
+ */
+k3moe_status k3moe_device_status(void *ws, void *stream);
+
+/* Static text for a status code. */
+const char *k3moe_status_string(k3moe_status status);
+
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char *k3moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* K3MOE_H */

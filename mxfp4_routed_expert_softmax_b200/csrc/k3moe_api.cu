@@ -1,0 +1,440 @@
+// C ABI of the k3moe library: argument validation, workspace layout and the
+// launch sequence of each entry point.  Declarations and the contract of
+// every function are in include/k3moe.h.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "decode_kernels.cuh"
+#include "k3moe.h"
+#include "layout.cuh"
+
+namespace {
+
+using namespace k3;
+
+thread_local std::string g_last_error;
+
+constexpr int kMaxDevices = 64;
+constexpr int kSmemLimit = 227 * 1024;
+
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+k3moe_status cuda_fail(cudaError_t e) {
+    g_last_error = cudaGetErrorString(e);
+    return K3MOE_ERR_CUDA;
+}
+
+template <typename Kern>
+cudaError_t set_smem(Kern kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// One-time per-device set-up: SM count and the shared-memory opt-ins.
+k3moe_status device_info(DeviceInfo **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return K3MOE_ERR_INVALID_ARGUMENT;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo &di = g_dev[dev];
+    if (!di.ready) {
+        e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e);
+        const int big = kSmemLimit;
+        cudaError_t r = cudaSuccess;
+        r = set_smem(route_shared_kernel, kRouteTok * 8192 * 4);
+        if (r == cudaSuccess) r = set_smem(expert_gu_kernel<1>, big);
+        if (r == cudaSuccess) r = set_smem(expert_gu_kernel<2>, big);
+        if (r == cudaSuccess) r = set_smem(expert_gu_kernel<4>, big);
+        if (r == cudaSuccess) r = set_smem(expert_gu_kernel<8>, big);
+        if (r == cudaSuccess) r = set_smem(expert_gu_kernel<16>, big);
+        if (r == cudaSuccess) r = set_smem(expert_down_kernel<1>, big);
+        if (r == cudaSuccess) r = set_smem(expert_down_kernel<2>, big);
+        if (r == cudaSuccess) r = set_smem(expert_down_kernel<4>, big);
+        if (r == cudaSuccess) r = set_smem(expert_down_kernel<8>, big);
+        if (r != cudaSuccess) return cuda_fail(r);
+        di.ready = true;
+    }
+    *out = &di;
+    return K3MOE_OK;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int shared_ff(const k3moe_dims *dm) {
+    return (dm->flags & K3MOE_NO_SHARED) ? 0 : dm->ff_shared;
+}
+
+k3moe_status check_dims(const k3moe_dims *dm) {
+    if (!dm) return K3MOE_ERR_INVALID_ARGUMENT;
+    if (dm->flags & ~(K3MOE_OUT_FP32 | K3MOE_NO_SHARED)) return K3MOE_ERR_INVALID_ARGUMENT;
+    if (dm->d < 64 || dm->d > 8192 || dm->d % 64) return K3MOE_ERR_UNSUPPORTED_SHAPE;
+    if (dm->ff < 64 || dm->ff > 8192 || dm->ff % 64) return K3MOE_ERR_UNSUPPORTED_SHAPE;
+    if (dm->n_experts < 1 || dm->n_experts > 1024) return K3MOE_ERR_UNSUPPORTED_SHAPE;
+    if (dm->top_k < 1 || dm->top_k > 32 || dm->top_k > dm->n_experts)
+        return K3MOE_ERR_INVALID_ARGUMENT;
+    if (dm->ff_shared < 0 || dm->ff_shared > 8192 || dm->ff_shared % 64)
+        return K3MOE_ERR_UNSUPPORTED_SHAPE;
+    if (gu_smem_bytes(dm->d) > kSmemLimit) return K3MOE_ERR_UNSUPPORTED_SHAPE;
+    if (dn_smem_bytes(dm->ff, dm->ff_shared) > kSmemLimit) return K3MOE_ERR_UNSUPPORTED_SHAPE;
+    return K3MOE_OK;
+}
+
+Layout layout_for(const k3moe_dims *dm, int k_eff) {
+    return make_layout(dm->d, dm->ff, dm->n_experts, k_eff, dm->ff_shared);
+}
+
+size_t staging_bytes(const k3moe_dims *dm) {
+    return align256((size_t)kChunk * dm->d * 2) + align256((size_t)kChunk * dm->d * 4);
+}
+
+template <typename Kern, typename P>
+cudaError_t launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                   const P &params) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, params);
+}
+
+int pow2_at_least(int v) {
+    int p = 1;
+    while (p < v) p <<= 1;
+    return p;
+}
+
+cudaError_t launch_gu(const DeviceInfo &di, const GUParams &gp, cudaStream_t st) {
+    const int need = (gp.d / 32 + 15) / 16;
+    const int smem = gu_smem_bytes(gp.d);
+    const dim3 grid(di.sms), block(kGUThreads);
+    switch (pow2_at_least(need)) {
+        case 1: return launch(expert_gu_kernel<1>, grid, block, smem, st, true, gp);
+        case 2: return launch(expert_gu_kernel<2>, grid, block, smem, st, true, gp);
+        case 4: return launch(expert_gu_kernel<4>, grid, block, smem, st, true, gp);
+        case 8: return launch(expert_gu_kernel<8>, grid, block, smem, st, true, gp);
+        default: return launch(expert_gu_kernel<16>, grid, block, smem, st, true, gp);
+    }
+}
+
+cudaError_t launch_down(const DeviceInfo &di, const DownParams &dp, cudaStream_t st) {
+    const int kmax = dp.ff > dp.ffs ? dp.ff : dp.ffs;
+    const int need = (kmax / 32 + 15) / 16;
+    const int smem = dn_smem_bytes(dp.ff, dp.ffs);
+    const dim3 grid(di.sms), block(kDownThreads);
+    switch (pow2_at_least(need)) {
+        case 1: return launch(expert_down_kernel<1>, grid, block, smem, st, true, dp);
+        case 2: return launch(expert_down_kernel<2>, grid, block, smem, st, true, dp);
+        case 4: return launch(expert_down_kernel<4>, grid, block, smem, st, true, dp);
+        default: return launch(expert_down_kernel<8>, grid, block, smem, st, true, dp);
+    }
+}
+
+// Router (+ shared gate/up + top-k + dispatch) for one chunk.
+cudaError_t launch_route(const DeviceInfo &di, const RouteParams &rp, cudaStream_t st) {
+    const int N = rp.E + rp.ffs;
+    const int nt = rp.Tc < kRouteTok ? rp.Tc : kRouteTok;
+    const int smem = nt * rp.d * 4;
+    const int per_sm = smem <= 64 * 1024 ? 2 : 1;
+    int G = di.sms * per_sm;
+    if (G > N) G = N;
+    return launch(route_shared_kernel, dim3(G), dim3(kRouteThreads), smem, st, false, rp);
+}
+
+struct EventHook {
+    cudaEvent_t *ev = nullptr;
+    int n = 0;
+    int next = 0;
+    cudaError_t record(cudaStream_t st) {
+        if (!ev || next >= n) return cudaSuccess;
+        return cudaEventRecord(ev[next++], st);
+    }
+};
+
+k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const float *bias,
+                        const uint8_t *const *expert_blobs, const void *shared_wg,
+                        const void *shared_wu, const void *shared_wd, const k3moe_dims *dims,
+                        void *y, int32_t *idx_out, float *w_out, void *ws, size_t ws_bytes,
+                        void *stream, const void *x_host, void *y_host, EventHook *hook = nullptr) {
+    k3moe_status s = check_dims(dims);
+    if (s != K3MOE_OK) return s;
+    const bool from_host = x_host != nullptr;
+    if (T < 1) return K3MOE_ERR_INVALID_ARGUMENT;
+    if (!from_host && (!x || !y || !aligned(x, 16) || !aligned(y, 16)))
+        return K3MOE_ERR_INVALID_ARGUMENT;
+    if (from_host && !y_host) return K3MOE_ERR_INVALID_ARGUMENT;
+    if (!w_router || !aligned(w_router, 16) || !expert_blobs || !aligned(expert_blobs, 8))
+        return K3MOE_ERR_INVALID_ARGUMENT;
+    if (bias && !aligned(bias, 4)) return K3MOE_ERR_INVALID_ARGUMENT;
+    if ((idx_out && !aligned(idx_out, 4)) || (w_out && !aligned(w_out, 4)))
+        return K3MOE_ERR_INVALID_ARGUMENT;
+    const int ffs = shared_ff(dims);
+    if (ffs > 0) {
+        if (!shared_wg || !shared_wu || !shared_wd || !aligned(shared_wg, 16) ||
+            !aligned(shared_wu, 16) || !aligned(shared_wd, 16))
+            return K3MOE_ERR_INVALID_ARGUMENT;
+    }
+    if (!ws || !aligned(ws, 256)) return K3MOE_ERR_INVALID_ARGUMENT;
+    const Layout L = layout_for(dims, dims->top_k);
+    const size_t need = L.total + (from_host ? staging_bytes(dims) : 0);
+    if (ws_bytes < need) return K3MOE_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo *di = nullptr;
+    s = device_info(&di);
+    if (s != K3MOE_OK) return s;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
+    const int d = dims->d;
+    const bool out32 = (dims->flags & K3MOE_OUT_FP32) != 0;
+    const size_t ybytes = out32 ? 4 : 2;
+    uint8_t *xstage = wsb + L.total;
+    uint8_t *ystage = xstage + align256((size_t)kChunk * d * 2);
+
+    for (int c0 = 0; c0 < T; c0 += kChunk) {
+        const int Tc = (T - c0) < kChunk ? (T - c0) : kChunk;
+        const uint16_t *xc;
+        void *yc;
+        cudaError_t e;
+        if (from_host) {
+            e = cudaMemcpyAsync(xstage, reinterpret_cast<const uint8_t *>(x_host) + (size_t)c0 * d * 2,
+                                (size_t)Tc * d * 2, cudaMemcpyHostToDevice, st);
+            if (e != cudaSuccess) return cuda_fail(e);
+            xc = reinterpret_cast<const uint16_t *>(xstage);
+            yc = ystage;
+        } else {
+            xc = reinterpret_cast<const uint16_t *>(x) + (size_t)c0 * d;
+            yc = reinterpret_cast<uint8_t *>(y) + (size_t)c0 * d * ybytes;
+        }
+        RouteParams rp{};
+        rp.x = xc;
+        rp.Tc = Tc;
+        rp.wr = w_router;
+        rp.bias = bias;
+        rp.swg = reinterpret_cast<const uint16_t *>(shared_wg);
+        rp.swu = reinterpret_cast<const uint16_t *>(shared_wu);
+        rp.ffs = ffs;
+        rp.d = d;
+        rp.E = dims->n_experts;
+        rp.k = dims->top_k;
+        rp.ws = wsb;
+        rp.L = L;
+        rp.blobs = expert_blobs;
+        rp.idx_out = idx_out ? idx_out + (size_t)c0 * dims->top_k : nullptr;
+        rp.w_out = w_out ? w_out + (size_t)c0 * dims->top_k : nullptr;
+        EventHook none;
+        EventHook &hk = hook ? *hook : none;
+        if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
+        e = launch_route(*di, rp, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
+
+        GUParams gp{xc, Tc, d, dims->ff, wsb, L};
+        e = launch_gu(*di, gp, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
+
+        DownParams dp{Tc, d, dims->ff, ffs, reinterpret_cast<const uint16_t *>(shared_wd), wsb, L};
+        e = launch_down(*di, dp, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
+
+        CombineParams cp{Tc, d, dims->top_k, ffs > 0, out32, wsb, L, yc};
+        e = launch(combine_kernel, dim3((d + 1023) / 1024, Tc), dim3(256), 0, st, true, cp);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
+
+        if (from_host) {
+            e = cudaMemcpyAsync(reinterpret_cast<uint8_t *>(y_host) + (size_t)c0 * d * ybytes, ystage,
+                                (size_t)Tc * d * ybytes, cudaMemcpyDeviceToHost, st);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+    }
+    return K3MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int k3moe_abi_version(void) { return K3MOE_ABI_VERSION; }
+
+size_t k3moe_blob_bytes(const k3moe_dims *dims) {
+    if (check_dims(dims) != K3MOE_OK) return 0;
+    return (size_t)3 * dims->d * dims->ff * 17 / 32;
+}
+
+size_t k3moe_workspace_size(const k3moe_dims *dims, int32_t T_max) {
+    if (check_dims(dims) != K3MOE_OK || T_max < 1) return 0;
+    return layout_for(dims, dims->top_k).total;
+}
+
+size_t k3moe_host_staging_bytes(const k3moe_dims *dims, int32_t T) {
+    if (check_dims(dims) != K3MOE_OK || T < 1) return 0;
+    return staging_bytes(dims);
+}
+
+k3moe_status k3moe_route(const void *x, int32_t T, const float *w_router, const float *bias,
+                         const k3moe_dims *dims, int32_t *idx, float *weight, void *ws,
+                         size_t ws_bytes, void *stream) {
+    k3moe_status s = check_dims(dims);
+    if (s != K3MOE_OK) return s;
+    if (T < 1 || !x || !aligned(x, 16) || !w_router || !aligned(w_router, 16) || !idx ||
+        !weight || !aligned(idx, 4) || !aligned(weight, 4) || (bias && !aligned(bias, 4)))
+        return K3MOE_ERR_INVALID_ARGUMENT;
+    if (!ws || !aligned(ws, 256)) return K3MOE_ERR_INVALID_ARGUMENT;
+    const Layout L = layout_for(dims, dims->top_k);
+    if (ws_bytes < L.total) return K3MOE_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo *di = nullptr;
+    s = device_info(&di);
+    if (s != K3MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    for (int c0 = 0; c0 < T; c0 += kChunk) {
+        const int Tc = (T - c0) < kChunk ? (T - c0) : kChunk;
+        RouteParams rp{};
+        rp.x = reinterpret_cast<const uint16_t *>(x) + (size_t)c0 * dims->d;
+        rp.Tc = Tc;
+        rp.wr = w_router;
+        rp.bias = bias;
+        rp.ffs = 0;
+        rp.d = dims->d;
+        rp.E = dims->n_experts;
+        rp.k = dims->top_k;
+        rp.ws = reinterpret_cast<uint8_t *>(ws);
+        rp.L = L;
+        rp.blobs = nullptr;
+        rp.idx_out = idx + (size_t)c0 * dims->top_k;
+        rp.w_out = weight + (size_t)c0 * dims->top_k;
+        cudaError_t e = launch_route(*di, rp, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return K3MOE_OK;
+}
+
+k3moe_status k3moe_expert_ffn(const void *x, int32_t T, const uint8_t *blob,
+                              const k3moe_dims *dims, void *out, void *ws, size_t ws_bytes,
+                              void *stream) {
+    k3moe_status s = check_dims(dims);
+    if (s != K3MOE_OK) return s;
+    if (T < 1 || !x || !aligned(x, 16) || !blob || !aligned(blob, 16) || !out || !aligned(out, 16))
+        return K3MOE_ERR_INVALID_ARGUMENT;
+    if (!ws || !aligned(ws, 256)) return K3MOE_ERR_INVALID_ARGUMENT;
+    if (ws_bytes < layout_for(dims, dims->top_k).total) return K3MOE_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo *di = nullptr;
+    s = device_info(&di);
+    if (s != K3MOE_OK) return s;
+    const Layout L = layout_for(dims, 1);  // one slot per token, weight 1
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
+    const int d = dims->d;
+    const bool out32 = (dims->flags & K3MOE_OUT_FP32) != 0;
+    for (int c0 = 0; c0 < T; c0 += kChunk) {
+        const int Tc = (T - c0) < kChunk ? (T - c0) : kChunk;
+        const uint16_t *xc = reinterpret_cast<const uint16_t *>(x) + (size_t)c0 * d;
+        void *yc = reinterpret_cast<uint8_t *>(out) + (size_t)c0 * d * (out32 ? 4 : 2);
+        SingleParams sp{xc, Tc, d, blob, wsb, L};
+        cudaError_t e = launch(single_expert_setup_kernel, dim3(1), dim3(256), 0, st, false, sp);
+        if (e != cudaSuccess) return cuda_fail(e);
+        GUParams gp{xc, Tc, d, dims->ff, wsb, L};
+        e = launch_gu(*di, gp, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+        DownParams dp{Tc, d, dims->ff, 0, nullptr, wsb, L};
+        e = launch_down(*di, dp, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+        CombineParams cp{Tc, d, 1, false, out32, wsb, L, yc};
+        e = launch(combine_kernel, dim3((d + 1023) / 1024, Tc), dim3(256), 0, st, true, cp);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return K3MOE_OK;
+}
+
+k3moe_status k3moe_layer(const void *x, int32_t T, const float *w_router, const float *bias,
+                         const uint8_t *const *expert_blobs, const void *shared_wg,
+                         const void *shared_wu, const void *shared_wd, const k3moe_dims *dims,
+                         void *y, int32_t *idx_out, float *w_out, void *ws, size_t ws_bytes,
+                         void *stream) {
+    return layer_impl(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu, shared_wd, dims, y,
+                      idx_out, w_out, ws, ws_bytes, stream, nullptr, nullptr);
+}
+
+k3moe_status k3moe_layer_from_host(const void *x_host, int32_t T, const float *w_router,
+                                   const float *bias, const uint8_t *const *expert_blobs,
+                                   const void *shared_wg, const void *shared_wu,
+                                   const void *shared_wd, const k3moe_dims *dims, void *y_host,
+                                   void *ws, size_t ws_bytes, void *stream) {
+    if (!x_host) return K3MOE_ERR_INVALID_ARGUMENT;
+    return layer_impl(nullptr, T, w_router, bias, expert_blobs, shared_wg, shared_wu, shared_wd,
+                      dims, nullptr, nullptr, nullptr, ws, ws_bytes, stream, x_host, y_host);
+}
+
+k3moe_status k3moe_layer_timed(const void *x, int32_t T, const float *w_router, const float *bias,
+                               const uint8_t *const *expert_blobs, const void *shared_wg,
+                               const void *shared_wu, const void *shared_wd,
+                               const k3moe_dims *dims, void *y, void *ws, size_t ws_bytes,
+                               void *stream, void *const *events, int32_t n_events,
+                               int32_t *n_kernels) {
+    if (T > kChunk || !events || n_events < 1 || !n_kernels) return K3MOE_ERR_INVALID_ARGUMENT;
+    for (int i = 0; i < n_events; ++i)
+        if (!events[i]) return K3MOE_ERR_INVALID_ARGUMENT;
+    EventHook hk;
+    hk.ev = reinterpret_cast<cudaEvent_t *>(const_cast<void **>(events));
+    hk.n = n_events;
+    k3moe_status s = layer_impl(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu,
+                                shared_wd, dims, y, nullptr, nullptr, ws, ws_bytes, stream, nullptr,
+                                nullptr, &hk);
+    *n_kernels = 4;
+    return s;
+}
+
+k3moe_status k3moe_device_status(void *ws, void *stream) {
+    if (!ws || !aligned(ws, 256)) return K3MOE_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    WsHeader h;
+    e = cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (h.status != 0u) {
+        // clear the status; after a timeout also restore the counters
+        WsHeader z;
+        memset(&z, 0, sizeof(z));
+        z.n_unique = h.n_unique;
+        e = cudaMemcpy(ws, &z, sizeof(z), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    if (h.status & kStTimeout) return K3MOE_ERR_DEVICE_TIMEOUT;
+    if (h.status & kStDeviceCheck) return K3MOE_ERR_DEVICE_CHECK;
+    return K3MOE_OK;
+}
+
+const char *k3moe_status_string(k3moe_status status) {
+    switch (status) {
+        case K3MOE_OK: return "ok";
+        case K3MOE_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case K3MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case K3MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case K3MOE_ERR_CUDA: return "CUDA error";
+        case K3MOE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        case K3MOE_ERR_DEVICE_CHECK: return "device-side argument check failed";
+    }
+    return "unknown status";
+}
+
+const char *k3moe_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"
