@@ -127,7 +127,10 @@ def cpu_oracle_time(cfg, seconds=10.0):
     until ~`seconds` of work; -> (tokens/s, threads, n_tokens)."""
     import oracle
     orc = oracle.oracle()
-    x = k3gen.hidden(cfg)
+    # tokens beyond the workload's own T are further draws of the same
+    # distribution (stream 0), so a small-T workload still gives a sample of
+    # ~`seconds` of oracle work
+    x = k3gen.hidden(cfg, T=max(cfg.T, 256))
     w = k3gen.router(cfg)
     b = k3gen.bias(cfg)
     sh = k3gen.shared(cfg) if cfg.ff_shared else None
@@ -135,7 +138,7 @@ def cpu_oracle_time(cfg, seconds=10.0):
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     done = 0
     t_total = 0.0
-    while t_total < seconds and done < cfg.T:
+    while t_total < seconds and done < x.shape[0]:
         xs = x[done:done + 1]
         # blob generation is input preparation, kept outside the timed region
         _, _, idx, _ = orc.route(xs, w, b, cfg.k)

@@ -40,9 +40,14 @@
  *              fp32 with K3MOE_OUT_FP32
  *   idx        int32 [T][k], weight fp32 [T][k]
  *
- * Precision: routed-expert weights are decoded exactly (E2M1 x 2^(e-127) is
- * exact); products are formed exactly and summed in fp32.  Router logits are
- * summed in fp32 from the exact fp32 weights and bf16 inputs.
+ * Precision: routed-expert weights enter the tensor cores exactly (each
+ * E2M1 code is re-placed as the E4M3 value 2^-6 * E2M1, the E8M0 scale
+ * multiplies each 32-weight block sum in fp32).  Activations enter as sums of
+ * E4M3 pieces after a per-token power-of-two prescale: x as two pieces (exact
+ * for every bf16 element down to 2^-17 of the token's largest |x|, below that
+ * off by at most 2^-18 of it), the SwiGLU activations h as four pieces (about
+ * 16 significant bits); the bf16 shared expert's h as bf16 hi + lo.  All sums
+ * are fp32.  Router logits are fp32 sums of exact fp32 x bf16 products.
  *
  * Ownership and ordering: the caller owns every buffer and the stream.  Calls
  * allocate nothing, never synchronise, and are ordered on `stream`; results
@@ -88,11 +93,10 @@ typedef enum {
 
 /*
  * Layer dimensions.  d and ff: multiples of 64, 64 <= d <= 8192,
- * 64 <= ff <= 8192; 1 <= n_experts <= 1024; 1 <= top_k <= min(n_experts, 32);
- * ff_shared: 0 (no shared expert) or a multiple of 64 up to 8192.  Shapes
- * whose staging tiles do not fit in one SM's shared memory (large ff or
- * ff_shared) return K3MOE_ERR_UNSUPPORTED_SHAPE.  Unknown flag bits are
- * rejected.
+ * 64 <= ff <= 3072; 1 <= n_experts <= 1024; 1 <= top_k <= min(n_experts, 32);
+ * ff_shared: 0 (no shared expert) or a multiple of 64 up to 3072.  Shapes
+ * whose staging tiles do not fit in one SM's shared memory return
+ * K3MOE_ERR_UNSUPPORTED_SHAPE.  Unknown flag bits are rejected.
  */
 typedef struct {
     int32_t d;
@@ -186,7 +190,9 @@ k3moe_status k3moe_layer_timed(const void *x, int32_t T, const float *w_router, 
 
 /*
  * Synchronises `stream`, then reads and clears the workspace status word:
- * K3MOE_OK, K3MOE_ERR_DEVICE_CHECK or K3MOE_ERR_DEVICE_TIMEOUT.
+ * K3MOE_OK, K3MOE_ERR_DEVICE_CHECK or K3MOE_ERR_DEVICE_TIMEOUT.  After
+ * K3MOE_ERR_DEVICE_TIMEOUT the outputs of the calls since the last check are
+ * undefined and the workspace must be zero-filled again before its next use.
  */
 k3moe_status k3moe_device_status(void *ws, void *stream);
 

@@ -9,6 +9,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp4.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -77,13 +78,15 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
+// try_wait with a suspend-time hint: the warp sleeps in hardware until the
+// phase completes (or ~1 ms passes) instead of spinning on the barrier.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
         " selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
         : "memory");
     return ok != 0;
 }
@@ -102,6 +105,23 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
+// ------------------------------------------------- gpu-scope atomics --
+// Release: this thread's earlier writes are visible to whoever acquires the
+// counter after it; acquire: writes released by others are visible after.
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ void red_add_release(uint32_t *p, uint32_t v) {
+    asm volatile("red.add.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // ------------------------------------------------- programmatic launches --
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
@@ -114,6 +134,61 @@ __device__ __forceinline__ void pdl_trigger() {
 __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
     __half2_raw r = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(byte), __NV_E2M1);
     return static_cast<uint32_t>(r.x) | (static_cast<uint32_t>(r.y) << 16);
+}
+
+// E2M1 nibbles -> E4M3 bytes by bit placement (ALU only, no conversion unit).
+// An E2M1 code s.e1e0.m becomes the E4M3 byte s.00e1e0.m00, whose value is
+// exactly 2^-6 times the E2M1 value: for exponent field e >= 1 both are
+// 2^(e-1)(1+m/2) resp. 2^(e-7)(1+m/2), and the E2M1 subnormal 0.5 (e=0, m=1)
+// lands on the E4M3 subnormal 4/8 * 2^-6.  The four even (low) nibbles of a
+// word give one word of four E4M3 bytes, the four odd (high) nibbles another.
+__device__ __forceinline__ uint32_t e2m1_even_to_e4m3(uint32_t w) {
+    return ((w << 4) & 0x80808080u) | ((w << 2) & 0x1C1C1C1Cu);
+}
+__device__ __forceinline__ uint32_t e2m1_odd_to_e4m3(uint32_t w) {
+    return (w & 0x80808080u) | ((w >> 2) & 0x1C1C1C1Cu);
+}
+
+// fp32 <-> E4M3 (OCP E4M3FN: bias 7, subnormals, no infinities) on the ALU
+// and FMA pipes.  Scaling by 2^-120 maps every E4M3 value, normal or
+// subnormal, onto fp32 bit patterns whose bits 30..20 are the E4M3 bits 6..0
+// (fp32 subnormals included, which fp32 arithmetic keeps when not flushing),
+// so rounding is an integer add at bit 20 (ties to even).  |v| <= 448.
+__device__ __forceinline__ uint32_t f32_to_e4m3_rn(float v) {
+    const uint32_t u = __float_as_uint(v * 0x1p-120f);
+    uint32_t m = u & 0x7FFFFFFFu;
+    m += 0x7FFFFu + ((m >> 20) & 1u);
+    return ((u >> 24) & 0x80u) | (m >> 20);
+}
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+    return __uint_as_float(((b & 0x80u) << 24) | ((b & 0x7Fu) << 20)) * 0x1p120f;
+}
+
+// Piece `piece` (0-based) of v written as a greedy sum of E4M3 values (each
+// step rounds the remaining residual to nearest; every residual is exact in
+// fp32).  Each piece carries 4 significant bits, so n pieces reproduce v
+// exactly while its low bits stay at or above the E4M3 step 2^-9.
+__device__ __forceinline__ uint32_t e4m3_piece(float v, int piece) {
+    uint32_t b = 0;
+    for (int i = 0; i <= piece; ++i) {
+        b = f32_to_e4m3_rn(v);
+        v -= e4m3_to_f32(b);
+    }
+    return b;
+}
+
+// Power-of-two exponent s with max_abs * 2^s in [128, 256): the largest
+// prescaled activation then fits E4M3 (max 448) with room for rounding up.
+__device__ __forceinline__ int e4m3_prescale(float max_abs) {
+    if (!(max_abs > 0.0f) || !isfinite(max_abs)) return 0;
+    int e;
+    frexpf(max_abs, &e);
+    int s = 8 - e;
+    return s < -100 ? -100 : (s > 100 ? 100 : s);
+}
+
+__device__ __forceinline__ float exp2i(int s) {  // 2^s for -126 <= s <= 127
+    return __uint_as_float((uint32_t)(127 + s) << 23);
 }
 
 // E8M0 byte -> 2^(e-127) as fp32 (e = 0 -> 2^-127, a subnormal; e = 255 -> NaN).
@@ -151,6 +226,16 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
                                         uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D = A(16x32, row) * B(32x8, col) + C, E4M3 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_e4m3(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));

@@ -1,27 +1,34 @@
 // Decode path of the MoE layer (up to kChunk tokens per pass).
 //
-//   route_shared  router GEMV (fp32 weights, CUDA cores) + the shared
-//                 expert's gate/up rows (bf16) + SwiGLU; the CTA that
-//                 finishes the last router row then runs softmax, top-k and
-//                 the expert dispatch for the chunk
-//   expert_gu     routed experts' gate/up on the packed MXFP4 rows: bulk
-//                 asynchronous copies into a shared-memory ring, E2M1 decoded
-//                 exactly to f16 in registers, mma.sync with the tokens as
-//                 the n dimension, E8M0 applied per 32-element block in fp32,
-//                 SwiGLU fused
-//   expert_down   down projection of every selected expert and of the shared
-//                 expert, same ring + mma scheme, activations split hi/lo
+//   route_shared  router GEMV (fp32 weights) and the shared expert's gate/up
+//                 rows (bf16) + SwiGLU on CUDA cores, streamed by warps over
+//                 equal slices of the weight bytes (a row split between warps
+//                 is summed by the last one to finish, in a fixed order); one
+//                 CTA waits for the router rows and runs softmax, top-k and the
+//                 expert dispatch while the others stream the shared expert
+//   expert_gu     gate/up of every selected expert on its packed MXFP4 rows:
+//                 bulk asynchronous copies into a shared-memory ring, E2M1
+//                 nibbles re-placed as E4M3 bytes by ALU bit operations (exact),
+//                 mma.sync m16n8k32 (E4M3) against the tokens, each token's x
+//                 carried as two E4M3 pieces, E8M0 block scales applied to the
+//                 fp32 block sums, SwiGLU fused
+//   expert_down   down projections of the selected experts (same scheme, the
+//                 activations h as four E4M3 pieces) and of the bf16 shared
+//                 expert (mma.sync bf16, h as hi + lo bf16)
 //   combine       y = S + sum_j w_j o_j in slot order, rounded once
-// Prior art: the kimi-k3-in-c project card ("P053"), core features (routed
-// experts multiplied directly on the packed nibbles, never dequantised to a
-// resident buffer); the tutorial page's section 2.4 moe_forward (route, then
-// per selected expert FFN, then weighted combine).
+// The routed weights are never expanded into a resident buffer: each 4-bit
+// code goes from shared memory to a register operand and into the MMA (the
+// kimi-k3-in-c project card ("P053"), core features: multiply directly on the
+// packed nibbles).  Layer structure: the tutorial page's section 2.4
+// moe_forward (route, per selected expert FFN, weighted combine).
 #pragma once
 
 #include "common.cuh"
 #include "layout.cuh"
 
 namespace k3 {
+
+constexpr int kMaxStages = 3;
 
 // =========================================================== route_shared ==
 
@@ -38,6 +45,7 @@ struct RouteParams {
     const uint8_t *const *blobs;  // device array [E], null: no dispatch (route only)
     int32_t *idx_out;   // optional [Tc][k]
     float *w_out;       // optional [Tc][k]
+    int nwarps;         // streaming warps: 8 per CTA, CTAs 1.. of the grid
 };
 
 constexpr int kRouteThreads = 256;
@@ -101,13 +109,50 @@ __device__ void warp_topk(const float *row, int E, int k, int lane, int32_t *idx
     }
 }
 
+// Byte position of column c inside an even/odd-permuted row: within each
+// group of 8 columns the even ones come first, then the odd ones, matching the
+// even/odd nibble split of the MMA A operand.
+__device__ __forceinline__ int perm8(int c) { return (c & ~7) + ((c & 1) ? 4 : 0) + ((c & 7) >> 1); }
+
+// Per-token E4M3 prescale exponent of x and x * 2^s as two E4M3 pieces,
+// written to the workspace for the gate/up pass.  Run by one whole CTA.
+__device__ void build_x_pieces(const uint16_t *x, int Tc, int d, uint8_t *ws, const Layout &L) {
+    __shared__ int s_sig[kChunk];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int t = warp; t < Tc; t += nw) {
+        const uint16_t *xr = x + (size_t)t * d;
+        float mx = 0.f;
+        for (int j = lane; j < d; j += 32) mx = fmaxf(mx, fabsf(__uint_as_float((uint32_t)xr[j] << 16)));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) {
+            const int sg = e4m3_prescale(mx);
+            s_sig[t] = sg;
+            reinterpret_cast<int32_t *>(ws + L.sigx)[t] = sg;
+        }
+    }
+    __syncthreads();
+    uint8_t *xp = ws + L.xp;
+    for (int i = threadIdx.x; i < Tc * d; i += blockDim.x) {
+        const int t = i / d, c = i - t * d;
+        float v = __uint_as_float((uint32_t)x[i] << 16) * exp2i(s_sig[t]);
+        const uint32_t p0 = f32_to_e4m3_rn(v);
+        v -= e4m3_to_f32(p0);
+        const uint32_t p1 = f32_to_e4m3_rn(v);
+        xp[((size_t)t * 2 + 0) * d + perm8(c)] = (uint8_t)p0;
+        xp[((size_t)t * 2 + 1) * d + perm8(c)] = (uint8_t)p1;
+    }
+}
+
+// Top-k of every token of the chunk, then the dispatch: distinct experts in
+// ascending id, their token masks, the slot of each (expert, token), the
+// per-token E4M3 prescale of x, zeroed |h| maxima.  Run by one whole CTA.
 __device__ void topk_dispatch(const RouteParams &p, WsHeader *hdr) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Layout &L = p.L;
     float *logits = reinterpret_cast<float *>(p.ws + L.logits);
     int32_t *idx = reinterpret_cast<int32_t *>(p.ws + L.idx);
     float *wt = reinterpret_cast<float *>(p.ws + L.wt);
-    __threadfence();
     if (warp < p.Tc) {
         const int t = warp;
         const float *row = logits + (size_t)t * p.E;
@@ -123,17 +168,7 @@ __device__ void topk_dispatch(const RouteParams &p, WsHeader *hdr) {
         else warp_topk<32>(row, p.E, p.k, lane, i1, w1, i2, w2);
     }
     if (p.blobs == nullptr) return;  // route only: no dispatch
-    // per-token f16 prescale of x (used by the gate/up pass)
-    if (warp < p.Tc) {
-        const uint16_t *xr = p.x + (size_t)warp * p.d;
-        float mx = 0.f;
-        for (int j = lane; j < p.d; j += 32) mx = fmaxf(mx, fabsf(__uint_as_float((uint32_t)xr[j] << 16)));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) reinterpret_cast<int32_t *>(p.ws + L.sigx)[warp] = f16_prescale(mx);
-    }
     __syncthreads();
-    // distinct experts of the chunk, ascending expert id
     __shared__ uint32_t bitmap[32];
     __shared__ uint32_t prefix[32];
     __shared__ uint32_t umask[kChunk * 32];
@@ -172,7 +207,6 @@ __device__ void topk_dispatch(const RouteParams &p, WsHeader *hdr) {
         atomicOr(&umask[u], 1u << t);
     }
     __syncthreads();
-    const uint32_t U = hdr->n_unique;
     const uint8_t **ublob = reinterpret_cast<const uint8_t **>(p.ws + L.uniq_blob);
     uint32_t *gmask = reinterpret_cast<uint32_t *>(p.ws + L.uniq_mask);
     for (int w = threadIdx.x; w < nwords * 32; w += blockDim.x) {
@@ -187,135 +221,221 @@ __device__ void topk_dispatch(const RouteParams &p, WsHeader *hdr) {
             gmask[u] = umask[u];
         }
     }
-    (void)U;
 }
 
-__global__ void __launch_bounds__(kRouteThreads) route_shared_kernel(RouteParams p) {
-    extern __shared__ __align__(16) float xs[];  // [kRouteTok][d]
-    __shared__ float red[kRouteThreads / 32][2 * kRouteTok];
-    __shared__ int s_last;
-    WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + p.L.hdr);
-    float *logits = reinterpret_cast<float *>(p.ws + p.L.logits);
-    float *hs = reinterpret_cast<float *>(p.ws + p.L.hs);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int N = p.E + p.ffs;
-    const int G = gridDim.x;
-    const int u0 = (int)(((long long)blockIdx.x * N) / G);
-    const int u1 = (int)(((long long)(blockIdx.x + 1) * N) / G);
-    const int nrouter = max(0, min(u1, p.E) - u0);
-    const int d = p.d;
-    pdl_trigger();
+// Warp that holds chunk c when N chunks are split evenly over W warps
+// (warp j holds [floor(jN/W), floor((j+1)N/W))).
+__device__ __forceinline__ int chunk_owner(long long c, long long N, int W) {
+    return (int)(((c + 1) * (long long)W - 1) / N);
+}
 
-    for (int t0 = 0; t0 < p.Tc; t0 += kRouteTok) {
-        const int nt = min(kRouteTok, p.Tc - t0);
-        __syncthreads();
-        for (int i = threadIdx.x; i < nt * d / 2; i += blockDim.x) {
-            int t = (2 * i) / d, j = (2 * i) % d;
-            uint32_t w = reinterpret_cast<const uint32_t *>(p.x + (size_t)(t0 + t) * d)[j / 2];
-            xs[t * d + j] = bf16_lo(w);
-            xs[t * d + j + 1] = bf16_hi(w);
-        }
-        __syncthreads();
-        const bool last_pass = (t0 + kRouteTok >= p.Tc);
-        for (int u = u0; u < u1; ++u) {
-            float a0[kRouteTok], a1[kRouteTok];
+// Row sums are ready: write the logit (router) or the SwiGLU activation (shared).
+template <bool ROUTER>
+__device__ __forceinline__ void finalize_row(const RouteParams &p, WsHeader *hdr, int row, int t0,
+                                             int nt, const float *v0, const float *v1) {
+    if (ROUTER) {
+        float *logits = reinterpret_cast<float *>(p.ws + p.L.logits);
+        const float b = p.bias ? p.bias[row] : 0.f;
+        for (int t = 0; t < nt; ++t) logits[(size_t)(t0 + t) * p.E + row] = v0[t] + b;
+    } else {
+        float *hs = reinterpret_cast<float *>(p.ws + p.L.hs);
+        for (int t = 0; t < nt; ++t) hs[(size_t)(t0 + t) * p.ffs + row] = silu_mul(v0[t], v1[t]);
+    }
+}
+
+// One warp streams its slice of a phase's rows (router rows, or shared rows
+// = [W_g,s row | W_u,s row]); every row is d*4 bytes = d/4 chunks of 16 B.
+// Returns (in lane 0) the number of rows this warp finished.
+template <bool ROUTER>
+__device__ int stream_phase(const RouteParams &p, WsHeader *hdr, const float *xs, int t0, int nt,
+                            int pass, int nrows, int j, int lane) {
+    int finished = 0;
+    const int d = p.d;
+    const int cpr = d / 4;
+    const int W = p.nwarps;
+    const long long N = (long long)nrows * cpr;
+    long long c = (long long)j * N / W;
+    const long long cend = (long long)(j + 1) * N / W;
+    const int NR = p.E + p.ffs;
+    const int row_base = ROUTER ? 0 : p.E;
+    float *part = reinterpret_cast<float *>(p.ws + p.L.part);    // [2][NR][kMaxSeg][8]
+    uint32_t *cnt = reinterpret_cast<uint32_t *>(p.ws + p.L.cnt);  // [2][NR]
+    while (c < cend) {
+        const int r = (int)(c / cpr);
+        const int a = (int)(c - (long long)r * cpr);
+        const int b = (int)min((long long)cpr, (long long)a + (cend - c));
+        float a0[kRouteTok], a1[kRouteTok];
 #pragma unroll
-            for (int t = 0; t < kRouteTok; ++t) a0[t] = a1[t] = 0.f;
-            if (u < p.E) {
-                // router row u: 4 fp32 weights per 16-byte chunk
-                const float4 *wr = reinterpret_cast<const float4 *>(p.wr + (size_t)u * d);
-                const int nc = d / 4;
-#pragma unroll 4
-                for (int c = threadIdx.x; c < nc; c += kRouteThreads) {
-                    float4 w = __ldg(wr + c);
+        for (int t = 0; t < kRouteTok; ++t) a0[t] = a1[t] = 0.f;
+        if (ROUTER) {
+            const float4 *wrow = reinterpret_cast<const float4 *>(p.wr + (size_t)r * d);
+            for (int cc = a + lane; cc < b; cc += 32 * 8) {
+                float4 w[8];
 #pragma unroll
-                    for (int t = 0; t < kRouteTok; ++t) {
-                        if (t < nt) {
-                            float4 xv = *reinterpret_cast<const float4 *>(xs + t * d + 4 * c);
-                            a0[t] = fmaf(w.x, xv.x, a0[t]);
-                            a0[t] = fmaf(w.y, xv.y, a0[t]);
-                            a0[t] = fmaf(w.z, xv.z, a0[t]);
-                            a0[t] = fmaf(w.w, xv.w, a0[t]);
-                        }
-                    }
+                for (int u = 0; u < 8; ++u) {
+                    const int ci = cc + 32 * u;
+                    w[u] = ci < b ? __ldg(wrow + ci) : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-            } else {
-                // shared expert rows r of W_g,s and W_u,s: 8 bf16 per chunk
-                const int r = u - p.E;
-                const uint4 *wg = reinterpret_cast<const uint4 *>(p.swg + (size_t)r * d);
-                const uint4 *wu = reinterpret_cast<const uint4 *>(p.swu + (size_t)r * d);
-                const int nc = d / 8;
-#pragma unroll 2
-                for (int c = threadIdx.x; c < nc; c += kRouteThreads) {
-                    uint4 g = __ldg(wg + c), v = __ldg(wu + c);
-                    float gf[8] = {bf16_lo(g.x), bf16_hi(g.x), bf16_lo(g.y), bf16_hi(g.y),
-                                   bf16_lo(g.z), bf16_hi(g.z), bf16_lo(g.w), bf16_hi(g.w)};
-                    float uf[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                                   bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
 #pragma unroll
-                    for (int t = 0; t < kRouteTok; ++t) {
-                        if (t < nt) {
-                            float4 x0 = *reinterpret_cast<const float4 *>(xs + t * d + 8 * c);
-                            float4 x1 = *reinterpret_cast<const float4 *>(xs + t * d + 8 * c + 4);
-                            float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                for (int u = 0; u < 8; ++u) {
+                    const int ci = cc + 32 * u;
+                    if (ci < b) {
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                a0[t] = fmaf(gf[i], xv[i], a0[t]);
-                                a1[t] = fmaf(uf[i], xv[i], a1[t]);
+                        for (int t = 0; t < kRouteTok; ++t) {
+                            if (t < nt) {
+                                const float4 xv = *reinterpret_cast<const float4 *>(xs + t * d + 4 * ci);
+                                a0[t] = fmaf(w[u].x, xv.x, a0[t]);
+                                a0[t] = fmaf(w[u].y, xv.y, a0[t]);
+                                a0[t] = fmaf(w[u].z, xv.z, a0[t]);
+                                a0[t] = fmaf(w[u].w, xv.w, a0[t]);
                             }
                         }
                     }
                 }
             }
-            // block reduction, fixed order
+        } else {
+            const int half = cpr / 2;  // chunks of one bf16 row
+            const uint4 *wg = reinterpret_cast<const uint4 *>(p.swg + (size_t)r * d);
+            const uint4 *wu = reinterpret_cast<const uint4 *>(p.swu + (size_t)r * d);
+            for (int cc = a + lane; cc < b; cc += 32 * 4) {
+                uint4 w[4];
 #pragma unroll
-            for (int t = 0; t < kRouteTok; ++t) {
+                for (int u = 0; u < 4; ++u) {
+                    const int ci = cc + 32 * u;
+                    w[u] = ci < b ? __ldg(ci < half ? wg + ci : wu + (ci - half)) : make_uint4(0, 0, 0, 0);
+                }
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    a0[t] += __shfl_xor_sync(0xffffffffu, a0[t], o);
-                    a1[t] += __shfl_xor_sync(0xffffffffu, a1[t], o);
-                }
-            }
-            if (lane == 0) {
+                for (int u = 0; u < 4; ++u) {
+                    const int ci = cc + 32 * u;
+                    if (ci < b) {
+                        const bool is_g = ci < half;
+                        const int col = 8 * (is_g ? ci : ci - half);
+                        const float wf[8] = {bf16_lo(w[u].x), bf16_hi(w[u].x), bf16_lo(w[u].y),
+                                             bf16_hi(w[u].y), bf16_lo(w[u].z), bf16_hi(w[u].z),
+                                             bf16_lo(w[u].w), bf16_hi(w[u].w)};
 #pragma unroll
-                for (int t = 0; t < kRouteTok; ++t) {
-                    red[warp][t] = a0[t];
-                    red[warp][kRouteTok + t] = a1[t];
-                }
-            }
-            __syncthreads();
-            if (threadIdx.x < nt) {
-                const int t = threadIdx.x;
-                float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-                for (int w = 0; w < kRouteThreads / 32; ++w) {
-                    s0 += red[w][t];
-                    s1 += red[w][kRouteTok + t];
-                }
-                if (u < p.E) {
-                    if (p.bias) s0 += p.bias[u];
-                    logits[(size_t)(t0 + t) * p.E + u] = s0;
-                } else {
-                    hs[(size_t)(t0 + t) * p.ffs + (u - p.E)] = silu_mul(s0, s1);
-                }
-            }
-            __syncthreads();
-            // after this CTA's last router row of the last pass: count it, and the
-            // CTA that completes the count runs top-k + dispatch
-            if (last_pass && nrouter > 0 && u == u0 + nrouter - 1) {
-                if (threadIdx.x == 0) {
-                    __threadfence();
-                    uint32_t old = atomicAdd(&hdr->router_done, (uint32_t)nrouter);
-                    s_last = (old + (uint32_t)nrouter == (uint32_t)p.E);
-                }
-                __syncthreads();
-                if (s_last) {
-                    topk_dispatch(p, hdr);
-                    __syncthreads();
-                    if (threadIdx.x == 0) hdr->router_done = 0u;
+                        for (int t = 0; t < kRouteTok; ++t) {
+                            if (t < nt) {
+                                const float4 x0 = *reinterpret_cast<const float4 *>(xs + t * d + col);
+                                const float4 x1 = *reinterpret_cast<const float4 *>(xs + t * d + col + 4);
+                                float s = 0.f;
+                                s = fmaf(wf[0], x0.x, s);
+                                s = fmaf(wf[1], x0.y, s);
+                                s = fmaf(wf[2], x0.z, s);
+                                s = fmaf(wf[3], x0.w, s);
+                                s = fmaf(wf[4], x1.x, s);
+                                s = fmaf(wf[5], x1.y, s);
+                                s = fmaf(wf[6], x1.z, s);
+                                s = fmaf(wf[7], x1.w, s);
+                                if (is_g) a0[t] += s;
+                                else a1[t] += s;
+                            }
+                        }
+                    }
                 }
             }
         }
+#pragma unroll
+        for (int t = 0; t < kRouteTok; ++t) {
+            if (t < nt) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    a0[t] += __shfl_xor_sync(0xffffffffu, a0[t], o);
+                    if (!ROUTER) a1[t] += __shfl_xor_sync(0xffffffffu, a1[t], o);
+                }
+            }
+        }
+        if (a == 0 && b == cpr) {
+            if (lane == 0) {
+                finalize_row<ROUTER>(p, hdr, r, t0, nt, a0, a1);
+                ++finished;
+            }
+        } else if (lane == 0) {
+            // the row is split between warps: park the partial; the last to
+            // arrive sums all parts in slot order and finishes the row
+            const long long rs = (long long)r * cpr;
+            const int first = chunk_owner(rs, N, W);
+            const int nseg = chunk_owner(rs + cpr - 1, N, W) - first + 1;
+            const int slot = j - first;
+            const int grow = row_base + r;
+            float *pp = part + (((size_t)(pass & 1) * NR + grow) * kMaxSeg) * 8;
+            uint32_t *pc = cnt + (size_t)(pass & 1) * NR + grow;
+#pragma unroll
+            for (int t = 0; t < kRouteTok; ++t) {
+                pp[slot * 8 + 2 * t] = a0[t];
+                pp[slot * 8 + 2 * t + 1] = a1[t];
+            }
+            const uint32_t old = atom_add_acq_rel(pc, 1u);  // publish the part, see the others
+            if (old == (uint32_t)(nseg - 1)) {
+                float s0[kRouteTok], s1[kRouteTok];
+#pragma unroll
+                for (int t = 0; t < kRouteTok; ++t) s0[t] = s1[t] = 0.f;
+                for (int sl = 0; sl < nseg; ++sl) {
+#pragma unroll
+                    for (int t = 0; t < kRouteTok; ++t) {
+                        s0[t] += __ldcg(pp + sl * 8 + 2 * t);
+                        s1[t] += __ldcg(pp + sl * 8 + 2 * t + 1);
+                    }
+                }
+                *pc = 0u;
+                finalize_row<ROUTER>(p, hdr, r, t0, nt, s0, s1);
+                ++finished;
+            }
+        }
+        c += b - a;
+    }
+    return finished;
+}
+
+__global__ void __launch_bounds__(kRouteThreads) route_shared_kernel(RouteParams p) {
+    extern __shared__ __align__(16) float xs[];  // [kRouteTok][d]
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + p.L.hdr);
+    pdl_trigger();
+    const int npass = (p.Tc + kRouteTok - 1) / kRouteTok;
+    if (blockIdx.x == 0) {
+        // x pieces for the gate/up pass need no routing: build them first
+        if (p.blobs != nullptr) build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L);
+        // wait (bounded) for every router row of every pass, then route and dispatch
+        __shared__ int s_ok;
+        if (threadIdx.x == 0) {
+            const uint32_t target = (uint32_t)(p.E * npass);
+            const uint64_t t0 = globaltimer();
+            int ok = 1;
+            while (ld_acquire(&hdr->router_done) < target) {
+                __nanosleep(128);
+                if (globaltimer() - t0 > kWaitLimitNs) {
+                    set_status(hdr, kStTimeout);
+                    ok = 0;
+                    break;
+                }
+            }
+            s_ok = ok;
+        }
+        __syncthreads();
+        if (!s_ok) return;
+        topk_dispatch(p, hdr);
+        __syncthreads();
+        if (threadIdx.x == 0) hdr->router_done = 0u;
+        return;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j = (blockIdx.x - 1) * (kRouteThreads / 32) + warp;
+    const int d = p.d;
+    for (int pass = 0; pass < npass; ++pass) {
+        const int t0 = pass * kRouteTok;
+        const int nt = min(kRouteTok, p.Tc - t0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < nt * d / 2; i += blockDim.x) {
+            const int t = (2 * i) / d, c = (2 * i) % d;
+            const uint32_t w = reinterpret_cast<const uint32_t *>(p.x + (size_t)(t0 + t) * d)[c / 2];
+            xs[t * d + c] = bf16_lo(w);
+            xs[t * d + c + 1] = bf16_hi(w);
+        }
+        __syncthreads();
+        const int nr = stream_phase<true>(p, hdr, xs, t0, nt, pass, p.E, j, lane);
+        // one release per warp: its logits are visible before they are counted
+        if (lane == 0 && nr > 0) red_add_release(&hdr->router_done, (uint32_t)nr);
+        if (p.ffs > 0) stream_phase<false>(p, hdr, xs, t0, nt, pass, p.ffs, j, lane);
     }
 }
 
@@ -326,30 +446,52 @@ struct GUParams {
     int Tc, d, ff;
     uint8_t *ws;
     Layout L;
+    int nst;  // pipeline stages
 };
 
 constexpr int kGUThreads = 512;  // 16 warps split each item's d columns
-constexpr int kStages = 3;
 
 __host__ __device__ inline int gu_pitch(int d) { return d / 2 + 16; }
+__host__ __device__ inline int gu_scp(int d) { return d / 32 + 1; }
 __host__ __device__ inline int gu_stage_bytes(int d) {
-    return (16 * gu_pitch(d) + 2 * 8 * (d / 32) + 127) & ~127;
+    return (16 * gu_pitch(d) + 16 * (d / 32) + 127) & ~127;
 }
-__host__ __device__ inline int gu_smem_bytes(int d) {
-    return kStages * gu_stage_bytes(d) + 2 * 16 * 8 * kChunk * 2 * 4 + kStages * 8;
+__host__ __device__ inline int gu_red_floats() { return 16 * 8 * kChunk * 2; }
+__host__ __device__ inline int gu_smem_bytes(int d, int nst) {
+    return nst * gu_stage_bytes(d) + 2 * 16 * gu_scp(d) * 4 + 2 * gu_red_floats() * 4 +
+           kMaxStages * 8;
 }
 
-template <int NBW>
+// E8M0 bytes [rows][nb] of a stage -> fp32 [rows][SCP], all threads of the
+// CTA, walking (row, block) without divisions.
+__device__ __forceinline__ void convert_scales(const uint8_t *sc8, float *dst, int rows, int nb,
+                                               int scp, int nthreads) {
+    const int step_r = nthreads / nb, step_b = nthreads - step_r * nb;
+    int r = threadIdx.x / nb, b = threadIdx.x - r * nb;
+    for (int i = threadIdx.x; i < rows * nb; i += nthreads) {
+        dst[r * scp + b] = e8m0_to_f32(sc8[i]);
+        r += step_r;
+        b += step_b;
+        if (b >= nb) {
+            b -= nb;
+            ++r;
+        }
+    }
+}
+
+// NBW: blocks of 32 columns per warp (>= d/32/16); NG: token groups of 4.
+template <int NBW, int NG>
 __global__ void __launch_bounds__(kGUThreads, 1) expert_gu_kernel(GUParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const int d = p.d, ff = p.ff, nb = d / 32;
-    const int P = gu_pitch(d), SB = gu_stage_bytes(d);
-    float *red = reinterpret_cast<float *>(smem + kStages * SB);  // [2][16][8][kChunk][2]
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * SB + 2 * 16 * 8 * kChunk * 2 * 4);
+    const int d = p.d, ff = p.ff, nb = d / 32, nst = p.nst;
+    const int P = gu_pitch(d), SB = gu_stage_bytes(d), SCP = gu_scp(d);
+    float *scf = reinterpret_cast<float *>(smem + nst * SB);  // [2][16][SCP]
+    float *red = scf + 2 * 16 * SCP;                           // [2][16][8][kChunk][2]
+    uint64_t *full = reinterpret_cast<uint64_t *>(red + 2 * gu_red_floats());
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + p.L.hdr);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < nst; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -371,22 +513,25 @@ __global__ void __launch_bounds__(kGUThreads, 1) expert_gu_kernel(GUParams p) {
     const int k = p.L.k;
     const size_t mat = (size_t)d * ff;
 
-    // B fragments: token n = g, columns 8q..8q+7 of each of this warp's blocks,
-    // as f16 prescaled by 2^sigx[n] (exact for the bf16 inputs in range)
-    uint32_t bx[NBW][2][2];
+    // B operand: column n = g of token group ng is token 4*ng + g/2, piece g&1
+    // of its prescaled x (x * 2^sigx = piece0 + piece1, E4M3).  Register 0
+    // holds the even columns 8q, 8q+2, 8q+4, 8q+6 of a block, register 1 the
+    // odd ones, matching the even/odd nibble split of the A operand.
+    uint32_t bx[NBW][NG][2];
     {
-        const bool tok_ok = g < p.Tc;
-        const float sc = tok_ok ? __uint_as_float((uint32_t)(127 + sigx[g]) << 23) : 0.f;
+        const uint8_t *xp = p.ws + p.L.xp;
 #pragma unroll
-        for (int i = 0; i < NBW; ++i) {
-            const int b = warp + 16 * i;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (tok_ok && b < nb)
-                v = *reinterpret_cast<const uint4 *>(p.x + (size_t)g * d + 32 * b + 8 * q);
-            bx[i][0][0] = pack_f16x2(bf16_lo(v.x) * sc, bf16_hi(v.x) * sc);
-            bx[i][0][1] = pack_f16x2(bf16_lo(v.y) * sc, bf16_hi(v.y) * sc);
-            bx[i][1][0] = pack_f16x2(bf16_lo(v.z) * sc, bf16_hi(v.z) * sc);
-            bx[i][1][1] = pack_f16x2(bf16_lo(v.w) * sc, bf16_hi(v.w) * sc);
+        for (int ng = 0; ng < NG; ++ng) {
+            const int t = 4 * ng + (g >> 1), piece = g & 1;
+#pragma unroll
+            for (int i = 0; i < NBW; ++i) {
+                const int b = warp + 16 * i;
+                uint2 v = make_uint2(0, 0);
+                if (t < p.Tc && b < nb)
+                    v = __ldcg(reinterpret_cast<const uint2 *>(xp + ((size_t)t * 2 + piece) * d + 32 * b + 8 * q));
+                bx[i][ng][0] = v.x;
+                bx[i][ng][1] = v.y;
+            }
         }
     }
 
@@ -395,7 +540,7 @@ __global__ void __launch_bounds__(kGUThreads, 1) expert_gu_kernel(GUParams p) {
         const int u = it / nrg, rg = it - (it / nrg) * nrg;
         const uint8_t *blob = ublob[u];
         uint8_t *st = smem + s * SB;
-        const uint32_t bytes = (uint32_t)(16 * (d / 2) + 2 * 8 * (d / 32));
+        const uint32_t bytes = (uint32_t)(16 * (d / 2) + 16 * (d / 32));
         if (lane == 0) {
             fence_proxy_async();
             if (blob) mbar_arrive_expect_tx(&full[s], bytes);
@@ -419,14 +564,25 @@ __global__ void __launch_bounds__(kGUThreads, 1) expert_gu_kernel(GUParams p) {
     };
 
     if (warp == 0)
-        for (int s = 0; s < kStages && i0 + s < i1; ++s) issue(i0 + s, s);
+        for (int s = 0; s < nst && i0 + s < i1; ++s) issue(i0 + s, s);
 
+    // The scales of item it+1 are converted before the barrier that ends item
+    // it, so each item needs one barrier: it protects the stage being
+    // refilled, the reduction buffer and the next item's scales.
+    bool ok = true;
+    if (i0 < i1) {
+        ok = mbar_wait_bounded(&full[0], 0u, hdr);
+        convert_scales(smem + 16 * P, scf, 16, nb, SCP, kGUThreads);
+        __syncthreads();
+    }
     for (int it = i0; it < i1; ++it) {
-        const int s = (it - i0) % kStages;
-        const uint32_t par = (uint32_t)(((it - i0) / kStages) & 1);
-        const bool ok = mbar_wait_bounded(&full[s], par, hdr);
+        const int s = (it - i0) % nst;
         const uint8_t *st = smem + s * SB;
-        float ag0 = 0.f, ag1 = 0.f, au0 = 0.f, au1 = 0.f;
+        const float *sc = scf + ((it - i0) & 1) * 16 * SCP;
+        float *rb = red + ((it - i0) & 1) * gu_red_floats();
+        float ag[NG], au[NG];
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) ag[ng] = au[ng] = 0.f;
         if (ok) {
 #pragma unroll
             for (int i = 0; i < NBW; ++i) {
@@ -435,27 +591,32 @@ __global__ void __launch_bounds__(kGUThreads, 1) expert_gu_kernel(GUParams p) {
                     const uint32_t wg = *reinterpret_cast<const uint32_t *>(st + g * P + 16 * b + 4 * q);
                     const uint32_t wu =
                         *reinterpret_cast<const uint32_t *>(st + (8 + g) * P + 16 * b + 4 * q);
-                    const float fg = e8m0_to_f32(st[16 * P + g * (d / 32) + b]);
-                    const float fu = e8m0_to_f32(st[16 * P + 8 * (d / 32) + g * (d / 32) + b]);
-                    float c[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_f16(c, e2m1x2_to_f16x2(wg & 0xFFu), e2m1x2_to_f16x2(wu & 0xFFu),
-                            e2m1x2_to_f16x2((wg >> 8) & 0xFFu), e2m1x2_to_f16x2((wu >> 8) & 0xFFu),
-                            bx[i][0][0], bx[i][0][1]);
-                    mma_f16(c, e2m1x2_to_f16x2((wg >> 16) & 0xFFu), e2m1x2_to_f16x2((wu >> 16) & 0xFFu),
-                            e2m1x2_to_f16x2(wg >> 24), e2m1x2_to_f16x2(wu >> 24), bx[i][1][0],
-                            bx[i][1][1]);
-                    ag0 = fmaf(c[0], fg, ag0);
-                    ag1 = fmaf(c[1], fg, ag1);
-                    au0 = fmaf(c[2], fu, au0);
-                    au1 = fmaf(c[3], fu, au1);
+                    const uint32_t a0 = e2m1_even_to_e4m3(wg), a1 = e2m1_even_to_e4m3(wu);
+                    const uint32_t a2 = e2m1_odd_to_e4m3(wg), a3 = e2m1_odd_to_e4m3(wu);
+                    const float fg = sc[g * SCP + b], fu = sc[(8 + g) * SCP + b];
+#pragma unroll
+                    for (int ng = 0; ng < NG; ++ng) {
+                        float c[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_e4m3(c, a0, a1, a2, a3, bx[i][ng][0], bx[i][ng][1]);
+                        ag[ng] = fmaf(c[0] + c[1], fg, ag[ng]);
+                        au[ng] = fmaf(c[2] + c[3], fu, au[ng]);
+                    }
                 }
             }
         }
-        float *rb = red + ((it - i0) & 1) * (16 * 8 * kChunk * 2);
-        *reinterpret_cast<float2 *>(rb + ((warp * 8 + g) * kChunk + 2 * q) * 2) = make_float2(ag0, au0);
-        *reinterpret_cast<float2 *>(rb + ((warp * 8 + g) * kChunk + 2 * q + 1) * 2) = make_float2(ag1, au1);
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng)
+            *reinterpret_cast<float2 *>(rb + ((warp * 8 + g) * kChunk + 4 * ng + q) * 2) =
+                make_float2(ag[ng], au[ng]);
+        bool ok_next = true;
+        if (it + 1 < i1) {
+            const int sn = (it + 1 - i0) % nst;
+            ok_next = mbar_wait_bounded(&full[sn], (uint32_t)(((it + 1 - i0) / nst) & 1), hdr);
+            convert_scales(smem + sn * SB + 16 * P, scf + ((it + 1 - i0) & 1) * 16 * SCP, 16, nb,
+                           SCP, kGUThreads);
+        }
         __syncthreads();
-        if (warp == 0 && it + kStages < i1) issue(it + kStages, s);
+        if (warp == 0 && it + nst < i1) issue(it + nst, s);
         if (threadIdx.x < 8 * kChunk) {
             const int r = threadIdx.x / kChunk, t = threadIdx.x % kChunk;
             const int u = it / nrg, rg = it - u * nrg;
@@ -463,17 +624,19 @@ __global__ void __launch_bounds__(kGUThreads, 1) expert_gu_kernel(GUParams p) {
                 float sg = 0.f, su = 0.f;
 #pragma unroll
                 for (int w = 0; w < 16; ++w) {
-                    float2 v = *reinterpret_cast<const float2 *>(rb + ((w * 8 + r) * kChunk + t) * 2);
+                    const float2 v = *reinterpret_cast<const float2 *>(rb + ((w * 8 + r) * kChunk + t) * 2);
                     sg += v.x;
                     su += v.y;
                 }
-                const float inv = __uint_as_float((uint32_t)(127 - sigx[t]) << 23);
+                // undo the 2^-6 of the E4M3 placement and the x prescale
+                const float inv = exp2i(6 - sigx[t]);
                 const float h = silu_mul(sg * inv, su * inv);
                 const int j = uslot[u * kChunk + t];
                 hbuf[((size_t)t * k + j) * ff + rg * 8 + r] = h;
                 atomicMax(&hmax[t * k + j], __float_as_uint(fabsf(h)));
             }
         }
+        ok = ok_next;
     }
 }
 
@@ -484,35 +647,50 @@ struct DownParams {
     const uint16_t *swd;  // bf16 [d][ffs] or null
     uint8_t *ws;
     Layout L;
+    int nst;
 };
 
 constexpr int kDownThreads = 512;
-constexpr int kDownRowsQ = 32;  // MXFP4 rows per item
-constexpr int kDownRowsS = 16;  // bf16 shared rows per item
+constexpr int kDownRowsQ = 64;  // MXFP4 rows per routed item (4 row groups)
+constexpr int kDownRowsS = 16;  // bf16 rows per shared item
 
 __host__ __device__ inline int dn_pitch_q(int ff) { return ff / 2 + 16; }
 __host__ __device__ inline int dn_pitch_s(int ffs) { return 2 * ffs + 64; }
+__host__ __device__ inline int dn_scp(int ff) { return ff / 32 + 1; }
+__host__ __device__ inline int dn_pc_pitch(int ff) { return ff + 32; }  // one (token, piece) row
 __host__ __device__ inline int dn_stage_bytes(int ff, int ffs) {
     int a = kDownRowsQ * dn_pitch_q(ff) + kDownRowsQ * (ff / 32);
     int b = ffs > 0 ? kDownRowsS * dn_pitch_s(ffs) : 0;
     return ((a > b ? a : b) + 127) & ~127;
 }
-__host__ __device__ inline int dn_smem_bytes(int ff, int ffs) {
-    return kStages * dn_stage_bytes(ff, ffs) + 2 * 16 * kDownRowsQ * kChunk * 4 + kStages * 8;
+// partial sums of one pass: routed [4 K-quarters][64 rows][4 tokens][2 halves],
+// shared [16 warps][16 rows][8 tokens]
+__host__ __device__ inline int dn_red_floats() {
+    const int a = 16 * 16 * kChunk, b = 4 * kDownRowsQ * 4 * 2;
+    return a > b ? a : b;
+}
+__host__ __device__ inline int dn_smem_bytes(int ff, int ffs, int nst) {
+    return nst * dn_stage_bytes(ff, ffs) + 2 * kDownRowsQ * dn_scp(ff) * 4 +
+           16 * dn_pc_pitch(ff) + 2 * dn_red_floats() * 4 + kMaxStages * 8;
 }
 
-template <int NBC>
+// NBQ: blocks per K-quarter for routed items (>= ff/32/4); NBS: blocks per warp
+// for shared items (>= ffs/32/16).
+template <int NBQ, int NBS>
 __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const int d = p.d, ff = p.ff, ffs = p.ffs;
+    const int d = p.d, ff = p.ff, ffs = p.ffs, nst = p.nst;
     const int SB = dn_stage_bytes(ff, ffs);
-    const int PQ = dn_pitch_q(ff), PS = dn_pitch_s(ffs);
-    float *red = reinterpret_cast<float *>(smem + kStages * SB);  // [2][16][32][kChunk]
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * SB + 2 * 16 * kDownRowsQ * kChunk * 4);
+    const int PQ = dn_pitch_q(ff), PS = dn_pitch_s(ffs), SCP = dn_scp(ff), PCP = dn_pc_pitch(ff);
+    const int nbk = ff / 32;
+    float *scf = reinterpret_cast<float *>(smem + nst * SB);                // [2][64][SCP]
+    uint8_t *pcs = reinterpret_cast<uint8_t *>(scf + 2 * kDownRowsQ * SCP);  // [4 tok][4 piece][PCP]
+    float *red = reinterpret_cast<float *>(pcs + 16 * PCP);                 // [2][dn_red_floats]
+    uint64_t *full = reinterpret_cast<uint64_t *>(red + 2 * dn_red_floats());
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + p.L.hdr);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < nst; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -521,8 +699,8 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
 
     const int k = p.L.k;
     const int U = (int)hdr->n_unique;
-    const int nq = d / kDownRowsQ;                 // items per routed expert
-    const int ns = ffs > 0 ? d / kDownRowsS : 0;   // shared items
+    const int nq = d / kDownRowsQ;
+    const int ns = ffs > 0 ? d / kDownRowsS : 0;
     const int N = U * nq + ns;
     const int G = gridDim.x;
     const int i0 = (int)(((long long)blockIdx.x * N) / G);
@@ -553,6 +731,7 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
             if (!blob) return;
             const uint8_t *dn = blob + mat + mat / 16;  // W_d nibble plane
             bulk_g2s(st + lane * PQ, dn + (size_t)(r0 + lane) * (ff / 2), ff / 2, &full[s]);
+            bulk_g2s(st + (lane + 32) * PQ, dn + (size_t)(r0 + lane + 32) * (ff / 2), ff / 2, &full[s]);
             if (lane == 0)
                 bulk_g2s(st + kDownRowsQ * PQ, dn + mat / 2 + (size_t)r0 * (ff / 32),
                          kDownRowsQ * (ff / 32), &full[s]);
@@ -569,179 +748,234 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
     };
 
     if (warp == 0)
-        for (int s = 0; s < kStages && i0 + s < i1; ++s) issue(i0 + s, s);
+        for (int s = 0; s < nst && i0 + s < i1; ++s) issue(i0 + s, s);
 
-    // B fragments of the current expert: [block][n-group][step][2]
-    uint32_t bh[NBC][2][2][2];
-    int cur = -1;     // current expert slot (U = shared)
-    int ntok = 0;     // tokens of the current expert
-    int tok[kChunk];  // token of each column pair
+    // routed items: warp = (row group rgw, K-quarter kq); column n = g of
+    // token group ng is token 2*ng + g/4 of the pass, piece g&3 of its h
+    const int rgw = warp & 3, kq = warp >> 2;
+    uint32_t bq[NBQ][2][2];
+    uint32_t bs[NBS][2][2][2];  // shared: [block][token group][step][2], bf16 hi/lo
+    int cur_key = -1;           // (expert, pass) whose pieces are loaded
+    bool shared_loaded = false;
+
+    // Reduce one pass of a routed item (tokens tb.. of the expert) into ob.
+    auto reduce_routed = [&](const float *rb, int u, int it, int tb, int nt, const int *tok) {
+        for (int i = threadIdx.x; i < kDownRowsQ * nt; i += kDownThreads) {
+            const int r = i / nt, mi = i - r * nt;
+            float sum = 0.f;
 #pragma unroll
-    for (int i = 0; i < kChunk; ++i) tok[i] = 0;
+            for (int qq = 0; qq < 4; ++qq)
+                sum += rb[((qq * kDownRowsQ + r) * 4 + mi) * 2] + rb[((qq * kDownRowsQ + r) * 4 + mi) * 2 + 1];
+            const int t = tok[tb + mi];
+            const int j = uslot[u * kChunk + t];
+            const int sgm = e4m3_prescale(__uint_as_float(__ldcg(hmax + t * k + j)));
+            const int r0 = (it - u * nq) * kDownRowsQ;
+            ob[((size_t)t * (k + 1) + 1 + j) * d + r0 + r] = sum * exp2i(6 - sgm);
+        }
+    };
 
+    // The E8M0 scales of item it+1 are converted before the barrier that ends
+    // item it: one barrier per item protects the refilled stage, the
+    // reduction buffer and the next item's scales.
+    bool ok = true;
+    if (i0 < i1) {
+        ok = mbar_wait_bounded(&full[0], 0u, hdr);
+        if (i0 < U * nq) convert_scales(smem + kDownRowsQ * PQ, scf, kDownRowsQ, nbk, SCP, kDownThreads);
+        __syncthreads();
+    }
     for (int it = i0; it < i1; ++it) {
         const bool shared_item = it >= U * nq;
         const int u = shared_item ? U : it / nq;
-        const int K = shared_item ? ffs : ff;
-        const int nbk = K / 32;
-        if (u != cur) {
-            cur = u;
-            // token list of this expert
-            uint32_t m = shared_item ? ((1u << p.Tc) - 1u) : umask[u];
+        const int s = (it - i0) % nst;
+        const uint8_t *st = smem + s * SB;
+        const float *sc = scf + ((it - i0) & 1) * kDownRowsQ * SCP;
+        float *rb = red + ((it - i0) & 1) * dn_red_floats();
+        const bool valid = ok && (shared_item || ublob[u] != nullptr);
+        int ntok;
+        int tok[kChunk];
+        if (!shared_item) {
+            const uint32_t m = umask[u];
             ntok = 0;
 #pragma unroll
             for (int t = 0; t < kChunk; ++t)
                 if ((m >> t) & 1u) tok[ntok++] = t;
+        } else {
+            ntok = p.Tc;
 #pragma unroll
-            for (int gi = 0; gi < 2; ++gi) {
-                const int mi = gi * 4 + (g >> 1);
-                const bool lo_part = g & 1;
-                const bool col_ok = mi < ntok && (shared_item || ublob[u] != nullptr);
-                int t = 0, j = 0;
-                float sc = 1.f;
-                if (col_ok) {
-                    t = tok[mi];
-                    if (!shared_item) {
-                        j = uslot[u * kChunk + t];
-                        const int sg = f16_prescale(__uint_as_float(__ldcg(hmax + t * k + j)));
-                        sc = __uint_as_float((uint32_t)(127 + sg) << 23);
-                    }
-                }
-                const float *src = shared_item ? hs + (size_t)t * ffs : hbuf + ((size_t)t * k + j) * ff;
+            for (int t = 0; t < kChunk; ++t) tok[t] = t;
+        }
+        const int npass = shared_item ? 1 : (ntok + 3) / 4;
+        for (int pass = 0; pass < npass; ++pass) {
+            const int tb = pass * 4;
+            const int nt = min(4, ntok - tb);
+            if (!shared_item) {
+                const int key = u * 2 + pass;
+                if (key != cur_key) {
+                    // h of up to 4 of this expert's tokens as four E4M3 pieces in
+                    // smem, each lane's 8 bytes of a block being the even then the
+                    // odd columns of its 8-column group
+                    __syncthreads();  // earlier reads of the pieces are done
+                    for (int i = threadIdx.x; i < nt * ff; i += kDownThreads) {
+                        const int mi = i / ff, c = i - mi * ff;
+                        float v = 0.f;
+                        if (ublob[u] != nullptr) {
+                            const int t = tok[tb + mi];
+                            const int j = uslot[u * kChunk + t];
+                            const int sgm = e4m3_prescale(__uint_as_float(__ldcg(hmax + t * k + j)));
+                            v = __ldcg(hbuf + ((size_t)t * k + j) * ff + c) * exp2i(sgm);
+                        }
+                        const int off = perm8(c);
 #pragma unroll
-                for (int i = 0; i < NBC; ++i) {
-                    const int b = warp + 16 * i;
-                    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    if (col_ok && b < nbk) {
-                        float4 a = __ldcg(reinterpret_cast<const float4 *>(src + 32 * b + 8 * q));
-                        float4 c = __ldcg(reinterpret_cast<const float4 *>(src + 32 * b + 8 * q + 4));
-                        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-                        v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
-                    }
-                    uint32_t r[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float x0 = v[2 * e] * sc, x1 = v[2 * e + 1] * sc;
-                        if (shared_item) {
-                            __nv_bfloat162 hi = __floats2bfloat162_rn(x0, x1);
-                            if (!lo_part) {
-                                r[e] = *reinterpret_cast<uint32_t *>(&hi);
-                            } else {
-                                float2 hf = __bfloat1622float2(hi);
-                                r[e] = pack_bf16x2(x0 - hf.x, x1 - hf.y);
-                            }
-                        } else {
-                            __half2 hi = __floats2half2_rn(x0, x1);
-                            if (!lo_part) {
-                                r[e] = *reinterpret_cast<uint32_t *>(&hi);
-                            } else {
-                                float2 hf = __half22float2(hi);
-                                r[e] = pack_f16x2(x0 - hf.x, x1 - hf.y);
-                            }
+                        for (int pc = 0; pc < 4; ++pc) {
+                            const uint32_t b8 = f32_to_e4m3_rn(v);
+                            pcs[(mi * 4 + pc) * PCP + off] = (uint8_t)b8;
+                            v -= e4m3_to_f32(b8);
                         }
                     }
-                    bh[i][gi][0][0] = r[0];
-                    bh[i][gi][0][1] = r[1];
-                    bh[i][gi][1][0] = r[2];
-                    bh[i][gi][1][1] = r[3];
+                    __syncthreads();
+#pragma unroll
+                    for (int ng = 0; ng < 2; ++ng) {
+                        const int mi = 2 * ng + (g >> 2), pc = g & 3;
+#pragma unroll
+                        for (int i = 0; i < NBQ; ++i) {
+                            const int b = kq + 4 * i;
+                            uint2 v = make_uint2(0, 0);
+                            if (b < nbk && mi < nt)
+                                v = *reinterpret_cast<const uint2 *>(pcs + (mi * 4 + pc) * PCP + b * 32 + q * 8);
+                            bq[i][ng][0] = v.x;
+                            bq[i][ng][1] = v.y;
+                        }
+                    }
+                    cur_key = key;
                 }
+            } else if (!shared_loaded) {
+                // shared expert: h as bf16 hi + lo; token group ng = tokens 4ng..4ng+3
+#pragma unroll
+                for (int ng = 0; ng < 2; ++ng) {
+                    const int t = 4 * ng + (g >> 1);
+                    const bool lo_part = g & 1;
+                    const bool col_ok = t < p.Tc;
+#pragma unroll
+                    for (int i = 0; i < NBS; ++i) {
+                        const int b = warp + 16 * i;
+                        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        if (col_ok && b < ffs / 32) {
+                            const float *src = hs + (size_t)t * ffs + 32 * b + 8 * q;
+                            const float4 a = __ldcg(reinterpret_cast<const float4 *>(src));
+                            const float4 c = __ldcg(reinterpret_cast<const float4 *>(src + 4));
+                            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+                            v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
+                        }
+                        uint32_t r[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            __nv_bfloat162 hi = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+                            if (!lo_part) {
+                                r[e] = *reinterpret_cast<uint32_t *>(&hi);
+                            } else {
+                                const float2 hf = __bfloat1622float2(hi);
+                                r[e] = pack_bf16x2(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
+                            }
+                        }
+                        bs[i][ng][0][0] = r[0];
+                        bs[i][ng][0][1] = r[1];
+                        bs[i][ng][1][0] = r[2];
+                        bs[i][ng][1][1] = r[3];
+                    }
+                }
+                shared_loaded = true;
             }
-        }
-        const int ngroups = ntok > 4 ? 2 : 1;
-        const int s = (it - i0) % kStages;
-        const uint32_t par = (uint32_t)(((it - i0) / kStages) & 1);
-        const bool ok = mbar_wait_bounded(&full[s], par, hdr);
-        const uint8_t *st = smem + s * SB;
-        float acc[2][2][2];  // [row group][n-group][row g / g+8]
+            float acc[2][2];  // [token group][row g / g+8]
 #pragma unroll
-        for (int a = 0; a < 2; ++a)
+            for (int a = 0; a < 2; ++a) acc[a][0] = acc[a][1] = 0.f;
+            if (valid && !shared_item) {
+                const int ng_n = (nt + 1) / 2;
+                const int ra = rgw * 16 + g;
 #pragma unroll
-            for (int b2 = 0; b2 < 2; ++b2) acc[a][b2][0] = acc[a][b2][1] = 0.f;
-        const bool valid = ok && (shared_item || ublob[u] != nullptr);
-        if (valid && !shared_item) {
-#pragma unroll
-            for (int i = 0; i < NBC; ++i) {
-                const int b = warp + 16 * i;
-                if (b < nbk) {
-#pragma unroll
-                    for (int rg = 0; rg < 2; ++rg) {
-                        const int ra = rg * 16 + g;
+                for (int i = 0; i < NBQ; ++i) {
+                    const int b = kq + 4 * i;
+                    if (b < nbk) {
                         const uint32_t w0 = *reinterpret_cast<const uint32_t *>(st + ra * PQ + 16 * b + 4 * q);
                         const uint32_t w1 = *reinterpret_cast<const uint32_t *>(st + (ra + 8) * PQ + 16 * b + 4 * q);
-                        const float f0 = e8m0_to_f32(st[kDownRowsQ * PQ + ra * (ff / 32) + b]);
-                        const float f1 = e8m0_to_f32(st[kDownRowsQ * PQ + (ra + 8) * (ff / 32) + b]);
-                        const uint32_t a00 = e2m1x2_to_f16x2(w0 & 0xFFu), a01 = e2m1x2_to_f16x2(w1 & 0xFFu);
-                        const uint32_t a02 = e2m1x2_to_f16x2((w0 >> 8) & 0xFFu), a03 = e2m1x2_to_f16x2((w1 >> 8) & 0xFFu);
-                        const uint32_t a10 = e2m1x2_to_f16x2((w0 >> 16) & 0xFFu), a11 = e2m1x2_to_f16x2((w1 >> 16) & 0xFFu);
-                        const uint32_t a12 = e2m1x2_to_f16x2(w0 >> 24), a13 = e2m1x2_to_f16x2(w1 >> 24);
+                        const uint32_t a0 = e2m1_even_to_e4m3(w0), a1 = e2m1_even_to_e4m3(w1);
+                        const uint32_t a2 = e2m1_odd_to_e4m3(w0), a3 = e2m1_odd_to_e4m3(w1);
+                        const float f0 = sc[ra * SCP + b], f1 = sc[(ra + 8) * SCP + b];
 #pragma unroll
-                        for (int gi = 0; gi < 2; ++gi) {
-                            if (gi < ngroups) {
+                        for (int ng = 0; ng < 2; ++ng) {
+                            if (ng < ng_n) {
                                 float c[4] = {0.f, 0.f, 0.f, 0.f};
-                                mma_f16(c, a00, a01, a02, a03, bh[i][gi][0][0], bh[i][gi][0][1]);
-                                mma_f16(c, a10, a11, a12, a13, bh[i][gi][1][0], bh[i][gi][1][1]);
-                                acc[rg][gi][0] = fmaf(c[0] + c[1], f0, acc[rg][gi][0]);
-                                acc[rg][gi][1] = fmaf(c[2] + c[3], f1, acc[rg][gi][1]);
+                                mma_e4m3(c, a0, a1, a2, a3, bq[i][ng][0], bq[i][ng][1]);
+                                acc[ng][0] = fmaf(c[0] + c[1], f0, acc[ng][0]);
+                                acc[ng][1] = fmaf(c[2] + c[3], f1, acc[ng][1]);
                             }
                         }
                     }
                 }
-            }
-        } else if (valid) {
+                // rb[kq][row][token of the pass][half]: columns 2q, 2q+1 hold
+                // pieces 2(q&1), 2(q&1)+1 of token 2*ng + q/2
 #pragma unroll
-            for (int i = 0; i < NBC; ++i) {
-                const int b = warp + 16 * i;
-                if (b < nbk) {
-                    const uint4 r0 = *reinterpret_cast<const uint4 *>(st + g * PS + 64 * b + 16 * q);
-                    const uint4 r1 = *reinterpret_cast<const uint4 *>(st + (g + 8) * PS + 64 * b + 16 * q);
+                for (int ng = 0; ng < 2; ++ng) {
+                    const int mi = 2 * ng + (q >> 1), hf = q & 1;
+                    rb[((kq * kDownRowsQ + ra) * 4 + mi) * 2 + hf] = acc[ng][0];
+                    rb[((kq * kDownRowsQ + ra + 8) * 4 + mi) * 2 + hf] = acc[ng][1];
+                }
+                if (pass + 1 < npass) {
+                    // more tokens follow in another pass: reduce this one now
+                    __syncthreads();
+                    reduce_routed(rb, u, it, tb, nt, tok);
+                    __syncthreads();
+                }
+            } else if (valid) {
 #pragma unroll
-                    for (int gi = 0; gi < 2; ++gi) {
-                        if (gi < ngroups) {
-                            float c[4] = {0.f, 0.f, 0.f, 0.f};
-                            mma_bf16(c, r0.x, r1.x, r0.y, r1.y, bh[i][gi][0][0], bh[i][gi][0][1]);
-                            mma_bf16(c, r0.z, r1.z, r0.w, r1.w, bh[i][gi][1][0], bh[i][gi][1][1]);
-                            acc[0][gi][0] += c[0] + c[1];
-                            acc[0][gi][1] += c[2] + c[3];
+                for (int i = 0; i < NBS; ++i) {
+                    const int b = warp + 16 * i;
+                    if (b < ffs / 32) {
+                        const uint4 r0 = *reinterpret_cast<const uint4 *>(st + g * PS + 64 * b + 16 * q);
+                        const uint4 r1 = *reinterpret_cast<const uint4 *>(st + (g + 8) * PS + 64 * b + 16 * q);
+#pragma unroll
+                        for (int ng = 0; ng < 2; ++ng) {
+                            if (4 * ng < p.Tc) {
+                                float c[4] = {0.f, 0.f, 0.f, 0.f};
+                                mma_bf16(c, r0.x, r1.x, r0.y, r1.y, bs[i][ng][0][0], bs[i][ng][0][1]);
+                                mma_bf16(c, r0.z, r1.z, r0.w, r1.w, bs[i][ng][1][0], bs[i][ng][1][1]);
+                                acc[ng][0] += c[0] + c[1];
+                                acc[ng][1] += c[2] + c[3];
+                            }
                         }
                     }
                 }
-            }
-        }
-        float *rb = red + ((it - i0) & 1) * (16 * kDownRowsQ * kChunk);
-        const int nrg = shared_item ? 1 : 2;
 #pragma unroll
-        for (int rg = 0; rg < 2; ++rg) {
-            if (rg < nrg) {
-#pragma unroll
-                for (int gi = 0; gi < 2; ++gi) {
-                    const int mi = gi * 4 + q;
-                    rb[(warp * kDownRowsQ + rg * 16 + g) * kChunk + mi] = acc[rg][gi][0];
-                    rb[(warp * kDownRowsQ + rg * 16 + g + 8) * kChunk + mi] = acc[rg][gi][1];
+                for (int ng = 0; ng < 2; ++ng) {
+                    const int t = 4 * ng + q;
+                    rb[(warp * 16 + g) * kChunk + t] = acc[ng][0];
+                    rb[(warp * 16 + g + 8) * kChunk + t] = acc[ng][1];
                 }
             }
+        }
+        bool ok_next = true;
+        if (it + 1 < i1) {
+            const int sn = (it + 1 - i0) % nst;
+            ok_next = mbar_wait_bounded(&full[sn], (uint32_t)(((it + 1 - i0) / nst) & 1), hdr);
+            if (it + 1 < U * nq)
+                convert_scales(smem + sn * SB + kDownRowsQ * PQ, scf + ((it + 1 - i0) & 1) * kDownRowsQ * SCP,
+                               kDownRowsQ, nbk, SCP, kDownThreads);
         }
         __syncthreads();
-        if (warp == 0 && it + kStages < i1) issue(it + kStages, s);
-        const int rows = shared_item ? kDownRowsS : kDownRowsQ;
-        if (threadIdx.x < rows * kChunk && valid) {
-            const int r = threadIdx.x / kChunk, mi = threadIdx.x % kChunk;
-            if (mi < ntok) {
+        if (warp == 0 && it + nst < i1) issue(it + nst, s);
+        if (valid && !shared_item) {
+            const int tb = (npass - 1) * 4;
+            reduce_routed(rb, u, it, tb, ntok - tb, tok);
+        } else if (valid) {
+            for (int i = threadIdx.x; i < kDownRowsS * p.Tc; i += kDownThreads) {
+                const int r = i / p.Tc, t = i - r * p.Tc;
                 float sum = 0.f;
 #pragma unroll
-                for (int w = 0; w < 16; ++w) sum += rb[(w * kDownRowsQ + r) * kChunk + mi];
-                const int t = tok[mi];
-                if (shared_item) {
-                    const int r0 = (it - U * nq) * kDownRowsS;
-                    ob[((size_t)t * (k + 1) + 0) * d + r0 + r] = sum;
-                } else {
-                    const int j = uslot[u * kChunk + t];
-                    const int sg = f16_prescale(__uint_as_float(__ldcg(hmax + t * k + j)));
-                    const float inv = __uint_as_float((uint32_t)(127 - sg) << 23);
-                    const int r0 = (it - u * nq) * kDownRowsQ;
-                    ob[((size_t)t * (k + 1) + 1 + j) * d + r0 + r] = sum * inv;
-                }
+                for (int w = 0; w < 16; ++w) sum += rb[(w * 16 + r) * kChunk + t];
+                const int r0 = (it - U * nq) * kDownRowsS;
+                ob[((size_t)t * (k + 1) + 0) * d + r0 + r] = sum;
             }
         }
+        ok = ok_next;
     }
 }
 
@@ -794,7 +1028,6 @@ struct SingleParams {
 
 __global__ void single_expert_setup_kernel(SingleParams p) {
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + p.L.hdr);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();
     if (threadIdx.x == 0) {
         hdr->n_unique = 1u;
@@ -812,14 +1045,7 @@ __global__ void single_expert_setup_kernel(SingleParams p) {
         reinterpret_cast<float *>(p.ws + p.L.wt)[t * p.L.k] = 1.0f;
         reinterpret_cast<uint32_t *>(p.ws + p.L.hmax)[t * p.L.k] = 0u;
     }
-    if (warp < p.Tc) {
-        const uint16_t *xr = p.x + (size_t)warp * p.d;
-        float mx = 0.f;
-        for (int j = lane; j < p.d; j += 32) mx = fmaxf(mx, fabsf(__uint_as_float((uint32_t)xr[j] << 16)));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) reinterpret_cast<int32_t *>(p.ws + p.L.sigx)[warp] = f16_prescale(mx);
-    }
+    build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L);
     __threadfence();
     pdl_trigger();
 }

@@ -25,6 +25,8 @@ constexpr int kSmemLimit = 227 * 1024;
 struct DeviceInfo {
     bool ready = false;
     int sms = 0;
+    int route_smem = -1;  // dynamic smem of the last occupancy query
+    int route_occ = 0;    // resident route_shared CTAs per SM at that size
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -39,6 +41,11 @@ cudaError_t set_smem(Kern kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+#define K3_GU_LIST(X) X(1, 1) X(1, 2) X(2, 1) X(2, 2) X(4, 1) X(4, 2) X(8, 1) X(8, 2) \
+    X(14, 1) X(14, 2) X(16, 1) X(16, 2)
+#define K3_DN_LIST(X) X(2, 1) X(2, 3) X(2, 6) X(4, 1) X(4, 3) X(4, 6) X(12, 1) X(12, 3) \
+    X(12, 6) X(24, 1) X(24, 3) X(24, 6)
+
 // One-time per-device set-up: SM count and the shared-memory opt-ins.
 k3moe_status device_info(DeviceInfo **out) {
     int dev = 0;
@@ -51,17 +58,13 @@ k3moe_status device_info(DeviceInfo **out) {
         e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return cuda_fail(e);
         const int big = kSmemLimit;
-        cudaError_t r = cudaSuccess;
-        r = set_smem(route_shared_kernel, kRouteTok * 8192 * 4);
-        if (r == cudaSuccess) r = set_smem(expert_gu_kernel<1>, big);
-        if (r == cudaSuccess) r = set_smem(expert_gu_kernel<2>, big);
-        if (r == cudaSuccess) r = set_smem(expert_gu_kernel<4>, big);
-        if (r == cudaSuccess) r = set_smem(expert_gu_kernel<8>, big);
-        if (r == cudaSuccess) r = set_smem(expert_gu_kernel<16>, big);
-        if (r == cudaSuccess) r = set_smem(expert_down_kernel<1>, big);
-        if (r == cudaSuccess) r = set_smem(expert_down_kernel<2>, big);
-        if (r == cudaSuccess) r = set_smem(expert_down_kernel<4>, big);
-        if (r == cudaSuccess) r = set_smem(expert_down_kernel<8>, big);
+        cudaError_t r = set_smem(route_shared_kernel, kRouteTok * 8192 * 4);
+#define K3_SET_GU(a, b) if (r == cudaSuccess) r = set_smem(expert_gu_kernel<a, b>, big);
+#define K3_SET_DN(a, b) if (r == cudaSuccess) r = set_smem(expert_down_kernel<a, b>, big);
+        K3_GU_LIST(K3_SET_GU)
+        K3_DN_LIST(K3_SET_DN)
+#undef K3_SET_GU
+#undef K3_SET_DN
         if (r != cudaSuccess) return cuda_fail(r);
         di.ready = true;
     }
@@ -75,18 +78,29 @@ int shared_ff(const k3moe_dims *dm) {
     return (dm->flags & K3MOE_NO_SHARED) ? 0 : dm->ff_shared;
 }
 
+int gu_stages(int d) {
+    for (int n = kMaxStages; n >= 2; --n)
+        if (gu_smem_bytes(d, n) <= kSmemLimit) return n;
+    return 0;
+}
+int dn_stages(int ff, int ffs) {
+    for (int n = kMaxStages; n >= 2; --n)
+        if (dn_smem_bytes(ff, ffs, n) <= kSmemLimit) return n;
+    return 0;
+}
+
 k3moe_status check_dims(const k3moe_dims *dm) {
     if (!dm) return K3MOE_ERR_INVALID_ARGUMENT;
     if (dm->flags & ~(K3MOE_OUT_FP32 | K3MOE_NO_SHARED)) return K3MOE_ERR_INVALID_ARGUMENT;
     if (dm->d < 64 || dm->d > 8192 || dm->d % 64) return K3MOE_ERR_UNSUPPORTED_SHAPE;
-    if (dm->ff < 64 || dm->ff > 8192 || dm->ff % 64) return K3MOE_ERR_UNSUPPORTED_SHAPE;
+    if (dm->ff < 64 || dm->ff > 3072 || dm->ff % 64) return K3MOE_ERR_UNSUPPORTED_SHAPE;
     if (dm->n_experts < 1 || dm->n_experts > 1024) return K3MOE_ERR_UNSUPPORTED_SHAPE;
     if (dm->top_k < 1 || dm->top_k > 32 || dm->top_k > dm->n_experts)
         return K3MOE_ERR_INVALID_ARGUMENT;
-    if (dm->ff_shared < 0 || dm->ff_shared > 8192 || dm->ff_shared % 64)
+    if (dm->ff_shared < 0 || dm->ff_shared > 3072 || dm->ff_shared % 64)
         return K3MOE_ERR_UNSUPPORTED_SHAPE;
-    if (gu_smem_bytes(dm->d) > kSmemLimit) return K3MOE_ERR_UNSUPPORTED_SHAPE;
-    if (dn_smem_bytes(dm->ff, dm->ff_shared) > kSmemLimit) return K3MOE_ERR_UNSUPPORTED_SHAPE;
+    if (gu_stages(dm->d) == 0) return K3MOE_ERR_UNSUPPORTED_SHAPE;
+    if (dn_stages(dm->ff, dm->ff_shared) == 0) return K3MOE_ERR_UNSUPPORTED_SHAPE;
     return K3MOE_OK;
 }
 
@@ -114,47 +128,69 @@ cudaError_t launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
     return cudaLaunchKernelEx(&cfg, kernel, params);
 }
 
-int pow2_at_least(int v) {
-    int p = 1;
-    while (p < v) p <<= 1;
-    return p;
-}
 
-cudaError_t launch_gu(const DeviceInfo &di, const GUParams &gp, cudaStream_t st) {
+cudaError_t launch_gu(const DeviceInfo &di, GUParams gp, cudaStream_t st) {
     const int need = (gp.d / 32 + 15) / 16;
-    const int smem = gu_smem_bytes(gp.d);
+    const int nbw = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : need <= 8 ? 8 : need <= 14 ? 14 : 16;
+    const int ng = gp.Tc <= 4 ? 1 : 2;
+    gp.nst = gu_stages(gp.d);
+    const int smem = gu_smem_bytes(gp.d, gp.nst);
     const dim3 grid(di.sms), block(kGUThreads);
-    switch (pow2_at_least(need)) {
-        case 1: return launch(expert_gu_kernel<1>, grid, block, smem, st, true, gp);
-        case 2: return launch(expert_gu_kernel<2>, grid, block, smem, st, true, gp);
-        case 4: return launch(expert_gu_kernel<4>, grid, block, smem, st, true, gp);
-        case 8: return launch(expert_gu_kernel<8>, grid, block, smem, st, true, gp);
-        default: return launch(expert_gu_kernel<16>, grid, block, smem, st, true, gp);
-    }
+#define K3_LAUNCH_GU(a, b) \
+    if (nbw == a && ng == b) return launch(expert_gu_kernel<a, b>, grid, block, smem, st, true, gp);
+    K3_GU_LIST(K3_LAUNCH_GU)
+#undef K3_LAUNCH_GU
+    return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_down(const DeviceInfo &di, const DownParams &dp, cudaStream_t st) {
-    const int kmax = dp.ff > dp.ffs ? dp.ff : dp.ffs;
-    const int need = (kmax / 32 + 15) / 16;
-    const int smem = dn_smem_bytes(dp.ff, dp.ffs);
+cudaError_t launch_down(const DeviceInfo &di, DownParams dp, cudaStream_t st) {
+    const int nq = (dp.ff / 32 + 3) / 4;
+    const int nbq = nq <= 2 ? 2 : nq <= 4 ? 4 : nq <= 12 ? 12 : 24;
+    const int ns = (dp.ffs / 32 + 15) / 16;
+    const int nbs = ns <= 1 ? 1 : ns <= 3 ? 3 : 6;
+    dp.nst = dn_stages(dp.ff, dp.ffs);
+    const int smem = dn_smem_bytes(dp.ff, dp.ffs, dp.nst);
     const dim3 grid(di.sms), block(kDownThreads);
-    switch (pow2_at_least(need)) {
-        case 1: return launch(expert_down_kernel<1>, grid, block, smem, st, true, dp);
-        case 2: return launch(expert_down_kernel<2>, grid, block, smem, st, true, dp);
-        case 4: return launch(expert_down_kernel<4>, grid, block, smem, st, true, dp);
-        default: return launch(expert_down_kernel<8>, grid, block, smem, st, true, dp);
-    }
+#define K3_LAUNCH_DN(a, b) \
+    if (nbq == a && nbs == b) return launch(expert_down_kernel<a, b>, grid, block, smem, st, true, dp);
+    K3_DN_LIST(K3_LAUNCH_DN)
+#undef K3_LAUNCH_DN
+    return cudaErrorInvalidValue;
 }
 
-// Router (+ shared gate/up + top-k + dispatch) for one chunk.
-cudaError_t launch_route(const DeviceInfo &di, const RouteParams &rp, cudaStream_t st) {
-    const int N = rp.E + rp.ffs;
+// Router (+ shared gate/up + top-k + dispatch) for one chunk.  Cooperative
+// launch: CTA 0 waits on the other CTAs' router rows, so all must be resident.
+cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st) {
     const int nt = rp.Tc < kRouteTok ? rp.Tc : kRouteTok;
     const int smem = nt * rp.d * 4;
-    const int per_sm = smem <= 64 * 1024 ? 2 : 1;
-    int G = di.sms * per_sm;
-    if (G > N) G = N;
-    return launch(route_shared_kernel, dim3(G), dim3(kRouteThreads), smem, st, false, rp);
+    if (di.route_smem != smem) {
+        int occ = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, route_shared_kernel,
+                                                                       kRouteThreads, smem);
+        if (e != cudaSuccess) return e;
+        di.route_occ = occ;
+        di.route_smem = smem;
+    }
+    const int per_sm = di.route_occ < 3 ? di.route_occ : 3;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    int gs = per_sm * di.sms - 1;  // streaming CTAs
+    // every streaming warp takes at least a quarter row of the smaller phase,
+    // so a row is split between at most 5 warps (kMaxSeg slots)
+    const int rows_min = rp.ffs > 0 && rp.ffs < rp.E ? rp.ffs : rp.E;
+    const int wmax = rows_min * 4;
+    if (gs * 8 > wmax) gs = wmax / 8 > 0 ? wmax / 8 : 1;
+    rp.nwarps = gs * 8;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(gs + 1);
+    cfg.blockDim = dim3(kRouteThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, route_shared_kernel, rp);
 }
 
 struct EventHook {
