@@ -149,6 +149,27 @@ __device__ __forceinline__ uint32_t e2m1_odd_to_e4m3(uint32_t w) {
     return (w & 0x80808080u) | ((w >> 2) & 0x1C1C1C1Cu);
 }
 
+// E2M1 nibbles -> f16 by bit placement (ALU only).  The code s.e1e0.m is put
+// at f16 bits 15 (sign) and 11..9 (low exponent bits, top mantissa bit): the
+// f16 value is exactly 2^-14 times the E2M1 value (the E2M1 subnormal 0.5
+// becomes the f16 subnormal 2^-15).  One register holds nibbles i and i+4 of
+// a word (16 bits apart), so both halves take the same shifts:
+//   pair 0: columns 0,4   pair 1: columns 1,5   pair 2: 2,6   pair 3: 3,7
+__device__ __forceinline__ uint32_t e2m1_pair0_f16(uint32_t w) {
+    return ((w << 9) & 0x0E000E00u) | ((w << 12) & 0x80008000u);
+}
+__device__ __forceinline__ uint32_t e2m1_pair1_f16(uint32_t w) {
+    return ((w << 5) & 0x0E000E00u) | ((w << 8) & 0x80008000u);
+}
+__device__ __forceinline__ uint32_t e2m1_pair2_f16(uint32_t w) {
+    return ((w << 1) & 0x0E000E00u) | ((w << 4) & 0x80008000u);
+}
+__device__ __forceinline__ uint32_t e2m1_pair3_f16(uint32_t w) {
+    return ((w >> 3) & 0x0E000E00u) | (w & 0x80008000u);
+}
+// Position of column c of an 8-column group in the pair order 0,4,1,5,2,6,3,7.
+__device__ __forceinline__ int pairpos(int c) { return (c & ~7) + 2 * (c & 3) + ((c >> 2) & 1); }
+
 // fp32 <-> E4M3 (OCP E4M3FN: bias 7, subnormals, no infinities) on the ALU
 // and FMA pipes.  Scaling by 2^-120 maps every E4M3 value, normal or
 // subnormal, onto fp32 bit patterns whose bits 30..20 are the E4M3 bits 6..0

@@ -114,9 +114,11 @@ __device__ void warp_topk(const float *row, int E, int k, int lane, int32_t *idx
 // even/odd nibble split of the MMA A operand.
 __device__ __forceinline__ int perm8(int c) { return (c & ~7) + ((c & 1) ? 4 : 0) + ((c & 7) >> 1); }
 
-// Per-token E4M3 prescale exponent of x and x * 2^s as two E4M3 pieces,
-// written to the workspace for the gate/up pass.  Run by one whole CTA.
-__device__ void build_x_pieces(const uint16_t *x, int Tc, int d, uint8_t *ws, const Layout &L) {
+// Per-token f16 prescale exponent s of x (max |x| 2^s in [2^14, 2^15)) and
+// x * 2^s as f16 in pair order (columns 0,4,1,5,2,6,3,7 of each group of 8),
+// written to the workspace for the gate/up pass.  Exact for every bf16
+// element at or above 2^-17 of the token's largest |x|.  Run by one CTA.
+__device__ void build_x_f16(const uint16_t *x, int Tc, int d, uint8_t *ws, const Layout &L) {
     __shared__ int s_sig[kChunk];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int t = warp; t < Tc; t += nw) {
@@ -126,21 +128,17 @@ __device__ void build_x_pieces(const uint16_t *x, int Tc, int d, uint8_t *ws, co
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         if (lane == 0) {
-            const int sg = e4m3_prescale(mx);
+            const int sg = f16_prescale(mx);
             s_sig[t] = sg;
             reinterpret_cast<int32_t *>(ws + L.sigx)[t] = sg;
         }
     }
     __syncthreads();
-    uint8_t *xp = ws + L.xp;
+    __half *xp = reinterpret_cast<__half *>(ws + L.xp);
     for (int i = threadIdx.x; i < Tc * d; i += blockDim.x) {
         const int t = i / d, c = i - t * d;
-        float v = __uint_as_float((uint32_t)x[i] << 16) * exp2i(s_sig[t]);
-        const uint32_t p0 = f32_to_e4m3_rn(v);
-        v -= e4m3_to_f32(p0);
-        const uint32_t p1 = f32_to_e4m3_rn(v);
-        xp[((size_t)t * 2 + 0) * d + perm8(c)] = (uint8_t)p0;
-        xp[((size_t)t * 2 + 1) * d + perm8(c)] = (uint8_t)p1;
+        const float v = __uint_as_float((uint32_t)x[i] << 16) * exp2i(s_sig[t]);
+        xp[(size_t)t * d + pairpos(c)] = __float2half_rn(v);
     }
 }
 
@@ -387,14 +385,14 @@ __device__ int stream_phase(const RouteParams &p, WsHeader *hdr, const float *xs
     return finished;
 }
 
-__global__ void __launch_bounds__(kRouteThreads) route_shared_kernel(RouteParams p) {
+__global__ void __launch_bounds__(kRouteThreads, 3) route_shared_kernel(RouteParams p) {
     extern __shared__ __align__(16) float xs[];  // [kRouteTok][d]
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + p.L.hdr);
     pdl_trigger();
     const int npass = (p.Tc + kRouteTok - 1) / kRouteTok;
     if (blockIdx.x == 0) {
         // x pieces for the gate/up pass need no routing: build them first
-        if (p.blobs != nullptr) build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L);
+        if (p.blobs != nullptr) build_x_f16(p.x, p.Tc, p.d, p.ws, p.L);
         // wait (bounded) for every router row of every pass, then route and dispatch
         __shared__ int s_ok;
         if (threadIdx.x == 0) {
@@ -479,8 +477,8 @@ __device__ __forceinline__ void convert_scales(const uint8_t *sc8, float *dst, i
     }
 }
 
-// NBW: blocks of 32 columns per warp (>= d/32/16); NG: token groups of 4.
-template <int NBW, int NG>
+// NBW: blocks of 32 columns per warp (>= d/32/16).
+template <int NBW>
 __global__ void __launch_bounds__(kGUThreads, 1) expert_gu_kernel(GUParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int d = p.d, ff = p.ff, nb = d / 32, nst = p.nst;
@@ -513,25 +511,22 @@ __global__ void __launch_bounds__(kGUThreads, 1) expert_gu_kernel(GUParams p) {
     const int k = p.L.k;
     const size_t mat = (size_t)d * ff;
 
-    // B operand: column n = g of token group ng is token 4*ng + g/2, piece g&1
-    // of its prescaled x (x * 2^sigx = piece0 + piece1, E4M3).  Register 0
-    // holds the even columns 8q, 8q+2, 8q+4, 8q+6 of a block, register 1 the
-    // odd ones, matching the even/odd nibble split of the A operand.
-    uint32_t bx[NBW][NG][2];
+    // B operand (column n = g = token): the lane's 8 columns 8q..8q+7 of a
+    // block as f16 pairs (0,4) (1,5) (2,6) (3,7), matching the nibble pairs
+    // the A operand is decoded into.
+    uint32_t bx[NBW][2][2];
     {
         const uint8_t *xp = p.ws + p.L.xp;
 #pragma unroll
-        for (int ng = 0; ng < NG; ++ng) {
-            const int t = 4 * ng + (g >> 1), piece = g & 1;
-#pragma unroll
-            for (int i = 0; i < NBW; ++i) {
-                const int b = warp + 16 * i;
-                uint2 v = make_uint2(0, 0);
-                if (t < p.Tc && b < nb)
-                    v = __ldcg(reinterpret_cast<const uint2 *>(xp + ((size_t)t * 2 + piece) * d + 32 * b + 8 * q));
-                bx[i][ng][0] = v.x;
-                bx[i][ng][1] = v.y;
-            }
+        for (int i = 0; i < NBW; ++i) {
+            const int b = warp + 16 * i;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (g < p.Tc && b < nb)
+                v = __ldcg(reinterpret_cast<const uint4 *>(xp + ((size_t)g * d + 32 * b + 8 * q) * 2));
+            bx[i][0][0] = v.x;
+            bx[i][0][1] = v.y;
+            bx[i][1][0] = v.z;
+            bx[i][1][1] = v.w;
         }
     }
 
@@ -580,9 +575,7 @@ __global__ void __launch_bounds__(kGUThreads, 1) expert_gu_kernel(GUParams p) {
         const uint8_t *st = smem + s * SB;
         const float *sc = scf + ((it - i0) & 1) * 16 * SCP;
         float *rb = red + ((it - i0) & 1) * gu_red_floats();
-        float ag[NG], au[NG];
-#pragma unroll
-        for (int ng = 0; ng < NG; ++ng) ag[ng] = au[ng] = 0.f;
+        float ag0 = 0.f, ag1 = 0.f, au0 = 0.f, au1 = 0.f;
         if (ok) {
 #pragma unroll
             for (int i = 0; i < NBW; ++i) {
@@ -591,23 +584,22 @@ __global__ void __launch_bounds__(kGUThreads, 1) expert_gu_kernel(GUParams p) {
                     const uint32_t wg = *reinterpret_cast<const uint32_t *>(st + g * P + 16 * b + 4 * q);
                     const uint32_t wu =
                         *reinterpret_cast<const uint32_t *>(st + (8 + g) * P + 16 * b + 4 * q);
-                    const uint32_t a0 = e2m1_even_to_e4m3(wg), a1 = e2m1_even_to_e4m3(wu);
-                    const uint32_t a2 = e2m1_odd_to_e4m3(wg), a3 = e2m1_odd_to_e4m3(wu);
                     const float fg = sc[g * SCP + b], fu = sc[(8 + g) * SCP + b];
-#pragma unroll
-                    for (int ng = 0; ng < NG; ++ng) {
-                        float c[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_e4m3(c, a0, a1, a2, a3, bx[i][ng][0], bx[i][ng][1]);
-                        ag[ng] = fmaf(c[0] + c[1], fg, ag[ng]);
-                        au[ng] = fmaf(c[2] + c[3], fu, au[ng]);
-                    }
+                    float c[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_f16(c, e2m1_pair0_f16(wg), e2m1_pair0_f16(wu), e2m1_pair1_f16(wg),
+                            e2m1_pair1_f16(wu), bx[i][0][0], bx[i][0][1]);
+                    mma_f16(c, e2m1_pair2_f16(wg), e2m1_pair2_f16(wu), e2m1_pair3_f16(wg),
+                            e2m1_pair3_f16(wu), bx[i][1][0], bx[i][1][1]);
+                    ag0 = fmaf(c[0], fg, ag0);
+                    ag1 = fmaf(c[1], fg, ag1);
+                    au0 = fmaf(c[2], fu, au0);
+                    au1 = fmaf(c[3], fu, au1);
                 }
             }
         }
-#pragma unroll
-        for (int ng = 0; ng < NG; ++ng)
-            *reinterpret_cast<float2 *>(rb + ((warp * 8 + g) * kChunk + 4 * ng + q) * 2) =
-                make_float2(ag[ng], au[ng]);
+        // columns 2q, 2q+1 are tokens 2q, 2q+1
+        *reinterpret_cast<float2 *>(rb + ((warp * 8 + g) * kChunk + 2 * q) * 2) = make_float2(ag0, au0);
+        *reinterpret_cast<float2 *>(rb + ((warp * 8 + g) * kChunk + 2 * q + 1) * 2) = make_float2(ag1, au1);
         bool ok_next = true;
         if (it + 1 < i1) {
             const int sn = (it + 1 - i0) % nst;
@@ -628,8 +620,8 @@ __global__ void __launch_bounds__(kGUThreads, 1) expert_gu_kernel(GUParams p) {
                     sg += v.x;
                     su += v.y;
                 }
-                // undo the 2^-6 of the E4M3 placement and the x prescale
-                const float inv = exp2i(6 - sigx[t]);
+                // undo the 2^-14 of the f16 placement and the x prescale
+                const float inv = exp2i(14 - sigx[t]);
                 const float h = silu_mul(sg * inv, su * inv);
                 const int j = uslot[u * kChunk + t];
                 hbuf[((size_t)t * k + j) * ff + rg * 8 + r] = h;
@@ -657,21 +649,21 @@ constexpr int kDownRowsS = 16;  // bf16 rows per shared item
 __host__ __device__ inline int dn_pitch_q(int ff) { return ff / 2 + 16; }
 __host__ __device__ inline int dn_pitch_s(int ffs) { return 2 * ffs + 64; }
 __host__ __device__ inline int dn_scp(int ff) { return ff / 32 + 1; }
-__host__ __device__ inline int dn_pc_pitch(int ff) { return ff + 32; }  // one (token, piece) row
+__host__ __device__ inline int dn_pc_pitch(int ff) { return 2 * ff + 64; }  // one (token, part) f16 row
 __host__ __device__ inline int dn_stage_bytes(int ff, int ffs) {
     int a = kDownRowsQ * dn_pitch_q(ff) + kDownRowsQ * (ff / 32);
     int b = ffs > 0 ? kDownRowsS * dn_pitch_s(ffs) : 0;
     return ((a > b ? a : b) + 127) & ~127;
 }
-// partial sums of one pass: routed [4 K-quarters][64 rows][4 tokens][2 halves],
+// partial sums of one pass: routed [4 K-quarters][64 rows][4 tokens],
 // shared [16 warps][16 rows][8 tokens]
 __host__ __device__ inline int dn_red_floats() {
-    const int a = 16 * 16 * kChunk, b = 4 * kDownRowsQ * 4 * 2;
+    const int a = 16 * 16 * kChunk, b = 4 * kDownRowsQ * 4;
     return a > b ? a : b;
 }
 __host__ __device__ inline int dn_smem_bytes(int ff, int ffs, int nst) {
     return nst * dn_stage_bytes(ff, ffs) + 2 * kDownRowsQ * dn_scp(ff) * 4 +
-           16 * dn_pc_pitch(ff) + 2 * dn_red_floats() * 4 + kMaxStages * 8;
+           8 * dn_pc_pitch(ff) + 2 * dn_red_floats() * 4 + kMaxStages * 8;
 }
 
 // NBQ: blocks per K-quarter for routed items (>= ff/32/4); NBS: blocks per warp
@@ -684,8 +676,8 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
     const int PQ = dn_pitch_q(ff), PS = dn_pitch_s(ffs), SCP = dn_scp(ff), PCP = dn_pc_pitch(ff);
     const int nbk = ff / 32;
     float *scf = reinterpret_cast<float *>(smem + nst * SB);                // [2][64][SCP]
-    uint8_t *pcs = reinterpret_cast<uint8_t *>(scf + 2 * kDownRowsQ * SCP);  // [4 tok][4 piece][PCP]
-    float *red = reinterpret_cast<float *>(pcs + 16 * PCP);                 // [2][dn_red_floats]
+    uint8_t *pcs = reinterpret_cast<uint8_t *>(scf + 2 * kDownRowsQ * SCP);  // [4 tok][hi,lo][PCP]
+    float *red = reinterpret_cast<float *>(pcs + 8 * PCP);                  // [2][dn_red_floats]
     uint64_t *full = reinterpret_cast<uint64_t *>(red + 2 * dn_red_floats());
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + p.L.hdr);
@@ -750,8 +742,8 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
     if (warp == 0)
         for (int s = 0; s < nst && i0 + s < i1; ++s) issue(i0 + s, s);
 
-    // routed items: warp = (row group rgw, K-quarter kq); column n = g of
-    // token group ng is token 2*ng + g/4 of the pass, piece g&3 of its h
+    // routed items: warp = (row group rgw, K-quarter kq); B column n = g is
+    // token g/2 of the pass, part g&1 (hi, lo) of its prescaled h in f16
     const int rgw = warp & 3, kq = warp >> 2;
     uint32_t bq[NBQ][2][2];
     uint32_t bs[NBS][2][2][2];  // shared: [block][token group][step][2], bf16 hi/lo
@@ -764,13 +756,13 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
             const int r = i / nt, mi = i - r * nt;
             float sum = 0.f;
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq)
-                sum += rb[((qq * kDownRowsQ + r) * 4 + mi) * 2] + rb[((qq * kDownRowsQ + r) * 4 + mi) * 2 + 1];
+            for (int qq = 0; qq < 4; ++qq) sum += rb[(qq * kDownRowsQ + r) * 4 + mi];
             const int t = tok[tb + mi];
             const int j = uslot[u * kChunk + t];
-            const int sgm = e4m3_prescale(__uint_as_float(__ldcg(hmax + t * k + j)));
+            const int sgm = f16_prescale(__uint_as_float(__ldcg(hmax + t * k + j)));
             const int r0 = (it - u * nq) * kDownRowsQ;
-            ob[((size_t)t * (k + 1) + 1 + j) * d + r0 + r] = sum * exp2i(6 - sgm);
+            // undo the 2^-14 of the f16 placement and the h prescale
+            ob[((size_t)t * (k + 1) + 1 + j) * d + r0 + r] = sum * exp2i(14 - sgm);
         }
     };
 
@@ -811,9 +803,8 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
             if (!shared_item) {
                 const int key = u * 2 + pass;
                 if (key != cur_key) {
-                    // h of up to 4 of this expert's tokens as four E4M3 pieces in
-                    // smem, each lane's 8 bytes of a block being the even then the
-                    // odd columns of its 8-column group
+                    // h of up to 4 of this expert's tokens, prescaled, as f16 hi + lo
+                    // in pair order, one smem row per (token, part)
                     __syncthreads();  // earlier reads of the pieces are done
                     for (int i = threadIdx.x; i < nt * ff; i += kDownThreads) {
                         const int mi = i / ff, c = i - mi * ff;
@@ -821,29 +812,27 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
                         if (ublob[u] != nullptr) {
                             const int t = tok[tb + mi];
                             const int j = uslot[u * kChunk + t];
-                            const int sgm = e4m3_prescale(__uint_as_float(__ldcg(hmax + t * k + j)));
+                            const int sgm = f16_prescale(__uint_as_float(__ldcg(hmax + t * k + j)));
                             v = __ldcg(hbuf + ((size_t)t * k + j) * ff + c) * exp2i(sgm);
                         }
-                        const int off = perm8(c);
-#pragma unroll
-                        for (int pc = 0; pc < 4; ++pc) {
-                            const uint32_t b8 = f32_to_e4m3_rn(v);
-                            pcs[(mi * 4 + pc) * PCP + off] = (uint8_t)b8;
-                            v -= e4m3_to_f32(b8);
-                        }
+                        const __half hi = __float2half_rn(v);
+                        const __half lo = __float2half_rn(v - __half2float(hi));
+                        reinterpret_cast<__half *>(pcs + (mi * 2 + 0) * PCP)[pairpos(c)] = hi;
+                        reinterpret_cast<__half *>(pcs + (mi * 2 + 1) * PCP)[pairpos(c)] = lo;
                     }
                     __syncthreads();
-#pragma unroll
-                    for (int ng = 0; ng < 2; ++ng) {
-                        const int mi = 2 * ng + (g >> 2), pc = g & 3;
+                    {
+                        const int mi = g >> 1, part = g & 1;
 #pragma unroll
                         for (int i = 0; i < NBQ; ++i) {
                             const int b = kq + 4 * i;
-                            uint2 v = make_uint2(0, 0);
+                            uint4 v = make_uint4(0, 0, 0, 0);
                             if (b < nbk && mi < nt)
-                                v = *reinterpret_cast<const uint2 *>(pcs + (mi * 4 + pc) * PCP + b * 32 + q * 8);
-                            bq[i][ng][0] = v.x;
-                            bq[i][ng][1] = v.y;
+                                v = *reinterpret_cast<const uint4 *>(pcs + (mi * 2 + part) * PCP + (32 * b + 8 * q) * 2);
+                            bq[i][0][0] = v.x;
+                            bq[i][0][1] = v.y;
+                            bq[i][1][0] = v.z;
+                            bq[i][1][1] = v.w;
                         }
                     }
                     cur_key = key;
@@ -889,36 +878,27 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
 #pragma unroll
             for (int a = 0; a < 2; ++a) acc[a][0] = acc[a][1] = 0.f;
             if (valid && !shared_item) {
-                const int ng_n = (nt + 1) / 2;
                 const int ra = rgw * 16 + g;
+                float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
                 for (int i = 0; i < NBQ; ++i) {
                     const int b = kq + 4 * i;
                     if (b < nbk) {
                         const uint32_t w0 = *reinterpret_cast<const uint32_t *>(st + ra * PQ + 16 * b + 4 * q);
                         const uint32_t w1 = *reinterpret_cast<const uint32_t *>(st + (ra + 8) * PQ + 16 * b + 4 * q);
-                        const uint32_t a0 = e2m1_even_to_e4m3(w0), a1 = e2m1_even_to_e4m3(w1);
-                        const uint32_t a2 = e2m1_odd_to_e4m3(w0), a3 = e2m1_odd_to_e4m3(w1);
                         const float f0 = sc[ra * SCP + b], f1 = sc[(ra + 8) * SCP + b];
-#pragma unroll
-                        for (int ng = 0; ng < 2; ++ng) {
-                            if (ng < ng_n) {
-                                float c[4] = {0.f, 0.f, 0.f, 0.f};
-                                mma_e4m3(c, a0, a1, a2, a3, bq[i][ng][0], bq[i][ng][1]);
-                                acc[ng][0] = fmaf(c[0] + c[1], f0, acc[ng][0]);
-                                acc[ng][1] = fmaf(c[2] + c[3], f1, acc[ng][1]);
-                            }
-                        }
+                        float c[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_f16(c, e2m1_pair0_f16(w0), e2m1_pair0_f16(w1), e2m1_pair1_f16(w0),
+                                e2m1_pair1_f16(w1), bq[i][0][0], bq[i][0][1]);
+                        mma_f16(c, e2m1_pair2_f16(w0), e2m1_pair2_f16(w1), e2m1_pair3_f16(w0),
+                                e2m1_pair3_f16(w1), bq[i][1][0], bq[i][1][1]);
+                        // columns 2q, 2q+1: hi and lo part of token q of the pass
+                        acc0 = fmaf(c[0] + c[1], f0, acc0);
+                        acc1 = fmaf(c[2] + c[3], f1, acc1);
                     }
                 }
-                // rb[kq][row][token of the pass][half]: columns 2q, 2q+1 hold
-                // pieces 2(q&1), 2(q&1)+1 of token 2*ng + q/2
-#pragma unroll
-                for (int ng = 0; ng < 2; ++ng) {
-                    const int mi = 2 * ng + (q >> 1), hf = q & 1;
-                    rb[((kq * kDownRowsQ + ra) * 4 + mi) * 2 + hf] = acc[ng][0];
-                    rb[((kq * kDownRowsQ + ra + 8) * 4 + mi) * 2 + hf] = acc[ng][1];
-                }
+                rb[(kq * kDownRowsQ + ra) * 4 + q] = acc0;
+                rb[(kq * kDownRowsQ + ra + 8) * 4 + q] = acc1;
                 if (pass + 1 < npass) {
                     // more tokens follow in another pass: reduce this one now
                     __syncthreads();
@@ -1045,7 +1025,7 @@ __global__ void single_expert_setup_kernel(SingleParams p) {
         reinterpret_cast<float *>(p.ws + p.L.wt)[t * p.L.k] = 1.0f;
         reinterpret_cast<uint32_t *>(p.ws + p.L.hmax)[t * p.L.k] = 0u;
     }
-    build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L);
+    build_x_f16(p.x, p.Tc, p.d, p.ws, p.L);
     __threadfence();
     pdl_trigger();
 }

@@ -41,8 +41,7 @@ cudaError_t set_smem(Kern kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-#define K3_GU_LIST(X) X(1, 1) X(1, 2) X(2, 1) X(2, 2) X(4, 1) X(4, 2) X(8, 1) X(8, 2) \
-    X(14, 1) X(14, 2) X(16, 1) X(16, 2)
+#define K3_GU_LIST(X) X(1) X(2) X(4) X(8) X(14) X(16)
 #define K3_DN_LIST(X) X(2, 1) X(2, 3) X(2, 6) X(4, 1) X(4, 3) X(4, 6) X(12, 1) X(12, 3) \
     X(12, 6) X(24, 1) X(24, 3) X(24, 6)
 
@@ -59,7 +58,7 @@ k3moe_status device_info(DeviceInfo **out) {
         if (e != cudaSuccess) return cuda_fail(e);
         const int big = kSmemLimit;
         cudaError_t r = set_smem(route_shared_kernel, kRouteTok * 8192 * 4);
-#define K3_SET_GU(a, b) if (r == cudaSuccess) r = set_smem(expert_gu_kernel<a, b>, big);
+#define K3_SET_GU(a) if (r == cudaSuccess) r = set_smem(expert_gu_kernel<a>, big);
 #define K3_SET_DN(a, b) if (r == cudaSuccess) r = set_smem(expert_down_kernel<a, b>, big);
         K3_GU_LIST(K3_SET_GU)
         K3_DN_LIST(K3_SET_DN)
@@ -132,12 +131,11 @@ cudaError_t launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
 cudaError_t launch_gu(const DeviceInfo &di, GUParams gp, cudaStream_t st) {
     const int need = (gp.d / 32 + 15) / 16;
     const int nbw = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : need <= 8 ? 8 : need <= 14 ? 14 : 16;
-    const int ng = gp.Tc <= 4 ? 1 : 2;
     gp.nst = gu_stages(gp.d);
     const int smem = gu_smem_bytes(gp.d, gp.nst);
     const dim3 grid(di.sms), block(kGUThreads);
-#define K3_LAUNCH_GU(a, b) \
-    if (nbw == a && ng == b) return launch(expert_gu_kernel<a, b>, grid, block, smem, st, true, gp);
+#define K3_LAUNCH_GU(a) \
+    if (nbw == a) return launch(expert_gu_kernel<a>, grid, block, smem, st, true, gp);
     K3_GU_LIST(K3_LAUNCH_GU)
 #undef K3_LAUNCH_GU
     return cudaErrorInvalidValue;
