@@ -3,7 +3,7 @@
 
 One step = one k3moe_layer call over one batch of the workload's tokens (the
 whole hot path: router, softmax, top-k, dispatch, routed gate/up + SwiGLU,
-down projections, shared expert, combine).  Default workload: the K3-shape
+down projections with the weighted combine, shared expert).  Default workload: the K3-shape
 decode layer (d=7168, ff=1536, 896 experts, top-16, bf16 shared expert
 ff=1536, T=1 token), all 896 experts resident in HBM (15.7 GB).
 
@@ -274,7 +274,8 @@ def main():
     value = world * T * args.steps / (total_ms / 1000.0)
 
     # per-kernel durations (events recorded between the library's kernels)
-    kernels = ["route_shared", "expert_gu", "expert_down", "combine"]
+    kernels = (["route_shared", "expert_gu", "shared_down", "expert_down"] if cfg.ff_shared > 0
+               else ["route_shared", "expert_gu", "expert_down"])
     per_kernel = {}
     if single_pass:
         for j, name in enumerate(kernels):
@@ -328,7 +329,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f16/bf16 mma, f32 accumulate",
+        "scaling": "weak", "vs_baseline": None, "dtype": "mxf4 (E2M1 x E2M1, E8M0 block scales) tcgen05 MMA, f32 accumulate",
         "data": "synthetic",
         "config": {"workload": workload_desc(cfg), "global_batch": world * T, "seq_len": 1,
                    "parallelism": f"replicas x{world}",
@@ -340,7 +341,7 @@ def main():
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 4 * chunks * args.steps,
+        "gpu_launches": (4 if cfg.ff_shared > 0 else 3) * chunks * args.steps,
         "clocks": clk,
     }
     if rank == 0:

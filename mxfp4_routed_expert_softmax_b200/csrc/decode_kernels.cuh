@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "layout.cuh"
+#include "umma_kernels.cuh"
 
 namespace k3 {
 
@@ -46,6 +47,7 @@ struct RouteParams {
     int32_t *idx_out;   // optional [Tc][k]
     float *w_out;       // optional [Tc][k]
     int nwarps;         // streaming warps: 8 per CTA, CTAs 1.. of the grid
+    uint4 tmpl[2][8];   // tensor-map templates: W_g/W_u plane, W_d plane
 };
 
 constexpr int kRouteThreads = 256;
@@ -217,6 +219,7 @@ __device__ void topk_dispatch(const RouteParams &p, WsHeader *hdr) {
             }
             ublob[u] = b;
             gmask[u] = umask[u];
+            if (b != nullptr) write_expert_tmaps(p.ws, L, (int)u, b, p.tmpl);
         }
     }
 }
@@ -385,14 +388,16 @@ __device__ int stream_phase(const RouteParams &p, WsHeader *hdr, const float *xs
     return finished;
 }
 
-__global__ void __launch_bounds__(kRouteThreads, 3) route_shared_kernel(RouteParams p) {
+__global__ void __launch_bounds__(kRouteThreads, 3) route_shared_kernel(const __grid_constant__ RouteParams p) {
     extern __shared__ __align__(16) float xs[];  // [kRouteTok][d]
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + p.L.hdr);
     pdl_trigger();
     const int npass = (p.Tc + kRouteTok - 1) / kRouteTok;
+    // the gate/up pass's pieces of x need no routing: every CTA builds a share
+    if (p.blobs != nullptr)
+        build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L, blockIdx.x * (kRouteThreads / 32) + (threadIdx.x >> 5),
+                       gridDim.x * (kRouteThreads / 32));
     if (blockIdx.x == 0) {
-        // x pieces for the gate/up pass need no routing: build them first
-        if (p.blobs != nullptr) build_x_f16(p.x, p.Tc, p.d, p.ws, p.L);
         // wait (bounded) for every router row of every pass, then route and dispatch
         __shared__ int s_ok;
         if (threadIdx.x == 0) {
@@ -640,6 +645,7 @@ struct DownParams {
     uint8_t *ws;
     Layout L;
     int nst;
+    int skip_routed;  // only the shared expert's rows (the routed ones run on the tensor cores)
 };
 
 constexpr int kDownThreads = 512;
@@ -693,7 +699,8 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
     const int U = (int)hdr->n_unique;
     const int nq = d / kDownRowsQ;
     const int ns = ffs > 0 ? d / kDownRowsS : 0;
-    const int N = U * nq + ns;
+    const int NQ = p.skip_routed ? 0 : U * nq;
+    const int N = NQ + ns;
     const int G = gridDim.x;
     const int i0 = (int)(((long long)blockIdx.x * N) / G);
     const int i1 = (int)(((long long)(blockIdx.x + 1) * N) / G);
@@ -708,7 +715,7 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
 
     auto issue = [&](int it, int s) {
         uint8_t *st = smem + s * SB;
-        if (it < U * nq) {
+        if (it < NQ) {
             const int u = it / nq, rb = it - u * nq;
             const uint8_t *blob = ublob[u];
             const int r0 = rb * kDownRowsQ;
@@ -728,7 +735,7 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
                 bulk_g2s(st + kDownRowsQ * PQ, dn + mat / 2 + (size_t)r0 * (ff / 32),
                          kDownRowsQ * (ff / 32), &full[s]);
         } else {
-            const int r0 = (it - U * nq) * kDownRowsS;
+            const int r0 = (it - NQ) * kDownRowsS;
             if (lane == 0) {
                 fence_proxy_async();
                 mbar_arrive_expect_tx(&full[s], (uint32_t)(kDownRowsS * 2 * ffs));
@@ -772,11 +779,11 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
     bool ok = true;
     if (i0 < i1) {
         ok = mbar_wait_bounded(&full[0], 0u, hdr);
-        if (i0 < U * nq) convert_scales(smem + kDownRowsQ * PQ, scf, kDownRowsQ, nbk, SCP, kDownThreads);
+        if (i0 < NQ) convert_scales(smem + kDownRowsQ * PQ, scf, kDownRowsQ, nbk, SCP, kDownThreads);
         __syncthreads();
     }
     for (int it = i0; it < i1; ++it) {
-        const bool shared_item = it >= U * nq;
+        const bool shared_item = it >= NQ;
         const int u = shared_item ? U : it / nq;
         const int s = (it - i0) % nst;
         const uint8_t *st = smem + s * SB;
@@ -936,7 +943,7 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
         if (it + 1 < i1) {
             const int sn = (it + 1 - i0) % nst;
             ok_next = mbar_wait_bounded(&full[sn], (uint32_t)(((it + 1 - i0) / nst) & 1), hdr);
-            if (it + 1 < U * nq)
+            if (it + 1 < NQ)
                 convert_scales(smem + sn * SB + kDownRowsQ * PQ, scf + ((it + 1 - i0) & 1) * kDownRowsQ * SCP,
                                kDownRowsQ, nbk, SCP, kDownThreads);
         }
@@ -951,7 +958,7 @@ __global__ void __launch_bounds__(kDownThreads, 1) expert_down_kernel(DownParams
                 float sum = 0.f;
 #pragma unroll
                 for (int w = 0; w < 16; ++w) sum += rb[(w * 16 + r) * kChunk + t];
-                const int r0 = (it - U * nq) * kDownRowsS;
+                const int r0 = (it - NQ) * kDownRowsS;
                 ob[((size_t)t * (k + 1) + 0) * d + r0 + r] = sum;
             }
         }
@@ -1004,29 +1011,32 @@ struct SingleParams {
     const uint8_t *blob;
     uint8_t *ws;
     Layout L;
+    uint4 tmpl[2][8];
 };
 
-__global__ void single_expert_setup_kernel(SingleParams p) {
+__global__ void single_expert_setup_kernel(const __grid_constant__ SingleParams p) {
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + p.L.hdr);
     pdl_wait();
-    if (threadIdx.x == 0) {
-        hdr->n_unique = 1u;
-        const uint8_t *b = p.blob;
-        if ((reinterpret_cast<uintptr_t>(b) & 15u) != 0u) {
-            set_status(hdr, kStDeviceCheck);
-            b = nullptr;
+    if (blockIdx.x == 0) {
+        if (threadIdx.x == 0) {
+            hdr->n_unique = 1u;
+            const uint8_t *b = p.blob;
+            if ((reinterpret_cast<uintptr_t>(b) & 15u) != 0u) {
+                set_status(hdr, kStDeviceCheck);
+                b = nullptr;
+            }
+            reinterpret_cast<const uint8_t **>(p.ws + p.L.uniq_blob)[0] = b;
+            reinterpret_cast<uint32_t *>(p.ws + p.L.uniq_mask)[0] = (1u << p.Tc) - 1u;
+            if (b != nullptr) write_expert_tmaps(p.ws, p.L, 0, b, p.tmpl);
         }
-        reinterpret_cast<const uint8_t **>(p.ws + p.L.uniq_blob)[0] = b;
-        reinterpret_cast<uint32_t *>(p.ws + p.L.uniq_mask)[0] = (1u << p.Tc) - 1u;
+        if (threadIdx.x < kChunk) {
+            const int t = threadIdx.x;
+            reinterpret_cast<int8_t *>(p.ws + p.L.uniq_slot)[t] = t < p.Tc ? 0 : -1;
+            reinterpret_cast<float *>(p.ws + p.L.wt)[t * p.L.k] = 1.0f;
+        }
     }
-    if (threadIdx.x < kChunk) {
-        const int t = threadIdx.x;
-        reinterpret_cast<int8_t *>(p.ws + p.L.uniq_slot)[t] = t < p.Tc ? 0 : -1;
-        reinterpret_cast<float *>(p.ws + p.L.wt)[t * p.L.k] = 1.0f;
-        reinterpret_cast<uint32_t *>(p.ws + p.L.hmax)[t * p.L.k] = 0u;
-    }
-    build_x_f16(p.x, p.Tc, p.d, p.ws, p.L);
-    __threadfence();
+    build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L, blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5),
+                   gridDim.x * (blockDim.x >> 5));
     pdl_trigger();
 }
 

@@ -1,6 +1,8 @@
 // C ABI of the k3moe library: argument validation, workspace layout and the
 // launch sequence of each entry point.  Declarations and the contract of
 // every function are in include/k3moe.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -31,8 +33,9 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
 
-k3moe_status cuda_fail(cudaError_t e) {
+k3moe_status cuda_fail(cudaError_t e, const char *where = nullptr) {
     g_last_error = cudaGetErrorString(e);
+    if (where) g_last_error = std::string(where) + ": " + g_last_error;
     return K3MOE_ERR_CUDA;
 }
 
@@ -41,7 +44,6 @@ cudaError_t set_smem(Kern kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-#define K3_GU_LIST(X) X(1) X(2) X(4) X(8) X(14) X(16)
 #define K3_DN_LIST(X) X(2, 1) X(2, 3) X(2, 6) X(4, 1) X(4, 3) X(4, 6) X(12, 1) X(12, 3) \
     X(12, 6) X(24, 1) X(24, 3) X(24, 6)
 
@@ -58,11 +60,10 @@ k3moe_status device_info(DeviceInfo **out) {
         if (e != cudaSuccess) return cuda_fail(e);
         const int big = kSmemLimit;
         cudaError_t r = set_smem(route_shared_kernel, kRouteTok * 8192 * 4);
-#define K3_SET_GU(a) if (r == cudaSuccess) r = set_smem(expert_gu_kernel<a>, big);
+        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<true>, big);
+        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<false>, big);
 #define K3_SET_DN(a, b) if (r == cudaSuccess) r = set_smem(expert_down_kernel<a, b>, big);
-        K3_GU_LIST(K3_SET_GU)
         K3_DN_LIST(K3_SET_DN)
-#undef K3_SET_GU
 #undef K3_SET_DN
         if (r != cudaSuccess) return cuda_fail(r);
         di.ready = true;
@@ -77,10 +78,12 @@ int shared_ff(const k3moe_dims *dm) {
     return (dm->flags & K3MOE_NO_SHARED) ? 0 : dm->ff_shared;
 }
 
-int gu_stages(int d) {
-    for (int n = kMaxStages; n >= 2; --n)
-        if (gu_smem_bytes(d, n) <= kSmemLimit) return n;
-    return 0;
+// Pipeline depth of the tensor-core kernels: as many stages as fit in shared
+// memory and in the TMEM scale columns (8 stages after the accumulators).
+int umma_stages(bool gu) {
+    int n = (kSmemLimit - umma_smem_bytes(gu, 0)) / umma_stage_bytes(gu);
+    const int cap = 8;
+    return n < cap ? n : cap;
 }
 int dn_stages(int ff, int ffs) {
     for (int n = kMaxStages; n >= 2; --n)
@@ -98,7 +101,6 @@ k3moe_status check_dims(const k3moe_dims *dm) {
         return K3MOE_ERR_INVALID_ARGUMENT;
     if (dm->ff_shared < 0 || dm->ff_shared > 3072 || dm->ff_shared % 64)
         return K3MOE_ERR_UNSUPPORTED_SHAPE;
-    if (gu_stages(dm->d) == 0) return K3MOE_ERR_UNSUPPORTED_SHAPE;
     if (dn_stages(dm->ff, dm->ff_shared) == 0) return K3MOE_ERR_UNSUPPORTED_SHAPE;
     return K3MOE_OK;
 }
@@ -128,22 +130,78 @@ cudaError_t launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
 }
 
 
-cudaError_t launch_gu(const DeviceInfo &di, GUParams gp, cudaStream_t st) {
-    const int need = (gp.d / 32 + 15) / 16;
-    const int nbw = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : need <= 8 ? 8 : need <= 14 ? 14 : 16;
-    gp.nst = gu_stages(gp.d);
-    const int smem = gu_smem_bytes(gp.d, gp.nst);
-    const dim3 grid(di.sms), block(kGUThreads);
-#define K3_LAUNCH_GU(a) \
-    if (nbw == a) return launch(expert_gu_kernel<a>, grid, block, smem, st, true, gp);
-    K3_GU_LIST(K3_LAUNCH_GU)
-#undef K3_LAUNCH_GU
-    return cudaErrorInvalidValue;
+// ------------------------------------------------------ tensor maps --
+// Templates of the two nibble-plane tensor maps (u8 elements, 128 x 128-byte
+// boxes, 128-byte swizzle): W_g / W_u (ff rows of d/2 bytes) and W_d (d rows
+// of ff/2 bytes).  The device copies them per selected expert and points the
+// copy at that expert's plane, so the encoded address is a placeholder.
+// The encoder is reached through the runtime's driver entry point, so the
+// library does not link the driver library itself.
+struct TmapCache {
+    int d = 0, ff = 0;
+    uint4 t[2][8];
+};
+TmapCache g_tmaps[16];
+int g_ntmaps = 0;
+
+k3moe_status tmap_templates(int d, int ff, void *placeholder, uint4 (&out)[2][8]) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (int i = 0; i < g_ntmaps; ++i)
+        if (g_tmaps[i].d == d && g_tmaps[i].ff == ff) {
+            memcpy(out, g_tmaps[i].t, sizeof(out));
+            return K3MOE_OK;
+        }
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (q != cudaDriverEntryPointSuccess || !fn) {
+            g_last_error = "cuTensorMapEncodeTiled is not available";
+            return K3MOE_ERR_CUDA;
+        }
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    CUtensorMap m[2];
+    for (int i = 0; i < 2; ++i) {
+        const cuuint64_t cols = (cuuint64_t)(i == 0 ? d : ff) / 2, rows = (cuuint64_t)(i == 0 ? ff : d);
+        const cuuint64_t dims[2] = {cols, rows};
+        const cuuint64_t strides[1] = {cols};
+        const cuuint32_t box[2] = {128, (cuuint32_t)kTileM};
+        const cuuint32_t es[2] = {1, 1};
+        CUresult r = encode(&m[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, placeholder, dims, strides, box, es,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            g_last_error = "cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")";
+            return K3MOE_ERR_CUDA;
+        }
+    }
+    static_assert(sizeof(CUtensorMap) == 128, "tensor map is 128 bytes");
+    memcpy(out, m, sizeof(out));
+    if (g_ntmaps < 16) {
+        g_tmaps[g_ntmaps].d = d;
+        g_tmaps[g_ntmaps].ff = ff;
+        memcpy(g_tmaps[g_ntmaps].t, m, sizeof(m));
+        ++g_ntmaps;
+    }
+    return K3MOE_OK;
+}
+
+template <bool GU>
+cudaError_t launch_umma(const DeviceInfo &di, UmmaParams up, cudaStream_t st) {
+    up.nst = umma_stages(GU);
+    const int smem = umma_smem_bytes(GU, up.nst);
+    const int g = di.sms < kMaxCtas ? di.sms : kMaxCtas;
+    return launch(umma_expert_kernel<GU>, dim3(g), dim3(kUThreads), smem, st, true, up);
 }
 
 cudaError_t launch_down(const DeviceInfo &di, DownParams dp, cudaStream_t st) {
+    dp.skip_routed = 1;
     const int nq = (dp.ff / 32 + 3) / 4;
-    const int nbq = nq <= 2 ? 2 : nq <= 4 ? 4 : nq <= 12 ? 12 : 24;
+    (void)nq;
+    const int nbq = 2;  // routed rows are skipped: the smallest variant
     const int ns = (dp.ffs / 32 + 15) / 16;
     const int nbs = ns <= 1 ? 1 : ns <= 3 ? 3 : 6;
     dp.nst = dn_stages(dp.ff, dp.ffs);
@@ -240,6 +298,10 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
     uint8_t *xstage = wsb + L.total;
     uint8_t *ystage = xstage + align256((size_t)kChunk * d * 2);
 
+    uint4 tmpl[2][8];
+    s = tmap_templates(d, dims->ff, ws, tmpl);
+    if (s != K3MOE_OK) return s;
+
     for (int c0 = 0; c0 < T; c0 += kChunk) {
         const int Tc = (T - c0) < kChunk ? (T - c0) : kChunk;
         const uint16_t *xc;
@@ -271,26 +333,37 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         rp.blobs = expert_blobs;
         rp.idx_out = idx_out ? idx_out + (size_t)c0 * dims->top_k : nullptr;
         rp.w_out = w_out ? w_out + (size_t)c0 * dims->top_k : nullptr;
+        memcpy(rp.tmpl, tmpl, sizeof(tmpl));
         EventHook none;
         EventHook &hk = hook ? *hook : none;
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
         e = launch_route(*di, rp, st);
-        if (e != cudaSuccess) return cuda_fail(e);
+        if (e != cudaSuccess) return cuda_fail(e, "router launch");
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
 
-        GUParams gp{xc, Tc, d, dims->ff, wsb, L};
-        e = launch_gu(*di, gp, st);
-        if (e != cudaSuccess) return cuda_fail(e);
+        UmmaParams up{};
+        up.Tc = Tc;
+        up.d = d;
+        up.ff = dims->ff;
+        up.k = dims->top_k;
+        up.ws = wsb;
+        up.L = L;
+        up.has_shared = ffs > 0;
+        up.out_fp32 = out32;
+        up.y = yc;
+        e = launch_umma<true>(*di, up, st);
+        if (e != cudaSuccess) return cuda_fail(e, "gate/up launch");
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
 
-        DownParams dp{Tc, d, dims->ff, ffs, reinterpret_cast<const uint16_t *>(shared_wd), wsb, L};
-        e = launch_down(*di, dp, st);
-        if (e != cudaSuccess) return cuda_fail(e);
-        if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
+        if (ffs > 0) {
+            DownParams dp{Tc, d, dims->ff, ffs, reinterpret_cast<const uint16_t *>(shared_wd), wsb, L};
+            e = launch_down(*di, dp, st);
+            if (e != cudaSuccess) return cuda_fail(e, "shared down launch");
+            if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
+        }
 
-        CombineParams cp{Tc, d, dims->top_k, ffs > 0, out32, wsb, L, yc};
-        e = launch(combine_kernel, dim3((d + 1023) / 1024, Tc), dim3(256), 0, st, true, cp);
-        if (e != cudaSuccess) return cuda_fail(e);
+        e = launch_umma<false>(*di, up, st);
+        if (e != cudaSuccess) return cuda_fail(e, "down launch");
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
 
         if (from_host) {
@@ -377,22 +450,39 @@ k3moe_status k3moe_expert_ffn(const void *x, int32_t T, const uint8_t *blob,
     uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
     const int d = dims->d;
     const bool out32 = (dims->flags & K3MOE_OUT_FP32) != 0;
+    uint4 tmpl[2][8];
+    s = tmap_templates(d, dims->ff, ws, tmpl);
+    if (s != K3MOE_OK) return s;
     for (int c0 = 0; c0 < T; c0 += kChunk) {
         const int Tc = (T - c0) < kChunk ? (T - c0) : kChunk;
         const uint16_t *xc = reinterpret_cast<const uint16_t *>(x) + (size_t)c0 * d;
         void *yc = reinterpret_cast<uint8_t *>(out) + (size_t)c0 * d * (out32 ? 4 : 2);
-        SingleParams sp{xc, Tc, d, blob, wsb, L};
-        cudaError_t e = launch(single_expert_setup_kernel, dim3(1), dim3(256), 0, st, false, sp);
-        if (e != cudaSuccess) return cuda_fail(e);
-        GUParams gp{xc, Tc, d, dims->ff, wsb, L};
-        e = launch_gu(*di, gp, st);
-        if (e != cudaSuccess) return cuda_fail(e);
-        DownParams dp{Tc, d, dims->ff, 0, nullptr, wsb, L};
-        e = launch_down(*di, dp, st);
-        if (e != cudaSuccess) return cuda_fail(e);
-        CombineParams cp{Tc, d, 1, false, out32, wsb, L, yc};
-        e = launch(combine_kernel, dim3((d + 1023) / 1024, Tc), dim3(256), 0, st, true, cp);
-        if (e != cudaSuccess) return cuda_fail(e);
+        SingleParams sp{};
+        sp.x = xc;
+        sp.Tc = Tc;
+        sp.d = d;
+        sp.blob = blob;
+        sp.ws = wsb;
+        sp.L = L;
+        memcpy(sp.tmpl, tmpl, sizeof(tmpl));
+        int nblk = (Tc * (d / 32) + 7) / 8;  // one warp per 32-element block
+        if (nblk > di->sms) nblk = di->sms;
+        cudaError_t e = launch(single_expert_setup_kernel, dim3(nblk), dim3(256), 0, st, false, sp);
+        if (e != cudaSuccess) return cuda_fail(e, "setup launch");
+        UmmaParams up{};
+        up.Tc = Tc;
+        up.d = d;
+        up.ff = dims->ff;
+        up.k = 1;
+        up.ws = wsb;
+        up.L = L;
+        up.has_shared = 0;
+        up.out_fp32 = out32;
+        up.y = yc;
+        e = launch_umma<true>(*di, up, st);
+        if (e != cudaSuccess) return cuda_fail(e, "gate/up launch");
+        e = launch_umma<false>(*di, up, st);
+        if (e != cudaSuccess) return cuda_fail(e, "down launch");
     }
     return K3MOE_OK;
 }
@@ -431,7 +521,7 @@ k3moe_status k3moe_layer_timed(const void *x, int32_t T, const float *w_router, 
     k3moe_status s = layer_impl(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu,
                                 shared_wd, dims, y, nullptr, nullptr, ws, ws_bytes, stream, nullptr,
                                 nullptr, &hk);
-    *n_kernels = 4;
+    *n_kernels = shared_ff(dims) > 0 ? 4 : 3;
     return s;
 }
 

@@ -9,6 +9,17 @@ namespace k3 {
 constexpr int kChunk = 8;   // tokens per decode pass
 constexpr int kMaxSeg = 8;  // most warps that share one router/shared row
 
+// Tensor-core path: each activation element enters the MMA as kPieces E2M1
+// values with their own per-32 E8M0 scales; B-operand row n = t*kPieces + p.
+constexpr int kPieces = 6;
+constexpr int kNMax = kChunk * kPieces;  // 48: widest MMA N of a chunk
+constexpr int kSfRow = 64;               // scale words per (K-tile, group): rows n < 64
+constexpr int kTileK = 256;              // weights per K-tile (128 bytes of nibbles per row)
+constexpr int kTileM = 128;              // MMA M: weight rows per item
+constexpr int kMaxCtas = 256;            // grid cap of the tensor-core kernels
+__host__ __device__ inline int act_n(int Tc) { return (Tc * kPieces + 7) & ~7; }
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
@@ -27,8 +38,15 @@ struct Layout {
     size_t ob;         // f32 [kChunk][k+1][d] expert outputs: [0] shared, [1+j] slot j
     size_t part;       // f32 [2][E+ffs][kMaxSeg][4][2] partial sums of rows split between warps
     size_t cnt;        // u32 [2][E+ffs] arrivals per split row (back to 0 after each row)
+    size_t tmap;       // 128-byte tensor maps [umax][3]: W_g, W_u, W_d nibble planes
+    size_t xb;         // u8  [nkt_d][N*128] E2M1 pieces of x (gate/up B operand)
+    size_t xsf;        // u32 [nkt_d][2][kSfRow] their E8M0 scales (byte = block in group)
+    size_t hb;         // u8  [umax][nkt_ff][N*128] pieces of w*h (down B operand)
+    size_t hsf;        // u32 [umax][nkt_ff][2][kSfRow]
+    size_t spart;      // f32 [kMaxCtas][2][2][kChunk][kTileM] split-item partial sums
+    size_t icnt;       // u32 [umax*nrb_ff + nrb_d] arrivals per split item (back to 0)
     size_t total;
-    int d, ff, E, k, ffs;
+    int d, ff, E, k, ffs, umax;
 };
 
 __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int ffs) {
@@ -70,6 +88,23 @@ __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int f
     o = align256(o + (size_t)2 * (E + ffs) * kMaxSeg * 4 * 2 * 4);
     L.cnt = o;
     o = align256(o + (size_t)2 * (E + ffs) * 4);
+    const int umax = E < kChunk * k ? E : kChunk * k;
+    const int nkt_d = ceil_div(d, kTileK), nkt_ff = ceil_div(ff, kTileK);
+    L.umax = umax;
+    L.tmap = o;
+    o = align256(o + (size_t)umax * 3 * 128);
+    L.xb = o;
+    o = align256(o + (size_t)nkt_d * kNMax * 128);
+    L.xsf = o;
+    o = align256(o + (size_t)nkt_d * 2 * kSfRow * 4);
+    L.hb = o;
+    o = align256(o + (size_t)umax * nkt_ff * kNMax * 128);
+    L.hsf = o;
+    o = align256(o + (size_t)umax * nkt_ff * 2 * kSfRow * 4);
+    L.spart = o;
+    o = align256(o + (size_t)kMaxCtas * 2 * 2 * kChunk * kTileM * 4);
+    L.icnt = o;
+    o = align256(o + ((size_t)umax * ceil_div(ff, kTileM) + ceil_div(d, kTileM)) * 4);
     L.total = o;
     return L;
 }

@@ -1,0 +1,486 @@
+// Routed-expert projections on the 5th-generation tensor cores
+// (tcgen05.mma kind::mxf4, block-scaled E2M1 x E2M1 with E8M0 scales).
+//
+// The packed expert blob goes straight into the tensor core: TMA copies
+// 128-row x 128-byte boxes of a nibble plane into shared memory (128-byte
+// swizzle) and the E8M0 scale bytes are written into tensor memory, so the
+// MMA itself decodes every 4-bit weight and applies its block scale -- no
+// per-weight thread work (the kimi-k3-in-c project card ("P053"), core
+// features: multiply directly on the packed nibbles, never dequantise).
+//
+// Activations (x for gate/up, w*h for down) are carried as kPieces E2M1
+// pieces per element, each 32-element block of each piece with its own E8M0
+// scale chosen from the block's remaining residual; the pieces sum exactly
+// to the activation up to the last residual (about 2^-19 of the block's
+// largest element).  Piece p of token t is B-operand row n = t*kPieces + p,
+// so a whole chunk of tokens and pieces is one MMA of N = act_n(Tc) columns
+// and the pieces are summed per token in the epilogue.
+//
+// Work: "items" of 128 weight rows, each a run of K-tiles (256 weights of
+// every row); the K-tiles of all items are split evenly over the CTAs
+// (stream-K).  An item split between CTAs is finished by the last one to
+// arrive, summing the per-token partials in piece order (deterministic).
+//
+// CTA roles (320 threads): warps 0-3 epilogue (one TMEM lane quadrant each),
+// warps 4-7 write the scale factors of each stage into TMEM (each writes the
+// same values into its own quadrant, as the MMA reads them replicated),
+// warp 8 issues the TMA / bulk copies, warp 9 issues the MMAs.
+#pragma once
+
+#include "common.cuh"
+#include "layout.cuh"
+#include "umma.cuh"
+
+namespace k3 {
+
+constexpr int kUThreads = 320;
+constexpr int kAtile = kTileM * 128;  // one A box: 128 rows x 128 bytes (16 KB)
+
+// ---------------------------------------------------------------- pieces --
+// One 32-element activation block (element = this lane's v) of token t ->
+// kPieces E2M1 pieces.  Piece p: scale exponent e from the largest |residual|
+// r of the block (smallest e with max|r| <= 6 * 2^e), codes = r / 2^e rounded
+// to the nearest E2M1 value, residual r -= code * 2^e (exact in fp32: the
+// subtracted value is a multiple of the residual's unit in the last place).
+// Writes the 16-byte nibble row of each piece into a K-tile of the B operand
+// (no-swizzle K-major core matrices, N rows, this block is 16-byte chunk c of
+// the tile) and its scale byte into the tile's scale words
+// (sfw[(c/4)*kSfRow + n], byte c%4).  All 32 lanes of the warp call it.
+__device__ __forceinline__ void quantize_pieces(float v, int lane, int t, int c, int N, uint8_t *tile,
+                                                uint8_t *sfw) {
+    float r = v;
+#pragma unroll
+    for (int p = 0; p < kPieces; ++p) {
+        float amax = fabsf(r);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const uint32_t bits = __float_as_uint(amax);
+        // amax = 1.f * 2^e0: 6 * 2^(e0-2) = 1.5 * 2^e0 covers 1.f <= 1.5
+        int e = (int)(bits >> 23) - 127 - 2 + ((bits & 0x7FFFFFu) > 0x400000u ? 1 : 0);
+        e = max(-126, min(126, e));
+        const float s = r * exp2i(-e);
+        const float m = fabsf(s);
+        float q;
+        if (m < 2.f) q = rintf(m * 2.f) * 0.5f;
+        else if (m < 4.f) q = rintf(m);
+        else q = rintf(m * 0.5f) * 2.f;
+        uint32_t code = q < 2.f ? (uint32_t)(q * 2.f) : (q < 4.f ? (uint32_t)q + 2u : (q < 5.f ? 6u : 7u));
+        if (s < 0.f && code != 0u) code |= 8u;
+        r -= copysignf(q, s) * exp2i(e);
+        uint32_t w = code << (4 * (lane & 7));
+        w |= __shfl_xor_sync(0xffffffffu, w, 1);
+        w |= __shfl_xor_sync(0xffffffffu, w, 2);
+        w |= __shfl_xor_sync(0xffffffffu, w, 4);
+        const int n = t * kPieces + p;
+        if ((lane & 7) == 0)
+            *reinterpret_cast<uint32_t *>(tile + (c * (N / 8) + n / 8) * 128 + (n % 8) * 16 + (lane >> 3) * 4) = w;
+        if (lane == 0) sfw[((c >> 2) * kSfRow + n) * 4 + (c & 3)] = (uint8_t)(e + 127);
+    }
+}
+
+// x of the chunk -> pieces (gate/up B operand), blocks spread over every warp
+// of the grid (warp index gw of nw).
+__device__ void build_x_pieces(const uint16_t *x, int Tc, int d, uint8_t *ws, const Layout &L, int gw,
+                               int nw) {
+    const int lane = threadIdx.x & 31, N = act_n(Tc), nb = d / 32;
+    for (int i = gw; i < Tc * nb; i += nw) {
+        const int t = i / nb, b = i - t * nb;
+        const float v = __uint_as_float((uint32_t)x[(size_t)t * d + 32 * b + lane] << 16);
+        const int kt = b >> 3;
+        quantize_pieces(v, lane, t, b & 7, N, ws + L.xb + (size_t)kt * N * 128,
+                        ws + L.xsf + (size_t)kt * 2 * kSfRow * 4);
+    }
+}
+
+// Tensor maps of distinct expert u: copies of the host-encoded templates
+// (W_g/W_u share one: ff rows of d/2 bytes; W_d: d rows of ff/2 bytes)
+// pointed at the expert's nibble planes.  One thread.
+__device__ void write_expert_tmaps(uint8_t *ws, const Layout &L, int u, const uint8_t *blob,
+                                   const uint4 (&tmpl)[2][8]) {
+    const size_t mat = (size_t)L.d * L.ff;
+    uint8_t *dst = ws + L.tmap + (size_t)u * 3 * 128;
+    const uint8_t *addr[3] = {blob, blob + mat / 2 + mat / 32, blob + mat + mat / 16};
+#pragma unroll
+    for (int m = 0; m < 3; ++m) {
+        uint4 *o = reinterpret_cast<uint4 *>(dst + m * 128);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j] = tmpl[m == 2 ? 1 : 0][j];
+        umma::tmap_set_address(dst + m * 128, addr[m]);
+    }
+    umma::tmap_release();
+}
+
+// ---------------------------------------------------------------- kernel --
+struct UmmaParams {
+    int Tc, d, ff, k;
+    uint8_t *ws;
+    Layout L;
+    int nst;          // pipeline stages
+    // down only
+    int has_shared;   // add the shared expert's output (ob slot 0)
+    int out_fp32;     // y in fp32 (else bf16, rounded once)
+    void *y;          // [Tc][d] of this chunk
+};
+
+__host__ __device__ inline int umma_stage_bytes(bool gu) { return (gu ? 2 : 1) * kAtile + kNMax * 128; }
+// TMEM scale columns of one stage, every group aligned: A scales 8 per matrix
+// (2 groups x 4 row blocks), then B scales (group g at +4g, up to 2 columns).
+__host__ __device__ inline int umma_sf_cols(bool gu) { return gu ? 32 : 16; }
+__host__ __device__ inline int umma_smem_bytes(bool gu, int nst) {
+    return 1024 + nst * umma_stage_bytes(gu) + 256;
+}
+
+// Load the (up to) 8 scale bytes of one weight row for one K-tile: nks valid
+// 2-byte pairs (one per MMA k-step); zero beyond.
+__device__ __forceinline__ uint2 load_sf8(const uint8_t *p, int nks) {
+    if (nks == 4 && (reinterpret_cast<uintptr_t>(p) & 7u) == 0u) return __ldg(reinterpret_cast<const uint2 *>(p));
+    const unsigned short *h = reinterpret_cast<const unsigned short *>(p);
+    uint32_t w0 = 0u, w1 = 0u;
+    if (nks > 0) w0 |= (uint32_t)__ldg(h);
+    if (nks > 1) w0 |= (uint32_t)__ldg(h + 1) << 16;
+    if (nks > 2) w1 |= (uint32_t)__ldg(h + 2);
+    if (nks > 3) w1 |= (uint32_t)__ldg(h + 3) << 16;
+    return make_uint2(w0, w1);
+}
+
+template <bool GU>
+__global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    constexpr int NMAT = GU ? 2 : 1;
+    constexpr int SB = NMAT * kAtile + kNMax * 128;
+    constexpr int SFC = GU ? 32 : 16;  // TMEM scale columns per stage (8-aligned)
+    const int nst = p.nst;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + nst * SB);
+    uint64_t *empty = full + nst;
+    uint64_t *afull = empty + nst;
+    uint64_t *aempty = afull + 2;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(aempty + 2);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(tslot + 1);
+    volatile int *s_last = s_abort + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Layout &L = p.L;
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + L.hdr);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nst; ++s) {
+            mbar_init(&full[s], 5);  // TMA thread + 4 scale warps
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&afull[b], 1);
+            mbar_init(&aempty[b], 4);
+        }
+        fence_mbar_init();
+        *s_abort = 0;
+    }
+    constexpr uint32_t kCols = GU ? 512u : 256u;
+    if (warp == 0) umma::tmem_alloc(tslot, kCols);
+    umma::fence_before();
+    __syncthreads();
+    umma::fence_after();
+    const uint32_t tbase = *tslot;
+    pdl_wait();
+    pdl_trigger();
+
+    const int Tc = p.Tc, N = act_n(Tc);
+    const int U = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_unique);
+    const int K = GU ? p.d : p.ff;   // reduction length
+    const int M = GU ? p.ff : p.d;   // weight rows
+    const int nkt = ceil_div(K, kTileK);
+    const int nrb = ceil_div(M, kTileM);
+    const int upi = GU ? nkt : U * nkt;  // units (K-tiles) per item
+    const int n_items = GU ? U * nrb : nrb;
+    const int total = n_items * upi;
+    const int G = min((int)gridDim.x, max(total, 1));
+    const int cta = blockIdx.x;
+    auto start = [&](int c) { return (int)(((long long)c * total) / G); };
+    auto owner = [&](int unit) { return (int)((((long long)unit + 1) * G - 1) / total); };
+    const int a = cta < G ? start(cta) : 0, b = cta < G ? start(cta + 1) : 0;
+    const size_t mat = (size_t)p.d * p.ff;
+    const uint8_t *const *ublob = reinterpret_cast<const uint8_t *const *>(p.ws + L.uniq_blob);
+    const uint32_t idesc = umma::idesc_mxf4(N);
+    // TMEM columns: accumulators [buf][mat] at (buf*NMAT + mat)*64 (N <= 64), then
+    // the scale columns of each stage from sf0
+    const uint32_t sf0 = GU ? 256u : 128u;
+
+    // Bounded wait that gives up at once after any role has given up, so a
+    // failure ends the kernel in bounded time.
+    auto wait = [&](uint64_t *bar, uint32_t parity) {
+        if (*s_abort) return false;
+        if (mbar_wait_bounded(bar, parity, hdr)) return true;
+        *s_abort = 1;
+        return false;
+    };
+
+    struct Unit {
+        int item, u, rb, kt;
+    };
+    auto decode = [&](int unit) {
+        Unit x;
+        x.item = unit / upi;
+        const int r = unit - x.item * upi;
+        if (GU) {
+            x.u = x.item / nrb;
+            x.rb = x.item - x.u * nrb;
+            x.kt = r;
+        } else {
+            x.u = r / nkt;
+            x.kt = r - x.u * nkt;
+            x.rb = x.item;
+        }
+        return x;
+    };
+
+    if (warp == 8) {
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            int last_u = -1;
+            for (int unit = a, it = 0; unit < b && !*s_abort; ++unit, ++it) {
+                const Unit x = decode(unit);
+                const int s = it % nst;
+                if (it >= nst && !wait(&empty[s], (uint32_t)(((it / nst) + 1) & 1))) break;
+                uint8_t *st = smem + s * SB;
+                const uint8_t *blob = ublob[x.u];
+                const uint8_t *bsrc = GU ? p.ws + L.xb + (size_t)x.kt * N * 128
+                                         : p.ws + L.hb + ((size_t)x.u * nkt + x.kt) * N * 128;
+                if (blob != nullptr) {
+                    const uint8_t *maps = p.ws + L.tmap + (size_t)x.u * 3 * 128;
+                    if (x.u != last_u) {
+                        if (GU) {
+                            umma::tmap_acquire(maps);
+                            umma::tmap_acquire(maps + 128);
+                        } else {
+                            umma::tmap_acquire(maps + 256);
+                        }
+                        last_u = x.u;
+                    }
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * kAtile + N * 128));
+                    if (GU) {
+                        umma::tma_load_2d(st, maps, x.kt * 128, x.rb * kTileM, &full[s]);
+                        umma::tma_load_2d(st + kAtile, maps + 128, x.kt * 128, x.rb * kTileM, &full[s]);
+                    } else {
+                        umma::tma_load_2d(st, maps + 256, x.kt * 128, x.rb * kTileM, &full[s]);
+                    }
+                } else {
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)(N * 128));
+                }
+                bulk_g2s(st + NMAT * kAtile, bsrc, (uint32_t)(N * 128), &full[s]);
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // --------------------------------------- scale factors -> TMEM --
+        const uint32_t lb = umma::lane_base(warp);
+        for (int unit = a, it = 0; unit < b; ++unit, ++it) {
+            const Unit x = decode(unit);
+            const int s = it % nst;
+            // lane 0 decides, the warp follows (the TMEM stores are warp-collective)
+            int go = 0;
+            if (lane == 0) go = it < nst ? !*s_abort : wait(&empty[s], (uint32_t)(((it / nst) + 1) & 1));
+            if (!__shfl_sync(0xffffffffu, go, 0)) break;
+            const uint8_t *blob = ublob[x.u];
+            const int nks = min(4, (K - x.kt * kTileK) / 64);
+            const uint32_t col = tbase + lb + sf0 + (uint32_t)(s * SFC);
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) {
+                const uint8_t *plane = nullptr;
+                if (blob != nullptr)
+                    plane = GU ? (m == 0 ? blob + mat / 2 : blob + mat + mat / 32) : blob + mat + mat / 16 + mat / 2;
+                uint32_t w[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int row = x.rb * kTileM + 32 * j + lane;
+                    uint2 v = make_uint2(0u, 0u);
+                    if (plane != nullptr && row < M) v = load_sf8(plane + (size_t)row * (K / 32) + x.kt * 8, nks);
+                    w[j] = v.x;      // group 0: k-steps 0, 1
+                    w[4 + j] = v.y;  // group 1: k-steps 2, 3
+                }
+                umma::st8(col + 8 * m, w);
+            }
+            const uint32_t *sfb = GU ? reinterpret_cast<const uint32_t *>(p.ws + L.xsf) + (size_t)x.kt * 2 * kSfRow
+                                     : reinterpret_cast<const uint32_t *>(p.ws + L.hsf) +
+                                           ((size_t)x.u * nkt + x.kt) * 2 * kSfRow;
+            {
+                // group g, row block j (rows 32j..) at column 8*NMAT + 4g + j
+                uint32_t w[8] = {__ldcg(sfb + lane), __ldcg(sfb + 32 + lane), 0u, 0u,
+                                 __ldcg(sfb + kSfRow + lane), __ldcg(sfb + kSfRow + 32 + lane), 0u, 0u};
+                umma::st8(col + 8 * NMAT, w);
+            }
+            umma::wait_st();
+            umma::fence_before();
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&full[s])) : "memory");
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------- MMA issuer --
+        if (lane == 0) {
+            int it = 0, seg = 0;
+            for (int unit = a; unit < b && !*s_abort; ++seg) {
+                const int item = unit / upi;
+                const int seg_end = min(b, (item + 1) * upi);
+                const int buf = seg & 1;
+                if (seg >= 2 && !wait(&aempty[buf], (uint32_t)(((seg >> 1) + 1) & 1))) break;
+                umma::fence_after();
+                const uint32_t dcol = tbase + (uint32_t)(buf * NMAT * 64);
+                for (int un = unit; un < seg_end; ++un, ++it) {
+                    const Unit x = decode(un);
+                    const int s = it % nst;
+                    if (!wait(&full[s], (uint32_t)((it / nst) & 1))) break;
+                    umma::fence_after();
+                    const uint32_t st = smem_u32(smem + s * SB);
+                    const uint32_t sfc = tbase + sf0 + (uint32_t)(s * SFC);
+                    const int nks = min(4, (K - x.kt * kTileK) / 64);
+                    for (int sk = 0; sk < nks; ++sk) {
+                        const uint32_t grp = (uint32_t)(sk >> 1), sfid = (uint32_t)(2 * (sk & 1));
+                        const uint32_t id = umma::idesc_sf_id(idesc, sfid);
+                        const uint64_t bdesc =
+                            umma::smem_desc(st + NMAT * kAtile + (uint32_t)(2 * sk * (N / 8) * 128),
+                                            (uint32_t)((N / 8) * 128), 128u, umma::kLayoutNone);
+                        const uint32_t sfb = (sfc + 8 * NMAT + grp * 4) | (sfid << 30);
+                        const uint32_t acc = (un != unit || sk != 0) ? 1u : 0u;
+#pragma unroll
+                        for (int m = 0; m < NMAT; ++m) {
+                            const uint64_t adesc = umma::smem_desc(st + (uint32_t)(m * kAtile + 32 * sk), 16u, 1024u,
+                                                                   umma::kLayoutSw128);
+                            const uint32_t sfa = (sfc + 8 * m + grp * 4) | (sfid << 30);
+                            umma::mma_mxf4(dcol + (uint32_t)(m * 64), adesc, bdesc, id, acc, sfa, sfb);
+                        }
+                    }
+                    umma::commit(&empty[s]);
+                }
+                umma::commit(&afull[buf]);
+                unit = seg_end;
+            }
+        }
+    } else {
+        // --------------------------------------------------- epilogue --
+        const uint32_t lb = umma::lane_base(warp);
+        const int rowl = 32 * warp + lane;  // row of the 128-row item
+        float* spart = reinterpret_cast<float *>(p.ws + L.spart);
+        uint32_t *icnt = reinterpret_cast<uint32_t *>(p.ws + L.icnt) + (GU ? 0 : L.umax * ceil_div(p.ff, kTileM));
+        int seg = 0;
+        for (int unit = a; unit < b; ++seg) {
+            const int item = unit / upi;
+            const int seg_end = min(b, (item + 1) * upi);
+            const int buf = seg & 1;
+            float acc[NMAT][kChunk];
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                for (int t = 0; t < kChunk; ++t) acc[m][t] = 0.f;
+            // every epilogue warp runs the same sequence of named barriers, so
+            // after a failed wait it carries on (with unused values)
+            if (lane == 0) wait(&afull[buf], (uint32_t)((seg >> 1) & 1));
+            __syncwarp();
+            umma::fence_after();
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) {
+#pragma unroll
+                for (int n0 = 0; n0 < kNMax; n0 += 8) {
+                    if (n0 < N) {
+                        uint32_t r[8];
+                        umma::ld8(tbase + lb + (uint32_t)((buf * NMAT + m) * 64 + n0), r);
+                        umma::wait_ld();
+#pragma unroll
+                        for (int jj = 0; jj < 8; ++jj) {
+                            const int t = (n0 + jj) / kPieces;
+                            if (t < kChunk) acc[m][t] += __uint_as_float(r[jj]);
+                        }
+                    }
+                }
+            }
+            umma::fence_before();
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&aempty[buf])) : "memory");
+
+            const bool whole = unit == item * upi && seg_end == (item + 1) * upi;
+            bool fin = whole;
+            if (!whole) {
+                const int slot = unit == a ? 0 : 1;
+                float *sp = spart + (size_t)((cta * 2 + slot) * 2) * kChunk * kTileM;
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                    for (int t = 0; t < kChunk; ++t)
+                        if (t < Tc) sp[(m * kChunk + t) * kTileM + rowl] = acc[m][t];
+                umma::bar_sync(1, 128);
+                if (threadIdx.x == 0) {
+                    const int c0 = owner(item * upi), c1 = owner((item + 1) * upi - 1);
+                    const uint32_t old = atom_add_acq_rel(icnt + item, 1u);
+                    const int last = old == (uint32_t)(c1 - c0);
+                    if (last) icnt[item] = 0u;
+                    *s_last = last;
+                }
+                umma::bar_sync(1, 128);
+                fin = *s_last != 0;
+                if (fin) {
+                    // sum every piece of the item in K order
+                    const int c0 = owner(item * upi), c1 = owner((item + 1) * upi - 1);
+#pragma unroll
+                    for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                        for (int t = 0; t < kChunk; ++t) acc[m][t] = 0.f;
+                    for (int cc = c0; cc <= c1; ++cc) {
+                        const int sl = start(cc) < item * upi ? 1 : 0;
+                        const float *q = spart + (size_t)((cc * 2 + sl) * 2) * kChunk * kTileM;
+#pragma unroll
+                        for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                            for (int t = 0; t < kChunk; ++t)
+                                if (t < Tc) acc[m][t] += __ldcg(q + (m * kChunk + t) * kTileM + rowl);
+                    }
+                }
+            }
+            if (fin) {
+                if constexpr (GU) {
+                    const Unit x = decode(item * upi);
+                    const int f = x.rb * kTileM + rowl;  // ff row of this thread
+                    const uint8_t *blob = ublob[x.u];
+                    const uint32_t msk = __ldcg(reinterpret_cast<const uint32_t *>(p.ws + L.uniq_mask) + x.u);
+                    const int8_t *uslot = reinterpret_cast<const int8_t *>(p.ws + L.uniq_slot) + x.u * kChunk;
+                    const float *wt = reinterpret_cast<const float *>(p.ws + L.wt);
+                    const int nkt_ff = ceil_div(p.ff, kTileK);
+                    const int blk = x.rb * 4 + warp;  // 32-row block of ff
+                    const int kt = blk >> 3;
+                    uint8_t *tile = p.ws + L.hb + ((size_t)x.u * nkt_ff + kt) * N * 128;
+                    uint8_t *sfw = p.ws + L.hsf + ((size_t)x.u * nkt_ff + kt) * 2 * kSfRow * 4;
+#pragma unroll
+                    for (int t = 0; t < kChunk; ++t) {
+                        if (t < Tc) {
+                            float h = 0.f;
+                            if (blob != nullptr && ((msk >> t) & 1u) && f < p.ff) {
+                                const int j = uslot[t];
+                                h = silu_mul(acc[0][t], acc[1][t]) * __ldcg(wt + t * p.k + j);
+                            }
+                            quantize_pieces(h, lane, t, blk & 7, N, tile, sfw);
+                        }
+                    }
+                } else {
+                    const int row = item * kTileM + rowl;
+                    if (row < p.d) {
+                        const float *ob = reinterpret_cast<const float *>(p.ws + L.ob);
+#pragma unroll
+                        for (int t = 0; t < kChunk; ++t) {
+                            if (t < Tc) {
+                                float y = acc[0][t];
+                                if (p.has_shared) y += __ldcg(ob + (size_t)t * (p.k + 1) * p.d + row);
+                                if (p.out_fp32)
+                                    reinterpret_cast<float *>(p.y)[(size_t)t * p.d + row] = y;
+                                else
+                                    reinterpret_cast<__nv_bfloat16 *>(p.y)[(size_t)t * p.d + row] = __float2bfloat16_rn(y);
+                            }
+                        }
+                    }
+                }
+            }
+            unit = seg_end;
+        }
+    }
+    umma::fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        umma::fence_after();
+        umma::tmem_dealloc(tbase, kCols);
+    }
+}
+
+}  // namespace k3
