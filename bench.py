@@ -55,9 +55,23 @@ def alg_bytes(cfg, U):
 
 
 def gu_bytes(cfg, U, pairs):
-    """Algorithmic bytes of one routed gate/up launch: W_g and W_u of each
-    distinct expert (nibbles + scales), x in, SwiGLU activations out."""
-    return U * 2 * cfg.d * cfg.ff * 17 // 32 + cfg.T * cfg.d * 2 + pairs * cfg.ff * 4
+    """Algorithmic bytes of one gate/up launch: W_g and W_u of each distinct
+    routed expert (nibbles + scales) and of the bf16 shared expert, x in, the
+    SwiGLU activations out (counted as fp32, one per selected pair and token)."""
+    return (U * 2 * cfg.d * cfg.ff * 17 // 32 + 2 * cfg.d * cfg.ff_shared * 2 + cfg.T * cfg.d * 2
+            + (pairs * cfg.ff + cfg.T * cfg.ff_shared) * 4)
+
+
+def down_bytes(cfg, U, pairs):
+    """Algorithmic bytes of one down launch: W_d of each distinct routed expert
+    and of the shared expert, the activations in (fp32 equivalent), y out."""
+    return (U * cfg.d * cfg.ff * 17 // 32 + cfg.d * cfg.ff_shared * 2
+            + (pairs * cfg.ff + cfg.T * cfg.ff_shared) * 4 + cfg.T * cfg.d * (4 if cfg.out_fp32 else 2))
+
+
+def route_bytes(cfg):
+    """Algorithmic bytes of one route launch: fp32 router weights, x in."""
+    return cfg.E * cfg.d * 4 + cfg.T * cfg.d * 2
 
 
 def load_peaks():
@@ -274,8 +288,7 @@ def main():
     value = world * T * args.steps / (total_ms / 1000.0)
 
     # per-kernel durations (events recorded between the library's kernels)
-    kernels = (["route_shared", "expert_gu", "shared_down", "expert_down"] if cfg.ff_shared > 0
-               else ["route_shared", "expert_gu", "expert_down"])
+    kernels = ["route", "expert_gu", "expert_down"]
     per_kernel = {}
     if single_pass:
         for j, name in enumerate(kernels):
@@ -338,10 +351,14 @@ def main():
         "layer_hbm_gbs": round(layer_gbs, 1),
         "layer_hbm_frac": round(layer_gbs / peak, 4),
         "per_kernel_ms": {k: round(v, 5) for k, v in per_kernel.items()},
+        "per_kernel_gbs": {k: round(b / (per_kernel[k] / 1000.0) / 1e9, 1)
+                           for k, b in (("route", route_bytes(cfg)), ("expert_gu", gu_bytes(cfg, U, pairs)),
+                                        ("expert_down", down_bytes(cfg, U, pairs)))
+                           if per_kernel.get(k)},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": (4 if cfg.ff_shared > 0 else 3) * chunks * args.steps,
+        "gpu_launches": 3 * chunks * args.steps,
         "clocks": clk,
     }
     if rank == 0:

@@ -40,14 +40,17 @@
  *              fp32 with K3MOE_OUT_FP32
  *   idx        int32 [T][k], weight fp32 [T][k]
  *
- * Precision: routed-expert weights enter the tensor cores exactly (each
- * E2M1 code is re-placed as the E4M3 value 2^-6 * E2M1, the E8M0 scale
- * multiplies each 32-weight block sum in fp32).  Activations enter as sums of
- * E4M3 pieces after a per-token power-of-two prescale: x as two pieces (exact
- * for every bf16 element down to 2^-17 of the token's largest |x|, below that
- * off by at most 2^-18 of it), the SwiGLU activations h as four pieces (about
- * 16 significant bits); the bf16 shared expert's h as bf16 hi + lo.  All sums
- * are fp32.  Router logits are fp32 sums of exact fp32 x bf16 products.
+ * Precision: routed-expert weights enter the tensor cores exactly, as their
+ * own E2M1 codes and E8M0 scales (block-scaled MMA, E2M1 x E2M1).  The
+ * activations they multiply (x, and w_j * h for the down projections, the
+ * routing weight folded in) enter as sums of 6 E2M1 pieces, each 32-element
+ * block of each piece with its own E8M0 scale taken from what the earlier
+ * pieces left over; the pieces reproduce each activation to about 2^-19 of
+ * the largest element of its 32-element block.  The bf16 shared expert runs
+ * on bf16 tensor-core MMAs with x exact and its h as bf16 hi + lo.  All
+ * accumulation is fp32 (the routed down projections and the shared one sum
+ * into one fp32 accumulator per output).  Router logits are fp32 sums of
+ * exact fp32 x bf16 products.
  *
  * Ownership and ordering: the caller owns every buffer and the stream.  Calls
  * allocate nothing, never synchronise, and are ordered on `stream`; results
@@ -177,8 +180,9 @@ k3moe_status k3moe_layer_from_host(const void *x_host, int32_t T, const float *w
  * i.e. one pass of the kernels): `events` are n_events cudaEvent_t handles
  * created by the caller; events[0] is recorded on `stream` before the first
  * kernel and events[i] after the i-th kernel, for i up to the number of
- * kernels the call launches, which is written to *n_kernels (4: router and
- * shared gate/up with top-k, routed gate/up, down projections, combine).
+ * kernels the call launches, which is written to *n_kernels (3: router with
+ * softmax, top-k and dispatch; gate/up of the routed and shared experts;
+ * down projections with the weighted combine).
  * The computation and its result are those of k3moe_layer.
  */
 k3moe_status k3moe_layer_timed(const void *x, int32_t T, const float *w_router, const float *bias,

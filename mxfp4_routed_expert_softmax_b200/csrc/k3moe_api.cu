@@ -44,8 +44,6 @@ cudaError_t set_smem(Kern kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-#define K3_DN_LIST(X) X(2, 1) X(2, 3) X(2, 6) X(4, 1) X(4, 3) X(4, 6) X(12, 1) X(12, 3) \
-    X(12, 6) X(24, 1) X(24, 3) X(24, 6)
 
 // One-time per-device set-up: SM count and the shared-memory opt-ins.
 k3moe_status device_info(DeviceInfo **out) {
@@ -59,12 +57,9 @@ k3moe_status device_info(DeviceInfo **out) {
         e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return cuda_fail(e);
         const int big = kSmemLimit;
-        cudaError_t r = set_smem(route_shared_kernel, kRouteTok * 8192 * 4);
+        cudaError_t r = set_smem(route_kernel, kRouteTok * 8192 * 4);
         if (r == cudaSuccess) r = set_smem(umma_expert_kernel<true>, big);
         if (r == cudaSuccess) r = set_smem(umma_expert_kernel<false>, big);
-#define K3_SET_DN(a, b) if (r == cudaSuccess) r = set_smem(expert_down_kernel<a, b>, big);
-        K3_DN_LIST(K3_SET_DN)
-#undef K3_SET_DN
         if (r != cudaSuccess) return cuda_fail(r);
         di.ready = true;
     }
@@ -85,11 +80,6 @@ int umma_stages(bool gu) {
     const int cap = 8;
     return n < cap ? n : cap;
 }
-int dn_stages(int ff, int ffs) {
-    for (int n = kMaxStages; n >= 2; --n)
-        if (dn_smem_bytes(ff, ffs, n) <= kSmemLimit) return n;
-    return 0;
-}
 
 k3moe_status check_dims(const k3moe_dims *dm) {
     if (!dm) return K3MOE_ERR_INVALID_ARGUMENT;
@@ -101,7 +91,6 @@ k3moe_status check_dims(const k3moe_dims *dm) {
         return K3MOE_ERR_INVALID_ARGUMENT;
     if (dm->ff_shared < 0 || dm->ff_shared > 3072 || dm->ff_shared % 64)
         return K3MOE_ERR_UNSUPPORTED_SHAPE;
-    if (dn_stages(dm->ff, dm->ff_shared) == 0) return K3MOE_ERR_UNSUPPORTED_SHAPE;
     return K3MOE_OK;
 }
 
@@ -189,6 +178,43 @@ k3moe_status tmap_templates(int d, int ff, void *placeholder, uint4 (&out)[2][8]
     return K3MOE_OK;
 }
 
+// Tensor maps of the bf16 shared expert at its real addresses (u8 elements,
+// 128 x 128-byte boxes, 128-byte swizzle): W_g, W_u (ff_s rows of 2d bytes),
+// W_d (d rows of 2 ff_s bytes).
+k3moe_status shared_tmaps(int d, int ffs, const void *wg, const void *wu, const void *wd, uint4 (&out)[3][8]) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (q != cudaDriverEntryPointSuccess || !fn) {
+            g_last_error = "cuTensorMapEncodeTiled is not available";
+            return K3MOE_ERR_CUDA;
+        }
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const void *addr[3] = {wg, wu, wd};
+    CUtensorMap m[3];
+    for (int i = 0; i < 3; ++i) {
+        const cuuint64_t cols = (cuuint64_t)(i < 2 ? d : ffs) * 2, rows = (cuuint64_t)(i < 2 ? ffs : d);
+        const cuuint64_t dims[2] = {cols, rows};
+        const cuuint64_t strides[1] = {cols};
+        const cuuint32_t box[2] = {128, (cuuint32_t)kTileM};
+        const cuuint32_t es[2] = {1, 1};
+        CUresult r = encode(&m[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(addr[i]), dims, strides, box,
+                            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            g_last_error = "cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")";
+            return K3MOE_ERR_CUDA;
+        }
+    }
+    memcpy(out, m, sizeof(out));
+    return K3MOE_OK;
+}
+
 template <bool GU>
 cudaError_t launch_umma(const DeviceInfo &di, UmmaParams up, cudaStream_t st) {
     up.nst = umma_stages(GU);
@@ -197,31 +223,15 @@ cudaError_t launch_umma(const DeviceInfo &di, UmmaParams up, cudaStream_t st) {
     return launch(umma_expert_kernel<GU>, dim3(g), dim3(kUThreads), smem, st, true, up);
 }
 
-cudaError_t launch_down(const DeviceInfo &di, DownParams dp, cudaStream_t st) {
-    dp.skip_routed = 1;
-    const int nq = (dp.ff / 32 + 3) / 4;
-    (void)nq;
-    const int nbq = 2;  // routed rows are skipped: the smallest variant
-    const int ns = (dp.ffs / 32 + 15) / 16;
-    const int nbs = ns <= 1 ? 1 : ns <= 3 ? 3 : 6;
-    dp.nst = dn_stages(dp.ff, dp.ffs);
-    const int smem = dn_smem_bytes(dp.ff, dp.ffs, dp.nst);
-    const dim3 grid(di.sms), block(kDownThreads);
-#define K3_LAUNCH_DN(a, b) \
-    if (nbq == a && nbs == b) return launch(expert_down_kernel<a, b>, grid, block, smem, st, true, dp);
-    K3_DN_LIST(K3_LAUNCH_DN)
-#undef K3_LAUNCH_DN
-    return cudaErrorInvalidValue;
-}
 
-// Router (+ shared gate/up + top-k + dispatch) for one chunk.  Cooperative
+// Router (+ top-k + dispatch + activation pieces) for one chunk.  Cooperative
 // launch: CTA 0 waits on the other CTAs' router rows, so all must be resident.
 cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st) {
     const int nt = rp.Tc < kRouteTok ? rp.Tc : kRouteTok;
     const int smem = nt * rp.d * 4;
     if (di.route_smem != smem) {
         int occ = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, route_shared_kernel,
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, route_kernel,
                                                                        kRouteThreads, smem);
         if (e != cudaSuccess) return e;
         di.route_occ = occ;
@@ -230,10 +240,9 @@ cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st) {
     const int per_sm = di.route_occ < 3 ? di.route_occ : 3;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     int gs = per_sm * di.sms - 1;  // streaming CTAs
-    // every streaming warp takes at least a quarter row of the smaller phase,
-    // so a row is split between at most 5 warps (kMaxSeg slots)
-    const int rows_min = rp.ffs > 0 && rp.ffs < rp.E ? rp.ffs : rp.E;
-    const int wmax = rows_min * 4;
+    // every streaming warp takes at least a quarter row, so a row is split
+    // between at most 5 warps (kMaxSeg slots)
+    const int wmax = rp.E * 4;
     if (gs * 8 > wmax) gs = wmax / 8 > 0 ? wmax / 8 : 1;
     rp.nwarps = gs * 8;
     cudaLaunchConfig_t cfg = {};
@@ -246,7 +255,7 @@ cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, route_shared_kernel, rp);
+    return cudaLaunchKernelEx(&cfg, route_kernel, rp);
 }
 
 struct EventHook {
@@ -301,6 +310,12 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
     uint4 tmpl[2][8];
     s = tmap_templates(d, dims->ff, ws, tmpl);
     if (s != K3MOE_OK) return s;
+    uint4 smap[3][8];
+    memset(smap, 0, sizeof(smap));
+    if (ffs > 0) {
+        s = shared_tmaps(d, ffs, shared_wg, shared_wu, shared_wd, smap);
+        if (s != K3MOE_OK) return s;
+    }
 
     for (int c0 = 0; c0 < T; c0 += kChunk) {
         const int Tc = (T - c0) < kChunk ? (T - c0) : kChunk;
@@ -322,9 +337,6 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         rp.Tc = Tc;
         rp.wr = w_router;
         rp.bias = bias;
-        rp.swg = reinterpret_cast<const uint16_t *>(shared_wg);
-        rp.swu = reinterpret_cast<const uint16_t *>(shared_wu);
-        rp.ffs = ffs;
         rp.d = d;
         rp.E = dims->n_experts;
         rp.k = dims->top_k;
@@ -334,6 +346,8 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         rp.idx_out = idx_out ? idx_out + (size_t)c0 * dims->top_k : nullptr;
         rp.w_out = w_out ? w_out + (size_t)c0 * dims->top_k : nullptr;
         memcpy(rp.tmpl, tmpl, sizeof(tmpl));
+        memcpy(rp.smap, smap, sizeof(smap));
+        rp.has_shared = ffs > 0;
         EventHook none;
         EventHook &hk = hook ? *hook : none;
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
@@ -346,21 +360,14 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         up.d = d;
         up.ff = dims->ff;
         up.k = dims->top_k;
+        up.ffs = ffs;
         up.ws = wsb;
         up.L = L;
-        up.has_shared = ffs > 0;
         up.out_fp32 = out32;
         up.y = yc;
         e = launch_umma<true>(*di, up, st);
         if (e != cudaSuccess) return cuda_fail(e, "gate/up launch");
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
-
-        if (ffs > 0) {
-            DownParams dp{Tc, d, dims->ff, ffs, reinterpret_cast<const uint16_t *>(shared_wd), wsb, L};
-            e = launch_down(*di, dp, st);
-            if (e != cudaSuccess) return cuda_fail(e, "shared down launch");
-            if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
-        }
 
         e = launch_umma<false>(*di, up, st);
         if (e != cudaSuccess) return cuda_fail(e, "down launch");
@@ -418,7 +425,6 @@ k3moe_status k3moe_route(const void *x, int32_t T, const float *w_router, const 
         rp.Tc = Tc;
         rp.wr = w_router;
         rp.bias = bias;
-        rp.ffs = 0;
         rp.d = dims->d;
         rp.E = dims->n_experts;
         rp.k = dims->top_k;
@@ -474,9 +480,9 @@ k3moe_status k3moe_expert_ffn(const void *x, int32_t T, const uint8_t *blob,
         up.d = d;
         up.ff = dims->ff;
         up.k = 1;
+        up.ffs = 0;
         up.ws = wsb;
         up.L = L;
-        up.has_shared = 0;
         up.out_fp32 = out32;
         up.y = yc;
         e = launch_umma<true>(*di, up, st);
@@ -521,7 +527,7 @@ k3moe_status k3moe_layer_timed(const void *x, int32_t T, const float *w_router, 
     k3moe_status s = layer_impl(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu,
                                 shared_wd, dims, y, nullptr, nullptr, ws, ws_bytes, stream, nullptr,
                                 nullptr, &hk);
-    *n_kernels = shared_ff(dims) > 0 ? 4 : 3;
+    *n_kernels = 3;
     return s;
 }
 

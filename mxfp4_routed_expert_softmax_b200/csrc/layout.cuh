@@ -14,10 +14,12 @@ constexpr int kMaxSeg = 8;  // most warps that share one router/shared row
 constexpr int kPieces = 6;
 constexpr int kNMax = kChunk * kPieces;  // 48: widest MMA N of a chunk
 constexpr int kSfRow = 64;               // scale words per (K-tile, group): rows n < 64
-constexpr int kTileK = 256;              // weights per K-tile (128 bytes of nibbles per row)
+constexpr int kTileK = 256;              // MXFP4 weights per K-tile (128 bytes of nibbles per row)
+constexpr int kTileKs = 64;              // bf16 weights per K-tile (128 bytes per row)
 constexpr int kTileM = 128;              // MMA M: weight rows per item
 constexpr int kMaxCtas = 256;            // grid cap of the tensor-core kernels
-__host__ __device__ inline int act_n(int Tc) { return (Tc * kPieces + 7) & ~7; }
+// MMA N of a chunk: a multiple of 16 (kind::f16 with M = 128 needs it)
+__host__ __device__ inline int act_n(int Tc) { return (Tc * kPieces + 15) & ~15; }
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -27,24 +29,21 @@ struct Layout {
     size_t logits;     // f32 [kChunk][E]
     size_t idx;        // i32 [kChunk][k]
     size_t wt;         // f32 [kChunk][k]
-    size_t sigx;       // i32 [kChunk]      E4M3 prescale exponent of each token's x
-    size_t xp;         // u8  [kChunk][2][d] x * 2^sigx as two E4M3 pieces (even/odd-permuted)
     size_t uniq_blob;  // u64 [kChunk*k]    blob pointer of each distinct selected expert
     size_t uniq_mask;  // u32 [kChunk*k]    tokens (bit t) that selected it
     size_t uniq_slot;  // i8  [kChunk*k][kChunk] slot j of token t for it, -1 if none
-    size_t hmax;       // u32 [kChunk][k]   max |h| of each (token, slot), as float bits
-    size_t h;          // f32 [kChunk][k][ff] SwiGLU activations of each (token, slot)
-    size_t hs;         // f32 [kChunk][ff_s] shared-expert activations
-    size_t ob;         // f32 [kChunk][k+1][d] expert outputs: [0] shared, [1+j] slot j
-    size_t part;       // f32 [2][E+ffs][kMaxSeg][4][2] partial sums of rows split between warps
-    size_t cnt;        // u32 [2][E+ffs] arrivals per split row (back to 0 after each row)
-    size_t tmap;       // 128-byte tensor maps [umax][3]: W_g, W_u, W_d nibble planes
+    size_t part;       // f32 [2][E][kMaxSeg][4] partial sums of router rows split between warps
+    size_t cnt;        // u32 [2][E] arrivals per split row (back to 0 after each row)
+    size_t tmap;       // 128-byte tensor maps [umax][3]: W_g, W_u, W_d nibble planes; then
+                       // the shared expert's W_g, W_u, W_d (bf16) at [umax*3 ..]
     size_t xb;         // u8  [nkt_d][N*128] E2M1 pieces of x (gate/up B operand)
     size_t xsf;        // u32 [nkt_d][2][kSfRow] their E8M0 scales (byte = block in group)
     size_t hb;         // u8  [umax][nkt_ff][N*128] pieces of w*h (down B operand)
     size_t hsf;        // u32 [umax][nkt_ff][2][kSfRow]
+    size_t xbf;        // u8  [ceil(d/64)][N*128] x as bf16 (rows t*kPieces), shared gate/up B
+    size_t hsb;        // u8  [ceil(ffs/64)][N*128] shared h as bf16 hi, lo (rows t*kPieces, +1)
     size_t spart;      // f32 [kMaxCtas][2][2][kChunk][kTileM] split-item partial sums
-    size_t icnt;       // u32 [umax*nrb_ff + nrb_d] arrivals per split item (back to 0)
+    size_t icnt;       // u32 [umax*nrb_ff + nrb_ffs + nrb_d] arrivals per split item (back to 0)
     size_t total;
     int d, ff, E, k, ffs, umax;
 };
@@ -66,33 +65,21 @@ __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int f
     o = align256(o + C * k * 4);
     L.wt = o;
     o = align256(o + C * k * 4);
-    L.sigx = o;
-    o = align256(o + C * 4);
-    L.xp = o;
-    o = align256(o + C * 2 * (size_t)d);
     L.uniq_blob = o;
     o = align256(o + C * k * 8);
     L.uniq_mask = o;
     o = align256(o + C * k * 4);
     L.uniq_slot = o;
     o = align256(o + C * k * C);
-    L.hmax = o;
-    o = align256(o + C * k * 4);
-    L.h = o;
-    o = align256(o + C * k * (size_t)ff * 4);
-    L.hs = o;
-    o = align256(o + C * (size_t)(ffs > 0 ? ffs : 1) * 4);
-    L.ob = o;
-    o = align256(o + C * (k + 1) * (size_t)d * 4);
     L.part = o;
-    o = align256(o + (size_t)2 * (E + ffs) * kMaxSeg * 4 * 2 * 4);
+    o = align256(o + (size_t)2 * E * kMaxSeg * 4 * 4);
     L.cnt = o;
-    o = align256(o + (size_t)2 * (E + ffs) * 4);
+    o = align256(o + (size_t)2 * E * 4);
     const int umax = E < kChunk * k ? E : kChunk * k;
     const int nkt_d = ceil_div(d, kTileK), nkt_ff = ceil_div(ff, kTileK);
     L.umax = umax;
     L.tmap = o;
-    o = align256(o + (size_t)umax * 3 * 128);
+    o = align256(o + ((size_t)umax * 3 + 3) * 128);
     L.xb = o;
     o = align256(o + (size_t)nkt_d * kNMax * 128);
     L.xsf = o;
@@ -101,10 +88,14 @@ __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int f
     o = align256(o + (size_t)umax * nkt_ff * kNMax * 128);
     L.hsf = o;
     o = align256(o + (size_t)umax * nkt_ff * 2 * kSfRow * 4);
+    L.xbf = o;
+    o = align256(o + (size_t)ceil_div(d, kTileKs) * kNMax * 128);
+    L.hsb = o;
+    o = align256(o + (size_t)(ffs > 0 ? ceil_div(ffs, kTileKs) : 1) * kNMax * 128);
     L.spart = o;
     o = align256(o + (size_t)kMaxCtas * 2 * 2 * kChunk * kTileM * 4);
     L.icnt = o;
-    o = align256(o + ((size_t)umax * ceil_div(ff, kTileM) + ceil_div(d, kTileM)) * 4);
+    o = align256(o + ((size_t)umax * ceil_div(ff, kTileM) + ceil_div(ffs, kTileM) + ceil_div(d, kTileM)) * 4);
     L.total = o;
     return L;
 }

@@ -37,6 +37,12 @@ __device__ __forceinline__ uint32_t idesc_sf_id(uint32_t idesc, uint32_t sf_id) 
     return idesc | (sf_id << 29) | (sf_id << 4);
 }
 
+// Instruction descriptor of kind::f16 with bf16 A and B (both K-major), f32
+// accumulate, M = 128, N (multiple of 16, <= 256).
+__host__ __device__ constexpr uint32_t idesc_bf16(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
+}
+
 // ------------------------------------------------------------ TMEM --
 // Warp-wide: allocate ncols columns (power of two >= 32); the base address
 // is written to *slot (shared memory).
@@ -63,6 +69,16 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d, uint64_t adesc, uint64_t bd
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
         " tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(d),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 operands (no output lane disabled).
+__device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n}\n" ::"r"(d), "l"(adesc),
+        "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u)
         : "memory");
 }
 

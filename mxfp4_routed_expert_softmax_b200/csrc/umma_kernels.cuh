@@ -78,18 +78,43 @@ __device__ __forceinline__ void quantize_pieces(float v, int lane, int t, int c,
     }
 }
 
-// x of the chunk -> pieces (gate/up B operand), blocks spread over every warp
-// of the grid (warp index gw of nw).
-__device__ void build_x_pieces(const uint16_t *x, int Tc, int d, uint8_t *ws, const Layout &L, int gw,
-                               int nw) {
+// x of the chunk -> pieces (routed gate/up B operand) and, with a shared
+// expert, x as bf16 in rows t*kPieces of the shared gate/up B operand (the
+// other piece rows zero).  Blocks spread over every warp of the grid (warp
+// index gw of nw).
+__device__ void build_x_pieces(const uint16_t *x, int Tc, int d, uint8_t *ws, const Layout &L, int gw, int nw,
+                               bool shared) {
     const int lane = threadIdx.x & 31, N = act_n(Tc), nb = d / 32;
     for (int i = gw; i < Tc * nb; i += nw) {
         const int t = i / nb, b = i - t * nb;
-        const float v = __uint_as_float((uint32_t)x[(size_t)t * d + 32 * b + lane] << 16);
+        const int col = 32 * b + lane;
+        const uint16_t xv = x[(size_t)t * d + col];
+        const float v = __uint_as_float((uint32_t)xv << 16);
         const int kt = b >> 3;
         quantize_pieces(v, lane, t, b & 7, N, ws + L.xb + (size_t)kt * N * 128,
                         ws + L.xsf + (size_t)kt * 2 * kSfRow * 4);
+        if (shared) {
+            uint8_t *tile = ws + L.xbf + (size_t)(col / kTileKs) * N * 128;
+            const int c = (col % kTileKs) / 8, e = col % 8;
+#pragma unroll
+            for (int pc = 0; pc < kPieces; ++pc) {
+                const int n = t * kPieces + pc;
+                *reinterpret_cast<uint16_t *>(tile + (c * (N / 8) + n / 8) * 128 + (n % 8) * 16 + e * 2) =
+                    pc == 0 ? xv : (uint16_t)0;
+            }
+        }
     }
+}
+
+// The shared expert's three tensor maps (encoded by the host with their real
+// addresses) into the workspace, where the tensor-core kernels read them.
+__device__ void write_shared_tmaps(uint8_t *ws, const Layout &L, const uint4 (&smap)[3][8]) {
+    uint4 *o = reinterpret_cast<uint4 *>(ws + L.tmap + (size_t)L.umax * 3 * 128);
+#pragma unroll
+    for (int m = 0; m < 3; ++m)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[m * 8 + j] = smap[m][j];
+    umma::tmap_release();
 }
 
 // Tensor maps of distinct expert u: copies of the host-encoded templates
@@ -113,11 +138,11 @@ __device__ void write_expert_tmaps(uint8_t *ws, const Layout &L, int u, const ui
 // ---------------------------------------------------------------- kernel --
 struct UmmaParams {
     int Tc, d, ff, k;
+    int ffs;          // shared expert rows (0: none)
     uint8_t *ws;
     Layout L;
     int nst;          // pipeline stages
     // down only
-    int has_shared;   // add the shared expert's output (ob slot 0)
     int out_fp32;     // y in fp32 (else bf16, rounded once)
     void *y;          // [Tc][d] of this chunk
 };
@@ -143,6 +168,13 @@ __device__ __forceinline__ uint2 load_sf8(const uint8_t *p, int nks) {
     return make_uint2(w0, w1);
 }
 
+// GU: routed items (distinct expert u, 128 rows of ff; K = d in 256-weight
+// tiles) then the shared expert's items (128 rows of ff_s; K = d in 64-weight
+// bf16 tiles).  Down: one item per 128 rows of d whose K runs over every
+// distinct routed expert's ff (256-weight tiles) and then the shared
+// expert's ff_s (64-weight bf16 tiles), all into one accumulator, so the
+// routing weights (folded into the routed pieces) and the shared expert are
+// combined by the tensor core itself.
 template <bool GU>
 __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -184,13 +216,16 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
 
     const int Tc = p.Tc, N = act_n(Tc);
     const int U = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_unique);
-    const int K = GU ? p.d : p.ff;   // reduction length
-    const int M = GU ? p.ff : p.d;   // weight rows
+    const int K = GU ? p.d : p.ff;   // routed reduction length
+    const int M = GU ? p.ff : p.d;   // routed weight rows
+    const int Ks = GU ? p.d : p.ffs; // shared reduction length
     const int nkt = ceil_div(K, kTileK);
     const int nrb = ceil_div(M, kTileM);
-    const int upi = GU ? nkt : U * nkt;  // units (K-tiles) per item
-    const int n_items = GU ? U * nrb : nrb;
-    const int total = n_items * upi;
+    const int nkts = p.ffs > 0 ? ceil_div(Ks, kTileKs) : 0;
+    const int nrbs = (GU && p.ffs > 0) ? ceil_div(p.ffs, kTileM) : 0;
+    const int R = GU ? U * nrb * nkt : 0;             // routed units (GU)
+    const int upi = GU ? 0 : U * nkt + nkts;          // units per item (down)
+    const int total = GU ? R + nrbs * nkts : nrb * upi;
     const int G = min((int)gridDim.x, max(total, 1));
     const int cta = blockIdx.x;
     auto start = [&](int c) { return (int)(((long long)c * total) / G); };
@@ -198,7 +233,8 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     const int a = cta < G ? start(cta) : 0, b = cta < G ? start(cta + 1) : 0;
     const size_t mat = (size_t)p.d * p.ff;
     const uint8_t *const *ublob = reinterpret_cast<const uint8_t *const *>(p.ws + L.uniq_blob);
-    const uint32_t idesc = umma::idesc_mxf4(N);
+    const uint8_t *smaps = p.ws + L.tmap + (size_t)L.umax * 3 * 128;
+    const uint32_t idesc4 = umma::idesc_mxf4(N), idesc16 = umma::idesc_bf16(N);
     // TMEM columns: accumulators [buf][mat] at (buf*NMAT + mat)*64 (N <= 64), then
     // the scale columns of each stage from sf0
     const uint32_t sf0 = GU ? 256u : 128u;
@@ -213,54 +249,80 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     };
 
     struct Unit {
-        int item, u, rb, kt;
+        int item, u, rb, kt, istart, iend;
+        bool shared;
     };
     auto decode = [&](int unit) {
         Unit x;
-        x.item = unit / upi;
-        const int r = unit - x.item * upi;
-        if (GU) {
-            x.u = x.item / nrb;
-            x.rb = x.item - x.u * nrb;
-            x.kt = r;
+        if constexpr (GU) {
+            if (unit < R) {
+                x.item = unit / nkt;
+                x.istart = x.item * nkt;
+                x.iend = x.istart + nkt;
+                x.u = x.item / nrb;
+                x.rb = x.item - x.u * nrb;
+                x.shared = false;
+            } else {
+                const int j = (unit - R) / nkts;
+                x.item = U * nrb + j;
+                x.istart = R + j * nkts;
+                x.iend = x.istart + nkts;
+                x.u = -1;
+                x.rb = j;
+                x.shared = true;
+            }
+            x.kt = unit - x.istart;
         } else {
-            x.u = r / nkt;
-            x.kt = r - x.u * nkt;
+            x.item = unit / upi;
+            x.istart = x.item * upi;
+            x.iend = x.istart + upi;
             x.rb = x.item;
+            const int r = unit - x.istart;
+            x.shared = r >= U * nkt;
+            if (!x.shared) {
+                x.u = r / nkt;
+                x.kt = r - x.u * nkt;
+            } else {
+                x.u = -1;
+                x.kt = r - U * nkt;
+            }
         }
         return x;
+    };
+    // MMA k-steps of a unit (32 bytes of every row each)
+    auto ksteps = [&](const Unit &x) {
+        return x.shared ? min(4, (Ks - x.kt * kTileKs) / 16) : min(4, (K - x.kt * kTileK) / 64);
     };
 
     if (warp == 8) {
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
-            int last_u = -1;
+            int last_u = -2;
             for (int unit = a, it = 0; unit < b && !*s_abort; ++unit, ++it) {
                 const Unit x = decode(unit);
                 const int s = it % nst;
                 if (it >= nst && !wait(&empty[s], (uint32_t)(((it / nst) + 1) & 1))) break;
                 uint8_t *st = smem + s * SB;
-                const uint8_t *blob = ublob[x.u];
-                const uint8_t *bsrc = GU ? p.ws + L.xb + (size_t)x.kt * N * 128
-                                         : p.ws + L.hb + ((size_t)x.u * nkt + x.kt) * N * 128;
-                if (blob != nullptr) {
-                    const uint8_t *maps = p.ws + L.tmap + (size_t)x.u * 3 * 128;
+                const uint8_t *blob = x.shared ? nullptr : ublob[x.u];
+                const uint8_t *maps = nullptr;
+                const uint8_t *bsrc;
+                if (x.shared) {
+                    maps = smaps + (GU ? 0 : 256);
+                    bsrc = (GU ? p.ws + L.xbf : p.ws + L.hsb) + (size_t)x.kt * N * 128;
+                } else {
+                    maps = p.ws + L.tmap + (size_t)x.u * 3 * 128 + (GU ? 0 : 256);
+                    bsrc = GU ? p.ws + L.xb + (size_t)x.kt * N * 128
+                              : p.ws + L.hb + ((size_t)x.u * nkt + x.kt) * N * 128;
+                }
+                if (x.shared || blob != nullptr) {
                     if (x.u != last_u) {
-                        if (GU) {
-                            umma::tmap_acquire(maps);
-                            umma::tmap_acquire(maps + 128);
-                        } else {
-                            umma::tmap_acquire(maps + 256);
-                        }
+                        umma::tmap_acquire(maps);
+                        if (GU) umma::tmap_acquire(maps + 128);
                         last_u = x.u;
                     }
                     mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * kAtile + N * 128));
-                    if (GU) {
-                        umma::tma_load_2d(st, maps, x.kt * 128, x.rb * kTileM, &full[s]);
-                        umma::tma_load_2d(st + kAtile, maps + 128, x.kt * 128, x.rb * kTileM, &full[s]);
-                    } else {
-                        umma::tma_load_2d(st, maps + 256, x.kt * 128, x.rb * kTileM, &full[s]);
-                    }
+                    umma::tma_load_2d(st, maps, x.kt * 128, x.rb * kTileM, &full[s]);
+                    if (GU) umma::tma_load_2d(st + kAtile, maps + 128, x.kt * 128, x.rb * kTileM, &full[s]);
                 } else {
                     mbar_arrive_expect_tx(&full[s], (uint32_t)(N * 128));
                 }
@@ -269,54 +331,86 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         }
     } else if (warp >= 4 && warp < 8) {
         // --------------------------------------- scale factors -> TMEM --
+        // The global loads of a unit's scales are issued kLook units ahead of
+        // its TMEM stores (a ring of registers), so their latency overlaps the
+        // pipeline instead of adding to every stage.  Shared (bf16) units have
+        // no scales: the warps only keep the stage protocol.
+        constexpr int kLook = 3;
+        struct SfRegs {
+            uint32_t a[NMAT][8];  // column 8m + 4g + j: group g, row block j
+            uint32_t b[4];        // B scales: (g0, rows 0-31), (g0, 32-63), (g1, ...), (g1, ...)
+            bool on;
+        };
         const uint32_t lb = umma::lane_base(warp);
-        for (int unit = a, it = 0; unit < b; ++unit, ++it) {
+        auto load = [&](int unit, SfRegs &r) {
             const Unit x = decode(unit);
-            const int s = it % nst;
-            // lane 0 decides, the warp follows (the TMEM stores are warp-collective)
-            int go = 0;
-            if (lane == 0) go = it < nst ? !*s_abort : wait(&empty[s], (uint32_t)(((it / nst) + 1) & 1));
-            if (!__shfl_sync(0xffffffffu, go, 0)) break;
+            r.on = !x.shared;
+            if (x.shared) return;
             const uint8_t *blob = ublob[x.u];
-            const int nks = min(4, (K - x.kt * kTileK) / 64);
-            const uint32_t col = tbase + lb + sf0 + (uint32_t)(s * SFC);
+            const int nks = ksteps(x);
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
                 const uint8_t *plane = nullptr;
                 if (blob != nullptr)
                     plane = GU ? (m == 0 ? blob + mat / 2 : blob + mat + mat / 32) : blob + mat + mat / 16 + mat / 2;
-                uint32_t w[8];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int row = x.rb * kTileM + 32 * j + lane;
                     uint2 v = make_uint2(0u, 0u);
                     if (plane != nullptr && row < M) v = load_sf8(plane + (size_t)row * (K / 32) + x.kt * 8, nks);
-                    w[j] = v.x;      // group 0: k-steps 0, 1
-                    w[4 + j] = v.y;  // group 1: k-steps 2, 3
+                    r.a[m][j] = v.x;      // group 0: k-steps 0, 1
+                    r.a[m][4 + j] = v.y;  // group 1: k-steps 2, 3
                 }
-                umma::st8(col + 8 * m, w);
             }
             const uint32_t *sfb = GU ? reinterpret_cast<const uint32_t *>(p.ws + L.xsf) + (size_t)x.kt * 2 * kSfRow
                                      : reinterpret_cast<const uint32_t *>(p.ws + L.hsf) +
                                            ((size_t)x.u * nkt + x.kt) * 2 * kSfRow;
-            {
-                // group g, row block j (rows 32j..) at column 8*NMAT + 4g + j
-                uint32_t w[8] = {__ldcg(sfb + lane), __ldcg(sfb + 32 + lane), 0u, 0u,
-                                 __ldcg(sfb + kSfRow + lane), __ldcg(sfb + kSfRow + 32 + lane), 0u, 0u};
+            r.b[0] = __ldcg(sfb + lane);
+            r.b[1] = __ldcg(sfb + 32 + lane);
+            r.b[2] = __ldcg(sfb + kSfRow + lane);
+            r.b[3] = __ldcg(sfb + kSfRow + 32 + lane);
+        };
+        auto store = [&](int it, const SfRegs &r) {
+            const int s = it % nst;
+            // lane 0 decides, the warp follows (the TMEM stores are warp-collective)
+            int go = 0;
+            if (lane == 0) go = it < nst ? !*s_abort : wait(&empty[s], (uint32_t)(((it / nst) + 1) & 1));
+            if (!__shfl_sync(0xffffffffu, go, 0)) return false;
+            if (r.on) {
+                const uint32_t col = tbase + lb + sf0 + (uint32_t)(s * SFC);
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m) umma::st8(col + 8 * m, r.a[m]);
+                const uint32_t w[8] = {r.b[0], r.b[1], 0u, 0u, r.b[2], r.b[3], 0u, 0u};
                 umma::st8(col + 8 * NMAT, w);
+                umma::wait_st();
             }
-            umma::wait_st();
             umma::fence_before();
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&full[s])) : "memory");
+            return true;
+        };
+        SfRegs R4[kLook + 1];
+        const int n = b - a;
+#pragma unroll
+        for (int i = 0; i < kLook; ++i)
+            if (i < n) load(a + i, R4[i]);
+        bool go = true;
+        for (int it0 = 0; it0 < n && go; it0 += kLook + 1) {
+#pragma unroll
+            for (int q = 0; q <= kLook; ++q) {
+                const int it = it0 + q;
+                if (it < n && go) {
+                    if (it + kLook < n) load(a + it + kLook, R4[(q + kLook) % (kLook + 1)]);
+                    go = store(it, R4[q]);
+                }
+            }
         }
     } else if (warp == 9) {
         // ------------------------------------------------- MMA issuer --
         if (lane == 0) {
             int it = 0, seg = 0;
             for (int unit = a; unit < b && !*s_abort; ++seg) {
-                const int item = unit / upi;
-                const int seg_end = min(b, (item + 1) * upi);
+                const int seg_end = min(b, decode(unit).iend);
                 const int buf = seg & 1;
                 if (seg >= 2 && !wait(&aempty[buf], (uint32_t)(((seg >> 1) + 1) & 1))) break;
                 umma::fence_after();
@@ -328,21 +422,30 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     umma::fence_after();
                     const uint32_t st = smem_u32(smem + s * SB);
                     const uint32_t sfc = tbase + sf0 + (uint32_t)(s * SFC);
-                    const int nks = min(4, (K - x.kt * kTileK) / 64);
+                    const int nks = ksteps(x);
                     for (int sk = 0; sk < nks; ++sk) {
-                        const uint32_t grp = (uint32_t)(sk >> 1), sfid = (uint32_t)(2 * (sk & 1));
-                        const uint32_t id = umma::idesc_sf_id(idesc, sfid);
                         const uint64_t bdesc =
                             umma::smem_desc(st + NMAT * kAtile + (uint32_t)(2 * sk * (N / 8) * 128),
                                             (uint32_t)((N / 8) * 128), 128u, umma::kLayoutNone);
-                        const uint32_t sfb = (sfc + 8 * NMAT + grp * 4) | (sfid << 30);
                         const uint32_t acc = (un != unit || sk != 0) ? 1u : 0u;
+                        if (x.shared) {
 #pragma unroll
-                        for (int m = 0; m < NMAT; ++m) {
-                            const uint64_t adesc = umma::smem_desc(st + (uint32_t)(m * kAtile + 32 * sk), 16u, 1024u,
-                                                                   umma::kLayoutSw128);
-                            const uint32_t sfa = (sfc + 8 * m + grp * 4) | (sfid << 30);
-                            umma::mma_mxf4(dcol + (uint32_t)(m * 64), adesc, bdesc, id, acc, sfa, sfb);
+                            for (int m = 0; m < NMAT; ++m) {
+                                const uint64_t adesc = umma::smem_desc(st + (uint32_t)(m * kAtile + 32 * sk), 16u,
+                                                                       1024u, umma::kLayoutSw128);
+                                umma::mma_bf16(dcol + (uint32_t)(m * 64), adesc, bdesc, idesc16, acc);
+                            }
+                        } else {
+                            const uint32_t grp = (uint32_t)(sk >> 1), sfid = (uint32_t)(2 * (sk & 1));
+                            const uint32_t id = umma::idesc_sf_id(idesc4, sfid);
+                            const uint32_t sfb = (sfc + 8 * NMAT + grp * 4) | (sfid << 30);
+#pragma unroll
+                            for (int m = 0; m < NMAT; ++m) {
+                                const uint64_t adesc = umma::smem_desc(st + (uint32_t)(m * kAtile + 32 * sk), 16u,
+                                                                       1024u, umma::kLayoutSw128);
+                                const uint32_t sfa = (sfc + 8 * m + grp * 4) | (sfid << 30);
+                                umma::mma_mxf4(dcol + (uint32_t)(m * 64), adesc, bdesc, id, acc, sfa, sfb);
+                            }
                         }
                     }
                     umma::commit(&empty[s]);
@@ -355,12 +458,14 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         // --------------------------------------------------- epilogue --
         const uint32_t lb = umma::lane_base(warp);
         const int rowl = 32 * warp + lane;  // row of the 128-row item
-        float* spart = reinterpret_cast<float *>(p.ws + L.spart);
-        uint32_t *icnt = reinterpret_cast<uint32_t *>(p.ws + L.icnt) + (GU ? 0 : L.umax * ceil_div(p.ff, kTileM));
+        float *spart = reinterpret_cast<float *>(p.ws + L.spart);
+        uint32_t *icnt = reinterpret_cast<uint32_t *>(p.ws + L.icnt) +
+                         (GU ? 0 : L.umax * ceil_div(p.ff, kTileM) + ceil_div(L.ffs, kTileM));
         int seg = 0;
         for (int unit = a; unit < b; ++seg) {
-            const int item = unit / upi;
-            const int seg_end = min(b, (item + 1) * upi);
+            const Unit x = decode(unit);
+            const int item = x.item;
+            const int seg_end = min(b, x.iend);
             const int buf = seg & 1;
             float acc[NMAT][kChunk];
 #pragma unroll
@@ -392,7 +497,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&aempty[buf])) : "memory");
 
-            const bool whole = unit == item * upi && seg_end == (item + 1) * upi;
+            const bool whole = unit == x.istart && seg_end == x.iend;
             bool fin = whole;
             if (!whole) {
                 const int slot = unit == a ? 0 : 1;
@@ -403,8 +508,8 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     for (int t = 0; t < kChunk; ++t)
                         if (t < Tc) sp[(m * kChunk + t) * kTileM + rowl] = acc[m][t];
                 umma::bar_sync(1, 128);
+                const int c0 = owner(x.istart), c1 = owner(x.iend - 1);
                 if (threadIdx.x == 0) {
-                    const int c0 = owner(item * upi), c1 = owner((item + 1) * upi - 1);
                     const uint32_t old = atom_add_acq_rel(icnt + item, 1u);
                     const int last = old == (uint32_t)(c1 - c0);
                     if (last) icnt[item] = 0u;
@@ -414,13 +519,12 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 fin = *s_last != 0;
                 if (fin) {
                     // sum every piece of the item in K order
-                    const int c0 = owner(item * upi), c1 = owner((item + 1) * upi - 1);
 #pragma unroll
                     for (int m = 0; m < NMAT; ++m)
 #pragma unroll
                         for (int t = 0; t < kChunk; ++t) acc[m][t] = 0.f;
                     for (int cc = c0; cc <= c1; ++cc) {
-                        const int sl = start(cc) < item * upi ? 1 : 0;
+                        const int sl = start(cc) < x.istart ? 1 : 0;
                         const float *q = spart + (size_t)((cc * 2 + sl) * 2) * kChunk * kTileM;
 #pragma unroll
                         for (int m = 0; m < NMAT; ++m)
@@ -432,37 +536,55 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             }
             if (fin) {
                 if constexpr (GU) {
-                    const Unit x = decode(item * upi);
-                    const int f = x.rb * kTileM + rowl;  // ff row of this thread
-                    const uint8_t *blob = ublob[x.u];
-                    const uint32_t msk = __ldcg(reinterpret_cast<const uint32_t *>(p.ws + L.uniq_mask) + x.u);
-                    const int8_t *uslot = reinterpret_cast<const int8_t *>(p.ws + L.uniq_slot) + x.u * kChunk;
-                    const float *wt = reinterpret_cast<const float *>(p.ws + L.wt);
-                    const int nkt_ff = ceil_div(p.ff, kTileK);
-                    const int blk = x.rb * 4 + warp;  // 32-row block of ff
-                    const int kt = blk >> 3;
-                    uint8_t *tile = p.ws + L.hb + ((size_t)x.u * nkt_ff + kt) * N * 128;
-                    uint8_t *sfw = p.ws + L.hsf + ((size_t)x.u * nkt_ff + kt) * 2 * kSfRow * 4;
+                    const int f = x.rb * kTileM + rowl;  // ff (or ff_s) row of this thread
+                    if (!x.shared) {
+                        const uint8_t *blob = ublob[x.u];
+                        const uint32_t msk = __ldcg(reinterpret_cast<const uint32_t *>(p.ws + L.uniq_mask) + x.u);
+                        const int8_t *uslot = reinterpret_cast<const int8_t *>(p.ws + L.uniq_slot) + x.u * kChunk;
+                        const float *wt = reinterpret_cast<const float *>(p.ws + L.wt);
+                        const int nkt_ff = ceil_div(p.ff, kTileK);
+                        const int blk = x.rb * 4 + warp;  // 32-row block of ff
+                        const int kt = blk >> 3;
+                        uint8_t *tile = p.ws + L.hb + ((size_t)x.u * nkt_ff + kt) * N * 128;
+                        uint8_t *sfw = p.ws + L.hsf + ((size_t)x.u * nkt_ff + kt) * 2 * kSfRow * 4;
 #pragma unroll
-                    for (int t = 0; t < kChunk; ++t) {
-                        if (t < Tc) {
-                            float h = 0.f;
-                            if (blob != nullptr && ((msk >> t) & 1u) && f < p.ff) {
-                                const int j = uslot[t];
-                                h = silu_mul(acc[0][t], acc[1][t]) * __ldcg(wt + t * p.k + j);
+                        for (int t = 0; t < kChunk; ++t) {
+                            if (t < Tc) {
+                                float h = 0.f;
+                                if (blob != nullptr && ((msk >> t) & 1u) && f < p.ff) {
+                                    const int j = uslot[t];
+                                    h = silu_mul(acc[0][t], acc[1][t]) * __ldcg(wt + t * p.k + j);
+                                }
+                                quantize_pieces(h, lane, t, blk & 7, N, tile, sfw);
                             }
-                            quantize_pieces(h, lane, t, blk & 7, N, tile, sfw);
+                        }
+                    } else if (f < p.ffs) {
+                        // shared: h as bf16 hi + lo (pieces 0, 1; the others zero), weight 1
+                        uint8_t *tile = p.ws + L.hsb + (size_t)(f / kTileKs) * N * 128;
+                        const int c = (f % kTileKs) / 8, e = f % 8;
+#pragma unroll
+                        for (int t = 0; t < kChunk; ++t) {
+                            if (t < Tc) {
+                                const float h = silu_mul(acc[0][t], acc[1][t]);
+                                const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+                                const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
+#pragma unroll
+                                for (int pc = 0; pc < kPieces; ++pc) {
+                                    const int n = t * kPieces + pc;
+                                    const __nv_bfloat16 v = pc == 0 ? hi : (pc == 1 ? lo : __float2bfloat16_rn(0.f));
+                                    *reinterpret_cast<__nv_bfloat16 *>(tile + (c * (N / 8) + n / 8) * 128 +
+                                                                       (n % 8) * 16 + e * 2) = v;
+                                }
+                            }
                         }
                     }
                 } else {
                     const int row = item * kTileM + rowl;
                     if (row < p.d) {
-                        const float *ob = reinterpret_cast<const float *>(p.ws + L.ob);
 #pragma unroll
                         for (int t = 0; t < kChunk; ++t) {
                             if (t < Tc) {
-                                float y = acc[0][t];
-                                if (p.has_shared) y += __ldcg(ob + (size_t)t * (p.k + 1) * p.d + row);
+                                const float y = acc[0][t];
                                 if (p.out_fp32)
                                     reinterpret_cast<float *>(p.y)[(size_t)t * p.d + row] = y;
                                 else
