@@ -25,7 +25,8 @@ struct WsHeader {
     uint32_t status;
     uint32_t router_done;  // router rows finished in this call; back to 0 by its end
     uint32_t n_unique;     // distinct routed experts in the current token chunk
-    uint32_t pad[61];
+    uint32_t topk_done;    // tokens whose top-k other CTAs finished; back to 0 by its end
+    uint32_t pad[60];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -74,15 +75,16 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
-// try_wait with a suspend-time hint: the warp sleeps in hardware until the
-// phase completes (or ~1 ms passes) instead of spinning on the barrier.
+// try_wait without a time hint: the hardware's own short wait window, then
+// the caller polls again (no long suspension between phase completion and
+// wake-up on the pipeline's critical path).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
         " selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }

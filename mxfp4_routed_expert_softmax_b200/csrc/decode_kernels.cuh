@@ -37,89 +37,131 @@ struct RouteParams {
 constexpr int kRouteThreads = 256;
 constexpr int kRouteTok = 4;  // tokens per pass over the rows (x kept in smem as fp32)
 
-// Softmax over all E logits and the top-k (descending, ties to the lower
-// index) of one token, by one warp.  NPL logits per lane stay in registers.
+// Order-preserving 32-bit key of a float (larger float -> larger key; -0 is
+// first made +0 so that equal values have equal keys) and its inverse.
+__device__ __forceinline__ uint32_t fkey(float v) {
+    const uint32_t u = __float_as_uint(v + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float fkey_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+constexpr uint32_t kNone = 0xffffffffu;
+
+// The k largest keys among NPL (key, id) slots per lane (id kNone: empty),
+// ties to the lower id, written by lane 0 to okey/oid (kNone once the slots
+// run out).  Each lane keeps its best remaining slot; a round takes the
+// warp's largest key (redux max) and, among the lanes holding it, the lowest
+// id (redux min): two warp reductions and one lane's rescan of NPL slots.
 template <int NPL>
-__device__ void warp_topk(const float *row, int E, int k, int lane, int32_t *idx, float *wt,
-                          int32_t *idx2, float *wt2) {
-    float v[NPL];
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-        int e = lane + 32 * i;
-        v[i] = e < E ? __ldcg(row + e) : -INFINITY;
-    }
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) m = fmaxf(m, v[i]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < NPL; ++i)
-        if (lane + 32 * i < E) s += expf(v[i] - m);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    const float inv_s = 1.0f / s;
-    uint32_t taken = 0;
-    for (int j = 0; j < k; ++j) {
-        float bv = 0.f;
-        int bi = 0x7fffffff;
+__device__ void warp_select(const uint32_t (&key)[NPL], const uint32_t (&id)[NPL], int k, int lane,
+                            uint32_t *okey, uint32_t *oid) {
+    uint32_t taken = 0u, bk = 0u, bi = kNone;
+    int bs = 0;
+    auto best = [&]() {
+        bk = 0u;
+        bi = kNone;
 #pragma unroll
         for (int i = 0; i < NPL; ++i) {
-            int e = lane + 32 * i;
-            bool cand = e < E && !((taken >> i) & 1u);
-            if (cand && (bi == 0x7fffffff || v[i] > bv)) {
-                bv = v[i];
-                bi = e;
+            if (id[i] != kNone && !((taken >> i) & 1u) &&
+                (bi == kNone || key[i] > bk || (key[i] == bk && id[i] < bi))) {
+                bk = key[i];
+                bi = id[i];
+                bs = i;
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            bool better = (oi != 0x7fffffff) &&
-                          (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi));
-            if (better) {
-                bv = ov;
-                bi = oi;
-            }
+    };
+    best();
+    for (int j = 0; j < k; ++j) {
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, bi != kNone ? bk : 0u);
+        const uint32_t imin = __reduce_min_sync(0xffffffffu, (bi != kNone && bk == kmax) ? bi : kNone);
+        if (imin != kNone && bi == imin) {
+            taken |= 1u << bs;
+            best();
         }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
         if (lane == 0) {
-            float w = expf(bv - m) * inv_s;
-            idx[j] = bi;
-            wt[j] = w;
-            if (idx2) idx2[j] = bi;
-            if (wt2) wt2[j] = w;
+            okey[j] = kmax;
+            oid[j] = imin;
         }
     }
 }
 
-// Top-k of every token of the chunk, then the dispatch: distinct experts in
-// ascending id, their token masks, the slot of each (expert, token), the
-// per-token E4M3 prescale of x, zeroed |h| maxima.  Run by one whole CTA.
-__device__ void topk_dispatch(const RouteParams &p, WsHeader *hdr) {
+// Softmax over all E logits and the top-k (descending logit, ties to the
+// lower index) of token t, by one whole CTA: each warp selects the top-k of
+// its eighth of the experts (up to 4 logits per lane), warp 0 selects the
+// top-k of those 8k candidates.  Thread 0 writes the results.
+__device__ void cta_topk(const RouteParams &p, int t) {
+    __shared__ uint32_t s_ck[8][32], s_ci[8][32];
+    __shared__ float s_red[2][8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float *row = reinterpret_cast<const float *>(p.ws + p.L.logits) + (size_t)t * p.E;
+    const int S = (p.E + 7) / 8;  // <= 128: 4 per lane
+    float v[4];
+    uint32_t key[4], id[4];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int o = lane + 32 * i, e = warp * S + o;
+        const bool ok = o < S && e < p.E;
+        v[i] = ok ? __ldcg(row + e) : -INFINITY;
+        key[i] = fkey(v[i]);
+        id[i] = ok ? (uint32_t)e : kNone;
+        mx = fmaxf(mx, v[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) s_red[0][warp] = mx;
+    __syncthreads();
+    float m = s_red[0][0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, s_red[0][w]);
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        if (id[i] != kNone) sum += expf(v[i] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) s_red[1][warp] = sum;
+    warp_select<4>(key, id, p.k, lane, s_ck[warp], s_ci[warp]);
+    __syncthreads();
+    if (warp != 0) return;
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += s_red[1][w];
+    const float inv_s = 1.0f / s;
+    uint32_t ck[8], ci[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int c = lane + 32 * i, w = c / p.k, jj = c - w * p.k;
+        const bool ok = w < 8;
+        ck[i] = ok ? s_ck[w][jj] : 0u;
+        ci[i] = ok ? s_ci[w][jj] : kNone;
+    }
+    __syncwarp();
+    uint32_t *fk = s_ck[0], *fi = s_ci[0];  // reused for the result (lane 0 writes after reading)
+    warp_select<8>(ck, ci, p.k, lane, fk, fi);
+    __syncwarp();
+    if (lane == 0) {
+        int32_t *i1 = reinterpret_cast<int32_t *>(p.ws + p.L.idx) + t * p.k;
+        float *w1 = reinterpret_cast<float *>(p.ws + p.L.wt) + t * p.k;
+        for (int j = 0; j < p.k; ++j) {
+            const float w = expf(fkey_value(fk[j]) - m) * inv_s;
+            i1[j] = (int32_t)fi[j];
+            w1[j] = w;
+            if (p.idx_out) p.idx_out[(size_t)t * p.k + j] = (int32_t)fi[j];
+            if (p.w_out) p.w_out[(size_t)t * p.k + j] = w;
+        }
+    }
+}
+
+// The dispatch of a chunk whose top-k is done: distinct experts in ascending
+// id, their token masks, the slot of each (expert, token), their blob
+// pointers (checked) and ids.  Run by one whole CTA.
+__device__ void dispatch(const RouteParams &p, WsHeader *hdr) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Layout &L = p.L;
-    float *logits = reinterpret_cast<float *>(p.ws + L.logits);
-    int32_t *idx = reinterpret_cast<int32_t *>(p.ws + L.idx);
-    float *wt = reinterpret_cast<float *>(p.ws + L.wt);
-    if (warp < p.Tc) {
-        const int t = warp;
-        const float *row = logits + (size_t)t * p.E;
-        int32_t *i2 = p.idx_out ? p.idx_out + (size_t)t * p.k : nullptr;
-        float *w2 = p.w_out ? p.w_out + (size_t)t * p.k : nullptr;
-        int32_t *i1 = idx + t * p.k;
-        float *w1 = wt + t * p.k;
-        if (p.E <= 32) warp_topk<1>(row, p.E, p.k, lane, i1, w1, i2, w2);
-        else if (p.E <= 64) warp_topk<2>(row, p.E, p.k, lane, i1, w1, i2, w2);
-        else if (p.E <= 128) warp_topk<4>(row, p.E, p.k, lane, i1, w1, i2, w2);
-        else if (p.E <= 256) warp_topk<8>(row, p.E, p.k, lane, i1, w1, i2, w2);
-        else if (p.E <= 512) warp_topk<16>(row, p.E, p.k, lane, i1, w1, i2, w2);
-        else warp_topk<32>(row, p.E, p.k, lane, i1, w1, i2, w2);
-    }
-    if (p.blobs == nullptr) return;  // route only: no dispatch
-    if (threadIdx.x == 0 && p.has_shared) write_shared_tmaps(p.ws, L, p.smap);
+    const int32_t *idx = reinterpret_cast<const int32_t *>(p.ws + L.idx);
     __syncthreads();
     __shared__ uint32_t bitmap[32];
     __shared__ uint32_t prefix[32];
@@ -130,7 +172,7 @@ __device__ void topk_dispatch(const RouteParams &p, WsHeader *hdr) {
     for (int i = threadIdx.x; i < kChunk * 32; i += blockDim.x) umask[i] = 0u;
     __syncthreads();
     for (int i = threadIdx.x; i < TK; i += blockDim.x) {
-        int e = idx[i];
+        const int e = __ldcg(idx + i);
         atomicOr(&bitmap[e >> 5], 1u << (e & 31));
     }
     __syncthreads();
@@ -150,7 +192,7 @@ __device__ void topk_dispatch(const RouteParams &p, WsHeader *hdr) {
     for (int i = threadIdx.x; i < TK * kChunk; i += blockDim.x) uslot[i] = -1;
     __syncthreads();
     for (int i = threadIdx.x; i < TK; i += blockDim.x) {
-        int e = idx[i];
+        const int e = __ldcg(idx + i);
         int t = i / p.k, j = i - t * p.k;
         uint32_t u = prefix[e >> 5] + __popc(bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
         uslot[u * kChunk + t] = (int8_t)j;
@@ -158,6 +200,7 @@ __device__ void topk_dispatch(const RouteParams &p, WsHeader *hdr) {
     }
     __syncthreads();
     const uint8_t **ublob = reinterpret_cast<const uint8_t **>(p.ws + L.uniq_blob);
+    int32_t *ueid = reinterpret_cast<int32_t *>(p.ws + L.uniq_eid);
     uint32_t *gmask = reinterpret_cast<uint32_t *>(p.ws + L.uniq_mask);
     for (int w = threadIdx.x; w < nwords * 32; w += blockDim.x) {
         if ((bitmap[w >> 5] >> (w & 31)) & 1u) {
@@ -168,8 +211,8 @@ __device__ void topk_dispatch(const RouteParams &p, WsHeader *hdr) {
                 b = nullptr;
             }
             ublob[u] = b;
+            ueid[u] = w;
             gmask[u] = umask[u];
-            if (b != nullptr) write_expert_tmaps(p.ws, L, (int)u, b, p.tmpl);
         }
     }
 }
@@ -270,57 +313,91 @@ __device__ int stream_router(const RouteParams &p, const float *xs, int t0, int 
     return finished;
 }
 
+// Wait (bounded) until *ctr reaches target; false (timeout bit set) if not.
+__device__ bool wait_count(const uint32_t *ctr, uint32_t target, WsHeader *hdr) {
+    const uint64_t t0 = globaltimer();
+    while (ld_acquire(ctr) < target) {
+        __nanosleep(64);
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            set_status(hdr, kStTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Cooperative launch (every CTA resident).  CTAs 1.. stream the router rows;
+// once all rows are in, token t's top-k runs on CTA t mod G (all its warps),
+// and CTA 0, after its own tokens, waits for the others' and dispatches.
+// Meanwhile the streaming CTAs build the gate/up pass's activation pieces and
+// every expert's tensor maps, which need no routing.
 __global__ void __launch_bounds__(kRouteThreads, 3) route_kernel(const __grid_constant__ RouteParams p) {
     extern __shared__ __align__(16) float xs[];  // [kRouteTok][d]
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + p.L.hdr);
+    __shared__ int s_ok;
     pdl_trigger();
     const int npass = (p.Tc + kRouteTok - 1) / kRouteTok;
-    // the gate/up pass's pieces of x need no routing: every CTA builds a share
-    if (p.blobs != nullptr)
-        build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L, blockIdx.x * (kRouteThreads / 32) + (threadIdx.x >> 5),
-                       gridDim.x * (kRouteThreads / 32), p.has_shared != 0);
-    if (blockIdx.x == 0) {
-        // wait (bounded) for every router row of every pass, then route and dispatch
-        __shared__ int s_ok;
-        if (threadIdx.x == 0) {
-            const uint32_t target = (uint32_t)(p.E * npass);
-            const uint64_t t0 = globaltimer();
-            int ok = 1;
-            while (ld_acquire(&hdr->router_done) < target) {
-                __nanosleep(128);
-                if (globaltimer() - t0 > kWaitLimitNs) {
-                    set_status(hdr, kStTimeout);
-                    ok = 0;
-                    break;
-                }
+    const int G = gridDim.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (blockIdx.x > 0) {
+        const int j = (blockIdx.x - 1) * (kRouteThreads / 32) + warp;
+        const int d = p.d;
+        for (int pass = 0; pass < npass; ++pass) {
+            const int t0 = pass * kRouteTok;
+            const int nt = min(kRouteTok, p.Tc - t0);
+            __syncthreads();
+            for (int i = threadIdx.x; i < nt * d / 2; i += blockDim.x) {
+                const int t = (2 * i) / d, c = (2 * i) % d;
+                const uint32_t w = reinterpret_cast<const uint32_t *>(p.x + (size_t)(t0 + t) * d)[c / 2];
+                xs[t * d + c] = bf16_lo(w);
+                xs[t * d + c + 1] = bf16_hi(w);
             }
-            s_ok = ok;
+            __syncthreads();
+            const int nr = stream_router(p, xs, t0, nt, pass, j, lane);
+            // one release per warp: its logits are visible before they are counted
+            if (lane == 0 && nr > 0) red_add_release(&hdr->router_done, (uint32_t)nr);
         }
+    }
+    // top-k of this CTA's tokens once every router row is in
+    if ((int)blockIdx.x < p.Tc) {
+        __syncthreads();
+        if (threadIdx.x == 0) s_ok = wait_count(&hdr->router_done, (uint32_t)(p.E * npass), hdr);
         __syncthreads();
         if (!s_ok) return;
-        topk_dispatch(p, hdr);
+        for (int t = blockIdx.x; t < p.Tc; t += G) {
+            cta_topk(p, t);
+            __syncthreads();
+        }
+        if (blockIdx.x > 0 && threadIdx.x == 0) {
+            int mine = 0;
+            for (int t = blockIdx.x; t < p.Tc; t += G) ++mine;
+            red_add_release(&hdr->topk_done, (uint32_t)mine);  // after thread 0's own result stores
+        }
+    }
+    if (blockIdx.x == 0) {
+        int mine = 0;
+        for (int t = 0; t < p.Tc; t += G) ++mine;
+        if (threadIdx.x == 0) s_ok = wait_count(&hdr->topk_done, (uint32_t)(p.Tc - mine), hdr);
         __syncthreads();
-        if (threadIdx.x == 0) hdr->router_done = 0u;
+        if (!s_ok) return;
+        if (p.blobs != nullptr) dispatch(p, hdr);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            hdr->router_done = 0u;
+            hdr->topk_done = 0u;
+        }
         return;
     }
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (p.blobs == nullptr) return;
+    // work of the gate/up pass that needs no routing
     const int j = (blockIdx.x - 1) * (kRouteThreads / 32) + warp;
-    const int d = p.d;
-    for (int pass = 0; pass < npass; ++pass) {
-        const int t0 = pass * kRouteTok;
-        const int nt = min(kRouteTok, p.Tc - t0);
-        __syncthreads();
-        for (int i = threadIdx.x; i < nt * d / 2; i += blockDim.x) {
-            const int t = (2 * i) / d, c = (2 * i) % d;
-            const uint32_t w = reinterpret_cast<const uint32_t *>(p.x + (size_t)(t0 + t) * d)[c / 2];
-            xs[t * d + c] = bf16_lo(w);
-            xs[t * d + c + 1] = bf16_hi(w);
-        }
-        __syncthreads();
-        const int nr = stream_router(p, xs, t0, nt, pass, j, lane);
-        // one release per warp: its logits are visible before they are counted
-        if (lane == 0 && nr > 0) red_add_release(&hdr->router_done, (uint32_t)nr);
+    build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L, j, p.nwarps, p.has_shared != 0);
+    const int tid = (blockIdx.x - 1) * kRouteThreads + threadIdx.x;
+    for (int e = tid; e < p.E; e += (G - 1) * kRouteThreads) {
+        const uint8_t *b = p.blobs[e];
+        if (b != nullptr && (reinterpret_cast<uintptr_t>(b) & 15u) == 0u) write_expert_tmaps(p.ws, p.L, e, b, p.tmpl);
     }
+    if (tid == 0 && p.has_shared) write_shared_tmaps(p.ws, p.L, p.smap);
 }
 
 // ======================================================= single expert ==
@@ -347,6 +424,7 @@ __global__ void single_expert_setup_kernel(const __grid_constant__ SingleParams 
                 b = nullptr;
             }
             reinterpret_cast<const uint8_t **>(p.ws + p.L.uniq_blob)[0] = b;
+            reinterpret_cast<int32_t *>(p.ws + p.L.uniq_eid)[0] = 0;
             reinterpret_cast<uint32_t *>(p.ws + p.L.uniq_mask)[0] = (1u << p.Tc) - 1u;
             if (b != nullptr) write_expert_tmaps(p.ws, p.L, 0, b, p.tmpl);
         }

@@ -39,41 +39,42 @@ constexpr int kAtile = kTileM * 128;  // one A box: 128 rows x 128 bytes (16 KB)
 // ---------------------------------------------------------------- pieces --
 // One 32-element activation block (element = this lane's v) of token t ->
 // kPieces E2M1 pieces.  Piece p: scale exponent e from the largest |residual|
-// r of the block (smallest e with max|r| <= 6 * 2^e), codes = r / 2^e rounded
-// to the nearest E2M1 value, residual r -= code * 2^e (exact in fp32: the
+// r of the block (smallest e with max|r| <= 6 * 2^e; the order of
+// non-negative floats is the order of their bits, so one warp max-reduction
+// of the bits finds it), codes = r / 2^e rounded to the nearest E2M1 value
+// (ties to the even code), residual r -= code * 2^e (exact in fp32: the
 // subtracted value is a multiple of the residual's unit in the last place).
+// Rounding to the E2M1 grid: below 2 the grid step is 0.5, below 4 it is 1,
+// up to 6 it is 2; adding then subtracting 2^22, 2^23 or 2^24 rounds an fp32
+// of that size to a multiple of the step, ties to even.  The code of a grid
+// value q >= 1 is read off its fp32 bits (exponent and top mantissa bit),
+// below 1 it is 0 or 1 (0.5).
 // Writes the 16-byte nibble row of each piece into a K-tile of the B operand
 // (no-swizzle K-major core matrices, N rows, this block is 16-byte chunk c of
-// the tile) and its scale byte into the tile's scale words
-// (sfw[(c/4)*kSfRow + n], byte c%4).  All 32 lanes of the warp call it.
+// the tile; element 2i in the low nibble of byte i) and its scale byte into
+// the tile's scale words (sfw[(c/4)*kSfRow + n], byte c%4).  All 32 lanes of
+// the warp call it.
 __device__ __forceinline__ void quantize_pieces(float v, int lane, int t, int c, int N, uint8_t *tile,
                                                 uint8_t *sfw) {
     float r = v;
 #pragma unroll
     for (int p = 0; p < kPieces; ++p) {
-        float amax = fabsf(r);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const uint32_t bits = __float_as_uint(amax);
+        const uint32_t bits = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(r)));
         // amax = 1.f * 2^e0: 6 * 2^(e0-2) = 1.5 * 2^e0 covers 1.f <= 1.5
         int e = (int)(bits >> 23) - 127 - 2 + ((bits & 0x7FFFFFu) > 0x400000u ? 1 : 0);
         e = max(-126, min(126, e));
         const float s = r * exp2i(-e);
         const float m = fabsf(s);
-        float q;
-        if (m < 2.f) q = rintf(m * 2.f) * 0.5f;
-        else if (m < 4.f) q = rintf(m);
-        else q = rintf(m * 0.5f) * 2.f;
-        uint32_t code = q < 2.f ? (uint32_t)(q * 2.f) : (q < 4.f ? (uint32_t)q + 2u : (q < 5.f ? 6u : 7u));
-        if (s < 0.f && code != 0u) code |= 8u;
-        r -= copysignf(q, s) * exp2i(e);
-        uint32_t w = code << (4 * (lane & 7));
-        w |= __shfl_xor_sync(0xffffffffu, w, 1);
-        w |= __shfl_xor_sync(0xffffffffu, w, 2);
-        w |= __shfl_xor_sync(0xffffffffu, w, 4);
+        const float C = m < 2.f ? 4194304.f : (m < 4.f ? 8388608.f : 16777216.f);
+        const float q = __fsub_rn(__fadd_rn(m, C), C);
+        const uint32_t qb = __float_as_uint(q);
+        uint32_t code = q >= 1.f ? (qb >> 22) - 252u : (q > 0.f ? 1u : 0u);
+        code |= (s < 0.f && code != 0u) ? 8u : 0u;
+        r = __fmaf_rn(-copysignf(q, s), exp2i(e), r);
+        const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
         const int n = t * kPieces + p;
-        if ((lane & 7) == 0)
-            *reinterpret_cast<uint32_t *>(tile + (c * (N / 8) + n / 8) * 128 + (n % 8) * 16 + (lane >> 3) * 4) = w;
+        uint8_t *row = tile + (c * (N / 8) + n / 8) * 128 + (n % 8) * 16;
+        if ((lane & 1) == 0) row[lane >> 1] = (uint8_t)(code | (hi << 4));
         if (lane == 0) sfw[((c >> 2) * kSfRow + n) * 4 + (c & 3)] = (uint8_t)(e + 127);
     }
 }
@@ -109,7 +110,7 @@ __device__ void build_x_pieces(const uint16_t *x, int Tc, int d, uint8_t *ws, co
 // The shared expert's three tensor maps (encoded by the host with their real
 // addresses) into the workspace, where the tensor-core kernels read them.
 __device__ void write_shared_tmaps(uint8_t *ws, const Layout &L, const uint4 (&smap)[3][8]) {
-    uint4 *o = reinterpret_cast<uint4 *>(ws + L.tmap + (size_t)L.umax * 3 * 128);
+    uint4 *o = reinterpret_cast<uint4 *>(ws + L.tmap + (size_t)L.E * 3 * 128);
 #pragma unroll
     for (int m = 0; m < 3; ++m)
 #pragma unroll
@@ -117,13 +118,13 @@ __device__ void write_shared_tmaps(uint8_t *ws, const Layout &L, const uint4 (&s
     umma::tmap_release();
 }
 
-// Tensor maps of distinct expert u: copies of the host-encoded templates
-// (W_g/W_u share one: ff rows of d/2 bytes; W_d: d rows of ff/2 bytes)
-// pointed at the expert's nibble planes.  One thread.
-__device__ void write_expert_tmaps(uint8_t *ws, const Layout &L, int u, const uint8_t *blob,
+// Tensor maps of expert e: copies of the host-encoded templates (W_g/W_u
+// share one: ff rows of d/2 bytes; W_d: d rows of ff/2 bytes) pointed at the
+// expert's nibble planes.  One thread.
+__device__ void write_expert_tmaps(uint8_t *ws, const Layout &L, int e, const uint8_t *blob,
                                    const uint4 (&tmpl)[2][8]) {
     const size_t mat = (size_t)L.d * L.ff;
-    uint8_t *dst = ws + L.tmap + (size_t)u * 3 * 128;
+    uint8_t *dst = ws + L.tmap + (size_t)e * 3 * 128;
     const uint8_t *addr[3] = {blob, blob + mat / 2 + mat / 32, blob + mat + mat / 16};
 #pragma unroll
     for (int m = 0; m < 3; ++m) {
@@ -151,8 +152,14 @@ __host__ __device__ inline int umma_stage_bytes(bool gu) { return (gu ? 2 : 1) *
 // TMEM scale columns of one stage, every group aligned: A scales 8 per matrix
 // (2 groups x 4 row blocks), then B scales (group g at +4g, up to 2 columns).
 __host__ __device__ inline int umma_sf_cols(bool gu) { return gu ? 32 : 16; }
+// Per-call metadata copied into shared memory by every CTA: blob pointer,
+// expert id and per-token routing weight (0 where the token did not select
+// it) of each distinct expert.  Global loads issued while the weight stream
+// saturates HBM wait thousands of cycles, so the pipeline never makes them.
+constexpr int kMetaU = kChunk * 32;  // distinct experts of a chunk (top_k <= 32)
+constexpr int kMetaBytes = kMetaU * 8 + kMetaU * 4 + kMetaU * kChunk * 4;
 __host__ __device__ inline int umma_smem_bytes(bool gu, int nst) {
-    return 1024 + nst * umma_stage_bytes(gu) + 256;
+    return 1024 + nst * umma_stage_bytes(gu) + 256 + kMetaBytes;
 }
 
 // Load the (up to) 8 scale bytes of one weight row for one K-tile: nks valid
@@ -190,6 +197,9 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     uint32_t *tslot = reinterpret_cast<uint32_t *>(aempty + 2);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tslot + 1);
     volatile int *s_last = s_abort + 1;
+    const uint8_t **s_blob = reinterpret_cast<const uint8_t **>(smem + nst * SB + 256);
+    int32_t *s_eid = reinterpret_cast<int32_t *>(s_blob + kMetaU);
+    float *s_wu = reinterpret_cast<float *>(s_eid + kMetaU);  // [u][t]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Layout &L = p.L;
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + L.hdr);
@@ -216,6 +226,24 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
 
     const int Tc = p.Tc, N = act_n(Tc);
     const int U = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_unique);
+    {
+        const uint8_t *const *gb = reinterpret_cast<const uint8_t *const *>(p.ws + L.uniq_blob);
+        const int32_t *ge = reinterpret_cast<const int32_t *>(p.ws + L.uniq_eid);
+        const uint32_t *gm = reinterpret_cast<const uint32_t *>(p.ws + L.uniq_mask);
+        const int8_t *gs = reinterpret_cast<const int8_t *>(p.ws + L.uniq_slot);
+        const float *gw = reinterpret_cast<const float *>(p.ws + L.wt);
+        for (int i = threadIdx.x; i < U; i += kUThreads) {
+            s_blob[i] = gb[i];
+            s_eid[i] = ge[i];
+        }
+        for (int i = threadIdx.x; i < U * kChunk; i += kUThreads) {
+            const int u = i / kChunk, t = i - u * kChunk;
+            float w = 0.f;
+            if (t < Tc && ((gm[u] >> t) & 1u)) w = gw[t * p.k + gs[u * kChunk + t]];
+            s_wu[i] = w;
+        }
+        __syncthreads();
+    }
     const int K = GU ? p.d : p.ff;   // routed reduction length
     const int M = GU ? p.ff : p.d;   // routed weight rows
     const int Ks = GU ? p.d : p.ffs; // shared reduction length
@@ -232,8 +260,9 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     auto owner = [&](int unit) { return (int)((((long long)unit + 1) * G - 1) / total); };
     const int a = cta < G ? start(cta) : 0, b = cta < G ? start(cta + 1) : 0;
     const size_t mat = (size_t)p.d * p.ff;
-    const uint8_t *const *ublob = reinterpret_cast<const uint8_t *const *>(p.ws + L.uniq_blob);
-    const uint8_t *smaps = p.ws + L.tmap + (size_t)L.umax * 3 * 128;
+    const uint8_t *const *ublob = s_blob;
+    const uint8_t *smaps = p.ws + L.tmap + (size_t)L.E * 3 * 128;
+    const int32_t *ueid = s_eid;
     const uint32_t idesc4 = umma::idesc_mxf4(N), idesc16 = umma::idesc_bf16(N);
     // TMEM columns: accumulators [buf][mat] at (buf*NMAT + mat)*64 (N <= 64), then
     // the scale columns of each stage from sf0
@@ -293,15 +322,32 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     auto ksteps = [&](const Unit &x) {
         return x.shared ? min(4, (Ks - x.kt * kTileKs) / 16) : min(4, (K - x.kt * kTileK) / 64);
     };
+    // The unit after x (no divisions): next K-tile, then the next expert
+    // (down), then the shared K-tiles; at the end of an item, a full decode.
+    auto advance = [&](const Unit &x, int unit_next) {
+        Unit y = x;
+        if (unit_next >= x.iend) return unit_next < total ? decode(unit_next) : x;
+        ++y.kt;
+        if constexpr (!GU) {
+            if (!y.shared && y.kt == nkt) {
+                y.kt = 0;
+                if (++y.u == U) {
+                    y.u = -1;
+                    y.shared = true;
+                }
+            }
+        }
+        return y;
+    };
 
     if (warp == 8) {
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
             int last_u = -2;
-            for (int unit = a, it = 0; unit < b && !*s_abort; ++unit, ++it) {
-                const Unit x = decode(unit);
-                const int s = it % nst;
-                if (it >= nst && !wait(&empty[s], (uint32_t)(((it / nst) + 1) & 1))) break;
+            Unit x = a < b ? decode(a) : Unit{};
+            uint32_t ph = 0u;  // phase of the current pass over the stages
+            for (int unit = a, it = 0, s = 0; unit < b && !*s_abort; x = advance(x, ++unit), ++it) {
+                if (it >= nst && !wait(&empty[s], ph ^ 1u)) break;
                 uint8_t *st = smem + s * SB;
                 const uint8_t *blob = x.shared ? nullptr : ublob[x.u];
                 const uint8_t *maps = nullptr;
@@ -310,7 +356,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     maps = smaps + (GU ? 0 : 256);
                     bsrc = (GU ? p.ws + L.xbf : p.ws + L.hsb) + (size_t)x.kt * N * 128;
                 } else {
-                    maps = p.ws + L.tmap + (size_t)x.u * 3 * 128 + (GU ? 0 : 256);
+                    maps = p.ws + L.tmap + (size_t)ueid[x.u] * 3 * 128 + (GU ? 0 : 256);
                     bsrc = GU ? p.ws + L.xb + (size_t)x.kt * N * 128
                               : p.ws + L.hb + ((size_t)x.u * nkt + x.kt) * N * 128;
                 }
@@ -327,6 +373,17 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     mbar_arrive_expect_tx(&full[s], (uint32_t)(N * 128));
                 }
                 bulk_g2s(st + NMAT * kAtile, bsrc, (uint32_t)(N * 128), &full[s]);
+                if (++s == nst) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (*s_abort) {
+                // a wait gave up somewhere: let the copies this thread issued
+                // land (bounded) before the CTA's shared memory goes away
+                const uint64_t t0 = globaltimer();
+                while (globaltimer() - t0 < 200000ull) {
+                }
             }
         }
     } else if (warp >= 4 && warp < 8) {
@@ -407,48 +464,63 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         }
     } else if (warp == 9) {
         // ------------------------------------------------- MMA issuer --
+        // One thread; everything per MMA is an add on precomputed descriptors
+        // (the start-address field of a descriptor is its low 14 bits, and
+        // every operand address here stays below 256 KB).
         if (lane == 0) {
-            int it = 0, seg = 0;
+            const uint64_t adesc0 = umma::smem_desc(smem_u32(smem), 16u, 1024u, umma::kLayoutSw128);
+            const uint64_t bdesc0 = umma::smem_desc(smem_u32(smem) + NMAT * kAtile, (uint32_t)((N / 8) * 128), 128u,
+                                                    umma::kLayoutNone);
+            const uint32_t bstep = (uint32_t)(2 * (N / 8) * 128) >> 4;  // one k-step of B (2 chunks)
+            const uint32_t id4[2] = {umma::idesc_sf_id(idesc4, 0u), umma::idesc_sf_id(idesc4, 2u)};
+            int seg = 0, s = 0;
+            uint32_t ph = 0u;
             for (int unit = a; unit < b && !*s_abort; ++seg) {
-                const int seg_end = min(b, decode(unit).iend);
+                Unit x = decode(unit);
+                const int seg_end = min(b, x.iend);
                 const int buf = seg & 1;
                 if (seg >= 2 && !wait(&aempty[buf], (uint32_t)(((seg >> 1) + 1) & 1))) break;
                 umma::fence_after();
                 const uint32_t dcol = tbase + (uint32_t)(buf * NMAT * 64);
-                for (int un = unit; un < seg_end; ++un, ++it) {
-                    const Unit x = decode(un);
-                    const int s = it % nst;
-                    if (!wait(&full[s], (uint32_t)((it / nst) & 1))) break;
+                uint32_t acc = 0u;
+                for (int un = unit; un < seg_end; x = advance(x, ++un)) {
+                    if (!wait(&full[s], ph)) break;
                     umma::fence_after();
-                    const uint32_t st = smem_u32(smem + s * SB);
-                    const uint32_t sfc = tbase + sf0 + (uint32_t)(s * SFC);
+                    const uint32_t soff = (uint32_t)(s * SB) >> 4;
+                    const uint64_t a0 = adesc0 + soff, b0 = bdesc0 + soff;
                     const int nks = ksteps(x);
-                    for (int sk = 0; sk < nks; ++sk) {
-                        const uint64_t bdesc =
-                            umma::smem_desc(st + NMAT * kAtile + (uint32_t)(2 * sk * (N / 8) * 128),
-                                            (uint32_t)((N / 8) * 128), 128u, umma::kLayoutNone);
-                        const uint32_t acc = (un != unit || sk != 0) ? 1u : 0u;
-                        if (x.shared) {
+                    if (x.shared) {
 #pragma unroll
-                            for (int m = 0; m < NMAT; ++m) {
-                                const uint64_t adesc = umma::smem_desc(st + (uint32_t)(m * kAtile + 32 * sk), 16u,
-                                                                       1024u, umma::kLayoutSw128);
-                                umma::mma_bf16(dcol + (uint32_t)(m * 64), adesc, bdesc, idesc16, acc);
+                        for (int sk = 0; sk < 4; ++sk) {
+                            if (sk < nks) {
+                                const uint64_t bd = b0 + sk * bstep;
+                                umma::mma_bf16(dcol, a0 + 2 * sk, bd, idesc16, acc);
+                                if (GU) umma::mma_bf16(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, idesc16, acc);
+                                acc = 1u;
                             }
-                        } else {
-                            const uint32_t grp = (uint32_t)(sk >> 1), sfid = (uint32_t)(2 * (sk & 1));
-                            const uint32_t id = umma::idesc_sf_id(idesc4, sfid);
-                            const uint32_t sfb = (sfc + 8 * NMAT + grp * 4) | (sfid << 30);
+                        }
+                    } else {
+                        const uint32_t sfc = tbase + sf0 + (uint32_t)(s * SFC);
 #pragma unroll
-                            for (int m = 0; m < NMAT; ++m) {
-                                const uint64_t adesc = umma::smem_desc(st + (uint32_t)(m * kAtile + 32 * sk), 16u,
-                                                                       1024u, umma::kLayoutSw128);
-                                const uint32_t sfa = (sfc + 8 * m + grp * 4) | (sfid << 30);
-                                umma::mma_mxf4(dcol + (uint32_t)(m * 64), adesc, bdesc, id, acc, sfa, sfb);
+                        for (int sk = 0; sk < 4; ++sk) {
+                            if (sk < nks) {
+                                const uint64_t bd = b0 + sk * bstep;
+                                const uint32_t sfid = (uint32_t)(2 * (sk & 1)) << 30;
+                                const uint32_t sfb = (sfc + 8 * NMAT + (sk >> 1) * 4) | sfid;
+                                umma::mma_mxf4(dcol, a0 + 2 * sk, bd, id4[sk & 1], acc, (sfc + (sk >> 1) * 4) | sfid,
+                                               sfb);
+                                if (GU)
+                                    umma::mma_mxf4(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, id4[sk & 1], acc,
+                                                   (sfc + 8 + (sk >> 1) * 4) | sfid, sfb);
+                                acc = 1u;
                             }
                         }
                     }
                     umma::commit(&empty[s]);
+                    if (++s == nst) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 umma::commit(&afull[buf]);
                 unit = seg_end;
@@ -539,9 +611,6 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     const int f = x.rb * kTileM + rowl;  // ff (or ff_s) row of this thread
                     if (!x.shared) {
                         const uint8_t *blob = ublob[x.u];
-                        const uint32_t msk = __ldcg(reinterpret_cast<const uint32_t *>(p.ws + L.uniq_mask) + x.u);
-                        const int8_t *uslot = reinterpret_cast<const int8_t *>(p.ws + L.uniq_slot) + x.u * kChunk;
-                        const float *wt = reinterpret_cast<const float *>(p.ws + L.wt);
                         const int nkt_ff = ceil_div(p.ff, kTileK);
                         const int blk = x.rb * 4 + warp;  // 32-row block of ff
                         const int kt = blk >> 3;
@@ -551,10 +620,8 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                         for (int t = 0; t < kChunk; ++t) {
                             if (t < Tc) {
                                 float h = 0.f;
-                                if (blob != nullptr && ((msk >> t) & 1u) && f < p.ff) {
-                                    const int j = uslot[t];
-                                    h = silu_mul(acc[0][t], acc[1][t]) * __ldcg(wt + t * p.k + j);
-                                }
+                                const float w = s_wu[x.u * kChunk + t];
+                                if (blob != nullptr && w != 0.f && f < p.ff) h = silu_mul(acc[0][t], acc[1][t]) * w;
                                 quantize_pieces(h, lane, t, blk & 7, N, tile, sfw);
                             }
                         }
