@@ -193,6 +193,39 @@ k3moe_status k3moe_layer_timed(const void *x, int32_t T, const float *w_router, 
                                int32_t *n_kernels);
 
 /*
+ * k3moe_layer without a caller-supplied workspace.  The pages this library
+ * follows have no counterpart of this call; it exists for callers that cannot
+ * allocate device memory at the point where they run the layer (code that
+ * must not call an allocator on its hot path, or a host framework whose
+ * allocator is not reachable through a C ABI).  Neither the library nor the
+ * caller allocates anything: the scratch is a fixed 16 MiB buffer in the
+ * library's own device data, one per device.
+ *   - The first call on a device looks up that buffer's device address for
+ *     the current device (cudaGetSymbolAddress) and clears it on `stream`;
+ *     make that first call before any stream capture begins.  A call whose
+ *     shape (d, ff, n_experts, top_k, ff_shared) differs from the previous
+ *     call's on that device also clears it first (the scratch layout and the
+ *     counters in it that must start at zero depend on the shape).
+ *   - Shapes whose scratch (k3moe_workspace_size(dims, 8)) exceeds 16 MiB are
+ *     rejected with K3MOE_ERR_WORKSPACE_TOO_SMALL before anything runs; the
+ *     K3 shape (d=7168, ff=1536, 896 experts, top-16, shared ff=1536) needs
+ *     about 10.5 MiB.
+ *   - All calls on one device share the buffer: two calls that may overlap
+ *     (other streams, other host threads) race and give wrong results.
+ *     Serialise them, or use k3moe_layer with a workspace per stream.
+ *   - Conditions only the device can see (misaligned blob pointers, a
+ *     bounded wait that ran out) are recorded in the buffer's status word,
+ *     which this interface does not read back; k3moe_layer reports them
+ *     through k3moe_device_status.
+ * Arguments, layouts, results and ordering are those of k3moe_layer without
+ * the routing copies (idx_out, w_out).
+ */
+k3moe_status k3moe_layer_noalloc(const void *x, int32_t T, const float *w_router, const float *bias,
+                                 const uint8_t *const *expert_blobs, const void *shared_wg,
+                                 const void *shared_wu, const void *shared_wd,
+                                 const k3moe_dims *dims, void *y, void *stream);
+
+/*
  * Synchronises `stream`, then reads and clears the workspace status word:
  * K3MOE_OK, K3MOE_ERR_DEVICE_CHECK or K3MOE_ERR_DEVICE_TIMEOUT.  After
  * K3MOE_ERR_DEVICE_TIMEOUT the outputs of the calls since the last check are

@@ -68,6 +68,7 @@ _SIGS = {
                               ctypes.c_int),
     "k3moe_layer_timed": ([_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _dp, _vp, _vp, _sz, _vp,
                            ctypes.POINTER(_vp), _i32, ctypes.POINTER(_i32)], ctypes.c_int),
+    "k3moe_layer_noalloc": ([_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _dp, _vp, _vp], ctypes.c_int),
     "k3moe_device_status": ([_vp, _vp], ctypes.c_int),
     "k3moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "k3moe_last_error": ([], ctypes.c_char_p),
@@ -143,6 +144,13 @@ def k3moe_layer(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu, shared
                            _ptr(shared_wg), _ptr(shared_wu), _ptr(shared_wd), ctypes.byref(dims),
                            _ptr(y), _ptr(idx_out), _ptr(w_out), _ptr(ws), ws_bytes,
                            _stream(stream))
+
+
+def k3moe_layer_noalloc(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu, shared_wd, dims, y,
+                        stream=None) -> int:
+    return lib.k3moe_layer_noalloc(_ptr(x), T, _ptr(w_router), _ptr(bias), _ptr(expert_blobs),
+                                   _ptr(shared_wg), _ptr(shared_wu), _ptr(shared_wd),
+                                   ctypes.byref(dims), _ptr(y), _stream(stream))
 
 
 def k3moe_layer_from_host(x_host, T, w_router, bias, expert_blobs, shared_wg, shared_wu,

@@ -24,8 +24,15 @@ thread_local std::string g_last_error;
 constexpr int kMaxDevices = 64;
 constexpr int kSmemLimit = 227 * 1024;
 
+// Scratch of k3moe_layer_noalloc: one buffer per device, in the library's own
+// device data (no allocation by the library or the caller).
+constexpr size_t kNoAllocBytes = (size_t)16 << 20;
+static __device__ __align__(256) uint8_t g_noalloc_ws[kNoAllocBytes];
+
 struct DeviceInfo {
     bool ready = false;
+    uint8_t *noalloc = nullptr;  // device address of g_noalloc_ws on this device, once set up
+    int noalloc_shape[5] = {0, 0, 0, 0, 0};  // (d, ff, E, k, ff_shared) its layout was last used for
     int sms = 0;
     int route_smem = -1;  // dynamic smem of the last occupancy query
     int route_occ = 0;    // resident route_shared CTAs per SM at that size
@@ -382,6 +389,29 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
     return K3MOE_OK;
 }
 
+// The built-in scratch of k3moe_layer_noalloc on this device.  The first
+// call looks up its device address.  The workspace layout depends on the
+// shape, and every layout keeps counters that must start at zero, so the
+// buffer is cleared (on the call's stream) whenever the shape differs from
+// the one it last served, the first call included.
+k3moe_status noalloc_scratch(DeviceInfo &di, const k3moe_dims *dm, cudaStream_t st, uint8_t **out) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!di.noalloc) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_ws);
+        if (e != cudaSuccess) return cuda_fail(e, "scratch address");
+        di.noalloc = reinterpret_cast<uint8_t *>(p);
+    }
+    const int shape[5] = {dm->d, dm->ff, dm->n_experts, dm->top_k, dm->ff_shared};
+    if (memcmp(shape, di.noalloc_shape, sizeof(shape)) != 0) {
+        cudaError_t e = cudaMemsetAsync(di.noalloc, 0, kNoAllocBytes, st);
+        if (e != cudaSuccess) return cuda_fail(e, "scratch clear");
+        memcpy(di.noalloc_shape, shape, sizeof(shape));
+    }
+    *out = di.noalloc;
+    return K3MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -529,6 +559,30 @@ k3moe_status k3moe_layer_timed(const void *x, int32_t T, const float *w_router, 
                                 nullptr, &hk);
     *n_kernels = 3;
     return s;
+}
+
+k3moe_status k3moe_layer_noalloc(const void *x, int32_t T, const float *w_router, const float *bias,
+                                 const uint8_t *const *expert_blobs, const void *shared_wg,
+                                 const void *shared_wu, const void *shared_wd,
+                                 const k3moe_dims *dims, void *y, void *stream) {
+    k3moe_status s = check_dims(dims);
+    if (s != K3MOE_OK) return s;
+    const size_t need = layout_for(dims, dims->top_k).total;
+    if (need > kNoAllocBytes) {
+        g_last_error = "k3moe_layer_noalloc: this shape needs " + std::to_string(need) +
+                       " bytes of scratch, the built-in buffer holds " + std::to_string(kNoAllocBytes);
+        return K3MOE_ERR_WORKSPACE_TOO_SMALL;
+    }
+    if (T < 1 || !x || !y || !aligned(x, 16) || !aligned(y, 16)) return K3MOE_ERR_INVALID_ARGUMENT;
+    DeviceInfo *di = nullptr;
+    s = device_info(&di);
+    if (s != K3MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = nullptr;
+    s = noalloc_scratch(*di, dims, st, &ws);
+    if (s != K3MOE_OK) return s;
+    return layer_impl(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu, shared_wd, dims, y,
+                      nullptr, nullptr, ws, kNoAllocBytes, stream, nullptr, nullptr);
 }
 
 k3moe_status k3moe_device_status(void *ws, void *stream) {
