@@ -193,10 +193,16 @@ def main():
     ap.add_argument("--config", default="k3_decode", choices=list(k3gen.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="profiling mode: no e2e/cpu legs")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="profiling: keep only this many experts resident (same d, ff, top-k); the "
+                         "routed and shared bytes per token stay those of the workload, the router shrinks")
     args = ap.parse_args()
     if args.warmup < 3 and not args.quick:
         args.warmup = 3
     cfg = k3gen.CONFIGS[args.config]
+    if args.experts is not None:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, name=f"{cfg.name}_e{args.experts}", E=args.experts)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

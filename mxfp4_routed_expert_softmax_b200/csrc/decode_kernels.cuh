@@ -29,7 +29,8 @@ struct RouteParams {
     int32_t *idx_out;   // optional [Tc][k]
     float *w_out;       // optional [Tc][k]
     int nwarps;         // streaming warps: 8 per CTA, CTAs 1.. of the grid
-    uint4 tmpl[2][8];   // tensor-map templates: W_g/W_u plane, W_d plane
+    uint4 tmpl[4][8];   // tensor-map templates: W_g/W_u, W_d nibble planes; their scale planes
+    int scale_mask;     // which scale-plane templates exist (bit 0: W_g/W_u, bit 1: W_d)
     uint4 smap[3][8];   // shared expert tensor maps (W_g, W_u, W_d), when has_shared
     int has_shared;     // the tensor-core kernels run a shared expert
 };
@@ -395,7 +396,7 @@ __global__ void __launch_bounds__(kRouteThreads, 3) route_kernel(const __grid_co
     const int tid = (blockIdx.x - 1) * kRouteThreads + threadIdx.x;
     for (int e = tid; e < p.E; e += (G - 1) * kRouteThreads) {
         const uint8_t *b = p.blobs[e];
-        if (b != nullptr && (reinterpret_cast<uintptr_t>(b) & 15u) == 0u) write_expert_tmaps(p.ws, p.L, e, b, p.tmpl);
+        if (b != nullptr && (reinterpret_cast<uintptr_t>(b) & 15u) == 0u) write_expert_tmaps(p.ws, p.L, e, b, p.tmpl, p.scale_mask);
     }
     if (tid == 0 && p.has_shared) write_shared_tmaps(p.ws, p.L, p.smap);
 }
@@ -409,7 +410,8 @@ struct SingleParams {
     const uint8_t *blob;
     uint8_t *ws;
     Layout L;
-    uint4 tmpl[2][8];
+    uint4 tmpl[4][8];
+    int scale_mask;
 };
 
 __global__ void single_expert_setup_kernel(const __grid_constant__ SingleParams p) {
@@ -426,7 +428,7 @@ __global__ void single_expert_setup_kernel(const __grid_constant__ SingleParams 
             reinterpret_cast<const uint8_t **>(p.ws + p.L.uniq_blob)[0] = b;
             reinterpret_cast<int32_t *>(p.ws + p.L.uniq_eid)[0] = 0;
             reinterpret_cast<uint32_t *>(p.ws + p.L.uniq_mask)[0] = (1u << p.Tc) - 1u;
-            if (b != nullptr) write_expert_tmaps(p.ws, p.L, 0, b, p.tmpl);
+            if (b != nullptr) write_expert_tmaps(p.ws, p.L, 0, b, p.tmpl, p.scale_mask);
         }
         if (threadIdx.x < kChunk) {
             const int t = threadIdx.x;

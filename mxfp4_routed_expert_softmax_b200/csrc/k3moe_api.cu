@@ -82,8 +82,8 @@ int shared_ff(const k3moe_dims *dm) {
 
 // Pipeline depth of the tensor-core kernels: as many stages as fit in shared
 // memory and in the TMEM scale columns (8 stages after the accumulators).
-int umma_stages(bool gu) {
-    int n = (kSmemLimit - umma_smem_bytes(gu, 0)) / umma_stage_bytes(gu);
+int umma_stages(bool gu, int N) {
+    int n = (kSmemLimit - umma_smem_bytes(gu, N, 0)) / umma_stage_bytes(gu, N);
     const int cap = 8;
     return n < cap ? n : cap;
 }
@@ -135,12 +135,12 @@ cudaError_t launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
 // library does not link the driver library itself.
 struct TmapCache {
     int d = 0, ff = 0;
-    uint4 t[2][8];
+    uint4 t[4][8];
 };
 TmapCache g_tmaps[16];
 int g_ntmaps = 0;
 
-k3moe_status tmap_templates(int d, int ff, void *placeholder, uint4 (&out)[2][8]) {
+k3moe_status tmap_templates(int d, int ff, void *placeholder, uint4 (&out)[4][8]) {
     std::lock_guard<std::mutex> lock(g_mu);
     for (int i = 0; i < g_ntmaps; ++i)
         if (g_tmaps[i].d == d && g_tmaps[i].ff == ff) {
@@ -159,15 +159,23 @@ k3moe_status tmap_templates(int d, int ff, void *placeholder, uint4 (&out)[2][8]
         }
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    CUtensorMap m[2];
-    for (int i = 0; i < 2; ++i) {
-        const cuuint64_t cols = (cuuint64_t)(i == 0 ? d : ff) / 2, rows = (cuuint64_t)(i == 0 ? ff : d);
+    // [0], [1]: nibble planes, 128 rows x 128 bytes, 128-byte swizzle (the
+    // MMA's K-major layout); [2], [3]: scale planes, 128 rows x 16 bytes, no
+    // swizzle, only when the row of scales is a multiple of 16 bytes (the
+    // reduction length a multiple of 512), else left zero.
+    CUtensorMap m[4];
+    memset(m, 0, sizeof(m));
+    for (int i = 0; i < 4; ++i) {
+        const int kdim = (i % 2 == 0) ? d : ff, rdim = (i % 2 == 0) ? ff : d;
+        const bool scale = i >= 2;
+        if (scale && kdim % 512 != 0) continue;
+        const cuuint64_t cols = (cuuint64_t)(scale ? kdim / 32 : kdim / 2), rows = (cuuint64_t)rdim;
         const cuuint64_t dims[2] = {cols, rows};
         const cuuint64_t strides[1] = {cols};
-        const cuuint32_t box[2] = {128, (cuuint32_t)kTileM};
+        const cuuint32_t box[2] = {scale ? 16u : 128u, (cuuint32_t)kTileM};
         const cuuint32_t es[2] = {1, 1};
         CUresult r = encode(&m[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, placeholder, dims, strides, box, es,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, scale ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) {
             g_last_error = "cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")";
@@ -224,8 +232,11 @@ k3moe_status shared_tmaps(int d, int ffs, const void *wg, const void *wu, const 
 
 template <bool GU>
 cudaError_t launch_umma(const DeviceInfo &di, UmmaParams up, cudaStream_t st) {
-    up.nst = umma_stages(GU);
-    const int smem = umma_smem_bytes(GU, up.nst);
+    const int N = act_n(up.Tc);
+    up.nst = umma_stages(GU, N);
+    up.sb = umma_stage_bytes(GU, N);
+    up.sf_tma = (GU ? up.d : up.ff) % 512 == 0;
+    const int smem = umma_smem_bytes(GU, N, up.nst);
     const int g = di.sms < kMaxCtas ? di.sms : kMaxCtas;
     return launch(umma_expert_kernel<GU>, dim3(g), dim3(kUThreads), smem, st, true, up);
 }
@@ -314,7 +325,7 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
     uint8_t *xstage = wsb + L.total;
     uint8_t *ystage = xstage + align256((size_t)kChunk * d * 2);
 
-    uint4 tmpl[2][8];
+    uint4 tmpl[4][8];
     s = tmap_templates(d, dims->ff, ws, tmpl);
     if (s != K3MOE_OK) return s;
     uint4 smap[3][8];
@@ -353,6 +364,7 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         rp.idx_out = idx_out ? idx_out + (size_t)c0 * dims->top_k : nullptr;
         rp.w_out = w_out ? w_out + (size_t)c0 * dims->top_k : nullptr;
         memcpy(rp.tmpl, tmpl, sizeof(tmpl));
+        rp.scale_mask = (d % 512 == 0 ? 1 : 0) | (dims->ff % 512 == 0 ? 2 : 0);
         memcpy(rp.smap, smap, sizeof(smap));
         rp.has_shared = ffs > 0;
         EventHook none;
@@ -486,7 +498,7 @@ k3moe_status k3moe_expert_ffn(const void *x, int32_t T, const uint8_t *blob,
     uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
     const int d = dims->d;
     const bool out32 = (dims->flags & K3MOE_OUT_FP32) != 0;
-    uint4 tmpl[2][8];
+    uint4 tmpl[4][8];
     s = tmap_templates(d, dims->ff, ws, tmpl);
     if (s != K3MOE_OK) return s;
     for (int c0 = 0; c0 < T; c0 += kChunk) {
@@ -501,6 +513,7 @@ k3moe_status k3moe_expert_ffn(const void *x, int32_t T, const uint8_t *blob,
         sp.ws = wsb;
         sp.L = L;
         memcpy(sp.tmpl, tmpl, sizeof(tmpl));
+        sp.scale_mask = (d % 512 == 0 ? 1 : 0) | (dims->ff % 512 == 0 ? 2 : 0);
         int nblk = (Tc * (d / 32) + 7) / 8;  // one warp per 32-element block
         if (nblk > di->sms) nblk = di->sms;
         cudaError_t e = launch(single_expert_setup_kernel, dim3(nblk), dim3(256), 0, st, false, sp);

@@ -35,8 +35,9 @@ struct Layout {
     size_t uniq_slot;  // i8  [kChunk*k][kChunk] slot j of token t for it, -1 if none
     size_t part;       // f32 [2][E][kMaxSeg][4] partial sums of router rows split between warps
     size_t cnt;        // u32 [2][E] arrivals per split row (back to 0 after each row)
-    size_t tmap;       // 128-byte tensor maps [E][3]: W_g, W_u, W_d nibble planes of each
-                       // expert; then the shared expert's W_g, W_u, W_d (bf16) at [E*3 ..]
+    size_t tmap;       // 128-byte tensor maps [E][6]: W_g, W_u, W_d nibble planes and their
+                       // scale planes, of each expert; then the shared expert's W_g, W_u,
+                       // W_d (bf16) at [E*6 ..]
     size_t xb;         // u8  [nkt_d][N*128] E2M1 pieces of x (gate/up B operand)
     size_t xsf;        // u32 [nkt_d][2][kSfRow] their E8M0 scales (byte = block in group)
     size_t hb;         // u8  [umax][nkt_ff][N*128] pieces of w*h (down B operand)
@@ -82,7 +83,7 @@ __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int f
     const int nkt_d = ceil_div(d, kTileK), nkt_ff = ceil_div(ff, kTileK);
     L.umax = umax;
     L.tmap = o;
-    o = align256(o + ((size_t)E * 3 + 3) * 128);
+    o = align256(o + ((size_t)E * 6 + 3) * 128);
     L.xb = o;
     o = align256(o + (size_t)nkt_d * kNMax * 128);
     L.xsf = o;

@@ -34,6 +34,9 @@
 namespace k3 {
 
 constexpr int kUThreads = 320;
+// Tensor maps per expert in the workspace: W_g, W_u, W_d nibble planes, then
+// (used when the reduction lengths are multiples of 512) their scale planes.
+constexpr int kMapsPerExpert = 6;
 constexpr int kAtile = kTileM * 128;  // one A box: 128 rows x 128 bytes (16 KB)
 
 // ---------------------------------------------------------------- pieces --
@@ -110,7 +113,7 @@ __device__ void build_x_pieces(const uint16_t *x, int Tc, int d, uint8_t *ws, co
 // The shared expert's three tensor maps (encoded by the host with their real
 // addresses) into the workspace, where the tensor-core kernels read them.
 __device__ void write_shared_tmaps(uint8_t *ws, const Layout &L, const uint4 (&smap)[3][8]) {
-    uint4 *o = reinterpret_cast<uint4 *>(ws + L.tmap + (size_t)L.E * 3 * 128);
+    uint4 *o = reinterpret_cast<uint4 *>(ws + L.tmap + (size_t)L.E * kMapsPerExpert * 128);
 #pragma unroll
     for (int m = 0; m < 3; ++m)
 #pragma unroll
@@ -118,19 +121,27 @@ __device__ void write_shared_tmaps(uint8_t *ws, const Layout &L, const uint4 (&s
     umma::tmap_release();
 }
 
-// Tensor maps of expert e: copies of the host-encoded templates (W_g/W_u
-// share one: ff rows of d/2 bytes; W_d: d rows of ff/2 bytes) pointed at the
-// expert's nibble planes.  One thread.
+// Tensor maps of expert e: copies of the host-encoded templates pointed at
+// the expert's planes.  Templates: [0] W_g/W_u nibbles (ff rows of d/2 bytes),
+// [1] W_d nibbles (d rows of ff/2 bytes), [2] W_g/W_u scales (ff rows of d/32
+// bytes), [3] W_d scales (d rows of ff/32 bytes); the scale maps are written
+// only where scale_mask says their template exists (bit 0: W_g/W_u, bit 1:
+// W_d; the reduction length a multiple of 512).  One thread.
 __device__ void write_expert_tmaps(uint8_t *ws, const Layout &L, int e, const uint8_t *blob,
-                                   const uint4 (&tmpl)[2][8]) {
+                                   const uint4 (&tmpl)[4][8], int scale_mask) {
     const size_t mat = (size_t)L.d * L.ff;
-    uint8_t *dst = ws + L.tmap + (size_t)e * 3 * 128;
-    const uint8_t *addr[3] = {blob, blob + mat / 2 + mat / 32, blob + mat + mat / 16};
+    uint8_t *dst = ws + L.tmap + (size_t)e * kMapsPerExpert * 128;
+    const uint8_t *addr[kMapsPerExpert] = {blob,           blob + mat / 2 + mat / 32, blob + mat + mat / 16,
+                                           blob + mat / 2, blob + mat + mat / 32,     blob + mat + mat / 16 + mat / 2};
+    const int which[kMapsPerExpert] = {0, 0, 1, 2, 2, 3};
 #pragma unroll
-    for (int m = 0; m < 3; ++m) {
+    for (int m = 0; m < kMapsPerExpert; ++m) {
+        if (which[m] == 2 && !(scale_mask & 1)) continue;
+        if (which[m] == 3 && !(scale_mask & 2)) continue;
+        const uint4 *src = tmpl[which[m]];
         uint4 *o = reinterpret_cast<uint4 *>(dst + m * 128);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) o[j] = tmpl[m == 2 ? 1 : 0][j];
+        for (int j = 0; j < 8; ++j) o[j] = src[j];
         umma::tmap_set_address(dst + m * 128, addr[m]);
     }
     umma::tmap_release();
@@ -143,12 +154,23 @@ struct UmmaParams {
     uint8_t *ws;
     Layout L;
     int nst;          // pipeline stages
+    int sb;           // bytes per stage (umma_stage_bytes for this N)
+    int sf_tma;       // A scales arrive by TMA with the stage (K a multiple of 512)
     // down only
     int out_fp32;     // y in fp32 (else bf16, rounded once)
     void *y;          // [Tc][d] of this chunk
 };
 
-__host__ __device__ inline int umma_stage_bytes(bool gu) { return (gu ? 2 : 1) * kAtile + kNMax * 128; }
+// One pipeline stage for MMA width N: the A boxes (16 KB per matrix, first,
+// so they stay 1024-byte aligned for the 128-byte swizzle), the B tile (N rows
+// x 128 bytes), the A scale boxes (128 rows x 16 bytes per matrix: the scales
+// of this K-tile and its neighbour) and the B scale words (2 x kSfRow words),
+// rounded up to 1024 bytes.
+__host__ __device__ inline int umma_sfa_off(bool gu, int N) { return (gu ? 2 : 1) * kAtile + N * 128; }
+__host__ __device__ inline int umma_sfb_off(bool gu, int N) { return umma_sfa_off(gu, N) + (gu ? 2 : 1) * 2048; }
+__host__ __device__ inline int umma_stage_bytes(bool gu, int N) {
+    return (umma_sfb_off(gu, N) + 2 * kSfRow * 4 + 1023) & ~1023;
+}
 // TMEM scale columns of one stage, every group aligned: A scales 8 per matrix
 // (2 groups x 4 row blocks), then B scales (group g at +4g, up to 2 columns).
 __host__ __device__ inline int umma_sf_cols(bool gu) { return gu ? 32 : 16; }
@@ -158,8 +180,8 @@ __host__ __device__ inline int umma_sf_cols(bool gu) { return gu ? 32 : 16; }
 // saturates HBM wait thousands of cycles, so the pipeline never makes them.
 constexpr int kMetaU = kChunk * 32;  // distinct experts of a chunk (top_k <= 32)
 constexpr int kMetaBytes = kMetaU * 8 + kMetaU * 4 + kMetaU * kChunk * 4;
-__host__ __device__ inline int umma_smem_bytes(bool gu, int nst) {
-    return 1024 + nst * umma_stage_bytes(gu) + 256 + kMetaBytes;
+__host__ __device__ inline int umma_smem_bytes(bool gu, int N, int nst) {
+    return 1024 + nst * umma_stage_bytes(gu, N) + 256 + kMetaBytes;
 }
 
 // Load the (up to) 8 scale bytes of one weight row for one K-tile: nks valid
@@ -187,11 +209,11 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     constexpr int NMAT = GU ? 2 : 1;
-    constexpr int SB = NMAT * kAtile + kNMax * 128;
     constexpr int SFC = GU ? 32 : 16;  // TMEM scale columns per stage (8-aligned)
-    const int nst = p.nst;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + nst * SB);
-    uint64_t *empty = full + nst;
+    const int nst = p.nst, SB = p.sb;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + nst * SB);  // stage bytes landed (TMA)
+    uint64_t *sfr = full + nst;                                        // stage scales in TMEM (4 warps)
+    uint64_t *empty = sfr + nst;                                       // stage consumed (MMA commit)
     uint64_t *afull = empty + nst;
     uint64_t *aempty = afull + 2;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(aempty + 2);
@@ -205,7 +227,8 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + L.hdr);
     if (threadIdx.x == 0) {
         for (int s = 0; s < nst; ++s) {
-            mbar_init(&full[s], 5);  // TMA thread + 4 scale warps
+            mbar_init(&full[s], 1);
+            mbar_init(&sfr[s], 4);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -261,7 +284,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     const int a = cta < G ? start(cta) : 0, b = cta < G ? start(cta + 1) : 0;
     const size_t mat = (size_t)p.d * p.ff;
     const uint8_t *const *ublob = s_blob;
-    const uint8_t *smaps = p.ws + L.tmap + (size_t)L.E * 3 * 128;
+    const uint8_t *smaps = p.ws + L.tmap + (size_t)L.E * kMapsPerExpert * 128;
     const int32_t *ueid = s_eid;
     const uint32_t idesc4 = umma::idesc_mxf4(N), idesc16 = umma::idesc_bf16(N);
     // TMEM columns: accumulators [buf][mat] at (buf*NMAT + mat)*64 (N <= 64), then
@@ -352,23 +375,42 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 const uint8_t *blob = x.shared ? nullptr : ublob[x.u];
                 const uint8_t *maps = nullptr;
                 const uint8_t *bsrc;
+                const uint8_t *scmaps = nullptr;  // the A scale planes' maps (TMA scale path)
+                const uint8_t *sfbsrc = nullptr;  // the B scale words of this K-tile
                 if (x.shared) {
                     maps = smaps + (GU ? 0 : 256);
                     bsrc = (GU ? p.ws + L.xbf : p.ws + L.hsb) + (size_t)x.kt * N * 128;
                 } else {
-                    maps = p.ws + L.tmap + (size_t)ueid[x.u] * 3 * 128 + (GU ? 0 : 256);
+                    const uint8_t *em = p.ws + L.tmap + (size_t)ueid[x.u] * kMapsPerExpert * 128;
+                    maps = em + (GU ? 0 : 256);
+                    scmaps = em + (GU ? 384 : 640);
                     bsrc = GU ? p.ws + L.xb + (size_t)x.kt * N * 128
                               : p.ws + L.hb + ((size_t)x.u * nkt + x.kt) * N * 128;
+                    sfbsrc = GU ? p.ws + L.xsf + (size_t)x.kt * 2 * kSfRow * 4
+                                : p.ws + L.hsf + ((size_t)x.u * nkt + x.kt) * 2 * kSfRow * 4;
                 }
+                const bool sf_dma = p.sf_tma && !x.shared && blob != nullptr;
                 if (x.shared || blob != nullptr) {
                     if (x.u != last_u) {
                         umma::tmap_acquire(maps);
                         if (GU) umma::tmap_acquire(maps + 128);
+                        if (sf_dma) {
+                            umma::tmap_acquire(scmaps);
+                            if (GU) umma::tmap_acquire(scmaps + 128);
+                        }
                         last_u = x.u;
                     }
-                    mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * kAtile + N * 128));
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * kAtile + N * 128 +
+                                                               (sf_dma ? NMAT * 2048 + 2 * kSfRow * 4 : 0)));
                     umma::tma_load_2d(st, maps, x.kt * 128, x.rb * kTileM, &full[s]);
                     if (GU) umma::tma_load_2d(st + kAtile, maps + 128, x.kt * 128, x.rb * kTileM, &full[s]);
+                    if (sf_dma) {
+                        // 16 scale bytes per row: this K-tile's 8 and its neighbour's
+                        uint8_t *sfa = st + umma_sfa_off(GU, N);
+                        umma::tma_load_2d(sfa, scmaps, (x.kt >> 1) * 16, x.rb * kTileM, &full[s]);
+                        if (GU) umma::tma_load_2d(sfa + 2048, scmaps + 128, (x.kt >> 1) * 16, x.rb * kTileM, &full[s]);
+                        bulk_g2s(st + umma_sfb_off(GU, N), sfbsrc, (uint32_t)(2 * kSfRow * 4), &full[s]);
+                    }
                 } else {
                     mbar_arrive_expect_tx(&full[s], (uint32_t)(N * 128));
                 }
@@ -388,6 +430,50 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         }
     } else if (warp >= 4 && warp < 8) {
         // --------------------------------------- scale factors -> TMEM --
+        const uint32_t lb = umma::lane_base(warp);
+        if (p.sf_tma) {
+            // The scales came with the stage's TMA copy: wait for the stage,
+            // then move this K-tile's 8 scale bytes of each row (and the B
+            // scales) into TMEM.  An expert whose blob failed its check gets
+            // zero scale bytes (finite 2^-127), so it adds exactly nothing.
+            Unit x = a < b ? decode(a) : Unit{};
+            uint32_t ph = 0u;
+            for (int unit = a, s = 0; unit < b; x = advance(x, ++unit)) {
+                int go = 0;
+                if (lane == 0) go = wait(&full[s], ph);
+                if (!__shfl_sync(0xffffffffu, go, 0)) break;
+                if (!x.shared) {
+                    const uint8_t *st = smem + s * SB;
+                    const bool has = ublob[x.u] != nullptr;
+                    const uint32_t col = tbase + lb + sf0 + (uint32_t)(s * SFC);
+#pragma unroll
+                    for (int m = 0; m < NMAT; ++m) {
+                        const uint8_t *sfa = st + umma_sfa_off(GU, N) + m * 2048 + (x.kt & 1) * 8;
+                        uint32_t w[8];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint2 v = has ? *reinterpret_cast<const uint2 *>(sfa + (32 * j + lane) * 16)
+                                                : make_uint2(0u, 0u);
+                            w[j] = v.x;      // group 0: k-steps 0, 1
+                            w[4 + j] = v.y;  // group 1: k-steps 2, 3
+                        }
+                        umma::st8(col + 8 * m, w);
+                    }
+                    const uint32_t *sb = reinterpret_cast<const uint32_t *>(st + umma_sfb_off(GU, N));
+                    const uint32_t w[8] = {has ? sb[lane] : 0u,          has ? sb[32 + lane] : 0u,          0u, 0u,
+                                           has ? sb[kSfRow + lane] : 0u, has ? sb[kSfRow + 32 + lane] : 0u, 0u, 0u};
+                    umma::st8(col + 8 * NMAT, w);
+                    umma::wait_st();
+                }
+                umma::fence_before();
+                __syncwarp();
+                if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sfr[s])) : "memory");
+                if (++s == nst) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        } else {
         // The global loads of a unit's scales are issued kLook units ahead of
         // its TMEM stores (a ring of registers), so their latency overlaps the
         // pipeline instead of adding to every stage.  Shared (bf16) units have
@@ -398,7 +484,6 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             uint32_t b[4];        // B scales: (g0, rows 0-31), (g0, 32-63), (g1, ...), (g1, ...)
             bool on;
         };
-        const uint32_t lb = umma::lane_base(warp);
         auto load = [&](int unit, SfRegs &r) {
             const Unit x = decode(unit);
             r.on = !x.shared;
@@ -443,7 +528,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             }
             umma::fence_before();
             __syncwarp();
-            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&full[s])) : "memory");
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sfr[s])) : "memory");
             return true;
         };
         SfRegs R4[kLook + 1];
@@ -461,6 +546,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     go = store(it, R4[q]);
                 }
             }
+        }
         }
     } else if (warp == 9) {
         // ------------------------------------------------- MMA issuer --
@@ -484,7 +570,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 const uint32_t dcol = tbase + (uint32_t)(buf * NMAT * 64);
                 uint32_t acc = 0u;
                 for (int un = unit; un < seg_end; x = advance(x, ++un)) {
-                    if (!wait(&full[s], ph)) break;
+                    if (!wait(&full[s], ph) || !wait(&sfr[s], ph)) break;
                     umma::fence_after();
                     const uint32_t soff = (uint32_t)(s * SB) >> 4;
                     const uint64_t a0 = adesc0 + soff, b0 = bdesc0 + soff;
