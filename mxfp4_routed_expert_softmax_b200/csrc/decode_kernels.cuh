@@ -28,11 +28,12 @@ struct RouteParams {
     const uint8_t *const *blobs;  // device array [E], null: no dispatch (route only)
     int32_t *idx_out;   // optional [Tc][k]
     float *w_out;       // optional [Tc][k]
-    int nwarps;         // streaming warps: 8 per CTA, CTAs 1.. of the grid
+    int nstage;         // router ring stages (kRStage bytes each)
     uint4 tmpl[4][8];   // tensor-map templates: W_g/W_u, W_d nibble planes; their scale planes
     int scale_mask;     // which scale-plane templates exist (bit 0: W_g/W_u, bit 1: W_d)
     uint4 smap[3][8];   // shared expert tensor maps (W_g, W_u, W_d), when has_shared
     int has_shared;     // the tensor-core kernels run a shared expert
+    const uint8_t *sw[3];  // the shared expert's W_g, W_u, W_d (the key of its cached maps)
 };
 
 constexpr int kRouteThreads = 256;
@@ -48,71 +49,54 @@ __device__ __forceinline__ float fkey_value(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-constexpr uint32_t kNone = 0xffffffffu;
-
-// The k largest keys among NPL (key, id) slots per lane (id kNone: empty),
-// ties to the lower id, written by lane 0 to okey/oid (kNone once the slots
-// run out).  Each lane keeps its best remaining slot; a round takes the
-// warp's largest key (redux max) and, among the lanes holding it, the lowest
-// id (redux min): two warp reductions and one lane's rescan of NPL slots.
-template <int NPL>
-__device__ void warp_select(const uint32_t (&key)[NPL], const uint32_t (&id)[NPL], int k, int lane,
-                            uint32_t *okey, uint32_t *oid) {
-    uint32_t taken = 0u, bk = 0u, bi = kNone;
-    int bs = 0;
-    auto best = [&]() {
-        bk = 0u;
-        bi = kNone;
+// Block-wide inclusive scan of v over the 256 threads in thread order.
+__device__ __forceinline__ uint32_t block_scan_incl(uint32_t v, uint32_t *s_tot) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-            if (id[i] != kNone && !((taken >> i) & 1u) &&
-                (bi == kNone || key[i] > bk || (key[i] == bk && id[i] < bi))) {
-                bk = key[i];
-                bi = id[i];
-                bs = i;
-            }
-        }
-    };
-    best();
-    for (int j = 0; j < k; ++j) {
-        const uint32_t kmax = __reduce_max_sync(0xffffffffu, bi != kNone ? bk : 0u);
-        const uint32_t imin = __reduce_min_sync(0xffffffffu, (bi != kNone && bk == kmax) ? bi : kNone);
-        if (imin != kNone && bi == imin) {
-            taken |= 1u << bs;
-            best();
-        }
-        if (lane == 0) {
-            okey[j] = kmax;
-            oid[j] = imin;
-        }
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
     }
+    if (lane == 31) s_tot[warp] = v;
+    __syncthreads();
+    uint32_t add = 0;
+    for (int w = 0; w < warp; ++w) add += s_tot[w];
+    __syncthreads();
+    return v + add;
 }
 
 // Softmax over all E logits and the top-k (descending logit, ties to the
-// lower index) of token t, by one whole CTA: each warp selects the top-k of
-// its eighth of the experts (up to 4 logits per lane), warp 0 selects the
-// top-k of those 8k candidates.  Thread 0 writes the results.
+// lower index) of token t, by one whole CTA (E <= 1024: 4 consecutive experts
+// per thread).  Radix select on the order-preserving keys: four 8-bit digit
+// passes (shared histogram, one warp's suffix scan) find the k-th largest key
+// K exactly; every key above K is taken, and of the keys equal to K the
+// lowest indices (a prefix count in index order).  The k winners are then
+// ranked by (key descending, index ascending) for the output order.
 __device__ void cta_topk(const RouteParams &p, int t) {
-    __shared__ uint32_t s_ck[8][32], s_ci[8][32];
+    __shared__ uint32_t s_hist[256];
+    __shared__ uint32_t s_tot[8];
     __shared__ float s_red[2][8];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const float *row = reinterpret_cast<const float *>(p.ws + p.L.logits) + (size_t)t * p.E;
-    const int S = (p.E + 7) / 8;  // <= 128: 4 per lane
+    __shared__ uint32_t s_pref, s_need, s_cnt;
+    __shared__ uint32_t s_selk[32], s_seli[32];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int E = p.E, k = p.k;
+    const float *row = reinterpret_cast<const float *>(p.ws + p.L.logits) + (size_t)t * E;
     float v[4];
-    uint32_t key[4], id[4];
+    uint32_t key[4];
+    bool ok[4];
     float mx = -INFINITY;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int o = lane + 32 * i, e = warp * S + o;
-        const bool ok = o < S && e < p.E;
-        v[i] = ok ? __ldcg(row + e) : -INFINITY;
-        key[i] = fkey(v[i]);
-        id[i] = ok ? (uint32_t)e : kNone;
+        const int e = 4 * tid + i;
+        ok[i] = e < E;
+        v[i] = ok[i] ? __ldcg(row + e) : -INFINITY;
+        key[i] = ok[i] ? fkey(v[i]) : 0u;  // real keys are > 0
         mx = fmaxf(mx, v[i]);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if (lane == 0) s_red[0][warp] = mx;
+    if (tid == 0) s_cnt = 0u;
     __syncthreads();
     float m = s_red[0][0];
 #pragma unroll
@@ -120,39 +104,90 @@ __device__ void cta_topk(const RouteParams &p, int t) {
     float sum = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        if (id[i] != kNone) sum += expf(v[i] - m);
+        if (ok[i]) sum += expf(v[i] - m);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     if (lane == 0) s_red[1][warp] = sum;
-    warp_select<4>(key, id, p.k, lane, s_ck[warp], s_ci[warp]);
+    // radix select of the k-th largest key
+    uint32_t pref = 0u, pmask = 0u;
+    uint32_t need = (uint32_t)k;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int sh = 24 - 8 * pass;
+        s_hist[tid] = 0u;
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (ok[i] && (key[i] & pmask) == pref) atomicAdd(&s_hist[(key[i] >> sh) & 255u], 1u);
+        __syncthreads();
+        if (warp == 0) {
+            // lane l holds digits 255-8l down to 248-8l (descending)
+            uint32_t c[8], lsum = 0u;
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                c[jj] = s_hist[255 - 8 * lane - jj];
+                lsum += c[jj];
+            }
+            uint32_t incl = lsum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            const uint32_t excl = incl - lsum;
+            if (excl < need && need <= incl) {
+                uint32_t acc = excl;
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    if (acc < need && acc + c[jj] >= need) {
+                        s_pref = pref | ((uint32_t)(255 - 8 * lane - jj) << sh);
+                        s_need = need - acc;
+                    }
+                    acc += c[jj];
+                }
+            }
+        }
+        __syncthreads();
+        pref = s_pref;
+        need = s_need;
+        pmask |= 0xFFu << sh;
+    }
+    // pref = the k-th largest key; take every key above it and the `need`
+    // lowest-index keys equal to it
+    uint32_t ties = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ties += (ok[i] && key[i] == pref) ? 1u : 0u;
+    uint32_t rank = block_scan_incl(ties, s_tot) - ties;  // ties at lower indices
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        bool take = ok[i] && key[i] > pref;
+        if (ok[i] && key[i] == pref) {
+            take = rank < need;
+            ++rank;
+        }
+        if (take) {
+            const uint32_t slot = atomicAdd(&s_cnt, 1u);
+            s_selk[slot] = key[i];
+            s_seli[slot] = (uint32_t)(4 * tid + i);
+        }
+    }
     __syncthreads();
     if (warp != 0) return;
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) s += s_red[1][w];
     const float inv_s = 1.0f / s;
-    uint32_t ck[8], ci[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int c = lane + 32 * i, w = c / p.k, jj = c - w * p.k;
-        const bool ok = w < 8;
-        ck[i] = ok ? s_ck[w][jj] : 0u;
-        ci[i] = ok ? s_ci[w][jj] : kNone;
-    }
-    __syncwarp();
-    uint32_t *fk = s_ck[0], *fi = s_ci[0];  // reused for the result (lane 0 writes after reading)
-    warp_select<8>(ck, ci, p.k, lane, fk, fi);
-    __syncwarp();
-    if (lane == 0) {
-        int32_t *i1 = reinterpret_cast<int32_t *>(p.ws + p.L.idx) + t * p.k;
-        float *w1 = reinterpret_cast<float *>(p.ws + p.L.wt) + t * p.k;
-        for (int j = 0; j < p.k; ++j) {
-            const float w = expf(fkey_value(fk[j]) - m) * inv_s;
-            i1[j] = (int32_t)fi[j];
-            w1[j] = w;
-            if (p.idx_out) p.idx_out[(size_t)t * p.k + j] = (int32_t)fi[j];
-            if (p.w_out) p.w_out[(size_t)t * p.k + j] = w;
+    if (lane < k) {
+        const uint32_t mk = s_selk[lane], mi = s_seli[lane];
+        int r = 0;
+        for (int q = 0; q < k; ++q) {
+            const uint32_t qk = s_selk[q], qi = s_seli[q];
+            r += (qk > mk || (qk == mk && qi < mi)) ? 1 : 0;
         }
+        const float w = expf(fkey_value(mk) - m) * inv_s;
+        reinterpret_cast<int32_t *>(p.ws + p.L.idx)[t * k + r] = (int32_t)mi;
+        reinterpret_cast<float *>(p.ws + p.L.wt)[t * k + r] = w;
+        if (p.idx_out) p.idx_out[(size_t)t * k + r] = (int32_t)mi;
+        if (p.w_out) p.w_out[(size_t)t * k + r] = w;
     }
 }
 
@@ -224,94 +259,236 @@ __device__ __forceinline__ int chunk_owner(long long c, long long N, int W) {
     return (int)(((c + 1) * (long long)W - 1) / N);
 }
 
-// A router row's sums are ready: write its logits (bias added).
-__device__ __forceinline__ void finalize_row(const RouteParams &p, int row, int t0, int nt, const float *v) {
-    float *logits = reinterpret_cast<float *>(p.ws + p.L.logits);
-    const float b = p.bias ? p.bias[row] : 0.f;
-    for (int t = 0; t < nt; ++t) logits[(size_t)(t0 + t) * p.E + row] = v[t] + b;
+// ------------------------------------------------------ router stream --
+// Router GEMV l = W_r x + b.  The fp32 router is one array of E*d floats; CTA
+// c of G owns the contiguous units [c*U/G, (c+1)*U/G) of 16 floats (U =
+// E*d/16; rows are whole units since d is a multiple of 64).  Its slice goes
+// through a ring of kRStage-byte shared-memory stages filled by bulk
+// asynchronous copies, so one thread keeps the SM's memory pipe full.  Thread
+// i of a stage takes its 16 floats (one row), the warp sums lanes of equal
+// row with a fixed shuffle tree (segmented), and after the stage's barrier
+// threads fold the warps' row sums into the CTA's row accumulators in warp
+// order, so every sum has a fixed order.  Rows cut by a CTA boundary are
+// finished by the last of their CTAs to arrive, summing the CTAs' parts in
+// CTA order.
+constexpr int kRStage = 16384;               // bytes per ring stage
+constexpr int kRFloats = kRStage / 4;        // 4096 floats: 256 units of 16
+constexpr int kRSegs = 16;                   // row segments per warp and stage (512 floats, d >= 64)
+constexpr int kRMaxRows = 72;                // rows of one CTA's slice (E/G + 2 <= 66)
+constexpr int kRFast = 8;                    // slices of at most this many rows: per-thread row sums
+
+struct RouteSmem {
+    float acc[kRMaxRows][kRouteTok];
+    int seg_row[2][8][kRSegs];
+    float seg_val[2][8][kRSegs][kRouteTok];
+    int seg_n[2][8];
+};
+
+__host__ __device__ inline int route_smem_bytes(int d, int nt, int nstage) {
+    return nstage * kRStage + nt * d * 4 + (int)sizeof(RouteSmem) + nstage * 8 + 64;
 }
 
-// One warp streams its slice of the router rows; every row is d*4 bytes =
-// d/4 chunks of 16 B.  Returns (in lane 0) the number of rows it finished.
-__device__ int stream_router(const RouteParams &p, const float *xs, int t0, int nt, int pass, int j, int lane) {
-    int finished = 0;
-    const int d = p.d;
-    const int cpr = d / 4;
-    const int W = p.nwarps;
-    const long long N = (long long)p.E * cpr;
-    long long c = (long long)j * N / W;
-    const long long cend = (long long)(j + 1) * N / W;
-    float *part = reinterpret_cast<float *>(p.ws + p.L.part);    // [2][E][kMaxSeg][kRouteTok]
-    uint32_t *cnt = reinterpret_cast<uint32_t *>(p.ws + p.L.cnt);  // [2][E]
-    while (c < cend) {
-        const int r = (int)(c / cpr);
-        const int a = (int)(c - (long long)r * cpr);
-        const int b = (int)min((long long)cpr, (long long)a + (cend - c));
-        float a0[kRouteTok];
+// This CTA's router slice: units [u0, u1) of 16 floats, in stages of 256.
+__device__ __forceinline__ void router_slice(const RouteParams &p, long long &u0, long long &u1) {
+    const long long U = (long long)p.E * p.d / 16;
+    u0 = (long long)blockIdx.x * U / gridDim.x;
+    u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;
+}
+__device__ __forceinline__ void router_issue(const RouteParams &p, uint8_t *ring, uint64_t *full, long long u0,
+                                             long long u1, int j, int slot) {
+    const long long a = u0 + 256LL * j;
+    const long long e = min(u1, a + 256);
+    const uint32_t bytes = (uint32_t)((e - a) * 64);
+    mbar_arrive_expect_tx(&full[slot], bytes);
+    bulk_g2s(ring + (size_t)slot * kRStage, p.wr + a * 16, bytes, &full[slot]);
+}
+// One thread: the first stages of a pass (the ring is free), issued before
+// anything else so the weight stream starts at once.
+__device__ void router_prefetch(const RouteParams &p, uint8_t *ring, uint64_t *full, int nstage, int chunk) {
+    long long u0, u1;
+    router_slice(p, u0, u1);
+    const int nch = (int)((u1 - u0 + 255) / 256);
+    for (int j = 0; j < nch && j < nstage; ++j) router_issue(p, ring, full, u0, u1, j, (chunk + j) % nstage);
+}
+
+// Streams this CTA's router slice once for tokens t0 .. t0+nt-1 (x in xs as
+// fp32 [nt][d]; the first stages already issued by router_prefetch);
+// finishes the rows it can and counts them on router_done.  `chunk` numbers
+// the CTA's stages across passes (ring phase).  All threads.
+__device__ void stream_router(const RouteParams &p, WsHeader *hdr, uint8_t *ring, uint64_t *full, int nstage,
+                              const float *xs, RouteSmem &sm, int t0, int nt, int pass, int &chunk) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+    const int d = p.d, G = gridDim.x, c = blockIdx.x;
+    const long long U = (long long)p.E * d / 16;
+    long long u0, u1;
+    router_slice(p, u0, u1);
+    const int row_base = (int)(u0 * 16 / d);
+    const int nrows = u1 > u0 ? (int)((u1 * 16 - 1) / d) - row_base + 1 : 0;
+    const int nch = (int)((u1 - u0 + 255) / 256);
+    for (int i = tid; i < kRMaxRows * kRouteTok; i += blockDim.x) (&sm.acc[0][0])[i] = 0.f;
+    bool timed_out = false;
+    auto issue = [&](int j, int slot) { router_issue(p, ring, full, u0, u1, j, slot); };
+    // Few rows per slice (the usual case): each thread keeps its own sum per
+    // row of the slice across all stages, and the warps reduce once at the
+    // end.  Otherwise the row sums are reduced and folded stage by stage.
+    const bool fast = nrows <= kRFast;
+    float racc[kRFast][kRouteTok];
 #pragma unroll
-        for (int t = 0; t < kRouteTok; ++t) a0[t] = 0.f;
-        const float4 *wrow = reinterpret_cast<const float4 *>(p.wr + (size_t)r * d);
-        for (int cc = a + lane; cc < b; cc += 32 * 8) {
-            float4 w[8];
+    for (int k = 0; k < kRFast; ++k)
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int ci = cc + 32 * u;
-                w[u] = ci < b ? __ldg(wrow + ci) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+        for (int t = 0; t < kRouteTok; ++t) racc[k][t] = 0.f;
+    __syncthreads();  // the accumulators are cleared
+    for (int j = 0; j < nch; ++j, ++chunk) {
+        const int slot = chunk % nstage;
+        const uint32_t par = (uint32_t)((chunk / nstage) & 1);
+        // bounded; after a timeout the CTA keeps going (its barriers stay in
+        // step) with unused values, the status word says so
+        {
+            // lane 0 polls; the others then take the completed phase themselves
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait_bounded(&full[slot], par, hdr) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (ok && lane != 0) ok = mbar_try_wait(&full[slot], par) ? 1 : 0;
+            if (!ok) timed_out = true;
+        }
+        const long long unit = u0 + 256LL * j + tid;
+        int row = -1;
+        float v[kRouteTok];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int ci = cc + 32 * u;
-                if (ci < b) {
+        for (int t = 0; t < kRouteTok; ++t) v[t] = 0.f;
+        if (unit < u1) {
+            const uint32_t f = (uint32_t)unit * 16u;  // E*d < 2^31 floats
+            row = (int)(f / (uint32_t)d);
+            const int col = (int)(f - (uint32_t)row * (uint32_t)d);
+            const float4 *w4 = reinterpret_cast<const float4 *>(ring + (size_t)slot * kRStage) + tid * 4;
 #pragma unroll
-                    for (int t = 0; t < kRouteTok; ++t) {
-                        if (t < nt) {
-                            const float4 xv = *reinterpret_cast<const float4 *>(xs + t * d + 4 * ci);
-                            a0[t] = fmaf(w[u].x, xv.x, a0[t]);
-                            a0[t] = fmaf(w[u].y, xv.y, a0[t]);
-                            a0[t] = fmaf(w[u].z, xv.z, a0[t]);
-                            a0[t] = fmaf(w[u].w, xv.w, a0[t]);
-                        }
+            for (int q = 0; q < 4; ++q) {
+                const float4 w = w4[q];
+#pragma unroll
+                for (int t = 0; t < kRouteTok; ++t) {
+                    if (t < nt) {
+                        const float4 xv = *reinterpret_cast<const float4 *>(xs + t * d + col + 4 * q);
+                        v[t] = fmaf(w.x, xv.x, v[t]);
+                        v[t] = fmaf(w.y, xv.y, v[t]);
+                        v[t] = fmaf(w.z, xv.z, v[t]);
+                        v[t] = fmaf(w.w, xv.w, v[t]);
                     }
                 }
             }
         }
+        if (fast) {
+            if (row >= 0) {
+                const int k = row - row_base;
 #pragma unroll
-        for (int t = 0; t < kRouteTok; ++t)
-            if (t < nt)
+                for (int kk = 0; kk < kRFast; ++kk)
+                    if (kk == k)
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) a0[t] += __shfl_xor_sync(0xffffffffu, a0[t], o);
-        if (a == 0 && b == cpr) {
-            if (lane == 0) {
-                finalize_row(p, r, t0, nt, a0);
-                ++finished;
+                        for (int t = 0; t < kRouteTok; ++t) racc[kk][t] += v[t];
             }
-        } else if (lane == 0) {
-            // the row is split between warps: park the partial; the last to
-            // arrive sums all parts in slot order and finishes the row
-            const long long rs = (long long)r * cpr;
-            const int first = chunk_owner(rs, N, W);
-            const int nseg = chunk_owner(rs + cpr - 1, N, W) - first + 1;
-            const int slot = j - first;
-            float *pp = part + (((size_t)(pass & 1) * p.E + r) * kMaxSeg) * kRouteTok;
-            uint32_t *pc = cnt + (size_t)(pass & 1) * p.E + r;
+            if (j + nstage < nch) {
+                __syncthreads();  // every thread is done with this stage: refill it
+                if (tid == 0) issue(j + nstage, slot);
+            }
+            continue;
+        }
+        // segmented sum over lanes of equal row (rows do not decrease along lanes)
 #pragma unroll
-            for (int t = 0; t < kRouteTok; ++t) pp[slot * kRouteTok + t] = a0[t];
-            const uint32_t old = atom_add_acq_rel(pc, 1u);  // publish the part, see the others
-            if (old == (uint32_t)(nseg - 1)) {
-                float s0[kRouteTok];
+        for (int o = 1; o < 32; o <<= 1) {
+            const int rn = __shfl_down_sync(0xffffffffu, row, o);
 #pragma unroll
-                for (int t = 0; t < kRouteTok; ++t) s0[t] = 0.f;
-                for (int sl = 0; sl < nseg; ++sl)
-#pragma unroll
-                    for (int t = 0; t < kRouteTok; ++t) s0[t] += __ldcg(pp + sl * kRouteTok + t);
-                *pc = 0u;
-                finalize_row(p, r, t0, nt, s0);
-                ++finished;
+            for (int t = 0; t < kRouteTok; ++t) {
+                const float vn = __shfl_down_sync(0xffffffffu, v[t], o);
+                if (lane + o < 32 && rn == row) v[t] += vn;
             }
         }
-        c += b - a;
+        const int rprev = __shfl_up_sync(0xffffffffu, row, 1);
+        const bool head = row >= 0 && (lane == 0 || rprev != row);
+        const uint32_t heads = __ballot_sync(0xffffffffu, head);
+        const int b = j & 1;
+        if (head) {
+            const int k = __popc(heads & ((1u << lane) - 1u));
+            sm.seg_row[b][warp][k] = row;
+#pragma unroll
+            for (int t = 0; t < kRouteTok; ++t) sm.seg_val[b][warp][k][t] = v[t];
+        }
+        if (lane == 0) sm.seg_n[b][warp] = __popc(heads);
+        __syncthreads();  // this stage is read and its row sums posted
+        if (tid == 0 && j + nstage < nch) issue(j + nstage, slot);
+        if (tid < nrows) {
+            const int r = row_base + tid;
+            for (int w = 0; w < 8; ++w)
+                for (int k = 0; k < sm.seg_n[b][w]; ++k)
+                    if (sm.seg_row[b][w][k] == r)
+#pragma unroll
+                        for (int t = 0; t < kRouteTok; ++t) sm.acc[tid][t] += sm.seg_val[b][w][k][t];
+        }
     }
-    return finished;
+    if (fast) {
+        // per row: the warp's sum (fixed butterfly), then the warps in order
+#pragma unroll
+        for (int k = 0; k < kRFast; ++k) {
+            if (k < nrows) {
+#pragma unroll
+                for (int t = 0; t < kRouteTok; ++t) {
+                    if (t < nt) {
+                        float v = racc[k][t];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                        if (lane == 0) sm.seg_val[0][warp][k][t] = v;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (tid < nrows)
+            for (int w = 0; w < 8; ++w)
+#pragma unroll
+                for (int t = 0; t < kRouteTok; ++t)
+                    if (t < nt) sm.acc[tid][t] += sm.seg_val[0][w][tid][t];
+    }
+    __syncthreads();  // every fold is done
+    if (timed_out && tid == 0) {
+        // copies may still be in flight: let them land (bounded) first
+        const uint64_t tw = globaltimer();
+        while (globaltimer() - tw < 200000ull) {
+        }
+    }
+    if (tid < nrows) {
+        const int r = row_base + tid;
+        const long long rs = (long long)r * d / 16, re = (long long)(r + 1) * d / 16;  // its units
+        float *logits = reinterpret_cast<float *>(p.ws + p.L.logits);
+        const float bias = p.bias ? p.bias[r] : 0.f;
+        bool done = false;
+        float out[kRouteTok];
+        if (rs >= u0 && re <= u1) {
+#pragma unroll
+            for (int t = 0; t < kRouteTok; ++t) out[t] = sm.acc[tid][t];
+            done = true;
+        } else {
+            // cut by a CTA boundary: park this CTA's part; the last to arrive
+            // sums the parts in CTA order
+            const int first = chunk_owner(rs, U, G);
+            const int nseg = chunk_owner(re - 1, U, G) - first + 1;
+            float *pp = reinterpret_cast<float *>(p.ws + p.L.part) + (((size_t)(pass & 1) * p.E + r) * kMaxSeg) * kRouteTok;
+            uint32_t *pc = reinterpret_cast<uint32_t *>(p.ws + p.L.cnt) + (size_t)(pass & 1) * p.E + r;
+#pragma unroll
+            for (int t = 0; t < kRouteTok; ++t) pp[(c - first) * kRouteTok + t] = sm.acc[tid][t];
+            const uint32_t old = atom_add_acq_rel(pc, 1u);
+            if (old == (uint32_t)(nseg - 1)) {
+#pragma unroll
+                for (int t = 0; t < kRouteTok; ++t) out[t] = 0.f;
+                for (int sl = 0; sl < nseg; ++sl)
+#pragma unroll
+                    for (int t = 0; t < kRouteTok; ++t) out[t] += __ldcg(pp + sl * kRouteTok + t);
+                *pc = 0u;
+                done = true;
+            }
+        }
+        if (done) {
+            for (int t = 0; t < nt; ++t) logits[(size_t)(t0 + t) * p.E + r] = out[t] + bias;
+            red_add_release(&hdr->router_done, 1u);  // after this thread's logit stores
+        }
+    }
 }
 
 // Wait (bounded) until *ctr reaches target; false (timeout bit set) if not.
@@ -327,38 +504,83 @@ __device__ bool wait_count(const uint32_t *ctr, uint32_t target, WsHeader *hdr) 
     return true;
 }
 
-// Cooperative launch (every CTA resident).  CTAs 1.. stream the router rows;
-// once all rows are in, token t's top-k runs on CTA t mod G (all its warps),
-// and CTA 0, after its own tokens, waits for the others' and dispatches.
-// Meanwhile the streaming CTAs build the gate/up pass's activation pieces and
-// every expert's tensor maps, which need no routing.
-__global__ void __launch_bounds__(kRouteThreads, 3) route_kernel(const __grid_constant__ RouteParams p) {
-    extern __shared__ __align__(16) float xs[];  // [kRouteTok][d]
+// Cooperative launch (every CTA resident), one CTA per SM.  Every CTA
+// streams its slice of the router; once all rows are in, token t's top-k runs
+// on CTA t mod G (all its warps), and CTA 0, after its own tokens, waits for
+// the others' and dispatches.  Meanwhile CTAs 1.. (CTA 0 when it is alone)
+// build the gate/up pass's activation pieces and every expert's tensor maps,
+// which need no routing.
+__global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_constant__ RouteParams p) {
+    extern __shared__ __align__(128) uint8_t rsm[];
+    const int nstage = p.nstage;
+    const int ntmax = min(p.Tc, kRouteTok);
+    uint8_t *ring = rsm;
+    float *xs = reinterpret_cast<float *>(rsm + (size_t)nstage * kRStage);  // [ntmax][d]
+    RouteSmem &sm = *reinterpret_cast<RouteSmem *>(xs + (size_t)ntmax * p.d);
+    uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(&sm) + sizeof(RouteSmem));
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + p.L.hdr);
     __shared__ int s_ok;
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < nstage; ++st) mbar_init(&full[st], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
     pdl_trigger();
     const int npass = (p.Tc + kRouteTok - 1) / kRouteTok;
     const int G = gridDim.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (blockIdx.x > 0) {
-        const int j = (blockIdx.x - 1) * (kRouteThreads / 32) + warp;
-        const int d = p.d;
-        for (int pass = 0; pass < npass; ++pass) {
-            const int t0 = pass * kRouteTok;
-            const int nt = min(kRouteTok, p.Tc - t0);
-            __syncthreads();
-            for (int i = threadIdx.x; i < nt * d / 2; i += blockDim.x) {
-                const int t = (2 * i) / d, c = (2 * i) % d;
-                const uint32_t w = reinterpret_cast<const uint32_t *>(p.x + (size_t)(t0 + t) * d)[c / 2];
-                xs[t * d + c] = bf16_lo(w);
-                xs[t * d + c + 1] = bf16_hi(w);
+    const int warp = threadIdx.x >> 5;
+    int chunk = 0;
+    if (threadIdx.x == 0) router_prefetch(p, ring, full, nstage, 0);  // pass 0's first stages
+    if (p.blobs != nullptr) {
+        // Tensor maps hold only plane addresses: an expert's maps are rewritten
+        // only when its blob pointer differs from the one they were written for
+        // (kept in the workspace), by threads spread over every CTA, while the
+        // first router stages are in flight.
+        const uint8_t **cache = reinterpret_cast<const uint8_t **>(p.ws + p.L.tcache);
+        for (int e = blockIdx.x * kRouteThreads + threadIdx.x; e < p.E + 1; e += G * kRouteThreads) {
+            if (e < p.E) {
+                const uint8_t *b = p.blobs[e];
+                if (b != cache[e] && b != nullptr && (reinterpret_cast<uintptr_t>(b) & 15u) == 0u) {
+                    write_expert_tmaps(p.ws, p.L, e, b, p.tmpl, p.scale_mask);
+                    cache[e] = b;
+                }
+            } else if (p.has_shared) {
+                if (cache[p.E] != p.sw[0] || cache[p.E + 1] != p.sw[1] || cache[p.E + 2] != p.sw[2]) {
+                    write_shared_tmaps(p.ws, p.L, p.smap);
+                    cache[p.E] = p.sw[0];
+                    cache[p.E + 1] = p.sw[1];
+                    cache[p.E + 2] = p.sw[2];
+                }
             }
-            __syncthreads();
-            const int nr = stream_router(p, xs, t0, nt, pass, j, lane);
-            // one release per warp: its logits are visible before they are counted
-            if (lane == 0 && nr > 0) red_add_release(&hdr->router_done, (uint32_t)nr);
         }
     }
+    for (int pass = 0; pass < npass; ++pass) {
+        const int t0 = pass * kRouteTok;
+        const int nt = min(kRouteTok, p.Tc - t0);
+        __syncthreads();  // the previous pass no longer reads xs or the ring
+        if (pass > 0 && threadIdx.x == 0) router_prefetch(p, ring, full, nstage, chunk);
+        // x of these tokens as fp32: 16-byte loads, several in flight per thread
+        const uint4 *xv = reinterpret_cast<const uint4 *>(p.x + (size_t)t0 * p.d);
+        const int n8 = nt * p.d / 8;
+#pragma unroll 4
+        for (int i = threadIdx.x; i < n8; i += blockDim.x) {
+            const uint4 w = __ldg(xv + i);
+            float4 *o = reinterpret_cast<float4 *>(xs + 8 * i);
+            o[0] = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+            o[1] = make_float4(bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w));
+        }
+        __syncthreads();
+        stream_router(p, hdr, ring, full, nstage, xs, sm, t0, nt, pass, chunk);
+    }
+    // work of the gate/up pass that needs no routing (before the top-k wait
+    // on a lone CTA, after it elsewhere is not needed: other CTAs do it)
+    auto prep = [&](int first_cta) {
+        if (p.blobs == nullptr) return;
+        const int nworkers = G - first_cta;
+        const int wi = (blockIdx.x - first_cta) * (kRouteThreads / 32) + warp;
+        build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L, wi, nworkers * (kRouteThreads / 32), p.has_shared != 0);
+    };
+    if (G == 1) prep(0);
     // top-k of this CTA's tokens once every router row is in
     if ((int)blockIdx.x < p.Tc) {
         __syncthreads();
@@ -389,20 +611,8 @@ __global__ void __launch_bounds__(kRouteThreads, 3) route_kernel(const __grid_co
         }
         return;
     }
-    if (p.blobs == nullptr) return;
-    // work of the gate/up pass that needs no routing
-    const int j = (blockIdx.x - 1) * (kRouteThreads / 32) + warp;
-    build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L, j, p.nwarps, p.has_shared != 0);
-    const int tid = (blockIdx.x - 1) * kRouteThreads + threadIdx.x;
-    for (int e = tid; e < p.E; e += (G - 1) * kRouteThreads) {
-        const uint8_t *b = p.blobs[e];
-        if (b != nullptr && (reinterpret_cast<uintptr_t>(b) & 15u) == 0u) write_expert_tmaps(p.ws, p.L, e, b, p.tmpl, p.scale_mask);
-    }
-    if (tid == 0 && p.has_shared) write_shared_tmaps(p.ws, p.L, p.smap);
+    prep(1);
 }
-
-// ======================================================= single expert ==
-// Dispatch for k3moe_expert_ffn: one expert, every token of the chunk, weight 1.
 
 struct SingleParams {
     const uint16_t *x;
@@ -428,7 +638,11 @@ __global__ void single_expert_setup_kernel(const __grid_constant__ SingleParams 
             reinterpret_cast<const uint8_t **>(p.ws + p.L.uniq_blob)[0] = b;
             reinterpret_cast<int32_t *>(p.ws + p.L.uniq_eid)[0] = 0;
             reinterpret_cast<uint32_t *>(p.ws + p.L.uniq_mask)[0] = (1u << p.Tc) - 1u;
-            if (b != nullptr) write_expert_tmaps(p.ws, p.L, 0, b, p.tmpl, p.scale_mask);
+            if (b != nullptr) {
+                // slot 0's maps now hold this blob (the layer's map cache sees it)
+                write_expert_tmaps(p.ws, p.L, 0, b, p.tmpl, p.scale_mask);
+                reinterpret_cast<const uint8_t **>(p.ws + p.L.tcache)[0] = b;
+            }
         }
         if (threadIdx.x < kChunk) {
             const int t = threadIdx.x;

@@ -31,11 +31,10 @@ static __device__ __align__(256) uint8_t g_noalloc_ws[kNoAllocBytes];
 
 struct DeviceInfo {
     bool ready = false;
+    int route_dyn_max = 0;       // dynamic smem the route kernel may take beside its static arrays
     uint8_t *noalloc = nullptr;  // device address of g_noalloc_ws on this device, once set up
     int noalloc_shape[5] = {0, 0, 0, 0, 0};  // (d, ff, E, k, ff_shared) its layout was last used for
     int sms = 0;
-    int route_smem = -1;  // dynamic smem of the last occupancy query
-    int route_occ = 0;    // resident route_shared CTAs per SM at that size
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -64,7 +63,12 @@ k3moe_status device_info(DeviceInfo **out) {
         e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return cuda_fail(e);
         const int big = kSmemLimit;
-        cudaError_t r = set_smem(route_kernel, kRouteTok * 8192 * 4);
+        cudaFuncAttributes fa;
+        cudaError_t r = cudaFuncGetAttributes(&fa, route_kernel);
+        if (r == cudaSuccess) {
+            di.route_dyn_max = big - (int)fa.sharedSizeBytes;
+            r = set_smem(route_kernel, di.route_dyn_max);
+        }
         if (r == cudaSuccess) r = set_smem(umma_expert_kernel<true>, big);
         if (r == cudaSuccess) r = set_smem(umma_expert_kernel<false>, big);
         if (r != cudaSuccess) return cuda_fail(r);
@@ -245,28 +249,22 @@ cudaError_t launch_umma(const DeviceInfo &di, UmmaParams up, cudaStream_t st) {
 // Router (+ top-k + dispatch + activation pieces) for one chunk.  Cooperative
 // launch: CTA 0 waits on the other CTAs' router rows, so all must be resident.
 cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st) {
+    // one CTA per SM, at most one per router row and one per stage of router
+    // bytes; as many ring stages as fit beside x (12 at most)
     const int nt = rp.Tc < kRouteTok ? rp.Tc : kRouteTok;
-    const int smem = nt * rp.d * 4;
-    if (di.route_smem != smem) {
-        int occ = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, route_kernel,
-                                                                       kRouteThreads, smem);
-        if (e != cudaSuccess) return e;
-        di.route_occ = occ;
-        di.route_smem = smem;
-    }
-    const int per_sm = di.route_occ < 3 ? di.route_occ : 3;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    int gs = per_sm * di.sms - 1;  // streaming CTAs
-    // every streaming warp takes at least a quarter row, so a row is split
-    // between at most 5 warps (kMaxSeg slots)
-    const int wmax = rp.E * 4;
-    if (gs * 8 > wmax) gs = wmax / 8 > 0 ? wmax / 8 : 1;
-    rp.nwarps = gs * 8;
+    const long long bytes = (long long)rp.E * rp.d * 4;
+    long long g = (bytes + kRStage - 1) / kRStage;
+    if (g > di.sms) g = di.sms;
+    if (g > rp.E) g = rp.E;
+    if (g < 1) g = 1;
+    int nstage = 12;
+    while (nstage > 2 && route_smem_bytes(rp.d, nt, nstage) > di.route_dyn_max) --nstage;
+    if (route_smem_bytes(rp.d, nt, nstage) > di.route_dyn_max) return cudaErrorInvalidConfiguration;
+    rp.nstage = nstage;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(gs + 1);
+    cfg.gridDim = dim3((unsigned)g);
     cfg.blockDim = dim3(kRouteThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = route_smem_bytes(rp.d, nt, nstage);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
@@ -367,6 +365,9 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         rp.scale_mask = (d % 512 == 0 ? 1 : 0) | (dims->ff % 512 == 0 ? 2 : 0);
         memcpy(rp.smap, smap, sizeof(smap));
         rp.has_shared = ffs > 0;
+        rp.sw[0] = reinterpret_cast<const uint8_t *>(shared_wg);
+        rp.sw[1] = reinterpret_cast<const uint8_t *>(shared_wu);
+        rp.sw[2] = reinterpret_cast<const uint8_t *>(shared_wd);
         EventHook none;
         EventHook &hk = hook ? *hook : none;
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
@@ -493,7 +494,7 @@ k3moe_status k3moe_expert_ffn(const void *x, int32_t T, const uint8_t *blob,
     DeviceInfo *di = nullptr;
     s = device_info(&di);
     if (s != K3MOE_OK) return s;
-    const Layout L = layout_for(dims, 1);  // one slot per token, weight 1
+    const Layout L = layout_for(dims, dims->top_k);  // the layer's layout: one workspace serves every call
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
     const int d = dims->d;
@@ -522,7 +523,7 @@ k3moe_status k3moe_expert_ffn(const void *x, int32_t T, const uint8_t *blob,
         up.Tc = Tc;
         up.d = d;
         up.ff = dims->ff;
-        up.k = 1;
+        up.k = dims->top_k;
         up.ffs = 0;
         up.ws = wsb;
         up.L = L;

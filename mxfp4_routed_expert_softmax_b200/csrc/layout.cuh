@@ -38,6 +38,7 @@ struct Layout {
     size_t tmap;       // 128-byte tensor maps [E][6]: W_g, W_u, W_d nibble planes and their
                        // scale planes, of each expert; then the shared expert's W_g, W_u,
                        // W_d (bf16) at [E*6 ..]
+    size_t tcache;     // u64 [E+3] the blob (and shared-expert) pointers the maps were written for
     size_t xb;         // u8  [nkt_d][N*128] E2M1 pieces of x (gate/up B operand)
     size_t xsf;        // u32 [nkt_d][2][kSfRow] their E8M0 scales (byte = block in group)
     size_t hb;         // u8  [umax][nkt_ff][N*128] pieces of w*h (down B operand)
@@ -84,6 +85,8 @@ __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int f
     L.umax = umax;
     L.tmap = o;
     o = align256(o + ((size_t)E * 6 + 3) * 128);
+    L.tcache = o;
+    o = align256(o + ((size_t)E + 3) * 8);
     L.xb = o;
     o = align256(o + (size_t)nkt_d * kNMax * 128);
     L.xsf = o;
