@@ -76,6 +76,30 @@ def route_bytes(cfg):
     return cfg.E * cfg.d * 4 + cfg.T * cfg.d * 2
 
 
+def captured_traffic(cfg):
+    """DRAM bytes (read + write) of one gate/up launch from the committed ncu
+    summary, while the kernel sources still hash to the captured ones and the
+    launch moves the same bytes (d, ff, k, shared ff, T and 16 distinct
+    experts); otherwise None."""
+    import hashlib
+    here = os.path.dirname(os.path.abspath(__file__))
+    try:
+        text = open(os.path.join(here, "profiles", "expert_gu_k3_decode_e64.md")).read()
+    except OSError:
+        return None
+    fields = dict(line.split(": ", 1) for line in text.splitlines()
+                  if line.startswith(("traffic_bytes_per_launch: ", "source_sha256: ")))
+    src = os.path.join(here, "mxfp4_routed_expert_softmax_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("umma_kernels.cuh", "umma.cuh", "common.cuh", "layout.cuh"):
+        h.update(open(os.path.join(src, f), "rb").read())
+    if fields.get("source_sha256", "").strip() != h.hexdigest():
+        return None
+    if (cfg.d, cfg.ff, cfg.k, cfg.ff_shared, cfg.T) != (7168, 1536, 16, 1536, 1):
+        return None
+    return int(fields["traffic_bytes_per_launch"])
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -322,7 +346,8 @@ def main():
                     "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 4),
                     "peak_kind": f"{peak_kind} (burst copy, MEASURED_PEAKS.json hbm_gbs)"
                     if peak_kind == "measured" else "fallback 6.65 TB/s",
-                    "traffic": None, "alg_bytes_per_launch": gb}
+                    "traffic": captured_traffic(cfg) if U == 16 else None,
+                    "alg_bytes_per_launch": gb}
     layer_gbs = alg_bytes(cfg, U) / (ms_per_step / 1000.0) / 1e9
 
     # end to end: host activations in and out through the C ABI, copies timed
