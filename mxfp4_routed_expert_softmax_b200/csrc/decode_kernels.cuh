@@ -72,15 +72,14 @@ __device__ __forceinline__ uint32_t block_scan_incl(uint32_t v, uint32_t *s_tot)
 // K exactly; every key above K is taken, and of the keys equal to K the
 // lowest indices (a prefix count in index order).  The k winners are then
 // ranked by (key descending, index ascending) for the output order.
-__device__ void cta_topk(const RouteParams &p, int t) {
+__device__ void cta_topk_row(const float *row, int E, int k, int32_t *idx_row, float *w_row, int32_t *idx_out_row,
+                             float *w_out_row) {
     __shared__ uint32_t s_hist[256];
     __shared__ uint32_t s_tot[8];
     __shared__ float s_red[2][8];
     __shared__ uint32_t s_pref, s_need, s_cnt;
     __shared__ uint32_t s_selk[32], s_seli[32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int E = p.E, k = p.k;
-    const float *row = reinterpret_cast<const float *>(p.ws + p.L.logits) + (size_t)t * E;
     float v[4];
     uint32_t key[4];
     bool ok[4];
@@ -184,11 +183,18 @@ __device__ void cta_topk(const RouteParams &p, int t) {
             r += (qk > mk || (qk == mk && qi < mi)) ? 1 : 0;
         }
         const float w = expf(fkey_value(mk) - m) * inv_s;
-        reinterpret_cast<int32_t *>(p.ws + p.L.idx)[t * k + r] = (int32_t)mi;
-        reinterpret_cast<float *>(p.ws + p.L.wt)[t * k + r] = w;
-        if (p.idx_out) p.idx_out[(size_t)t * k + r] = (int32_t)mi;
-        if (p.w_out) p.w_out[(size_t)t * k + r] = w;
+        idx_row[r] = (int32_t)mi;
+        w_row[r] = w;
+        if (idx_out_row) idx_out_row[r] = (int32_t)mi;
+        if (w_out_row) w_out_row[r] = w;
     }
+}
+// Token t of a decode chunk: logits, picks and weights in the workspace.
+__device__ void cta_topk(const RouteParams &p, int t) {
+    const int k = p.k;
+    cta_topk_row(reinterpret_cast<const float *>(p.ws + p.L.logits) + (size_t)t * p.E, p.E, k,
+                 reinterpret_cast<int32_t *>(p.ws + p.L.idx) + t * k, reinterpret_cast<float *>(p.ws + p.L.wt) + t * k,
+                 p.idx_out ? p.idx_out + (size_t)t * k : nullptr, p.w_out ? p.w_out + (size_t)t * k : nullptr);
 }
 
 // The dispatch of a chunk whose top-k is done: distinct experts in ascending
@@ -249,6 +255,30 @@ __device__ void dispatch(const RouteParams &p, WsHeader *hdr) {
             ublob[u] = b;
             ueid[u] = w;
             gmask[u] = umask[u];
+        }
+    }
+}
+
+// Tensor maps hold only plane addresses: an expert's maps are rewritten only
+// when its blob pointer differs from the one they were written for (kept in
+// the workspace).  Thread i of n takes experts i, i + n, ...; index E is the
+// shared expert.
+__device__ void refresh_tmaps(const RouteParams &p, int i0, int n) {
+    const uint8_t **cache = reinterpret_cast<const uint8_t **>(p.ws + p.L.tcache);
+    for (int e = i0; e < p.E + 1; e += n) {
+        if (e < p.E) {
+            const uint8_t *b = p.blobs[e];
+            if (b != cache[e] && b != nullptr && (reinterpret_cast<uintptr_t>(b) & 15u) == 0u) {
+                write_expert_tmaps(p.ws, p.L, e, b, p.tmpl, p.scale_mask);
+                cache[e] = b;
+            }
+        } else if (p.has_shared) {
+            if (cache[p.E] != p.sw[0] || cache[p.E + 1] != p.sw[1] || cache[p.E + 2] != p.sw[2]) {
+                write_shared_tmaps(p.ws, p.L, p.smap);
+                cache[p.E] = p.sw[0];
+                cache[p.E + 1] = p.sw[1];
+                cache[p.E + 2] = p.sw[2];
+            }
         }
     }
 }
@@ -531,29 +561,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
     const int warp = threadIdx.x >> 5;
     int chunk = 0;
     if (threadIdx.x == 0) router_prefetch(p, ring, full, nstage, 0);  // pass 0's first stages
-    if (p.blobs != nullptr) {
-        // Tensor maps hold only plane addresses: an expert's maps are rewritten
-        // only when its blob pointer differs from the one they were written for
-        // (kept in the workspace), by threads spread over every CTA, while the
-        // first router stages are in flight.
-        const uint8_t **cache = reinterpret_cast<const uint8_t **>(p.ws + p.L.tcache);
-        for (int e = blockIdx.x * kRouteThreads + threadIdx.x; e < p.E + 1; e += G * kRouteThreads) {
-            if (e < p.E) {
-                const uint8_t *b = p.blobs[e];
-                if (b != cache[e] && b != nullptr && (reinterpret_cast<uintptr_t>(b) & 15u) == 0u) {
-                    write_expert_tmaps(p.ws, p.L, e, b, p.tmpl, p.scale_mask);
-                    cache[e] = b;
-                }
-            } else if (p.has_shared) {
-                if (cache[p.E] != p.sw[0] || cache[p.E + 1] != p.sw[1] || cache[p.E + 2] != p.sw[2]) {
-                    write_shared_tmaps(p.ws, p.L, p.smap);
-                    cache[p.E] = p.sw[0];
-                    cache[p.E + 1] = p.sw[1];
-                    cache[p.E + 2] = p.sw[2];
-                }
-            }
-        }
-    }
+    // while the first router stages are in flight
+    if (p.blobs != nullptr) refresh_tmaps(p, blockIdx.x * kRouteThreads + threadIdx.x, G * kRouteThreads);
     for (int pass = 0; pass < npass; ++pass) {
         const int t0 = pass * kRouteTok;
         const int nt = min(kRouteTok, p.Tc - t0);

@@ -14,6 +14,7 @@
 #include "decode_kernels.cuh"
 #include "k3moe.h"
 #include "layout.cuh"
+#include "prefill_kernels.cuh"
 
 namespace {
 
@@ -69,8 +70,10 @@ k3moe_status device_info(DeviceInfo **out) {
             di.route_dyn_max = big - (int)fa.sharedSizeBytes;
             r = set_smem(route_kernel, di.route_dyn_max);
         }
-        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<true>, big);
-        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<false>, big);
+        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<true, false>, big);
+        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<false, false>, big);
+        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<true, true>, big);
+        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<false, true>, big);
         if (r != cudaSuccess) return cuda_fail(r);
         di.ready = true;
     }
@@ -109,8 +112,55 @@ Layout layout_for(const k3moe_dims *dm, int k_eff) {
     return make_layout(dm->d, dm->ff, dm->n_experts, k_eff, dm->ff_shared);
 }
 
-size_t staging_bytes(const k3moe_dims *dm) {
-    return align256((size_t)kChunk * dm->d * 2) + align256((size_t)kChunk * dm->d * 4);
+// ---------------------------------------------------------- prefill pass --
+// The grouped prefill kernels run on a fixed grid; a pass takes as many
+// tokens (up to kPfMaxTokens) as keep every CTA's share of groups within its
+// shared-memory table (a bound over the worst case of the routing).
+constexpr int kPfCtas = 148;
+
+int pf_groups_per_cta_bound(const k3moe_dims *dm, int Tp) {
+    const int d = dm->d, ff = dm->ff, E = dm->n_experts, k = dm->top_k;
+    const int ffs = (dm->flags & K3MOE_NO_SHARED) ? 0 : dm->ff_shared;
+    const long long ngr = pf_routed_groups_max(Tp, E, k), ngs = ffs > 0 ? ceil_div(Tp, kGroup) : 0;
+    int worst = 0;
+    for (int gu = 0; gu < 2; ++gu) {
+        const long long upr = gu ? (long long)ceil_div(ff, kTileM) * ceil_div(d, kTileK)
+                                 : (long long)ceil_div(d, kTileM) * ceil_div(ff, kTileK);
+        const long long ups = ffs == 0 ? 0
+                              : gu ? (long long)ceil_div(ffs, kTileM) * ceil_div(d, kTileKs)
+                                   : (long long)ceil_div(d, kTileM) * ceil_div(ffs, kTileKs);
+        const long long total = ngr * upr + ngs * ups;
+        const long long per = (total + kPfCtas - 1) / kPfCtas;
+        const long long mn = ups > 0 && ups < upr ? ups : upr;
+        const long long g = (per + mn - 1) / mn + 1;
+        if (g > worst) worst = (int)(g > (1 << 30) ? (1 << 30) : g);
+    }
+    return worst;
+}
+
+int pf_pass_tokens(const k3moe_dims *dm, int T) {
+    int Tp = T < kPfMaxTokens ? T : kPfMaxTokens;
+    while (Tp > kChunk && pf_groups_per_cta_bound(dm, Tp) > kPfMetaG) Tp -= kGroup;
+    return Tp;
+}
+
+PLayout playout_for(const k3moe_dims *dm, int Tp) {
+    const Layout L = layout_for(dm, dm->top_k);
+    const int ffs = (dm->flags & K3MOE_NO_SHARED) ? 0 : dm->ff_shared;
+    return make_playout(L.total, dm->d, dm->ff, dm->n_experts, dm->top_k, ffs, Tp);
+}
+
+// Scratch for a call of T tokens on the grouped prefill path (0: T is one chunk).
+size_t pf_need(const k3moe_dims *dm, int T) {
+    if (T <= kChunk) return 0;
+    const int Tp = pf_pass_tokens(dm, T);
+    if (Tp <= kChunk) return 0;
+    return playout_for(dm, Tp).total;
+}
+
+size_t staging_bytes(const k3moe_dims *dm, int T) {
+    const size_t n = T > kChunk ? (size_t)T : (size_t)kChunk;
+    return align256(n * dm->d * 2) + align256(n * dm->d * 4);
 }
 
 template <typename Kern, typename P>
@@ -236,13 +286,14 @@ k3moe_status shared_tmaps(int d, int ffs, const void *wg, const void *wu, const 
 
 template <bool GU>
 cudaError_t launch_umma(const DeviceInfo &di, UmmaParams up, cudaStream_t st) {
+    up.ngs = 0;
     const int N = act_n(up.Tc);
     up.nst = umma_stages(GU, N);
     up.sb = umma_stage_bytes(GU, N);
     up.sf_tma = (GU ? up.d : up.ff) % 512 == 0;
     const int smem = umma_smem_bytes(GU, N, up.nst);
     const int g = di.sms < kMaxCtas ? di.sms : kMaxCtas;
-    return launch(umma_expert_kernel<GU>, dim3(g), dim3(kUThreads), smem, st, true, up);
+    return launch(umma_expert_kernel<GU, false>, dim3(g), dim3(kUThreads), smem, st, true, up);
 }
 
 
@@ -272,6 +323,99 @@ cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, route_kernel, rp);
+}
+
+// Launches of the grouped prefill, pass after pass; rp carries the shapes,
+// blobs and tensor-map templates.  routing_only: stop after the top-k.
+k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims, const uint16_t *x, int T,
+                          void *y, int32_t *idx_out, float *w_out, cudaStream_t st, bool routing_only = false) {
+    const int d = dims->d, E = dims->n_experts, k = dims->top_k;
+    const int ffs = rp.has_shared ? dims->ff_shared : 0;
+    const bool out32 = (dims->flags & K3MOE_OUT_FP32) != 0;
+    const int Tp = pf_pass_tokens(dims, T);
+    const PLayout P = playout_for(dims, Tp);
+    uint8_t *wsb = rp.ws;
+    cudaError_t e;
+    for (int t0 = 0; t0 < T; t0 += Tp) {
+        const int Tq = (T - t0) < Tp ? (T - t0) : Tp;
+        PfRouteParams pp{};
+        pp.r = rp;
+        pp.r.x = x + (size_t)t0 * d;
+        pp.r.Tc = Tq;
+        pp.r.idx_out = idx_out ? idx_out + (size_t)t0 * k : nullptr;
+        pp.r.w_out = w_out ? w_out + (size_t)t0 * k : nullptr;
+        pp.P = P;
+        pp.T = Tq;
+        pp.ngs = ffs > 0 ? ceil_div(Tq, kGroup) : 0;
+        // router: split K until the grid covers the GPU twice; the split
+        // partials go where the expert outputs go later (not in use yet)
+        PfRouterParams rr{};
+        rr.x = pp.r.x;
+        rr.wr = rp.wr;
+        rr.bias = rp.bias;
+        rr.T = Tq;
+        rr.d = d;
+        rr.E = E;
+        const int gx = ceil_div(E, kPrBM), gy = ceil_div(Tq, kPrBN);
+        int ns = (2 * di.sms + gx * gy - 1) / (gx * gy);
+        if (ns > 8) ns = 8;
+        if (ns > d / 256) ns = d / 256;
+        if (ns < 1) ns = 1;
+        while (ns > 1 && (size_t)ns * Tq * E * 4 > P.icnt - P.o) --ns;
+        rr.nsplit = ns;
+        rr.out = reinterpret_cast<float *>(wsb + (ns > 1 ? P.o : P.lg));
+        e = launch(pf_router_kernel, dim3(gx, gy, ns), dim3(kPrThreads), 0, st, false, rr);
+        if (e != cudaSuccess) return cuda_fail(e, "prefill router launch");
+        if (ns > 1) {
+            const PfRouterSumParams sp{rr.out, ns, rp.bias, Tq, E, reinterpret_cast<float *>(wsb + P.lg)};
+            e = launch(pf_router_sum_kernel, dim3(4 * di.sms), dim3(256), 0, st, false, sp);
+            if (e != cudaSuccess) return cuda_fail(e, "prefill router sum launch");
+        }
+        e = launch(pf_topk_kernel, dim3(Tq), dim3(kRouteThreads), 0, st, false, pp);
+        if (e != cudaSuccess) return cuda_fail(e, "prefill top-k launch");
+        if (routing_only) continue;
+        const int nhb = ceil_div(Tq, kPfHistTok);
+        e = launch(pf_hist_kernel, dim3(nhb), dim3(kRouteThreads), 0, st, false, pp);
+        if (e == cudaSuccess) e = launch(pf_scan_kernel, dim3(1), dim3(kPfScanThreads), 0, st, false, pp);
+        if (e == cudaSuccess) e = launch(pf_place_kernel, dim3(nhb), dim3(kRouteThreads), 0, st, false, pp);
+        if (e == cudaSuccess) e = launch(pf_prep_kernel, dim3(2 * di.sms), dim3(kRouteThreads), 0, st, false, pp);
+        if (e != cudaSuccess) return cuda_fail(e, "prefill dispatch launch");
+        e = cudaMemsetAsync(wsb + P.icnt, 0, P.total - P.icnt, st);
+        if (e != cudaSuccess) return cuda_fail(e, "prefill counters");
+        UmmaParams up{};
+        up.Tc = 0;
+        up.d = d;
+        up.ff = dims->ff;
+        up.k = k;
+        up.ffs = ffs;
+        up.ws = wsb;
+        up.L = rp.L;
+        up.out_fp32 = out32;
+        up.y = nullptr;
+        up.P = P;
+        up.ngs = pp.ngs;
+        up.blobs = rp.blobs;
+        for (int gu = 1; gu >= 0; --gu) {
+            up.nst = umma_stages(gu != 0, kPfN);
+            up.sb = umma_stage_bytes(gu != 0, kPfN);
+            up.sf_tma = (gu ? d : dims->ff) % 512 == 0;
+            const int smem = umma_smem_bytes(gu != 0, kPfN, up.nst);
+            e = gu ? launch(umma_expert_kernel<true, true>, dim3(kPfCtas), dim3(kUThreads), smem, st, true, up)
+                   : launch(umma_expert_kernel<false, true>, dim3(kPfCtas), dim3(kUThreads), smem, st, true, up);
+            if (e != cudaSuccess) return cuda_fail(e, gu ? "prefill gate/up launch" : "prefill down launch");
+        }
+        PfCombineParams cp{};
+        cp.o = reinterpret_cast<const float *>(wsb + P.o);
+        cp.T = Tq;
+        cp.d = d;
+        cp.k = k;
+        cp.has_shared = ffs > 0;
+        cp.out_fp32 = out32;
+        cp.y = reinterpret_cast<uint8_t *>(y) + (size_t)t0 * d * (out32 ? 4 : 2);
+        e = launch(pf_combine_kernel, dim3(4 * di.sms), dim3(256), 0, st, false, cp);
+        if (e != cudaSuccess) return cuda_fail(e, "prefill combine launch");
+    }
+    return K3MOE_OK;
 }
 
 struct EventHook {
@@ -309,7 +453,11 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
     }
     if (!ws || !aligned(ws, 256)) return K3MOE_ERR_INVALID_ARGUMENT;
     const Layout L = layout_for(dims, dims->top_k);
-    const size_t need = L.total + (from_host ? staging_bytes(dims) : 0);
+    // grouped prefill when the workspace holds its region (else 8-token passes)
+    const size_t pfn = hook ? 0 : pf_need(dims, T);
+    const bool grouped = pfn > 0 && ws_bytes >= pfn + (from_host ? staging_bytes(dims, T) : 0);
+    const size_t base = grouped ? pfn : L.total;
+    const size_t need = base + (from_host ? staging_bytes(dims, grouped ? T : kChunk) : 0);
     if (ws_bytes < need) return K3MOE_ERR_WORKSPACE_TOO_SMALL;
     DeviceInfo *di = nullptr;
     s = device_info(&di);
@@ -320,8 +468,8 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
     const int d = dims->d;
     const bool out32 = (dims->flags & K3MOE_OUT_FP32) != 0;
     const size_t ybytes = out32 ? 4 : 2;
-    uint8_t *xstage = wsb + L.total;
-    uint8_t *ystage = xstage + align256((size_t)kChunk * d * 2);
+    uint8_t *xstage = wsb + base;
+    uint8_t *ystage = xstage + align256((size_t)(grouped ? T : kChunk) * d * 2);
 
     uint4 tmpl[4][8];
     s = tmap_templates(d, dims->ff, ws, tmpl);
@@ -331,6 +479,39 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
     if (ffs > 0) {
         s = shared_tmaps(d, ffs, shared_wg, shared_wu, shared_wd, smap);
         if (s != K3MOE_OK) return s;
+    }
+
+    if (grouped) {
+        RouteParams rp{};
+        rp.wr = w_router;
+        rp.bias = bias;
+        rp.d = d;
+        rp.E = dims->n_experts;
+        rp.k = dims->top_k;
+        rp.ws = wsb;
+        rp.L = L;
+        rp.blobs = expert_blobs;
+        memcpy(rp.tmpl, tmpl, sizeof(tmpl));
+        rp.scale_mask = (d % 512 == 0 ? 1 : 0) | (dims->ff % 512 == 0 ? 2 : 0);
+        memcpy(rp.smap, smap, sizeof(smap));
+        rp.has_shared = ffs > 0;
+        rp.sw[0] = reinterpret_cast<const uint8_t *>(shared_wg);
+        rp.sw[1] = reinterpret_cast<const uint8_t *>(shared_wu);
+        rp.sw[2] = reinterpret_cast<const uint8_t *>(shared_wd);
+        cudaError_t e;
+        if (from_host) {
+            e = cudaMemcpyAsync(xstage, x_host, (size_t)T * d * 2, cudaMemcpyHostToDevice, st);
+            if (e != cudaSuccess) return cuda_fail(e);
+            x = xstage;
+            y = ystage;
+        }
+        s = prefill_impl(*di, rp, dims, reinterpret_cast<const uint16_t *>(x), T, y, idx_out, w_out, st);
+        if (s != K3MOE_OK) return s;
+        if (from_host) {
+            e = cudaMemcpyAsync(y_host, ystage, (size_t)T * d * ybytes, cudaMemcpyDeviceToHost, st);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        return K3MOE_OK;
     }
 
     for (int c0 = 0; c0 < T; c0 += kChunk) {
@@ -438,12 +619,13 @@ size_t k3moe_blob_bytes(const k3moe_dims *dims) {
 
 size_t k3moe_workspace_size(const k3moe_dims *dims, int32_t T_max) {
     if (check_dims(dims) != K3MOE_OK || T_max < 1) return 0;
-    return layout_for(dims, dims->top_k).total;
+    const size_t dec = layout_for(dims, dims->top_k).total, pf = pf_need(dims, T_max);
+    return pf > dec ? pf : dec;
 }
 
 size_t k3moe_host_staging_bytes(const k3moe_dims *dims, int32_t T) {
     if (check_dims(dims) != K3MOE_OK || T < 1) return 0;
-    return staging_bytes(dims);
+    return staging_bytes(dims, T);
 }
 
 k3moe_status k3moe_route(const void *x, int32_t T, const float *w_router, const float *bias,
@@ -461,6 +643,19 @@ k3moe_status k3moe_route(const void *x, int32_t T, const float *w_router, const 
     s = device_info(&di);
     if (s != K3MOE_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t pfn = pf_need(dims, T);
+    if (pfn > 0 && ws_bytes >= pfn) {
+        // many tokens: the prefill router (a GEMM over all of them) and top-k
+        RouteParams rp{};
+        rp.wr = w_router;
+        rp.bias = bias;
+        rp.d = dims->d;
+        rp.E = dims->n_experts;
+        rp.k = dims->top_k;
+        rp.ws = reinterpret_cast<uint8_t *>(ws);
+        rp.L = L;
+        return prefill_impl(*di, rp, dims, reinterpret_cast<const uint16_t *>(x), T, nullptr, idx, weight, st, true);
+    }
     for (int c0 = 0; c0 < T; c0 += kChunk) {
         const int Tc = (T - c0) < kChunk ? (T - c0) : kChunk;
         RouteParams rp{};

@@ -54,6 +54,20 @@ def test_sizes(m):
     assert m.k3moe_workspace_size(d, 0) == 0
 
 
+def test_workspace_grows_with_the_grouped_prefill_region(m):
+    """Up to 8 tokens: the decode scratch only; more: plus the grouped prefill
+    region (per-token pieces, groups, per-(token, slot) outputs), which grows
+    with the pass size and stops growing at the pass limit."""
+    d = m.make_dims(7168, 1536, 896, 16, 1536)
+    w8 = m.k3moe_workspace_size(d, 8)
+    assert m.k3moe_workspace_size(d, 1) == w8
+    w9, w512, w4096 = (m.k3moe_workspace_size(d, t) for t in (9, 512, 4096))
+    assert w8 < w9 < w512 < w4096
+    # outputs per (token, slot) dominate: (k+1)*d fp32 per token
+    assert w4096 - w512 > (4096 - 512) * 17 * 7168 * 4
+    assert m.k3moe_workspace_size(d, 8192) == m.k3moe_workspace_size(d, 100000)
+
+
 BIG = 1 << 30
 A16 = 0x10000  # a fake 16-byte aligned address: never dereferenced, calls fail validation first
 

@@ -247,3 +247,78 @@ def test_misaligned_blob_is_reported_not_read():
     # the status is cleared by reading it, and the workspace is usable again
     y2, _, _ = run_layer(cfg, W, inp.x, inp.bias, inp.T, 0)
     assert m.k3moe_device_status(ws) == m.K3MOE_OK
+
+
+# ----------------------------------------------------------- grouped prefill --
+# More than 8 tokens with a workspace sized for them: tokens sorted by expert,
+# groups of up to 8 tokens per tensor-core item, expert outputs summed per
+# token at the end.  Shapes cover both scale paths (reduction length a
+# multiple of 512: scales by TMA; otherwise loaded by the scale warps).
+
+@pytest.mark.parametrize("cfg,T", [
+    (k3gen.Config("pf_tiny", d=256, ff=128, E=32, k=4, ff_shared=128, T=0), 64),
+    (SMALL, 200),
+    (k3gen.Config("pf_k32", d=256, ff=192, E=64, k=32, ff_shared=0, T=0, bias="normal"), 37),
+    (k3gen.Config("pf_skew", d=512, ff=512, E=128, k=6, ff_shared=64, T=0, bias="zipf"), 300),
+])
+def test_grouped_prefill_parity(orc, cfg, T):
+    W = kdev.weights(cfg)
+    inp = kdev.DeviceInputs(cfg, T=T)
+    y32, idx, w = run_layer(cfg, W, inp.x, inp.bias, T, m.K3MOE_OUT_FP32)
+    y16, idx2, _ = run_layer(cfg, W, inp.x, inp.bias, T, 0)
+    assert np.array_equal(idx, idx2)
+    r = torch.from_numpy(y32).to(torch.bfloat16).view(torch.int16).numpy()
+    assert np.array_equal(r, y16), "bf16 output is not RNE(fp32 output)"
+    tokens = sample_tokens(T, 24)
+    yo, problems, _, probs, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx, tokens,
+                                                 shared=cfg.ff_shared > 0)
+    assert not problems, problems[:3]
+    wref = np.take_along_axis(probs, idx[tokens].astype(np.int64), axis=1)
+    assert np.allclose(w[tokens], wref, rtol=1e-5, atol=1e-7)
+    err = g1_error(y32[tokens], yo)
+    assert err.max() <= G1_TOL, (err.max(), err)
+
+
+def test_grouped_prefill_matches_chunked_path(orc):
+    """The same call with a workspace too small for the grouped region runs
+    8-token passes; both must meet the oracle, and routing must agree."""
+    cfg = SMALL
+    T = 45
+    W = kdev.weights(cfg)
+    inp = kdev.DeviceInputs(cfg, T=T)
+    dims = dims_of(cfg, m.K3MOE_OUT_FP32)
+    outs = []
+    for wsT in (T, 8):
+        ws = m.new_workspace(dims, wsT)
+        y = torch.empty((T, cfg.d), dtype=torch.float32, device="cuda")
+        idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
+        m.check(m.k3moe_layer(inp.x, T, W.w_router, inp.bias, W.blob_ptrs, *W.shared, dims, y, idx, w, ws),
+                "layer")
+        torch.cuda.synchronize()
+        m.check(m.k3moe_device_status(ws), "device status")
+        outs.append((y.cpu().numpy(), idx.cpu().numpy()))
+    assert np.array_equal(outs[0][1], outs[1][1])
+    yo, problems, _, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, outs[0][1],
+                                             list(range(T)))
+    assert not problems
+    for y, _ in outs:
+        assert g1_error(y, yo).max() <= G1_TOL
+
+
+def test_grouped_prefill_deterministic_and_multi_pass(orc):
+    """k=32 of 64 experts on a tiny shape needs several passes for 6000 tokens
+    (each CTA's group table is bounded); two calls give the same bytes."""
+    cfg = k3gen.Config("pf_pass", d=256, ff=128, E=64, k=32, ff_shared=128, T=0, bias="normal")
+    T = 6000
+    W = kdev.weights(cfg)
+    inp = kdev.DeviceInputs(cfg, T=T)
+    a = run_layer(cfg, W, inp.x, inp.bias, T, m.K3MOE_OUT_FP32)
+    b = run_layer(cfg, W, inp.x, inp.bias, T, m.K3MOE_OUT_FP32)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+    y, idx, _ = a
+    tokens = sample_tokens(T, 16)
+    yo, problems, _, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx, tokens)
+    assert not problems
+    assert g1_error(y[tokens], yo).max() <= G1_TOL
