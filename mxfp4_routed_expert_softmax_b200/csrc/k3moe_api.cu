@@ -70,10 +70,10 @@ k3moe_status device_info(DeviceInfo **out) {
             di.route_dyn_max = big - (int)fa.sharedSizeBytes;
             r = set_smem(route_kernel, di.route_dyn_max);
         }
-        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<true, false>, big);
-        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<false, false>, big);
-        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<true, true>, big);
-        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<false, true>, big);
+        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<true>, big);
+        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<false>, big);
+        if (r == cudaSuccess) r = set_smem(pf_expert_kernel<true>, big);
+        if (r == cudaSuccess) r = set_smem(pf_expert_kernel<false>, big);
         if (r != cudaSuccess) return cuda_fail(r);
         di.ready = true;
     }
@@ -113,35 +113,10 @@ Layout layout_for(const k3moe_dims *dm, int k_eff) {
 }
 
 // ---------------------------------------------------------- prefill pass --
-// The grouped prefill kernels run on a fixed grid; a pass takes as many
-// tokens (up to kPfMaxTokens) as keep every CTA's share of groups within its
-// shared-memory table (a bound over the worst case of the routing).
-constexpr int kPfCtas = 148;
-
-int pf_groups_per_cta_bound(const k3moe_dims *dm, int Tp) {
-    const int d = dm->d, ff = dm->ff, E = dm->n_experts, k = dm->top_k;
-    const int ffs = (dm->flags & K3MOE_NO_SHARED) ? 0 : dm->ff_shared;
-    const long long ngr = pf_routed_groups_max(Tp, E, k), ngs = ffs > 0 ? ceil_div(Tp, kGroup) : 0;
-    int worst = 0;
-    for (int gu = 0; gu < 2; ++gu) {
-        const long long upr = gu ? (long long)ceil_div(ff, kTileM) * ceil_div(d, kTileK)
-                                 : (long long)ceil_div(d, kTileM) * ceil_div(ff, kTileK);
-        const long long ups = ffs == 0 ? 0
-                              : gu ? (long long)ceil_div(ffs, kTileM) * ceil_div(d, kTileKs)
-                                   : (long long)ceil_div(d, kTileM) * ceil_div(ffs, kTileKs);
-        const long long total = ngr * upr + ngs * ups;
-        const long long per = (total + kPfCtas - 1) / kPfCtas;
-        const long long mn = ups > 0 && ups < upr ? ups : upr;
-        const long long g = (per + mn - 1) / mn + 1;
-        if (g > worst) worst = (int)(g > (1 << 30) ? (1 << 30) : g);
-    }
-    return worst;
-}
-
+// A pass of the grouped prefill takes up to kPfMaxTokens tokens.
 int pf_pass_tokens(const k3moe_dims *dm, int T) {
-    int Tp = T < kPfMaxTokens ? T : kPfMaxTokens;
-    while (Tp > kChunk && pf_groups_per_cta_bound(dm, Tp) > kPfMetaG) Tp -= kGroup;
-    return Tp;
+    (void)dm;
+    return T < kPfMaxTokens ? T : kPfMaxTokens;
 }
 
 PLayout playout_for(const k3moe_dims *dm, int Tp) {
@@ -286,14 +261,13 @@ k3moe_status shared_tmaps(int d, int ffs, const void *wg, const void *wu, const 
 
 template <bool GU>
 cudaError_t launch_umma(const DeviceInfo &di, UmmaParams up, cudaStream_t st) {
-    up.ngs = 0;
     const int N = act_n(up.Tc);
     up.nst = umma_stages(GU, N);
     up.sb = umma_stage_bytes(GU, N);
     up.sf_tma = (GU ? up.d : up.ff) % 512 == 0;
     const int smem = umma_smem_bytes(GU, N, up.nst);
     const int g = di.sms < kMaxCtas ? di.sms : kMaxCtas;
-    return launch(umma_expert_kernel<GU, false>, dim3(g), dim3(kUThreads), smem, st, true, up);
+    return launch(umma_expert_kernel<GU>, dim3(g), dim3(kUThreads), smem, st, true, up);
 }
 
 
@@ -347,6 +321,8 @@ k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims
         pp.P = P;
         pp.T = Tq;
         pp.ngs = ffs > 0 ? ceil_div(Tq, kGroup) : 0;
+        pp.ff = dims->ff;
+        pp.ffs = ffs;
         // router: split K until the grid covers the GPU twice; the split
         // partials go where the expert outputs go later (not in use yet)
         PfRouterParams rr{};
@@ -361,7 +337,7 @@ k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims
         if (ns > 8) ns = 8;
         if (ns > d / 256) ns = d / 256;
         if (ns < 1) ns = 1;
-        while (ns > 1 && (size_t)ns * Tq * E * 4 > P.icnt - P.o) --ns;
+        while (ns > 1 && (size_t)ns * Tq * E * 4 > P.total - P.o) --ns;
         rr.nsplit = ns;
         rr.out = reinterpret_cast<float *>(wsb + (ns > 1 ? P.o : P.lg));
         e = launch(pf_router_kernel, dim3(gx, gy, ns), dim3(kPrThreads), 0, st, false, rr);
@@ -378,30 +354,29 @@ k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims
         e = launch(pf_hist_kernel, dim3(nhb), dim3(kRouteThreads), 0, st, false, pp);
         if (e == cudaSuccess) e = launch(pf_scan_kernel, dim3(1), dim3(kPfScanThreads), 0, st, false, pp);
         if (e == cudaSuccess) e = launch(pf_place_kernel, dim3(nhb), dim3(kRouteThreads), 0, st, false, pp);
+        if (e == cudaSuccess) e = launch(pf_items_kernel, dim3(2 * di.sms), dim3(256), 0, st, false, pp);
         if (e == cudaSuccess) e = launch(pf_prep_kernel, dim3(2 * di.sms), dim3(kRouteThreads), 0, st, false, pp);
         if (e != cudaSuccess) return cuda_fail(e, "prefill dispatch launch");
-        e = cudaMemsetAsync(wsb + P.icnt, 0, P.total - P.icnt, st);
-        if (e != cudaSuccess) return cuda_fail(e, "prefill counters");
-        UmmaParams up{};
-        up.Tc = 0;
+        PfUmmaParams up{};
         up.d = d;
         up.ff = dims->ff;
         up.k = k;
         up.ffs = ffs;
         up.ws = wsb;
         up.L = rp.L;
-        up.out_fp32 = out32;
-        up.y = nullptr;
         up.P = P;
         up.ngs = pp.ngs;
         up.blobs = rp.blobs;
         for (int gu = 1; gu >= 0; --gu) {
-            up.nst = umma_stages(gu != 0, kPfN);
-            up.sb = umma_stage_bytes(gu != 0, kPfN);
+            const int sb = umma_stage_bytes(gu != 0, kPfN);
+            int nst = (kSmemLimit - pf_smem_bytes(gu != 0, 0)) / sb;
+            if (nst > 8) nst = 8;
+            up.nst = nst;
+            up.sb = sb;
             up.sf_tma = (gu ? d : dims->ff) % 512 == 0;
-            const int smem = umma_smem_bytes(gu != 0, kPfN, up.nst);
-            e = gu ? launch(umma_expert_kernel<true, true>, dim3(kPfCtas), dim3(kUThreads), smem, st, true, up)
-                   : launch(umma_expert_kernel<false, true>, dim3(kPfCtas), dim3(kUThreads), smem, st, true, up);
+            const int smem = pf_smem_bytes(gu != 0, nst);
+            e = gu ? launch(pf_expert_kernel<true>, dim3(di.sms), dim3(kPfThreads), smem, st, true, up)
+                   : launch(pf_expert_kernel<false>, dim3(di.sms), dim3(kPfThreads), smem, st, true, up);
             if (e != cudaSuccess) return cuda_fail(e, gu ? "prefill gate/up launch" : "prefill down launch");
         }
         PfCombineParams cp{};

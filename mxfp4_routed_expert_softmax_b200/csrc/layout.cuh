@@ -109,23 +109,24 @@ __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int f
 
 // ---------------------------------------------------------------- prefill --
 // Grouped prefill (more than kChunk tokens): the pairs (token, slot) are
-// sorted by expert, each expert's pairs cut into groups of up to kGroup
-// tokens; a tensor-core item is (group, 128 weight rows), so each expert's
-// weights stream once per call while its groups run side by side.  The
-// shared expert takes groups of kGroup consecutive tokens.  Activations enter
-// as kPfPieces E2M1 pieces per element: token j of a group owns B rows
-// 8j..8j+7, one 1024-byte block per K-tile ([16-byte chunk c][piece][16 B]),
-// so a token's block of a K-tile is one contiguous copy.
-constexpr int kGroup = 8;       // tokens per group
-constexpr int kPfPieces = 8;    // pieces per activation element (rows per token)
+// sorted by expert and each expert's pairs cut into groups of up to kGroup
+// tokens; a tensor-core item is (group, 128 weight rows), and the items of
+// one expert's row block are consecutive, so the CTAs that run them side by
+// side read each weight tile from HBM once and from L2 for the other groups.
+// The shared expert takes groups of kGroup consecutive tokens.  Activations
+// enter as kPfPieces E2M1 pieces per element: token j of a group owns B rows
+// 4j..4j+3 (half a core matrix), so its 64 bytes per 16-byte chunk of a
+// K-tile are one contiguous copy.
+constexpr int kGroup = 16;      // tokens per group
+constexpr int kPfPieces = 4;    // pieces per activation element (rows per token)
 constexpr int kPfN = kGroup * kPfPieces;  // 64: MMA N of a routed group
-constexpr int kPfNs = 16;       // MMA N of a shared-expert group (bf16 rows 0-7, 8-15)
-constexpr int kPfMetaG = 160;   // groups one CTA's share of a pass may touch (shared memory)
-constexpr int kPfMaxTokens = 8192;  // tokens per prefill pass
-constexpr int kPfHistTok = 16;  // tokens per block of the dispatch histogram
+constexpr int kPfNsGU = kGroup;           // 16: shared gate/up (x as bf16, one row per token)
+constexpr int kPfNsDn = 2 * kGroup;       // 32: shared down (h as bf16 high rows, then low rows)
+constexpr int kPfMaxTokens = 8192;        // tokens per prefill pass
+constexpr int kPfHistTok = 16;            // tokens per block of the dispatch histogram
 
 struct PLayout {
-    size_t lg;     // f32 [Tp][E] router logits
+    size_t lg;     // f32 [Tp][E] router logits (or the router's split-K partials: see o)
     size_t idx;    // i32 [Tp][k]
     size_t wt;     // f32 [Tp][k]
     size_t hist;   // u32 [nhb][E] picks per (16-token block, expert), then their exclusive
@@ -134,16 +135,17 @@ struct PLayout {
     size_t eoff;   // u32 [E] first position of each expert in perm
     size_t goff;   // u32 [E] first group of each expert
     size_t perm;   // i32 [Tp*k] pair ids t*k+j sorted by (expert, token)
-    size_t grp;    // int4 [ngmax] routed groups then shared groups: (expert or -1, first
-                   // position / first token, tokens, blob ok)
-    size_t xp;     // u8 [Tp][nkt_d][1024] pieces of x, one block per (token, K-tile)
-    size_t xps;    // u8 [Tp][nkt_d][2][8][4] their scales ([group of 4 blocks][piece][block])
-    size_t xbf;    // u8 [ngs][nkts_d][kPfNs*128] x as bf16 per shared group (rows 0-7)
+    size_t grp;    // int4 [ngr + ngs] routed groups then shared groups: (expert or -1,
+                   // first position / first token, tokens, blob ok)
+    size_t itg;    // i32 [ngr*nrb_ff + ngs*nrbs_ff] gate/up items in run order: group | rb << 20
+    size_t itd;    // i32 [(ngr + ngs)*nrb_d] down items in run order
+    size_t xp;     // u8 [Tp][nkt_d][8 chunks][4 pieces][16 B] pieces of x per token
+    size_t xps;    // u8 [Tp][nkt_d][2][4 pieces][4] their scales ([group of 4 blocks][piece][block])
+    size_t xbf;    // u8 [ngs][nkts_d][kPfNsGU*128] x as bf16 per shared group
     size_t hb;     // u8 [ngr][nkt_ff][kPfN*128] w*h pieces per routed group (down B)
     size_t hsf;    // u32 [ngr][nkt_ff][2][kSfRow]
-    size_t hsb;    // u8 [ngs][nkts_ff][kPfNs*128] shared h as bf16 hi (rows 0-7), lo (8-15)
+    size_t hsb;    // u8 [ngs][nkts_ff][kPfNsDn*128] shared h as bf16 high (rows 0-15), low (16-31)
     size_t o;      // f32 [Tp][k+1][d] expert outputs per (token, slot); slot k: shared
-    size_t icnt;   // u32 [gate/up items + down items] arrivals per split item (back to 0)
     size_t total;  // end offset (absolute: the prefill region follows the decode layout)
     int Tp, ngr, ngs, nhb;
 };
@@ -161,43 +163,31 @@ __host__ __device__ inline PLayout make_playout(size_t base, int d, int ff, int 
     P.nhb = ceil_div(Tp, kPfHistTok);
     const int nkt_d = ceil_div(d, kTileK), nkt_ff = ceil_div(ff, kTileK);
     const int nkts_d = ceil_div(d, kTileKs), nkts_ff = ffs > 0 ? ceil_div(ffs, kTileKs) : 0;
+    const size_t nrb_ff = ceil_div(ff, kTileM), nrbs_ff = ffs > 0 ? ceil_div(ffs, kTileM) : 0;
+    const size_t nrb_d = ceil_div(d, kTileM);
     size_t o = align256(base);
-    P.lg = o;
-    o = align256(o + (size_t)Tp * E * 4);
-    P.idx = o;
-    o = align256(o + (size_t)Tp * k * 4);
-    P.wt = o;
-    o = align256(o + (size_t)Tp * k * 4);
-    P.hist = o;
-    o = align256(o + (size_t)P.nhb * E * 4);
-    P.ecnt = o;
-    o = align256(o + (size_t)E * 4);
-    P.eoff = o;
-    o = align256(o + (size_t)E * 4);
-    P.goff = o;
-    o = align256(o + (size_t)E * 4);
-    P.perm = o;
-    o = align256(o + (size_t)Tp * k * 4);
-    P.grp = o;
-    o = align256(o + (size_t)(P.ngr + P.ngs) * 16);
-    P.xp = o;
-    o = align256(o + (size_t)Tp * nkt_d * 1024);
-    P.xps = o;
-    o = align256(o + (size_t)Tp * nkt_d * 64);
-    P.xbf = o;
-    o = align256(o + (size_t)P.ngs * nkts_d * kPfNs * 128);
-    P.hb = o;
-    o = align256(o + (size_t)P.ngr * nkt_ff * kPfN * 128);
-    P.hsf = o;
-    o = align256(o + (size_t)P.ngr * nkt_ff * 2 * kSfRow * 4);
-    P.hsb = o;
-    o = align256(o + (size_t)P.ngs * nkts_ff * kPfNs * 128);
-    P.o = o;
-    o = align256(o + (size_t)Tp * (k + 1) * d * 4);
-    P.icnt = o;
-    const size_t items = (size_t)P.ngr * ceil_div(ff, kTileM) + (size_t)P.ngs * (ffs > 0 ? ceil_div(ffs, kTileM) : 0) +
-                         (size_t)(P.ngr + P.ngs) * ceil_div(d, kTileM);
-    o = align256(o + items * 4);
+    auto take = [&](size_t &field, size_t bytes) {
+        field = o;
+        o = align256(o + bytes);
+    };
+    take(P.lg, (size_t)Tp * E * 4);
+    take(P.idx, (size_t)Tp * k * 4);
+    take(P.wt, (size_t)Tp * k * 4);
+    take(P.hist, (size_t)P.nhb * E * 4);
+    take(P.ecnt, (size_t)E * 4);
+    take(P.eoff, (size_t)E * 4);
+    take(P.goff, (size_t)E * 4);
+    take(P.perm, (size_t)Tp * k * 4);
+    take(P.grp, (size_t)(P.ngr + P.ngs) * 16);
+    take(P.itg, ((size_t)P.ngr * nrb_ff + (size_t)P.ngs * nrbs_ff) * 4);
+    take(P.itd, (size_t)(P.ngr + P.ngs) * nrb_d * 4);
+    take(P.xp, (size_t)Tp * nkt_d * 8 * kPfPieces * 16);
+    take(P.xps, (size_t)Tp * nkt_d * 2 * kPfPieces * 4);
+    take(P.xbf, (size_t)P.ngs * nkts_d * kPfNsGU * 128);
+    take(P.hb, (size_t)P.ngr * nkt_ff * kPfN * 128);
+    take(P.hsf, (size_t)P.ngr * nkt_ff * 2 * kSfRow * 4);
+    take(P.hsb, (size_t)P.ngs * nkts_ff * kPfNsDn * 128);
+    take(P.o, (size_t)Tp * (k + 1) * d * 4);
     P.total = o;
     return P;
 }

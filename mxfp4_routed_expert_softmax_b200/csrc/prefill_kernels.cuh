@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "decode_kernels.cuh"
 #include "layout.cuh"
+#include "prefill_umma.cuh"
 #include "umma_kernels.cuh"
 
 namespace k3 {
@@ -145,6 +146,7 @@ struct PfRouteParams {
     PLayout P;
     int T;               // tokens of this pass
     int ngs;             // shared groups of this pass (0: no shared expert)
+    int ff, ffs;         // expert and shared-expert hidden sizes
 };
 
 // One CTA per token: softmax over all E and the top-k (as in decode).
@@ -257,11 +259,45 @@ __global__ void __launch_bounds__(kRouteThreads) pf_place_kernel(const __grid_co
     }
 }
 
+// Items of the expert kernels in run order: for each expert, for each 128-row
+// block, its groups (so the groups sharing a weight tile run side by side);
+// then the shared expert's items, row block by row block.  Entry: group |
+// row block << 20.  One thread per (group, row block).
+__global__ void pf_items_kernel(const __grid_constant__ PfRouteParams p) {
+    const uint8_t *ws = p.r.ws;
+    const int NG = (int)*reinterpret_cast<const volatile uint32_t *>(
+        &reinterpret_cast<const WsHeader *>(ws + p.r.L.hdr)->n_unique);
+    const int4 *grp = reinterpret_cast<const int4 *>(ws + p.P.grp);
+    const uint32_t *ecnt = reinterpret_cast<const uint32_t *>(ws + p.P.ecnt);
+    const uint32_t *goff = reinterpret_cast<const uint32_t *>(ws + p.P.goff);
+    int32_t *itg = reinterpret_cast<int32_t *>(p.r.ws + p.P.itg);
+    int32_t *itd = reinterpret_cast<int32_t *>(p.r.ws + p.P.itd);
+    const int nrb_ff = ceil_div(p.ff, kTileM), nrb_d = ceil_div(p.r.d, kTileM);
+    const int nrbs_ff = p.ngs > 0 ? ceil_div(p.ffs, kTileM) : 0;
+    const int per = nrb_ff > nrb_d ? nrb_ff : nrb_d;
+    const long long n = (long long)(NG + p.ngs) * per;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const int g = (int)(i / per), rb = (int)(i - (long long)g * per);
+        if (g < NG) {
+            const int e = __ldcg(&grp[g].x);
+            const int ng = (int)((__ldcg(ecnt + e) + kGroup - 1) / kGroup), j = g - (int)__ldcg(goff + e);
+            const int base = (int)__ldcg(goff + e);
+            if (rb < nrb_ff) itg[base * nrb_ff + rb * ng + j] = g | (rb << 20);
+            if (rb < nrb_d) itd[base * nrb_d + rb * ng + j] = g | (rb << 20);
+        } else {
+            const int s = g - NG;
+            if (rb < nrbs_ff) itg[NG * nrb_ff + rb * p.ngs + s] = g | (rb << 20);
+            if (rb < nrb_d) itd[NG * nrb_d + rb * p.ngs + s] = g | (rb << 20);
+        }
+    }
+}
+
 // -------------------------------------------------------------- x pieces --
-// Every token's x as kPfPieces E2M1 pieces, one 1024-byte block per K-tile
-// (token row group of the prefill B layout) plus 64 scale bytes; with a
-// shared expert, x as bf16 in the shared groups' tiles (rows 0-7; rows 8-15
-// and the rows of absent tokens zero).  Warps over (token, 32-block).
+// Every token's x as kPfPieces E2M1 pieces: per K-tile, [chunk][piece][16 B]
+// (64 contiguous bytes per chunk: the token's half core matrix) and the
+// scales [group of 4 blocks][piece][block]; with a shared expert, x as bf16
+// in the shared groups' tiles (MMA N = 16 rows, one per token; the rows of
+// absent tokens zero).  Warps over (token, 32-block).
 __global__ void __launch_bounds__(kRouteThreads) pf_prep_kernel(const __grid_constant__ PfRouteParams p) {
     const int lane = threadIdx.x & 31, d = p.r.d, nb = d / 32, nkt = ceil_div(d, kTileK);
     const int nkts = ceil_div(d, kTileKs);
@@ -276,15 +312,14 @@ __global__ void __launch_bounds__(kRouteThreads) pf_prep_kernel(const __grid_con
         if (real) {
             const float v = __uint_as_float((uint32_t)xv << 16);
             const size_t blk = (size_t)t * nkt + (b >> 3);
-            quantize_pieces_t<kPfPieces, true>(v, lane, 0, b & 7, kPfN, kPfPieces, ws + p.P.xp + blk * 1024,
-                                               ws + p.P.xps + blk * 64);
+            quantize_pieces_t<kPfPieces>(v, lane, 0, b & 7, kPfPieces * 16, 0, kPfPieces,
+                                         ws + p.P.xp + blk * (8 * kPfPieces * 16), ws + p.P.xps + blk * (2 * kPfPieces * 4));
         }
         if (p.ngs > 0) {
             const int gs = t / kGroup, j = t - gs * kGroup;
-            uint8_t *tile = ws + p.P.xbf + ((size_t)gs * nkts + col / kTileKs) * kPfNs * 128;
+            uint8_t *tile = ws + p.P.xbf + ((size_t)gs * nkts + col / kTileKs) * kPfNsGU * 128;
             const int c = (col % kTileKs) / 8, e = col % 8;
-            *reinterpret_cast<uint16_t *>(tile + (c * 2) * 128 + j * 16 + e * 2) = xv;
-            *reinterpret_cast<uint16_t *>(tile + (c * 2 + 1) * 128 + j * 16 + e * 2) = (uint16_t)0;
+            *reinterpret_cast<uint16_t *>(tile + c * (kPfNsGU / 8) * 128 + (j / 8) * 128 + (j % 8) * 16 + e * 2) = xv;
         }
     }
 }

@@ -53,16 +53,14 @@ constexpr int kAtile = kTileM * 128;  // one A box: 128 rows x 128 bytes (16 KB)
 // value q >= 1 is read off its fp32 bits (exponent and top mantissa bit),
 // below 1 it is 0 or 1 (0.5).
 // Writes the 16-byte nibble row of each piece into a K-tile of the B operand
-// (no-swizzle K-major core matrices, this block is 16-byte chunk c of the
-// tile; element 2i in the low nibble of byte i) and its scale byte into the
-// tile's scale words (sfw[(c/4)*sfrow + n], byte c%4).  B row n = t*P + p.
-// Core-matrix order: decode tiles put the N/8 row groups of one chunk side by
-// side (chunk c, row group n/8 at (c*N/8 + n/8)*128); prefill tiles (FLIP)
-// keep each row group's 8 chunks together (at (n/8)*1024 + c*128), so one
-// token's K-tile is one 1024-byte block.  All 32 lanes of the warp call it.
-template <int P, bool FLIP>
-__device__ __forceinline__ void quantize_pieces_t(float v, int lane, int t, int c, int N, int sfrow, uint8_t *tile,
-                                                  uint8_t *sfw) {
+// (no-swizzle K-major core matrices; this block is 16-byte chunk c of the
+// tile; element 2i in the low nibble of byte i): B row n = t*P + p goes to
+// tile + c*cs + (n/8)*gs + (n%8)*16 (an MMA tile of N rows: cs = N/8*128,
+// gs = 128), and its scale byte to the tile's scale words (sfw[(c/4)*sfrow +
+// n], byte c%4).  All 32 lanes of the warp call it.
+template <int P>
+__device__ __forceinline__ void quantize_pieces_t(float v, int lane, int t, int c, int cs, int gs, int sfrow,
+                                                  uint8_t *tile, uint8_t *sfw) {
     float r = v;
 #pragma unroll
     for (int p = 0; p < P; ++p) {
@@ -80,14 +78,14 @@ __device__ __forceinline__ void quantize_pieces_t(float v, int lane, int t, int 
         r = __fmaf_rn(-copysignf(q, s), exp2i(e), r);
         const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
         const int n = t * P + p;
-        uint8_t *row = tile + (FLIP ? (n / 8) * 1024 + c * 128 : (c * (N / 8) + n / 8) * 128) + (n % 8) * 16;
+        uint8_t *row = tile + c * cs + (n / 8) * gs + (n % 8) * 16;
         if ((lane & 1) == 0) row[lane >> 1] = (uint8_t)(code | (hi << 4));
         if (lane == 0) sfw[((c >> 2) * sfrow + n) * 4 + (c & 3)] = (uint8_t)(e + 127);
     }
 }
 __device__ __forceinline__ void quantize_pieces(float v, int lane, int t, int c, int N, uint8_t *tile,
                                                 uint8_t *sfw) {
-    quantize_pieces_t<kPieces, false>(v, lane, t, c, N, kSfRow, tile, sfw);
+    quantize_pieces_t<kPieces>(v, lane, t, c, (N / 8) * 128, 128, kSfRow, tile, sfw);
 }
 
 // x of the chunk -> pieces (routed gate/up B operand) and, with a shared
@@ -167,10 +165,6 @@ struct UmmaParams {
     // down only
     int out_fp32;     // y in fp32 (else bf16, rounded once)
     void *y;          // [Tc][d] of this chunk
-    // grouped prefill only
-    PLayout P;        // the prefill region of the workspace
-    int ngs;          // shared-expert groups of this pass (0: no shared expert)
-    const uint8_t *const *blobs;  // device array [E] of expert blobs (scale loads without TMA)
 };
 
 // One pipeline stage for MMA width N: the A boxes (16 KB per matrix, first,
@@ -191,12 +185,7 @@ __host__ __device__ inline int umma_sf_cols(bool gu) { return gu ? 32 : 16; }
 // it) of each distinct expert.  Global loads issued while the weight stream
 // saturates HBM wait thousands of cycles, so the pipeline never makes them.
 constexpr int kMetaU = kChunk * 32;  // distinct experts of a chunk (top_k <= 32)
-// Grouped prefill: per group of this CTA's share, its expert (or -1: shared),
-// token count | blob ok << 8, pair ids (t*k+j; shared: token ids) and
-// routing weights.
-constexpr int kMetaBytesDecode = kMetaU * 8 + kMetaU * 4 + kMetaU * kChunk * 4;
-constexpr int kMetaBytesPf = kPfMetaG * (4 + 4 + kGroup * 4 + kGroup * 4);
-constexpr int kMetaBytes = kMetaBytesDecode > kMetaBytesPf ? kMetaBytesDecode : kMetaBytesPf;
+constexpr int kMetaBytes = kMetaU * 8 + kMetaU * 4 + kMetaU * kChunk * 4;
 __host__ __device__ inline int umma_smem_bytes(bool gu, int N, int nst) {
     return 1024 + nst * umma_stage_bytes(gu, N) + 256 + kMetaBytes;
 }
@@ -221,12 +210,7 @@ __device__ __forceinline__ uint2 load_sf8(const uint8_t *p, int nks) {
 // expert's ff_s (64-weight bf16 tiles), all into one accumulator, so the
 // routing weights (folded into the routed pieces) and the shared expert are
 // combined by the tensor core itself.
-// PF (grouped prefill): items are (group, 128 weight rows), the routed groups
-// (K-tiles of 256, B = the group's tokens' pieces, N = kPfN) and then the
-// shared expert's groups (bf16 K-tiles of 64, N = kPfNs); every item has its
-// own tokens, so a down item writes its tokens' (token, slot) outputs and a
-// separate pass sums them.
-template <bool GU, bool PF>
+template <bool GU>
 __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -244,11 +228,6 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     const uint8_t **s_blob = reinterpret_cast<const uint8_t **>(smem + nst * SB + 256);
     int32_t *s_eid = reinterpret_cast<int32_t *>(s_blob + kMetaU);
     float *s_wu = reinterpret_cast<float *>(s_eid + kMetaU);  // [u][t]
-    // grouped prefill: the same region holds this CTA's groups
-    int32_t *g_eid = reinterpret_cast<int32_t *>(smem + nst * SB + 256);  // expert, -1: shared
-    int32_t *g_nok = g_eid + kPfMetaG;                                     // tokens | blob ok << 8
-    int32_t *g_pair = g_nok + kPfMetaG;                                    // [g][j] pair (shared: token)
-    float *g_w = reinterpret_cast<float *>(g_pair + kPfMetaG * kGroup);   // [g][j] routing weight
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Layout &L = p.L;
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + L.hdr);
@@ -274,10 +253,9 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     pdl_wait();
     pdl_trigger();
 
-    const int Tc = p.Tc, N = PF ? kPfN : act_n(Tc);
-    // distinct experts of the chunk (decode) or routed groups of the pass (PF)
+    const int Tc = p.Tc, N = act_n(Tc);
     const int U = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_unique);
-    if constexpr (!PF) {
+    {
         const uint8_t *const *gb = reinterpret_cast<const uint8_t *const *>(p.ws + L.uniq_blob);
         const int32_t *ge = reinterpret_cast<const int32_t *>(p.ws + L.uniq_eid);
         const uint32_t *gm = reinterpret_cast<const uint32_t *>(p.ws + L.uniq_mask);
@@ -301,23 +279,20 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     const int nkt = ceil_div(K, kTileK);
     const int nrb = ceil_div(M, kTileM);
     const int nkts = p.ffs > 0 ? ceil_div(Ks, kTileKs) : 0;
-    // shared-expert row blocks: decode gate/up only (the decode down items
-    // append the shared K-tiles); PF both (down: d rows per shared group)
-    const int nrbs = p.ffs > 0 ? (PF ? (GU ? ceil_div(p.ffs, kTileM) : nrb) : (GU ? ceil_div(p.ffs, kTileM) : 0)) : 0;
-    const int R = (GU || PF) ? U * nrb * nkt : 0;     // routed units (GU, PF)
-    const int upi = (GU || PF) ? 0 : U * nkt + nkts;  // units per item (decode down)
-    const int total = PF ? R + p.ngs * nrbs * nkts : (GU ? R + nrbs * nkts : nrb * upi);
+    const int nrbs = (GU && p.ffs > 0) ? ceil_div(p.ffs, kTileM) : 0;
+    const int R = GU ? U * nrb * nkt : 0;             // routed units (GU)
+    const int upi = GU ? 0 : U * nkt + nkts;          // units per item (down)
+    const int total = GU ? R + nrbs * nkts : nrb * upi;
     const int G = min((int)gridDim.x, max(total, 1));
     const int cta = blockIdx.x;
     auto start = [&](int c) { return (int)(((long long)c * total) / G); };
     auto owner = [&](int unit) { return (int)((((long long)unit + 1) * G - 1) / total); };
-    const int a = cta < G ? start(cta) : 0;
-    int b = cta < G ? start(cta + 1) : 0;
+    const int a = cta < G ? start(cta) : 0, b = cta < G ? start(cta + 1) : 0;
     const size_t mat = (size_t)p.d * p.ff;
     const uint8_t *const *ublob = s_blob;
     const uint8_t *smaps = p.ws + L.tmap + (size_t)L.E * kMapsPerExpert * 128;
     const int32_t *ueid = s_eid;
-    const uint32_t idesc4 = umma::idesc_mxf4(N), idesc16 = umma::idesc_bf16(PF ? kPfNs : N);
+    const uint32_t idesc4 = umma::idesc_mxf4(N), idesc16 = umma::idesc_bf16(N);
     // TMEM columns: accumulators [buf][mat] at (buf*NMAT + mat)*64 (N <= 64), then
     // the scale columns of each stage from sf0
     const uint32_t sf0 = GU ? 256u : 128u;
@@ -337,25 +312,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     };
     auto decode = [&](int unit) {
         Unit x;
-        if constexpr (PF) {
-            if (unit < R) {
-                x.item = unit / nkt;
-                x.istart = x.item * nkt;
-                x.iend = x.istart + nkt;
-                x.u = x.item / nrb;  // routed group
-                x.rb = x.item - x.u * nrb;
-                x.shared = false;
-            } else {
-                const int j = (unit - R) / nkts;
-                x.item = U * nrb + j;
-                x.istart = R + j * nkts;
-                x.iend = x.istart + nkts;
-                x.u = U + j / nrbs;  // shared groups follow the routed ones
-                x.rb = j - (j / nrbs) * nrbs;
-                x.shared = true;
-            }
-            x.kt = unit - x.istart;
-        } else if constexpr (GU) {
+        if constexpr (GU) {
             if (unit < R) {
                 x.item = unit / nkt;
                 x.istart = x.item * nkt;
@@ -400,7 +357,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         Unit y = x;
         if (unit_next >= x.iend) return unit_next < total ? decode(unit_next) : x;
         ++y.kt;
-        if constexpr (!GU && !PF) {
+        if constexpr (!GU) {
             if (!y.shared && y.kt == nkt) {
                 y.kt = 0;
                 if (++y.u == U) {
@@ -412,48 +369,6 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         return y;
     };
 
-    // PF: this CTA's groups (a contiguous range) into shared memory, so the
-    // pipeline never waits on a global load for them
-    int g_lo = 0;
-    if constexpr (PF) {
-        const int4 *grp = reinterpret_cast<const int4 *>(p.ws + p.P.grp);
-        const int32_t *perm = reinterpret_cast<const int32_t *>(p.ws + p.P.perm);
-        const float *pwt = reinterpret_cast<const float *>(p.ws + p.P.wt);
-        int ng = 0;
-        if (a < b) {
-            g_lo = decode(a).u;
-            ng = decode(b - 1).u - g_lo + 1;
-        }
-        if (ng > kPfMetaG) {
-            // the host sizes passes so that this cannot happen; never overrun
-            if (threadIdx.x == 0) set_status(hdr, kStDeviceCheck);
-            ng = 0;
-            b = a;
-        }
-        for (int i = threadIdx.x; i < ng; i += kUThreads) {
-            const int4 gr = grp[g_lo + i];  // (expert or -1, first position / token, tokens, blob ok)
-            g_eid[i] = gr.x;
-            g_nok[i] = gr.z | (gr.w << 8);
-#pragma unroll
-            for (int j = 0; j < kGroup; ++j) {
-                int pid = 0;
-                float w = 0.f;
-                if (j < gr.z) {
-                    if (gr.x >= 0) {
-                        pid = __ldcg(perm + gr.y + j);
-                        w = __ldcg(pwt + pid);
-                    } else {
-                        pid = gr.y + j;
-                        w = 1.f;
-                    }
-                }
-                g_pair[i * kGroup + j] = pid;
-                g_w[i * kGroup + j] = w;
-            }
-        }
-        __syncthreads();
-    }
-
     if (warp == 8) {
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
@@ -463,74 +378,6 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             for (int unit = a, it = 0, s = 0; unit < b && !*s_abort; x = advance(x, ++unit), ++it) {
                 if (it >= nst && !wait(&empty[s], ph ^ 1u)) break;
                 uint8_t *st = smem + s * SB;
-                if constexpr (PF) {
-                    const int gl = x.u - g_lo;
-                    uint8_t *bdst = st + NMAT * kAtile;
-                    if (x.shared) {
-                        const uint8_t *maps = smaps + (GU ? 0 : 256);
-                        const int gs = x.u - U;
-                        const uint8_t *bsrc = p.ws + (GU ? p.P.xbf : p.P.hsb) + ((size_t)gs * nkts + x.kt) * kPfNs * 128;
-                        if (x.u != last_u) {
-                            umma::tmap_acquire(maps);
-                            if (GU) umma::tmap_acquire(maps + 128);
-                            last_u = x.u;
-                        }
-                        mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * kAtile + kPfNs * 128));
-                        umma::tma_load_2d(st, maps, x.kt * 128, x.rb * kTileM, &full[s]);
-                        if (GU) umma::tma_load_2d(st + kAtile, maps + 128, x.kt * 128, x.rb * kTileM, &full[s]);
-                        bulk_g2s(bdst, bsrc, (uint32_t)(kPfNs * 128), &full[s]);
-                    } else {
-                        const bool ok = (g_nok[gl] >> 8) != 0;
-                        const int ntok = g_nok[gl] & 255;
-                        const bool sf_dma = p.sf_tma && ok;
-                        const uint8_t *em = p.ws + L.tmap + (size_t)g_eid[gl] * kMapsPerExpert * 128;
-                        const uint8_t *maps = em + (GU ? 0 : 256);
-                        const uint8_t *scmaps = em + (GU ? 384 : 640);
-                        uint32_t tx = GU ? (uint32_t)ntok * (1024u + (sf_dma ? 64u : 0u))
-                                         : (uint32_t)(kPfN * 128 + (sf_dma ? 2 * kSfRow * 4 : 0));
-                        if (ok) tx += (uint32_t)(NMAT * kAtile + (sf_dma ? NMAT * 2048 : 0));
-                        mbar_arrive_expect_tx(&full[s], tx);
-                        if (ok) {
-                            if (x.u != last_u) {
-                                umma::tmap_acquire(maps);
-                                if (GU) umma::tmap_acquire(maps + 128);
-                                if (sf_dma) {
-                                    umma::tmap_acquire(scmaps);
-                                    if (GU) umma::tmap_acquire(scmaps + 128);
-                                }
-                                last_u = x.u;
-                            }
-                            umma::tma_load_2d(st, maps, x.kt * 128, x.rb * kTileM, &full[s]);
-                            if (GU) umma::tma_load_2d(st + kAtile, maps + 128, x.kt * 128, x.rb * kTileM, &full[s]);
-                            if (sf_dma) {
-                                uint8_t *sfa = st + umma_sfa_off(GU, kPfN);
-                                umma::tma_load_2d(sfa, scmaps, (x.kt >> 1) * 16, x.rb * kTileM, &full[s]);
-                                if (GU)
-                                    umma::tma_load_2d(sfa + 2048, scmaps + 128, (x.kt >> 1) * 16, x.rb * kTileM,
-                                                      &full[s]);
-                            }
-                        }
-                        uint8_t *sfb = st + umma_sfb_off(GU, kPfN);
-                        if (GU) {
-                            // gather: token j's 1024-byte block of this K-tile (and its
-                            // 2 x 32 scale bytes) from the per-token pieces of x
-                            for (int j = 0; j < ntok; ++j) {
-                                const int tok = g_pair[gl * kGroup + j] / p.k;
-                                const size_t blk = (size_t)tok * nkt + x.kt;
-                                bulk_g2s(bdst + j * 1024, p.ws + p.P.xp + blk * 1024, 1024u, &full[s]);
-                                if (sf_dma) {
-                                    bulk_g2s(sfb + 8 * j * 4, p.ws + p.P.xps + blk * 64, 32u, &full[s]);
-                                    bulk_g2s(sfb + (kSfRow + 8 * j) * 4, p.ws + p.P.xps + blk * 64 + 32, 32u, &full[s]);
-                                }
-                            }
-                        } else {
-                            const size_t blk = (size_t)x.u * nkt + x.kt;
-                            bulk_g2s(bdst, p.ws + p.P.hb + blk * kPfN * 128, (uint32_t)(kPfN * 128), &full[s]);
-                            if (sf_dma)
-                                bulk_g2s(sfb, p.ws + p.P.hsf + blk * 2 * kSfRow * 4, (uint32_t)(2 * kSfRow * 4), &full[s]);
-                        }
-                    }
-                } else {
                 const uint8_t *blob = x.shared ? nullptr : ublob[x.u];
                 const uint8_t *maps = nullptr;
                 const uint8_t *bsrc;
@@ -574,7 +421,6 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     mbar_arrive_expect_tx(&full[s], (uint32_t)(N * 128));
                 }
                 bulk_g2s(st + NMAT * kAtile, bsrc, (uint32_t)(N * 128), &full[s]);
-                }
                 if (++s == nst) {
                     s = 0;
                     ph ^= 1u;
@@ -604,11 +450,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 if (!__shfl_sync(0xffffffffu, go, 0)) break;
                 if (!x.shared) {
                     const uint8_t *st = smem + s * SB;
-                    bool has;
-                    if constexpr (PF)
-                        has = (g_nok[x.u - g_lo] >> 8) != 0;
-                    else
-                        has = ublob[x.u] != nullptr;
+                    const bool has = ublob[x.u] != nullptr;
                     const uint32_t col = tbase + lb + sf0 + (uint32_t)(s * SFC);
 #pragma unroll
                     for (int m = 0; m < NMAT; ++m) {
@@ -652,13 +494,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             const Unit x = decode(unit);
             r.on = !x.shared;
             if (x.shared) return;
-            const uint8_t *blob;
-            if constexpr (PF) {
-                const int gl = x.u - g_lo;
-                blob = (g_nok[gl] >> 8) ? p.blobs[g_eid[gl]] : nullptr;
-            } else {
-                blob = ublob[x.u];
-            }
+            const uint8_t *blob = ublob[x.u];
             const int nks = ksteps(x);
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
@@ -674,30 +510,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     r.a[m][4 + j] = v.y;  // group 1: k-steps 2, 3
                 }
             }
-            if constexpr (PF) {
-                if (GU) {
-                    // B row n = 8j + piece: token j's scale words of this K-tile
-                    const int gl = x.u - g_lo, ntok = g_nok[gl] & 255;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int n = 32 * h + lane, j = n >> 3;
-                        uint32_t w0 = 0u, w1 = 0u;
-                        if (j < ntok) {
-                            const int tok = g_pair[gl * kGroup + j] / p.k;
-                            const uint32_t *q = reinterpret_cast<const uint32_t *>(
-                                p.ws + p.P.xps + ((size_t)tok * nkt + x.kt) * 64);
-                            w0 = __ldcg(q + (n & 7));
-                            w1 = __ldcg(q + 8 + (n & 7));
-                        }
-                        r.b[h] = w0;
-                        r.b[2 + h] = w1;
-                    }
-                    return;
-                }
-            }
-            const uint32_t *sfb = PF ? reinterpret_cast<const uint32_t *>(p.ws + p.P.hsf) +
-                                           ((size_t)x.u * nkt + x.kt) * 2 * kSfRow
-                                     : GU ? reinterpret_cast<const uint32_t *>(p.ws + L.xsf) + (size_t)x.kt * 2 * kSfRow
+            const uint32_t *sfb = GU ? reinterpret_cast<const uint32_t *>(p.ws + L.xsf) + (size_t)x.kt * 2 * kSfRow
                                      : reinterpret_cast<const uint32_t *>(p.ws + L.hsf) +
                                            ((size_t)x.u * nkt + x.kt) * 2 * kSfRow;
             r.b[0] = __ldcg(sfb + lane);
@@ -748,17 +561,9 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         // every operand address here stays below 256 KB).
         if (lane == 0) {
             const uint64_t adesc0 = umma::smem_desc(smem_u32(smem), 16u, 1024u, umma::kLayoutSw128);
-            // B: decode tiles put a chunk's row groups side by side (LBO = N/8
-            // core matrices, SBO = 128); prefill routed tiles keep a row
-            // group's chunks together (LBO = 128, SBO = 1024); prefill shared
-            // tiles are decode-style with N = kPfNs
-            const uint32_t bbase = smem_u32(smem) + NMAT * kAtile;
-            const uint64_t bdesc0 = PF ? umma::smem_desc(bbase, 128u, 1024u, umma::kLayoutNone)
-                                       : umma::smem_desc(bbase, (uint32_t)((N / 8) * 128), 128u, umma::kLayoutNone);
-            const uint32_t bstep = PF ? (256u >> 4) : (uint32_t)(2 * (N / 8) * 128) >> 4;  // one k-step (2 chunks)
-            const uint64_t bdesc0s =
-                PF ? umma::smem_desc(bbase, (uint32_t)((kPfNs / 8) * 128), 128u, umma::kLayoutNone) : bdesc0;
-            const uint32_t bsteps = PF ? (uint32_t)(2 * (kPfNs / 8) * 128) >> 4 : bstep;
+            const uint64_t bdesc0 = umma::smem_desc(smem_u32(smem) + NMAT * kAtile, (uint32_t)((N / 8) * 128), 128u,
+                                                    umma::kLayoutNone);
+            const uint32_t bstep = (uint32_t)(2 * (N / 8) * 128) >> 4;  // one k-step of B (2 chunks)
             const uint32_t id4[2] = {umma::idesc_sf_id(idesc4, 0u), umma::idesc_sf_id(idesc4, 2u)};
             int seg = 0, s = 0;
             uint32_t ph = 0u;
@@ -777,11 +582,10 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     const uint64_t a0 = adesc0 + soff, b0 = bdesc0 + soff;
                     const int nks = ksteps(x);
                     if (x.shared) {
-                        const uint64_t b0s = bdesc0s + soff;
 #pragma unroll
                         for (int sk = 0; sk < 4; ++sk) {
                             if (sk < nks) {
-                                const uint64_t bd = b0s + sk * bsteps;
+                                const uint64_t bd = b0 + sk * bstep;
                                 umma::mma_bf16(dcol, a0 + 2 * sk, bd, idesc16, acc);
                                 if (GU) umma::mma_bf16(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, idesc16, acc);
                                 acc = 1u;
@@ -819,13 +623,8 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         const uint32_t lb = umma::lane_base(warp);
         const int rowl = 32 * warp + lane;  // row of the 128-row item
         float *spart = reinterpret_cast<float *>(p.ws + L.spart);
-        uint32_t *icnt;
-        if constexpr (PF)
-            icnt = reinterpret_cast<uint32_t *>(p.ws + p.P.icnt) +
-                   (GU ? 0 : (size_t)p.P.ngr * ceil_div(p.ff, kTileM) + (size_t)p.P.ngs * ceil_div(p.ffs, kTileM));
-        else
-            icnt = reinterpret_cast<uint32_t *>(p.ws + L.icnt) +
-                   (GU ? 0 : L.umax * ceil_div(p.ff, kTileM) + ceil_div(L.ffs, kTileM));
+        uint32_t *icnt = reinterpret_cast<uint32_t *>(p.ws + L.icnt) +
+                         (GU ? 0 : L.umax * ceil_div(p.ff, kTileM) + ceil_div(L.ffs, kTileM));
         int seg = 0;
         for (int unit = a; unit < b; ++seg) {
             const Unit x = decode(unit);
@@ -842,42 +641,8 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             if (lane == 0) wait(&afull[buf], (uint32_t)((seg >> 1) & 1));
             __syncwarp();
             umma::fence_after();
-            // tokens of the item (PF: the group's; decode: the chunk's)
-            int tv = Tc;
-            if constexpr (PF) {
-                tv = g_nok[x.u - g_lo] & 255;
-                if (!x.shared) {
-                    // token j: the sum of its kPfPieces columns 8j..8j+7, in a fixed order
 #pragma unroll
-                    for (int m = 0; m < NMAT; ++m) {
-#pragma unroll
-                        for (int j = 0; j < kGroup; ++j) {
-                            uint32_t r[8];
-                            umma::ld8(tbase + lb + (uint32_t)((buf * NMAT + m) * 64 + 8 * j), r);
-                            umma::wait_ld();
-                            const float s01 = __uint_as_float(r[0]) + __uint_as_float(r[1]);
-                            const float s23 = __uint_as_float(r[2]) + __uint_as_float(r[3]);
-                            const float s45 = __uint_as_float(r[4]) + __uint_as_float(r[5]);
-                            const float s67 = __uint_as_float(r[6]) + __uint_as_float(r[7]);
-                            acc[m][j] = (s01 + s23) + (s45 + s67);
-                        }
-                    }
-                } else {
-                    // token j: column j (x, or h's bf16 high part) + column 8 + j
-                    // (zero for gate/up, h's low part for down)
-#pragma unroll
-                    for (int m = 0; m < NMAT; ++m) {
-                        uint32_t r[8], q[8];
-                        umma::ld8(tbase + lb + (uint32_t)((buf * NMAT + m) * 64), r);
-                        umma::ld8(tbase + lb + (uint32_t)((buf * NMAT + m) * 64 + 8), q);
-                        umma::wait_ld();
-#pragma unroll
-                        for (int j = 0; j < kGroup; ++j) acc[m][j] = __uint_as_float(r[j]) + __uint_as_float(q[j]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int m = 0; m < (PF ? 0 : NMAT); ++m) {
+            for (int m = 0; m < NMAT; ++m) {
 #pragma unroll
                 for (int n0 = 0; n0 < kNMax; n0 += 8) {
                     if (n0 < N) {
@@ -905,7 +670,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 for (int m = 0; m < NMAT; ++m)
 #pragma unroll
                     for (int t = 0; t < kChunk; ++t)
-                        if (t < tv) sp[(m * kChunk + t) * kTileM + rowl] = acc[m][t];
+                        if (t < Tc) sp[(m * kChunk + t) * kTileM + rowl] = acc[m][t];
                 umma::bar_sync(1, 128);
                 const int c0 = owner(x.istart), c1 = owner(x.iend - 1);
                 if (threadIdx.x == 0) {
@@ -929,66 +694,12 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                         for (int m = 0; m < NMAT; ++m)
 #pragma unroll
                             for (int t = 0; t < kChunk; ++t)
-                                if (t < tv) acc[m][t] += __ldcg(q + (m * kChunk + t) * kTileM + rowl);
+                                if (t < Tc) acc[m][t] += __ldcg(q + (m * kChunk + t) * kTileM + rowl);
                     }
                 }
             }
             if (fin) {
-                if constexpr (PF) {
-                    const int gl = x.u - g_lo;
-                    const bool ok = (g_nok[gl] >> 8) != 0;
-                    if constexpr (GU) {
-                        const int f = x.rb * kTileM + rowl;  // ff (or ff_s) row of this thread
-                        if (!x.shared) {
-                            // w*h of the group's tokens -> the group's down B operand
-                            const int nkt_ff = ceil_div(p.ff, kTileK);
-                            const int blk = x.rb * 4 + warp;  // 32-row block of ff
-                            const int kt = blk >> 3;
-                            const size_t tb = (size_t)x.u * nkt_ff + kt;
-                            uint8_t *tile = p.ws + p.P.hb + tb * kPfN * 128;
-                            uint8_t *sfw = p.ws + p.P.hsf + tb * 2 * kSfRow * 4;
-#pragma unroll
-                            for (int j = 0; j < kGroup; ++j) {
-                                if (j < tv) {
-                                    float h = 0.f;
-                                    if (ok && f < p.ff) h = silu_mul(acc[0][j], acc[1][j]) * g_w[gl * kGroup + j];
-                                    quantize_pieces_t<kPfPieces, true>(h, lane, j, blk & 7, kPfN, kSfRow, tile, sfw);
-                                }
-                            }
-                        } else if (f < p.ffs) {
-                            // shared: h as bf16 hi (row j) + lo (row 8 + j), weight 1
-                            const int gs = x.u - U;
-                            const int nkts_ff = ceil_div(p.ffs, kTileKs);
-                            uint8_t *tile = p.ws + p.P.hsb + ((size_t)gs * nkts_ff + f / kTileKs) * kPfNs * 128;
-                            const int c = (f % kTileKs) / 8, e = f % 8;
-#pragma unroll
-                            for (int j = 0; j < kGroup; ++j) {
-                                if (j < tv) {
-                                    const float h = silu_mul(acc[0][j], acc[1][j]);
-                                    const __nv_bfloat16 hi = __float2bfloat16_rn(h);
-                                    const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
-                                    *reinterpret_cast<__nv_bfloat16 *>(tile + (c * 2) * 128 + j * 16 + e * 2) = hi;
-                                    *reinterpret_cast<__nv_bfloat16 *>(tile + (c * 2 + 1) * 128 + j * 16 + e * 2) = lo;
-                                }
-                            }
-                        }
-                    } else {
-                        // down: this item's rows of o[token][slot] (slot k: the shared expert)
-                        const int row = x.rb * kTileM + rowl;
-                        if (row < p.d) {
-                            float *o = reinterpret_cast<float *>(p.ws + p.P.o);
-#pragma unroll
-                            for (int j = 0; j < kGroup; ++j) {
-                                if (j < tv) {
-                                    const int pid = g_pair[gl * kGroup + j];
-                                    const int t = x.shared ? pid : pid / p.k;
-                                    const int slot = x.shared ? p.k : pid - t * p.k;
-                                    o[((size_t)t * (p.k + 1) + slot) * p.d + row] = acc[0][j];
-                                }
-                            }
-                        }
-                    }
-                } else if constexpr (GU) {
+                if constexpr (GU) {
                     const int f = x.rb * kTileM + rowl;  // ff (or ff_s) row of this thread
                     if (!x.shared) {
                         const uint8_t *blob = ublob[x.u];

@@ -307,10 +307,10 @@ def test_grouped_prefill_matches_chunked_path(orc):
 
 
 def test_grouped_prefill_deterministic_and_multi_pass(orc):
-    """k=32 of 64 experts on a tiny shape needs several passes for 6000 tokens
-    (each CTA's group table is bounded); two calls give the same bytes."""
+    """More tokens than one prefill pass takes (8192): two passes; two calls
+    give the same bytes."""
     cfg = k3gen.Config("pf_pass", d=256, ff=128, E=64, k=32, ff_shared=128, T=0, bias="normal")
-    T = 6000
+    T = 8192 + 700
     W = kdev.weights(cfg)
     inp = kdev.DeviceInputs(cfg, T=T)
     a = run_layer(cfg, W, inp.x, inp.bias, T, m.K3MOE_OUT_FP32)
