@@ -368,7 +368,7 @@ k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims
         up.ngs = pp.ngs;
         up.blobs = rp.blobs;
         for (int gu = 1; gu >= 0; --gu) {
-            const int sb = umma_stage_bytes(gu != 0, kPfN);
+            const int sb = pf_stage_bytes(gu != 0);
             int nst = (kSmemLimit - pf_smem_bytes(gu != 0, 0)) / sb;
             if (nst > 8) nst = 8;
             up.nst = nst;

@@ -110,18 +110,18 @@ __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int f
 // ---------------------------------------------------------------- prefill --
 // Grouped prefill (more than kChunk tokens): the pairs (token, slot) are
 // sorted by expert and each expert's pairs cut into groups of up to kGroup
-// tokens; a tensor-core item is (group, 128 weight rows), and the items of
-// one expert's row block are consecutive, so the CTAs that run them side by
-// side read each weight tile from HBM once and from L2 for the other groups.
-// The shared expert takes groups of kGroup consecutive tokens.  Activations
-// enter as kPfPieces E2M1 pieces per element: token j of a group owns B rows
-// 4j..4j+3 (half a core matrix), so its 64 bytes per 16-byte chunk of a
-// K-tile are one contiguous copy.
-constexpr int kGroup = 16;      // tokens per group
+// tokens; a tensor-core item is (group, 128 weight rows).  Items run in group
+// order, row blocks innermost, dealt round-robin to the CTAs: the CTAs that
+// run side by side share the groups' B tiles and the experts' weight tiles
+// through L2.  The shared expert takes groups of kGroup consecutive tokens.
+// Activations enter as kPfPieces E2M1 pieces per element (B rows 4j..4j+3 for
+// token j of a group); each group's B operand is written once per call, in
+// the MMA's layout, by the pass that quantises x.
+constexpr int kGroup = 32;      // tokens per group
 constexpr int kPfPieces = 4;    // pieces per activation element (rows per token)
-constexpr int kPfN = kGroup * kPfPieces;  // 64: MMA N of a routed group
-constexpr int kPfNsGU = kGroup;           // 16: shared gate/up (x as bf16, one row per token)
-constexpr int kPfNsDn = 2 * kGroup;       // 32: shared down (h as bf16 high rows, then low rows)
+constexpr int kPfN = kGroup * kPfPieces;  // 128: MMA N of a routed group
+constexpr int kPfNsGU = kGroup;           // 32: shared gate/up (x as bf16, one row per token)
+constexpr int kPfNsDn = 2 * kGroup;       // 64: shared down (h as bf16 high rows, then low rows)
 constexpr int kPfMaxTokens = 8192;        // tokens per prefill pass
 constexpr int kPfHistTok = 16;            // tokens per block of the dispatch histogram
 
@@ -135,16 +135,19 @@ struct PLayout {
     size_t eoff;   // u32 [E] first position of each expert in perm
     size_t goff;   // u32 [E] first group of each expert
     size_t perm;   // i32 [Tp*k] pair ids t*k+j sorted by (expert, token)
+    size_t pw;     // f32 [Tp*k] their routing weights, in the same order
     size_t grp;    // int4 [ngr + ngs] routed groups then shared groups: (expert or -1,
                    // first position / first token, tokens, blob ok)
-    size_t itg;    // i32 [ngr*nrb_ff + ngs*nrbs_ff] gate/up items in run order: group | rb << 20
-    size_t itd;    // i32 [(ngr + ngs)*nrb_d] down items in run order
-    size_t xp;     // u8 [Tp][nkt_d][8 chunks][4 pieces][16 B] pieces of x per token
-    size_t xps;    // u8 [Tp][nkt_d][2][4 pieces][4] their scales ([group of 4 blocks][piece][block])
+    size_t itg;    // int4 [ngr*nrb_ff + ngs*nrbs_ff] gate/up items in run order: (group | rb << 20,
+                   // expert or -1, first position / first token, tokens | blob ok << 8)
+    size_t itd;    // int4 [(ngr + ngs)*nrb_d] down items in run order
+    size_t ploc;   // i32 [Tp*k] group * kGroup + slot in the group of each pair t*k+j
+    size_t xg;     // u8 [ngr][nkt_d][kPfN*128] pieces of x per routed group (gate/up B)
+    size_t xgs;    // u32 [ngr][nkt_d][2][kPfN] their scales (word = 4 blocks of one row)
     size_t xbf;    // u8 [ngs][nkts_d][kPfNsGU*128] x as bf16 per shared group
     size_t hb;     // u8 [ngr][nkt_ff][kPfN*128] w*h pieces per routed group (down B)
-    size_t hsf;    // u32 [ngr][nkt_ff][2][kSfRow]
-    size_t hsb;    // u8 [ngs][nkts_ff][kPfNsDn*128] shared h as bf16 high (rows 0-15), low (16-31)
+    size_t hsf;    // u32 [ngr][nkt_ff][2][kPfN] their scales (word = 4 blocks of one row)
+    size_t hsb;    // u8 [ngs][nkts_ff][kPfNsDn*128] shared h as bf16 high (rows 0-31), low (32-63)
     size_t o;      // f32 [Tp][k+1][d] expert outputs per (token, slot); slot k: shared
     size_t total;  // end offset (absolute: the prefill region follows the decode layout)
     int Tp, ngr, ngs, nhb;
@@ -178,14 +181,16 @@ __host__ __device__ inline PLayout make_playout(size_t base, int d, int ff, int 
     take(P.eoff, (size_t)E * 4);
     take(P.goff, (size_t)E * 4);
     take(P.perm, (size_t)Tp * k * 4);
+    take(P.pw, (size_t)Tp * k * 4);
     take(P.grp, (size_t)(P.ngr + P.ngs) * 16);
-    take(P.itg, ((size_t)P.ngr * nrb_ff + (size_t)P.ngs * nrbs_ff) * 4);
-    take(P.itd, (size_t)(P.ngr + P.ngs) * nrb_d * 4);
-    take(P.xp, (size_t)Tp * nkt_d * 8 * kPfPieces * 16);
-    take(P.xps, (size_t)Tp * nkt_d * 2 * kPfPieces * 4);
+    take(P.itg, ((size_t)P.ngr * nrb_ff + (size_t)P.ngs * nrbs_ff) * 16);
+    take(P.itd, (size_t)(P.ngr + P.ngs) * nrb_d * 16);
+    take(P.ploc, (size_t)Tp * k * 4);
+    take(P.xg, (size_t)P.ngr * nkt_d * kPfN * 128);
+    take(P.xgs, (size_t)P.ngr * nkt_d * 2 * kPfN * 4);
     take(P.xbf, (size_t)P.ngs * nkts_d * kPfNsGU * 128);
     take(P.hb, (size_t)P.ngr * nkt_ff * kPfN * 128);
-    take(P.hsf, (size_t)P.ngr * nkt_ff * 2 * kSfRow * 4);
+    take(P.hsf, (size_t)P.ngr * nkt_ff * 2 * kPfN * 4);
     take(P.hsb, (size_t)P.ngs * nkts_ff * kPfNsDn * 128);
     take(P.o, (size_t)Tp * (k + 1) * d * 4);
     P.total = o;

@@ -250,77 +250,109 @@ __global__ void __launch_bounds__(kRouteThreads) pf_place_kernel(const __grid_co
     __syncthreads();
     const uint32_t *hist = reinterpret_cast<const uint32_t *>(p.r.ws + p.P.hist) + (size_t)blockIdx.x * E;
     const uint32_t *eoff = reinterpret_cast<const uint32_t *>(p.r.ws + p.P.eoff);
+    const uint32_t *goff = reinterpret_cast<const uint32_t *>(p.r.ws + p.P.goff);
+    int32_t *ploc = reinterpret_cast<int32_t *>(p.r.ws + p.P.ploc);
     int32_t *perm = reinterpret_cast<int32_t *>(p.r.ws + p.P.perm);
+    float *pw = reinterpret_cast<float *>(p.r.ws + p.P.pw);
+    const float *wt = reinterpret_cast<const float *>(p.r.ws + p.P.wt);
     for (int i = threadIdx.x; i < (t1 - t0) * k; i += blockDim.x) {
         const int e = s_idx[i], tl = i / k;
         uint32_t r = 0u;  // pairs of expert e at earlier tokens of the block (one per token at most)
         for (int q = 0; q < tl * k; ++q) r += s_idx[q] == e ? 1u : 0u;
-        perm[eoff[e] + hist[e] + r] = (t0 + tl) * k + (i - tl * k);
+        const int pid = (t0 + tl) * k + (i - tl * k);
+        const uint32_t rel = hist[e] + r;  // rank among expert e's pairs
+        perm[eoff[e] + rel] = pid;
+        pw[eoff[e] + rel] = wt[pid];
+        ploc[pid] = (int)((goff[e] + rel / kGroup) * kGroup + rel % kGroup);
     }
 }
 
-// Items of the expert kernels in run order: for each expert, for each 128-row
-// block, its groups (so the groups sharing a weight tile run side by side);
-// then the shared expert's items, row block by row block.  Entry: group |
-// row block << 20.  One thread per (group, row block).
+// Items of the expert kernels in run order: group by group (an expert's
+// groups are consecutive), its 128-row blocks innermost; the shared expert's
+// groups last.  Entry: (group | row block << 20, expert or -1, first position
+// or token, tokens | blob ok << 8).  One thread per (group, row block).
 __global__ void pf_items_kernel(const __grid_constant__ PfRouteParams p) {
     const uint8_t *ws = p.r.ws;
     const int NG = (int)*reinterpret_cast<const volatile uint32_t *>(
         &reinterpret_cast<const WsHeader *>(ws + p.r.L.hdr)->n_unique);
     const int4 *grp = reinterpret_cast<const int4 *>(ws + p.P.grp);
-    const uint32_t *ecnt = reinterpret_cast<const uint32_t *>(ws + p.P.ecnt);
-    const uint32_t *goff = reinterpret_cast<const uint32_t *>(ws + p.P.goff);
-    int32_t *itg = reinterpret_cast<int32_t *>(p.r.ws + p.P.itg);
-    int32_t *itd = reinterpret_cast<int32_t *>(p.r.ws + p.P.itd);
+    int4 *itg = reinterpret_cast<int4 *>(p.r.ws + p.P.itg);
+    int4 *itd = reinterpret_cast<int4 *>(p.r.ws + p.P.itd);
     const int nrb_ff = ceil_div(p.ff, kTileM), nrb_d = ceil_div(p.r.d, kTileM);
     const int nrbs_ff = p.ngs > 0 ? ceil_div(p.ffs, kTileM) : 0;
     const int per = nrb_ff > nrb_d ? nrb_ff : nrb_d;
     const long long n = (long long)(NG + p.ngs) * per;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
         const int g = (int)(i / per), rb = (int)(i - (long long)g * per);
+        const int4 gr = __ldcg(grp + g);  // (expert or -1, first position / token, tokens, blob ok)
+        const int4 rec = make_int4(g | (rb << 20), gr.x, gr.y, gr.z | (gr.w << 8));
         if (g < NG) {
-            const int e = __ldcg(&grp[g].x);
-            const int ng = (int)((__ldcg(ecnt + e) + kGroup - 1) / kGroup), j = g - (int)__ldcg(goff + e);
-            const int base = (int)__ldcg(goff + e);
-            if (rb < nrb_ff) itg[base * nrb_ff + rb * ng + j] = g | (rb << 20);
-            if (rb < nrb_d) itd[base * nrb_d + rb * ng + j] = g | (rb << 20);
+            if (rb < nrb_ff) itg[(size_t)g * nrb_ff + rb] = rec;
+            if (rb < nrb_d) itd[(size_t)g * nrb_d + rb] = rec;
         } else {
             const int s = g - NG;
-            if (rb < nrbs_ff) itg[NG * nrb_ff + rb * p.ngs + s] = g | (rb << 20);
-            if (rb < nrb_d) itd[NG * nrb_d + rb * p.ngs + s] = g | (rb << 20);
+            if (rb < nrbs_ff) itg[(size_t)NG * nrb_ff + (size_t)s * nrbs_ff + rb] = rec;
+            if (rb < nrb_d) itd[(size_t)NG * nrb_d + (size_t)s * nrb_d + rb] = rec;
         }
     }
 }
 
 // -------------------------------------------------------------- x pieces --
-// Every token's x as kPfPieces E2M1 pieces: per K-tile, [chunk][piece][16 B]
-// (64 contiguous bytes per chunk: the token's half core matrix) and the
-// scales [group of 4 blocks][piece][block]; with a shared expert, x as bf16
-// in the shared groups' tiles (MMA N = 16 rows, one per token; the rows of
-// absent tokens zero).  Warps over (token, 32-block).
+// x as kPfPieces E2M1 pieces, written straight into the B tile of every group
+// that has the token (the gate/up MMA's layout: chunk c of B row 4s + piece
+// at c*(kPfN/8)*128 + (row/8)*128 + (row%8)*16, scale words [2][kPfN]).  One
+// warp per (token, K-tile): the 8 blocks of 32 are quantised into a
+// shared-memory staging block, then lane 4c + piece holds chunk c's 16 bytes
+// of that piece and stores them for each of the token's k groups.  With a
+// shared expert, x also goes as bf16 into the shared groups' tiles (MMA N =
+// 32 rows, one per token; rows of absent tokens zero).
+constexpr int kPrepWarps = kRouteThreads / 32;
+
 __global__ void __launch_bounds__(kRouteThreads) pf_prep_kernel(const __grid_constant__ PfRouteParams p) {
-    const int lane = threadIdx.x & 31, d = p.r.d, nb = d / 32, nkt = ceil_div(d, kTileK);
+    __shared__ __align__(16) uint8_t stage[kPrepWarps][8][kPfPieces][16];
+    __shared__ __align__(16) uint8_t sstage[kPrepWarps][2][kPfPieces][4];
+    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5, d = p.r.d, k = p.r.k;
+    const int nkt = ceil_div(d, kTileK), nb = d / 32;
     const int nkts = ceil_div(d, kTileKs);
-    const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), nw = gridDim.x * (blockDim.x >> 5);
+    const int gw = blockIdx.x * kPrepWarps + wl, nw = gridDim.x * kPrepWarps;
     uint8_t *ws = p.r.ws;
+    const int32_t *ploc = reinterpret_cast<const int32_t *>(ws + p.P.ploc);
     const int Tpad = p.ngs > 0 ? p.ngs * kGroup : p.T;
-    for (int i = gw; i < Tpad * nb; i += nw) {
-        const int t = i / nb, b = i - t * nb;
-        const int col = 32 * b + lane;
+    for (int i = gw; i < Tpad * nkt; i += nw) {
+        const int t = i / nkt, kt = i - t * nkt;
         const bool real = t < p.T;
-        const uint16_t xv = real ? p.r.x[(size_t)t * d + col] : (uint16_t)0;
-        if (real) {
-            const float v = __uint_as_float((uint32_t)xv << 16);
-            const size_t blk = (size_t)t * nkt + (b >> 3);
-            quantize_pieces_t<kPfPieces>(v, lane, 0, b & 7, kPfPieces * 16, 0, kPfPieces,
-                                         ws + p.P.xp + blk * (8 * kPfPieces * 16), ws + p.P.xps + blk * (2 * kPfPieces * 4));
+        const int nbk = min(8, nb - kt * 8);  // 32-blocks in this K-tile
+        if (lane < 8) *reinterpret_cast<uint32_t *>(&sstage[wl][lane >> 2][lane & 3][0]) = 0u;
+        __syncwarp();
+        for (int c = 0; c < nbk; ++c) {
+            const int col = 32 * (kt * 8 + c) + lane;
+            const uint16_t xv = real ? p.r.x[(size_t)t * d + col] : (uint16_t)0;
+            if (real)
+                quantize_pieces_t<kPfPieces>(__uint_as_float((uint32_t)xv << 16), lane, 0, c, kPfPieces * 16, 0,
+                                             kPfPieces, &stage[wl][0][0][0], &sstage[wl][0][0][0]);
+            if (p.ngs > 0) {
+                const int gs = t / kGroup, j = t - gs * kGroup;
+                uint8_t *tile = ws + p.P.xbf + ((size_t)gs * nkts + col / kTileKs) * kPfNsGU * 128;
+                const int cc = (col % kTileKs) / 8, e = col % 8;
+                *reinterpret_cast<uint16_t *>(tile + cc * (kPfNsGU / 8) * 128 + (j / 8) * 128 + (j % 8) * 16 + e * 2) = xv;
+            }
         }
-        if (p.ngs > 0) {
-            const int gs = t / kGroup, j = t - gs * kGroup;
-            uint8_t *tile = ws + p.P.xbf + ((size_t)gs * nkts + col / kTileKs) * kPfNsGU * 128;
-            const int c = (col % kTileKs) / 8, e = col % 8;
-            *reinterpret_cast<uint16_t *>(tile + c * (kPfNsGU / 8) * 128 + (j / 8) * 128 + (j % 8) * 16 + e * 2) = xv;
+        if (!real) continue;
+        __syncwarp();
+        const int c = lane >> 2, pc = lane & 3;
+        const uint4 row = c < nbk ? *reinterpret_cast<const uint4 *>(&stage[wl][c][pc][0]) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t sw = lane < 8 ? *reinterpret_cast<const uint32_t *>(&sstage[wl][lane >> 2][lane & 3][0]) : 0u;
+        const int myloc = lane < k ? __ldcg(ploc + (size_t)t * k + lane) : 0;
+        for (int j = 0; j < k; ++j) {
+            const int loc = __shfl_sync(0xffffffffu, myloc, j);
+            const int g = loc / kGroup, s = loc - g * kGroup;
+            const size_t tb = (size_t)g * nkt + kt;
+            uint8_t *tile = ws + p.P.xg + tb * kPfN * 128;
+            *reinterpret_cast<uint4 *>(tile + c * (kPfN / 8) * 128 + (s >> 1) * 128 + (s & 1) * 64 + pc * 16) = row;
+            if (lane < 8)
+                reinterpret_cast<uint32_t *>(ws + p.P.xgs + tb * 2 * kPfN * 4)[(lane >> 2) * kPfN + 4 * s + (lane & 3)] = sw;
         }
+        __syncwarp();
     }
 }
 

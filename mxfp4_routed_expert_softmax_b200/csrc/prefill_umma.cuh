@@ -5,18 +5,17 @@
 //
 // Items are (group of up to kGroup tokens of one expert, 128 weight rows) and
 // run whole on one CTA; CTA c takes items c, c + G, c + 2G, ... of a list in
-// which the groups of one expert's row block are consecutive.  So at any time
-// the CTAs work on the same few weight tiles for different token groups, in
-// step (every routed item has the same length): each tile comes from HBM once
-// and from L2 for the other groups.  The shared expert's items (bf16 weights,
+// group order with the row blocks innermost.  So at any time the CTAs work on
+// a few groups of a few experts, in step (every routed item has the same
+// length): a group's B tile is read by the CTAs of its row blocks at about
+// the same time, and an expert's weight tiles by the CTAs of its groups, so
+// most of both come from L2.  The shared expert's items (bf16 weights,
 // kind::f16) follow the routed ones.
 //
 // Warps: 0-3 epilogue (TMEM lane quadrants), 4-7 scale factors into TMEM,
-// 8 copies (lane 0: weight tiles by TMA; all lanes: the gather of the group's
-// token pieces by 16-byte asynchronous copies, whose completion each lane
-// reports to the stage's barrier -- a bulk copy per 64-byte piece would
-// serialise on the TMA unit), 9 MMA issue, 10 loads each item's group
-// description into a ring of shared-memory slots ahead of use.
+// 8 copies (TMA weight tiles, bulk copies of the group's B tile), 9 MMA issue,
+// 10 loads each item's group description into a ring of shared-memory slots
+// ahead of use.
 #pragma once
 
 #include "common.cuh"
@@ -28,22 +27,6 @@ namespace k3 {
 
 constexpr int kPfThreads = 352;
 constexpr int kPfSlots = 4;  // group descriptions in flight
-
-// 16-byte asynchronous copy global -> shared (L2 only), and the arrival on
-// `bar` once every such copy this thread issued has landed (the barrier's
-// expected count includes it).
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-// Generic-proxy writes to shared memory (the copies above) -> visible to the
-// tensor core's reads (async proxy) after this fence.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 struct PfUmmaParams {
     int d, ff, k, ffs;
@@ -58,17 +41,25 @@ struct PfUmmaParams {
 
 struct PfSlot {
     int32_t eid;         // expert (-1: shared)
-    int32_t g;           // group index (shared: ngr_used + s)
+    int32_t g;           // group index (shared: routed groups + s)
     int32_t rb;          // 128-row block of the item
     int32_t n;           // tokens
     int32_t ok;          // the expert's blob passed its check
     int32_t pad[3];
     int32_t pair[kGroup];  // t*k + slot (shared: token)
+    int32_t orow[kGroup];  // output row t*(k+1) + slot (shared: slot k)
     float w[kGroup];       // routing weight (shared: 1)
 };
 
+// One pipeline stage: the weight boxes (16 KB per matrix, 1024-byte aligned
+// for the 128-byte swizzle), the B tile (kPfN rows x 128 bytes), the weight
+// scale boxes (128 rows x 16 bytes per matrix) and the B scale words
+// (2 groups x kPfN rows), rounded up to 1024 bytes.
+__host__ __device__ inline int pf_sfa_off(bool gu) { return (gu ? 2 : 1) * kAtile + kPfN * 128; }
+__host__ __device__ inline int pf_sfb_off(bool gu) { return pf_sfa_off(gu) + (gu ? 2 : 1) * 2048; }
+__host__ __device__ inline int pf_stage_bytes(bool gu) { return (pf_sfb_off(gu) + 2 * kPfN * 4 + 1023) & ~1023; }
 __host__ __device__ inline int pf_smem_bytes(bool gu, int nst) {
-    return 1024 + nst * umma_stage_bytes(gu, kPfN) + 512 + kPfSlots * (int)sizeof(PfSlot);
+    return 1024 + nst * pf_stage_bytes(gu) + 512 + kPfSlots * (int)sizeof(PfSlot);
 }
 
 template <bool GU>
@@ -76,7 +67,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     constexpr int NMAT = GU ? 2 : 1;
-    constexpr int SFC = GU ? 32 : 16;   // TMEM scale columns per stage
+    // accumulators: gate/up one buffer (two matrices of kPfN columns), down two
+    // buffers; then the scale columns of each stage (8-aligned groups)
+    constexpr int NBUF = GU ? 1 : 2;
+    constexpr int SFC = GU ? 32 : 16;
     constexpr int NS = GU ? kPfNsGU : kPfNsDn;  // MMA N of a shared item
     const int nst = p.nst, SB = p.sb;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + nst * SB);
@@ -94,7 +88,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + L.hdr);
     if (threadIdx.x == 0) {
         for (int s = 0; s < nst; ++s) {
-            mbar_init(&full[s], GU ? 33 : 1);  // gate/up: + the 32 copy lanes
+            mbar_init(&full[s], 1);
             mbar_init(&sfr[s], 4);
             mbar_init(&empty[s], 1);
         }
@@ -109,7 +103,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
         fence_mbar_init();
         *s_abort = 0;
     }
-    constexpr uint32_t kCols = GU ? 512u : 256u;
+    constexpr uint32_t kCols = 512u;
     if (warp == 0) umma::tmem_alloc(tslot, kCols);
     umma::fence_before();
     __syncthreads();
@@ -130,11 +124,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
     const int NI = IR + p.ngs * nrbs;        // all items
     const int G = gridDim.x, cta = blockIdx.x;
     const int nmine = cta < NI ? (NI - cta + G - 1) / G : 0;  // this CTA's items
-    const int32_t *items = reinterpret_cast<const int32_t *>(p.ws + (GU ? p.P.itg : p.P.itd));
+    const int4 *items = reinterpret_cast<const int4 *>(p.ws + (GU ? p.P.itg : p.P.itd));
     const size_t mat = (size_t)p.d * p.ff;
     const uint8_t *smaps = p.ws + L.tmap + (size_t)L.E * kMapsPerExpert * 128;
     const uint32_t idesc4 = umma::idesc_mxf4(kPfN), idesc16 = umma::idesc_bf16(NS);
-    const uint32_t sf0 = GU ? 256u : 128u;
+    const uint32_t sf0 = (uint32_t)(NBUF * NMAT * kPfN);
     auto item_of = [&](int q) { return cta + q * G; };
     auto nk_of = [&](int it) { return it < IR ? nkt : nkts; };
     auto wait = [&](uint64_t *bar, uint32_t parity) {
@@ -157,39 +151,50 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
 
     if (warp == 10) {
         // ---------------------------------------------- group descriptions --
-        const int4 *grp = reinterpret_cast<const int4 *>(p.ws + p.P.grp);
+        // Two items in flight: the record of item q+2 and the pairs of item
+        // q+1 load while item q's slot is written.
         const int32_t *perm = reinterpret_cast<const int32_t *>(p.ws + p.P.perm);
-        const float *pwt = reinterpret_cast<const float *>(p.ws + p.P.wt);
+        const float *pw = reinterpret_cast<const float *>(p.ws + p.P.pw);
+        auto pairs_of = [&](const int4 &rec, int &pid, float &w) {
+            const int n = rec.w & 255;
+            pid = 0;
+            w = 0.f;
+            if (lane < n) {
+                if (rec.y >= 0) {
+                    pid = __ldcg(perm + rec.z + lane);
+                    w = __ldcg(pw + rec.z + lane);
+                } else {
+                    pid = rec.z + lane;
+                    w = 1.f;
+                }
+            }
+        };
+        int4 r1 = make_int4(0, 0, 0, 0), r2 = make_int4(0, 0, 0, 0);
+        int pid1 = 0;
+        float w1 = 0.f;
+        if (nmine > 0) r1 = __ldcg(items + item_of(0));
+        if (nmine > 1) r2 = __ldcg(items + item_of(1));
+        if (nmine > 0) pairs_of(r1, pid1, w1);
         for (int q = 0; q < nmine; ++q) {
+            const int4 rec = r1;
+            const int pid = pid1;
+            const float w = w1;
+            r1 = r2;
+            if (q + 2 < nmine) r2 = __ldcg(items + item_of(q + 2));
+            if (q + 1 < nmine) pairs_of(r1, pid1, w1);
             int go = 1;
             if (lane == 0 && q >= kPfSlots) go = wait(&mempty[q % kPfSlots], (uint32_t)(((q / kPfSlots) + 1) & 1));
             if (!__shfl_sync(0xffffffffu, go, 0)) break;
-            const int it = item_of(q);
-            const int code = __ldcg(items + it);
-            const int g = code & 0xFFFFF, rb = code >> 20;
-            const int4 gr = __ldcg(grp + g);
             PfSlot &sl = slots[q % kPfSlots];
-            if (lane < kGroup) {
-                int pid = 0;
-                float w = 0.f;
-                if (lane < gr.z) {
-                    if (gr.x >= 0) {
-                        pid = __ldcg(perm + gr.y + lane);
-                        w = __ldcg(pwt + pid);
-                    } else {
-                        pid = gr.y + lane;
-                        w = 1.f;
-                    }
-                }
-                sl.pair[lane] = pid;
-                sl.w[lane] = w;
-            }
+            sl.pair[lane] = pid;
+            sl.orow[lane] = rec.y >= 0 ? pid + pid / p.k : pid * (p.k + 1) + p.k;
+            sl.w[lane] = w;
             if (lane == 0) {
-                sl.eid = gr.x;
-                sl.g = g;
-                sl.rb = rb;
-                sl.n = gr.z;
-                sl.ok = gr.w;
+                sl.eid = rec.y;
+                sl.g = rec.x & 0xFFFFF;
+                sl.rb = rec.x >> 20;
+                sl.n = rec.w & 255;
+                sl.ok = rec.w >> 8;
             }
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&mfull[q % kPfSlots])) : "memory");
@@ -214,10 +219,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
                 maps = em + (GU ? 0 : 256);
                 scmaps = em + (GU ? 384 : 640);
             }
-            // this lane's share of the token gather: token j = lane / 2, chunks
-            // 4*(lane & 1) .. +3 and scale group lane & 1
-            const int jt = lane >> 1, half = lane & 1;
-            const int tok = (!shared && jt < n) ? sl->pair[jt] / p.k : 0;
             if (lane == 0 && (shared || ok)) {
                 umma::tmap_acquire(maps);
                 if (GU) umma::tmap_acquire(maps + 128);
@@ -233,15 +234,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
                 if (!__shfl_sync(0xffffffffu, go, 0)) break;
                 uint8_t *st = smem + s * SB;
                 uint8_t *bdst = st + NMAT * kAtile;
-                uint8_t *sfb = st + umma_sfb_off(GU, kPfN);
+                uint8_t *sfb = st + pf_sfb_off(GU);
                 if (lane == 0) {
                     uint32_t tx;
                     if (shared) {
                         tx = (uint32_t)(NMAT * kAtile + NS * 128);
-                    } else if (GU) {
-                        tx = 0u;  // the token gather reports itself (32 lanes)
                     } else {
-                        tx = (uint32_t)(kPfN * 128 + 2 * kSfRow * 4);
+                        tx = (uint32_t)(kPfN * 128 + 2 * kPfN * 4);
                     }
                     if (!shared && ok) tx += (uint32_t)(NMAT * kAtile + (sf_dma ? NMAT * 2048 : 0));
                     mbar_arrive_expect_tx(&full[s], tx);
@@ -250,35 +249,20 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
                         if (GU) umma::tma_load_2d(st + kAtile, maps + 128, kt * 128, rb * kTileM, &full[s]);
                     }
                     if (sf_dma) {
-                        uint8_t *sfa = st + umma_sfa_off(GU, kPfN);
+                        uint8_t *sfa = st + pf_sfa_off(GU);
                         umma::tma_load_2d(sfa, scmaps, (kt >> 1) * 16, rb * kTileM, &full[s]);
                         if (GU) umma::tma_load_2d(sfa + 2048, scmaps + 128, (kt >> 1) * 16, rb * kTileM, &full[s]);
                     }
                     if (shared) {
                         const size_t off = (GU ? p.P.xbf : p.P.hsb) + ((size_t)(g - NG) * nkts + kt) * NS * 128;
                         bulk_g2s(bdst, p.ws + off, (uint32_t)(NS * 128), &full[s]);
-                    } else if (!GU) {
+                    } else {
+                        // the group's B tile (x pieces for gate/up, w*h pieces for down)
                         const size_t blk = (size_t)g * nkt + kt;
-                        bulk_g2s(bdst, p.ws + p.P.hb + blk * kPfN * 128, (uint32_t)(kPfN * 128), &full[s]);
-                        bulk_g2s(sfb, p.ws + p.P.hsf + blk * 2 * kSfRow * 4, (uint32_t)(2 * kSfRow * 4), &full[s]);
+                        bulk_g2s(bdst, p.ws + (GU ? p.P.xg : p.P.hb) + blk * kPfN * 128, (uint32_t)(kPfN * 128), &full[s]);
+                        bulk_g2s(sfb, p.ws + (GU ? p.P.xgs : p.P.hsf) + blk * 2 * kPfN * 4, (uint32_t)(2 * kPfN * 4),
+                                 &full[s]);
                     }
-                }
-                if (GU) {
-                    if (!shared && jt < n) {
-                        // B row 4j + p, chunk c at c*(N/8)*128 + (j/2)*128 + (j%2)*64 + p*16
-                        const size_t blk = (size_t)tok * nkt + kt;
-                        const uint8_t *src = p.ws + p.P.xp + blk * (8 * kPfPieces * 16);
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) {
-                            const int c = 4 * half + cc;
-                            uint8_t *dst = bdst + c * (kPfN / 8) * 128 + (jt >> 1) * 128 + (jt & 1) * 64;
-#pragma unroll
-                            for (int pc = 0; pc < kPfPieces; ++pc) cp_async16(dst + pc * 16, src + c * 64 + pc * 16);
-                        }
-                        // scale words: rows 4j.. of scale group `half`
-                        cp_async16(sfb + (half * kSfRow + 4 * jt) * 4, p.ws + p.P.xps + blk * (2 * kPfPieces * 4) + half * 16);
-                    }
-                    cp_async_arrive(&full[s]);  // every lane, every stage (the barrier expects 33)
                 }
                 if (++s == nst) {
                     s = 0;
@@ -287,7 +271,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
             }
             slot_done(q);
         }
-        cp_async_wait_all();
         if (*s_abort && lane == 0) {
             const uint64_t t0 = globaltimer();
             while (globaltimer() - t0 < 200000ull) {
@@ -322,7 +305,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
                     for (int m = 0; m < NMAT; ++m) {
                         uint32_t w[8];
                         if (p.sf_tma) {
-                            const uint8_t *sfa = st + umma_sfa_off(GU, kPfN) + m * 2048 + (kt & 1) * 8;
+                            const uint8_t *sfa = st + pf_sfa_off(GU) + m * 2048 + (kt & 1) * 8;
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 const uint2 v = ok ? *reinterpret_cast<const uint2 *>(sfa + (32 * j + lane) * 16)
@@ -347,8 +330,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
                         }
                         umma::st8(col + 8 * m, w);
                     }
-                    const uint32_t *sb = reinterpret_cast<const uint32_t *>(st + umma_sfb_off(GU, kPfN));
-                    const uint32_t w[8] = {sb[lane], sb[32 + lane], 0u, 0u, sb[kSfRow + lane], sb[kSfRow + 32 + lane], 0u, 0u};
+                    // B scales: column 4g + n/32, lane n%32
+                    const uint32_t *sb = reinterpret_cast<const uint32_t *>(st + pf_sfb_off(GU));
+                    const uint32_t w[8] = {sb[lane],        sb[32 + lane],        sb[64 + lane],        sb[96 + lane],
+                                           sb[kPfN + lane], sb[kPfN + 32 + lane], sb[kPfN + 64 + lane], sb[kPfN + 96 + lane]};
                     umma::st8(col + 8 * NMAT, w);
                     umma::wait_st();
                 }
@@ -378,10 +363,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
             for (int q = 0; q < nmine && !*s_abort; ++q) {
                 const int it = item_of(q);
                 const bool shared = it >= IR;
-                const int buf = q & 1;
-                if (q >= 2 && !wait(&aempty[buf], (uint32_t)(((q >> 1) + 1) & 1))) break;
+                const int buf = q % NBUF;
+                if (q >= NBUF && !wait(&aempty[buf], (uint32_t)(((q / NBUF) + 1) & 1))) break;
                 umma::fence_after();
-                const uint32_t dcol = tbase + (uint32_t)(buf * NMAT * 64);
+                const uint32_t dcol = tbase + (uint32_t)(buf * NMAT * kPfN);
                 uint32_t acc = 0u;
                 const int nk = nk_of(it);
                 bool go = true;
@@ -390,7 +375,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
                         go = false;
                         break;
                     }
-                    if (GU) fence_proxy_async_smem();  // the copy lanes' B tile
                     umma::fence_after();
                     const uint32_t soff = (uint32_t)(s * SB) >> 4;
                     const uint64_t a0 = adesc0 + soff;
@@ -402,7 +386,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
                             if (sk < nks) {
                                 const uint64_t bd = b0 + sk * bsteps;
                                 umma::mma_bf16(dcol, a0 + 2 * sk, bd, idesc16, acc);
-                                if (GU) umma::mma_bf16(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, idesc16, acc);
+                                if (GU) umma::mma_bf16(dcol + kPfN, a0 + (kAtile >> 4) + 2 * sk, bd, idesc16, acc);
                                 acc = 1u;
                             }
                         }
@@ -418,7 +402,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
                                 const uint32_t sfb = (sfc + 8 * NMAT + (sk >> 1) * 4) | sfid;
                                 umma::mma_mxf4(dcol, a0 + 2 * sk, bd, id4[sk & 1], acc, (sfc + (sk >> 1) * 4) | sfid, sfb);
                                 if (GU)
-                                    umma::mma_mxf4(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, id4[sk & 1], acc,
+                                    umma::mma_mxf4(dcol + kPfN, a0 + (kAtile >> 4) + 2 * sk, bd, id4[sk & 1], acc,
                                                    (sfc + 8 + (sk >> 1) * 4) | sfid, sfb);
                                 acc = 1u;
                             }
@@ -443,46 +427,44 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
             if (!sl) break;
             const int it = item_of(q);
             const bool shared = it >= IR;
-            const int buf = q & 1;
+            const int buf = q % NBUF;
             const int n = sl->n, rb = sl->rb;
             const bool ok = sl->ok != 0;
             int go = 0;
-            if (lane == 0) go = wait(&afull[buf], (uint32_t)((q >> 1) & 1));
+            if (lane == 0) go = wait(&afull[buf], (uint32_t)((q / NBUF) & 1));
             go = __shfl_sync(0xffffffffu, go, 0);
             umma::fence_after();
             float acc[NMAT][kGroup];
             if (!shared) {
-                // token j: the sum of its kPfPieces columns 4j..4j+3
+                // token j: the sum of its kPfPieces columns 4j..4j+3 (32 columns
+                // per TMEM load, one wait per load)
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) {
 #pragma unroll
-                    for (int c8 = 0; c8 < kPfN / 8; ++c8) {
-                        uint32_t r[8];
-                        umma::ld8(tbase + lb + (uint32_t)((buf * NMAT + m) * 64 + 8 * c8), r);
+                    for (int c32 = 0; c32 < kPfN / 32; ++c32) {
+                        uint32_t r[32];
+                        umma::ld32(tbase + lb + (uint32_t)((buf * NMAT + m) * kPfN + 32 * c32), r);
                         umma::wait_ld();
-                        acc[m][2 * c8] = (__uint_as_float(r[0]) + __uint_as_float(r[1])) +
-                                         (__uint_as_float(r[2]) + __uint_as_float(r[3]));
-                        acc[m][2 * c8 + 1] = (__uint_as_float(r[4]) + __uint_as_float(r[5])) +
-                                             (__uint_as_float(r[6]) + __uint_as_float(r[7]));
+#pragma unroll
+                        for (int t = 0; t < 8; ++t)
+                            acc[m][8 * c32 + t] = (__uint_as_float(r[4 * t]) + __uint_as_float(r[4 * t + 1])) +
+                                                  (__uint_as_float(r[4 * t + 2]) + __uint_as_float(r[4 * t + 3]));
                     }
                 }
             } else {
-                // gate/up: column j (x of token j); down: column j (h high) + 16 + j (h low)
+                // gate/up: column j (x of token j); down: column j (h high) + 32 + j (h low)
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) {
+                    uint32_t r[32];
+                    umma::ld32(tbase + lb + (uint32_t)((buf * NMAT + m) * kPfN), r);
+                    umma::wait_ld();
 #pragma unroll
-                    for (int c8 = 0; c8 < kGroup / 8; ++c8) {
-                        uint32_t r[8];
-                        umma::ld8(tbase + lb + (uint32_t)((buf * NMAT + m) * 64 + 8 * c8), r);
+                    for (int jj = 0; jj < kGroup; ++jj) acc[m][jj] = __uint_as_float(r[jj]);
+                    if (!GU) {
+                        umma::ld32(tbase + lb + (uint32_t)((buf * NMAT + m) * kPfN + kGroup), r);
                         umma::wait_ld();
 #pragma unroll
-                        for (int jj = 0; jj < 8; ++jj) acc[m][8 * c8 + jj] = __uint_as_float(r[jj]);
-                        if (!GU) {
-                            umma::ld8(tbase + lb + (uint32_t)((buf * NMAT + m) * 64 + kGroup + 8 * c8), r);
-                            umma::wait_ld();
-#pragma unroll
-                            for (int jj = 0; jj < 8; ++jj) acc[m][8 * c8 + jj] += __uint_as_float(r[jj]);
-                        }
+                        for (int jj = 0; jj < kGroup; ++jj) acc[m][jj] += __uint_as_float(r[jj]);
                     }
                 }
             }
@@ -498,18 +480,23 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
                         const int blk = rb * 4 + warp;  // 32-row block of ff
                         const size_t tb = (size_t)sl->g * nkt_ff + (blk >> 3);
                         uint8_t *tile = p.ws + p.P.hb + tb * kPfN * 128;
-                        uint8_t *sfw = p.ws + p.P.hsf + tb * 2 * kSfRow * 4;
+                        uint8_t *sfw = p.ws + p.P.hsf + tb * 2 * kPfN * 4;
+                        // 4 tokens at a time (absent tokens' rows get zeros; nothing reads them)
 #pragma unroll
-                        for (int j = 0; j < kGroup; ++j) {
-                            if (j < n) {
-                                float h = 0.f;
-                                if (ok && f < p.ff) h = silu_mul(acc[0][j], acc[1][j]) * sl->w[j];
-                                quantize_pieces_t<kPfPieces>(h, lane, j, blk & 7, (kPfN / 8) * 128, 128, kSfRow, tile,
-                                                             sfw);
+                        for (int j0 = 0; j0 < kGroup; j0 += 4) {
+                            if (j0 < n) {
+                                float h[4];
+#pragma unroll
+                                for (int b = 0; b < 4; ++b) {
+                                    const int j = j0 + b;
+                                    h[b] = (ok && f < p.ff && j < n) ? silu_mul(acc[0][j], acc[1][j]) * sl->w[j] : 0.f;
+                                }
+                                quantize_pieces_batch<kPfPieces, 4>(h, lane, j0, blk & 7, (kPfN / 8) * 128, 128, kPfN,
+                                                                    tile, sfw);
                             }
                         }
                     } else if (f < p.ffs) {
-                        // shared: h as bf16 high (row j) + low (row 16 + j), weight 1
+                        // shared: h as bf16 high (row j) + low (row 32 + j), weight 1
                         const int gs = sl->g - NG;
                         const int nkts_ff = ceil_div(p.ffs, kTileKs);
                         uint8_t *tile = p.ws + p.P.hsb + ((size_t)gs * nkts_ff + f / kTileKs) * kPfNsDn * 128;
@@ -535,10 +522,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
 #pragma unroll
                         for (int j = 0; j < kGroup; ++j) {
                             if (j < n) {
-                                const int pid = sl->pair[j];
-                                const int t = shared ? pid : pid / p.k;
-                                const int slot = shared ? p.k : pid - t * p.k;
-                                o[((size_t)t * (p.k + 1) + slot) * p.d + row] = acc[0][j];
+                                o[(size_t)sl->orow[j] * p.d + row] = acc[0][j];
                             }
                         }
                     }

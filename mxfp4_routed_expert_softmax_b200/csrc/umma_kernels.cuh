@@ -83,6 +83,40 @@ __device__ __forceinline__ void quantize_pieces_t(float v, int lane, int t, int 
         if (lane == 0) sfw[((c >> 2) * sfrow + n) * 4 + (c & 3)] = (uint8_t)(e + 127);
     }
 }
+// The same for NB tokens t0..t0+NB-1 at once (values v[b]): the NB chains
+// of dependent steps interleave, so one warp keeps its pipeline busy.
+template <int P, int NB>
+__device__ __forceinline__ void quantize_pieces_batch(const float (&v)[NB], int lane, int t0, int c, int cs, int gs,
+                                                      int sfrow, uint8_t *tile, uint8_t *sfw) {
+    float r[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) r[b] = v[b];
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        uint32_t bits[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) bits[b] = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(r[b])));
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            int e = (int)(bits[b] >> 23) - 127 - 2 + ((bits[b] & 0x7FFFFFu) > 0x400000u ? 1 : 0);
+            e = max(-126, min(126, e));
+            const float s = r[b] * exp2i(-e);
+            const float m = fabsf(s);
+            const float C = m < 2.f ? 4194304.f : (m < 4.f ? 8388608.f : 16777216.f);
+            const float q = __fsub_rn(__fadd_rn(m, C), C);
+            const uint32_t qb = __float_as_uint(q);
+            uint32_t code = q >= 1.f ? (qb >> 22) - 252u : (q > 0.f ? 1u : 0u);
+            code |= (s < 0.f && code != 0u) ? 8u : 0u;
+            r[b] = __fmaf_rn(-copysignf(q, s), exp2i(e), r[b]);
+            const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
+            const int n = (t0 + b) * P + p;
+            uint8_t *row = tile + c * cs + (n / 8) * gs + (n % 8) * 16;
+            if ((lane & 1) == 0) row[lane >> 1] = (uint8_t)(code | (hi << 4));
+            if (lane == 0) sfw[((c >> 2) * sfrow + n) * 4 + (c & 3)] = (uint8_t)(e + 127);
+        }
+    }
+}
+
 __device__ __forceinline__ void quantize_pieces(float v, int lane, int t, int c, int N, uint8_t *tile,
                                                 uint8_t *sfw) {
     quantize_pieces_t<kPieces>(v, lane, t, c, (N / 8) * 128, 128, kSfRow, tile, sfw);
