@@ -56,6 +56,30 @@ def alg_bytes(cfg, U):
     return router + shared + experts + act
 
 
+def launches_per_step(cfg, T):
+    """The library's kernel launches for one layer call: 3 per 8-token pass
+    (decode); for more tokens per grouped-prefill pass (up to 8192 tokens):
+    router GEMM (+ its split-K sum), top-k, 4 dispatch kernels, the
+    quantising pass, gate/up, down, combine."""
+    if T <= 8:
+        return 3
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    n = 0
+    for t0 in range(0, T, 8192):
+        tq = min(8192, T - t0)
+        gx, gy = -(-cfg.E // 128), -(-tq // 128)
+        ns = max(1, min(8, cfg.d // 256, -(-(2 * sms) // (gx * gy))))
+        n += 10 + (1 if ns > 1 else 0)
+    return n
+
+
+def layer_flops(cfg, T):
+    """Algorithmic FLOPs of one layer call (2 per multiply-add): router, the
+    k routed experts of every token (gate, up, down), the shared expert."""
+    return 2 * T * (cfg.E * cfg.d + cfg.k * 3 * cfg.d * cfg.ff + 3 * cfg.d * cfg.ff_shared)
+
+
 def gu_bytes(cfg, U, pairs):
     """Algorithmic bytes of one gate/up launch: W_g and W_u of each distinct
     routed expert (nibbles + scales) and of the bf16 shared expert, x in, the
@@ -98,6 +122,20 @@ def captured_traffic(cfg):
     if (cfg.d, cfg.ff, cfg.k, cfg.ff_shared, cfg.T) != (7168, 1536, 16, 1536, 1):
         return None
     return int(fields["traffic_bytes_per_launch"])
+
+
+def load_bf16_peak():
+    """Measured dense bf16 TFLOP/s (burst), else the fallback 1590."""
+    here = os.path.dirname(os.path.abspath(__file__))
+    try:
+        with open(os.path.join(here, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        v = d.get("bf16_tflops")
+        if isinstance(v, dict):
+            v = v.get("value")
+        return float(v)
+    except (OSError, ValueError, TypeError):
+        return 1590.0
 
 
 def load_peaks():
@@ -349,6 +387,25 @@ def main():
                     "traffic": captured_traffic(cfg) if U == 16 else None,
                     "alg_bytes_per_launch": gb}
     layer_gbs = alg_bytes(cfg, U) / (ms_per_step / 1000.0) / 1e9
+    if roofline is None:
+        # many tokens (grouped prefill): the whole layer against its bound.  The
+        # block-scaled fp4 tensor peak is the measured bf16 peak x 4 (the
+        # nominal dense ratio); the layer is HBM-bound when its bytes take
+        # longer at the copy peak than its FLOPs at that tensor peak.
+        fl = layer_flops(cfg, T)
+        tensor_peak = load_bf16_peak() * 4.0
+        t_hbm = alg_bytes(cfg, U) / (peak * 1e9)
+        t_tc = fl / (tensor_peak * 1e12)
+        if t_hbm >= t_tc:
+            roofline = {"bound": "hbm", "kernel": "layer (all kernels of the grouped prefill)",
+                        "achieved": round(layer_gbs, 1), "peak": peak, "unit": "GB/s",
+                        "frac": round(layer_gbs / peak, 4), "traffic": None,
+                        "alg_bytes_per_launch": alg_bytes(cfg, U)}
+        else:
+            tf = fl / (ms_per_step / 1000.0) / 1e12
+            roofline = {"bound": "tensor", "kernel": "layer (all kernels of the grouped prefill)",
+                        "achieved": round(tf, 2), "peak": round(tensor_peak, 1), "unit": "TFLOP/s",
+                        "frac": round(tf / tensor_peak, 4), "traffic": None, "alg_flops_per_launch": fl}
 
     # end to end: host activations in and out through the C ABI, copies timed
     e2e = None
@@ -381,7 +438,6 @@ def main():
                "sample": f"{n} token(s) of the workload ({t:.1f} s), fp64 scalar C oracle, "
                          f"OpenMP over output rows"}
 
-    chunks = (T + 7) // 8
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -401,7 +457,7 @@ def main():
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 3 * chunks * args.steps,
+        "gpu_launches": launches_per_step(cfg, T) * args.steps,
         "clocks": clk,
     }
     if rank == 0:
