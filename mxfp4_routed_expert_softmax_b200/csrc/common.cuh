@@ -26,7 +26,9 @@ struct WsHeader {
     uint32_t router_done;  // router rows finished in this call; back to 0 by its end
     uint32_t n_unique;     // distinct routed experts in the current token chunk
     uint32_t topk_done;    // tokens whose top-k other CTAs finished; back to 0 by its end
-    uint32_t pad[60];
+    uint32_t prep_done;    // router CTAs whose tensor maps and x pieces are written (decode;
+                           // reset by the down pass)
+    uint32_t pad[59];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 

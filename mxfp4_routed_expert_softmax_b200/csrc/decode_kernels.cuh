@@ -562,7 +562,15 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
     int chunk = 0;
     if (threadIdx.x == 0) router_prefetch(p, ring, full, nstage, 0);  // pass 0's first stages
     // while the first router stages are in flight
-    if (p.blobs != nullptr) refresh_tmaps(p, blockIdx.x * kRouteThreads + threadIdx.x, G * kRouteThreads);
+    if (p.blobs != nullptr) {
+        refresh_tmaps(p, blockIdx.x * kRouteThreads + threadIdx.x, G * kRouteThreads);
+        if (blockIdx.x == 0 && G > 1) {
+            // CTA 0 builds no x pieces: its maps are all it publishes to the
+            // gate/up pass's shared units (the other CTAs count after their pieces)
+            __syncthreads();
+            if (threadIdx.x == 0) red_add_release(&hdr->prep_done, 1u);
+        }
+    }
     for (int pass = 0; pass < npass; ++pass) {
         const int t0 = pass * kRouteTok;
         const int nt = min(kRouteTok, p.Tc - t0);
@@ -589,7 +597,11 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
         const int wi = (blockIdx.x - first_cta) * (kRouteThreads / 32) + warp;
         build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L, wi, nworkers * (kRouteThreads / 32), p.has_shared != 0);
     };
-    if (G == 1) prep(0);
+    if (G == 1 && p.blobs != nullptr) {
+        prep(0);
+        __syncthreads();
+        if (threadIdx.x == 0) red_add_release(&hdr->prep_done, 1u);
+    }
     // top-k of this CTA's tokens once every router row is in
     if ((int)blockIdx.x < p.Tc) {
         __syncthreads();
@@ -621,6 +633,10 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
         return;
     }
     prep(1);
+    if (p.blobs != nullptr) {
+        __syncthreads();
+        if (threadIdx.x == 0) red_add_release(&hdr->prep_done, 1u);  // after this CTA's pieces and maps
+    }
 }
 
 struct SingleParams {

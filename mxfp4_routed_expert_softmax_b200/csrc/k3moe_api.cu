@@ -273,7 +273,7 @@ cudaError_t launch_umma(const DeviceInfo &di, UmmaParams up, cudaStream_t st) {
 
 // Router (+ top-k + dispatch + activation pieces) for one chunk.  Cooperative
 // launch: CTA 0 waits on the other CTAs' router rows, so all must be resident.
-cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st) {
+cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st, int *grid_out = nullptr) {
     // one CTA per SM, at most one per router row and one per stage of router
     // bytes; as many ring stages as fit beside x (12 at most)
     const int nt = rp.Tc < kRouteTok ? rp.Tc : kRouteTok;
@@ -286,6 +286,7 @@ cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st) {
     while (nstage > 2 && route_smem_bytes(rp.d, nt, nstage) > di.route_dyn_max) --nstage;
     if (route_smem_bytes(rp.d, nt, nstage) > di.route_dyn_max) return cudaErrorInvalidConfiguration;
     rp.nstage = nstage;
+    if (grid_out) *grid_out = (int)g;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)g);
     cfg.blockDim = dim3(kRouteThreads);
@@ -527,7 +528,8 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         EventHook none;
         EventHook &hk = hook ? *hook : none;
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
-        e = launch_route(*di, rp, st);
+        int route_ctas = 0;
+        e = launch_route(*di, rp, st, &route_ctas);
         if (e != cudaSuccess) return cuda_fail(e, "router launch");
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
 
@@ -541,6 +543,7 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         up.L = L;
         up.out_fp32 = out32;
         up.y = yc;
+        up.route_ctas = route_ctas;
         e = launch_umma<true>(*di, up, st);
         if (e != cudaSuccess) return cuda_fail(e, "gate/up launch");
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);

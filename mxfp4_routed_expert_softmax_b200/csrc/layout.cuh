@@ -45,7 +45,8 @@ struct Layout {
     size_t hsf;        // u32 [umax][nkt_ff][2][kSfRow]
     size_t xbf;        // u8  [ceil(d/64)][N*128] x as bf16 (rows t*kPieces), shared gate/up B
     size_t hsb;        // u8  [ceil(ffs/64)][N*128] shared h as bf16 hi, lo (rows t*kPieces, +1)
-    size_t spart;      // f32 [kMaxCtas][2][2][kChunk][kTileM] split-item partial sums
+    size_t spart;      // f32 [kMaxCtas][4][2][kChunk][kTileM] split-item partial sums (2 unit
+                       // ranges x first/last item of a CTA)
     size_t icnt;       // u32 [umax*nrb_ff + nrb_ffs + nrb_d] arrivals per split item (back to 0)
     size_t total;
     int d, ff, E, k, ffs, umax;
@@ -100,7 +101,7 @@ __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int f
     L.hsb = o;
     o = align256(o + (size_t)(ffs > 0 ? ceil_div(ffs, kTileKs) : 1) * kNMax * 128);
     L.spart = o;
-    o = align256(o + (size_t)kMaxCtas * 2 * 2 * kChunk * kTileM * 4);
+    o = align256(o + (size_t)kMaxCtas * 4 * 2 * kChunk * kTileM * 4);
     L.icnt = o;
     o = align256(o + ((size_t)umax * ceil_div(ff, kTileM) + ceil_div(ffs, kTileM) + ceil_div(d, kTileM)) * 4);
     L.total = o;

@@ -21,10 +21,17 @@
 // (stream-K).  An item split between CTAs is finished by the last one to
 // arrive, summing the per-token partials in piece order (deterministic).
 //
-// CTA roles (320 threads): warps 0-3 epilogue (one TMEM lane quadrant each),
+// CTA roles (352 threads): warps 0-3 epilogue (one TMEM lane quadrant each),
 // warps 4-7 write the scale factors of each stage into TMEM (each writes the
 // same values into its own quadrant, as the MMA reads them replicated),
-// warp 8 issues the TMA / bulk copies, warp 9 issues the MMAs.
+// warp 8 issues the TMA / bulk copies, warp 9 issues the MMAs, warp 10 (gate/
+// up) loads the routing once the router kernel has finished.
+//
+// Gate/up runs two ranges of units, each split over the CTAs: first the
+// shared expert's (they need no routing: x as bf16 and the shared tensor maps
+// are published by the router kernel's CTAs through a counter), then the
+// routed experts'.  So the shared expert streams while the router kernel's
+// last CTAs still run the top-k and the dispatch.
 #pragma once
 
 #include "common.cuh"
@@ -33,7 +40,7 @@
 
 namespace k3 {
 
-constexpr int kUThreads = 320;
+constexpr int kUThreads = 352;
 // Tensor maps per expert in the workspace: W_g, W_u, W_d nibble planes, then
 // (used when the reduction lengths are multiples of 512) their scale planes.
 constexpr int kMapsPerExpert = 6;
@@ -199,6 +206,9 @@ struct UmmaParams {
     // down only
     int out_fp32;     // y in fp32 (else bf16, rounded once)
     void *y;          // [Tc][d] of this chunk
+    // gate/up: router-kernel CTAs that announce their x pieces and tensor maps
+    // in the header's prep_done (0: nothing to wait for)
+    int route_ctas;
 };
 
 // One pipeline stage for MMA width N: the A boxes (16 KB per matrix, first,
@@ -256,9 +266,11 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     uint64_t *empty = sfr + nst;                                       // stage consumed (MMA commit)
     uint64_t *afull = empty + nst;
     uint64_t *aempty = afull + 2;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(aempty + 2);
+    uint64_t *mready = aempty + 2;  // the routing is in shared memory (gate/up)
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(mready + 1);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tslot + 1);
     volatile int *s_last = s_abort + 1;
+    volatile int *s_U = s_last + 1;
     const uint8_t **s_blob = reinterpret_cast<const uint8_t **>(smem + nst * SB + 256);
     int32_t *s_eid = reinterpret_cast<int32_t *>(s_blob + kMetaU);
     float *s_wu = reinterpret_cast<float *>(s_eid + kMetaU);  // [u][t]
@@ -275,6 +287,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             mbar_init(&afull[b], 1);
             mbar_init(&aempty[b], 4);
         }
+        mbar_init(mready, 1);
         fence_mbar_init();
         *s_abort = 0;
     }
@@ -284,28 +297,45 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     __syncthreads();
     umma::fence_after();
     const uint32_t tbase = *tslot;
-    pdl_wait();
-    pdl_trigger();
-
     const int Tc = p.Tc, N = act_n(Tc);
-    const int U = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_unique);
-    {
+    // the routing of the chunk (written by the router kernel) -> shared memory
+    auto load_meta = [&](int i0, int nthr) {
+        const int U = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_unique);
         const uint8_t *const *gb = reinterpret_cast<const uint8_t *const *>(p.ws + L.uniq_blob);
         const int32_t *ge = reinterpret_cast<const int32_t *>(p.ws + L.uniq_eid);
         const uint32_t *gm = reinterpret_cast<const uint32_t *>(p.ws + L.uniq_mask);
         const int8_t *gs = reinterpret_cast<const int8_t *>(p.ws + L.uniq_slot);
         const float *gw = reinterpret_cast<const float *>(p.ws + L.wt);
-        for (int i = threadIdx.x; i < U; i += kUThreads) {
+        for (int i = i0; i < U; i += nthr) {
             s_blob[i] = gb[i];
             s_eid[i] = ge[i];
         }
-        for (int i = threadIdx.x; i < U * kChunk; i += kUThreads) {
+        for (int i = i0; i < U * kChunk; i += nthr) {
             const int u = i / kChunk, t = i - u * kChunk;
             float w = 0.f;
             if (t < Tc && ((gm[u] >> t) & 1u)) w = gw[t * p.k + gs[u * kChunk + t]];
             s_wu[i] = w;
         }
+        return U;
+    };
+    if constexpr (!GU) {
+        pdl_wait();
+        pdl_trigger();
+        const int U0 = load_meta(threadIdx.x, kUThreads);
+        if (threadIdx.x == 0) {
+            *s_U = U0;
+            hdr->prep_done = 0u;  // every gate/up CTA has read it (the gate/up grid is complete)
+        }
         __syncthreads();
+    } else {
+        pdl_trigger();
+        if (warp == 10) {
+            pdl_wait();
+            const int U0 = load_meta(lane, 32);
+            if (lane == 0) *s_U = U0;
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(mready)) : "memory");
+        }
     }
     const int K = GU ? p.d : p.ff;   // routed reduction length
     const int M = GU ? p.ff : p.d;   // routed weight rows
@@ -314,14 +344,48 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     const int nrb = ceil_div(M, kTileM);
     const int nkts = p.ffs > 0 ? ceil_div(Ks, kTileKs) : 0;
     const int nrbs = (GU && p.ffs > 0) ? ceil_div(p.ffs, kTileM) : 0;
-    const int R = GU ? U * nrb * nkt : 0;             // routed units (GU)
-    const int upi = GU ? 0 : U * nkt + nkts;          // units per item (down)
-    const int total = GU ? R + nrbs * nkts : nrb * upi;
-    const int G = min((int)gridDim.x, max(total, 1));
+    const int S = GU ? nrbs * nkts : 0;               // shared units (gate/up: the first range)
+    // down: the routing is known here; gate/up: only after mready
+    int U = GU ? 0 : *s_U;
+    int upi = GU ? 0 : U * nkt + nkts;                // units per item (down)
     const int cta = blockIdx.x;
-    auto start = [&](int c) { return (int)(((long long)c * total) / G); };
-    auto owner = [&](int unit) { return (int)((((long long)unit + 1) * G - 1) / total); };
-    const int a = cta < G ? start(cta) : 0, b = cta < G ? start(cta + 1) : 0;
+    // A range of units [base, base + n) split evenly over the CTAs (CTA c of
+    // G takes [start(c), start(c + 1))); an item cut between CTAs is finished
+    // by the last of them to arrive.
+    struct Range {
+        int base, n, G, a, b;
+    };
+    auto make_range = [&](int base, int n) {
+        Range r;
+        r.base = base;
+        r.n = n;
+        r.G = min((int)gridDim.x, max(n, 1));
+        r.a = cta < r.G && n > 0 ? base + (int)(((long long)cta * n) / r.G) : base;
+        r.b = cta < r.G && n > 0 ? base + (int)(((long long)(cta + 1) * n) / r.G) : base;
+        return r;
+    };
+    auto start = [&](const Range &r, int c) { return r.base + (int)(((long long)c * r.n) / r.G); };
+    auto owner = [&](const Range &r, int unit) {
+        return (int)((((long long)(unit - r.base) + 1) * r.G - 1) / r.n);
+    };
+    // gate/up: [shared units | routed units]; down: [all units | nothing]
+    Range rng[2];
+    rng[0] = GU ? make_range(0, S) : make_range(0, nrb * upi);
+    rng[1] = make_range(0, 0);
+    // gate/up, before the routed range: wait for the routing (lane 0 of the
+    // calling warp waits, the warp follows), then size the routed range
+    auto routed_range = [&](bool warp_wide) {
+        int ok = 1;
+        if (lane == 0) {
+            ok = (!*s_abort && mbar_wait_bounded(mready, 0u, hdr)) ? 1 : 0;
+            if (!ok) *s_abort = 1;
+        }
+        if (warp_wide) ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) return false;
+        U = *s_U;
+        rng[1] = make_range(S, U * nrb * nkt);
+        return true;
+    };
     const size_t mat = (size_t)p.d * p.ff;
     const uint8_t *const *ublob = s_blob;
     const uint8_t *smaps = p.ws + L.tmap + (size_t)L.E * kMapsPerExpert * 128;
@@ -347,21 +411,24 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     auto decode = [&](int unit) {
         Unit x;
         if constexpr (GU) {
-            if (unit < R) {
-                x.item = unit / nkt;
-                x.istart = x.item * nkt;
-                x.iend = x.istart + nkt;
-                x.u = x.item / nrb;
-                x.rb = x.item - x.u * nrb;
-                x.shared = false;
-            } else {
-                const int j = (unit - R) / nkts;
-                x.item = U * nrb + j;
-                x.istart = R + j * nkts;
+            if (unit < S) {
+                // shared item j (counter j), K-tiles of 64 bf16
+                const int j = unit / nkts;
+                x.item = j;
+                x.istart = j * nkts;
                 x.iend = x.istart + nkts;
                 x.u = -1;
                 x.rb = j;
                 x.shared = true;
+            } else {
+                // routed item (u, rb) (counter nrbs + u*nrb + rb)
+                const int ir = (unit - S) / nkt;
+                x.item = nrbs + ir;
+                x.istart = S + ir * nkt;
+                x.iend = x.istart + nkt;
+                x.u = ir / nrb;
+                x.rb = ir - x.u * nrb;
+                x.shared = false;
             }
             x.kt = unit - x.istart;
         } else {
@@ -387,9 +454,9 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     };
     // The unit after x (no divisions): next K-tile, then the next expert
     // (down), then the shared K-tiles; at the end of an item, a full decode.
-    auto advance = [&](const Unit &x, int unit_next) {
+    auto advance = [&](const Unit &x, int unit_next, int end) {
         Unit y = x;
-        if (unit_next >= x.iend) return unit_next < total ? decode(unit_next) : x;
+        if (unit_next >= x.iend) return unit_next < end ? decode(unit_next) : x;
         ++y.kt;
         if constexpr (!GU) {
             if (!y.shared && y.kt == nkt) {
@@ -407,9 +474,27 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
             int last_u = -2;
-            Unit x = a < b ? decode(a) : Unit{};
             uint32_t ph = 0u;  // phase of the current pass over the stages
-            for (int unit = a, it = 0, s = 0; unit < b && !*s_abort; x = advance(x, ++unit), ++it) {
+            int it = 0, s = 0;
+            if (GU && rng[0].a < rng[0].b && p.route_ctas > 0) {
+                // the shared units read x as bf16 and the shared tensor maps,
+                // which the router kernel's CTAs publish by counting prep_done
+                const uint64_t t0 = globaltimer();
+                while (ld_acquire(&hdr->prep_done) < (uint32_t)p.route_ctas) {
+                    __nanosleep(32);
+                    if (globaltimer() - t0 > kWaitLimitNs) {
+                        set_status(hdr, kStTimeout);
+                        *s_abort = 1;
+                        break;
+                    }
+                }
+                asm volatile("fence.proxy.async.global;" ::: "memory");  // before the bulk copies read x
+            }
+            for (int ri = 0; ri < 2 && !*s_abort; ++ri) {
+            if (ri == 1 && (!GU || !routed_range(false))) break;
+            const Range rg = rng[ri];
+            Unit x = rg.a < rg.b ? decode(rg.a) : Unit{};
+            for (int unit = rg.a; unit < rg.b && !*s_abort; x = advance(x, ++unit, rg.b), ++it) {
                 if (it >= nst && !wait(&empty[s], ph ^ 1u)) break;
                 uint8_t *st = smem + s * SB;
                 const uint8_t *blob = x.shared ? nullptr : ublob[x.u];
@@ -460,6 +545,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     ph ^= 1u;
                 }
             }
+            }
             if (*s_abort) {
                 // a wait gave up somewhere: let the copies this thread issued
                 // land (bounded) before the CTA's shared memory goes away
@@ -476,12 +562,20 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             // then move this K-tile's 8 scale bytes of each row (and the B
             // scales) into TMEM.  An expert whose blob failed its check gets
             // zero scale bytes (finite 2^-127), so it adds exactly nothing.
-            Unit x = a < b ? decode(a) : Unit{};
             uint32_t ph = 0u;
-            for (int unit = a, s = 0; unit < b; x = advance(x, ++unit)) {
+            int s = 0;
+            for (int ri = 0; ri < 2; ++ri) {
+            if (ri == 1 && (!GU || !routed_range(true))) break;
+            const Range rg = rng[ri];
+            Unit x = rg.a < rg.b ? decode(rg.a) : Unit{};
+            bool go_on = true;
+            for (int unit = rg.a; unit < rg.b; x = advance(x, ++unit, rg.b)) {
                 int go = 0;
                 if (lane == 0) go = wait(&full[s], ph);
-                if (!__shfl_sync(0xffffffffu, go, 0)) break;
+                if (!__shfl_sync(0xffffffffu, go, 0)) {
+                    go_on = false;
+                    break;
+                }
                 if (!x.shared) {
                     const uint8_t *st = smem + s * SB;
                     const bool has = ublob[x.u] != nullptr;
@@ -512,6 +606,8 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     s = 0;
                     ph ^= 1u;
                 }
+            }
+            if (!go_on) break;
             }
         } else {
         // The global loads of a unit's scales are issued kLook units ahead of
@@ -572,20 +668,26 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             return true;
         };
         SfRegs R4[kLook + 1];
-        const int n = b - a;
-#pragma unroll
-        for (int i = 0; i < kLook; ++i)
-            if (i < n) load(a + i, R4[i]);
         bool go = true;
-        for (int it0 = 0; it0 < n && go; it0 += kLook + 1) {
+        int done = 0;  // stages passed in earlier ranges
+        for (int ri = 0; ri < 2 && go; ++ri) {
+            if (ri == 1 && (!GU || !routed_range(true))) break;
+            const Range rg = rng[ri];
+            const int a = rg.a, n = rg.b - rg.a;
 #pragma unroll
-            for (int q = 0; q <= kLook; ++q) {
-                const int it = it0 + q;
-                if (it < n && go) {
-                    if (it + kLook < n) load(a + it + kLook, R4[(q + kLook) % (kLook + 1)]);
-                    go = store(it, R4[q]);
+            for (int i = 0; i < kLook; ++i)
+                if (i < n) load(a + i, R4[i]);
+            for (int it0 = 0; it0 < n && go; it0 += kLook + 1) {
+#pragma unroll
+                for (int q = 0; q <= kLook; ++q) {
+                    const int it = it0 + q;
+                    if (it < n && go) {
+                        if (it + kLook < n) load(a + it + kLook, R4[(q + kLook) % (kLook + 1)]);
+                        go = store(done + it, R4[q]);
+                    }
                 }
             }
+            done += n;
         }
         }
     } else if (warp == 9) {
@@ -601,15 +703,18 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             const uint32_t id4[2] = {umma::idesc_sf_id(idesc4, 0u), umma::idesc_sf_id(idesc4, 2u)};
             int seg = 0, s = 0;
             uint32_t ph = 0u;
-            for (int unit = a; unit < b && !*s_abort; ++seg) {
+            for (int ri = 0; ri < 2 && !*s_abort; ++ri) {
+            if (ri == 1 && (!GU || !routed_range(false))) break;
+            const Range rg = rng[ri];
+            for (int unit = rg.a; unit < rg.b && !*s_abort; ++seg) {
                 Unit x = decode(unit);
-                const int seg_end = min(b, x.iend);
+                const int seg_end = min(rg.b, x.iend);
                 const int buf = seg & 1;
                 if (seg >= 2 && !wait(&aempty[buf], (uint32_t)(((seg >> 1) + 1) & 1))) break;
                 umma::fence_after();
                 const uint32_t dcol = tbase + (uint32_t)(buf * NMAT * 64);
                 uint32_t acc = 0u;
-                for (int un = unit; un < seg_end; x = advance(x, ++un)) {
+                for (int un = unit; un < seg_end; x = advance(x, ++un, rg.b)) {
                     if (!wait(&full[s], ph) || !wait(&sfr[s], ph)) break;
                     umma::fence_after();
                     const uint32_t soff = (uint32_t)(s * SB) >> 4;
@@ -651,8 +756,9 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 umma::commit(&afull[buf]);
                 unit = seg_end;
             }
+            }
         }
-    } else {
+    } else if (warp < 4) {
         // --------------------------------------------------- epilogue --
         const uint32_t lb = umma::lane_base(warp);
         const int rowl = 32 * warp + lane;  // row of the 128-row item
@@ -660,10 +766,13 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         uint32_t *icnt = reinterpret_cast<uint32_t *>(p.ws + L.icnt) +
                          (GU ? 0 : L.umax * ceil_div(p.ff, kTileM) + ceil_div(L.ffs, kTileM));
         int seg = 0;
-        for (int unit = a; unit < b; ++seg) {
+        for (int ri = 0; ri < 2; ++ri) {
+        if (ri == 1 && (!GU || !routed_range(true))) break;
+        const Range rg = rng[ri];
+        for (int unit = rg.a; unit < rg.b; ++seg) {
             const Unit x = decode(unit);
             const int item = x.item;
-            const int seg_end = min(b, x.iend);
+            const int seg_end = min(rg.b, x.iend);
             const int buf = seg & 1;
             float acc[NMAT][kChunk];
 #pragma unroll
@@ -698,15 +807,15 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             const bool whole = unit == x.istart && seg_end == x.iend;
             bool fin = whole;
             if (!whole) {
-                const int slot = unit == a ? 0 : 1;
-                float *sp = spart + (size_t)((cta * 2 + slot) * 2) * kChunk * kTileM;
+                const int slot = 2 * ri + (unit == rg.a ? 0 : 1);
+                float *sp = spart + (size_t)((cta * 4 + slot) * 2) * kChunk * kTileM;
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m)
 #pragma unroll
                     for (int t = 0; t < kChunk; ++t)
                         if (t < Tc) sp[(m * kChunk + t) * kTileM + rowl] = acc[m][t];
                 umma::bar_sync(1, 128);
-                const int c0 = owner(x.istart), c1 = owner(x.iend - 1);
+                const int c0 = owner(rg, x.istart), c1 = owner(rg, x.iend - 1);
                 if (threadIdx.x == 0) {
                     const uint32_t old = atom_add_acq_rel(icnt + item, 1u);
                     const int last = old == (uint32_t)(c1 - c0);
@@ -722,8 +831,8 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
 #pragma unroll
                         for (int t = 0; t < kChunk; ++t) acc[m][t] = 0.f;
                     for (int cc = c0; cc <= c1; ++cc) {
-                        const int sl = start(cc) < x.istart ? 1 : 0;
-                        const float *q = spart + (size_t)((cc * 2 + sl) * 2) * kChunk * kTileM;
+                        const int sl = 2 * ri + (start(rg, cc) < x.istart ? 1 : 0);
+                        const float *q = spart + (size_t)((cc * 4 + sl) * 2) * kChunk * kTileM;
 #pragma unroll
                         for (int m = 0; m < NMAT; ++m)
 #pragma unroll
@@ -788,6 +897,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 }
             }
             unit = seg_end;
+        }
         }
     }
     umma::fence_before();
