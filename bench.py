@@ -231,18 +231,65 @@ def cpu_oracle_time(cfg, seconds=10.0):
     return done / t_total, threads, done, t_total
 
 
-def run_reference(args, cfg, rank):
+def arm_config(cfg, world):
+    """The workload description both arms report."""
+    return {"workload": workload_desc(cfg), "global_batch": world * cfg.T, "seq_len": 1,
+            "parallelism": f"replicas x{world}"}
+
+
+def max_over_ranks(value, world, device):
+    """The largest of every rank's value (each rank calls it; the ranks are
+    independent replicas and exchange nothing else)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, T, steps, max_ms):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * T * steps / (max_ms / 1000.0)
+
+
+def run_reference(args, cfg, rank, world):
+    """The reference arm: the fp64 CPU oracle as it stands, on the host cores,
+    rank 0 only.  A step is one token of the workload (route + combine); W
+    untimed steps, then K timed ones."""
     if rank != 0:
         return
-    tok_s, threads, n, t = cpu_oracle_time(cfg, seconds=max(5.0, 2.0 * args.steps))
-    ms = 1000.0 * t / n
+    import oracle
+    orc = oracle.oracle()
+    n = args.warmup + args.steps
+    x = k3gen.hidden(cfg, T=max(cfg.T, n))
+    w = k3gen.router(cfg)
+    b = k3gen.bias(cfg)
+    sh = k3gen.shared(cfg) if cfg.ff_shared else None
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    cache = {}
+    t_total = 0.0
+    for i in range(n):
+        xs = x[i:i + 1]
+        _, _, idx, _ = orc.route(xs, w, b, cfg.k)
+        for e in idx[0]:  # input preparation (blob generation) outside the timed region
+            if int(e) not in cache:
+                cache[int(e)] = k3gen.expert_blob(cfg, int(e))
+        t0 = time.perf_counter()
+        _, _, idx, wt = orc.route(xs, w, b, cfg.k)
+        orc.combine(xs, wt, [cache[int(e)] for e in idx[0]], sh, cfg.d, cfg.ff)
+        if i >= args.warmup:
+            t_total += time.perf_counter() - t0
+    tok_s = args.steps / t_total
     line = {
-        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": n, "warmup": 0, "ms_per_step": ms * cfg.T, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_desc(cfg)},
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * t_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": arm_config(cfg, world),
         "cpu_baseline": {"value": tok_s, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"{n} token(s) of the workload, fp64 scalar C oracle"},
+                         "sample": f"one token of the workload per step, {args.steps} timed steps after "
+                                   f"{args.warmup} warm-up, fp64 scalar C oracle (OpenMP over output rows)"},
         "e2e": {"value": tok_s, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -273,7 +320,7 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
-        run_reference(args, cfg, rank)
+        run_reference(args, cfg, rank, world)
         return
 
     import torch
@@ -360,12 +407,9 @@ def main():
         k3.check(k3.k3moe_device_status(ws), "device status")
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, "cuda")
     ms_per_step = total_ms / args.steps
-    value = world * T * args.steps / (total_ms / 1000.0)
+    value = job_throughput(world, T, args.steps, total_ms)
 
     # per-kernel durations (events recorded between the library's kernels)
     kernels = ["route", "expert_gu", "expert_down"]
@@ -424,11 +468,8 @@ def main():
             b.synchronize()  # the result is on the host here
             if i >= args.warmup:
                 e_ms += a.elapsed_time(b)
-        if world > 1:
-            t = _t.tensor([e_ms], dtype=_t.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * T * args.steps / (e_ms / 1000.0), "unit": UNIT,
+        e_ms = max_over_ranks(e_ms, world, "cuda")
+        e2e = {"value": job_throughput(world, T, args.steps, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * ybytes}
 
     cpu = None
@@ -443,10 +484,9 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "mxf4 (E2M1 x E2M1, E8M0 block scales) tcgen05 MMA, f32 accumulate",
         "data": "synthetic",
-        "config": {"workload": workload_desc(cfg), "global_batch": world * T, "seq_len": 1,
-                   "parallelism": f"replicas x{world}",
-                   "l2": "256 MiB buffer written, then another 256 MiB read, before every step, outside the timed events",
-                   "distinct_experts": U},
+        "config": dict(arm_config(cfg, world),
+                       l2="256 MiB buffer written, then another 256 MiB read, before every step, outside the timed events",
+                       distinct_experts=U),
         "layer_hbm_gbs": round(layer_gbs, 1),
         "layer_hbm_frac": round(layer_gbs / peak, 4),
         "per_kernel_ms": {k: round(v, 5) for k, v in per_kernel.items()},
