@@ -52,6 +52,16 @@
  * into one fp32 accumulator per output).  Router logits are fp32 sums of
  * exact fp32 x bf16 products.
  *
+ * Many tokens (T > 8, with a workspace sized for T): the grouped path.  The
+ * router is a GEMM over all tokens (fp32, fixed summation order), the
+ * (token, slot) pairs are sorted by expert and cut into groups of up to 32
+ * tokens, and each group runs through the experts' packed weights on the
+ * tensor cores with its activations as 4 E2M1 pieces (about 2^-10 of the
+ * block's largest element); each (token, slot) output is kept in fp32 and
+ * the k + 1 outputs of a token are summed in slot order (shared expert last)
+ * before the one rounding.  A workspace sized for 8 tokens runs any T as
+ * 8-token passes of the path above.
+ *
  * Ownership and ordering: the caller owns every buffer and the stream.  Calls
  * allocate nothing, never synchronise, and are ordered on `stream`; results
  * are valid once the stream reaches them, and inputs must stay unmodified
@@ -116,7 +126,11 @@ int k3moe_abi_version(void);
 /* Bytes of one routed expert's blob: 3*d*ff*17/32; 0 if dims are invalid. */
 size_t k3moe_blob_bytes(const k3moe_dims *dims);
 
-/* Scratch bytes a call with up to T_max tokens needs; 0 if dims are invalid. */
+/* Scratch bytes a call with up to T_max tokens needs; 0 if dims are invalid.
+ * For T_max > 8 this includes the grouped path's region for passes of up to
+ * 8192 tokens (about 0.7 MB per token for the K3 shape, most of it the fp32
+ * output of every (token, slot)); a call with more tokens than its workspace
+ * was sized for falls back to 8-token passes when the workspace holds those. */
 size_t k3moe_workspace_size(const k3moe_dims *dims, int32_t T_max);
 
 /*
@@ -125,7 +139,8 @@ size_t k3moe_workspace_size(const k3moe_dims *dims, int32_t T_max);
  *               lower index), weight[t][j] = its softmax probability.
  * x: bf16 [T][d]; w_router: fp32 [E][d]; bias: fp32 [E] or NULL;
  * idx: int32 [T][k]; weight: fp32 [T][k].  All pointers 16-byte aligned
- * except bias, idx and weight (4-byte aligned).
+ * except bias, idx and weight (4-byte aligned).  With T > 8 and a workspace
+ * sized for T, the logits come from the grouped path's router GEMM.
  */
 k3moe_status k3moe_route(const void *x, int32_t T, const float *w_router, const float *bias,
                          const k3moe_dims *dims, int32_t *idx, float *weight, void *ws,
