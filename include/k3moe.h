@@ -128,7 +128,7 @@ size_t k3moe_blob_bytes(const k3moe_dims *dims);
 
 /* Scratch bytes a call with up to T_max tokens needs; 0 if dims are invalid.
  * For T_max > 8 this includes the grouped path's region for passes of up to
- * 8192 tokens (about 0.7 MB per token for the K3 shape, most of it the fp32
+ * 8192 tokens (about 0.9 MB per token for the K3 shape, most of it the fp32
  * output of every (token, slot)); a call with more tokens than its workspace
  * was sized for falls back to 8-token passes when the workspace holds those. */
 size_t k3moe_workspace_size(const k3moe_dims *dims, int32_t T_max);
@@ -224,7 +224,7 @@ k3moe_status k3moe_layer_timed(const void *x, int32_t T, const float *w_router, 
  *   - Shapes whose scratch (k3moe_workspace_size(dims, 8)) exceeds 16 MiB are
  *     rejected with K3MOE_ERR_WORKSPACE_TOO_SMALL before anything runs; the
  *     K3 shape (d=7168, ff=1536, 896 experts, top-16, shared ff=1536) needs
- *     about 10.5 MiB.
+ *     about 14.8 MiB.
  *   - All calls on one device share the buffer: two calls that may overlap
  *     (other streams, other host threads) race and give wrong results.
  *     Serialise them, or use k3moe_layer with a workspace per stream.
