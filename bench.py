@@ -100,23 +100,35 @@ def route_bytes(cfg):
     return cfg.E * cfg.d * 4 + cfg.T * cfg.d * 2
 
 
-def captured_traffic(cfg):
-    """DRAM bytes (read + write) of one gate/up launch from the committed ncu
-    summary, while the kernel sources still hash to the captured ones and the
-    launch moves the same bytes (d, ff, k, shared ff, T and 16 distinct
+# The committed ncu summary that holds the DRAM traffic of each timed kernel
+# (K3 decode shape, T=1, 16 distinct experts): kernel name -> profile file.
+TRAFFIC_PROFILES = {"expert_gu": "expert_gu_k3_decode_e64.md"}
+
+
+def captured_traffic(cfg, kernel):
+    """DRAM bytes (read + write) of one launch of `kernel` from its committed
+    ncu summary, while the kernel sources still hash to the captured ones and
+    the launch moves the same bytes (d, ff, k, shared ff, T and 16 distinct
     experts); otherwise None."""
     import hashlib
     here = os.path.dirname(os.path.abspath(__file__))
+    prof = TRAFFIC_PROFILES.get(kernel)
+    if prof is None:
+        return None
     try:
-        text = open(os.path.join(here, "profiles", "expert_gu_k3_decode_e64.md")).read()
+        text = open(os.path.join(here, "profiles", prof)).read()
     except OSError:
         return None
     fields = dict(line.split(": ", 1) for line in text.splitlines()
-                  if line.startswith(("traffic_bytes_per_launch: ", "source_sha256: ")))
+                  if line.startswith(("traffic_bytes_per_launch: ", "source_sha256: ", "source_files: ")))
+    files = fields.get("source_files", "umma_kernels.cuh umma.cuh common.cuh layout.cuh").split()
     src = os.path.join(here, "mxfp4_routed_expert_softmax_b200", "csrc")
     h = hashlib.sha256()
-    for f in ("umma_kernels.cuh", "umma.cuh", "common.cuh", "layout.cuh"):
-        h.update(open(os.path.join(src, f), "rb").read())
+    try:
+        for f in files:
+            h.update(open(os.path.join(src, f), "rb").read())
+    except OSError:
+        return None
     if fields.get("source_sha256", "").strip() != h.hexdigest():
         return None
     if (cfg.d, cfg.ff, cfg.k, cfg.ff_shared, cfg.T) != (7168, 1536, 16, 1536, 1):
@@ -125,7 +137,7 @@ def captured_traffic(cfg):
 
 
 def load_bf16_peak():
-    """Measured dense bf16 TFLOP/s (burst), else the fallback 1590."""
+    """Measured dense bf16 TFLOP/s (burst) and its kind, else the fallback 1590."""
     here = os.path.dirname(os.path.abspath(__file__))
     try:
         with open(os.path.join(here, "MEASURED_PEAKS.json")) as f:
@@ -133,9 +145,9 @@ def load_bf16_peak():
         v = d.get("bf16_tflops")
         if isinstance(v, dict):
             v = v.get("value")
-        return float(v)
+        return float(v), "measured"
     except (OSError, ValueError, TypeError):
-        return 1590.0
+        return 1590.0, "fallback"
 
 
 def load_peaks():
@@ -304,6 +316,8 @@ def main():
     ap.add_argument("--config", default="k3_decode", choices=list(k3gen.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="profiling mode: no e2e/cpu legs")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="measure the headline workload only (not the T=8 / prefill workloads)")
     ap.add_argument("--experts", type=int, default=None,
                     help="profiling: keep only this many experts resident (same d, ff, top-k); the "
                          "routed and shared bytes per token stay those of the workload, the router shrinks")
@@ -334,13 +348,6 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     W = kdev.weights(cfg)
-    inp = kdev.DeviceInputs(cfg)
-    T = inp.T
-    dims = k3.make_dims(cfg.d, cfg.ff, cfg.E, cfg.k, cfg.ff_shared,
-                        k3.K3MOE_OUT_FP32 if cfg.out_fp32 else 0)
-    ws = k3.new_workspace(dims, T, host_staging=True)
-    ybytes = 4 if cfg.out_fp32 else 2
-    y = torch.empty((T, cfg.d), dtype=torch.float32 if cfg.out_fp32 else torch.int16, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     rflush = torch.ones(64 << 20, dtype=torch.float32, device="cuda")  # 256 MiB, read after the write
 
@@ -349,39 +356,136 @@ def main():
         # leave L2 here (their write-back is not charged to the next step)
         flush.fill_(i & 255)
         rflush.sum()
+
     stream = torch.cuda.current_stream()
+    peak, _ = load_peaks()
+
+    # the headline workload, then (default run) the other K3 workloads on the
+    # same resident weights, each measured the same way
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    head = measure(cfg, W, k3, args, flush_l2, stream, world, e2e=not args.quick)
+    others = {}
+    if args.config == "k3_decode" and args.experts is None and not args.quick and not args.no_configs:
+        for name in ("k3_decode_t8", "k3_prefill_512", "k3_prefill_4096"):
+            others[name] = measure(k3gen.CONFIGS[name], W, k3, args, flush_l2, stream, world, e2e=False)
+    clk = clocks.stop()
+
+    T = head["T"]
+    ms_per_step = head["ms_per_step"]
+    value = head["value"]
+    roofline = head["roofline"]
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
+        tok_s, threads, n, t = cpu_oracle_time(cfg, seconds=10.0)
+        cpu = {"value": tok_s, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{n} token(s) of the workload ({t:.1f} s), fp64 scalar C oracle, "
+                         f"OpenMP over output rows",
+               "cpu_model": cpu_model()}
+        for name, r in others.items():
+            tok_s, threads, n, t = cpu_oracle_time(k3gen.CONFIGS[name], seconds=4.0)
+            r["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                 "sample": f"{n} token(s) of the workload ({t:.1f} s)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "mxf4 (E2M1 x E2M1, E8M0 block scales) tcgen05 MMA, f32 accumulate",
+        "data": "synthetic",
+        "config": dict(arm_config(cfg, world),
+                       l2="256 MiB buffer written, then another 256 MiB read, before every step, outside the timed events",
+                       distinct_experts=head["U"]),
+        "layer_hbm_gbs": head["layer_gbs"],
+        "layer_hbm_frac": round(head["layer_gbs"] / peak, 4),
+        "per_kernel_ms": head["per_kernel_ms"],
+        "per_kernel_gbs": head["per_kernel_gbs"],
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": head["e2e"],
+        "gpu_launches": head["launches"] * args.steps,
+        "clocks": clk,
+    }
+    if others:
+        line["configs"] = {name: summary(r, peak) for name, r in others.items()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def summary(r, peak):
+    """The per-workload record of the bench line's `configs` key."""
+    out = {"workload": workload_desc(r["cfg"]), "tokens": r["T"], "steps": r["steps"],
+           "ms_per_step": r["ms_per_step"], "value": r["value"], "unit": UNIT,
+           "distinct_experts": r["U"], "layer_hbm_gbs": r["layer_gbs"],
+           "layer_hbm_frac": round(r["layer_gbs"] / peak, 4), "roofline": r["roofline"],
+           "gpu_launches_per_step": r["launches"]}
+    if r["per_kernel_ms"]:
+        out["per_kernel_ms"] = r["per_kernel_ms"]
+        out["per_kernel_gbs"] = r["per_kernel_gbs"]
+    if "cpu_baseline" in r:
+        out["cpu_baseline"] = r["cpu_baseline"]
+    return out
+
+
+def kernel_names(n):
+    """Names of the library's kernels in launch order for an 8-token pass."""
+    return {3: ["route", "expert_gu", "expert_down"], 1: ["layer"]}.get(n, [f"k{i}" for i in range(n)])
+
+
+def kernel_bytes(cfg, U, pairs, name):
+    return {"route": route_bytes(cfg), "expert_gu": gu_bytes(cfg, U, pairs),
+            "expert_down": down_bytes(cfg, U, pairs), "layer": alg_bytes(cfg, U)}.get(name)
+
+
+def measure(cfg, W, k3, args, flush_l2, stream, world, e2e=False):
+    """W warm-up and K timed layer calls on one workload (L2 flushed before
+    each, CUDA events on the launching stream, max over ranks); for passes of
+    up to 8 tokens also K calls with events between the library's kernels,
+    and (e2e) K calls through k3moe_layer_from_host with the copies timed."""
+    import torch
+    from k3gen import device as kdev
+    inp = kdev.DeviceInputs(cfg)
+    T = inp.T
+    dims = k3.make_dims(cfg.d, cfg.ff, cfg.E, cfg.k, cfg.ff_shared,
+                        k3.K3MOE_OUT_FP32 if cfg.out_fp32 else 0)
+    ws = k3.new_workspace(dims, T, host_staging=e2e)
+    ybytes = 4 if cfg.out_fp32 else 2
+    y = torch.empty((T, cfg.d), dtype=torch.float32 if cfg.out_fp32 else torch.int16, device="cuda")
     sg, su, sd = W.shared
 
     def step_plain():
         k3.check(k3.k3moe_layer(inp.x, T, W.w_router, inp.bias, W.blob_ptrs, sg, su, sd, dims, y,
                                 None, None, ws), "k3moe_layer")
 
-    single_pass = T <= 8
-    nev = 5
-    # warm-up
     for _ in range(args.warmup):
         flush_l2(1)
         step_plain()
     torch.cuda.synchronize()
     k3.check(k3.k3moe_device_status(ws), "device status")
-
     # distinct experts of the batch (for the algorithmic byte count)
     idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
     wts = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
     k3.check(k3.k3moe_route(inp.x, T, W.w_router, inp.bias, dims, idx, wts, ws), "route")
-    idx_np = idx.cpu().numpy()
-    U = len(np.unique(idx_np))
+    U = len(np.unique(idx.cpu().numpy()))
     pairs = T * cfg.k
 
-    # timed region
-    clocks = ClockSampler(local_rank)
-    clocks.start()
-    time.sleep(0.3)
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
-    kern_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)]
-               for _ in range(args.steps)] if single_pass else None
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
@@ -392,75 +496,74 @@ def main():
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clk = clocks.stop()
     k3.check(k3.k3moe_device_status(ws), "device status")
-    # per-kernel durations: K more steps with events between the library's
-    # kernels (k3moe_layer_timed; the events serialise the kernels, so these
-    # steps are not part of the headline number)
-    if single_pass:
-        for i in range(args.steps):
-            flush_l2(i)
-            st, nk = k3.k3moe_layer_timed(inp.x, T, W.w_router, inp.bias, W.blob_ptrs, sg, su, sd,
-                                          dims, y, ws, kern_ev[i])
-            k3.check(st, "k3moe_layer_timed")
-        torch.cuda.synchronize()
-        k3.check(k3.k3moe_device_status(ws), "device status")
-    step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    total_ms = sum(step_ms)
-    total_ms = max_over_ranks(total_ms, world, "cuda")
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in step_ev), world, "cuda")
     ms_per_step = total_ms / args.steps
     value = job_throughput(world, T, args.steps, total_ms)
 
-    # per-kernel durations (events recorded between the library's kernels)
-    kernels = ["route", "expert_gu", "expert_down"]
+    # per-kernel durations: K more calls with events between the library's
+    # kernels (k3moe_layer_timed; the events serialise the kernels, so these
+    # calls are not part of the headline number)
     per_kernel = {}
-    if single_pass:
-        for j, name in enumerate(kernels):
+    n_kernels = None
+    if T <= 8:
+        nev = 6
+        kern_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush_l2(i)
+            st, n_kernels = k3.k3moe_layer_timed(inp.x, T, W.w_router, inp.bias, W.blob_ptrs, sg, su,
+                                                 sd, dims, y, ws, kern_ev[i])
+            k3.check(st, "k3moe_layer_timed")
+        torch.cuda.synchronize()
+        k3.check(k3.k3moe_device_status(ws), "device status")
+        for j, name in enumerate(kernel_names(n_kernels)):
             per_kernel[name] = statistics.mean(kern_ev[i][j].elapsed_time(kern_ev[i][j + 1])
                                                for i in range(args.steps))
+
     peak, peak_kind = load_peaks()
-    gu_ms = per_kernel.get("expert_gu")
-    gb = gu_bytes(cfg, U, pairs)
+    layer_gbs = alg_bytes(cfg, U) / (ms_per_step / 1000.0) / 1e9
     roofline = None
-    if gu_ms:
-        ach = gb / (gu_ms / 1000.0) / 1e9
-        roofline = {"bound": "hbm", "kernel": "expert_gu", "achieved": round(ach, 1),
-                    "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 4),
+    if per_kernel:
+        # the dominant kernel against the HBM copy peak
+        name = max(per_kernel, key=per_kernel.get)
+        gb = kernel_bytes(cfg, U, pairs, name)
+        ach = gb / (per_kernel[name] / 1000.0) / 1e9
+        roofline = {"bound": "hbm", "kernel": name, "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                    "frac": round(ach / peak, 4),
                     "peak_kind": f"{peak_kind} (burst copy, MEASURED_PEAKS.json hbm_gbs)"
                     if peak_kind == "measured" else "fallback 6.65 TB/s",
-                    "traffic": captured_traffic(cfg) if U == 16 else None,
+                    "traffic": captured_traffic(cfg, name) if U == 16 else None,
                     "alg_bytes_per_launch": gb}
-    layer_gbs = alg_bytes(cfg, U) / (ms_per_step / 1000.0) / 1e9
-    if roofline is None:
+    else:
         # many tokens (grouped prefill): the whole layer against its bound.  The
         # block-scaled fp4 tensor peak is the measured bf16 peak x 4 (the
-        # nominal dense ratio); the layer is HBM-bound when its bytes take
-        # longer at the copy peak than its FLOPs at that tensor peak.
+        # nominal dense fp4/bf16 ratio, 9 / 2.25 PFLOP/s); the layer is
+        # HBM-bound when its bytes take longer at the copy peak than its FLOPs
+        # at that tensor peak.  Both fractions are reported.
         fl = layer_flops(cfg, T)
-        tensor_peak = load_bf16_peak() * 4.0
+        bf16_peak, bf16_kind = load_bf16_peak()
+        tensor_peak = bf16_peak * 4.0
         t_hbm = alg_bytes(cfg, U) / (peak * 1e9)
         t_tc = fl / (tensor_peak * 1e12)
-        if t_hbm >= t_tc:
-            roofline = {"bound": "hbm", "kernel": "layer (all kernels of the grouped prefill)",
-                        "achieved": round(layer_gbs, 1), "peak": peak, "unit": "GB/s",
-                        "frac": round(layer_gbs / peak, 4), "traffic": None,
-                        "alg_bytes_per_launch": alg_bytes(cfg, U)}
-        else:
-            tf = fl / (ms_per_step / 1000.0) / 1e12
-            roofline = {"bound": "tensor", "kernel": "layer (all kernels of the grouped prefill)",
-                        "achieved": round(tf, 2), "peak": round(tensor_peak, 1), "unit": "TFLOP/s",
-                        "frac": round(tf / tensor_peak, 4), "traffic": None, "alg_flops_per_launch": fl}
+        tf = fl / (ms_per_step / 1000.0) / 1e12
+        hb = {"bound": "hbm", "kernel": "layer (all kernels of the grouped prefill)",
+              "achieved": round(layer_gbs, 1), "peak": peak, "unit": "GB/s",
+              "frac": round(layer_gbs / peak, 4), "traffic": None, "alg_bytes_per_launch": alg_bytes(cfg, U)}
+        tc = {"bound": "tensor", "kernel": "layer (all kernels of the grouped prefill)",
+              "achieved": round(tf, 2), "peak": round(tensor_peak, 1), "unit": "TFLOP/s",
+              "frac": round(tf / tensor_peak, 4), "traffic": None, "alg_flops_per_launch": fl,
+              "peak_kind": f"{bf16_kind} dense bf16 x 4 (nominal dense fp4 / bf16 ratio)"}
+        roofline = dict(hb if t_hbm >= t_tc else tc)
+        roofline["other_bound"] = tc if t_hbm >= t_tc else hb
 
-    # end to end: host activations in and out through the C ABI, copies timed
-    e2e = None
-    if not args.quick:
-        import torch as _t
-        xh = _t.from_numpy(inp.x_host.view(np.int16)).pin_memory()
-        yh = _t.empty((T, cfg.d), dtype=_t.float32 if cfg.out_fp32 else _t.int16).pin_memory()
+    e2e_rec = None
+    if e2e:
+        xh = torch.from_numpy(inp.x_host.view(np.int16)).pin_memory()
+        yh = torch.empty((T, cfg.d), dtype=torch.float32 if cfg.out_fp32 else torch.int16).pin_memory()
         e_ms = 0.0
         for i in range(args.warmup + args.steps):
             flush_l2(i)
-            a, b = _t.cuda.Event(enable_timing=True), _t.cuda.Event(enable_timing=True)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             k3.check(k3.k3moe_layer_from_host(xh, T, W.w_router, inp.bias, W.blob_ptrs, sg, su, sd,
                                               dims, yh, ws), "from_host")
@@ -469,41 +572,15 @@ def main():
             if i >= args.warmup:
                 e_ms += a.elapsed_time(b)
         e_ms = max_over_ranks(e_ms, world, "cuda")
-        e2e = {"value": job_throughput(world, T, args.steps, e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * ybytes}
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
-        tok_s, threads, n, t = cpu_oracle_time(cfg, seconds=10.0)
-        cpu = {"value": tok_s, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"{n} token(s) of the workload ({t:.1f} s), fp64 scalar C oracle, "
-                         f"OpenMP over output rows"}
-
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "mxf4 (E2M1 x E2M1, E8M0 block scales) tcgen05 MMA, f32 accumulate",
-        "data": "synthetic",
-        "config": dict(arm_config(cfg, world),
-                       l2="256 MiB buffer written, then another 256 MiB read, before every step, outside the timed events",
-                       distinct_experts=U),
-        "layer_hbm_gbs": round(layer_gbs, 1),
-        "layer_hbm_frac": round(layer_gbs / peak, 4),
-        "per_kernel_ms": {k: round(v, 5) for k, v in per_kernel.items()},
-        "per_kernel_gbs": {k: round(b / (per_kernel[k] / 1000.0) / 1e9, 1)
-                           for k, b in (("route", route_bytes(cfg)), ("expert_gu", gu_bytes(cfg, U, pairs)),
-                                        ("expert_down", down_bytes(cfg, U, pairs)))
-                           if per_kernel.get(k)},
-        "roofline": roofline,
-        "cpu_baseline": cpu,
-        "e2e": e2e,
-        "gpu_launches": launches_per_step(cfg, T) * args.steps,
-        "clocks": clk,
-    }
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+        e2e_rec = {"value": job_throughput(world, T, args.steps, e_ms), "unit": UNIT,
+                   "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * ybytes}
+    launches = n_kernels if (T <= 8 and n_kernels) else launches_per_step(cfg, T)
+    del ws
+    return {"cfg": cfg, "T": T, "U": U, "steps": args.steps, "ms_per_step": ms_per_step, "value": value,
+            "layer_gbs": round(layer_gbs, 1), "per_kernel_ms": {k: round(v, 5) for k, v in per_kernel.items()},
+            "per_kernel_gbs": {k: round(kernel_bytes(cfg, U, pairs, k) / (v / 1000.0) / 1e9, 1)
+                               for k, v in per_kernel.items() if kernel_bytes(cfg, U, pairs, k)},
+            "roofline": roofline, "e2e": e2e_rec, "launches": launches}
 
 
 if __name__ == "__main__":

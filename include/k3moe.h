@@ -103,6 +103,22 @@ typedef enum {
 /* flags */
 #define K3MOE_OUT_FP32 1u  /* y (and expert_ffn's out) in fp32 instead of bf16 */
 #define K3MOE_NO_SHARED 2u /* skip the shared expert (its pointers may be NULL) */
+/* Check every E8M0 scale byte the call reads for 0xFF (the encoding of NaN,
+ * OCP Microscaling Formats v1.0): a call that meets one records
+ * K3MOE_ERR_DEVICE_CHECK in the workspace status word (its outputs are then
+ * undefined).  Without the flag the byte is handed to the tensor core as it
+ * is, and the outputs it reaches are whatever the hardware makes of a NaN
+ * scale. */
+#define K3MOE_STRICT 4u
+/* Routing variants (the pages' routing uses neither; both are common in MoE
+ * models).  K3MOE_RENORM_TOPK: the k weights of a token are divided by their
+ * sum, w_j = p_idx_j / sum_j' p_idx_j' (summed in pick order).
+ * K3MOE_BIAS_SELECT_ONLY: `bias` moves only the selection -- the top-k is
+ * taken on l_e + b_e, while the weights come from the softmax of the unbiased
+ * logits l (without the flag the bias is part of the logits and so moves
+ * both). */
+#define K3MOE_RENORM_TOPK 8u
+#define K3MOE_BIAS_SELECT_ONLY 16u
 
 /*
  * Layer dimensions.  d and ff: multiples of 64, 64 <= d <= 8192,
@@ -245,8 +261,25 @@ k3moe_status k3moe_layer_noalloc(const void *x, int32_t T, const float *w_router
  * K3MOE_OK, K3MOE_ERR_DEVICE_CHECK or K3MOE_ERR_DEVICE_TIMEOUT.  After
  * K3MOE_ERR_DEVICE_TIMEOUT the outputs of the calls since the last check are
  * undefined and the workspace must be zero-filled again before its next use.
+ * ws == NULL reads the built-in scratch of k3moe_layer_noalloc on the
+ * current device instead; there, after K3MOE_ERR_DEVICE_TIMEOUT, this call
+ * itself zero-fills the whole built-in buffer (synchronously), so the next
+ * k3moe_layer_noalloc call starts clean.
  */
 k3moe_status k3moe_device_status(void *ws, void *stream);
+
+/*
+ * For tests of the failure paths only (process-wide; leave at 0, 0 in
+ * production).  Makes a bounded device wait run out without any GPU fault:
+ *   mode 0: normal operation;
+ *   mode 1: the routed gate/up work of every later layer call waits for a
+ *           "routing loaded" signal that is never given, so its waits run
+ *           out and the call records K3MOE_ERR_DEVICE_TIMEOUT (the kernels
+ *           then finish early with undefined outputs; nothing faults).
+ * wait_limit_ns bounds every device wait of later calls (0: the default of
+ * 2 seconds).  Returns K3MOE_ERR_INVALID_ARGUMENT for an unknown mode.
+ */
+k3moe_status k3moe_debug_set_fault(int32_t mode, uint64_t wait_limit_ns);
 
 /* Static text for a status code. */
 const char *k3moe_status_string(k3moe_status status);

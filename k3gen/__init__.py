@@ -94,6 +94,8 @@ class Config:
     "zipf" (b_e = -1.1 ln r_e for a seeded rank permutation, stream 6).
     out_fp32: the output mode the workload is quoted in (the parity tests
     check both modes on every config).
+    scale_lo, scale_count: the experts' E8M0 bytes are uniform in
+    [scale_lo, scale_lo + scale_count) (the workloads: 118..124).
     """
     name: str
     d: int
@@ -105,6 +107,8 @@ class Config:
     bias: str | None = None
     zipf_s: float = 1.1
     out_fp32: bool = False
+    scale_lo: int = SCALE_LO
+    scale_count: int = SCALE_COUNT
 
     @property
     def blob_bytes(self) -> int:
@@ -186,7 +190,9 @@ def expert_blob(cfg: Config, e: int, seed: int = 0, out: np.ndarray | None = Non
     if out is None:
         out = np.empty((nb,), dtype=np.uint8)
     assert out.dtype == np.uint8 and out.size == nb
-    _load().k3gen_expert_blob(seed, e, cfg.d, cfg.ff, SCALE_LO, SCALE_COUNT, _ptr(out))
+    if not (0 <= cfg.scale_lo and cfg.scale_count >= 1 and cfg.scale_lo + cfg.scale_count <= 256):
+        raise ValueError("E8M0 byte range outside 0..255")
+    _load().k3gen_expert_blob(seed, e, cfg.d, cfg.ff, cfg.scale_lo, cfg.scale_count, _ptr(out))
     return out
 
 

@@ -47,7 +47,7 @@ class DeviceWeights:
 
 def weights(cfg: k3gen.Config, seed: int = 0, device="cuda") -> DeviceWeights:
     """Device weights shared by every workload with the same layer shape."""
-    key = (cfg.d, cfg.ff, cfg.E, cfg.ff_shared, seed, str(device))
+    key = (cfg.d, cfg.ff, cfg.E, cfg.ff_shared, cfg.scale_lo, cfg.scale_count, seed, str(device))
     w = _WEIGHTS.get(key)
     if w is None:
         w = DeviceWeights(cfg, seed, device)

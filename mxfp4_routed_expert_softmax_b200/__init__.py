@@ -25,6 +25,9 @@ K3MOE_ERR_DEVICE_CHECK = 6
 
 K3MOE_OUT_FP32 = 1
 K3MOE_NO_SHARED = 2
+K3MOE_STRICT = 4
+K3MOE_RENORM_TOPK = 8
+K3MOE_BIAS_SELECT_ONLY = 16
 
 
 class K3moeError(RuntimeError):
@@ -72,6 +75,7 @@ _SIGS = {
     "k3moe_device_status": ([_vp, _vp], ctypes.c_int),
     "k3moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "k3moe_last_error": ([], ctypes.c_char_p),
+    "k3moe_debug_set_fault": ([_i32, ctypes.c_uint64], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -179,7 +183,15 @@ def k3moe_layer_timed(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu, 
 
 
 def k3moe_device_status(ws, stream=None) -> int:
+    """ws=None: the built-in scratch of k3moe_layer_noalloc on this device."""
     return lib.k3moe_device_status(_ptr(ws), _stream(stream))
+
+
+def k3moe_debug_set_fault(mode: int, wait_limit_ns: int = 0) -> int:
+    """Failure-path tests only: mode 1 makes the next layer calls' bounded
+    device waits run out (no GPU fault); wait_limit_ns bounds every wait
+    (0: the default).  Reset with (0, 0)."""
+    return lib.k3moe_debug_set_fault(mode, wait_limit_ns)
 
 
 def new_workspace(dims: k3moe_dims, T_max: int, device="cuda", host_staging: bool = False):

@@ -18,7 +18,8 @@ namespace k3 {
 constexpr uint32_t kStDeviceCheck = 1u;  // a device-side argument check failed
 constexpr uint32_t kStTimeout = 2u;      // a bounded wait gave up
 
-// Bounded waits give up after this many nanoseconds of wall time.
+// Bounded waits give up after this many nanoseconds of wall time (the
+// default; every kernel takes its limit as a launch parameter).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 struct WsHeader {
@@ -26,9 +27,11 @@ struct WsHeader {
     uint32_t router_done;  // router rows finished in this call; back to 0 by its end
     uint32_t n_unique;     // distinct routed experts in the current token chunk
     uint32_t topk_done;    // tokens whose top-k other CTAs finished; back to 0 by its end
-    uint32_t prep_done;    // router CTAs whose tensor maps and x pieces are written (decode;
-                           // reset by the down pass)
-    uint32_t pad[59];
+    uint32_t prep_done;    // CTAs whose tensor maps and x pieces are written (decode; back to 0
+                           // by the end of the call)
+    uint32_t gu_done;      // gate/up items whose activations are written (layer kernel)
+    uint32_t exit_cnt;     // CTAs of the layer kernel that have finished (the last resets)
+    uint32_t pad[57];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -91,20 +94,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for phase `parity` of `bar` to complete, for at most kWaitLimitNs.
+// Wait for phase `parity` of `bar` to complete, for at most limit_ns.
 // Returns false (and sets the timeout bit) when the limit is reached.
 // The clock is read only every 64 polls: the waits sit on the pipelines'
 // critical paths.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, WsHeader *h) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, WsHeader *h,
+                                                  uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0u && globaltimer() - t0 > kWaitLimitNs) {
+        if ((i & 63u) == 0u && globaltimer() - t0 > limit_ns) {
             set_status(h, kStTimeout);
             return false;
         }
     }
+}
+
+// Wait (bounded, no status) for phase `parity` of `bar`: used on the way
+// out of a kernel whose pipeline gave up, so that bulk copies this thread
+// issued have landed before the CTA's shared memory is released.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer() - t0 > limit_ns) return;
+    }
+}
+
+// E8M0 byte 0xFF encodes NaN: nonzero when any of the 8 bytes of (a, b) is.
+__device__ __forceinline__ uint32_t e8m0_nan8(uint32_t a, uint32_t b) {
+    return __vcmpeq4(a, 0xFFFFFFFFu) | __vcmpeq4(b, 0xFFFFFFFFu);
 }
 
 // ------------------------------------------------- gpu-scope atomics --

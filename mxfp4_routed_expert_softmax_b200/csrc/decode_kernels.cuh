@@ -34,9 +34,15 @@ struct RouteParams {
     uint4 smap[3][8];   // shared expert tensor maps (W_g, W_u, W_d), when has_shared
     int has_shared;     // the tensor-core kernels run a shared expert
     const uint8_t *sw[3];  // the shared expert's W_g, W_u, W_d (the key of its cached maps)
+    uint64_t wait_ns;   // bound of every device wait
+    int route_flags;    // kRouteRenorm | kRouteBiasSelect
 };
 
 constexpr int kRouteThreads = 256;
+// Routing variants: the k weights renormalised over the picks; the bias
+// moving only the selection (the logits and the softmax stay unbiased).
+constexpr int kRouteRenorm = 1;
+constexpr int kRouteBiasSelect = 2;
 constexpr int kRouteTok = 4;  // tokens per pass over the rows (x kept in smem as fp32)
 
 // Order-preserving 32-bit key of a float (larger float -> larger key; -0 is
@@ -72,8 +78,11 @@ __device__ __forceinline__ uint32_t block_scan_incl(uint32_t v, uint32_t *s_tot)
 // K exactly; every key above K is taken, and of the keys equal to K the
 // lowest indices (a prefix count in index order).  The k winners are then
 // ranked by (key descending, index ascending) for the output order.
+// sel_bias (non-null): the selection runs on logit + sel_bias[e] while the
+// softmax stays on the logits; renorm: the k weights are divided by their
+// sum (in pick order).
 __device__ void cta_topk_row(const float *row, int E, int k, int32_t *idx_row, float *w_row, int32_t *idx_out_row,
-                             float *w_out_row) {
+                             float *w_out_row, const float *sel_bias = nullptr, bool renorm = false) {
     __shared__ uint32_t s_hist[256];
     __shared__ uint32_t s_tot[8];
     __shared__ float s_red[2][8];
@@ -89,7 +98,7 @@ __device__ void cta_topk_row(const float *row, int E, int k, int32_t *idx_row, f
         const int e = 4 * tid + i;
         ok[i] = e < E;
         v[i] = ok[i] ? __ldcg(row + e) : -INFINITY;
-        key[i] = ok[i] ? fkey(v[i]) : 0u;  // real keys are > 0
+        key[i] = ok[i] ? fkey(sel_bias ? v[i] + __ldg(sel_bias + e) : v[i]) : 0u;  // real keys are > 0
         mx = fmaxf(mx, v[i]);
     }
 #pragma unroll
@@ -175,14 +184,31 @@ __device__ void cta_topk_row(const float *row, int E, int k, int32_t *idx_row, f
 #pragma unroll
     for (int w = 0; w < 8; ++w) s += s_red[1][w];
     const float inv_s = 1.0f / s;
+    uint32_t mk = 0u, mi = 0u;
+    int r = 0;
     if (lane < k) {
-        const uint32_t mk = s_selk[lane], mi = s_seli[lane];
-        int r = 0;
+        mk = s_selk[lane];
+        mi = s_seli[lane];
         for (int q = 0; q < k; ++q) {
             const uint32_t qk = s_selk[q], qi = s_seli[q];
             r += (qk > mk || (qk == mk && qi < mi)) ? 1 : 0;
         }
-        const float w = expf(fkey_value(mk) - m) * inv_s;
+    }
+    // the pick's softmax numerator (its own logit: the key holds it unless
+    // the selection was biased)
+    const float lv = lane < k ? (sel_bias ? __ldcg(row + mi) : fkey_value(mk)) : 0.f;
+    float num = lane < k ? expf(lv - m) : 0.f;
+    float w = num * inv_s;
+    if (renorm) {
+        // sum of the k numerators in pick order (lane r holds pick r)
+        __shared__ float s_num[32];
+        if (lane < k) s_num[r] = num;
+        __syncwarp();
+        float z = 0.f;
+        for (int q = 0; q < k; ++q) z += s_num[q];
+        w = num / z;
+    }
+    if (lane < k) {
         idx_row[r] = (int32_t)mi;
         w_row[r] = w;
         if (idx_out_row) idx_out_row[r] = (int32_t)mi;
@@ -194,7 +220,8 @@ __device__ void cta_topk(const RouteParams &p, int t) {
     const int k = p.k;
     cta_topk_row(reinterpret_cast<const float *>(p.ws + p.L.logits) + (size_t)t * p.E, p.E, k,
                  reinterpret_cast<int32_t *>(p.ws + p.L.idx) + t * k, reinterpret_cast<float *>(p.ws + p.L.wt) + t * k,
-                 p.idx_out ? p.idx_out + (size_t)t * k : nullptr, p.w_out ? p.w_out + (size_t)t * k : nullptr);
+                 p.idx_out ? p.idx_out + (size_t)t * k : nullptr, p.w_out ? p.w_out + (size_t)t * k : nullptr,
+                 (p.route_flags & kRouteBiasSelect) ? p.bias : nullptr, (p.route_flags & kRouteRenorm) != 0);
 }
 
 // The dispatch of a chunk whose top-k is done: distinct experts in ascending
@@ -356,7 +383,6 @@ __device__ void stream_router(const RouteParams &p, WsHeader *hdr, uint8_t *ring
     const int nrows = u1 > u0 ? (int)((u1 * 16 - 1) / d) - row_base + 1 : 0;
     const int nch = (int)((u1 - u0 + 255) / 256);
     for (int i = tid; i < kRMaxRows * kRouteTok; i += blockDim.x) (&sm.acc[0][0])[i] = 0.f;
-    bool timed_out = false;
     auto issue = [&](int j, int slot) { router_issue(p, ring, full, u0, u1, j, slot); };
     // Few rows per slice (the usual case): each thread keeps its own sum per
     // row of the slice across all stages, and the warps reduce once at the
@@ -376,10 +402,9 @@ __device__ void stream_router(const RouteParams &p, WsHeader *hdr, uint8_t *ring
         {
             // lane 0 polls; the others then take the completed phase themselves
             int ok = 1;
-            if (lane == 0) ok = mbar_wait_bounded(&full[slot], par, hdr) ? 1 : 0;
+            if (lane == 0) ok = mbar_wait_bounded(&full[slot], par, hdr, p.wait_ns) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (ok && lane != 0) ok = mbar_try_wait(&full[slot], par) ? 1 : 0;
-            if (!ok) timed_out = true;
+            if (ok && lane != 0) (void)mbar_try_wait(&full[slot], par);
         }
         const long long unit = u0 + 256LL * j + tid;
         int row = -1;
@@ -476,18 +501,14 @@ __device__ void stream_router(const RouteParams &p, WsHeader *hdr, uint8_t *ring
                 for (int t = 0; t < kRouteTok; ++t)
                     if (t < nt) sm.acc[tid][t] += sm.seg_val[0][w][tid][t];
     }
+    // every stage this CTA issued has been waited for above (a stage whose
+    // wait ran out is the only copy that may not have landed)
     __syncthreads();  // every fold is done
-    if (timed_out && tid == 0) {
-        // copies may still be in flight: let them land (bounded) first
-        const uint64_t tw = globaltimer();
-        while (globaltimer() - tw < 200000ull) {
-        }
-    }
     if (tid < nrows) {
         const int r = row_base + tid;
         const long long rs = (long long)r * d / 16, re = (long long)(r + 1) * d / 16;  // its units
         float *logits = reinterpret_cast<float *>(p.ws + p.L.logits);
-        const float bias = p.bias ? p.bias[r] : 0.f;
+        const float bias = (p.bias && !(p.route_flags & kRouteBiasSelect)) ? p.bias[r] : 0.f;
         bool done = false;
         float out[kRouteTok];
         if (rs >= u0 && re <= u1) {
@@ -522,11 +543,11 @@ __device__ void stream_router(const RouteParams &p, WsHeader *hdr, uint8_t *ring
 }
 
 // Wait (bounded) until *ctr reaches target; false (timeout bit set) if not.
-__device__ bool wait_count(const uint32_t *ctr, uint32_t target, WsHeader *hdr) {
+__device__ bool wait_count(const uint32_t *ctr, uint32_t target, WsHeader *hdr, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer();
     while (ld_acquire(ctr) < target) {
         __nanosleep(64);
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             set_status(hdr, kStTimeout);
             return false;
         }
@@ -605,7 +626,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
     // top-k of this CTA's tokens once every router row is in
     if ((int)blockIdx.x < p.Tc) {
         __syncthreads();
-        if (threadIdx.x == 0) s_ok = wait_count(&hdr->router_done, (uint32_t)(p.E * npass), hdr);
+        if (threadIdx.x == 0) s_ok = wait_count(&hdr->router_done, (uint32_t)(p.E * npass), hdr, p.wait_ns);
         __syncthreads();
         if (!s_ok) return;
         for (int t = blockIdx.x; t < p.Tc; t += G) {
@@ -621,7 +642,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
     if (blockIdx.x == 0) {
         int mine = 0;
         for (int t = 0; t < p.Tc; t += G) ++mine;
-        if (threadIdx.x == 0) s_ok = wait_count(&hdr->topk_done, (uint32_t)(p.Tc - mine), hdr);
+        if (threadIdx.x == 0) s_ok = wait_count(&hdr->topk_done, (uint32_t)(p.Tc - mine), hdr, p.wait_ns);
         __syncthreads();
         if (!s_ok) return;
         if (p.blobs != nullptr) dispatch(p, hdr);

@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -13,6 +14,7 @@
 #include "common.cuh"
 #include "decode_kernels.cuh"
 #include "k3moe.h"
+#include "layer_kernel.cuh"
 #include "layout.cuh"
 #include "prefill_kernels.cuh"
 
@@ -39,6 +41,16 @@ struct DeviceInfo {
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
+
+// Failure-path test settings (k3moe_debug_set_fault): the injected fault and
+// the bound of every device wait, read at each launch.
+std::atomic<int> g_fault_mode{0};
+std::atomic<uint64_t> g_wait_ns{0};
+
+uint64_t wait_limit() {
+    const uint64_t v = g_wait_ns.load(std::memory_order_relaxed);
+    return v ? v : kWaitLimitNs;
+}
 
 k3moe_status cuda_fail(cudaError_t e, const char *where = nullptr) {
     g_last_error = cudaGetErrorString(e);
@@ -74,6 +86,7 @@ k3moe_status device_info(DeviceInfo **out) {
         if (r == cudaSuccess) r = set_smem(umma_expert_kernel<false>, big);
         if (r == cudaSuccess) r = set_smem(pf_expert_kernel<true>, big);
         if (r == cudaSuccess) r = set_smem(pf_expert_kernel<false>, big);
+        if (r == cudaSuccess) r = set_smem(layer_kernel, big);
         if (r != cudaSuccess) return cuda_fail(r);
         di.ready = true;
     }
@@ -97,7 +110,8 @@ int umma_stages(bool gu, int N) {
 
 k3moe_status check_dims(const k3moe_dims *dm) {
     if (!dm) return K3MOE_ERR_INVALID_ARGUMENT;
-    if (dm->flags & ~(K3MOE_OUT_FP32 | K3MOE_NO_SHARED)) return K3MOE_ERR_INVALID_ARGUMENT;
+    if (dm->flags & ~(K3MOE_OUT_FP32 | K3MOE_NO_SHARED | K3MOE_STRICT | K3MOE_RENORM_TOPK | K3MOE_BIAS_SELECT_ONLY))
+        return K3MOE_ERR_INVALID_ARGUMENT;
     if (dm->d < 64 || dm->d > 8192 || dm->d % 64) return K3MOE_ERR_UNSUPPORTED_SHAPE;
     if (dm->ff < 64 || dm->ff > 3072 || dm->ff % 64) return K3MOE_ERR_UNSUPPORTED_SHAPE;
     if (dm->n_experts < 1 || dm->n_experts > 1024) return K3MOE_ERR_UNSUPPORTED_SHAPE;
@@ -106,6 +120,12 @@ k3moe_status check_dims(const k3moe_dims *dm) {
     if (dm->ff_shared < 0 || dm->ff_shared > 3072 || dm->ff_shared % 64)
         return K3MOE_ERR_UNSUPPORTED_SHAPE;
     return K3MOE_OK;
+}
+
+// Routing-variant bits of the kernels' parameters from the call's flags.
+int route_flags(const k3moe_dims *dm) {
+    return ((dm->flags & K3MOE_RENORM_TOPK) ? kRouteRenorm : 0) |
+           ((dm->flags & K3MOE_BIAS_SELECT_ONLY) ? kRouteBiasSelect : 0);
 }
 
 Layout layout_for(const k3moe_dims *dm, int k_eff) {
@@ -265,6 +285,8 @@ cudaError_t launch_umma(const DeviceInfo &di, UmmaParams up, cudaStream_t st) {
     up.nst = umma_stages(GU, N);
     up.sb = umma_stage_bytes(GU, N);
     up.sf_tma = (GU ? up.d : up.ff) % 512 == 0;
+    up.wait_ns = wait_limit();
+    up.inject = GU ? g_fault_mode.load(std::memory_order_relaxed) : 0;
     const int smem = umma_smem_bytes(GU, N, up.nst);
     const int g = di.sms < kMaxCtas ? di.sms : kMaxCtas;
     return launch(umma_expert_kernel<GU>, dim3(g), dim3(kUThreads), smem, st, true, up);
@@ -286,6 +308,7 @@ cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st, int *g
     while (nstage > 2 && route_smem_bytes(rp.d, nt, nstage) > di.route_dyn_max) --nstage;
     if (route_smem_bytes(rp.d, nt, nstage) > di.route_dyn_max) return cudaErrorInvalidConfiguration;
     rp.nstage = nstage;
+    rp.wait_ns = wait_limit();
     if (grid_out) *grid_out = (int)g;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)g);
@@ -298,6 +321,45 @@ cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st, int *g
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, route_kernel, rp);
+}
+
+// The one-launch decode pass (layer_kernel) for this shape, if it fits: the
+// pipeline stages and the routing tables in one SM's shared memory, and the
+// rows of one CTA's router slice in its row accumulators.  0: not supported
+// (the three-kernel pass runs instead).
+int layer_stages(const DeviceInfo &di, const k3moe_dims *dm, int Tc) {
+    const int N = act_n(Tc);
+    const int rest = kSmemLimit - 1024 - lk_smem(dm->n_experts, dm->top_k, Tc, dm->d).total;
+    int nst = rest / lk_stage_bytes(N);
+    if (nst > 8) nst = 8;
+    if (nst < 2) return 0;
+    const long long rf = (long long)dm->n_experts * dm->d;
+    const long long n0 = (rf + kLRUnit - 1) / kLRUnit;
+    const int G = di.sms < kLMaxCtas ? di.sms : kLMaxCtas;
+    const long long g0 = n0 < G ? n0 : G;
+    const long long upc = (n0 + g0 - 1) / g0;  // router units of one CTA at most
+    const long long rows = (upc * kLRUnit + dm->d - 1) / dm->d + 1;
+    if (rows > kRMaxRows) return 0;
+    return nst;
+}
+
+// Cooperative launch: the CTAs wait on each other's counters (router rows,
+// activation pieces, gate/up items), so all of them must be resident.
+cudaError_t launch_layer(const DeviceInfo &di, LayerParams lp, int nst, cudaStream_t st) {
+    const int N = act_n(lp.r.Tc);
+    lp.nst = nst;
+    lp.sb = lk_stage_bytes(N);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(di.sms < kLMaxCtas ? di.sms : kLMaxCtas));
+    cfg.blockDim = dim3(kLThreads);
+    cfg.dynamicSmemBytes = lk_smem_bytes(N, nst, lp.r.E, lp.r.k, lp.r.Tc, lp.r.d);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, layer_kernel, lp);
 }
 
 // Launches of the grouped prefill, pass after pass; rp carries the shapes,
@@ -329,7 +391,7 @@ k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims
         PfRouterParams rr{};
         rr.x = pp.r.x;
         rr.wr = rp.wr;
-        rr.bias = rp.bias;
+        rr.bias = (rp.route_flags & kRouteBiasSelect) ? nullptr : rp.bias;  // in the logits or not
         rr.T = Tq;
         rr.d = d;
         rr.E = E;
@@ -344,7 +406,7 @@ k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims
         e = launch(pf_router_kernel, dim3(gx, gy, ns), dim3(kPrThreads), 0, st, false, rr);
         if (e != cudaSuccess) return cuda_fail(e, "prefill router launch");
         if (ns > 1) {
-            const PfRouterSumParams sp{rr.out, ns, rp.bias, Tq, E, reinterpret_cast<float *>(wsb + P.lg)};
+            const PfRouterSumParams sp{rr.out, ns, rr.bias, Tq, E, reinterpret_cast<float *>(wsb + P.lg)};
             e = launch(pf_router_sum_kernel, dim3(4 * di.sms), dim3(256), 0, st, false, sp);
             if (e != cudaSuccess) return cuda_fail(e, "prefill router sum launch");
         }
@@ -368,6 +430,8 @@ k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims
         up.P = P;
         up.ngs = pp.ngs;
         up.blobs = rp.blobs;
+        up.wait_ns = wait_limit();
+        up.strict = (dims->flags & K3MOE_STRICT) != 0;
         for (int gu = 1; gu >= 0; --gu) {
             const int sb = pf_stage_bytes(gu != 0);
             int nst = (kSmemLimit - pf_smem_bytes(gu != 0, 0)) / sb;
@@ -398,6 +462,7 @@ struct EventHook {
     cudaEvent_t *ev = nullptr;
     int n = 0;
     int next = 0;
+    int kernels = 0;  // kernels of the last pass
     cudaError_t record(cudaStream_t st) {
         if (!ev || next >= n) return cudaSuccess;
         return cudaEventRecord(ev[next++], st);
@@ -467,6 +532,7 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         rp.ws = wsb;
         rp.L = L;
         rp.blobs = expert_blobs;
+        rp.route_flags = route_flags(dims);
         memcpy(rp.tmpl, tmpl, sizeof(tmpl));
         rp.scale_mask = (d % 512 == 0 ? 1 : 0) | (dims->ff % 512 == 0 ? 2 : 0);
         memcpy(rp.smap, smap, sizeof(smap));
@@ -528,6 +594,32 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         EventHook none;
         EventHook &hk = hook ? *hook : none;
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
+        const int lst = 0 * layer_stages(*di, dims, Tc);  // TEMP: layer kernel off until reviewed
+        if (lst > 0) {
+            // the whole pass in one launch
+            LayerParams lp{};
+            lp.r = rp;
+            lp.r.wait_ns = wait_limit();
+            lp.ff = dims->ff;
+            lp.ffs = ffs;
+            lp.sf_tma_gu = d % 512 == 0;
+            lp.sf_tma_dn = dims->ff % 512 == 0;
+            lp.out_fp32 = out32;
+            lp.y = yc;
+            lp.strict = (dims->flags & K3MOE_STRICT) != 0;
+            lp.inject = g_fault_mode.load(std::memory_order_relaxed);
+            e = launch_layer(*di, lp, lst, st);
+            if (e != cudaSuccess) return cuda_fail(e, "layer launch");
+            if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
+            hk.kernels = 1;
+            if (from_host) {
+                e = cudaMemcpyAsync(reinterpret_cast<uint8_t *>(y_host) + (size_t)c0 * d * ybytes, ystage,
+                                    (size_t)Tc * d * ybytes, cudaMemcpyDeviceToHost, st);
+                if (e != cudaSuccess) return cuda_fail(e);
+            }
+            continue;
+        }
+        hk.kernels = 3;
         int route_ctas = 0;
         e = launch_route(*di, rp, st, &route_ctas);
         if (e != cudaSuccess) return cuda_fail(e, "router launch");
@@ -544,6 +636,7 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         up.out_fp32 = out32;
         up.y = yc;
         up.route_ctas = route_ctas;
+        up.strict = (dims->flags & K3MOE_STRICT) != 0;
         e = launch_umma<true>(*di, up, st);
         if (e != cudaSuccess) return cuda_fail(e, "gate/up launch");
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
@@ -561,24 +654,38 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
     return K3MOE_OK;
 }
 
-// The built-in scratch of k3moe_layer_noalloc on this device.  The first
-// call looks up its device address.  The workspace layout depends on the
-// shape, and every layout keeps counters that must start at zero, so the
-// buffer is cleared (on the call's stream) whenever the shape differs from
-// the one it last served, the first call included.
-k3moe_status noalloc_scratch(DeviceInfo &di, const k3moe_dims *dm, cudaStream_t st, uint8_t **out) {
-    std::lock_guard<std::mutex> lock(g_mu);
+// Device address of the built-in scratch of k3moe_layer_noalloc on the
+// current device (looked up on the first use; the caller holds g_mu).
+k3moe_status noalloc_address(DeviceInfo &di) {
     if (!di.noalloc) {
         void *p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_ws);
         if (e != cudaSuccess) return cuda_fail(e, "scratch address");
         di.noalloc = reinterpret_cast<uint8_t *>(p);
     }
+    return K3MOE_OK;
+}
+
+// The built-in scratch of k3moe_layer_noalloc on this device.  The workspace
+// layout depends on the shape, and every layout keeps counters that must
+// start at zero, so the buffer is cleared (on the call's stream) whenever the
+// shape differs from the one it last served, the first call included.  Every
+// call also clears the header's counters (not its status word): a call that
+// gave up part-way (a bounded wait ran out) may have left them raised, and
+// the next call must not take them for its own progress.
+k3moe_status noalloc_scratch(DeviceInfo &di, const k3moe_dims *dm, cudaStream_t st, uint8_t **out) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    k3moe_status s = noalloc_address(di);
+    if (s != K3MOE_OK) return s;
     const int shape[5] = {dm->d, dm->ff, dm->n_experts, dm->top_k, dm->ff_shared};
+    cudaError_t e;
     if (memcmp(shape, di.noalloc_shape, sizeof(shape)) != 0) {
-        cudaError_t e = cudaMemsetAsync(di.noalloc, 0, kNoAllocBytes, st);
+        e = cudaMemsetAsync(di.noalloc, 0, kNoAllocBytes, st);
         if (e != cudaSuccess) return cuda_fail(e, "scratch clear");
         memcpy(di.noalloc_shape, shape, sizeof(shape));
+    } else {
+        e = cudaMemsetAsync(di.noalloc + sizeof(uint32_t), 0, sizeof(WsHeader) - sizeof(uint32_t), st);
+        if (e != cudaSuccess) return cuda_fail(e, "scratch header clear");
     }
     *out = di.noalloc;
     return K3MOE_OK;
@@ -632,6 +739,7 @@ k3moe_status k3moe_route(const void *x, int32_t T, const float *w_router, const 
         rp.k = dims->top_k;
         rp.ws = reinterpret_cast<uint8_t *>(ws);
         rp.L = L;
+        rp.route_flags = route_flags(dims);
         return prefill_impl(*di, rp, dims, reinterpret_cast<const uint16_t *>(x), T, nullptr, idx, weight, st, true);
     }
     for (int c0 = 0; c0 < T; c0 += kChunk) {
@@ -647,6 +755,7 @@ k3moe_status k3moe_route(const void *x, int32_t T, const float *w_router, const 
         rp.ws = reinterpret_cast<uint8_t *>(ws);
         rp.L = L;
         rp.blobs = nullptr;
+        rp.route_flags = route_flags(dims);
         rp.idx_out = idx + (size_t)c0 * dims->top_k;
         rp.w_out = weight + (size_t)c0 * dims->top_k;
         cudaError_t e = launch_route(*di, rp, st);
@@ -702,6 +811,7 @@ k3moe_status k3moe_expert_ffn(const void *x, int32_t T, const uint8_t *blob,
         up.L = L;
         up.out_fp32 = out32;
         up.y = yc;
+        up.strict = (dims->flags & K3MOE_STRICT) != 0;
         e = launch_umma<true>(*di, up, st);
         if (e != cudaSuccess) return cuda_fail(e, "gate/up launch");
         e = launch_umma<false>(*di, up, st);
@@ -744,7 +854,7 @@ k3moe_status k3moe_layer_timed(const void *x, int32_t T, const float *w_router, 
     k3moe_status s = layer_impl(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu,
                                 shared_wd, dims, y, nullptr, nullptr, ws, ws_bytes, stream, nullptr,
                                 nullptr, &hk);
-    *n_kernels = 3;
+    *n_kernels = hk.kernels;
     return s;
 }
 
@@ -768,13 +878,47 @@ k3moe_status k3moe_layer_noalloc(const void *x, int32_t T, const float *w_router
     uint8_t *ws = nullptr;
     s = noalloc_scratch(*di, dims, st, &ws);
     if (s != K3MOE_OK) return s;
+    // a workspace sized for one 8-token pass: any T runs as 8-token decode
+    // passes (the grouped path's region would not fit in the buffer)
     return layer_impl(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu, shared_wd, dims, y,
-                      nullptr, nullptr, ws, kNoAllocBytes, stream, nullptr, nullptr);
+                      nullptr, nullptr, ws, need, stream, nullptr, nullptr);
 }
 
 k3moe_status k3moe_device_status(void *ws, void *stream) {
-    if (!ws || !aligned(ws, 256)) return K3MOE_ERR_INVALID_ARGUMENT;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (ws == nullptr) {
+        // the built-in scratch of k3moe_layer_noalloc on the current device
+        DeviceInfo *di = nullptr;
+        k3moe_status s = device_info(&di);
+        if (s != K3MOE_OK) return s;
+        uint8_t *buf = nullptr;
+        {
+            std::lock_guard<std::mutex> lock(g_mu);
+            s = noalloc_address(*di);
+            if (s != K3MOE_OK) return s;
+            buf = di->noalloc;
+        }
+        cudaError_t e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cuda_fail(e);
+        WsHeader h;
+        e = cudaMemcpy(&h, buf, sizeof(h), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (h.status & kStTimeout) {
+            // a call gave up part-way: every counter in the buffer may be
+            // raised, so the whole buffer starts again from zero
+            e = cudaMemset(buf, 0, kNoAllocBytes);
+            if (e == cudaSuccess) e = cudaDeviceSynchronize();
+            if (e != cudaSuccess) return cuda_fail(e, "scratch clear");
+            return K3MOE_ERR_DEVICE_TIMEOUT;
+        }
+        if (h.status != 0u) {
+            const uint32_t zero = 0u;
+            e = cudaMemcpy(buf, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        return (h.status & kStDeviceCheck) ? K3MOE_ERR_DEVICE_CHECK : K3MOE_OK;
+    }
+    if (!aligned(ws, 256)) return K3MOE_ERR_INVALID_ARGUMENT;
     cudaError_t e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e);
     WsHeader h;
@@ -807,5 +951,12 @@ const char *k3moe_status_string(k3moe_status status) {
 }
 
 const char *k3moe_last_error(void) { return g_last_error.c_str(); }
+
+k3moe_status k3moe_debug_set_fault(int32_t mode, uint64_t wait_limit_ns) {
+    if (mode < 0 || mode > 1) return K3MOE_ERR_INVALID_ARGUMENT;
+    g_fault_mode.store(mode, std::memory_order_relaxed);
+    g_wait_ns.store(wait_limit_ns, std::memory_order_relaxed);
+    return K3MOE_OK;
+}
 
 }  // extern "C"

@@ -1,0 +1,1100 @@
+// The whole decode layer for one pass of up to kChunk tokens in ONE
+// persistent launch (one CTA per SM): router GEMV, softmax and top-k, the
+// dispatch, the shared expert and the routed experts' gate/up + SwiGLU and
+// down projections with the weighted combine.  Layer structure: the tutorial
+// page's section 2.4 moe_forward (gate scores over all experts, softmax,
+// top-k, each selected expert's FFN, weighted combine) and section 1.2's
+// always-on shared expert; the routed experts' packed MXFP4 weights go
+// straight into the tensor cores (the kimi-k3-in-c project card, core
+// features).
+//
+// Every CTA runs the same four ranges of "units" (each range split evenly
+// over the CTAs, stream-K) through one ring of shared-memory stages:
+//   R0  the fp32 router, 32 KB per unit (bulk copies), summed on the CUDA
+//       cores by the scale warps (their tensor-memory work starts later);
+//   R1  the shared expert's gate/up (bf16 MMAs, x as bf16);
+//   R2  the routed experts' gate/up (block-scaled kind::mxf4 MMAs, x as E2M1
+//       pieces), once the routing is known;
+//   R3  the down projections: one accumulator per 128 rows of d, K running
+//       over every distinct routed expert's ff (two 256-weight K-tiles per
+//       unit) and then the shared expert's ff_s (two 64-weight bf16 K-tiles
+//       per unit), so the routing weights (folded into the activation pieces)
+//       and the shared expert are combined by the tensor core itself.
+// So the router bytes and the shared expert stream while the routing is
+// still being decided, and the W_d tiles of the first down units are loaded
+// before the gate/up results they multiply are complete (only their B tiles
+// wait).
+//
+// Routing in every CTA: once all router rows are in (a counter in the
+// workspace header), warps 0-3 and 10 each take a token and find its top-k
+// with warp reductions, then warp 10 builds the dispatch (distinct experts in
+// ascending id, each token's weight per expert) in shared memory -- every CTA
+// derives the same routing from the same logits, so no further grid-wide
+// exchange is needed before the routed units start.
+//
+// Roles (352 threads): warps 0-3 epilogue (one TMEM lane quadrant each; they
+// also take part in the top-k), warps 4-7 router sums (R0) and scale factors
+// into TMEM (R2, R3), warp 8 copies (TMA, bulk), warp 9 MMA issue, warp 10
+// set-up (tensor maps, activation pieces), top-k and dispatch.
+#pragma once
+
+#include "common.cuh"
+#include "decode_kernels.cuh"
+#include "layout.cuh"
+#include "umma.cuh"
+#include "umma_kernels.cuh"
+
+namespace k3 {
+
+constexpr int kLThreads = 352;
+constexpr int kLMaxCtas = 160;        // grid cap (one CTA per SM)
+constexpr int kLRUnit = 8192;         // router floats per R0 unit (32 KB)
+constexpr int kLSfc = 32;             // TMEM scale columns per stage
+constexpr int kLSegMax = 32;          // row segments per warp and router unit (d >= 64)
+constexpr int kLTopkWarps = 5;        // warps 0-3 and 10
+
+struct LayerParams {
+    RouteParams r;     // x, Tc, router, shapes, workspace, blobs, maps, wait_ns
+    int ff, ffs;       // expert and shared-expert hidden sizes (ffs 0: none)
+    int nst, sb;       // pipeline stages, bytes per stage
+    int sf_tma_gu;     // W_g / W_u scales by TMA (d a multiple of 512)
+    int sf_tma_dn;     // W_d scales by TMA (ff a multiple of 512)
+    int out_fp32;
+    void *y;           // [Tc][d] of this pass
+    int strict;        // flag E8M0 NaN bytes among the weight scales read
+    int inject;        // failure-path tests: 1 = the routing is never signalled
+};
+
+// ---------------------------------------------------------- smem layout --
+// One stage: two A boxes (2 x 16 KB, 1024-byte aligned for the 128-byte
+// swizzle; a router unit fills both), two B tiles of N rows x 128 bytes, two
+// A scale boxes (128 rows x 16 bytes), two B scale blocks (2 x kSfRow words).
+__host__ __device__ inline int lk_b_off() { return 2 * kAtile; }
+__host__ __device__ inline int lk_sfa_off(int N) { return 2 * kAtile + 2 * N * 128; }
+__host__ __device__ inline int lk_sfb_off(int N) { return lk_sfa_off(N) + 2 * 2048; }
+__host__ __device__ inline int lk_stage_bytes(int N) { return (lk_sfb_off(N) + 2 * 2 * kSfRow * 4 + 1023) & ~1023; }
+
+// The rest, after the stages (byte offsets from the end of the stages),
+// sized for this pass: E experts, top-k, Tc tokens, hidden size d.
+struct LkSmem {
+    int segs;  // row segments one warp's 2048 router floats can touch
+    int bars, ptab, blob, eid, wu, tidx, tw, racc, segr, segv, segn, misc, total;
+};
+__host__ __device__ inline LkSmem lk_smem(int E, int k, int Tc, int d) {
+    LkSmem s;
+    const int umax = E < Tc * k ? E : Tc * k;
+    s.segs = 2047 / d + 2 < kLSegMax ? 2047 / d + 2 : kLSegMax;
+    auto a16 = [](int v) { return (v + 15) & ~15; };
+    int o = 0;
+    s.bars = o;   o += 512;                           // mbarriers, TMEM slot, flags
+    s.ptab = o;   o += a16(E * 8);                    // blob pointer of every expert
+    s.blob = o;   o += a16(umax * 8);                 // per distinct expert: blob pointer,
+    s.eid = o;    o += a16(umax * 4);                 //   expert id,
+    s.wu = o;     o += a16(umax * Tc * 4);            //   weight of each token (0: not selected)
+    s.tidx = o;   o += Tc * 32 * 4;                   // top-k of each token: experts
+    s.tw = o;     o += Tc * 32 * 4;                   //   and weights
+    s.racc = o;   o += a16(kRMaxRows * Tc * 4);       // router row sums of this CTA's slice
+    s.segr = o;   o += a16(2 * 4 * s.segs * 4);       // per-warp row segments of a unit (x2)
+    s.segv = o;   o += a16(2 * 4 * s.segs * Tc * 4);
+    s.segn = o;   o += 2 * 4 * 4;
+    s.misc = o;   o += 64 * 4;                        // dispatch bitmap / prefix
+    s.total = o;
+    return s;
+}
+__host__ __device__ inline int lk_smem_bytes(int N, int nst, int E, int k, int Tc, int d) {
+    return 1024 + nst * lk_stage_bytes(N) + lk_smem(E, k, Tc, d).total;
+}
+
+// --------------------------------------------------------------- top-k --
+// Softmax over all E logits and the top-k of one token, by one warp.  Lane l
+// holds experts l, l + 32, ...  The k winners come out one per round: the
+// largest key (order-preserving bits of the logit) over every lane's best,
+// the lowest expert id among equal keys, so the picks are in descending
+// logit with ties to the lower index.  Each lane keeps its best and second
+// best candidates: on a win the second becomes the best, so a lane rescans
+// its values only on every other win.  w = exp(l - max) / sum over all E of
+// exp(l_e - max), fp32.  sel_bias (non-null): the selection runs on
+// l + sel_bias[e], the softmax on l; renorm: the k weights are divided by
+// their sum.
+__device__ void warp_topk(const float *row, int E, int k, int32_t *idx_out, float *w_out,
+                          const float *sel_bias, bool renorm) {
+    const int lane = threadIdx.x & 31;
+    constexpr int kPer = 32;  // E <= 1024
+    uint32_t key[kPer];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int e = lane + 32 * i;
+        const float v = e < E ? __ldcg(row + e) : -INFINITY;
+        key[i] = e < E ? fkey(sel_bias ? v + __ldg(sel_bias + e) : v) : 0u;  // real keys are > 0
+        mx = fmaxf(mx, v);
+    }
+    const float m = fkey_value(__reduce_max_sync(0xffffffffu, fkey(mx)));
+    // the softmax runs on the logits themselves (read again when the keys
+    // hold biased scores)
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) sum += expf((sel_bias ? __ldcg(row + e) : fkey_value(key[i])) - m);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float inv_s = 1.0f / sum;
+    uint32_t taken = 0u;
+    // best and second best (key, slot) of this lane, first slot on equal keys
+    auto rescan = [&](uint32_t &k1, int &i1, uint32_t &k2, int &i2) {
+        k1 = 0u; i1 = -1; k2 = 0u; i2 = -1;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const uint32_t kv = ((taken >> i) & 1u) ? 0u : key[i];
+            if (kv > k1) {
+                k2 = k1; i2 = i1; k1 = kv; i1 = i;
+            } else if (kv > k2) {
+                k2 = kv; i2 = i;
+            }
+        }
+    };
+    uint32_t k1, k2;
+    int i1, i2;
+    rescan(k1, i1, k2, i2);
+    for (int j = 0; j < k; ++j) {
+        const uint32_t K = __reduce_max_sync(0xffffffffu, k1);
+        const uint32_t cand = (k1 == K && i1 >= 0) ? (uint32_t)(lane + 32 * i1) : 0xFFFFFFFFu;
+        const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+        if (lane == 0) {
+            idx_out[j] = (int32_t)win;
+            w_out[j] = fkey_value(K);  // the pick's key value (its logit when unbiased)
+        }
+        if ((int)(win & 31u) == lane) {
+            taken |= 1u << i1;
+            if (i2 >= 0) {
+                // the second best becomes the best; the lane looks for a new
+                // second only if it wins again
+                k1 = k2; i1 = i2; k2 = 0u; i2 = -1;
+            } else {
+                rescan(k1, i1, k2, i2);
+            }
+        }
+        __syncwarp();
+    }
+    // weights: lane j takes pick j
+    float num = 0.f;
+    if (lane < k) {
+        const float lv = sel_bias ? __ldcg(row + idx_out[lane]) : w_out[lane];
+        num = expf(lv - m);
+    }
+    float w = num * inv_s;
+    if (renorm) {
+        float z = num;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        w = num / z;
+    }
+    __syncwarp();
+    if (lane < k) w_out[lane] = w;
+    __syncwarp();
+}
+
+// --------------------------------------------------------------- kernel --
+__global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_constant__ LayerParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const RouteParams &rp = p.r;
+    const Layout &L = rp.L;
+    const int nst = p.nst, SB = p.sb, Tc = rp.Tc, N = act_n(Tc);
+    const int d = rp.d, E = rp.E, k = rp.k;
+    const LkSmem so = lk_smem(E, k, Tc, d);
+    const int SG = so.segs;
+    uint8_t *tail = smem + nst * SB;
+    uint64_t *full = reinterpret_cast<uint64_t *>(tail + so.bars);  // stage bytes landed
+    uint64_t *sfr = full + 8;                                        // stage scales in TMEM (4 warps)
+    uint64_t *empty = sfr + 8;                                       // stage consumed
+    uint64_t *afull = empty + 8;
+    uint64_t *aempty = afull + 2;
+    uint64_t *mready = aempty + 2;  // the routing is in shared memory
+    uint64_t *mdone = mready + 1;   // every MMA this CTA issued has completed
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(mdone + 1);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(tslot + 1);
+    volatile int *s_U = s_abort + 1;
+    volatile int *s_last = s_abort + 2;
+    const uint8_t **s_ptab = reinterpret_cast<const uint8_t **>(tail + so.ptab);
+    const uint8_t **s_blob = reinterpret_cast<const uint8_t **>(tail + so.blob);
+    int32_t *s_eid = reinterpret_cast<int32_t *>(tail + so.eid);
+    float *s_wu = reinterpret_cast<float *>(tail + so.wu);      // [u][Tc]
+    int32_t *s_tidx = reinterpret_cast<int32_t *>(tail + so.tidx);  // [t][32]
+    float *s_tw = reinterpret_cast<float *>(tail + so.tw);
+    float *s_racc = reinterpret_cast<float *>(tail + so.racc);  // [row][Tc]
+    int *s_segr = reinterpret_cast<int *>(tail + so.segr);      // [2][4][SG]
+    float *s_segv = reinterpret_cast<float *>(tail + so.segv);  // [2][4][SG][Tc]
+    int *s_segn = reinterpret_cast<int *>(tail + so.segn);      // [2][4]
+    uint32_t *s_misc = reinterpret_cast<uint32_t *>(tail + so.misc);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(rp.ws + L.hdr);
+    const int G = gridDim.x, cta = blockIdx.x;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nst; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&sfr[s], 4);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&afull[b], 1);
+            mbar_init(&aempty[b], 4);
+        }
+        mbar_init(mready, 1);
+        mbar_init(mdone, 1);
+        fence_mbar_init();
+        *s_abort = 0;
+        *s_U = 0;
+    }
+    constexpr uint32_t kCols = 512u;
+    if (warp == 0) umma::tmem_alloc(tslot, kCols);
+    umma::fence_before();
+    __syncthreads();
+    umma::fence_after();
+    const uint32_t tbase = *tslot;
+    // TMEM columns: accumulators [buf][mat] at (2*buf + mat) * 64 (N <= 48),
+    // then kLSfc scale columns per stage: A box 0 (+0), A box 1 (+8), B tile
+    // 0 (+16), B tile 1 (+24).
+    const uint32_t sf0 = 256u;
+
+    // ------------------------------------------------------------ shapes --
+    const int ffs = p.ffs, ff = p.ff;
+    const long long rfloats = (long long)E * d;
+    const int n0 = (int)((rfloats + kLRUnit - 1) / kLRUnit);   // router units
+    const int nkts_d = ceil_div(d, kTileKs);                    // shared gate/up K-tiles (64)
+    const int nrbs = ffs > 0 ? ceil_div(ffs, kTileM) : 0;       // shared gate/up items
+    const int nkt_d = ceil_div(d, kTileK);                      // routed gate/up K-tiles (256)
+    const int nrb_ff = ceil_div(ff, kTileM);                    // routed gate/up items per expert
+    const int nkt_ff = ceil_div(ff, kTileK);                    // routed down K-tiles per expert
+    const int ndu = (nkt_ff + 1) / 2;                           // ... in units of two
+    const int nkts_ffs = ffs > 0 ? ceil_div(ffs, kTileKs) : 0;  // shared down K-tiles (64)
+    const int nsdu = (nkts_ffs + 1) / 2;
+    const int nrb_d = ceil_div(d, kTileM);                      // down items
+    int U = 0;                                                  // distinct routed experts (after mready)
+
+    // A range of n units split evenly over the CTAs (CTA c of G' = min(G, n)
+    // takes [c n / G', (c+1) n / G')); an item cut between CTAs is finished
+    // by the last of them to arrive.
+    struct Range {
+        int n, G, a, b;
+    };
+    auto make_range = [&](int n) {
+        Range r;
+        r.n = n;
+        r.G = min(G, max(n, 1));
+        r.a = cta < r.G && n > 0 ? (int)(((long long)cta * n) / r.G) : 0;
+        r.b = cta < r.G && n > 0 ? (int)(((long long)(cta + 1) * n) / r.G) : 0;
+        return r;
+    };
+    auto start_of = [&](const Range &r, int c) { return (int)(((long long)c * r.n) / r.G); };
+    auto owner = [&](const Range &r, int unit) { return (int)((((long long)unit + 1) * r.G - 1) / r.n); };
+    Range rg[4];
+    rg[0] = make_range(n0);
+    rg[1] = make_range(nrbs * nkts_d);
+    rg[2] = make_range(0);
+    rg[3] = make_range(0);
+    // units per item of the ranges with items (R1, R2, R3)
+    auto upi = [&](int r) { return r == 1 ? nkts_d : (r == 2 ? nkt_d : U * ndu + nsdu); };
+    // Bounded wait that gives up at once after any role has given up.
+    auto wait = [&](uint64_t *bar, uint32_t parity) {
+        if (*s_abort) return false;
+        if (mbar_wait_bounded(bar, parity, hdr, rp.wait_ns)) return true;
+        *s_abort = 1;
+        return false;
+    };
+    // Before R2: the routing (one lane waits, its warp follows when warp_wide).
+    auto routed_ranges = [&](bool warp_wide) {
+        int ok = 1;
+        if (lane == 0) {
+            ok = (!*s_abort && mbar_wait_bounded(mready, 0u, hdr, rp.wait_ns)) ? 1 : 0;
+            if (!ok) *s_abort = 1;
+        }
+        if (warp_wide) ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) return false;
+        U = *s_U;
+        rg[2] = make_range(U * nrb_ff * nkt_d);
+        rg[3] = make_range(nrb_d * (U * ndu + nsdu));
+        return true;
+    };
+    // Unit u of range r (r >= 1): item, its unit span, expert, row block,
+    // first K-tile and K-tiles in the unit; kind 1 shared gate/up, 2 routed
+    // gate/up, 3 routed down, 4 shared down.
+    struct Unit {
+        int kind, item, istart, iend, u, rb, kt, nt;
+    };
+    auto decode = [&](int r, int unit) {
+        Unit x;
+        const int per = upi(r);
+        x.item = unit / per;
+        x.istart = x.item * per;
+        x.iend = x.istart + per;
+        const int j = unit - x.istart;
+        if (r == 1) {
+            x.kind = 1; x.u = -1; x.rb = x.item; x.kt = j; x.nt = 1;
+        } else if (r == 2) {
+            x.kind = 2; x.u = x.item / nrb_ff; x.rb = x.item - x.u * nrb_ff; x.kt = j; x.nt = 1;
+        } else {
+            x.rb = x.item;
+            if (j < U * ndu) {
+                x.kind = 3; x.u = j / ndu; x.kt = 2 * (j - x.u * ndu); x.nt = min(2, nkt_ff - x.kt);
+            } else {
+                x.kind = 4; x.u = -1; x.kt = 2 * (j - U * ndu); x.nt = min(2, nkts_ffs - x.kt);
+            }
+        }
+        return x;
+    };
+    const size_t mat = (size_t)d * ff;
+    const uint8_t *smaps = rp.ws + L.tmap + (size_t)E * kMapsPerExpert * 128;
+
+    if (warp == 10) {
+        // ================================================= set-up, routing --
+        // blob pointers of every expert -> shared memory (the dispatch reads
+        // them); tensor maps of this CTA's share of the experts (and, in CTA
+        // 0, the shared expert's); this CTA's share of the activation pieces
+        // (x as E2M1 pieces for R2, as bf16 for R1).  Then counted on
+        // prep_done, which the copies warps wait for before their first
+        // B tile or tensor map.
+        for (int e = lane; e < E; e += 32) s_ptab[e] = rp.blobs[e];
+        refresh_tmaps(rp, cta * 32 + lane, G * 32);
+        build_x_pieces(rp.x, Tc, d, rp.ws, L, cta, G, rp.has_shared != 0);
+        __syncwarp();
+        if (lane == 0) red_add_release(&hdr->prep_done, 1u);
+    }
+
+    if (warp < 4 || warp == 10) {
+        // top-k of the tokens, warps 0-3 and 10 (160 threads) once every
+        // router row is in
+        const int tw = warp == 10 ? 4 : warp;
+        int ok = 1;
+        if (lane == 0) {
+            const uint64_t t0 = globaltimer();
+            while (ld_acquire(&hdr->router_done) < (uint32_t)E) {
+                if (*s_abort || globaltimer() - t0 > rp.wait_ns) {
+                    set_status(hdr, kStTimeout);
+                    *s_abort = 1;
+                    ok = 0;
+                    break;
+                }
+            }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (ok) {
+            const float *logits = reinterpret_cast<const float *>(rp.ws + L.logits);
+            for (int t = tw; t < Tc; t += kLTopkWarps)
+                warp_topk(logits + (size_t)t * E, E, k, s_tidx + t * 32, s_tw + t * 32,
+                          (rp.route_flags & kRouteBiasSelect) ? rp.bias : nullptr, (rp.route_flags & kRouteRenorm) != 0);
+        }
+        umma::bar_sync(3, 32 * kLTopkWarps);
+        if (warp == 10 && ok && !*s_abort) {
+            // dispatch: distinct experts in ascending id (bitmap + prefix),
+            // each one's blob (checked) and per-token weight
+            uint32_t *bitmap = s_misc, *prefix = s_misc + 32;
+            const int nwords = (E + 31) >> 5;
+            bitmap[lane] = 0u;
+            __syncwarp();
+            for (int i = lane; i < Tc * k; i += 32) {
+                const int e = s_tidx[(i / k) * 32 + i % k];
+                atomicOr(&bitmap[e >> 5], 1u << (e & 31));
+            }
+            __syncwarp();
+            const uint32_t c = lane < nwords ? __popc(bitmap[lane]) : 0u;
+            uint32_t incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            prefix[lane] = incl - c;
+            const int Ut = (int)__shfl_sync(0xffffffffu, incl, 31);
+            __syncwarp();
+            for (int i = lane; i < Ut * Tc; i += 32) s_wu[i] = 0.f;
+            for (int w = lane; w < nwords * 32; w += 32) {
+                if ((bitmap[w >> 5] >> (w & 31)) & 1u) {
+                    const uint32_t u = prefix[w >> 5] + __popc(bitmap[w >> 5] & ((1u << (w & 31)) - 1u));
+                    const uint8_t *b = s_ptab[w];
+                    if (b == nullptr || (reinterpret_cast<uintptr_t>(b) & 15u) != 0u) {
+                        set_status(hdr, kStDeviceCheck);
+                        b = nullptr;
+                    }
+                    s_blob[u] = b;
+                    s_eid[u] = w;
+                }
+            }
+            __syncwarp();
+            for (int i = lane; i < Tc * k; i += 32) {
+                const int t = i / k, j = i - t * k;
+                const int e = s_tidx[t * 32 + j];
+                const uint32_t u = prefix[e >> 5] + __popc(bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
+                s_wu[u * Tc + t] = s_tw[t * 32 + j];
+                if (cta == 0) {
+                    if (rp.idx_out) rp.idx_out[(size_t)t * k + j] = e;
+                    if (rp.w_out) rp.w_out[(size_t)t * k + j] = s_tw[t * 32 + j];
+                }
+            }
+            if (lane == 0) {
+                *s_U = Ut;
+                if (cta == 0) hdr->n_unique = (uint32_t)Ut;
+            }
+            __syncwarp();
+            if (lane == 0 && p.inject != 1)
+                asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(mready)) : "memory");
+        }
+    }
+
+    if (warp == 8) {
+        // ========================================================= copies --
+        if (lane == 0) {
+            int i = 0;  // this CTA's unit counter over all ranges (stage i % nst)
+            bool prep_ok = false, gu_ok = false;
+            uint32_t gu_total = 0u;
+            // B tiles of down units whose weights are issued but whose
+            // activations were not ready yet (at most nst, in stage order)
+            int pend_s[8], pend_unit[8];
+            int npend = 0;
+            auto issue_b = [&](int s, const Unit &x) {
+                uint8_t *st = smem + s * SB;
+                // the B scale words travel with the stage when the A scales do
+                const bool sfb = x.kind == 3 && p.sf_tma_dn && s_blob[x.u] != nullptr;
+                for (int tt = 0; tt < x.nt; ++tt) {
+                    const size_t bt = x.kind == 3 ? (size_t)x.u * nkt_ff + x.kt + tt : (size_t)(x.kt + tt);
+                    const uint8_t *bsrc = x.kind == 3 ? rp.ws + L.hb + bt * N * 128 : rp.ws + L.hsb + bt * N * 128;
+                    bulk_g2s(st + lk_b_off() + tt * N * 128, bsrc, (uint32_t)(N * 128), &full[s]);
+                    if (sfb)
+                        bulk_g2s(st + lk_sfb_off(N) + tt * 2 * kSfRow * 4, rp.ws + L.hsf + bt * 2 * kSfRow * 4,
+                                 (uint32_t)(2 * kSfRow * 4), &full[s]);
+                }
+            };
+            auto gu_ready = [&](bool block) {
+                if (gu_ok) return true;
+                const uint64_t t0 = globaltimer();
+                while (ld_acquire(&hdr->gu_done) < gu_total) {
+                    if (!block) return false;
+                    if (*s_abort || globaltimer() - t0 > rp.wait_ns) {
+                        set_status(hdr, kStTimeout);
+                        *s_abort = 1;
+                        return false;
+                    }
+                }
+                asm volatile("fence.proxy.async.global;" ::: "memory");  // before bulk copies read h
+                gu_ok = true;
+                return true;
+            };
+            for (int r = 0; r < 4 && !*s_abort; ++r) {
+                if (r == 2) {
+                    if (!routed_ranges(false)) break;
+                    gu_total = (uint32_t)(nrbs + U * nrb_ff);
+                }
+                const Range R = rg[r];
+                for (int unit = R.a; unit < R.b && !*s_abort; ++unit, ++i) {
+                    const int s = i % nst;
+                    const uint32_t ph = (uint32_t)((i / nst) & 1);
+                    if (r == 3 && npend == nst) {
+                        // every stage waits for activations: wait for them
+                        if (!gu_ready(true)) break;
+                        for (int q = 0; q < npend; ++q) issue_b(pend_s[q], decode(3, pend_unit[q]));
+                        npend = 0;
+                    }
+                    if (r == 3 && npend > 0 && gu_ready(false)) {
+                        for (int q = 0; q < npend; ++q) issue_b(pend_s[q], decode(3, pend_unit[q]));
+                        npend = 0;
+                    }
+                    if (i >= nst && !wait(&empty[s], ph ^ 1u)) break;
+                    uint8_t *st = smem + s * SB;
+                    if (r == 0) {
+                        const long long f0 = (long long)unit * kLRUnit;
+                        const long long f1 = min(rfloats, f0 + kLRUnit);
+                        const uint32_t bytes = (uint32_t)((f1 - f0) * 4);
+                        mbar_arrive_expect_tx(&full[s], bytes);
+                        bulk_g2s(st, rp.wr + f0, bytes, &full[s]);
+                        continue;
+                    }
+                    if (!prep_ok) {
+                        // x pieces, x as bf16 and the tensor maps are published
+                        // by every CTA's set-up warp
+                        const uint64_t t0 = globaltimer();
+                        bool ok = true;
+                        while (ld_acquire(&hdr->prep_done) < (uint32_t)G) {
+                            if (globaltimer() - t0 > rp.wait_ns) {
+                                set_status(hdr, kStTimeout);
+                                *s_abort = 1;
+                                ok = false;
+                                break;
+                            }
+                        }
+                        if (!ok) break;
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                        prep_ok = true;
+                    }
+                    const Unit x = decode(r, unit);
+                    const uint8_t *maps, *scmaps = nullptr;
+                    bool blob_ok = true;
+                    if (x.kind == 1 || x.kind == 4) {
+                        maps = smaps + (x.kind == 1 ? 0 : 256);
+                    } else {
+                        const uint8_t *em = rp.ws + L.tmap + (size_t)s_eid[x.u] * kMapsPerExpert * 128;
+                        maps = em + (x.kind == 2 ? 0 : 256);
+                        scmaps = em + (x.kind == 2 ? 384 : 640);
+                        blob_ok = s_blob[x.u] != nullptr;
+                    }
+                    const bool sf_dma = blob_ok && ((x.kind == 2 && p.sf_tma_gu) || (x.kind == 3 && p.sf_tma_dn));
+                    // bytes: A boxes, B tiles, A scale box(es), B scale words
+                    uint32_t tx = 0u;
+                    const int nbox = (x.kind == 1 || x.kind == 2) ? 2 : x.nt;
+                    const int nb = (x.kind == 1 || x.kind == 2) ? 1 : x.nt;
+                    if (blob_ok) tx += (uint32_t)(nbox * kAtile);
+                    tx += (uint32_t)(nb * N * 128);
+                    if (sf_dma) tx += (uint32_t)((x.kind == 2 ? 2 : 1) * 2048 + nb * 2 * kSfRow * 4);
+                    mbar_arrive_expect_tx(&full[s], tx);
+                    if (blob_ok) {
+                        umma::tmap_acquire(maps);
+                        if (x.kind <= 2) {
+                            // gate/up: W_g box and W_u box of K-tile kt (128 bytes of every row)
+                            umma::tmap_acquire(maps + 128);
+                            umma::tma_load_2d(st, maps, x.kt * 128, x.rb * kTileM, &full[s]);
+                            umma::tma_load_2d(st + kAtile, maps + 128, x.kt * 128, x.rb * kTileM, &full[s]);
+                        } else {
+                            for (int tt = 0; tt < x.nt; ++tt)
+                                umma::tma_load_2d(st + tt * kAtile, maps, (x.kt + tt) * 128, x.rb * kTileM, &full[s]);
+                        }
+                        if (sf_dma) {
+                            uint8_t *sfa = st + lk_sfa_off(N);
+                            umma::tmap_acquire(scmaps);
+                            umma::tma_load_2d(sfa, scmaps, (x.kt >> 1) * 16, x.rb * kTileM, &full[s]);
+                            if (x.kind == 2) {
+                                umma::tmap_acquire(scmaps + 128);
+                                umma::tma_load_2d(sfa + 2048, scmaps + 128, (x.kt >> 1) * 16, x.rb * kTileM, &full[s]);
+                            }
+                        }
+                    }
+                    if (x.kind == 1) {
+                        bulk_g2s(st + lk_b_off(), rp.ws + L.xbf + (size_t)x.kt * N * 128, (uint32_t)(N * 128), &full[s]);
+                    } else if (x.kind == 2) {
+                        bulk_g2s(st + lk_b_off(), rp.ws + L.xb + (size_t)x.kt * N * 128, (uint32_t)(N * 128), &full[s]);
+                        if (sf_dma)
+                            bulk_g2s(st + lk_sfb_off(N), rp.ws + L.xsf + (size_t)x.kt * 2 * kSfRow * 4,
+                                     (uint32_t)(2 * kSfRow * 4), &full[s]);
+                    } else if (gu_ready(false)) {
+                        issue_b(s, x);
+                    } else {
+                        pend_s[npend] = s;
+                        pend_unit[npend] = unit;
+                        ++npend;
+                    }
+                }
+            }
+            if (npend > 0 && !*s_abort && gu_ready(true)) {
+                for (int q = 0; q < npend; ++q) issue_b(pend_s[q], decode(3, pend_unit[q]));
+                npend = 0;
+            }
+            if (*s_abort) {
+                // a wait gave up somewhere: wait (bounded) for the last copy
+                // issued into each stage, so none lands after the CTA's
+                // shared memory is released
+                for (int q = 0; q < nst && q < i; ++q) {
+                    const int last = q + ((i - 1 - q) / nst) * nst;
+                    mbar_drain(&full[q], (uint32_t)((last / nst) & 1), rp.wait_ns);
+                }
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ============================ router sums (R0), scales -> TMEM =====
+        const int tid = threadIdx.x - 128;  // 0..127
+        const int wl = warp - 4;
+        const uint32_t lb = umma::lane_base(warp);
+        uint32_t nanb = 0u;
+        // this CTA's router slice: floats [f_lo, f_hi), rows row_base ..
+        const Range R0 = rg[0];
+        const long long f_lo = (long long)R0.a * kLRUnit, f_hi = min(rfloats, (long long)R0.b * kLRUnit);
+        const int row_base = R0.a < R0.b ? (int)(f_lo / d) : 0;
+        const int nrows = R0.a < R0.b ? (int)((f_hi - 1) / d) - row_base + 1 : 0;
+        for (int q = tid; q < kRMaxRows * Tc; q += 128) s_racc[q] = 0.f;
+        umma::bar_sync(2, 128);
+        int i = 0;
+        bool go = true;
+        bool act_ok[2] = {false, false};  // x pieces' scales / h pieces' scales seen (no-TMA path)
+        for (int r = 0; r < 4 && go; ++r) {
+            if (r == 2 && !routed_ranges(true)) break;
+            const Range R = rg[r];
+            for (int unit = R.a; unit < R.b; ++unit, ++i) {
+                const int s = i % nst;
+                const uint32_t ph = (uint32_t)((i / nst) & 1);
+                int ok = 0;
+                if (lane == 0) ok = wait(&full[s], ph) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                // router units end in a barrier of the four warps: they agree
+                // on going on, so none is left waiting at it
+                if (r == 0) ok = umma::bar_red_and(2, 128, ok != 0) ? 1 : 0;
+                if (!ok) {
+                    go = false;
+                    break;
+                }
+                (void)mbar_try_wait(&full[s], ph);  // every lane sees the landed bytes
+                const uint8_t *st = smem + s * SB;
+                if (r == 0) {
+                    // 64 consecutive floats per thread (one row: d is a multiple
+                    // of 64), every token; then the warp's sums per row
+                    // (segmented, fixed order) into this unit's buffers
+                    const long long f = (long long)unit * kLRUnit + 64LL * tid;
+                    int row = -1;
+                    float v[kChunk];
+#pragma unroll
+                    for (int t = 0; t < kChunk; ++t) v[t] = 0.f;
+                    if (f < f_hi) {
+                        row = (int)(f / d);
+                        const int col = (int)(f - (long long)row * d);
+                        // the 16 float4 of this thread's 64 floats, starting at
+                        // (lane mod 16) so that a warp's loads spread over the
+                        // banks; each product is exact, each sum fp32 in this order
+                        const float4 *w4 = reinterpret_cast<const float4 *>(st) + tid * 16;
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const int jq = (q + lane) & 15;
+                            const float4 a = w4[jq];
+#pragma unroll
+                            for (int t = 0; t < kChunk; ++t) {
+                                if (t < Tc) {
+                                    const uint2 xw = __ldg(reinterpret_cast<const uint2 *>(rp.x + (size_t)t * d + col) + jq);
+                                    v[t] = fmaf(a.x, bf16_lo(xw.x), v[t]);
+                                    v[t] = fmaf(a.y, bf16_hi(xw.x), v[t]);
+                                    v[t] = fmaf(a.z, bf16_lo(xw.y), v[t]);
+                                    v[t] = fmaf(a.w, bf16_hi(xw.y), v[t]);
+                                }
+                            }
+                        }
+                    }
+                    // segmented sum over lanes of equal row (rows do not decrease along lanes)
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int rn = __shfl_down_sync(0xffffffffu, row, o);
+#pragma unroll
+                        for (int t = 0; t < kChunk; ++t) {
+                            const float vn = __shfl_down_sync(0xffffffffu, v[t], o);
+                            if (lane + o < 32 && rn == row) v[t] += vn;
+                        }
+                    }
+                    const int rprev = __shfl_up_sync(0xffffffffu, row, 1);
+                    const bool head = row >= 0 && (lane == 0 || rprev != row);
+                    const uint32_t heads = __ballot_sync(0xffffffffu, head);
+                    const int b = i & 1;
+                    if (head) {
+                        const int q = __popc(heads & ((1u << lane) - 1u));
+                        s_segr[(b * 4 + wl) * SG + q] = row;
+#pragma unroll
+                        for (int t = 0; t < kChunk; ++t)
+                            if (t < Tc) s_segv[((b * 4 + wl) * SG + q) * Tc + t] = v[t];
+                    }
+                    if (lane == 0) s_segn[b * 4 + wl] = __popc(heads);
+                    umma::bar_sync(2, 128);  // the stage is read and the row sums posted
+                    if (tid == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[s])) : "memory");
+                    // fold the warps' row sums into the slice's rows, warps in order
+                    if (tid < nrows) {
+                        const int rr = row_base + tid;
+                        for (int w2 = 0; w2 < 4; ++w2)
+                            for (int q = 0; q < s_segn[b * 4 + w2]; ++q)
+                                if (s_segr[(b * 4 + w2) * SG + q] == rr)
+                                    for (int t = 0; t < Tc; ++t)
+                                        s_racc[tid * Tc + t] += s_segv[((b * 4 + w2) * SG + q) * Tc + t];
+                    }
+                } else {
+                    const Unit x = decode(r, unit);
+                    if (x.kind == 2 || x.kind == 3) {
+                        const uint8_t *blob = s_blob[x.u];
+                        const bool has = blob != nullptr;
+                        const bool tma_sc = x.kind == 2 ? p.sf_tma_gu : p.sf_tma_dn;
+                        const uint32_t col = tbase + lb + sf0 + (uint32_t)(s * kLSfc);
+                        const int K = x.kind == 2 ? d : ff, M = x.kind == 2 ? ff : d;
+                        const int nbox = x.kind == 2 ? 2 : x.nt;
+                        // A scales: box m holds matrix m (gate/up) or K-tile kt + m (down)
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) {
+                            if (m < nbox) {
+                                const int ktm = x.kind == 2 ? x.kt : x.kt + m;
+                                uint32_t w[8];
+                                if (tma_sc) {
+                                    const uint8_t *sfa = st + lk_sfa_off(N) + (x.kind == 2 ? m * 2048 : 0) + (ktm & 1) * 8;
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        const uint2 v = has ? *reinterpret_cast<const uint2 *>(sfa + (32 * j + lane) * 16)
+                                                            : make_uint2(0u, 0u);
+                                        nanb |= e8m0_nan8(v.x, v.y);
+                                        w[j] = v.x;
+                                        w[4 + j] = v.y;
+                                    }
+                                } else {
+                                    const uint8_t *plane = nullptr;
+                                    if (has)
+                                        plane = x.kind == 2 ? (m == 0 ? blob + mat / 2 : blob + mat + mat / 32)
+                                                            : blob + mat + mat / 16 + mat / 2;
+                                    const int nks = min(4, (K - ktm * kTileK) / 64);
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        const int row = x.rb * kTileM + 32 * j + lane;
+                                        uint2 v = make_uint2(0u, 0u);
+                                        if (plane != nullptr && row < M) v = load_sf8(plane + (size_t)row * (K / 32) + ktm * 8, nks);
+                                        nanb |= e8m0_nan8(v.x, v.y);
+                                        w[j] = v.x;
+                                        w[4 + j] = v.y;
+                                    }
+                                }
+                                umma::st8(col + 8 * m, w);
+                            }
+                        }
+                        // B scales: tile tt at column 16 + 8 tt (rows 0-31, 32-63 per group)
+                        const int nbt = x.kind == 2 ? 1 : x.nt;
+#pragma unroll
+                        for (int tt = 0; tt < 2; ++tt) {
+                            if (tt < nbt) {
+                                uint32_t b0, b1, b2, b3;
+                                if (tma_sc) {
+                                    const uint32_t *sb = reinterpret_cast<const uint32_t *>(st + lk_sfb_off(N) + tt * 2 * kSfRow * 4);
+                                    b0 = sb[lane]; b1 = sb[32 + lane]; b2 = sb[kSfRow + lane]; b3 = sb[kSfRow + 32 + lane];
+                                } else {
+                                    // written by other CTAs: acquire their counter once
+                                    const int ai = x.kind == 2 ? 0 : 1;
+                                    if (!act_ok[ai]) {
+                                        const uint32_t *ctr = ai == 0 ? &hdr->prep_done : &hdr->gu_done;
+                                        const uint32_t want = ai == 0 ? (uint32_t)G : (uint32_t)(nrbs + U * nrb_ff);
+                                        const uint64_t t0 = globaltimer();
+                                        while (ld_acquire(ctr) < want && globaltimer() - t0 <= rp.wait_ns) {
+                                        }
+                                        act_ok[ai] = true;
+                                    }
+                                    const uint32_t *sb = x.kind == 2
+                                        ? reinterpret_cast<const uint32_t *>(rp.ws + L.xsf) + (size_t)x.kt * 2 * kSfRow
+                                        : reinterpret_cast<const uint32_t *>(rp.ws + L.hsf) +
+                                              ((size_t)x.u * nkt_ff + x.kt + tt) * 2 * kSfRow;
+                                    b0 = __ldcg(sb + lane); b1 = __ldcg(sb + 32 + lane);
+                                    b2 = __ldcg(sb + kSfRow + lane); b3 = __ldcg(sb + kSfRow + 32 + lane);
+                                }
+                                if (!has) b0 = b1 = b2 = b3 = 0u;
+                                const uint32_t w[8] = {b0, b1, 0u, 0u, b2, b3, 0u, 0u};
+                                umma::st8(col + 16 + 8 * tt, w);
+                            }
+                        }
+                        umma::wait_st();
+                    }
+                    umma::fence_before();
+                }
+                __syncwarp();
+                if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sfr[s])) : "memory");
+            }
+            if (r == 0) {
+                // the slice's rows: finished here, or (cut by a CTA boundary)
+                // parked for the last of their CTAs, which sums the parts in
+                // CTA order; each finished row counts on router_done
+                umma::bar_sync(2, 128);
+                if (go && tid < nrows) {
+                    const int rr = row_base + tid;
+                    const long long rs = (long long)rr * d, re = rs + d;  // its floats
+                    float *logits = reinterpret_cast<float *>(rp.ws + L.logits);
+                    const float bias = (rp.bias && !(rp.route_flags & kRouteBiasSelect)) ? rp.bias[rr] : 0.f;
+                    bool done = false;
+                    float out[kChunk];
+                    if (rs >= f_lo && re <= f_hi) {
+#pragma unroll
+                        for (int t = 0; t < kChunk; ++t) out[t] = t < Tc ? s_racc[tid * Tc + t] : 0.f;
+                        done = true;
+                    } else {
+                        const int first = owner(R0, (int)(rs / kLRUnit));
+                        const int nseg = owner(R0, (int)((re - 1) / kLRUnit)) - first + 1;
+                        float *pp = reinterpret_cast<float *>(rp.ws + L.part) + ((size_t)rr * kMaxSeg) * kChunk;
+                        uint32_t *pc = reinterpret_cast<uint32_t *>(rp.ws + L.cnt) + rr;
+#pragma unroll
+                        for (int t = 0; t < kChunk; ++t) pp[(cta - first) * kChunk + t] = t < Tc ? s_racc[tid * Tc + t] : 0.f;
+                        const uint32_t old = atom_add_acq_rel(pc, 1u);
+                        if (old == (uint32_t)(nseg - 1)) {
+#pragma unroll
+                            for (int t = 0; t < kChunk; ++t) out[t] = 0.f;
+                            for (int sl = 0; sl < nseg; ++sl)
+#pragma unroll
+                                for (int t = 0; t < kChunk; ++t) out[t] += __ldcg(pp + sl * kChunk + t);
+                            *pc = 0u;
+                            done = true;
+                        }
+                    }
+                    if (done) {
+                        for (int t = 0; t < Tc; ++t) logits[(size_t)t * E + rr] = out[t] + bias;
+                        red_add_release(&hdr->router_done, 1u);  // after this thread's logit stores
+                    }
+                }
+            }
+        }
+        if (p.strict && __any_sync(0xffffffffu, nanb != 0u) && lane == 0) set_status(hdr, kStDeviceCheck);
+    } else if (warp == 9) {
+        // ====================================================== MMA issue --
+        if (lane == 0) {
+            const uint64_t adesc0 = umma::smem_desc(smem_u32(smem), 16u, 1024u, umma::kLayoutSw128);
+            const uint64_t bdesc0 = umma::smem_desc(smem_u32(smem) + lk_b_off(), (uint32_t)((N / 8) * 128), 128u,
+                                                    umma::kLayoutNone);
+            const uint32_t bstep = (uint32_t)(2 * (N / 8) * 128) >> 4;  // one k-step of B (2 chunks)
+            const uint32_t btile = (uint32_t)(N * 128) >> 4;            // B tile 1 after tile 0
+            const uint32_t idesc4 = umma::idesc_mxf4(N), idesc16 = umma::idesc_bf16(N);
+            const uint32_t id4[2] = {umma::idesc_sf_id(idesc4, 0u), umma::idesc_sf_id(idesc4, 2u)};
+            int i = 0, seg = 0;
+            for (int r = 0; r < 4 && !*s_abort; ++r) {
+                if (r == 2 && !routed_ranges(false)) break;
+                const Range R = rg[r];
+                if (r == 0) {
+                    i += R.b - R.a;  // router units are consumed by the scale warps
+                    continue;
+                }
+                for (int unit = R.a; unit < R.b && !*s_abort; ++seg) {
+                    Unit x = decode(r, unit);
+                    const int seg_end = min(R.b, x.iend);
+                    const int buf = seg & 1;
+                    if (seg >= 2 && !wait(&aempty[buf], (uint32_t)(((seg >> 1) + 1) & 1))) break;
+                    umma::fence_after();
+                    const uint32_t dcol = tbase + (uint32_t)(buf * 128);
+                    uint32_t acc = 0u;
+                    for (int un = unit; un < seg_end; ++un, ++i) {
+                        if (un != unit) x = decode(r, un);
+                        const int s = i % nst;
+                        const uint32_t ph = (uint32_t)((i / nst) & 1);
+                        if (!wait(&full[s], ph) || !wait(&sfr[s], ph)) break;
+                        umma::fence_after();
+                        const uint32_t soff = (uint32_t)(s * SB) >> 4;
+                        const uint64_t a0 = adesc0 + soff, b0 = bdesc0 + soff;
+                        const uint32_t sfc = tbase + sf0 + (uint32_t)(s * kLSfc);
+                        if (x.kind == 1) {
+                            // shared gate/up: bf16, W_g -> acc 0, W_u -> acc 1
+                            const int nks = min(4, (d - x.kt * kTileKs) / 16);
+#pragma unroll
+                            for (int sk = 0; sk < 4; ++sk) {
+                                if (sk < nks) {
+                                    const uint64_t bd = b0 + sk * bstep;
+                                    umma::mma_bf16(dcol, a0 + 2 * sk, bd, idesc16, acc);
+                                    umma::mma_bf16(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, idesc16, acc);
+                                    acc = 1u;
+                                }
+                            }
+                        } else if (x.kind == 2) {
+                            const int nks = min(4, (d - x.kt * kTileK) / 64);
+#pragma unroll
+                            for (int sk = 0; sk < 4; ++sk) {
+                                if (sk < nks) {
+                                    const uint64_t bd = b0 + sk * bstep;
+                                    const uint32_t sfid = (uint32_t)(2 * (sk & 1)) << 30;
+                                    const uint32_t sfb = (sfc + 16 + (sk >> 1) * 4) | sfid;
+                                    umma::mma_mxf4(dcol, a0 + 2 * sk, bd, id4[sk & 1], acc, (sfc + (sk >> 1) * 4) | sfid, sfb);
+                                    umma::mma_mxf4(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, id4[sk & 1], acc,
+                                                   (sfc + 8 + (sk >> 1) * 4) | sfid, sfb);
+                                    acc = 1u;
+                                }
+                            }
+                        } else {
+                            // down: K-tiles kt, kt + 1 (A box tt, B tile tt) into acc 0
+                            for (int tt = 0; tt < x.nt; ++tt) {
+                                const uint64_t at = a0 + (uint32_t)(tt * (kAtile >> 4));
+                                const uint64_t bt = b0 + tt * btile;
+                                if (x.kind == 3) {
+                                    const int nks = min(4, (ff - (x.kt + tt) * kTileK) / 64);
+#pragma unroll
+                                    for (int sk = 0; sk < 4; ++sk) {
+                                        if (sk < nks) {
+                                            const uint32_t sfid = (uint32_t)(2 * (sk & 1)) << 30;
+                                            umma::mma_mxf4(dcol, at + 2 * sk, bt + sk * bstep, id4[sk & 1], acc,
+                                                           (sfc + 8 * tt + (sk >> 1) * 4) | sfid,
+                                                           (sfc + 16 + 8 * tt + (sk >> 1) * 4) | sfid);
+                                            acc = 1u;
+                                        }
+                                    }
+                                } else {
+                                    const int nks = min(4, (ffs - (x.kt + tt) * kTileKs) / 16);
+#pragma unroll
+                                    for (int sk = 0; sk < 4; ++sk) {
+                                        if (sk < nks) {
+                                            umma::mma_bf16(dcol, at + 2 * sk, bt + sk * bstep, idesc16, acc);
+                                            acc = 1u;
+                                        }
+                                    }
+                                }
+                            }
+                        }
+                        umma::commit(&empty[s]);
+                    }
+                    umma::commit(&afull[buf]);
+                    unit = seg_end;
+                }
+            }
+            // the CTA frees its tensor memory only after every MMA issued here
+            // has completed (on an early exit too)
+            umma::commit(mdone);
+            mbar_drain(mdone, 0u, rp.wait_ns);
+        }
+    }
+
+    if (warp < 4) {
+        // ======================================================= epilogue --
+        const uint32_t lb = umma::lane_base(warp);
+        const int rowl = 32 * warp + lane;  // row of the 128-row item
+        float *spart = reinterpret_cast<float *>(rp.ws + L.spart);
+        int seg = 0;
+        for (int r = 1; r < 4; ++r) {
+            // the four warps agree on going on (they share named barrier 1)
+            if (r == 2 && !umma::bar_red_and(1, 128, routed_ranges(true))) break;
+            const Range R = rg[r];
+            uint32_t *icnt = reinterpret_cast<uint32_t *>(rp.ws + L.icnt) +
+                             (r == 1 ? L.umax * nrb_ff : (r == 2 ? 0 : L.umax * nrb_ff + nrbs));
+            const int NM = r == 3 ? 1 : 2;
+            for (int unit = R.a; unit < R.b; ++seg) {
+                const Unit x = decode(r, unit);
+                const int item = x.item;
+                const int seg_end = min(R.b, x.iend);
+                const int buf = seg & 1;
+                float acc[2][kChunk];
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+#pragma unroll
+                    for (int t = 0; t < kChunk; ++t) acc[m][t] = 0.f;
+                // every epilogue warp runs the same sequence of named barriers,
+                // so after a failed wait it carries on (with unused values)
+                if (lane == 0) wait(&afull[buf], (uint32_t)((seg >> 1) & 1));
+                __syncwarp();
+                umma::fence_after();
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    if (m < NM) {
+#pragma unroll
+                        for (int n0 = 0; n0 < kNMax; n0 += 8) {
+                            if (n0 < N) {
+                                uint32_t v[8];
+                                umma::ld8(tbase + lb + (uint32_t)((buf * 2 + m) * 64 + n0), v);
+                                umma::wait_ld();
+#pragma unroll
+                                for (int jj = 0; jj < 8; ++jj) {
+                                    const int t = (n0 + jj) / kPieces;
+                                    if (t < kChunk) acc[m][t] += __uint_as_float(v[jj]);
+                                }
+                            }
+                        }
+                    }
+                }
+                umma::fence_before();
+                __syncwarp();
+                if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&aempty[buf])) : "memory");
+
+                const bool whole = unit == x.istart && seg_end == x.iend;
+                bool fin = whole;
+                if (!whole) {
+                    const int slot = 2 * (r - 1) + (unit == R.a ? 0 : 1);
+                    float *sp = spart + (size_t)((cta * 6 + slot) * 2) * kChunk * kTileM;
+#pragma unroll
+                    for (int m = 0; m < 2; ++m)
+#pragma unroll
+                        for (int t = 0; t < kChunk; ++t)
+                            if (m < NM && t < Tc) sp[(m * kChunk + t) * kTileM + rowl] = acc[m][t];
+                    umma::bar_sync(1, 128);
+                    const int c0 = owner(R, x.istart), c1 = owner(R, x.iend - 1);
+                    if (threadIdx.x == 0) {
+                        const uint32_t old = atom_add_acq_rel(icnt + item, 1u);
+                        const int last = old == (uint32_t)(c1 - c0);
+                        if (last) icnt[item] = 0u;
+                        *s_last = last;
+                    }
+                    umma::bar_sync(1, 128);
+                    fin = *s_last != 0;
+                    if (fin) {
+                        // sum every part of the item in K order
+#pragma unroll
+                        for (int m = 0; m < 2; ++m)
+#pragma unroll
+                            for (int t = 0; t < kChunk; ++t) acc[m][t] = 0.f;
+                        for (int cc = c0; cc <= c1; ++cc) {
+                            const int sl = 2 * (r - 1) + (start_of(R, cc) < x.istart ? 1 : 0);
+                            const float *q = spart + (size_t)((cc * 6 + sl) * 2) * kChunk * kTileM;
+#pragma unroll
+                            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                                for (int t = 0; t < kChunk; ++t)
+                                    if (m < NM && t < Tc) acc[m][t] += __ldcg(q + (m * kChunk + t) * kTileM + rowl);
+                        }
+                    }
+                }
+                if (fin) {
+                    if (r == 2) {
+                        const int f = x.rb * kTileM + rowl;  // ff row of this thread
+                        const uint8_t *blob = s_blob[x.u];
+                        const int blk = x.rb * 4 + warp;  // 32-row block of ff
+                        const int kt = blk >> 3;
+                        uint8_t *tile = rp.ws + L.hb + ((size_t)x.u * nkt_ff + kt) * N * 128;
+                        uint8_t *sfw = rp.ws + L.hsf + ((size_t)x.u * nkt_ff + kt) * 2 * kSfRow * 4;
+#pragma unroll
+                        for (int t = 0; t < kChunk; ++t) {
+                            if (t < Tc) {
+                                float h = 0.f;
+                                const float w = s_wu[x.u * Tc + t];
+                                if (blob != nullptr && w != 0.f && f < ff) h = silu_mul(acc[0][t], acc[1][t]) * w;
+                                quantize_pieces(h, lane, t, blk & 7, N, tile, sfw);
+                            }
+                        }
+                    } else if (r == 1) {
+                        const int f = x.rb * kTileM + rowl;  // ff_s row of this thread
+                        if (f < ffs) {
+                            // h as bf16 hi + lo (pieces 0, 1; the others zero), weight 1
+                            uint8_t *tile = rp.ws + L.hsb + (size_t)(f / kTileKs) * N * 128;
+                            const int c = (f % kTileKs) / 8, e = f % 8;
+#pragma unroll
+                            for (int t = 0; t < kChunk; ++t) {
+                                if (t < Tc) {
+                                    const float h = silu_mul(acc[0][t], acc[1][t]);
+                                    const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+                                    const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
+#pragma unroll
+                                    for (int pc = 0; pc < kPieces; ++pc) {
+                                        const int n = t * kPieces + pc;
+                                        const __nv_bfloat16 v = pc == 0 ? hi : (pc == 1 ? lo : __float2bfloat16_rn(0.f));
+                                        *reinterpret_cast<__nv_bfloat16 *>(tile + (c * (N / 8) + n / 8) * 128 +
+                                                                           (n % 8) * 16 + e * 2) = v;
+                                    }
+                                }
+                            }
+                        }
+                    } else {
+                        const int row = item * kTileM + rowl;
+                        if (row < d) {
+#pragma unroll
+                            for (int t = 0; t < kChunk; ++t) {
+                                if (t < Tc) {
+                                    const float yv = acc[0][t];
+                                    if (p.out_fp32)
+                                        reinterpret_cast<float *>(p.y)[(size_t)t * d + row] = yv;
+                                    else
+                                        reinterpret_cast<__nv_bfloat16 *>(p.y)[(size_t)t * d + row] = __float2bfloat16_rn(yv);
+                                }
+                            }
+                        }
+                    }
+                    if (r != 3) {
+                        // this gate/up item's activations are written: count it
+                        // for the down units' copies
+                        umma::bar_sync(1, 128);
+                        if (threadIdx.x == 0) red_add_release(&hdr->gu_done, 1u);
+                    }
+                }
+                unit = seg_end;
+            }
+        }
+    }
+
+    umma::fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        umma::fence_after();
+        umma::tmem_dealloc(tbase, kCols);
+    }
+    if (threadIdx.x == 0) {
+        // the last CTA out returns the header's counters to zero for the next call
+        const uint32_t old = atom_add_acq_rel(&hdr->exit_cnt, 1u);
+        if (old == (uint32_t)(G - 1)) {
+            hdr->router_done = 0u;
+            hdr->prep_done = 0u;
+            hdr->gu_done = 0u;
+            hdr->exit_cnt = 0u;
+        }
+    }
+}
+
+}  // namespace k3

@@ -156,7 +156,8 @@ __global__ void __launch_bounds__(kRouteThreads) pf_topk_kernel(const __grid_con
     cta_topk_row(reinterpret_cast<const float *>(ws + p.P.lg) + (size_t)t * E, E, k,
                  reinterpret_cast<int32_t *>(ws + p.P.idx) + (size_t)t * k,
                  reinterpret_cast<float *>(ws + p.P.wt) + (size_t)t * k,
-                 p.r.idx_out ? p.r.idx_out + (size_t)t * k : nullptr, p.r.w_out ? p.r.w_out + (size_t)t * k : nullptr);
+                 p.r.idx_out ? p.r.idx_out + (size_t)t * k : nullptr, p.r.w_out ? p.r.w_out + (size_t)t * k : nullptr,
+                 (p.r.route_flags & kRouteBiasSelect) ? p.r.bias : nullptr, (p.r.route_flags & kRouteRenorm) != 0);
 }
 
 // --------------------------------------------------------------- dispatch --

@@ -37,6 +37,8 @@ struct PfUmmaParams {
     int nst, sb;       // pipeline stages and bytes per stage
     int sf_tma;        // weight scales by TMA (reduction length a multiple of 512)
     const uint8_t *const *blobs;  // device array [E] (weight-scale loads without TMA)
+    uint64_t wait_ns;  // bound of every device wait
+    int strict;        // flag E8M0 NaN bytes (0xFF) among the weight scales read
 };
 
 struct PfSlot {
@@ -80,7 +82,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
     uint64_t *aempty = afull + 2;
     uint64_t *mfull = aempty + 2;
     uint64_t *mempty = mfull + kPfSlots;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(mempty + kPfSlots);
+    uint64_t *mdone = mempty + kPfSlots;  // every MMA this CTA issued has completed
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(mdone + 1);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tslot + 1);
     PfSlot *slots = reinterpret_cast<PfSlot *>(smem + nst * SB + 512);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -100,6 +103,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
             mbar_init(&mfull[s], 1);
             mbar_init(&mempty[s], 9);  // copies warp, 4 scale warps, 4 epilogue warps
         }
+        mbar_init(mdone, 1);
         fence_mbar_init();
         *s_abort = 0;
     }
@@ -133,7 +137,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
     auto nk_of = [&](int it) { return it < IR ? nkt : nkts; };
     auto wait = [&](uint64_t *bar, uint32_t parity) {
         if (*s_abort) return false;
-        if (mbar_wait_bounded(bar, parity, hdr)) return true;
+        if (mbar_wait_bounded(bar, parity, hdr, p.wait_ns)) return true;
         *s_abort = 1;
         return false;
     };
@@ -272,8 +276,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
             slot_done(q);
         }
         if (*s_abort && lane == 0) {
-            const uint64_t t0 = globaltimer();
-            while (globaltimer() - t0 < 200000ull) {
+            // wait (bounded) for the last copy issued into each stage, so none
+            // lands after the CTA's shared memory is released
+            for (int q = 0; q < nst && q < it_stage; ++q) {
+                const int last = q + ((it_stage - 1 - q) / nst) * nst;
+                mbar_drain(&full[q], (uint32_t)((last / nst) & 1), p.wait_ns);
             }
         }
     } else if (warp >= 4 && warp < 8) {
@@ -281,6 +288,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
         const uint32_t lb = umma::lane_base(warp);
         int s = 0;
         uint32_t ph = 0u;
+        uint32_t nanb = 0u;  // E8M0 NaN bytes met among the weight scales (strict mode)
         for (int q = 0; q < nmine; ++q) {
             const PfSlot *sl = slot_wait(q);
             if (!sl) break;
@@ -310,6 +318,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
                             for (int j = 0; j < 4; ++j) {
                                 const uint2 v = ok ? *reinterpret_cast<const uint2 *>(sfa + (32 * j + lane) * 16)
                                                    : make_uint2(0u, 0u);
+                                nanb |= e8m0_nan8(v.x, v.y);
                                 w[j] = v.x;
                                 w[4 + j] = v.y;
                             }
@@ -324,6 +333,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
                                 const int row = rb * kTileM + 32 * j + lane;
                                 uint2 v = make_uint2(0u, 0u);
                                 if (plane != nullptr && row < M) v = load_sf8(plane + (size_t)row * (K / 32) + kt * 8, nks);
+                                nanb |= e8m0_nan8(v.x, v.y);
                                 w[j] = v.x;
                                 w[4 + j] = v.y;
                             }
@@ -348,6 +358,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
             slot_done(q);
             if (!go) break;
         }
+        if (p.strict && __any_sync(0xffffffffu, nanb != 0u) && lane == 0) set_status(hdr, kStDeviceCheck);
     } else if (warp == 9) {
         // ------------------------------------------------- MMA issuer --
         if (lane == 0) {
@@ -417,6 +428,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_expert_kernel(const __grid_c
                 umma::commit(&afull[buf]);
                 if (!go) break;
             }
+            // the CTA frees its tensor memory only after every MMA issued here
+            // has completed (on an early exit too)
+            umma::commit(mdone);
+            mbar_drain(mdone, 0u, p.wait_ns);
         }
     } else {
         // --------------------------------------------------- epilogue --

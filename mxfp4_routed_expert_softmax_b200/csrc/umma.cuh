@@ -157,6 +157,18 @@ __device__ __forceinline__ void tmap_acquire(const void *gmap) {
 __device__ __forceinline__ void bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Named barrier that also ANDs a predicate over its `count` threads: every
+// thread gets true only if every thread passed true.
+__device__ __forceinline__ bool bar_red_and(int id, int count, bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n"
+        " selp.u32 %0, 1, 0, q;\n}"
+        : "=r"(out)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return out != 0u;
+}
 
 }  // namespace umma
 }  // namespace k3

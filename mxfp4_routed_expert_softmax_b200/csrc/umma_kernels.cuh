@@ -209,6 +209,9 @@ struct UmmaParams {
     // gate/up: router-kernel CTAs that announce their x pieces and tensor maps
     // in the header's prep_done (0: nothing to wait for)
     int route_ctas;
+    uint64_t wait_ns;  // bound of every device wait
+    int strict;        // flag E8M0 NaN bytes (0xFF) among the weight scales read
+    int inject;        // failure-path tests: 1 = never signal "routing loaded"
 };
 
 // One pipeline stage for MMA width N: the A boxes (16 KB per matrix, first,
@@ -230,8 +233,9 @@ __host__ __device__ inline int umma_sf_cols(bool gu) { return gu ? 32 : 16; }
 // saturates HBM wait thousands of cycles, so the pipeline never makes them.
 constexpr int kMetaU = kChunk * 32;  // distinct experts of a chunk (top_k <= 32)
 constexpr int kMetaBytes = kMetaU * 8 + kMetaU * 4 + kMetaU * kChunk * 4;
+constexpr int kUBarBytes = 512;  // mbarriers, the TMEM address and flags after the stages
 __host__ __device__ inline int umma_smem_bytes(bool gu, int N, int nst) {
-    return 1024 + nst * umma_stage_bytes(gu, N) + 256 + kMetaBytes;
+    return 1024 + nst * umma_stage_bytes(gu, N) + kUBarBytes + kMetaBytes;
 }
 
 // Load the (up to) 8 scale bytes of one weight row for one K-tile: nks valid
@@ -267,11 +271,12 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     uint64_t *afull = empty + nst;
     uint64_t *aempty = afull + 2;
     uint64_t *mready = aempty + 2;  // the routing is in shared memory (gate/up)
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(mready + 1);
+    uint64_t *mdone = mready + 1;   // every MMA this CTA issued has completed
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(mdone + 1);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tslot + 1);
     volatile int *s_last = s_abort + 1;
     volatile int *s_U = s_last + 1;
-    const uint8_t **s_blob = reinterpret_cast<const uint8_t **>(smem + nst * SB + 256);
+    const uint8_t **s_blob = reinterpret_cast<const uint8_t **>(smem + nst * SB + kUBarBytes);
     int32_t *s_eid = reinterpret_cast<int32_t *>(s_blob + kMetaU);
     float *s_wu = reinterpret_cast<float *>(s_eid + kMetaU);  // [u][t]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -288,6 +293,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             mbar_init(&aempty[b], 4);
         }
         mbar_init(mready, 1);
+        mbar_init(mdone, 1);
         fence_mbar_init();
         *s_abort = 0;
     }
@@ -334,7 +340,8 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             const int U0 = load_meta(lane, 32);
             if (lane == 0) *s_U = U0;
             __syncwarp();
-            if (lane == 0) asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(mready)) : "memory");
+            if (lane == 0 && p.inject != 1)
+                asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(mready)) : "memory");
         }
     }
     const int K = GU ? p.d : p.ff;   // routed reduction length
@@ -377,7 +384,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     auto routed_range = [&](bool warp_wide) {
         int ok = 1;
         if (lane == 0) {
-            ok = (!*s_abort && mbar_wait_bounded(mready, 0u, hdr)) ? 1 : 0;
+            ok = (!*s_abort && mbar_wait_bounded(mready, 0u, hdr, p.wait_ns)) ? 1 : 0;
             if (!ok) *s_abort = 1;
         }
         if (warp_wide) ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -399,7 +406,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     // failure ends the kernel in bounded time.
     auto wait = [&](uint64_t *bar, uint32_t parity) {
         if (*s_abort) return false;
-        if (mbar_wait_bounded(bar, parity, hdr)) return true;
+        if (mbar_wait_bounded(bar, parity, hdr, p.wait_ns)) return true;
         *s_abort = 1;
         return false;
     };
@@ -482,7 +489,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 const uint64_t t0 = globaltimer();
                 while (ld_acquire(&hdr->prep_done) < (uint32_t)p.route_ctas) {
                     __nanosleep(32);
-                    if (globaltimer() - t0 > kWaitLimitNs) {
+                    if (globaltimer() - t0 > p.wait_ns) {
                         set_status(hdr, kStTimeout);
                         *s_abort = 1;
                         break;
@@ -547,16 +554,19 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             }
             }
             if (*s_abort) {
-                // a wait gave up somewhere: let the copies this thread issued
-                // land (bounded) before the CTA's shared memory goes away
-                const uint64_t t0 = globaltimer();
-                while (globaltimer() - t0 < 200000ull) {
+                // a wait gave up somewhere: wait (bounded) for the last copy
+                // issued into each stage, so none lands after the CTA's
+                // shared memory is released
+                for (int q = 0; q < nst && q < it; ++q) {
+                    const int last = q + ((it - 1 - q) / nst) * nst;  // its last use
+                    mbar_drain(&full[q], (uint32_t)((last / nst) & 1), p.wait_ns);
                 }
             }
         }
     } else if (warp >= 4 && warp < 8) {
         // --------------------------------------- scale factors -> TMEM --
         const uint32_t lb = umma::lane_base(warp);
+        uint32_t nanb = 0u;  // E8M0 NaN bytes met among the weight scales (strict mode)
         if (p.sf_tma) {
             // The scales came with the stage's TMA copy: wait for the stage,
             // then move this K-tile's 8 scale bytes of each row (and the B
@@ -588,6 +598,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                         for (int j = 0; j < 4; ++j) {
                             const uint2 v = has ? *reinterpret_cast<const uint2 *>(sfa + (32 * j + lane) * 16)
                                                 : make_uint2(0u, 0u);
+                            nanb |= e8m0_nan8(v.x, v.y);
                             w[j] = v.x;      // group 0: k-steps 0, 1
                             w[4 + j] = v.y;  // group 1: k-steps 2, 3
                         }
@@ -636,6 +647,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     const int row = x.rb * kTileM + 32 * j + lane;
                     uint2 v = make_uint2(0u, 0u);
                     if (plane != nullptr && row < M) v = load_sf8(plane + (size_t)row * (K / 32) + x.kt * 8, nks);
+                    nanb |= e8m0_nan8(v.x, v.y);
                     r.a[m][j] = v.x;      // group 0: k-steps 0, 1
                     r.a[m][4 + j] = v.y;  // group 1: k-steps 2, 3
                 }
@@ -690,6 +702,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             done += n;
         }
         }
+        if (p.strict && __any_sync(0xffffffffu, nanb != 0u) && lane == 0) set_status(hdr, kStDeviceCheck);
     } else if (warp == 9) {
         // ------------------------------------------------- MMA issuer --
         // One thread; everything per MMA is an add on precomputed descriptors
@@ -757,6 +770,10 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 unit = seg_end;
             }
             }
+            // the CTA frees its tensor memory only after every MMA issued here
+            // has completed (on an early exit too)
+            umma::commit(mdone);
+            mbar_drain(mdone, 0u, p.wait_ns);
         }
     } else if (warp < 4) {
         // --------------------------------------------------- epilogue --

@@ -62,6 +62,8 @@ def load(path: str | None = None):
     lib.oracle_softmax.argtypes = [vp, i64, vp]
     lib.oracle_topk.argtypes = [vp, i64, i64, vp]
     lib.oracle_route.argtypes = [vp, i64, vp, vp, i64, i64, i64, vp, vp, vp, vp]
+    lib.oracle_route_variant.argtypes = [vp, i64, vp, vp, i64, i64, i64, ctypes.c_int, ctypes.c_int,
+                                         vp, vp, vp, vp]
     lib.oracle_expert_ffn_vec.argtypes = [vp, vp, i64, i64, vp]
     lib.oracle_expert_ffn.argtypes = [vp, i64, vp, i64, i64, vp]
     lib.oracle_shared_ffn.argtypes = [vp, i64, vp, vp, vp, i64, i64, vp]
@@ -69,7 +71,8 @@ def load(path: str | None = None):
     lib.oracle_layer.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64,
                                  vp, vp, vp]
     for name in ("oracle_mxfp4_matvec", "oracle_bf16_matvec", "oracle_router_logits",
-                 "oracle_softmax", "oracle_topk", "oracle_route", "oracle_expert_ffn_vec",
+                 "oracle_softmax", "oracle_topk", "oracle_route", "oracle_route_variant",
+                 "oracle_expert_ffn_vec",
                  "oracle_expert_ffn", "oracle_shared_ffn", "oracle_combine", "oracle_layer"):
         getattr(lib, name).restype = None
     if path is None:
@@ -167,6 +170,25 @@ class Oracle:
         weight = np.empty((T, k), dtype=np.float64)
         self.lib.oracle_route(_p(x), T, _p(w), _p(b), d, E, k, _p(logits), _p(probs), _p(idx),
                               _p(weight))
+        return logits, probs, idx, weight
+
+    def route_variant(self, x, w, bias, k, renorm=False, bias_select_only=False):
+        """route() with the routing variants: the bias moving only the
+        selection, and/or the k weights renormalised over the picks.
+        -> (logits [T,E] f64 (unbiased when bias_select_only), probs [T,E],
+            idx [T,k] i32, weight [T,k] f64)"""
+        x = _bf(x)
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+        T, d = x.shape
+        E = w.shape[0]
+        logits = np.empty((T, E), dtype=np.float64)
+        probs = np.empty((T, E), dtype=np.float64)
+        idx = np.empty((T, k), dtype=np.int32)
+        weight = np.empty((T, k), dtype=np.float64)
+        self.lib.oracle_route_variant(_p(x), T, _p(w), _p(b), d, E, k, int(bool(renorm)),
+                                      int(bool(bias_select_only)), _p(logits), _p(probs), _p(idx),
+                                      _p(weight))
         return logits, probs, idx, weight
 
     def expert_ffn(self, x, blob, d, ff) -> np.ndarray:

@@ -171,6 +171,43 @@ void oracle_route(const uint16_t *x, int64_t T, const float *w, const float *bia
     free(l);
 }
 
+/*
+ * Two routing variants the pages leave open (their routing formula uses the
+ * raw softmax probability of each pick and adds no bias), written out for
+ * parity with the library's flags:
+ *   bias_select_only: the bias moves only the selection -- the top-k is taken
+ *     on s_e = l_e + b_e, while p is the softmax of the unbiased l;
+ *   renorm: the k weights are rescaled to sum to one over the picks,
+ *     w_j = p_idx_j / sum_j' p_idx_j' (the sum in pick order).
+ * With both off this is oracle_route.  logits_out receives l (unbiased when
+ * bias_select_only, else l + b); probs_out the softmax p.
+ */
+void oracle_route_variant(const uint16_t *x, int64_t T, const float *w, const float *bias,
+                          int64_t d, int64_t E, int64_t k, int renorm, int bias_select_only,
+                          double *logits_out, double *probs_out, int32_t *idx, double *weight) {
+    double *l = (double *)malloc((size_t)(T * E) * sizeof(double));
+    double *sel = (double *)malloc((size_t)E * sizeof(double));
+    double *p = (double *)malloc((size_t)E * sizeof(double));
+    oracle_router_logits(x, T, w, bias_select_only ? NULL : bias, d, E, l);
+    for (int64_t t = 0; t < T; ++t) {
+        const double *lt = l + t * E;
+        for (int64_t e = 0; e < E; ++e) sel[e] = lt[e] + ((bias_select_only && bias) ? (double)bias[e] : 0.0);
+        oracle_softmax(lt, E, p);
+        oracle_topk(sel, E, k, idx + t * k);
+        double z = 0.0;
+        for (int64_t j = 0; j < k; ++j) z += p[idx[t * k + j]];
+        for (int64_t j = 0; j < k; ++j) {
+            const double pj = p[idx[t * k + j]];
+            weight[t * k + j] = renorm ? pj / z : pj;
+        }
+        if (probs_out) memcpy(probs_out + t * E, p, (size_t)E * sizeof(double));
+    }
+    if (logits_out) memcpy(logits_out, l, (size_t)(T * E) * sizeof(double));
+    free(p);
+    free(sel);
+    free(l);
+}
+
 static double silu(double z) { return z / (1.0 + exp(-z)); }
 
 /* Byte offsets of the six planes of a routed expert's blob:

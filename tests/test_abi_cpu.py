@@ -81,7 +81,7 @@ A16 = 0x10000  # a fake 16-byte aligned address: never dereferenced, calls fail 
     ((7168, 1536, 896, 33, 1536, 0), 1),     # k > 32
     ((256, 128, 4, 5, 128, 0), 1),           # k > E
     ((7168, 1536, 896, 16, 100, 0), 2),      # shared width not a multiple of 64
-    ((7168, 1536, 896, 16, 1536, 8), 1),     # unknown flag
+    ((7168, 1536, 896, 16, 1536, 32), 1),    # unknown flag
     ((7168, 8192, 896, 16, 1536, 0), 2),     # down tile does not fit shared memory
 ])
 def test_layer_rejects_bad_dims(m, dims, want):
@@ -138,3 +138,20 @@ def test_product_path_has_no_oracle_reference():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.lower(), f
+
+
+@pytest.mark.parametrize("flag", ["K3MOE_STRICT", "K3MOE_RENORM_TOPK", "K3MOE_BIAS_SELECT_ONLY"])
+def test_option_flags_are_accepted(m, flag):
+    """The option flags pass validation (the call then fails only on the tiny
+    workspace size, before anything is launched)."""
+    d = m.make_dims(256, 128, 32, 4, 128, getattr(m, flag) | m.K3MOE_OUT_FP32)
+    st = m.lib.k3moe_layer(A16, 4, A16, None, A16, A16, A16, A16, ctypes.byref(d), A16, None, None,
+                           A16 * 16, 16, None)
+    assert st == m.K3MOE_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_fault_hook_validates_and_resets(m):
+    assert m.k3moe_debug_set_fault(2, 0) == m.K3MOE_ERR_INVALID_ARGUMENT
+    assert m.k3moe_debug_set_fault(-1, 0) == m.K3MOE_ERR_INVALID_ARGUMENT
+    assert m.k3moe_debug_set_fault(1, 1000000) == m.K3MOE_OK
+    assert m.k3moe_debug_set_fault(0, 0) == m.K3MOE_OK

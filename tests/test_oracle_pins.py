@@ -391,3 +391,84 @@ def test_torch_fp64_second_opinion_k3_route_and_one_expert(orc):
     h = torch.nn.functional.silu(Wg @ xt[0]) * (Wu @ xt[0])
     ot = (Wd @ h).numpy()
     assert np.allclose(o, ot, rtol=1e-12, atol=1e-12 * np.abs(ot).max())
+
+
+# ------------------------------------------------------ routing variants --
+# The pages' routing adds no bias and weights each pick by its raw softmax
+# probability; the library also offers a bias that moves only the selection
+# and weights renormalised over the k picks.  Pins: closed forms on a
+# hand-built router, and invariants on random ones.
+
+def _variant_case():
+    """x = (1, 0), W_r rows (e, 0): logits exactly (0, 1, 2, 3)."""
+    x = np.array([[k3gen.bf16_bits(1.0), 0]], dtype=np.uint16)
+    w = np.array([[0.0, 0.0], [1.0, 0.0], [2.0, 0.0], [3.0, 0.0]], dtype=np.float32)
+    b = np.array([10.0, 0.0, 0.0, -10.0], dtype=np.float32)
+    return x, w, b
+
+
+def test_route_variants_closed_forms(orc):
+    x, w, b = _variant_case()
+    e = math.e
+    # no bias: picks 3, 2; renormalised weights e^3, e^2 over their sum
+    _, _, idx, wt = orc.route_variant(x, w, None, 2, renorm=True)
+    assert idx[0].tolist() == [3, 2]
+    assert np.allclose(wt[0], [e ** 3 / (e ** 3 + e ** 2), e ** 2 / (e ** 3 + e ** 2)], rtol=1e-15, atol=0)
+    # bias in the logits (the library's default): s = (10, 1, 2, -7), picks 0, 2
+    zs = e ** 10 + e + e ** 2 + e ** -7
+    _, _, idx, wt = orc.route_variant(x, w, b, 2)
+    assert idx[0].tolist() == [0, 2]
+    assert np.allclose(wt[0], [e ** 10 / zs, e ** 2 / zs], rtol=1e-14, atol=0)
+    _, _, idx, wt = orc.route_variant(x, w, b, 2, renorm=True)
+    assert np.allclose(wt[0], [e ** 10 / (e ** 10 + e ** 2), e ** 2 / (e ** 10 + e ** 2)], rtol=1e-14, atol=0)
+    # selection-only bias: the same picks, weights from the unbiased softmax
+    z = 1 + e + e ** 2 + e ** 3
+    lg, _, idx, wt = orc.route_variant(x, w, b, 2, bias_select_only=True)
+    assert idx[0].tolist() == [0, 2]
+    assert np.array_equal(lg[0], [0.0, 1.0, 2.0, 3.0])
+    assert np.allclose(wt[0], [1 / z, e ** 2 / z], rtol=1e-15, atol=0)
+    _, _, idx, wt = orc.route_variant(x, w, b, 2, renorm=True, bias_select_only=True)
+    assert idx[0].tolist() == [0, 2]
+    assert np.allclose(wt[0], [1 / (1 + e ** 2), e ** 2 / (1 + e ** 2)], rtol=1e-15, atol=0)
+
+
+def test_route_variants_selection_ties_go_to_lower_index(orc):
+    """Selection scores tied by the bias: (0+2, 1+1, 2+0, 3-1) all equal 2."""
+    x, w, _ = _variant_case()
+    b = np.array([2.0, 1.0, 0.0, -1.0], dtype=np.float32)
+    _, _, idx, _ = orc.route_variant(x, w, b, 3, bias_select_only=True)
+    assert idx[0].tolist() == [0, 1, 2]
+
+
+def test_route_variants_invariants(orc):
+    rng = np.random.default_rng(21)
+    T, d, E, k = 5, 64, 40, 6
+    x = np.array([[k3gen.bf16_bits(v) for v in row] for row in rng.standard_normal((T, d))],
+                 dtype=np.uint16)
+    w = (rng.standard_normal((E, d)) / 8).astype(np.float32)
+    b = rng.standard_normal(E).astype(np.float32)
+    # plain variant = the pages' routing
+    l0, p0, i0, w0 = orc.route(x, w, b, k)
+    l1, p1, i1, w1 = orc.route_variant(x, w, b, k)
+    assert np.array_equal(i0, i1) and np.array_equal(w0, w1) and np.array_equal(l0, l1)
+    # renormalised: same picks, weights proportional to p, summing to one
+    _, _, i2, w2 = orc.route_variant(x, w, b, k, renorm=True)
+    assert np.array_equal(i2, i0)
+    assert np.allclose(w2.sum(1), 1.0, rtol=0, atol=1e-15)
+    assert np.allclose(w2 / w2[:, :1], w0 / w0[:, :1], rtol=1e-14)
+    # k = E: renormalising changes nothing (the probabilities already sum to one)
+    _, _, _, wa = orc.route_variant(x, w, b, E)
+    _, _, _, wb = orc.route_variant(x, w, b, E, renorm=True)
+    assert np.allclose(wa, wb, rtol=1e-14, atol=0)
+    # selection-only bias with a zero bias, or none, is the unbiased routing
+    l3, _, i3, w3 = orc.route_variant(x, w, np.zeros(E, np.float32), k, bias_select_only=True)
+    l4, _, i4, w4 = orc.route(x, w, None, k)
+    assert np.array_equal(i3, i4) and np.array_equal(w3, w4) and np.array_equal(l3, l4)
+    # selection-only: picks = top-k of (l + b); weights = the unbiased softmax at the picks
+    l5, p5, i5, w5 = orc.route_variant(x, w, b, k, bias_select_only=True)
+    s = l5 + b.astype(np.float64)
+    for t in range(T):
+        assert i5[t].tolist() == sorted(range(E), key=lambda e: (-s[t, e], e))[:k]
+    unb = np.exp(l5 - l5.max(1, keepdims=True))
+    unb /= unb.sum(1, keepdims=True)
+    assert np.allclose(w5, np.take_along_axis(unb, i5.astype(np.int64), 1), rtol=1e-13)

@@ -8,7 +8,9 @@ import torch
 
 import k3gen
 from k3gen import device as kdev
-from parity import G1_TOL, bf16_bits_to_f64, check_topk_row, g1_error
+from gpu_helpers import (dims_of, last_group_of_busiest_expert, oracle_reference, run_layer,
+                         sample_tokens)
+from parity import G1_TOL, check_topk_row, g1_error
 
 pytestmark = pytest.mark.gpu
 
@@ -23,62 +25,9 @@ def _need_gpu():
     kdev.release_all()
 
 
-def dims_of(cfg, flags=0):
-    return m.make_dims(cfg.d, cfg.ff, cfg.E, cfg.k, cfg.ff_shared, flags)
-
-
-def run_layer(cfg, W, x, bias, T, flags=0, ptrs=None):
-    dims = dims_of(cfg, flags)
-    ws = m.new_workspace(dims, T)
-    out32 = bool(flags & m.K3MOE_OUT_FP32)
-    y = torch.empty((T, cfg.d), dtype=torch.float32 if out32 else torch.int16, device="cuda")
-    idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
-    w = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
-    sg, su, sd = W.shared if not (flags & m.K3MOE_NO_SHARED) else (None, None, None)
-    st = m.k3moe_layer(x, T, W.w_router, bias, W.blob_ptrs if ptrs is None else ptrs, sg, su, sd,
-                       dims, y, idx, w, ws)
-    m.check(st, "k3moe_layer")
-    torch.cuda.synchronize()
-    m.check(m.k3moe_device_status(ws), "device status")
-    return y.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy()
-
-
-def oracle_reference(orc, cfg, W, x_host, bias_host, gpu_idx, tokens, shared=True):
-    """Oracle y for the given tokens, routed with the GPU's selection when the
-    oracle agrees it is a valid top-k (C14), else with the oracle's own."""
-    xs = x_host[tokens]
-    logits, probs, idx_o, w_o = orc.route(xs, W.w_router_host, bias_host, cfg.k)
-    problems = []
-    idx_use = np.empty_like(idx_o)
-    n_decisive = 0
-    for i, t in enumerate(tokens):
-        decisive, pr = check_topk_row(logits[i], gpu_idx[t], cfg.k)
-        n_decisive += decisive
-        problems += [f"token {t}: {p}" for p in pr]
-        idx_use[i] = gpu_idx[t]
-    weight = np.take_along_axis(probs, idx_use.astype(np.int64), axis=1)
-    cache = {}
-    slot_blobs = []
-    for i in range(len(tokens)):
-        for j in range(cfg.k):
-            e = int(idx_use[i, j])
-            if e not in cache:
-                cache[e] = W.blob_host(e)
-            slot_blobs.append(cache[e])
-    sh = W.shared_host if shared else None
-    y = orc.combine(xs, weight, slot_blobs, sh, cfg.d, cfg.ff)
-    return y, problems, n_decisive, probs, idx_use
-
-
-def sample_tokens(T, n):
-    if T <= n:
-        return list(range(T))
-    rng = np.random.default_rng(T)
-    s = set(rng.choice(T, n - 2, replace=False).tolist()) | {0, T - 1}
-    return sorted(s)
-
-
-SAMPLES = {"tiny": 4, "k3_decode": 1, "k3_decode_t8": 8, "k3_prefill_512": 12, "k3_prefill_4096": 8}
+# tokens compared with the oracle per workload; on the grouped-prefill
+# workloads the tokens of the busiest expert's last (ragged) group are added
+SAMPLES = {"tiny": 4, "k3_decode": 1, "k3_decode_t8": 8, "k3_prefill_512": 64, "k3_prefill_4096": 64}
 
 
 @pytest.mark.parametrize("name", list(k3gen.CONFIGS))
@@ -94,7 +43,10 @@ def test_layer_parity(orc, name):
     r = torch.from_numpy(y32).to(torch.bfloat16).view(torch.int16).numpy()
     assert np.array_equal(r, y16), "bf16 output is not RNE(fp32 output)"
     tokens = sample_tokens(T, SAMPLES[name])
-    yo, problems, nd, probs, idx_use = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx,
+    if T > 8:
+        tail, _, _ = last_group_of_busiest_expert(idx)
+        tokens = sorted(set(tokens) | set(tail))
+    yo, problems, nd, probs, idx_use, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx,
                                                          tokens)
     assert not problems, problems[:5]
     # routing weights: fp32 softmax vs fp64
@@ -150,7 +102,7 @@ def test_layer_no_shared_routed_only(orc):
     inp = kdev.DeviceInputs(cfg)
     y, idx, w = run_layer(cfg, W, inp.x, inp.bias, inp.T, m.K3MOE_OUT_FP32 | m.K3MOE_NO_SHARED)
     tokens = list(range(inp.T))
-    yo, problems, _, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx, tokens,
+    yo, problems, _, _, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx, tokens,
                                              shared=False)
     assert not problems
     assert g1_error(y, yo).max() <= G1_TOL
@@ -165,7 +117,7 @@ def test_ragged_token_counts(orc, T):
     W = kdev.weights(cfg)
     inp = kdev.DeviceInputs(cfg, T=T)
     y, idx, w = run_layer(cfg, W, inp.x, inp.bias, T, m.K3MOE_OUT_FP32)
-    yo, problems, _, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx,
+    yo, problems, _, _, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx,
                                              list(range(T)))
     assert not problems, problems[:3]
     assert g1_error(y, yo).max() <= G1_TOL
@@ -177,7 +129,7 @@ def test_degenerate_k(orc, E, k):
     W = kdev.weights(cfg)
     inp = kdev.DeviceInputs(cfg, T=6)
     y, idx, w = run_layer(cfg, W, inp.x, inp.bias, 6, m.K3MOE_OUT_FP32)
-    yo, problems, _, probs, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx,
+    yo, problems, _, probs, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx,
                                                  list(range(6)))
     assert not problems
     if k == E:
@@ -270,7 +222,7 @@ def test_grouped_prefill_parity(orc, cfg, T):
     r = torch.from_numpy(y32).to(torch.bfloat16).view(torch.int16).numpy()
     assert np.array_equal(r, y16), "bf16 output is not RNE(fp32 output)"
     tokens = sample_tokens(T, 24)
-    yo, problems, _, probs, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx, tokens,
+    yo, problems, _, probs, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx, tokens,
                                                  shared=cfg.ff_shared > 0)
     assert not problems, problems[:3]
     wref = np.take_along_axis(probs, idx[tokens].astype(np.int64), axis=1)
@@ -299,7 +251,7 @@ def test_grouped_prefill_matches_chunked_path(orc):
         m.check(m.k3moe_device_status(ws), "device status")
         outs.append((y.cpu().numpy(), idx.cpu().numpy()))
     assert np.array_equal(outs[0][1], outs[1][1])
-    yo, problems, _, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, outs[0][1],
+    yo, problems, _, _, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, outs[0][1],
                                              list(range(T)))
     assert not problems
     for y, _ in outs:
@@ -319,6 +271,6 @@ def test_grouped_prefill_deterministic_and_multi_pass(orc):
         assert np.array_equal(u, v)
     y, idx, _ = a
     tokens = sample_tokens(T, 16)
-    yo, problems, _, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx, tokens)
+    yo, problems, _, _, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx, tokens)
     assert not problems
     assert g1_error(y[tokens], yo).max() <= G1_TOL

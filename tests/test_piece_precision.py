@@ -67,3 +67,34 @@ def test_three_pieces_would_not_do(data):
     """Why not fewer: 3 pieces leave the SwiGLU activations near the gate."""
     _, _, h, Wd = data
     assert g1_like(h, 3, Wd) > 1e-3
+
+
+def _outliers_every_block(x, rng):
+    """One element x2^8 and one x2^10 in every 32-element block."""
+    xo = x.copy().reshape(x.shape[0], -1, 32)
+    T, nb, _ = xo.shape
+    for t in range(T):
+        for b in range(nb):
+            i, j = rng.choice(32, 2, replace=False)
+            xo[t, b, i] *= 2.0 ** 8
+            xo[t, b, j] *= 2.0 ** 10
+    return xo.reshape(x.shape)
+
+
+def test_pieces_with_outlier_activations(data):
+    """Outliers: a 32-element block whose largest element is 2^10 above the
+    others spends its first pieces on that element, so the small ones are
+    resolved later; the error is measured against the largest output, which
+    the outliers also dominate.  With every block holding a 2^8 and a 2^10
+    outlier, or with 8 hidden channels 1000x the others, 4 pieces stay 6x
+    inside the 2e-3 gate and 6 pieces ~100x."""
+    x, W, h, Wd = data
+    rng = np.random.default_rng(11)
+    xb = _outliers_every_block(x, rng)
+    xc = x.copy()
+    xc[:, rng.choice(x.shape[1], 8, replace=False)] *= 1000.0
+    hb = _outliers_every_block(h, rng)
+    for P, bound in ((4, 3.5e-4 * 1.5), (6, 2e-5)):
+        assert g1_like(xb, P, W) < bound, P
+        assert g1_like(xc, P, W) < bound, P
+        assert g1_like(hb, P, Wd) < bound, P
