@@ -316,6 +316,10 @@ def main():
     ap.add_argument("--config", default="k3_decode", choices=list(k3gen.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="profiling mode: no e2e/cpu legs")
+    ap.add_argument("--layers", type=int, default=92,
+                    help="also time one token through this many K3 MoE layers in a row (0: skip)")
+    ap.add_argument("--cache-slots", type=int, nargs="*", default=[64, 128, 256],
+                    help="expert-cache slot counts to simulate (the middle one also timed); none: skip")
     ap.add_argument("--no-configs", action="store_true",
                     help="measure the headline workload only (not the T=8 / prefill workloads)")
     ap.add_argument("--experts", type=int, default=None,
@@ -370,6 +374,12 @@ def main():
     if args.config == "k3_decode" and args.experts is None and not args.quick and not args.no_configs:
         for name in ("k3_decode_t8", "k3_prefill_512", "k3_prefill_4096"):
             others[name] = measure(k3gen.CONFIGS[name], W, k3, args, flush_l2, stream, world, e2e=False)
+    model = None
+    if args.config == "k3_decode" and args.experts is None and not args.quick and args.layers > 0:
+        model = measure_model(cfg, W, k3, args, flush_l2, stream, world, args.layers)
+    cache = None
+    if args.config == "k3_decode" and args.experts is None and not args.quick and args.cache_slots:
+        cache = measure_cache(W, k3, args, stream)
     clk = clocks.stop()
 
     T = head["T"]
@@ -408,10 +418,158 @@ def main():
     }
     if others:
         line["configs"] = {name: summary(r, peak) for name, r in others.items()}
+    if model is not None:
+        line["model_decode"] = model
+    if cache is not None:
+        line["expert_cache"] = cache
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def measure_model(cfg, W, k3, args, flush_l2, stream, world, n_layers):
+    """One decode token through n_layers K3 MoE layers in a row (the steps of
+    a pre-norm block: RMSNorm, the layer, the residual add; k3moe_layer_residual
+    with the residual stream updated in place), every layer with its own router,
+    shared expert and norm weights and its own permutation of the resident
+    experts, captured in a CUDA graph.  L2 is flushed before each token, not
+    between layers: consecutive layers stream different weights."""
+    import torch
+    E, d = cfg.E, cfg.d
+    dims = k3.make_dims(cfg.d, cfg.ff, cfg.E, cfg.k, cfg.ff_shared, 0)
+    ws = k3.new_workspace(dims, 1)
+    layers = []
+    for l in range(n_layers):
+        seed = 1000 + l
+        wr = torch.from_numpy(k3gen.router(cfg, seed)).cuda()
+        sg, su, sd = (torch.from_numpy(a.view(np.int16)).cuda() for a in k3gen.shared(cfg, seed))
+        g = torch.from_numpy(k3gen.norm_weights(cfg, seed).view(np.int16)).cuda()
+        perm = np.random.default_rng(seed).permutation(E)
+        ptrs = W.blob_ptrs[torch.from_numpy(perm).cuda()].contiguous()
+        layers.append((wr, sg, su, sd, g, ptrs))
+    h0 = torch.from_numpy(k3gen.hidden(cfg, T=1).view(np.int16)).cuda()
+    h = h0.clone()
+
+    def token():
+        for (wr, sg, su, sd, g, ptrs) in layers:
+            k3.check(k3.k3moe_layer_residual(h, 1, g, 1e-6, wr, None, ptrs, sg, su, sd, dims, h, ws),
+                     "k3moe_layer_residual")
+
+    for _ in range(2):
+        h.copy_(h0)
+        token()
+    torch.cuda.synchronize()
+    k3.check(k3.k3moe_device_status(ws), "device status")
+    graph = None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            token()
+        graph.replay()
+        torch.cuda.synchronize()
+        k3.check(k3.k3moe_device_status(ws), "device status")
+    except Exception as ex:  # capture refused: time the launches themselves
+        graph = None
+        capture_error = str(ex).splitlines()[0][:200]
+    steps = max(3, min(args.steps, 10))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        h.copy_(h0)
+        flush_l2(i)
+        ev[i][0].record(stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            token()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    k3.check(k3.k3moe_device_status(ws), "device status")
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, "cuda")
+    ms = total_ms / steps
+    peak, _ = load_peaks()
+    gbs = n_layers * alg_bytes(cfg, cfg.k) / (ms / 1000.0) / 1e9  # 16 distinct experts per layer at T=1
+    out = {"layers": n_layers, "tokens_per_step": 1, "steps": steps, "ms_per_token": round(ms, 4),
+           "value": round(world * 1000.0 / ms, 2), "unit": "tokens/s (all layers)",
+           "us_per_layer": round(1000.0 * ms / n_layers, 2), "hbm_gbs": round(gbs, 1),
+           "hbm_frac": round(gbs / peak, 4), "cuda_graph": graph is not None,
+           "gpu_launches_per_token": n_layers}
+    if graph is None:
+        out["cuda_graph_error"] = capture_error
+    del graph, layers
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_cache(W, k3, args, stream):
+    """The expert cache under the Zipf-skewed routing of the 512-token K3
+    workload, decoded one token at a time: the hit rate of the cache's own
+    policy (k3moe_cache_plan over the tokens' routing) for each slot count,
+    and, for the middle one, real k3moe_layer_cached calls with the experts in
+    page-locked host memory (only the experts these tokens ever select are
+    materialised on the host; the others are never fetched)."""
+    import torch
+    cfg = k3gen.CONFIGS["k3_prefill_512"]
+    inp = kdev_inputs(cfg)
+    T = inp.T
+    dims = k3.make_dims(cfg.d, cfg.ff, cfg.E, cfg.k, cfg.ff_shared, 0)
+    ws = k3.new_workspace(dims, 8)
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
+    k3.check(k3.k3moe_route(inp.x, T, W.w_router, inp.bias, dims, idx, wts, ws), "route")
+    idx = idx.cpu().numpy()
+    used = sorted(set(idx.reshape(-1).tolist()))
+    sb = k3.k3moe_cache_slot_bytes(dims)
+    out = {"workload": workload_desc(cfg) + ", decoded one token per call", "tokens": T,
+           "distinct_experts": len(used), "policy": "least recently used over slots", "slots": {}}
+    for S in args.cache_slots:
+        fake = type("F", (), {"data_ptr": lambda self: 1 << 40, "numel": lambda self: S * sb,
+                              "element_size": lambda self: 1})()
+        c = k3.ExpertCache(dims, S, fake, [0x1000] * cfg.E)
+        for t in range(T):
+            k3.check(c.plan(idx[t])[0], "cache plan")
+        st = c.stats()
+        c.close()
+        out["slots"][str(S)] = {"hit_rate": round(st["hits"] / st["requests"], 4), "fills": st["fills"],
+                                "device_bytes": S * sb}
+    S = args.cache_slots[len(args.cache_slots) // 2]
+    host = torch.empty((len(used), cfg.blob_bytes), dtype=torch.uint8).pin_memory()
+    ptrs = [0] * cfg.E
+    for i, e in enumerate(used):
+        host[i].copy_(W.blobs[e].cpu())
+        ptrs[e] = host.data_ptr() + i * cfg.blob_bytes
+    dummy = torch.zeros(16, dtype=torch.uint8).pin_memory()  # never fetched: no token selects these
+    ptrs = [p if p else dummy.data_ptr() for p in ptrs]
+    slots = torch.empty(S * sb, dtype=torch.uint8, device="cuda")
+    table = torch.zeros(cfg.E, dtype=torch.int64, device="cuda")
+    cache = k3.ExpertCache(dims, S, slots, ptrs)
+    idx_host = torch.empty(cfg.k, dtype=torch.int32).pin_memory()
+    y = torch.empty((1, cfg.d), dtype=torch.int16, device="cuda")
+    sg, su, sd = W.shared
+    n = min(T, 256)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for t in range(n):
+        k3.check(k3.k3moe_layer_cached(cache, inp.x[t:t + 1], 1, W.w_router, inp.bias, table, sg, su, sd, dims,
+                                       y, idx_host, ws), "k3moe_layer_cached")
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    k3.check(k3.k3moe_device_status(ws), "device status")
+    st = cache.stats()
+    out["timed"] = {"slots": S, "tokens": n, "tokens_per_s": round(n / wall, 1),
+                    "ms_per_token": round(1000.0 * wall / n, 3), "hit_rate": round(st["hits"] / st["requests"], 4),
+                    "fills": st["fills"], "host_to_device_gb": round(st["fills"] * cfg.blob_bytes / 1e9, 3),
+                    "clock": "host wall clock (each call synchronises on its routing)"}
+    cache.close()
+    del host, slots
+    torch.cuda.empty_cache()
+    return out
+
+
+def kdev_inputs(cfg):
+    from k3gen import device as kdev
+    return kdev.DeviceInputs(cfg)
 
 
 def cpu_model():

@@ -191,6 +191,84 @@ k3moe_status k3moe_layer(const void *x, int32_t T, const float *w_router, const 
                          void *stream);
 
 /*
+ * The layer inside a pre-norm transformer block: the step before it (RMSNorm
+ * of the residual stream) and the one after it (the residual add) fused in
+ * (the kimi-k3-in-c project card lists RMSNorm among its kernels; the pages
+ * give no formula, so the standard one is used):
+ *   x      = RNE_bf16( h * norm_w / sqrt(mean(h^2) + eps) )   per token
+ *   h_out  = h + layer(x)                                      rounded once
+ * h: bf16 [T][d] (the residual stream); norm_w: bf16 [d], 16-byte aligned;
+ * eps >= 0; h_out: [T][d] bf16 (or fp32 with K3MOE_OUT_FP32), and may be h
+ * itself (updated in place).  The normalisation runs in fp32 inside the
+ * kernels that read x (1/rms as 1/sqrtf of the fp32 mean of squares, each
+ * element (h * r) * w rounded to bf16).  Other arguments as for k3moe_layer
+ * (no routing copies).  Up to 8 tokens per pass this needs the one-launch
+ * decode kernel's shape limits (K3MOE_ERR_UNSUPPORTED_SHAPE otherwise); with
+ * a workspace sized for more tokens the grouped path normalises each pass
+ * first and adds h in its final sum.
+ */
+k3moe_status k3moe_layer_residual(const void *h, int32_t T, const void *norm_w, float eps,
+                                  const float *w_router, const float *bias,
+                                  const uint8_t *const *expert_blobs, const void *shared_wg,
+                                  const void *shared_wu, const void *shared_wd,
+                                  const k3moe_dims *dims, void *h_out, void *ws, size_t ws_bytes,
+                                  void *stream);
+
+/*
+ * Expert cache: the routed experts live in host memory and only the most
+ * recently used ones in device memory, in n_slots slots -- the pages' defining
+ * idea (the kimi-k3-in-c project card: experts are streamed on demand, never
+ * all resident; their engine keeps an LRU of RAM slots fed from NVMe), one
+ * level up: host memory -> HBM by the copy engine.  The layer calls reach the
+ * experts through their device pointer table, which the cache rewrites.
+ *   k3moe_cache_slot_bytes: bytes of one slot (the blob size rounded up to 256).
+ *   k3moe_cache_create: slot_mem is caller-owned device memory of at least
+ *     n_slots * slot bytes, 256-byte aligned; host_blobs holds E host pointers
+ *     to the experts' blobs (page-locked memory makes the copies asynchronous;
+ *     it must stay valid while the cache is used).  The library allocates the
+ *     small host-side bookkeeping (freed by k3moe_cache_destroy) and no device
+ *     memory.  Starts empty.
+ *   k3moe_cache_fetch: makes every expert in experts[0..n) (host array,
+ *     repeats allowed) resident: experts already in a slot are marked used;
+ *     each missing one (in order of first appearance) takes a free slot or the
+ *     least recently used slot not holding a requested expert (lowest slot on
+ *     ties) and is copied in with one cudaMemcpyAsync on `stream`.  Then the
+ *     device pointer table ptr_table (E entries) is rewritten on `stream`:
+ *     each resident expert's slot address, NULL for the others (a call that
+ *     selects a non-resident expert reports K3MOE_ERR_DEVICE_CHECK through the
+ *     workspace status).  K3MOE_ERR_INVALID_ARGUMENT, with nothing changed,
+ *     when an id is out of range or more distinct experts than slots are asked.
+ *   k3moe_cache_plan: the same bookkeeping without any copy (simulation).
+ *   k3moe_layer_cached: k3moe_layer with the experts behind the cache: per
+ *     pass of up to 8 tokens, the routing (the same kernel and bits as the
+ *     layer's own), its picks copied to idx_host (host, [T][k] int32, page-
+ *     locked preferred), a SYNCHRONISATION of `stream`, a fetch of the picks,
+ *     then the layer on the fetched experts.  ws needs k3moe_workspace_size(dims, 8).
+ */
+typedef struct k3moe_cache k3moe_cache;
+typedef struct {
+    uint64_t requests;  /* distinct experts asked for, summed over fetches */
+    uint64_t hits;      /* of those, already resident */
+    uint64_t fills;     /* copied in */
+    uint64_t evictions; /* resident experts replaced */
+} k3moe_cache_stats;
+size_t k3moe_cache_slot_bytes(const k3moe_dims *dims);
+k3moe_status k3moe_cache_create(const k3moe_dims *dims, int32_t n_slots, void *slot_mem,
+                                size_t slot_mem_bytes, const void *const *host_blobs,
+                                k3moe_cache **cache);
+void k3moe_cache_destroy(k3moe_cache *cache);
+k3moe_status k3moe_cache_fetch(k3moe_cache *cache, const int32_t *experts, int32_t n,
+                               void *ptr_table, void *stream);
+k3moe_status k3moe_cache_plan(k3moe_cache *cache, const int32_t *experts, int32_t n,
+                              int32_t *filled, int32_t *n_filled);
+k3moe_status k3moe_cache_get_stats(const k3moe_cache *cache, k3moe_cache_stats *stats);
+k3moe_status k3moe_layer_cached(k3moe_cache *cache, const void *x, int32_t T, const float *w_router,
+                                const float *bias, void *ptr_table, const void *shared_wg,
+                                const void *shared_wu, const void *shared_wd,
+                                const k3moe_dims *dims, void *y, int32_t *idx_host, void *ws,
+                                size_t ws_bytes, void *stream);
+
+/*
  * k3moe_layer with the activations in HOST memory: copies x_host ([T][d]
  * bf16) into the workspace, runs the layer, and copies y back to y_host
  * ([T][d], bf16 or fp32 per flags), all ordered on `stream` (the copies are

@@ -29,7 +29,7 @@ _lock = threading.Lock()
 _lib = None
 
 # Streams of the counter-based generator.
-STREAM_X, STREAM_ROUTER, STREAM_BIAS, STREAM_NIB, STREAM_SCALE, STREAM_SHARED, STREAM_ZIPF = range(7)
+STREAM_X, STREAM_ROUTER, STREAM_BIAS, STREAM_NIB, STREAM_SCALE, STREAM_SHARED, STREAM_ZIPF, STREAM_NORM = range(8)
 
 # E8M0 exponents of the synthetic experts: uniform in [118, 124].
 SCALE_LO, SCALE_COUNT = 118, 7
@@ -201,6 +201,15 @@ def all_blobs(cfg: Config, seed: int = 0) -> np.ndarray:
     out = np.empty((cfg.E, cfg.blob_bytes), dtype=np.uint8)
     for e in range(cfg.E):
         expert_blob(cfg, e, seed, out[e])
+    return out
+
+
+def norm_weights(cfg: Config, seed: int = 0) -> np.ndarray:
+    """RMSNorm weights [d] as bf16 bits: bf16(1 + 0.1 N(0,1)), stream 7."""
+    out = np.empty((cfg.d,), dtype=np.uint16)
+    base = normal(seed, STREAM_NORM, 0, cfg.d)
+    for j in range(cfg.d):
+        out[j] = bf16_bits(1.0 + 0.1 * base[j])
     return out
 
 

@@ -50,6 +50,11 @@ def make_dims(d, ff, n_experts, top_k, ff_shared, flags=0) -> k3moe_dims:
     return k3moe_dims(d, ff, n_experts, top_k, ff_shared, flags)
 
 
+class k3moe_cache_stats(ctypes.Structure):
+    _fields_ = [("requests", ctypes.c_uint64), ("hits", ctypes.c_uint64), ("fills", ctypes.c_uint64),
+                ("evictions", ctypes.c_uint64)]
+
+
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
                       "`python mxfp4_routed_expert_softmax_b200/build.py` (nvcc, sm_100a)")
@@ -67,6 +72,8 @@ _SIGS = {
     "k3moe_expert_ffn": ([_vp, _i32, _vp, _dp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "k3moe_layer": ([_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _dp, _vp, _vp, _vp, _vp, _sz, _vp],
                     ctypes.c_int),
+    "k3moe_layer_residual": ([_vp, _i32, _vp, ctypes.c_float, _vp, _vp, _vp, _vp, _vp, _vp, _dp, _vp, _vp,
+                              _sz, _vp], ctypes.c_int),
     "k3moe_layer_from_host": ([_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _dp, _vp, _vp, _sz, _vp],
                               ctypes.c_int),
     "k3moe_layer_timed": ([_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _dp, _vp, _vp, _sz, _vp,
@@ -76,6 +83,14 @@ _SIGS = {
     "k3moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "k3moe_last_error": ([], ctypes.c_char_p),
     "k3moe_debug_set_fault": ([_i32, ctypes.c_uint64], ctypes.c_int),
+    "k3moe_cache_slot_bytes": ([_dp], _sz),
+    "k3moe_cache_create": ([_dp, _i32, _vp, _sz, _vp, ctypes.POINTER(_vp)], ctypes.c_int),
+    "k3moe_cache_destroy": ([_vp], None),
+    "k3moe_cache_fetch": ([_vp, _vp, _i32, _vp, _vp], ctypes.c_int),
+    "k3moe_cache_plan": ([_vp, _vp, _i32, _vp, ctypes.POINTER(_i32)], ctypes.c_int),
+    "k3moe_cache_get_stats": ([_vp, ctypes.POINTER(k3moe_cache_stats)], ctypes.c_int),
+    "k3moe_layer_cached": ([_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _dp, _vp, _vp, _vp, _sz, _vp],
+                           ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -150,6 +165,14 @@ def k3moe_layer(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu, shared
                            _stream(stream))
 
 
+def k3moe_layer_residual(h, T, norm_w, eps, w_router, bias, expert_blobs, shared_wg, shared_wu, shared_wd,
+                         dims, h_out, ws, ws_bytes=None, stream=None) -> int:
+    ws_bytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    return lib.k3moe_layer_residual(_ptr(h), T, _ptr(norm_w), float(eps), _ptr(w_router), _ptr(bias),
+                                    _ptr(expert_blobs), _ptr(shared_wg), _ptr(shared_wu), _ptr(shared_wd),
+                                    ctypes.byref(dims), _ptr(h_out), _ptr(ws), ws_bytes, _stream(stream))
+
+
 def k3moe_layer_noalloc(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu, shared_wd, dims, y,
                         stream=None) -> int:
     return lib.k3moe_layer_noalloc(_ptr(x), T, _ptr(w_router), _ptr(bias), _ptr(expert_blobs),
@@ -192,6 +215,60 @@ def k3moe_debug_set_fault(mode: int, wait_limit_ns: int = 0) -> int:
     device waits run out (no GPU fault); wait_limit_ns bounds every wait
     (0: the default).  Reset with (0, 0)."""
     return lib.k3moe_debug_set_fault(mode, wait_limit_ns)
+
+
+class ExpertCache:
+    """Handle of a k3moe_cache (argument marshalling only; the policy and the
+    copies are the library's).  slot_mem: device tensor of at least
+    n_slots * k3moe_cache_slot_bytes(dims) bytes; host_blob_ptrs: E host
+    addresses (kept alive by the caller)."""
+
+    def __init__(self, dims, n_slots, slot_mem, host_blob_ptrs):
+        import numpy as np
+        self._ptrs = np.ascontiguousarray(np.asarray(host_blob_ptrs, dtype=np.uint64))
+        h = ctypes.c_void_p()
+        nbytes = slot_mem.numel() * slot_mem.element_size() if hasattr(slot_mem, "numel") else 0
+        check(lib.k3moe_cache_create(ctypes.byref(dims), n_slots, _ptr(slot_mem), nbytes,
+                                     self._ptrs.ctypes.data, ctypes.byref(h)), "k3moe_cache_create")
+        self.handle = h
+
+    def plan(self, experts):
+        import numpy as np
+        e = np.ascontiguousarray(np.asarray(experts, dtype=np.int32))
+        out = np.empty(max(1, e.size), dtype=np.int32)
+        n = ctypes.c_int32(0)
+        st = lib.k3moe_cache_plan(self.handle, e.ctypes.data, e.size, out.ctypes.data, ctypes.byref(n))
+        return st, out[:n.value].tolist()
+
+    def fetch(self, experts, ptr_table, stream=None) -> int:
+        import numpy as np
+        e = np.ascontiguousarray(np.asarray(experts, dtype=np.int32))
+        return lib.k3moe_cache_fetch(self.handle, e.ctypes.data, e.size, _ptr(ptr_table), _stream(stream))
+
+    def stats(self) -> dict:
+        st = k3moe_cache_stats()
+        check(lib.k3moe_cache_get_stats(self.handle, ctypes.byref(st)), "k3moe_cache_get_stats")
+        return {"requests": st.requests, "hits": st.hits, "fills": st.fills, "evictions": st.evictions}
+
+    def close(self):
+        if self.handle:
+            lib.k3moe_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        self.close()
+
+
+def k3moe_cache_slot_bytes(dims: k3moe_dims) -> int:
+    return lib.k3moe_cache_slot_bytes(ctypes.byref(dims))
+
+
+def k3moe_layer_cached(cache, x, T, w_router, bias, ptr_table, shared_wg, shared_wu, shared_wd, dims, y,
+                       idx_host, ws, ws_bytes=None, stream=None) -> int:
+    ws_bytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    return lib.k3moe_layer_cached(cache.handle, _ptr(x), T, _ptr(w_router), _ptr(bias), _ptr(ptr_table),
+                                  _ptr(shared_wg), _ptr(shared_wu), _ptr(shared_wd), ctypes.byref(dims),
+                                  _ptr(y), _ptr(idx_host), _ptr(ws), ws_bytes, _stream(stream))
 
 
 def new_workspace(dims: k3moe_dims, T_max: int, device="cuda", host_staging: bool = False):

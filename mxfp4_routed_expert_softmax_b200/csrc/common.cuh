@@ -159,4 +159,25 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
+// ------------------------------------------------------------- RMSNorm --
+// 1 / sqrt(mean(h^2) + eps) of one token of d bf16 values, by one warp: lane
+// l sums the squares of elements l, l + 32, ... in fp32, then a fixed
+// butterfly adds the lanes, so every warp that runs it gets the same bits.
+__device__ __forceinline__ float warp_rms_inv(const uint16_t *h, int d, float eps) {
+    const int lane = threadIdx.x & 31;
+    float ss = 0.f;
+    for (int j = lane; j < d; j += 32) {
+        const float v = __uint_as_float((uint32_t)h[j] << 16);
+        ss = fmaf(v, v, ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    return 1.0f / sqrtf(ss / (float)d + eps);
+}
+// One element of the normalised token: RNE_bf16((h * r) * g), bf16 bits.
+__device__ __forceinline__ uint16_t rms_norm_bf16(uint16_t h, float r, uint16_t g) {
+    const float v = (__uint_as_float((uint32_t)h << 16) * r) * __uint_as_float((uint32_t)g << 16);
+    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
 }  // namespace k3

@@ -7,12 +7,14 @@
 
 #include <atomic>
 #include <cstdio>
+#include <new>
 #include <cstring>
 #include <mutex>
 #include <string>
 
 #include "common.cuh"
 #include "decode_kernels.cuh"
+#include "expert_cache.cuh"
 #include "k3moe.h"
 #include "layer_kernel.cuh"
 #include "layout.cuh"
@@ -323,6 +325,10 @@ cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st, int *g
     return cudaLaunchKernelEx(&cfg, route_kernel, rp);
 }
 
+// TEMP: the one-launch decode kernel serves only the pre-norm calls until it
+// has been checked on the GPU.
+constexpr bool kUseLayerKernel = false;
+
 // The one-launch decode pass (layer_kernel) for this shape, if it fits: the
 // pipeline stages and the routing tables in one SM's shared memory, and the
 // rows of one CTA's router slice in its row accumulators.  0: not supported
@@ -362,10 +368,24 @@ cudaError_t launch_layer(const DeviceInfo &di, LayerParams lp, int nst, cudaStre
     return cudaLaunchKernelEx(&cfg, layer_kernel, lp);
 }
 
+// The routing of one decode pass by the one-launch kernel stopped after its
+// top-k (the picks land in the workspace and in idx_out / w_out): the same
+// bits as the routing inside a full launch of the same pass.
+cudaError_t launch_layer_route(const DeviceInfo &di, const RouteParams &rp, int nst, cudaStream_t st) {
+    LayerParams lp{};
+    lp.r = rp;
+    lp.r.wait_ns = wait_limit();
+    lp.mode = kLayerRouteOnly;
+    return launch_layer(di, lp, nst, st);
+}
+
 // Launches of the grouped prefill, pass after pass; rp carries the shapes,
 // blobs and tensor-map templates.  routing_only: stop after the top-k.
+// norm_w (non-null): x holds the residual stream h; the layer runs on
+// RMSNorm(h) (written into the pass's xn region) and h is added to its output.
 k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims, const uint16_t *x, int T,
-                          void *y, int32_t *idx_out, float *w_out, cudaStream_t st, bool routing_only = false) {
+                          void *y, int32_t *idx_out, float *w_out, cudaStream_t st, bool routing_only = false,
+                          const uint16_t *norm_w = nullptr, float eps = 0.f) {
     const int d = dims->d, E = dims->n_experts, k = dims->top_k;
     const int ffs = rp.has_shared ? dims->ff_shared : 0;
     const bool out32 = (dims->flags & K3MOE_OUT_FP32) != 0;
@@ -375,9 +395,16 @@ k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims
     cudaError_t e;
     for (int t0 = 0; t0 < T; t0 += Tp) {
         const int Tq = (T - t0) < Tp ? (T - t0) : Tp;
+        const uint16_t *xq = x + (size_t)t0 * d;
+        if (norm_w) {
+            const PfNormParams np{xq, norm_w, eps, Tq, d, reinterpret_cast<uint16_t *>(wsb + P.xn)};
+            e = launch(pf_rmsnorm_kernel, dim3(ceil_div(Tq, 8)), dim3(256), 0, st, false, np);
+            if (e != cudaSuccess) return cuda_fail(e, "prefill norm launch");
+            xq = reinterpret_cast<const uint16_t *>(wsb + P.xn);
+        }
         PfRouteParams pp{};
         pp.r = rp;
-        pp.r.x = x + (size_t)t0 * d;
+        pp.r.x = xq;
         pp.r.Tc = Tq;
         pp.r.idx_out = idx_out ? idx_out + (size_t)t0 * k : nullptr;
         pp.r.w_out = w_out ? w_out + (size_t)t0 * k : nullptr;
@@ -452,6 +479,7 @@ k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims
         cp.has_shared = ffs > 0;
         cp.out_fp32 = out32;
         cp.y = reinterpret_cast<uint8_t *>(y) + (size_t)t0 * d * (out32 ? 4 : 2);
+        cp.resid = norm_w ? x + (size_t)t0 * d : nullptr;
         e = launch(pf_combine_kernel, dim3(4 * di.sms), dim3(256), 0, st, false, cp);
         if (e != cudaSuccess) return cuda_fail(e, "prefill combine launch");
     }
@@ -469,11 +497,14 @@ struct EventHook {
     }
 };
 
+// norm_w (non-null): x is the residual stream h, the layer runs on
+// RMSNorm(h) and y = h + layer (the decode passes need the one-launch kernel).
 k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const float *bias,
                         const uint8_t *const *expert_blobs, const void *shared_wg,
                         const void *shared_wu, const void *shared_wd, const k3moe_dims *dims,
                         void *y, int32_t *idx_out, float *w_out, void *ws, size_t ws_bytes,
-                        void *stream, const void *x_host, void *y_host, EventHook *hook = nullptr) {
+                        void *stream, const void *x_host, void *y_host, EventHook *hook = nullptr,
+                        const uint16_t *norm_w = nullptr, float eps = 0.f, int layer_mode = kLayerFull) {
     k3moe_status s = check_dims(dims);
     if (s != K3MOE_OK) return s;
     const bool from_host = x_host != nullptr;
@@ -547,7 +578,8 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
             x = xstage;
             y = ystage;
         }
-        s = prefill_impl(*di, rp, dims, reinterpret_cast<const uint16_t *>(x), T, y, idx_out, w_out, st);
+        s = prefill_impl(*di, rp, dims, reinterpret_cast<const uint16_t *>(x), T, y, idx_out, w_out, st, false,
+                         norm_w, eps);
         if (s != K3MOE_OK) return s;
         if (from_host) {
             e = cudaMemcpyAsync(y_host, ystage, (size_t)T * d * ybytes, cudaMemcpyDeviceToHost, st);
@@ -556,6 +588,7 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         return K3MOE_OK;
     }
 
+    if (norm_w && layer_stages(*di, dims, T < kChunk ? T : kChunk) == 0) return K3MOE_ERR_UNSUPPORTED_SHAPE;
     for (int c0 = 0; c0 < T; c0 += kChunk) {
         const int Tc = (T - c0) < kChunk ? (T - c0) : kChunk;
         const uint16_t *xc;
@@ -594,7 +627,8 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         EventHook none;
         EventHook &hk = hook ? *hook : none;
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
-        const int lst = 0 * layer_stages(*di, dims, Tc);  // TEMP: layer kernel off until reviewed
+        const int lst = (kUseLayerKernel || norm_w || layer_mode != kLayerFull) ? layer_stages(*di, dims, Tc) : 0;
+        if (layer_mode != kLayerFull && lst == 0) return K3MOE_ERR_UNSUPPORTED_SHAPE;
         if (lst > 0) {
             // the whole pass in one launch
             LayerParams lp{};
@@ -608,6 +642,10 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
             lp.y = yc;
             lp.strict = (dims->flags & K3MOE_STRICT) != 0;
             lp.inject = g_fault_mode.load(std::memory_order_relaxed);
+            lp.norm_w = norm_w;
+            lp.eps = eps;
+            lp.resid = norm_w ? xc : nullptr;
+            lp.mode = layer_mode;
             e = launch_layer(*di, lp, lst, st);
             if (e != cudaSuccess) return cuda_fail(e, "layer launch");
             if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
@@ -693,6 +731,13 @@ k3moe_status noalloc_scratch(DeviceInfo &di, const k3moe_dims *dm, cudaStream_t 
 
 }  // namespace
 
+// The opaque cache handle of the C ABI.
+struct k3moe_cache {
+    k3::ExpertCache c;
+    std::vector<uint64_t> table;  // the last pointer table written (host copy)
+    std::vector<int> fe, fs;      // the last fetch's fills
+};
+
 extern "C" {
 
 int k3moe_abi_version(void) { return K3MOE_ABI_VERSION; }
@@ -758,7 +803,8 @@ k3moe_status k3moe_route(const void *x, int32_t T, const float *w_router, const 
         rp.route_flags = route_flags(dims);
         rp.idx_out = idx + (size_t)c0 * dims->top_k;
         rp.w_out = weight + (size_t)c0 * dims->top_k;
-        cudaError_t e = launch_route(*di, rp, st);
+        const int lst = kUseLayerKernel ? layer_stages(*di, dims, Tc) : 0;
+        cudaError_t e = lst > 0 ? launch_layer_route(*di, rp, lst, st) : launch_route(*di, rp, st);
         if (e != cudaSuccess) return cuda_fail(e);
     }
     return K3MOE_OK;
@@ -829,6 +875,17 @@ k3moe_status k3moe_layer(const void *x, int32_t T, const float *w_router, const 
                       idx_out, w_out, ws, ws_bytes, stream, nullptr, nullptr);
 }
 
+k3moe_status k3moe_layer_residual(const void *h, int32_t T, const void *norm_w, float eps,
+                                  const float *w_router, const float *bias,
+                                  const uint8_t *const *expert_blobs, const void *shared_wg,
+                                  const void *shared_wu, const void *shared_wd, const k3moe_dims *dims,
+                                  void *h_out, void *ws, size_t ws_bytes, void *stream) {
+    if (!norm_w || !aligned(norm_w, 16) || !(eps >= 0.f) || !(eps < 1e30f)) return K3MOE_ERR_INVALID_ARGUMENT;
+    return layer_impl(h, T, w_router, bias, expert_blobs, shared_wg, shared_wu, shared_wd, dims, h_out, nullptr,
+                      nullptr, ws, ws_bytes, stream, nullptr, nullptr, nullptr,
+                      reinterpret_cast<const uint16_t *>(norm_w), eps);
+}
+
 k3moe_status k3moe_layer_from_host(const void *x_host, int32_t T, const float *w_router,
                                    const float *bias, const uint8_t *const *expert_blobs,
                                    const void *shared_wg, const void *shared_wu,
@@ -882,6 +939,133 @@ k3moe_status k3moe_layer_noalloc(const void *x, int32_t T, const float *w_router
     // passes (the grouped path's region would not fit in the buffer)
     return layer_impl(x, T, w_router, bias, expert_blobs, shared_wg, shared_wu, shared_wd, dims, y,
                       nullptr, nullptr, ws, need, stream, nullptr, nullptr);
+}
+
+size_t k3moe_cache_slot_bytes(const k3moe_dims *dims) {
+    if (check_dims(dims) != K3MOE_OK) return 0;
+    return align256((size_t)3 * dims->d * dims->ff * 17 / 32);
+}
+
+k3moe_status k3moe_cache_create(const k3moe_dims *dims, int32_t n_slots, void *slot_mem,
+                                size_t slot_mem_bytes, const void *const *host_blobs,
+                                k3moe_cache **cache) {
+    if (!cache) return K3MOE_ERR_INVALID_ARGUMENT;
+    *cache = nullptr;
+    k3moe_status s = check_dims(dims);
+    if (s != K3MOE_OK) return s;
+    const size_t sb = k3moe_cache_slot_bytes(dims);
+    if (n_slots < 1 || !slot_mem || !aligned(slot_mem, 256) || !host_blobs ||
+        slot_mem_bytes < (size_t)n_slots * sb)
+        return K3MOE_ERR_INVALID_ARGUMENT;
+    for (int e = 0; e < dims->n_experts; ++e)
+        if (!host_blobs[e]) return K3MOE_ERR_INVALID_ARGUMENT;
+    k3moe_cache *c = new (std::nothrow) k3moe_cache;
+    if (!c) return K3MOE_ERR_INVALID_ARGUMENT;
+    ExpertCache &x = c->c;
+    x.E = dims->n_experts;
+    x.S = n_slots;
+    x.blob_bytes = (size_t)3 * dims->d * dims->ff * 17 / 32;
+    x.slot_bytes = sb;
+    x.slots = reinterpret_cast<uint8_t *>(slot_mem);
+    x.host.assign(host_blobs, host_blobs + x.E);
+    x.slot_of.assign(x.E, -1);
+    x.expert_of.assign(n_slots, -1);
+    x.last.assign(n_slots, 0);
+    x.stamp.assign(x.E, 0);
+    *cache = c;
+    return K3MOE_OK;
+}
+
+void k3moe_cache_destroy(k3moe_cache *cache) { delete cache; }
+
+k3moe_status k3moe_cache_plan(k3moe_cache *cache, const int32_t *experts, int32_t n, int32_t *filled,
+                              int32_t *n_filled) {
+    if (!cache || (n > 0 && !experts) || n < 0 || !n_filled) return K3MOE_ERR_INVALID_ARGUMENT;
+    if (!cache->c.plan(experts, n, cache->fe, cache->fs)) return K3MOE_ERR_INVALID_ARGUMENT;
+    *n_filled = (int32_t)cache->fe.size();
+    if (filled)
+        for (size_t i = 0; i < cache->fe.size(); ++i) filled[i] = cache->fe[i];
+    return K3MOE_OK;
+}
+
+k3moe_status k3moe_cache_fetch(k3moe_cache *cache, const int32_t *experts, int32_t n, void *ptr_table,
+                               void *stream) {
+    if (!cache || (n > 0 && !experts) || n < 0 || !ptr_table || !aligned(ptr_table, 8))
+        return K3MOE_ERR_INVALID_ARGUMENT;
+    ExpertCache &x = cache->c;
+    if (!x.plan(experts, n, cache->fe, cache->fs)) return K3MOE_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    for (size_t i = 0; i < cache->fe.size(); ++i) {
+        cudaError_t e = cudaMemcpyAsync(x.slots + (size_t)cache->fs[i] * x.slot_bytes, x.host[cache->fe[i]],
+                                        x.blob_bytes, cudaMemcpyHostToDevice, st);
+        if (e != cudaSuccess) return cuda_fail(e, "expert copy");
+    }
+    x.table(cache->table);
+    cudaError_t e = cudaMemcpyAsync(ptr_table, cache->table.data(), (size_t)x.E * 8, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "pointer table copy");
+    return K3MOE_OK;
+}
+
+k3moe_status k3moe_cache_get_stats(const k3moe_cache *cache, k3moe_cache_stats *stats) {
+    if (!cache || !stats) return K3MOE_ERR_INVALID_ARGUMENT;
+    stats->requests = cache->c.requests;
+    stats->hits = cache->c.hits;
+    stats->fills = cache->c.fills;
+    stats->evictions = cache->c.evictions;
+    return K3MOE_OK;
+}
+
+k3moe_status k3moe_layer_cached(k3moe_cache *cache, const void *x, int32_t T, const float *w_router,
+                                const float *bias, void *ptr_table, const void *shared_wg,
+                                const void *shared_wu, const void *shared_wd, const k3moe_dims *dims,
+                                void *y, int32_t *idx_host, void *ws, size_t ws_bytes, void *stream) {
+    k3moe_status s = check_dims(dims);
+    if (s != K3MOE_OK) return s;
+    if (!cache || !idx_host || T < 1 || !x || !aligned(x, 16) || !y || !aligned(y, 16) || !ws ||
+        !aligned(ws, 256) || cache->c.E != dims->n_experts)
+        return K3MOE_ERR_INVALID_ARGUMENT;
+    const Layout L = layout_for(dims, dims->top_k);
+    if (ws_bytes < L.total) return K3MOE_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo *di = nullptr;
+    s = device_info(&di);
+    if (s != K3MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int k = dims->top_k, d = dims->d;
+    const size_t ybytes = (dims->flags & K3MOE_OUT_FP32) ? 4 : 2;
+    for (int c0 = 0; c0 < T; c0 += kChunk) {
+        const int Tc = (T - c0) < kChunk ? (T - c0) : kChunk;
+        const uint16_t *xc = reinterpret_cast<const uint16_t *>(x) + (size_t)c0 * d;
+        // 1. the routing of the pass, to the host
+        RouteParams rp{};
+        rp.x = xc;
+        rp.Tc = Tc;
+        rp.wr = w_router;
+        rp.bias = bias;
+        rp.d = d;
+        rp.E = dims->n_experts;
+        rp.k = k;
+        rp.ws = reinterpret_cast<uint8_t *>(ws);
+        rp.L = L;
+        rp.route_flags = route_flags(dims);
+        // the routing by the kernel the layer call will use, so the experts
+        // fetched are exactly the ones its dispatch takes
+        const int lst = kUseLayerKernel ? layer_stages(*di, dims, Tc) : 0;
+        cudaError_t e = lst > 0 ? launch_layer_route(*di, rp, lst, st) : launch_route(*di, rp, st);
+        if (e != cudaSuccess) return cuda_fail(e, "router launch");
+        e = cudaMemcpyAsync(idx_host + (size_t)c0 * k, reinterpret_cast<uint8_t *>(ws) + L.idx,
+                            (size_t)Tc * k * 4, cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cuda_fail(e, "routing to host");
+        // 2. its experts into the cache, 3. the layer on the cached experts
+        s = k3moe_cache_fetch(cache, idx_host + (size_t)c0 * k, Tc * k, ptr_table, stream);
+        if (s != K3MOE_OK) return s;
+        s = layer_impl(xc, Tc, w_router, bias, reinterpret_cast<const uint8_t *const *>(ptr_table), shared_wg,
+                       shared_wu, shared_wd, dims, reinterpret_cast<uint8_t *>(y) + (size_t)c0 * d * ybytes,
+                       nullptr, nullptr, ws, L.total, stream, nullptr, nullptr, nullptr, nullptr, 0.f,
+                       lst > 0 ? kLayerRouted : kLayerFull);
+        if (s != K3MOE_OK) return s;
+    }
+    return K3MOE_OK;
 }
 
 k3moe_status k3moe_device_status(void *ws, void *stream) {

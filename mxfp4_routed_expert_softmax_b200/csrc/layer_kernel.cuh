@@ -63,7 +63,19 @@ struct LayerParams {
     void *y;           // [Tc][d] of this pass
     int strict;        // flag E8M0 NaN bytes among the weight scales read
     int inject;        // failure-path tests: 1 = the routing is never signalled
+    // pre-norm and residual (null: the layer alone): r.x holds the residual
+    // stream h; the layer's input is x = RMSNorm(h) with these weights, and
+    // the output y + resid
+    const uint16_t *norm_w;  // bf16 [d]
+    float eps;
+    const uint16_t *resid;   // bf16 [Tc][d], added to the layer's output before its rounding
+    // kLayerFull; kLayerRouteOnly: stop after the top-k (CTA 0 writes the
+    // routing into the workspace); kLayerRouted: take the routing from the
+    // workspace (written by a route-only launch of the same pass) instead of
+    // computing it -- the two launches together give the bits of one full one
+    int mode;
 };
+constexpr int kLayerFull = 0, kLayerRouteOnly = 1, kLayerRouted = 2;
 
 // ---------------------------------------------------------- smem layout --
 // One stage: two A boxes (2 x 16 KB, 1024-byte aligned for the 128-byte
@@ -78,7 +90,7 @@ __host__ __device__ inline int lk_stage_bytes(int N) { return (lk_sfb_off(N) + 2
 // sized for this pass: E experts, top-k, Tc tokens, hidden size d.
 struct LkSmem {
     int segs;  // row segments one warp's 2048 router floats can touch
-    int bars, ptab, blob, eid, wu, tidx, tw, racc, segr, segv, segn, misc, total;
+    int bars, ptab, blob, eid, wu, tidx, tw, racc, segr, segv, segn, misc, rn, total;
 };
 __host__ __device__ inline LkSmem lk_smem(int E, int k, int Tc, int d) {
     LkSmem s;
@@ -98,6 +110,7 @@ __host__ __device__ inline LkSmem lk_smem(int E, int k, int Tc, int d) {
     s.segv = o;   o += a16(2 * 4 * s.segs * Tc * 4);
     s.segn = o;   o += 2 * 4 * 4;
     s.misc = o;   o += 64 * 4;                        // dispatch bitmap / prefix
+    s.rn = o;     o += kChunk * 4;                    // 1 / rms of each token (pre-norm)
     s.total = o;
     return s;
 }
@@ -214,7 +227,8 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
     uint64_t *aempty = afull + 2;
     uint64_t *mready = aempty + 2;  // the routing is in shared memory
     uint64_t *mdone = mready + 1;   // every MMA this CTA issued has completed
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(mdone + 1);
+    uint64_t *rnready = mdone + 1;  // the tokens' 1 / rms are in shared memory (pre-norm)
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(rnready + 1);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tslot + 1);
     volatile int *s_U = s_abort + 1;
     volatile int *s_last = s_abort + 2;
@@ -229,6 +243,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
     float *s_segv = reinterpret_cast<float *>(tail + so.segv);  // [2][4][SG][Tc]
     int *s_segn = reinterpret_cast<int *>(tail + so.segn);      // [2][4]
     uint32_t *s_misc = reinterpret_cast<uint32_t *>(tail + so.misc);
+    float *s_rn = reinterpret_cast<float *>(tail + so.rn);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     WsHeader *hdr = reinterpret_cast<WsHeader *>(rp.ws + L.hdr);
     const int G = gridDim.x, cta = blockIdx.x;
@@ -245,6 +260,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
         }
         mbar_init(mready, 1);
         mbar_init(mdone, 1);
+        mbar_init(rnready, 1);
         fence_mbar_init();
         *s_abort = 0;
         *s_U = 0;
@@ -292,8 +308,8 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
     auto start_of = [&](const Range &r, int c) { return (int)(((long long)c * r.n) / r.G); };
     auto owner = [&](const Range &r, int unit) { return (int)((((long long)unit + 1) * r.G - 1) / r.n); };
     Range rg[4];
-    rg[0] = make_range(n0);
-    rg[1] = make_range(nrbs * nkts_d);
+    rg[0] = make_range(p.mode == kLayerRouted ? 0 : n0);
+    rg[1] = make_range(p.mode == kLayerRouteOnly ? 0 : nrbs * nkts_d);
     rg[2] = make_range(0);
     rg[3] = make_range(0);
     // units per item of the ranges with items (R1, R2, R3)
@@ -307,6 +323,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
     };
     // Before R2: the routing (one lane waits, its warp follows when warp_wide).
     auto routed_ranges = [&](bool warp_wide) {
+        if (p.mode == kLayerRouteOnly) return false;  // nothing after the routing
         int ok = 1;
         if (lane == 0) {
             ok = (!*s_abort && mbar_wait_bounded(mready, 0u, hdr, rp.wait_ns)) ? 1 : 0;
@@ -357,19 +374,39 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
         // (x as E2M1 pieces for R2, as bf16 for R1).  Then counted on
         // prep_done, which the copies warps wait for before their first
         // B tile or tensor map.
-        for (int e = lane; e < E; e += 32) s_ptab[e] = rp.blobs[e];
-        refresh_tmaps(rp, cta * 32 + lane, G * 32);
-        build_x_pieces(rp.x, Tc, d, rp.ws, L, cta, G, rp.has_shared != 0);
-        __syncwarp();
-        if (lane == 0) red_add_release(&hdr->prep_done, 1u);
+        if (p.norm_w) {
+            // 1 / rms of every token (the same bits in every CTA)
+            for (int t = 0; t < Tc; ++t) {
+                const float r = warp_rms_inv(rp.x + (size_t)t * d, d, p.eps);
+                if (lane == 0) s_rn[t] = r;
+            }
+            __syncwarp();
+            if (lane == 0)
+                asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(rnready)) : "memory");
+        }
+        if (p.mode != kLayerRouteOnly) {
+            for (int e = lane; e < E; e += 32) s_ptab[e] = rp.blobs[e];
+            refresh_tmaps(rp, cta * 32 + lane, G * 32);
+            build_x_pieces(rp.x, Tc, d, rp.ws, L, cta, G, rp.has_shared != 0, p.norm_w, s_rn);
+            __syncwarp();
+            if (lane == 0) red_add_release(&hdr->prep_done, 1u);
+        }
     }
 
-    if (warp < 4 || warp == 10) {
+    if ((warp < 4 || warp == 10) && !(p.mode == kLayerRouteOnly && cta != 0)) {
         // top-k of the tokens, warps 0-3 and 10 (160 threads) once every
-        // router row is in
+        // router row is in (or the routing a route-only launch left)
         const int tw = warp == 10 ? 4 : warp;
         int ok = 1;
-        if (lane == 0) {
+        if (p.mode == kLayerRouted) {
+            const int32_t *gi = reinterpret_cast<const int32_t *>(rp.ws + L.idx);
+            const float *gw = reinterpret_cast<const float *>(rp.ws + L.wt);
+            for (int t = tw; t < Tc; t += kLTopkWarps)
+                if (lane < k) {
+                    s_tidx[t * 32 + lane] = __ldcg(gi + t * k + lane);
+                    s_tw[t * 32 + lane] = __ldcg(gw + t * k + lane);
+                }
+        } else if (lane == 0) {
             const uint64_t t0 = globaltimer();
             while (ld_acquire(&hdr->router_done) < (uint32_t)E) {
                 if (*s_abort || globaltimer() - t0 > rp.wait_ns) {
@@ -381,14 +418,23 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
             }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (ok) {
+        if (ok && p.mode != kLayerRouted) {
             const float *logits = reinterpret_cast<const float *>(rp.ws + L.logits);
             for (int t = tw; t < Tc; t += kLTopkWarps)
                 warp_topk(logits + (size_t)t * E, E, k, s_tidx + t * 32, s_tw + t * 32,
                           (rp.route_flags & kRouteBiasSelect) ? rp.bias : nullptr, (rp.route_flags & kRouteRenorm) != 0);
         }
         umma::bar_sync(3, 32 * kLTopkWarps);
-        if (warp == 10 && ok && !*s_abort) {
+        if (warp == 10 && ok && !*s_abort && p.mode == kLayerRouteOnly) {
+            // route only: the picks into the workspace (and the caller's copies)
+            for (int i = lane; i < Tc * k; i += 32) {
+                const int t = i / k, j = i - t * k;
+                reinterpret_cast<int32_t *>(rp.ws + L.idx)[i] = s_tidx[t * 32 + j];
+                reinterpret_cast<float *>(rp.ws + L.wt)[i] = s_tw[t * 32 + j];
+                if (rp.idx_out) rp.idx_out[i] = s_tidx[t * 32 + j];
+                if (rp.w_out) rp.w_out[i] = s_tw[t * 32 + j];
+            }
+        } else if (warp == 10 && ok && !*s_abort) {
             // dispatch: distinct experts in ascending id (bitmap + prefix),
             // each one's blob (checked) and per-token weight
             uint32_t *bitmap = s_misc, *prefix = s_misc + 32;
@@ -611,9 +657,19 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
         const int row_base = R0.a < R0.b ? (int)(f_lo / d) : 0;
         const int nrows = R0.a < R0.b ? (int)((f_hi - 1) / d) - row_base + 1 : 0;
         for (int q = tid; q < kRMaxRows * Tc; q += 128) s_racc[q] = 0.f;
-        umma::bar_sync(2, 128);
-        int i = 0;
         bool go = true;
+        if (p.norm_w) {
+            // the router reads x = RMSNorm(h): wait for the tokens' 1 / rms
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait_bounded(rnready, 0u, hdr, rp.wait_ns) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (ok) (void)mbar_try_wait(rnready, 0u);
+            go = umma::bar_red_and(2, 128, ok != 0);
+            if (!go) *s_abort = 1;
+        } else {
+            umma::bar_sync(2, 128);
+        }
+        int i = 0;
         bool act_ok[2] = {false, false};  // x pieces' scales / h pieces' scales seen (no-TMA path)
         for (int r = 0; r < 4 && go; ++r) {
             if (r == 2 && !routed_ranges(true)) break;
@@ -653,10 +709,20 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                         for (int q = 0; q < 16; ++q) {
                             const int jq = (q + lane) & 15;
                             const float4 a = w4[jq];
+                            uint2 gn = make_uint2(0u, 0u);
+                            if (p.norm_w) gn = __ldg(reinterpret_cast<const uint2 *>(p.norm_w + col) + jq);
 #pragma unroll
                             for (int t = 0; t < kChunk; ++t) {
                                 if (t < Tc) {
-                                    const uint2 xw = __ldg(reinterpret_cast<const uint2 *>(rp.x + (size_t)t * d + col) + jq);
+                                    uint2 xw = __ldg(reinterpret_cast<const uint2 *>(rp.x + (size_t)t * d + col) + jq);
+                                    if (p.norm_w) {
+                                        // x = RMSNorm(h), element by element
+                                        const float rt = s_rn[t];
+                                        xw.x = (uint32_t)rms_norm_bf16((uint16_t)(xw.x & 0xFFFFu), rt, (uint16_t)(gn.x & 0xFFFFu)) |
+                                               ((uint32_t)rms_norm_bf16((uint16_t)(xw.x >> 16), rt, (uint16_t)(gn.x >> 16)) << 16);
+                                        xw.y = (uint32_t)rms_norm_bf16((uint16_t)(xw.y & 0xFFFFu), rt, (uint16_t)(gn.y & 0xFFFFu)) |
+                                               ((uint32_t)rms_norm_bf16((uint16_t)(xw.y >> 16), rt, (uint16_t)(gn.y >> 16)) << 16);
+                                    }
                                     v[t] = fmaf(a.x, bf16_lo(xw.x), v[t]);
                                     v[t] = fmaf(a.y, bf16_hi(xw.x), v[t]);
                                     v[t] = fmaf(a.z, bf16_lo(xw.y), v[t]);
@@ -1058,7 +1124,8 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
 #pragma unroll
                             for (int t = 0; t < kChunk; ++t) {
                                 if (t < Tc) {
-                                    const float yv = acc[0][t];
+                                    float yv = acc[0][t];
+                                    if (p.resid) yv += __uint_as_float((uint32_t)p.resid[(size_t)t * d + row] << 16);
                                     if (p.out_fp32)
                                         reinterpret_cast<float *>(p.y)[(size_t)t * d + row] = yv;
                                     else

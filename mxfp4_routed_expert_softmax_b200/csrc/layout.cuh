@@ -150,6 +150,7 @@ struct PLayout {
     size_t hsf;    // u32 [ngr][nkt_ff][2][kPfN] their scales (word = 4 blocks of one row)
     size_t hsb;    // u8 [ngs][nkts_ff][kPfNsDn*128] shared h as bf16 high (rows 0-31), low (32-63)
     size_t o;      // f32 [Tp][k+1][d] expert outputs per (token, slot); slot k: shared
+    size_t xn;     // bf16 [Tp][d] the layer's input RMSNorm(h) (pre-norm calls)
     size_t total;  // end offset (absolute: the prefill region follows the decode layout)
     int Tp, ngr, ngs, nhb;
 };
@@ -194,6 +195,7 @@ __host__ __device__ inline PLayout make_playout(size_t base, int d, int ff, int 
     take(P.hsf, (size_t)P.ngr * nkt_ff * 2 * kPfN * 4);
     take(P.hsb, (size_t)P.ngs * nkts_ff * kPfNsDn * 128);
     take(P.o, (size_t)Tp * (k + 1) * d * 4);
+    take(P.xn, (size_t)Tp * d * 2);
     P.total = o;
     return P;
 }

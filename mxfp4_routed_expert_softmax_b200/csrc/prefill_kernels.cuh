@@ -357,13 +357,34 @@ __global__ void __launch_bounds__(kRouteThreads) pf_prep_kernel(const __grid_con
     }
 }
 
+// ------------------------------------------------------------- pre-norm --
+// xn[t] = RMSNorm(h[t]) rounded to bf16, one warp per token (the same
+// per-token arithmetic as the decode kernel's).
+struct PfNormParams {
+    const uint16_t *h;       // bf16 [T][d]
+    const uint16_t *norm_w;  // bf16 [d]
+    float eps;
+    int T, d;
+    uint16_t *xn;            // bf16 [T][d]
+};
+__global__ void pf_rmsnorm_kernel(const __grid_constant__ PfNormParams p) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= p.T) return;
+    const uint16_t *h = p.h + (size_t)t * p.d;
+    const float r = warp_rms_inv(h, p.d, p.eps);
+    for (int j = lane; j < p.d; j += 32) p.xn[(size_t)t * p.d + j] = rms_norm_bf16(h[j], r, p.norm_w[j]);
+}
+
 // -------------------------------------------------------------- combine --
 // y[t] = sum_j o[t][j] (j < k, routing weights already applied) + o[t][k]
-// (the shared expert), in that order, rounded once.
+// (the shared expert), in that order (+ the residual h[t] for pre-norm
+// calls), rounded once.
 struct PfCombineParams {
     const float *o;      // [T][k+1][d]
     int T, d, k, has_shared, out_fp32;
     void *y;             // [T][d]
+    const uint16_t *resid;  // bf16 [T][d] or null
 };
 
 __global__ void pf_combine_kernel(const __grid_constant__ PfCombineParams p) {
@@ -380,6 +401,13 @@ __global__ void pf_combine_kernel(const __grid_constant__ PfCombineParams p) {
             s.y += v.y;
             s.z += v.z;
             s.w += v.w;
+        }
+        if (p.resid) {
+            const uint2 hv = *reinterpret_cast<const uint2 *>(p.resid + 4 * i);
+            s.x += bf16_lo(hv.x);
+            s.y += bf16_hi(hv.x);
+            s.z += bf16_lo(hv.y);
+            s.w += bf16_hi(hv.y);
         }
         if (p.out_fp32) {
             reinterpret_cast<float4 *>(p.y)[i] = s;

@@ -132,14 +132,16 @@ __device__ __forceinline__ void quantize_pieces(float v, int lane, int t, int c,
 // x of the chunk -> pieces (routed gate/up B operand) and, with a shared
 // expert, x as bf16 in rows t*kPieces of the shared gate/up B operand (the
 // other piece rows zero).  Blocks spread over every warp of the grid (warp
-// index gw of nw).
+// index gw of nw).  norm_w (non-null): x is RMSNorm(h) of the given tokens,
+// x_j = RNE_bf16((h_j * rnorm[t]) * norm_w[j]).
 __device__ void build_x_pieces(const uint16_t *x, int Tc, int d, uint8_t *ws, const Layout &L, int gw, int nw,
-                               bool shared) {
+                               bool shared, const uint16_t *norm_w = nullptr, const float *rnorm = nullptr) {
     const int lane = threadIdx.x & 31, N = act_n(Tc), nb = d / 32;
     for (int i = gw; i < Tc * nb; i += nw) {
         const int t = i / nb, b = i - t * nb;
         const int col = 32 * b + lane;
-        const uint16_t xv = x[(size_t)t * d + col];
+        uint16_t xv = x[(size_t)t * d + col];
+        if (norm_w) xv = rms_norm_bf16(xv, rnorm[t], norm_w[col]);
         const float v = __uint_as_float((uint32_t)xv << 16);
         const int kt = b >> 3;
         quantize_pieces(v, lane, t, b & 7, N, ws + L.xb + (size_t)kt * N * 128,

@@ -64,6 +64,8 @@ def load(path: str | None = None):
     lib.oracle_route.argtypes = [vp, i64, vp, vp, i64, i64, i64, vp, vp, vp, vp]
     lib.oracle_route_variant.argtypes = [vp, i64, vp, vp, i64, i64, i64, ctypes.c_int, ctypes.c_int,
                                          vp, vp, vp, vp]
+    lib.oracle_rmsnorm.argtypes = [vp, i64, vp, dbl, i64, vp]
+    lib.oracle_residual_add.argtypes = [vp, i64, i64, vp, vp]
     lib.oracle_expert_ffn_vec.argtypes = [vp, vp, i64, i64, vp]
     lib.oracle_expert_ffn.argtypes = [vp, i64, vp, i64, i64, vp]
     lib.oracle_shared_ffn.argtypes = [vp, i64, vp, vp, vp, i64, i64, vp]
@@ -72,7 +74,7 @@ def load(path: str | None = None):
                                  vp, vp, vp]
     for name in ("oracle_mxfp4_matvec", "oracle_bf16_matvec", "oracle_router_logits",
                  "oracle_softmax", "oracle_topk", "oracle_route", "oracle_route_variant",
-                 "oracle_expert_ffn_vec",
+                 "oracle_rmsnorm", "oracle_residual_add", "oracle_expert_ffn_vec",
                  "oracle_expert_ffn", "oracle_shared_ffn", "oracle_combine", "oracle_layer"):
         getattr(lib, name).restype = None
     if path is None:
@@ -190,6 +192,23 @@ class Oracle:
                                       int(bool(bias_select_only)), _p(logits), _p(probs), _p(idx),
                                       _p(weight))
         return logits, probs, idx, weight
+
+    def rmsnorm(self, h, g, eps) -> np.ndarray:
+        """x = RNE_bf16(h * g / sqrt(mean(h^2) + eps)) per token: bf16 bits [T, d]."""
+        h, g = _bf(h), _bf(g)
+        T, d = h.shape
+        out = np.empty((T, d), dtype=np.uint16)
+        self.lib.oracle_rmsnorm(_p(h), T, _p(g), float(eps), d, _p(out))
+        return out
+
+    def residual_add(self, h, y) -> np.ndarray:
+        """h (bf16 bits) + y (fp64), fp64."""
+        h = _bf(h)
+        T, d = h.shape
+        y = np.ascontiguousarray(y, dtype=np.float64)
+        out = np.empty((T, d), dtype=np.float64)
+        self.lib.oracle_residual_add(_p(h), T, d, _p(y), _p(out))
+        return out
 
     def expert_ffn(self, x, blob, d, ff) -> np.ndarray:
         x = _bf(x)

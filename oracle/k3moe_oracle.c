@@ -294,6 +294,35 @@ void oracle_combine(const uint16_t *x, int64_t T, const double *weight, int64_t 
     free(xv);
 }
 
+/*
+ * The steps on either side of the layer in a pre-norm transformer block (the
+ * kimi-k3-in-c project card names RMSNorm among its k3_ops.c kernels and the
+ * dense trunk's normalisation parameters; the pages give no formula, so the
+ * standard one is taken):
+ *   x_j = RNE_bf16( h_j g_j / sqrt(mean_j h_j^2 + eps) )   (the layer's input)
+ *   out = h + y                                            (the residual add)
+ * h, g bf16; the norm in fp64, rounded once to bf16 (the layer takes bf16).
+ */
+void oracle_rmsnorm(const uint16_t *h, int64_t T, const uint16_t *g, double eps, int64_t d,
+                    uint16_t *x_out) {
+    for (int64_t t = 0; t < T; ++t) {
+        double ss = 0.0;
+        for (int64_t j = 0; j < d; ++j) {
+            const double v = oracle_bf16_value(h[t * d + j]);
+            ss += v * v;
+        }
+        const double r = 1.0 / sqrt(ss / (double)d + eps);
+        for (int64_t j = 0; j < d; ++j)
+            x_out[t * d + j] =
+                oracle_bf16_rne(oracle_bf16_value(h[t * d + j]) * r * oracle_bf16_value(g[j]));
+    }
+}
+
+/* out[t][j] = h[t][j] + y[t][j] in fp64 */
+void oracle_residual_add(const uint16_t *h, int64_t T, int64_t d, const double *y, double *out) {
+    for (int64_t i = 0; i < T * d; ++i) out[i] = oracle_bf16_value(h[i]) + y[i];
+}
+
 /* the whole layer; blobs[e] is expert e's blob (all E present) */
 void oracle_layer(const uint16_t *x, int64_t T, const float *w_router, const float *bias,
                   const uint8_t *const *blobs, const uint16_t *wg, const uint16_t *wu,

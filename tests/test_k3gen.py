@@ -91,3 +91,15 @@ def test_blob_layout_sizes():
         for o in offs:
             assert o % 16 == 0
     assert k3gen.CONFIGS["k3_decode"].blob_bytes == 17547264
+
+
+def test_norm_weights_stream():
+    """RMSNorm weights: bf16(1 + 0.1 N(0,1)) from stream 7, deterministic."""
+    cfg = k3gen.CONFIGS["tiny"]
+    g = k3gen.norm_weights(cfg)
+    assert g.dtype == np.uint16 and g.shape == (cfg.d,)
+    assert np.array_equal(g, k3gen.norm_weights(cfg))
+    v = k3gen.bf16_to_f32(g).astype(np.float64)
+    assert abs(v.mean() - 1.0) < 0.03 and 0.07 < v.std() < 0.13
+    n = k3gen.normal(0, k3gen.STREAM_NORM, 0, 4)
+    assert [int(b) for b in g[:4]] == [k3gen.bf16_bits(1.0 + 0.1 * z) for z in n]

@@ -472,3 +472,51 @@ def test_route_variants_invariants(orc):
     unb = np.exp(l5 - l5.max(1, keepdims=True))
     unb /= unb.sum(1, keepdims=True)
     assert np.allclose(w5, np.take_along_axis(unb, i5.astype(np.int64), 1), rtol=1e-13)
+
+
+# --------------------------------------------- RMSNorm and the residual add --
+
+def _bf16_row(vals):
+    return np.array([[k3gen.bf16_bits(v) for v in vals]], dtype=np.uint16)
+
+
+def test_rmsnorm_worked_example(orc):
+    """h = (3, 4), g = (1, 0.5), eps = 0: mean h^2 = 12.5, so x = (3, 2) / sqrt(12.5)
+    rounded to bf16 (the generator's own nearest-even rounding)."""
+    h = _bf16_row([3.0, 4.0])
+    g = np.array([k3gen.bf16_bits(1.0), k3gen.bf16_bits(0.5)], dtype=np.uint16)
+    x = orc.rmsnorm(h, g, 0.0)
+    r = 1.0 / math.sqrt(12.5)
+    assert x[0].tolist() == [k3gen.bf16_bits(3.0 * r), k3gen.bf16_bits(2.0 * r)]
+
+
+def test_rmsnorm_constant_token_gives_the_weights(orc):
+    """h_j = c for all j, eps = 0: x_j = sign(c) g_j exactly."""
+    rng = np.random.default_rng(3)
+    g = np.array([k3gen.bf16_bits(v) for v in rng.standard_normal(64)], dtype=np.uint16)
+    for c in (0.75, -3.0, 1024.0):
+        x = orc.rmsnorm(_bf16_row([c] * 64), g, 0.0)
+        want = g if c > 0 else (g ^ 0x8000)
+        assert np.array_equal(x[0], want)
+
+
+def test_rmsnorm_scale_invariance_and_eps(orc):
+    """Scaling a token by a power of two leaves its norm unchanged (eps = 0);
+    eps pulls a small token towards zero."""
+    rng = np.random.default_rng(4)
+    h = np.array([[k3gen.bf16_bits(v) for v in rng.standard_normal(128)]], dtype=np.uint16)
+    g = np.array([k3gen.bf16_bits(v) for v in 1 + 0.1 * rng.standard_normal(128)], dtype=np.uint16)
+    hf = k3gen.bf16_to_f32(h).astype(np.float64)
+    h8 = np.array([[k3gen.bf16_bits(v) for v in hf[0] * 8.0]], dtype=np.uint16)
+    assert np.array_equal(orc.rmsnorm(h, g, 0.0), orc.rmsnorm(h8, g, 0.0))
+    small = np.array([[k3gen.bf16_bits(v) for v in hf[0] * 1e-3]], dtype=np.uint16)
+    a = k3gen.bf16_to_f32(orc.rmsnorm(small, g, 0.0)).astype(np.float64)
+    b = k3gen.bf16_to_f32(orc.rmsnorm(small, g, 1e-4)).astype(np.float64)
+    ms = (hf[0] * 1e-3) ** 2
+    assert np.allclose(b / a, math.sqrt(ms.mean() / (ms.mean() + 1e-4)), rtol=2e-2)
+
+
+def test_residual_add(orc):
+    h = _bf16_row([1.5, -2.0, 0.25])
+    y = np.array([[0.125, 4.0, -0.25]])
+    assert np.array_equal(orc.residual_add(h, y), [[1.625, 2.0, 0.0]])
