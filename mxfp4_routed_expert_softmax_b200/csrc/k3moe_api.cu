@@ -19,6 +19,7 @@
 #include "layer_kernel.cuh"
 #include "layout.cuh"
 #include "prefill_kernels.cuh"
+#include "prefill_router_mma.cuh"
 
 namespace {
 
@@ -89,6 +90,7 @@ k3moe_status device_info(DeviceInfo **out) {
         if (r == cudaSuccess) r = set_smem(pf_expert_kernel<true>, big);
         if (r == cudaSuccess) r = set_smem(pf_expert_kernel<false>, big);
         if (r == cudaSuccess) r = set_smem(layer_kernel, big);
+        if (r == cudaSuccess) r = set_smem(pf_router_mma_kernel, rm_smem_bytes());
         if (r != cudaSuccess) return cuda_fail(r);
         di.ready = true;
     }
@@ -281,6 +283,39 @@ k3moe_status shared_tmaps(int d, int ffs, const void *wg, const void *wu, const 
     return K3MOE_OK;
 }
 
+// A 2-D tensor map of 16-bit elements [rows][cols] (row pitch cols * 2 bytes),
+// boxes of 64 columns x 128 rows with the 128-byte swizzle (the MMA's K-major
+// operand layout).
+k3moe_status tmap_bf16_rows(const void *addr, int cols, int rows, uint4 (&out)[8]) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (q != cudaDriverEntryPointSuccess || !fn) {
+            g_last_error = "cuTensorMapEncodeTiled is not available";
+            return K3MOE_ERR_CUDA;
+        }
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    CUtensorMap m;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kRmKStep, (cuuint32_t)kRmTile};
+    const cuuint32_t es[2] = {1, 1};
+    CUresult r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(addr), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_error = "cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")";
+        return K3MOE_ERR_CUDA;
+    }
+    memcpy(out, &m, sizeof(out));
+    return K3MOE_OK;
+}
+
 template <bool GU>
 cudaError_t launch_umma(const DeviceInfo &di, UmmaParams up, cudaStream_t st) {
     const int N = act_n(up.Tc);
@@ -393,6 +428,24 @@ k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims
     const PLayout P = playout_for(dims, Tp);
     uint8_t *wsb = rp.ws;
     cudaError_t e;
+    // the router as three exact bf16 parts, once per call, and their tensor maps
+    RouterMmaParams rm{};
+    {
+        uint16_t *w1 = reinterpret_cast<uint16_t *>(wsb + P.wsplit);
+        const size_t n = (size_t)E * d;
+        const RouterSplitParams spp{rp.wr, n, w1, w1 + n, w1 + 2 * n};
+        e = launch(pf_router_split_kernel, dim3(4 * di.sms), dim3(256), 0, st, false, spp);
+        if (e != cudaSuccess) return cuda_fail(e, "router split launch");
+        for (int q = 0; q < 3; ++q) {
+            k3moe_status s = tmap_bf16_rows(w1 + q * n, d, E, rm.tw[q]);
+            if (s != K3MOE_OK) return s;
+        }
+        rm.bias = (rp.route_flags & kRouteBiasSelect) ? nullptr : rp.bias;
+        rm.d = d;
+        rm.E = E;
+        rm.ws = wsb;
+        rm.wait_ns = wait_limit();
+    }
     for (int t0 = 0; t0 < T; t0 += Tp) {
         const int Tq = (T - t0) < Tp ? (T - t0) : Tp;
         const uint16_t *xq = x + (size_t)t0 * d;
@@ -413,29 +466,16 @@ k3moe_status prefill_impl(DeviceInfo &di, RouteParams rp, const k3moe_dims *dims
         pp.ngs = ffs > 0 ? ceil_div(Tq, kGroup) : 0;
         pp.ff = dims->ff;
         pp.ffs = ffs;
-        // router: split K until the grid covers the GPU twice; the split
-        // partials go where the expert outputs go later (not in use yet)
-        PfRouterParams rr{};
-        rr.x = pp.r.x;
-        rr.wr = rp.wr;
-        rr.bias = (rp.route_flags & kRouteBiasSelect) ? nullptr : rp.bias;  // in the logits or not
-        rr.T = Tq;
-        rr.d = d;
-        rr.E = E;
-        const int gx = ceil_div(E, kPrBM), gy = ceil_div(Tq, kPrBN);
-        int ns = (2 * di.sms + gx * gy - 1) / (gx * gy);
-        if (ns > 8) ns = 8;
-        if (ns > d / 256) ns = d / 256;
-        if (ns < 1) ns = 1;
-        while (ns > 1 && (size_t)ns * Tq * E * 4 > P.total - P.o) --ns;
-        rr.nsplit = ns;
-        rr.out = reinterpret_cast<float *>(wsb + (ns > 1 ? P.o : P.lg));
-        e = launch(pf_router_kernel, dim3(gx, gy, ns), dim3(kPrThreads), 0, st, false, rr);
-        if (e != cudaSuccess) return cuda_fail(e, "prefill router launch");
-        if (ns > 1) {
-            const PfRouterSumParams sp{rr.out, ns, rr.bias, Tq, E, reinterpret_cast<float *>(wsb + P.lg)};
-            e = launch(pf_router_sum_kernel, dim3(4 * di.sms), dim3(256), 0, st, false, sp);
-            if (e != cudaSuccess) return cuda_fail(e, "prefill router sum launch");
+        // router: tiles of 128 experts x 128 tokens on the tensor cores
+        {
+            k3moe_status s = tmap_bf16_rows(pp.r.x, d, Tq, rm.tx);
+            if (s != K3MOE_OK) return s;
+            rm.T = Tq;
+            rm.out = reinterpret_cast<float *>(wsb + P.lg);
+            const int tiles = ceil_div(E, kRmTile) * ceil_div(Tq, kRmTile);
+            e = launch(pf_router_mma_kernel, dim3(tiles < di.sms ? tiles : di.sms), dim3(kRmThreads), rm_smem_bytes(),
+                       st, false, rm);
+            if (e != cudaSuccess) return cuda_fail(e, "prefill router launch");
         }
         e = launch(pf_topk_kernel, dim3(Tq), dim3(kRouteThreads), 0, st, false, pp);
         if (e != cudaSuccess) return cuda_fail(e, "prefill top-k launch");
@@ -615,6 +655,7 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         rp.ws = wsb;
         rp.L = L;
         rp.blobs = expert_blobs;
+        rp.route_flags = route_flags(dims);
         rp.idx_out = idx_out ? idx_out + (size_t)c0 * dims->top_k : nullptr;
         rp.w_out = w_out ? w_out + (size_t)c0 * dims->top_k : nullptr;
         memcpy(rp.tmpl, tmpl, sizeof(tmpl));

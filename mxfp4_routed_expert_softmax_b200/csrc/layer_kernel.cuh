@@ -500,6 +500,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
             // activations were not ready yet (at most nst, in stage order)
             int pend_s[8], pend_unit[8];
             int npend = 0;
+            const uint8_t *acq_maps = nullptr, *acq_sc = nullptr;  // last tensor maps acquired
             auto issue_b = [&](int s, const Unit &x) {
                 uint8_t *st = smem + s * SB;
                 // the B scale words travel with the stage when the A scales do
@@ -595,10 +596,15 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                     if (sf_dma) tx += (uint32_t)((x.kind == 2 ? 2 : 1) * 2048 + nb * 2 * kSfRow * 4);
                     mbar_arrive_expect_tx(&full[s], tx);
                     if (blob_ok) {
-                        umma::tmap_acquire(maps);
+                        // the maps were written through the generic proxy (this
+                        // launch or an earlier one): one acquire per map and CTA
+                        if (maps != acq_maps) {
+                            umma::tmap_acquire(maps);
+                            if (x.kind <= 2) umma::tmap_acquire(maps + 128);
+                            acq_maps = maps;
+                        }
                         if (x.kind <= 2) {
                             // gate/up: W_g box and W_u box of K-tile kt (128 bytes of every row)
-                            umma::tmap_acquire(maps + 128);
                             umma::tma_load_2d(st, maps, x.kt * 128, x.rb * kTileM, &full[s]);
                             umma::tma_load_2d(st + kAtile, maps + 128, x.kt * 128, x.rb * kTileM, &full[s]);
                         } else {
@@ -607,10 +613,13 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                         }
                         if (sf_dma) {
                             uint8_t *sfa = st + lk_sfa_off(N);
-                            umma::tmap_acquire(scmaps);
+                            if (scmaps != acq_sc) {
+                                umma::tmap_acquire(scmaps);
+                                if (x.kind == 2) umma::tmap_acquire(scmaps + 128);
+                                acq_sc = scmaps;
+                            }
                             umma::tma_load_2d(sfa, scmaps, (x.kt >> 1) * 16, x.rb * kTileM, &full[s]);
                             if (x.kind == 2) {
-                                umma::tmap_acquire(scmaps + 128);
                                 umma::tma_load_2d(sfa + 2048, scmaps + 128, (x.kt >> 1) * 16, x.rb * kTileM, &full[s]);
                             }
                         }
@@ -701,33 +710,58 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                     if (f < f_hi) {
                         row = (int)(f / d);
                         const int col = (int)(f - (long long)row * d);
-                        // the 16 float4 of this thread's 64 floats, starting at
-                        // (lane mod 16) so that a warp's loads spread over the
-                        // banks; each product is exact, each sum fp32 in this order
+                        // This thread's 64 columns of x for a token: eight
+                        // 16-byte loads issued together, chunk (q + lane) mod 8
+                        // into register q, so the weight reads below (the same
+                        // rotated order) spread over the shared-memory banks
+                        // and every register index stays static; the next
+                        // token's loads are in flight while this one's FMAs run.
+                        // Each product is exact; each sum fp32 in this order.
                         const float4 *w4 = reinterpret_cast<const float4 *>(st) + tid * 16;
+                        auto load_x = [&](int t, uint4 (&xr)[8]) {
+                            const uint4 *xv = reinterpret_cast<const uint4 *>(rp.x + (size_t)t * d + col);
 #pragma unroll
-                        for (int q = 0; q < 16; ++q) {
-                            const int jq = (q + lane) & 15;
-                            const float4 a = w4[jq];
-                            uint2 gn = make_uint2(0u, 0u);
-                            if (p.norm_w) gn = __ldg(reinterpret_cast<const uint2 *>(p.norm_w + col) + jq);
+                            for (int q = 0; q < 8; ++q) xr[q] = __ldg(xv + ((q + lane) & 7));
+                            if (p.norm_w) {
+                                // x = RMSNorm(h), element by element
+                                const uint4 *gv = reinterpret_cast<const uint4 *>(p.norm_w + col);
+                                const float rt = s_rn[t];
 #pragma unroll
-                            for (int t = 0; t < kChunk; ++t) {
-                                if (t < Tc) {
-                                    uint2 xw = __ldg(reinterpret_cast<const uint2 *>(rp.x + (size_t)t * d + col) + jq);
-                                    if (p.norm_w) {
-                                        // x = RMSNorm(h), element by element
-                                        const float rt = s_rn[t];
-                                        xw.x = (uint32_t)rms_norm_bf16((uint16_t)(xw.x & 0xFFFFu), rt, (uint16_t)(gn.x & 0xFFFFu)) |
-                                               ((uint32_t)rms_norm_bf16((uint16_t)(xw.x >> 16), rt, (uint16_t)(gn.x >> 16)) << 16);
-                                        xw.y = (uint32_t)rms_norm_bf16((uint16_t)(xw.y & 0xFFFFu), rt, (uint16_t)(gn.y & 0xFFFFu)) |
-                                               ((uint32_t)rms_norm_bf16((uint16_t)(xw.y >> 16), rt, (uint16_t)(gn.y >> 16)) << 16);
-                                    }
-                                    v[t] = fmaf(a.x, bf16_lo(xw.x), v[t]);
-                                    v[t] = fmaf(a.y, bf16_hi(xw.x), v[t]);
-                                    v[t] = fmaf(a.z, bf16_lo(xw.y), v[t]);
-                                    v[t] = fmaf(a.w, bf16_hi(xw.y), v[t]);
+                                for (int q = 0; q < 8; ++q) {
+                                    const uint4 g = __ldg(gv + ((q + lane) & 7));
+                                    uint32_t *xw = reinterpret_cast<uint32_t *>(&xr[q]);
+                                    const uint32_t *gw = reinterpret_cast<const uint32_t *>(&g);
+#pragma unroll
+                                    for (int h = 0; h < 4; ++h)
+                                        xw[h] = (uint32_t)rms_norm_bf16((uint16_t)(xw[h] & 0xFFFFu), rt, (uint16_t)(gw[h] & 0xFFFFu)) |
+                                                ((uint32_t)rms_norm_bf16((uint16_t)(xw[h] >> 16), rt, (uint16_t)(gw[h] >> 16)) << 16);
                                 }
+                            }
+                        };
+                        auto dot = [&](const uint4 (&xr)[8]) {
+                            float acc = 0.f;
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const int jq = (q + lane) & 7;
+                                const float4 a = w4[2 * jq], b = w4[2 * jq + 1];
+                                acc = fmaf(a.x, bf16_lo(xr[q].x), acc);
+                                acc = fmaf(a.y, bf16_hi(xr[q].x), acc);
+                                acc = fmaf(a.z, bf16_lo(xr[q].y), acc);
+                                acc = fmaf(a.w, bf16_hi(xr[q].y), acc);
+                                acc = fmaf(b.x, bf16_lo(xr[q].z), acc);
+                                acc = fmaf(b.y, bf16_hi(xr[q].z), acc);
+                                acc = fmaf(b.z, bf16_lo(xr[q].w), acc);
+                                acc = fmaf(b.w, bf16_hi(xr[q].w), acc);
+                            }
+                            return acc;
+                        };
+                        uint4 xa[8], xb[8];
+                        load_x(0, xa);
+#pragma unroll
+                        for (int t = 0; t < kChunk; ++t) {
+                            if (t < Tc) {
+                                if (t + 1 < Tc) load_x(t + 1, (t & 1) ? xa : xb);
+                                v[t] = dot((t & 1) ? xb : xa);
                             }
                         }
                     }
@@ -843,9 +877,12 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                         umma::wait_st();
                     }
                     umma::fence_before();
+                    // sfr counts the stage's matrix units only: the MMA warp
+                    // never waits on a router unit, so a phase it does not
+                    // track could let a parity wait pass early
+                    __syncwarp();
+                    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sfr[s])) : "memory");
                 }
-                __syncwarp();
-                if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sfr[s])) : "memory");
             }
             if (r == 0) {
                 // the slice's rows: finished here, or (cut by a CTA boundary)
@@ -900,11 +937,15 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
             const uint32_t idesc4 = umma::idesc_mxf4(N), idesc16 = umma::idesc_bf16(N);
             const uint32_t id4[2] = {umma::idesc_sf_id(idesc4, 0u), umma::idesc_sf_id(idesc4, 2u)};
             int i = 0, seg = 0;
+            // router units (the first n0 of the ring) are consumed by the
+            // scale warps and do not complete sfr: stage s's matrix use
+            // number is its use number minus its router uses
+            const int n0 = rg[0].b - rg[0].a;
             for (int r = 0; r < 4 && !*s_abort; ++r) {
                 if (r == 2 && !routed_ranges(false)) break;
                 const Range R = rg[r];
                 if (r == 0) {
-                    i += R.b - R.a;  // router units are consumed by the scale warps
+                    i += n0;
                     continue;
                 }
                 for (int unit = R.a; unit < R.b && !*s_abort; ++seg) {
@@ -919,7 +960,12 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                         if (un != unit) x = decode(r, un);
                         const int s = i % nst;
                         const uint32_t ph = (uint32_t)((i / nst) & 1);
-                        if (!wait(&full[s], ph) || !wait(&sfr[s], ph)) break;
+                        const int r0s = n0 > s ? (n0 - 1 - s) / nst + 1 : 0;
+                        const uint32_t phs = (uint32_t)(((i / nst) - r0s) & 1);
+                        // sfr first: the scale warps arrive on it only after
+                        // this use's bytes landed, so full is then at most
+                        // this use's phase ahead and its parity wait is exact
+                        if (!wait(&sfr[s], phs) || !wait(&full[s], ph)) break;
                         umma::fence_after();
                         const uint32_t soff = (uint32_t)(s * SB) >> 4;
                         const uint64_t a0 = adesc0 + soff, b0 = bdesc0 + soff;

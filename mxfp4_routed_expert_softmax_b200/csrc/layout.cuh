@@ -151,6 +151,7 @@ struct PLayout {
     size_t hsb;    // u8 [ngs][nkts_ff][kPfNsDn*128] shared h as bf16 high (rows 0-31), low (32-63)
     size_t o;      // f32 [Tp][k+1][d] expert outputs per (token, slot); slot k: shared
     size_t xn;     // bf16 [Tp][d] the layer's input RMSNorm(h) (pre-norm calls)
+    size_t wsplit; // bf16 [3][E][d] the router split into three exact bf16 parts
     size_t total;  // end offset (absolute: the prefill region follows the decode layout)
     int Tp, ngr, ngs, nhb;
 };
@@ -196,6 +197,7 @@ __host__ __device__ inline PLayout make_playout(size_t base, int d, int ff, int 
     take(P.hsb, (size_t)P.ngs * nkts_ff * kPfNsDn * 128);
     take(P.o, (size_t)Tp * (k + 1) * d * 4);
     take(P.xn, (size_t)Tp * d * 2);
+    take(P.wsplit, (size_t)3 * E * d * 2);
     P.total = o;
     return P;
 }

@@ -30,11 +30,11 @@ int main(int argc, char **argv) {
     if (Tp > 0) {
         const PLayout P = make_playout(L.total, d, ff, E, k, ffs, Tp);
         const size_t pv[] = {P.lg, P.idx, P.wt, P.hist, P.ecnt, P.eoff, P.goff, P.perm, P.pw, P.grp, P.itg, P.itd,
-                             P.ploc, P.xg, P.xgs, P.xbf, P.hb, P.hsf, P.hsb, P.o, P.total};
+                             P.ploc, P.xg, P.xgs, P.xbf, P.hb, P.hsf, P.hsb, P.o, P.xn, P.total};
         const char *pn[] = {"lg", "idx", "wt", "hist", "ecnt", "eoff", "goff", "perm", "pw", "grp", "itg", "itd",
-                            "ploc", "xg", "xgs", "xbf", "hb", "hsf", "hsb", "o", "total"};
+                            "ploc", "xg", "xgs", "xbf", "hb", "hsf", "hsb", "o", "xn", "total"};
         printf(", \"prefill\": {");
-        for (int i = 0; i < 21; ++i) printf("%s\"%s\": %zu", i ? ", " : "", pn[i], pv[i]);
+        for (int i = 0; i < 22; ++i) printf("%s\"%s\": %zu", i ? ", " : "", pn[i], pv[i]);
         printf(", \"ngr\": %d, \"ngs\": %d}", P.ngr, P.ngs);
     }
     printf("}\n");

@@ -38,6 +38,19 @@ MUTANTS = {
                            "s += oracle_bf16_value(x[j]) * (double)w[e * d + j];"),
     "down_scale_rows": ("oracle_mxfp4_matvec(p[4], p[5], d, ff, g, out);",
                         "oracle_mxfp4_matvec(p[4], p[3], d, ff, g, out);"),
+    # routing variants, RMSNorm, residual add
+    "renorm_unscaled": ("weight[t * k + j] = renorm ? pj / z : pj;", "weight[t * k + j] = pj;"),
+    "select_bias_in_softmax": ("oracle_router_logits(x, T, w, bias_select_only ? NULL : bias, d, E, l);",
+                               "oracle_router_logits(x, T, w, bias, d, E, l);"),
+    "select_bias_ignored": ("sel[e] = lt[e] + ((bias_select_only && bias) ? (double)bias[e] : 0.0);",
+                            "sel[e] = lt[e];"),
+    "rmsnorm_sum_not_mean": ("const double r = 1.0 / sqrt(ss / (double)d + eps);",
+                             "const double r = 1.0 / sqrt(ss + eps);"),
+    "rmsnorm_eps_outside": ("const double r = 1.0 / sqrt(ss / (double)d + eps);",
+                            "const double r = 1.0 / sqrt(ss / (double)d) + eps;"),
+    "rmsnorm_no_weight": ("oracle_bf16_rne(oracle_bf16_value(h[t * d + j]) * r * oracle_bf16_value(g[j]));",
+                          "oracle_bf16_rne(oracle_bf16_value(h[t * d + j]) * r);"),
+    "residual_dropped": ("out[i] = oracle_bf16_value(h[i]) + y[i];", "out[i] = y[i];"),
 }
 
 BATTERY = [
@@ -50,6 +63,10 @@ BATTERY = [
     pins.test_bias_shifts_routing,
     lambda o: pins.test_torch_fp64_second_opinion(o, "tiny"),
     lambda o: pins.test_torch_fp64_second_opinion(o, "small_bias"),
+    pins.test_route_variants_closed_forms, pins.test_route_variants_selection_ties_go_to_lower_index,
+    pins.test_route_variants_invariants, pins.test_rmsnorm_worked_example,
+    pins.test_rmsnorm_constant_token_gives_the_weights, pins.test_rmsnorm_scale_invariance_and_eps,
+    pins.test_residual_add,
 ]
 
 

@@ -78,7 +78,13 @@ def check_layer(orc, cfg, W, x_bits, bias_dev, bias_host, flags, tokens=None, ws
                                                  shared=shared)
     assert not problems, problems[:3]
     wref = np.take_along_axis(probs, idx[tokens].astype(np.int64), axis=1)
-    assert np.allclose(w[tokens], wref, rtol=1e-5, atol=1e-7)
+    # the routing weights' relative error follows the fp32 error of the logits,
+    # bounded by 2^-24 log2(d) sum_j |x_j W_r[e, j]| (large with outliers)
+    xa = np.abs(k3gen.bf16_to_f32(x_bits[tokens]).astype(np.float64))
+    wa = np.abs(W.w_router_host.astype(np.float64))
+    lbound = np.array([(xa[i] @ wa[idx[t]].T).max() for i, t in enumerate(tokens)]) * 2.0 ** -24 * np.log2(cfg.d)
+    rtol = np.maximum(1e-5, 4 * lbound)[:, None]
+    assert np.all(np.abs(w[tokens] - wref) <= 1e-7 + rtol * np.abs(wref)), (rtol.max(), np.abs(w[tokens] - wref).max())
     err = g1_error(y[tokens], yo)
     assert err.max() <= G1_TOL, (err.max(), err)
     return err, idx
