@@ -98,12 +98,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Returns false (and sets the timeout bit) when the limit is reached.
 // The clock is read only every 64 polls: the waits sit on the pipelines'
 // critical paths.
+// try_wait that lets the hardware suspend the thread (up to about a
+// microsecond) until the phase completes, instead of returning at once.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(1000u)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, WsHeader *h,
                                                   uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity)) return true;
         if ((i & 63u) == 0u && globaltimer() - t0 > limit_ns) {
             set_status(h, kStTimeout);
             return false;
@@ -141,6 +154,29 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Wait until *ctr >= target: relaxed polls with a short sleep, then one
+// acquire fence (a relaxed read that sees the producers' release, followed by
+// the fence, orders everything they published before this thread's later
+// reads), so the acquire is paid once and not on every poll.  False after
+// limit_ns, or at once when *abort (if given) becomes nonzero.
+__device__ __forceinline__ bool spin_geq(const uint32_t *ctr, uint32_t target, uint64_t limit_ns,
+                                         const volatile int *abort = nullptr) {
+    if (ld_relaxed(ctr) < target) {
+        const uint64_t t0 = globaltimer();
+        do {
+            if ((abort && *abort) || globaltimer() - t0 > limit_ns) return false;
+            __nanosleep(32);
+        } while (ld_relaxed(ctr) < target);
+    }
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    return true;
 }
 
 // ------------------------------------------------- programmatic launches --

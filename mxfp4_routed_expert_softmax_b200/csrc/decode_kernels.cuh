@@ -544,15 +544,9 @@ __device__ void stream_router(const RouteParams &p, WsHeader *hdr, uint8_t *ring
 
 // Wait (bounded) until *ctr reaches target; false (timeout bit set) if not.
 __device__ bool wait_count(const uint32_t *ctr, uint32_t target, WsHeader *hdr, uint64_t limit_ns) {
-    const uint64_t t0 = globaltimer();
-    while (ld_acquire(ctr) < target) {
-        __nanosleep(64);
-        if (globaltimer() - t0 > limit_ns) {
-            set_status(hdr, kStTimeout);
-            return false;
-        }
-    }
-    return true;
+    if (spin_geq(ctr, target, limit_ns)) return true;
+    set_status(hdr, kStTimeout);
+    return false;
 }
 
 // Cooperative launch (every CTA resident), one CTA per SM.  Every CTA

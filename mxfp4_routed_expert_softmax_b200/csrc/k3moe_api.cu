@@ -374,13 +374,13 @@ int layer_stages(const DeviceInfo &di, const k3moe_dims *dm, int Tc) {
     int nst = rest / lk_stage_bytes(N);
     if (nst > 8) nst = 8;
     if (nst < 2) return 0;
-    const long long rf = (long long)dm->n_experts * dm->d;
-    const long long n0 = (rf + kLRUnit - 1) / kLRUnit;
+    if (dm->d > kLRUnit) return 0;  // a router unit holds whole rows
+    const int rpu = lk_rows_per_unit(dm->d);
+    const int n0 = (dm->n_experts + rpu - 1) / rpu;
     const int G = di.sms < kLMaxCtas ? di.sms : kLMaxCtas;
-    const long long g0 = n0 < G ? n0 : G;
-    const long long upc = (n0 + g0 - 1) / g0;  // router units of one CTA at most
-    const long long rows = (upc * kLRUnit + dm->d - 1) / dm->d + 1;
-    if (rows > kRMaxRows) return 0;
+    const int g0 = n0 < G ? n0 : G;
+    const int upc = (n0 + g0 - 1) / g0;  // router units of one CTA at most
+    if (upc * rpu > kRMaxRows) return 0;
     return nst;
 }
 

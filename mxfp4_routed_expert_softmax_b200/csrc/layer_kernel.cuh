@@ -48,10 +48,10 @@ namespace k3 {
 
 constexpr int kLThreads = 352;
 constexpr int kLMaxCtas = 160;        // grid cap (one CTA per SM)
-constexpr int kLRUnit = 8192;         // router floats per R0 unit (32 KB)
+constexpr int kLRUnit = 8192;         // router floats per R0 unit at most (32 KB): whole rows
 constexpr int kLSfc = 32;             // TMEM scale columns per stage
-constexpr int kLSegMax = 32;          // row segments per warp and router unit (d >= 64)
 constexpr int kLTopkWarps = 5;        // warps 0-3 and 10
+constexpr int kTkCand = 128;          // top-k candidates per warp (scratch: keys, then ids)
 
 struct LayerParams {
     RouteParams r;     // x, Tc, router, shapes, workspace, blobs, maps, wait_ns
@@ -86,16 +86,17 @@ __host__ __device__ inline int lk_sfa_off(int N) { return 2 * kAtile + 2 * N * 1
 __host__ __device__ inline int lk_sfb_off(int N) { return lk_sfa_off(N) + 2 * 2048; }
 __host__ __device__ inline int lk_stage_bytes(int N) { return (lk_sfb_off(N) + 2 * 2 * kSfRow * 4 + 1023) & ~1023; }
 
+// Router rows per R0 unit: as many whole rows of d floats as fit in kLRUnit.
+__host__ __device__ inline int lk_rows_per_unit(int d) { return d >= kLRUnit ? 1 : kLRUnit / d; }
+
 // The rest, after the stages (byte offsets from the end of the stages),
 // sized for this pass: E experts, top-k, Tc tokens, hidden size d.
 struct LkSmem {
-    int segs;  // row segments one warp's 2048 router floats can touch
-    int bars, ptab, blob, eid, wu, tidx, tw, racc, segr, segv, segn, misc, rn, total;
+    int bars, ptab, blob, eid, wu, tidx, tw, racc, misc, rn, tk, total;
 };
 __host__ __device__ inline LkSmem lk_smem(int E, int k, int Tc, int d) {
     LkSmem s;
     const int umax = E < Tc * k ? E : Tc * k;
-    s.segs = 2047 / d + 2 < kLSegMax ? 2047 / d + 2 : kLSegMax;
     auto a16 = [](int v) { return (v + 15) & ~15; };
     int o = 0;
     s.bars = o;   o += 512;                           // mbarriers, TMEM slot, flags
@@ -105,12 +106,10 @@ __host__ __device__ inline LkSmem lk_smem(int E, int k, int Tc, int d) {
     s.wu = o;     o += a16(umax * Tc * 4);            //   weight of each token (0: not selected)
     s.tidx = o;   o += Tc * 32 * 4;                   // top-k of each token: experts
     s.tw = o;     o += Tc * 32 * 4;                   //   and weights
-    s.racc = o;   o += a16(kRMaxRows * Tc * 4);       // router row sums of this CTA's slice
-    s.segr = o;   o += a16(2 * 4 * s.segs * 4);       // per-warp row segments of a unit (x2)
-    s.segv = o;   o += a16(2 * 4 * s.segs * Tc * 4);
-    s.segn = o;   o += 2 * 4 * 4;
+    s.racc = o;   o += a16(4 * kRMaxRows * Tc * 4);   // router row sums of this CTA's rows, per warp
     s.misc = o;   o += 64 * 4;                        // dispatch bitmap / prefix
     s.rn = o;     o += kChunk * 4;                    // 1 / rms of each token (pre-norm)
+    s.tk = o;     o += kLTopkWarps * 2 * kTkCand * 4;  // top-k candidates of each top-k warp
     s.total = o;
     return s;
 }
@@ -120,27 +119,32 @@ __host__ __device__ inline int lk_smem_bytes(int N, int nst, int E, int k, int T
 
 // --------------------------------------------------------------- top-k --
 // Softmax over all E logits and the top-k of one token, by one warp.  Lane l
-// holds experts l, l + 32, ...  The k winners come out one per round: the
-// largest key (order-preserving bits of the logit) over every lane's best,
-// the lowest expert id among equal keys, so the picks are in descending
-// logit with ties to the lower index.  Each lane keeps its best and second
-// best candidates: on a win the second becomes the best, so a lane rescans
-// its values only on every other win.  w = exp(l - max) / sum over all E of
-// exp(l_e - max), fp32.  sel_bias (non-null): the selection runs on
-// l + sel_bias[e], the softmax on l; renorm: the k weights are divided by
-// their sum.
-__device__ void warp_topk(const float *row, int E, int k, int32_t *idx_out, float *w_out,
-                          const float *sel_bias, bool renorm) {
+// holds experts l, l + 32, ...  Picks come out in descending key (the
+// order-preserving bits of the logit) with ties to the lower expert id.
+// w = exp(l - max) / sum over all E of exp(l_e - max), fp32.  sel_bias
+// (non-null): the selection runs on l + sel_bias[e], the softmax on l;
+// renorm: the k weights are divided by their sum.
+//
+// Selection: the k-th largest of the 32 lane maxima, L, is a lower bound of
+// the k-th largest key (k lanes hold a key >= L), so only keys >= L can be
+// picked; those candidates (about k plus a few for spread logits) go to the
+// warp's scratch and the k rounds (warp max of the lanes' best candidate,
+// lowest id among equal keys) run over at most four per lane.  More than
+// kTkCand candidates (many equal keys) take the rounds over all keys.
+__device__ __noinline__ void warp_topk(const float *row, int E, int k, int32_t *idx_out, float *w_out,
+                          const float *sel_bias, bool renorm, uint32_t *scratch) {
     const int lane = threadIdx.x & 31;
     constexpr int kPer = 32;  // E <= 1024
     uint32_t key[kPer];
     float mx = -INFINITY;
+    uint32_t lmax = 0u;
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
         const int e = lane + 32 * i;
         const float v = e < E ? __ldcg(row + e) : -INFINITY;
         key[i] = e < E ? fkey(sel_bias ? v + __ldg(sel_bias + e) : v) : 0u;  // real keys are > 0
         mx = fmaxf(mx, v);
+        lmax = max(lmax, key[i]);
     }
     const float m = fkey_value(__reduce_max_sync(0xffffffffu, fkey(mx)));
     // the softmax runs on the logits themselves (read again when the keys
@@ -154,43 +158,88 @@ __device__ void warp_topk(const float *row, int E, int k, int32_t *idx_out, floa
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float inv_s = 1.0f / sum;
-    uint32_t taken = 0u;
-    // best and second best (key, slot) of this lane, first slot on equal keys
-    auto rescan = [&](uint32_t &k1, int &i1, uint32_t &k2, int &i2) {
-        k1 = 0u; i1 = -1; k2 = 0u; i2 = -1;
+
+    // L: the lane maximum of rank k - 1 (larger first, lower lane first)
+    int rank = 0;
+#pragma unroll
+    for (int o = 0; o < 32; ++o) {
+        const uint32_t other = __shfl_sync(0xffffffffu, lmax, o);
+        rank += (other > lmax || (other == lmax && o < lane)) ? 1 : 0;
+    }
+    const uint32_t at = __ballot_sync(0xffffffffu, rank == k - 1);
+    const uint32_t L = __shfl_sync(0xffffffffu, lmax, __ffs(at) - 1);
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) c += key[i] >= L ? 1 : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (total <= kTkCand) {
+        int pos = incl - c;
 #pragma unroll
         for (int i = 0; i < kPer; ++i) {
-            const uint32_t kv = ((taken >> i) & 1u) ? 0u : key[i];
-            if (kv > k1) {
-                k2 = k1; i2 = i1; k1 = kv; i1 = i;
-            } else if (kv > k2) {
-                k2 = kv; i2 = i;
-            }
-        }
-    };
-    uint32_t k1, k2;
-    int i1, i2;
-    rescan(k1, i1, k2, i2);
-    for (int j = 0; j < k; ++j) {
-        const uint32_t K = __reduce_max_sync(0xffffffffu, k1);
-        const uint32_t cand = (k1 == K && i1 >= 0) ? (uint32_t)(lane + 32 * i1) : 0xFFFFFFFFu;
-        const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
-        if (lane == 0) {
-            idx_out[j] = (int32_t)win;
-            w_out[j] = fkey_value(K);  // the pick's key value (its logit when unbiased)
-        }
-        if ((int)(win & 31u) == lane) {
-            taken |= 1u << i1;
-            if (i2 >= 0) {
-                // the second best becomes the best; the lane looks for a new
-                // second only if it wins again
-                k1 = k2; i1 = i2; k2 = 0u; i2 = -1;
-            } else {
-                rescan(k1, i1, k2, i2);
+            if (key[i] >= L) {
+                scratch[pos] = key[i];
+                scratch[kTkCand + pos] = (uint32_t)(lane + 32 * i);
+                ++pos;
             }
         }
         __syncwarp();
+        uint32_t ck[kTkCand / 32], ci[kTkCand / 32];
+#pragma unroll
+        for (int q = 0; q < kTkCand / 32; ++q) {
+            const int j = 32 * q + lane;
+            ck[q] = j < total ? scratch[j] : 0u;
+            ci[q] = j < total ? scratch[kTkCand + j] : 0xFFFFFFFFu;
+        }
+        for (int j = 0; j < k; ++j) {
+            uint32_t bk = 0u, bi = 0xFFFFFFFFu;
+#pragma unroll
+            for (int q = 0; q < kTkCand / 32; ++q) {
+                if (ck[q] > bk || (ck[q] == bk && ci[q] < bi)) {
+                    bk = ck[q];
+                    bi = ci[q];
+                }
+            }
+            const uint32_t K = __reduce_max_sync(0xffffffffu, bk);
+            const uint32_t win = __reduce_min_sync(0xffffffffu, bk == K ? bi : 0xFFFFFFFFu);
+            if (lane == 0) {
+                idx_out[j] = (int32_t)win;
+                w_out[j] = fkey_value(K);  // the pick's key value (its logit when unbiased)
+            }
+#pragma unroll
+            for (int q = 0; q < kTkCand / 32; ++q)
+                if (ci[q] == win) ck[q] = 0u;
+        }
+    } else {
+        // every key is a candidate: the rounds over all of them
+        uint32_t taken = 0u;
+        for (int j = 0; j < k; ++j) {
+            uint32_t bk = 0u;
+            int bq = -1;
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
+                const uint32_t kv = ((taken >> i) & 1u) ? 0u : key[i];
+                if (kv > bk) {
+                    bk = kv;
+                    bq = i;
+                }
+            }
+            const uint32_t K = __reduce_max_sync(0xffffffffu, bk);
+            const uint32_t cand = (bk == K && bq >= 0) ? (uint32_t)(lane + 32 * bq) : 0xFFFFFFFFu;
+            const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+            if (lane == 0) {
+                idx_out[j] = (int32_t)win;
+                w_out[j] = fkey_value(K);
+            }
+            if ((int)(win & 31u) == lane) taken |= 1u << bq;
+        }
     }
+    __syncwarp();
     // weights: lane j takes pick j
     float num = 0.f;
     if (lane < k) {
@@ -218,7 +267,6 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
     const int nst = p.nst, SB = p.sb, Tc = rp.Tc, N = act_n(Tc);
     const int d = rp.d, E = rp.E, k = rp.k;
     const LkSmem so = lk_smem(E, k, Tc, d);
-    const int SG = so.segs;
     uint8_t *tail = smem + nst * SB;
     uint64_t *full = reinterpret_cast<uint64_t *>(tail + so.bars);  // stage bytes landed
     uint64_t *sfr = full + 8;                                        // stage scales in TMEM (4 warps)
@@ -228,22 +276,25 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
     uint64_t *mready = aempty + 2;  // the routing is in shared memory
     uint64_t *mdone = mready + 1;   // every MMA this CTA issued has completed
     uint64_t *rnready = mdone + 1;  // the tokens' 1 / rms are in shared memory (pre-norm)
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(rnready + 1);
+    uint64_t *rdready = rnready + 1;  // every router row is in (warp 0 polled router_done)
+    uint64_t *tkready = rdready + 1;  // the top-k warps are done (picks in shared memory)
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(tkready + 1);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tslot + 1);
     volatile int *s_U = s_abort + 1;
     volatile int *s_last = s_abort + 2;
+    volatile int *s_rdone = s_abort + 3;  // router rows this CTA finished
+    volatile int *s_rok = s_abort + 4;    // every router row is in (top-k warps)
+    int *s_r0c = const_cast<int *>(s_abort) + 8;  // [stage]: warps done with a router unit
     const uint8_t **s_ptab = reinterpret_cast<const uint8_t **>(tail + so.ptab);
     const uint8_t **s_blob = reinterpret_cast<const uint8_t **>(tail + so.blob);
     int32_t *s_eid = reinterpret_cast<int32_t *>(tail + so.eid);
     float *s_wu = reinterpret_cast<float *>(tail + so.wu);      // [u][Tc]
     int32_t *s_tidx = reinterpret_cast<int32_t *>(tail + so.tidx);  // [t][32]
     float *s_tw = reinterpret_cast<float *>(tail + so.tw);
-    float *s_racc = reinterpret_cast<float *>(tail + so.racc);  // [row][Tc]
-    int *s_segr = reinterpret_cast<int *>(tail + so.segr);      // [2][4][SG]
-    float *s_segv = reinterpret_cast<float *>(tail + so.segv);  // [2][4][SG][Tc]
-    int *s_segn = reinterpret_cast<int *>(tail + so.segn);      // [2][4]
+    float *s_racc = reinterpret_cast<float *>(tail + so.racc);  // [warp][row][Tc]
     uint32_t *s_misc = reinterpret_cast<uint32_t *>(tail + so.misc);
     float *s_rn = reinterpret_cast<float *>(tail + so.rn);
+    uint32_t *s_tk = reinterpret_cast<uint32_t *>(tail + so.tk);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     WsHeader *hdr = reinterpret_cast<WsHeader *>(rp.ws + L.hdr);
     const int G = gridDim.x, cta = blockIdx.x;
@@ -261,9 +312,13 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
         mbar_init(mready, 1);
         mbar_init(mdone, 1);
         mbar_init(rnready, 1);
+        mbar_init(rdready, 1);
+        mbar_init(tkready, kLTopkWarps);
         fence_mbar_init();
         *s_abort = 0;
         *s_U = 0;
+        *s_rdone = 0;
+        for (int q = 0; q < 8; ++q) s_r0c[q] = 0;
     }
     constexpr uint32_t kCols = 512u;
     if (warp == 0) umma::tmem_alloc(tslot, kCols);
@@ -278,8 +333,8 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
 
     // ------------------------------------------------------------ shapes --
     const int ffs = p.ffs, ff = p.ff;
-    const long long rfloats = (long long)E * d;
-    const int n0 = (int)((rfloats + kLRUnit - 1) / kLRUnit);   // router units
+    const int rpu = lk_rows_per_unit(d);                        // router rows per unit
+    const int n0 = (E + rpu - 1) / rpu;                         // router units
     const int nkts_d = ceil_div(d, kTileKs);                    // shared gate/up K-tiles (64)
     const int nrbs = ffs > 0 ? ceil_div(ffs, kTileM) : 0;       // shared gate/up items
     const int nkt_d = ceil_div(d, kTileK);                      // routed gate/up K-tiles (256)
@@ -307,11 +362,13 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
     };
     auto start_of = [&](const Range &r, int c) { return (int)(((long long)c * r.n) / r.G); };
     auto owner = [&](const Range &r, int unit) { return (int)((((long long)unit + 1) * r.G - 1) / r.n); };
-    Range rg[4];
-    rg[0] = make_range(p.mode == kLayerRouted ? 0 : n0);
-    rg[1] = make_range(p.mode == kLayerRouteOnly ? 0 : nrbs * nkts_d);
-    rg[2] = make_range(0);
-    rg[3] = make_range(0);
+    // (scalars, not an array: an array indexed by a loop counter would live
+    // in local memory)
+    Range rg0 = make_range(p.mode == kLayerRouted ? 0 : n0);
+    Range rg1 = make_range(p.mode == kLayerRouteOnly ? 0 : nrbs * nkts_d);
+    Range rg2 = make_range(0);
+    Range rg3 = make_range(0);
+    auto rgr = [&](int r) { return r == 0 ? rg0 : (r == 1 ? rg1 : (r == 2 ? rg2 : rg3)); };
     // units per item of the ranges with items (R1, R2, R3)
     auto upi = [&](int r) { return r == 1 ? nkts_d : (r == 2 ? nkt_d : U * ndu + nsdu); };
     // Bounded wait that gives up at once after any role has given up.
@@ -332,8 +389,8 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
         if (warp_wide) ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) return false;
         U = *s_U;
-        rg[2] = make_range(U * nrb_ff * nkt_d);
-        rg[3] = make_range(nrb_d * (U * ndu + nsdu));
+        rg2 = make_range(U * nrb_ff * nkt_d);
+        rg3 = make_range(nrb_d * (U * ndu + nsdu));
         return true;
     };
     // Unit u of range r (r >= 1): item, its unit span, expert, row block,
@@ -368,12 +425,8 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
 
     if (warp == 10) {
         // ================================================= set-up, routing --
-        // blob pointers of every expert -> shared memory (the dispatch reads
-        // them); tensor maps of this CTA's share of the experts (and, in CTA
-        // 0, the shared expert's); this CTA's share of the activation pieces
-        // (x as E2M1 pieces for R2, as bf16 for R1).  Then counted on
-        // prep_done, which the copies warps wait for before their first
-        // B tile or tensor map.
+        // the tokens' 1 / rms (pre-norm calls) and the blob pointer of every
+        // expert -> shared memory (the dispatch reads them)
         if (p.norm_w) {
             // 1 / rms of every token (the same bits in every CTA)
             for (int t = 0; t < Tc; ++t) {
@@ -384,13 +437,27 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
             if (lane == 0)
                 asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(rnready)) : "memory");
         }
-        if (p.mode != kLayerRouteOnly) {
+        if (p.mode != kLayerRouteOnly)
             for (int e = lane; e < E; e += 32) s_ptab[e] = rp.blobs[e];
+    } else if ((warp == 1 || warp == 2) && p.mode != kLayerRouteOnly) {
+        // set-up shared with two of the top-k warps (idle until the router
+        // rows are in): warp 1 this CTA's share of the tensor maps, warp 2
+        // its share of the activation pieces; each counts on prep_done
+        // (2 per CTA), which the copies warps wait for before their first
+        // B tile or tensor map
+        if (warp == 1) {
             refresh_tmaps(rp, cta * 32 + lane, G * 32);
-            build_x_pieces(rp.x, Tc, d, rp.ws, L, cta, G, rp.has_shared != 0, p.norm_w, s_rn);
-            __syncwarp();
-            if (lane == 0) red_add_release(&hdr->prep_done, 1u);
+        } else {
+            int ok = 1;
+            if (p.norm_w) {
+                if (lane == 0) ok = mbar_wait_bounded(rnready, 0u, hdr, rp.wait_ns) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (ok) (void)mbar_try_wait(rnready, 0u);
+            }
+            if (ok) build_x_pieces(rp.x, Tc, d, rp.ws, L, cta, G, rp.has_shared != 0, p.norm_w, s_rn);
         }
+        __syncwarp();
+        if (lane == 0) red_add_release(&hdr->prep_done, 1u);
     }
 
     if ((warp < 4 || warp == 10) && !(p.mode == kLayerRouteOnly && cta != 0)) {
@@ -406,25 +473,53 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                     s_tidx[t * 32 + lane] = __ldcg(gi + t * k + lane);
                     s_tw[t * 32 + lane] = __ldcg(gw + t * k + lane);
                 }
-        } else if (lane == 0) {
-            const uint64_t t0 = globaltimer();
-            while (ld_acquire(&hdr->router_done) < (uint32_t)E) {
-                if (*s_abort || globaltimer() - t0 > rp.wait_ns) {
-                    set_status(hdr, kStTimeout);
-                    *s_abort = 1;
-                    ok = 0;
-                    break;
+        } else {
+            // one poller per CTA (the counter's line is shared by the whole
+            // grid); the other top-k warps wait on rdready
+            if (warp == 0) {
+                // a first pass of the top-k code on a stand-in row (the first E
+                // router weights; picks overwritten below) while the router
+                // rows are summed: the code is fetched now, not on the path
+                warp_topk(rp.wr, E, k, s_tidx, s_tw, nullptr, false, s_tk);
+            }
+            if (lane == 0) {
+                if (warp == 0) {
+                    if (!spin_geq(&hdr->router_done, (uint32_t)E, rp.wait_ns, s_abort)) {
+                        set_status(hdr, kStTimeout);
+                        *s_abort = 1;
+                        ok = 0;
+                    }
+                    *s_rok = ok;
+                    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(rdready)) : "memory");
+                } else {
+                    ok = mbar_wait_bounded(rdready, 0u, hdr, rp.wait_ns) && *s_rok ? 1 : 0;
+                    if (!ok) *s_abort = 1;
                 }
             }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            // every lane acquires the poller's release (which follows its
+            // acquire of the other CTAs' logits)
+            if (ok) (void)mbar_try_wait(rdready, 0u);
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
         if (ok && p.mode != kLayerRouted) {
             const float *logits = reinterpret_cast<const float *>(rp.ws + L.logits);
             for (int t = tw; t < Tc; t += kLTopkWarps)
                 warp_topk(logits + (size_t)t * E, E, k, s_tidx + t * 32, s_tw + t * 32,
-                          (rp.route_flags & kRouteBiasSelect) ? rp.bias : nullptr, (rp.route_flags & kRouteRenorm) != 0);
+                          (rp.route_flags & kRouteBiasSelect) ? rp.bias : nullptr, (rp.route_flags & kRouteRenorm) != 0,
+                          s_tk + tw * 2 * kTkCand);
         }
-        umma::bar_sync(3, 32 * kLTopkWarps);
+        // the picks are in shared memory: each top-k warp counts on tkready,
+        // the dispatching warp waits for all of them
+        __syncwarp();
+        if (lane == 0)
+            asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(tkready)) : "memory");
+        if (warp == 10) {
+            int all = 1;
+            if (lane == 0) all = mbar_wait_bounded(tkready, 0u, hdr, rp.wait_ns) ? 1 : 0;
+            all = __shfl_sync(0xffffffffu, all, 0);
+            if (all) (void)mbar_try_wait(tkready, 0u);
+            else { ok = 0; *s_abort = 1; }
+        }
         if (warp == 10 && ok && !*s_abort && p.mode == kLayerRouteOnly) {
             // route only: the picks into the workspace (and the caller's copies)
             for (int i = lane; i < Tc * k; i += 32) {
@@ -457,9 +552,12 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
             const int Ut = (int)__shfl_sync(0xffffffffu, incl, 31);
             __syncwarp();
             for (int i = lane; i < Ut * Tc; i += 32) s_wu[i] = 0.f;
-            for (int w = lane; w < nwords * 32; w += 32) {
-                if ((bitmap[w >> 5] >> (w & 31)) & 1u) {
-                    const uint32_t u = prefix[w >> 5] + __popc(bitmap[w >> 5] & ((1u << (w & 31)) - 1u));
+            if (lane < nwords) {
+                // lane l: the set bits of word l, in ascending expert id
+                uint32_t bits = bitmap[lane], u = prefix[lane];
+                while (bits != 0u) {
+                    const int w = 32 * lane + __ffs(bits) - 1;
+                    bits &= bits - 1u;
                     const uint8_t *b = s_ptab[w];
                     if (b == nullptr || (reinterpret_cast<uintptr_t>(b) & 15u) != 0u) {
                         set_status(hdr, kStDeviceCheck);
@@ -467,6 +565,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                     }
                     s_blob[u] = b;
                     s_eid[u] = w;
+                    ++u;
                 }
             }
             __syncwarp();
@@ -516,14 +615,13 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
             };
             auto gu_ready = [&](bool block) {
                 if (gu_ok) return true;
-                const uint64_t t0 = globaltimer();
-                while (ld_acquire(&hdr->gu_done) < gu_total) {
-                    if (!block) return false;
-                    if (*s_abort || globaltimer() - t0 > rp.wait_ns) {
-                        set_status(hdr, kStTimeout);
-                        *s_abort = 1;
-                        return false;
-                    }
+                if (!block) {
+                    if (ld_relaxed(&hdr->gu_done) < gu_total) return false;
+                    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+                } else if (!spin_geq(&hdr->gu_done, gu_total, rp.wait_ns, s_abort)) {
+                    set_status(hdr, kStTimeout);
+                    *s_abort = 1;
+                    return false;
                 }
                 asm volatile("fence.proxy.async.global;" ::: "memory");  // before bulk copies read h
                 gu_ok = true;
@@ -534,7 +632,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                     if (!routed_ranges(false)) break;
                     gu_total = (uint32_t)(nrbs + U * nrb_ff);
                 }
-                const Range R = rg[r];
+                const Range R = rgr(r);
                 for (int unit = R.a; unit < R.b && !*s_abort; ++unit, ++i) {
                     const int s = i % nst;
                     const uint32_t ph = (uint32_t)((i / nst) & 1);
@@ -551,27 +649,20 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                     if (i >= nst && !wait(&empty[s], ph ^ 1u)) break;
                     uint8_t *st = smem + s * SB;
                     if (r == 0) {
-                        const long long f0 = (long long)unit * kLRUnit;
-                        const long long f1 = min(rfloats, f0 + kLRUnit);
-                        const uint32_t bytes = (uint32_t)((f1 - f0) * 4);
+                        const int ur0 = unit * rpu;
+                        const uint32_t bytes = (uint32_t)(min(rpu, E - ur0) * d * 4);
                         mbar_arrive_expect_tx(&full[s], bytes);
-                        bulk_g2s(st, rp.wr + f0, bytes, &full[s]);
+                        bulk_g2s(st, rp.wr + (size_t)ur0 * d, bytes, &full[s]);
                         continue;
                     }
                     if (!prep_ok) {
                         // x pieces, x as bf16 and the tensor maps are published
                         // by every CTA's set-up warp
-                        const uint64_t t0 = globaltimer();
-                        bool ok = true;
-                        while (ld_acquire(&hdr->prep_done) < (uint32_t)G) {
-                            if (globaltimer() - t0 > rp.wait_ns) {
-                                set_status(hdr, kStTimeout);
-                                *s_abort = 1;
-                                ok = false;
-                                break;
-                            }
+                        if (!spin_geq(&hdr->prep_done, (uint32_t)(2 * G), rp.wait_ns, s_abort)) {
+                            set_status(hdr, kStTimeout);
+                            *s_abort = 1;
+                            break;
                         }
-                        if (!ok) break;
                         asm volatile("fence.proxy.async.global;" ::: "memory");
                         prep_ok = true;
                     }
@@ -660,12 +751,12 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
         const int wl = warp - 4;
         const uint32_t lb = umma::lane_base(warp);
         uint32_t nanb = 0u;
-        // this CTA's router slice: floats [f_lo, f_hi), rows row_base ..
-        const Range R0 = rg[0];
-        const long long f_lo = (long long)R0.a * kLRUnit, f_hi = min(rfloats, (long long)R0.b * kLRUnit);
-        const int row_base = R0.a < R0.b ? (int)(f_lo / d) : 0;
-        const int nrows = R0.a < R0.b ? (int)((f_hi - 1) / d) - row_base + 1 : 0;
-        for (int q = tid; q < kRMaxRows * Tc; q += 128) s_racc[q] = 0.f;
+        // this CTA's router rows: row_base .. row_base + nrows - 1 (whole
+        // rows: a unit is rpu rows)
+        const Range R0 = rg0;
+        const int row_base = R0.a * rpu;
+        const int nrows = R0.a < R0.b ? min(E, R0.b * rpu) - row_base : 0;
+        for (int q = tid; q < 4 * kRMaxRows * Tc; q += 128) s_racc[q] = 0.f;
         bool go = true;
         if (p.norm_w) {
             // the router reads x = RMSNorm(h): wait for the tokens' 1 / rms
@@ -678,127 +769,168 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
         } else {
             umma::bar_sync(2, 128);
         }
+        // this thread's 64 floats of a unit: row rin_t of the unit, columns
+        // col_t .. col_t + 63 (the same in every unit)
+        const int f_t = 64 * tid;
+        const int rin_t = f_t / d, col_t = f_t - rin_t * d;
+        // Token t's 64 columns of x: eight 16-byte loads issued together,
+        // chunk (q + lane) mod 8 into register q, so the weight reads (the
+        // same rotated order) spread over the shared-memory banks and every
+        // register index stays static.  x = RMSNorm(h) on pre-norm calls.
+        auto load_x = [&](int t, uint4 (&xr)[8]) {
+            const uint4 *xv = reinterpret_cast<const uint4 *>(rp.x + (size_t)t * d + col_t);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) xr[q] = __ldg(xv + ((q + lane) & 7));
+            if (p.norm_w) {
+                const uint4 *gv = reinterpret_cast<const uint4 *>(p.norm_w + col_t);
+                const float rt = s_rn[t];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint4 g = __ldg(gv + ((q + lane) & 7));
+                    uint32_t *xw = reinterpret_cast<uint32_t *>(&xr[q]);
+                    const uint32_t *gw = reinterpret_cast<const uint32_t *>(&g);
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        xw[h] = (uint32_t)rms_norm_bf16((uint16_t)(xw[h] & 0xFFFFu), rt, (uint16_t)(gw[h] & 0xFFFFu)) |
+                                ((uint32_t)rms_norm_bf16((uint16_t)(xw[h] >> 16), rt, (uint16_t)(gw[h] >> 16)) << 16);
+                }
+            }
+        };
+        // 64 products (each exact), summed in fp32 in this order
+        auto dot_w = [&](const float4 *w4, const uint4 (&xr)[8]) {
+            float acc = 0.f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int jq = (q + lane) & 7;
+                const float4 a = w4[2 * jq], b = w4[2 * jq + 1];
+                acc = fmaf(a.x, bf16_lo(xr[q].x), acc);
+                acc = fmaf(a.y, bf16_hi(xr[q].x), acc);
+                acc = fmaf(a.z, bf16_lo(xr[q].y), acc);
+                acc = fmaf(a.w, bf16_hi(xr[q].y), acc);
+                acc = fmaf(b.x, bf16_lo(xr[q].z), acc);
+                acc = fmaf(b.y, bf16_hi(xr[q].z), acc);
+                acc = fmaf(b.z, bf16_lo(xr[q].w), acc);
+                acc = fmaf(b.w, bf16_hi(xr[q].w), acc);
+            }
+            return acc;
+        };
         int i = 0;
         bool act_ok[2] = {false, false};  // x pieces' scales / h pieces' scales seen (no-TMA path)
-        for (int r = 0; r < 4 && go; ++r) {
-            if (r == 2 && !routed_ranges(true)) break;
-            const Range R = rg[r];
+        // ---- R0: the router rows of this CTA.  One token (ONE): its columns
+        // of x stay in registers for the whole slice; more tokens: loaded per
+        // unit, the next token's loads in flight during this one's products.
+        auto router_units = [&](auto one) {
+            constexpr bool ONE = decltype(one)::value;
+            uint4 x0[8];
+            if (ONE && f_t < rpu * d) load_x(0, x0);
+            const Range R = rg0;
             for (int unit = R.a; unit < R.b; ++unit, ++i) {
                 const int s = i % nst;
                 const uint32_t ph = (uint32_t)((i / nst) & 1);
                 int ok = 0;
                 if (lane == 0) ok = wait(&full[s], ph) ? 1 : 0;
                 ok = __shfl_sync(0xffffffffu, ok, 0);
-                // router units end in a barrier of the four warps: they agree
-                // on going on, so none is left waiting at it
-                if (r == 0) ok = umma::bar_red_and(2, 128, ok != 0) ? 1 : 0;
                 if (!ok) {
                     go = false;
                     break;
                 }
                 (void)mbar_try_wait(&full[s], ph);  // every lane sees the landed bytes
                 const uint8_t *st = smem + s * SB;
-                if (r == 0) {
-                    // 64 consecutive floats per thread (one row: d is a multiple
-                    // of 64), every token; then the warp's sums per row
-                    // (segmented, fixed order) into this unit's buffers
-                    const long long f = (long long)unit * kLRUnit + 64LL * tid;
-                    int row = -1;
-                    float v[kChunk];
+                // Each warp on its own: 64 consecutive floats of the unit
+                // per thread (inside one row: d is a multiple of 64), the
+                // same columns of x in every unit; the warp's sums per row
+                // (segmented over lanes, fixed order) go into its own row
+                // accumulators, unit after unit; the last of the four warps
+                // to finish a unit releases its stage.
+                const int ur0 = unit * rpu;  // first row of the unit
+                const int ufl = min(rpu, E - ur0) * d;
+                int row = -1;
+                float v[kChunk];
 #pragma unroll
-                    for (int t = 0; t < kChunk; ++t) v[t] = 0.f;
-                    if (f < f_hi) {
-                        row = (int)(f / d);
-                        const int col = (int)(f - (long long)row * d);
-                        // This thread's 64 columns of x for a token: eight
-                        // 16-byte loads issued together, chunk (q + lane) mod 8
-                        // into register q, so the weight reads below (the same
-                        // rotated order) spread over the shared-memory banks
-                        // and every register index stays static; the next
-                        // token's loads are in flight while this one's FMAs run.
-                        // Each product is exact; each sum fp32 in this order.
-                        const float4 *w4 = reinterpret_cast<const float4 *>(st) + tid * 16;
-                        auto load_x = [&](int t, uint4 (&xr)[8]) {
-                            const uint4 *xv = reinterpret_cast<const uint4 *>(rp.x + (size_t)t * d + col);
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) xr[q] = __ldg(xv + ((q + lane) & 7));
-                            if (p.norm_w) {
-                                // x = RMSNorm(h), element by element
-                                const uint4 *gv = reinterpret_cast<const uint4 *>(p.norm_w + col);
-                                const float rt = s_rn[t];
-#pragma unroll
-                                for (int q = 0; q < 8; ++q) {
-                                    const uint4 g = __ldg(gv + ((q + lane) & 7));
-                                    uint32_t *xw = reinterpret_cast<uint32_t *>(&xr[q]);
-                                    const uint32_t *gw = reinterpret_cast<const uint32_t *>(&g);
-#pragma unroll
-                                    for (int h = 0; h < 4; ++h)
-                                        xw[h] = (uint32_t)rms_norm_bf16((uint16_t)(xw[h] & 0xFFFFu), rt, (uint16_t)(gw[h] & 0xFFFFu)) |
-                                                ((uint32_t)rms_norm_bf16((uint16_t)(xw[h] >> 16), rt, (uint16_t)(gw[h] >> 16)) << 16);
-                                }
-                            }
-                        };
-                        auto dot = [&](const uint4 (&xr)[8]) {
-                            float acc = 0.f;
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                const int jq = (q + lane) & 7;
-                                const float4 a = w4[2 * jq], b = w4[2 * jq + 1];
-                                acc = fmaf(a.x, bf16_lo(xr[q].x), acc);
-                                acc = fmaf(a.y, bf16_hi(xr[q].x), acc);
-                                acc = fmaf(a.z, bf16_lo(xr[q].y), acc);
-                                acc = fmaf(a.w, bf16_hi(xr[q].y), acc);
-                                acc = fmaf(b.x, bf16_lo(xr[q].z), acc);
-                                acc = fmaf(b.y, bf16_hi(xr[q].z), acc);
-                                acc = fmaf(b.z, bf16_lo(xr[q].w), acc);
-                                acc = fmaf(b.w, bf16_hi(xr[q].w), acc);
-                            }
-                            return acc;
-                        };
+                for (int t = 0; t < kChunk; ++t) v[t] = 0.f;
+                if (f_t < ufl) {
+                    row = ur0 + rin_t - row_base;
+                    const float4 *w4 = reinterpret_cast<const float4 *>(st) + tid * 16;
+                    if constexpr (ONE) {
+                        v[0] = dot_w(w4, x0);
+                    } else {
                         uint4 xa[8], xb[8];
                         load_x(0, xa);
 #pragma unroll
                         for (int t = 0; t < kChunk; ++t) {
                             if (t < Tc) {
                                 if (t + 1 < Tc) load_x(t + 1, (t & 1) ? xa : xb);
-                                v[t] = dot((t & 1) ? xb : xa);
+                                v[t] = dot_w(w4, (t & 1) ? xb : xa);
                             }
                         }
                     }
-                    // segmented sum over lanes of equal row (rows do not decrease along lanes)
+                }
+                // segmented sum over lanes of equal row (rows do not decrease along lanes)
 #pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const int rn = __shfl_down_sync(0xffffffffu, row, o);
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int rn = __shfl_down_sync(0xffffffffu, row, o);
 #pragma unroll
-                        for (int t = 0; t < kChunk; ++t) {
+                    for (int t = 0; t < kChunk; ++t) {
+                        if (t < Tc) {
                             const float vn = __shfl_down_sync(0xffffffffu, v[t], o);
                             if (lane + o < 32 && rn == row) v[t] += vn;
                         }
                     }
-                    const int rprev = __shfl_up_sync(0xffffffffu, row, 1);
-                    const bool head = row >= 0 && (lane == 0 || rprev != row);
-                    const uint32_t heads = __ballot_sync(0xffffffffu, head);
-                    const int b = i & 1;
-                    if (head) {
-                        const int q = __popc(heads & ((1u << lane) - 1u));
-                        s_segr[(b * 4 + wl) * SG + q] = row;
+                }
+                const int rprev = __shfl_up_sync(0xffffffffu, row, 1);
+                if (row >= 0 && (lane == 0 || rprev != row)) {
+                    float *acc = s_racc + ((size_t)wl * kRMaxRows + row) * Tc;
 #pragma unroll
-                        for (int t = 0; t < kChunk; ++t)
-                            if (t < Tc) s_segv[((b * 4 + wl) * SG + q) * Tc + t] = v[t];
-                    }
-                    if (lane == 0) s_segn[b * 4 + wl] = __popc(heads);
-                    umma::bar_sync(2, 128);  // the stage is read and the row sums posted
-                    if (tid == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[s])) : "memory");
-                    // fold the warps' row sums into the slice's rows, warps in order
-                    if (tid < nrows) {
-                        const int rr = row_base + tid;
-                        for (int w2 = 0; w2 < 4; ++w2)
-                            for (int q = 0; q < s_segn[b * 4 + w2]; ++q)
-                                if (s_segr[(b * 4 + w2) * SG + q] == rr)
-                                    for (int t = 0; t < Tc; ++t)
-                                        s_racc[tid * Tc + t] += s_segv[((b * 4 + w2) * SG + q) * Tc + t];
-                    }
-                } else {
+                    for (int t = 0; t < kChunk; ++t)
+                        if (t < Tc) acc[t] += v[t];
+                }
+                __syncwarp();
+                if (lane == 0 && atomicAdd(&s_r0c[s], 1) == 3) {
+                    s_r0c[s] = 0;
+                    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[s])) : "memory");
+                }
+            }
+        };
+        if (go) {
+            if (Tc == 1)
+                router_units(std::integral_constant<bool, true>{});
+            else
+                router_units(std::integral_constant<bool, false>{});
+            // the slice's rows: the four warps' sums in warp order, one
+            // release per CTA on router_done (the barrier orders every
+            // thread's logit stores before thread 0's release)
+            go = umma::bar_red_and(2, 128, go);
+            if (go && tid < nrows) {
+                const int rr = row_base + tid;
+                float *logits = reinterpret_cast<float *>(rp.ws + L.logits);
+                const float bias = (rp.bias && !(rp.route_flags & kRouteBiasSelect)) ? rp.bias[rr] : 0.f;
+                for (int t = 0; t < Tc; ++t) {
+                    float o = s_racc[(size_t)tid * Tc + t];
+#pragma unroll
+                    for (int w2 = 1; w2 < 4; ++w2) o += s_racc[((size_t)w2 * kRMaxRows + tid) * Tc + t];
+                    logits[(size_t)t * E + rr] = o + bias;
+                }
+            }
+            umma::bar_sync(2, 128);
+            if (tid == 0 && go && nrows > 0) red_add_release(&hdr->router_done, (uint32_t)nrows);
+        }
+        // ---- R1 .. R3: the scale factors of the matrix units
+        for (int r = 1; r < 4 && go; ++r) {
+            if (r == 2 && !routed_ranges(true)) break;
+            const Range R = rgr(r);
+            for (int unit = R.a; unit < R.b; ++unit, ++i) {
+                const int s = i % nst;
+                const uint32_t ph = (uint32_t)((i / nst) & 1);
+                int ok = 0;
+                if (lane == 0) ok = wait(&full[s], ph) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) {
+                    go = false;
+                    break;
+                }
+                (void)mbar_try_wait(&full[s], ph);  // every lane sees the landed bytes
+                const uint8_t *st = smem + s * SB;
+                {
                     const Unit x = decode(r, unit);
                     if (x.kind == 2 || x.kind == 3) {
                         const uint8_t *blob = s_blob[x.u];
@@ -856,10 +988,8 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                                     const int ai = x.kind == 2 ? 0 : 1;
                                     if (!act_ok[ai]) {
                                         const uint32_t *ctr = ai == 0 ? &hdr->prep_done : &hdr->gu_done;
-                                        const uint32_t want = ai == 0 ? (uint32_t)G : (uint32_t)(nrbs + U * nrb_ff);
-                                        const uint64_t t0 = globaltimer();
-                                        while (ld_acquire(ctr) < want && globaltimer() - t0 <= rp.wait_ns) {
-                                        }
+                                        const uint32_t want = ai == 0 ? (uint32_t)(2 * G) : (uint32_t)(nrbs + U * nrb_ff);
+                                        (void)spin_geq(ctr, want, rp.wait_ns);
                                         act_ok[ai] = true;
                                     }
                                     const uint32_t *sb = x.kind == 2
@@ -884,46 +1014,6 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                     if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sfr[s])) : "memory");
                 }
             }
-            if (r == 0) {
-                // the slice's rows: finished here, or (cut by a CTA boundary)
-                // parked for the last of their CTAs, which sums the parts in
-                // CTA order; each finished row counts on router_done
-                umma::bar_sync(2, 128);
-                if (go && tid < nrows) {
-                    const int rr = row_base + tid;
-                    const long long rs = (long long)rr * d, re = rs + d;  // its floats
-                    float *logits = reinterpret_cast<float *>(rp.ws + L.logits);
-                    const float bias = (rp.bias && !(rp.route_flags & kRouteBiasSelect)) ? rp.bias[rr] : 0.f;
-                    bool done = false;
-                    float out[kChunk];
-                    if (rs >= f_lo && re <= f_hi) {
-#pragma unroll
-                        for (int t = 0; t < kChunk; ++t) out[t] = t < Tc ? s_racc[tid * Tc + t] : 0.f;
-                        done = true;
-                    } else {
-                        const int first = owner(R0, (int)(rs / kLRUnit));
-                        const int nseg = owner(R0, (int)((re - 1) / kLRUnit)) - first + 1;
-                        float *pp = reinterpret_cast<float *>(rp.ws + L.part) + ((size_t)rr * kMaxSeg) * kChunk;
-                        uint32_t *pc = reinterpret_cast<uint32_t *>(rp.ws + L.cnt) + rr;
-#pragma unroll
-                        for (int t = 0; t < kChunk; ++t) pp[(cta - first) * kChunk + t] = t < Tc ? s_racc[tid * Tc + t] : 0.f;
-                        const uint32_t old = atom_add_acq_rel(pc, 1u);
-                        if (old == (uint32_t)(nseg - 1)) {
-#pragma unroll
-                            for (int t = 0; t < kChunk; ++t) out[t] = 0.f;
-                            for (int sl = 0; sl < nseg; ++sl)
-#pragma unroll
-                                for (int t = 0; t < kChunk; ++t) out[t] += __ldcg(pp + sl * kChunk + t);
-                            *pc = 0u;
-                            done = true;
-                        }
-                    }
-                    if (done) {
-                        for (int t = 0; t < Tc; ++t) logits[(size_t)t * E + rr] = out[t] + bias;
-                        red_add_release(&hdr->router_done, 1u);  // after this thread's logit stores
-                    }
-                }
-            }
         }
         if (p.strict && __any_sync(0xffffffffu, nanb != 0u) && lane == 0) set_status(hdr, kStDeviceCheck);
     } else if (warp == 9) {
@@ -940,10 +1030,10 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
             // router units (the first n0 of the ring) are consumed by the
             // scale warps and do not complete sfr: stage s's matrix use
             // number is its use number minus its router uses
-            const int n0 = rg[0].b - rg[0].a;
+            const int n0 = rg0.b - rg0.a;
             for (int r = 0; r < 4 && !*s_abort; ++r) {
                 if (r == 2 && !routed_ranges(false)) break;
-                const Range R = rg[r];
+                const Range R = rgr(r);
                 if (r == 0) {
                     i += n0;
                     continue;
@@ -1047,7 +1137,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
         for (int r = 1; r < 4; ++r) {
             // the four warps agree on going on (they share named barrier 1)
             if (r == 2 && !umma::bar_red_and(1, 128, routed_ranges(true))) break;
-            const Range R = rg[r];
+            const Range R = rgr(r);
             uint32_t *icnt = reinterpret_cast<uint32_t *>(rp.ws + L.icnt) +
                              (r == 1 ? L.umax * nrb_ff : (r == 2 ? 0 : L.umax * nrb_ff + nrbs));
             const int NM = r == 3 ? 1 : 2;

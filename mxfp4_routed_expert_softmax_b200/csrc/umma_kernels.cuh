@@ -378,9 +378,11 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         return (int)((((long long)(unit - r.base) + 1) * r.G - 1) / r.n);
     };
     // gate/up: [shared units | routed units]; down: [all units | nothing]
-    Range rng[2];
-    rng[0] = GU ? make_range(0, S) : make_range(0, nrb * upi);
-    rng[1] = make_range(0, 0);
+    // (two scalars, not an array: an array indexed by a loop counter would
+    // live in local memory)
+    Range rng0 = GU ? make_range(0, S) : make_range(0, nrb * upi);
+    Range rng1 = make_range(0, 0);
+    auto rng = [&](int ri) { return ri == 0 ? rng0 : rng1; };
     // gate/up, before the routed range: wait for the routing (lane 0 of the
     // calling warp waits, the warp follows), then size the routed range
     auto routed_range = [&](bool warp_wide) {
@@ -392,7 +394,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         if (warp_wide) ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) return false;
         U = *s_U;
-        rng[1] = make_range(S, U * nrb * nkt);
+        rng1 = make_range(S, U * nrb * nkt);
         return true;
     };
     const size_t mat = (size_t)p.d * p.ff;
@@ -485,23 +487,18 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             int last_u = -2;
             uint32_t ph = 0u;  // phase of the current pass over the stages
             int it = 0, s = 0;
-            if (GU && rng[0].a < rng[0].b && p.route_ctas > 0) {
+            if (GU && rng0.a < rng0.b && p.route_ctas > 0) {
                 // the shared units read x as bf16 and the shared tensor maps,
                 // which the router kernel's CTAs publish by counting prep_done
-                const uint64_t t0 = globaltimer();
-                while (ld_acquire(&hdr->prep_done) < (uint32_t)p.route_ctas) {
-                    __nanosleep(32);
-                    if (globaltimer() - t0 > p.wait_ns) {
-                        set_status(hdr, kStTimeout);
-                        *s_abort = 1;
-                        break;
-                    }
+                if (!spin_geq(&hdr->prep_done, (uint32_t)p.route_ctas, p.wait_ns)) {
+                    set_status(hdr, kStTimeout);
+                    *s_abort = 1;
                 }
                 asm volatile("fence.proxy.async.global;" ::: "memory");  // before the bulk copies read x
             }
             for (int ri = 0; ri < 2 && !*s_abort; ++ri) {
             if (ri == 1 && (!GU || !routed_range(false))) break;
-            const Range rg = rng[ri];
+            const Range rg = rng(ri);
             Unit x = rg.a < rg.b ? decode(rg.a) : Unit{};
             for (int unit = rg.a; unit < rg.b && !*s_abort; x = advance(x, ++unit, rg.b), ++it) {
                 if (it >= nst && !wait(&empty[s], ph ^ 1u)) break;
@@ -578,7 +575,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             int s = 0;
             for (int ri = 0; ri < 2; ++ri) {
             if (ri == 1 && (!GU || !routed_range(true))) break;
-            const Range rg = rng[ri];
+            const Range rg = rng(ri);
             Unit x = rg.a < rg.b ? decode(rg.a) : Unit{};
             bool go_on = true;
             for (int unit = rg.a; unit < rg.b; x = advance(x, ++unit, rg.b)) {
@@ -686,7 +683,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         int done = 0;  // stages passed in earlier ranges
         for (int ri = 0; ri < 2 && go; ++ri) {
             if (ri == 1 && (!GU || !routed_range(true))) break;
-            const Range rg = rng[ri];
+            const Range rg = rng(ri);
             const int a = rg.a, n = rg.b - rg.a;
 #pragma unroll
             for (int i = 0; i < kLook; ++i)
@@ -720,7 +717,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             uint32_t ph = 0u;
             for (int ri = 0; ri < 2 && !*s_abort; ++ri) {
             if (ri == 1 && (!GU || !routed_range(false))) break;
-            const Range rg = rng[ri];
+            const Range rg = rng(ri);
             for (int unit = rg.a; unit < rg.b && !*s_abort; ++seg) {
                 Unit x = decode(unit);
                 const int seg_end = min(rg.b, x.iend);
@@ -787,7 +784,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         int seg = 0;
         for (int ri = 0; ri < 2; ++ri) {
         if (ri == 1 && (!GU || !routed_range(true))) break;
-        const Range rg = rng[ri];
+        const Range rg = rng(ri);
         for (int unit = rg.a; unit < rg.b; ++seg) {
             const Unit x = decode(unit);
             const int item = x.item;
