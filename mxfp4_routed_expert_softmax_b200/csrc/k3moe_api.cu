@@ -89,7 +89,8 @@ k3moe_status device_info(DeviceInfo **out) {
         if (r == cudaSuccess) r = set_smem(umma_expert_kernel<false>, big);
         if (r == cudaSuccess) r = set_smem(pf_expert_kernel<true>, big);
         if (r == cudaSuccess) r = set_smem(pf_expert_kernel<false>, big);
-        if (r == cudaSuccess) r = set_smem(layer_kernel, big);
+        if (r == cudaSuccess) r = set_smem(layer_kernel<1, true>, big);
+        if (r == cudaSuccess) r = set_smem(layer_kernel<0, false>, big);
         if (r == cudaSuccess) r = set_smem(pf_router_mma_kernel, rm_smem_bytes());
         if (r != cudaSuccess) return cuda_fail(r);
         di.ready = true;
@@ -400,17 +401,21 @@ cudaError_t launch_layer(const DeviceInfo &di, LayerParams lp, int nst, cudaStre
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, layer_kernel, lp);
+    // one decode token with TMA scale boxes: the specialised instance
+    if (lp.r.Tc == 1 && lp.sf_tma_gu && lp.sf_tma_dn) return cudaLaunchKernelEx(&cfg, layer_kernel<1, true>, lp);
+    return cudaLaunchKernelEx(&cfg, layer_kernel<0, false>, lp);
 }
 
 // The routing of one decode pass by the one-launch kernel stopped after its
 // top-k (the picks land in the workspace and in idx_out / w_out): the same
 // bits as the routing inside a full launch of the same pass.
-cudaError_t launch_layer_route(const DeviceInfo &di, const RouteParams &rp, int nst, cudaStream_t st) {
+cudaError_t launch_layer_route(const DeviceInfo &di, const RouteParams &rp, int nst, cudaStream_t st, bool ff_tma) {
     LayerParams lp{};
     lp.r = rp;
     lp.r.wait_ns = wait_limit();
     lp.mode = kLayerRouteOnly;
+    // the instance a full launch of the same pass takes (same routing code)
+    lp.sf_tma_gu = lp.sf_tma_dn = rp.d % 512 == 0 && ff_tma;
     return launch_layer(di, lp, nst, st);
 }
 
@@ -845,7 +850,7 @@ k3moe_status k3moe_route(const void *x, int32_t T, const float *w_router, const 
         rp.idx_out = idx + (size_t)c0 * dims->top_k;
         rp.w_out = weight + (size_t)c0 * dims->top_k;
         const int lst = kUseLayerKernel ? layer_stages(*di, dims, Tc) : 0;
-        cudaError_t e = lst > 0 ? launch_layer_route(*di, rp, lst, st) : launch_route(*di, rp, st);
+        cudaError_t e = lst > 0 ? launch_layer_route(*di, rp, lst, st, dims->ff % 512 == 0) : launch_route(*di, rp, st);
         if (e != cudaSuccess) return cuda_fail(e);
     }
     return K3MOE_OK;
@@ -1091,7 +1096,7 @@ k3moe_status k3moe_layer_cached(k3moe_cache *cache, const void *x, int32_t T, co
         // the routing by the kernel the layer call will use, so the experts
         // fetched are exactly the ones its dispatch takes
         const int lst = kUseLayerKernel ? layer_stages(*di, dims, Tc) : 0;
-        cudaError_t e = lst > 0 ? launch_layer_route(*di, rp, lst, st) : launch_route(*di, rp, st);
+        cudaError_t e = lst > 0 ? launch_layer_route(*di, rp, lst, st, dims->ff % 512 == 0) : launch_route(*di, rp, st);
         if (e != cudaSuccess) return cuda_fail(e, "router launch");
         e = cudaMemcpyAsync(idx_host + (size_t)c0 * k, reinterpret_cast<uint8_t *>(ws) + L.idx,
                             (size_t)Tc * k * 4, cudaMemcpyDeviceToHost, st);

@@ -52,6 +52,7 @@ constexpr int kLRUnit = 8192;         // router floats per R0 unit at most (32 K
 constexpr int kLSfc = 32;             // TMEM scale columns per stage
 constexpr int kLTopkWarps = 5;        // warps 0-3 and 10
 constexpr int kTkCand = 128;          // top-k candidates per warp (scratch: keys, then ids)
+constexpr int kTkWords = 2 * kTkCand + 4;  // a top-k warp's scratch: candidates, count, max, sum
 
 struct LayerParams {
     RouteParams r;     // x, Tc, router, shapes, workspace, blobs, maps, wait_ns
@@ -109,7 +110,7 @@ __host__ __device__ inline LkSmem lk_smem(int E, int k, int Tc, int d) {
     s.racc = o;   o += a16(4 * kRMaxRows * Tc * 4);   // router row sums of this CTA's rows, per warp
     s.misc = o;   o += 64 * 4;                        // dispatch bitmap / prefix
     s.rn = o;     o += kChunk * 4;                    // 1 / rms of each token (pre-norm)
-    s.tk = o;     o += kLTopkWarps * 2 * kTkCand * 4;  // top-k candidates of each top-k warp
+    s.tk = o;     o += kLTopkWarps * kTkWords * 4;   // top-k candidates of each top-k warp
     s.total = o;
     return s;
 }
@@ -131,7 +132,7 @@ __host__ __device__ inline int lk_smem_bytes(int N, int nst, int E, int k, int T
 // warp's scratch and the k rounds (warp max of the lanes' best candidate,
 // lowest id among equal keys) run over at most four per lane.  More than
 // kTkCand candidates (many equal keys) take the rounds over all keys.
-__device__ __noinline__ void warp_topk(const float *row, int E, int k, int32_t *idx_out, float *w_out,
+__device__ void warp_topk(const float *row, int E, int k, int32_t *idx_out, float *w_out,
                           const float *sel_bias, bool renorm, uint32_t *scratch) {
     const int lane = threadIdx.x & 31;
     constexpr int kPer = 32;  // E <= 1024
@@ -258,13 +259,173 @@ __device__ __noinline__ void warp_topk(const float *row, int E, int k, int32_t *
     __syncwarp();
 }
 
+// One token's top-k by four warps (one token per pass is the decode case):
+// warp q takes the slice [e0, e1) of the row (lane l: e0 + l + 32 i) and
+// posts its candidates (keys >= the k-th largest of its 32 lane maxima, so
+// every key of the token's top-k that lies in the slice) with their ids,
+// their count (kTkCand + 1 when they do not fit) and its softmax partial:
+// max of the logits and sum of exp(l - max) over the slice.
+__device__ void warp_topk_part(const float *row, int e0, int e1, int k, const float *sel_bias, uint32_t *scratch) {
+    const int lane = threadIdx.x & 31;
+    constexpr int kPer = 8;  // slices of at most 256
+    uint32_t key[kPer];
+    float val[kPer];
+    float mx = -INFINITY;
+    uint32_t lmax = 0u;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int e = e0 + lane + 32 * i;
+        const float v = e < e1 ? __ldcg(row + e) : -INFINITY;
+        val[i] = v;
+        key[i] = e < e1 ? fkey(sel_bias ? v + __ldg(sel_bias + e) : v) : 0u;  // real keys are > 0
+        mx = fmaxf(mx, v);
+        lmax = max(lmax, key[i]);
+    }
+    const float m = fkey_value(__reduce_max_sync(0xffffffffu, fkey(mx)));
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+        if (e0 + lane + 32 * i < e1) sum += expf(val[i] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    int rank = 0;
+#pragma unroll
+    for (int o = 0; o < 32; ++o) {
+        const uint32_t other = __shfl_sync(0xffffffffu, lmax, o);
+        rank += (other > lmax || (other == lmax && o < lane)) ? 1 : 0;
+    }
+    const uint32_t at = __ballot_sync(0xffffffffu, rank == k - 1);
+    const uint32_t L = at ? __shfl_sync(0xffffffffu, lmax, __ffs(at) - 1) : 0u;
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) c += (key[i] != 0u && key[i] >= L) ? 1 : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (total <= kTkCand) {
+        int pos = incl - c;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            if (key[i] != 0u && key[i] >= L) {
+                scratch[pos] = key[i];
+                scratch[kTkCand + pos] = (uint32_t)(e0 + lane + 32 * i);
+                ++pos;
+            }
+        }
+    }
+    if (lane == 0) {
+        scratch[2 * kTkCand] = (uint32_t)(total <= kTkCand ? total : kTkCand + 1);
+        scratch[2 * kTkCand + 1] = __float_as_uint(m);
+        scratch[2 * kTkCand + 2] = __float_as_uint(sum);
+    }
+}
+
+// The merge of the four parts by one warp: the k rounds over the union of
+// the candidates (warp max of the lanes' best, lowest id among equal keys),
+// the softmax from the parts' partials (max over the parts, sums rescaled to
+// it).  False (nothing written) when the candidates do not fit: the caller
+// then runs warp_topk over the whole row.
+__device__ bool warp_topk_merge(const float *row, int k, int32_t *idx_out, float *w_out, const float *sel_bias,
+                                bool renorm, const uint32_t *scratch) {
+    const int lane = threadIdx.x & 31;
+    int cnt[4], off[4], C = 0;
+    bool fit = true;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        cnt[q] = (int)scratch[q * kTkWords + 2 * kTkCand];
+        fit = fit && cnt[q] <= kTkCand;
+        off[q] = C;
+        C += cnt[q];
+    }
+    if (!fit || C > kTkCand) return false;
+    float m = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) m = fmaxf(m, __uint_as_float(scratch[q * kTkWords + 2 * kTkCand + 1]));
+    float z = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float mq = __uint_as_float(scratch[q * kTkWords + 2 * kTkCand + 1]);
+        const float sq = __uint_as_float(scratch[q * kTkWords + 2 * kTkCand + 2]);
+        if (sq > 0.f) z += sq * expf(mq - m);
+    }
+    uint32_t ck[kTkCand / 32], ci[kTkCand / 32];
+#pragma unroll
+    for (int r = 0; r < kTkCand / 32; ++r) {
+        const int j = 32 * r + lane;
+        ck[r] = 0u;
+        ci[r] = 0xFFFFFFFFu;
+        if (j < C) {
+            int q = 0, base = 0;
+#pragma unroll
+            for (int qq = 1; qq < 4; ++qq) {
+                if (j >= off[qq]) {
+                    q = qq;
+                    base = off[qq];
+                }
+            }
+            ck[r] = scratch[q * kTkWords + (j - base)];
+            ci[r] = scratch[q * kTkWords + kTkCand + (j - base)];
+        }
+    }
+    for (int j = 0; j < k; ++j) {
+        uint32_t bk = 0u, bi = 0xFFFFFFFFu;
+#pragma unroll
+        for (int r = 0; r < kTkCand / 32; ++r) {
+            if (ck[r] > bk || (ck[r] == bk && ci[r] < bi)) {
+                bk = ck[r];
+                bi = ci[r];
+            }
+        }
+        const uint32_t K = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t win = __reduce_min_sync(0xffffffffu, bk == K ? bi : 0xFFFFFFFFu);
+        if (lane == 0) {
+            idx_out[j] = (int32_t)win;
+            w_out[j] = fkey_value(K);
+        }
+#pragma unroll
+        for (int r = 0; r < kTkCand / 32; ++r)
+            if (ci[r] == win) ck[r] = 0u;
+    }
+    __syncwarp();
+    float num = 0.f;
+    if (lane < k) {
+        const float lv = sel_bias ? __ldcg(row + idx_out[lane]) : w_out[lane];
+        num = expf(lv - m);
+    }
+    float w = num / z;
+    if (renorm) {
+        float zz = num;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
+        w = num / zz;
+    }
+    __syncwarp();
+    if (lane < k) w_out[lane] = w;
+    __syncwarp();
+    return true;
+}
+
 // --------------------------------------------------------------- kernel --
+// kTc: the tokens of the pass when fixed at compile time (1: one decode
+// token, every per-token loop folds to one iteration and the code the SM
+// fetches shrinks accordingly), 0: from the parameters.  kSf: the A scale
+// boxes come by TMA (both reduction lengths multiples of 512), fixed at
+// compile time; false: from the parameters.
+template <int kTc, bool kSf>
 __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_constant__ LayerParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const RouteParams &rp = p.r;
     const Layout &L = rp.L;
-    const int nst = p.nst, SB = p.sb, Tc = rp.Tc, N = act_n(Tc);
+    const int nst = p.nst, SB = p.sb, Tc = kTc > 0 ? kTc : rp.Tc, N = act_n(Tc);
+    const bool sf_gu = kSf || p.sf_tma_gu, sf_dn = kSf || p.sf_tma_dn;
+    // accumulator chains: each matrix slot of 64 columns holds Q chains of W
+    // columns (independent MMAs overlap in the tensor pipe; the epilogue sums)
+    const int Q = N <= 32 ? 2 : 1, W = 64 / Q;
     const int d = rp.d, E = rp.E, k = rp.k;
     const LkSmem so = lk_smem(E, k, Tc, d);
     uint8_t *tail = smem + nst * SB;
@@ -278,7 +439,8 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
     uint64_t *rnready = mdone + 1;  // the tokens' 1 / rms are in shared memory (pre-norm)
     uint64_t *rdready = rnready + 1;  // every router row is in (warp 0 polled router_done)
     uint64_t *tkready = rdready + 1;  // the top-k warps are done (picks in shared memory)
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(tkready + 1);
+    uint64_t *tkpart = tkready + 1;   // the four parts of a one-token top-k are posted
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(tkpart + 1);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tslot + 1);
     volatile int *s_U = s_abort + 1;
     volatile int *s_last = s_abort + 2;
@@ -314,6 +476,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
         mbar_init(rnready, 1);
         mbar_init(rdready, 1);
         mbar_init(tkready, kLTopkWarps);
+        mbar_init(tkpart, 4);
         fence_mbar_init();
         *s_abort = 0;
         *s_U = 0;
@@ -326,6 +489,27 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
     __syncthreads();
     umma::fence_after();
     const uint32_t tbase = *tslot;
+    // Zero a buffer's accumulator chains (this warp's lane quadrant): at the
+    // start, and by the epilogue after reading them, so every MMA accumulates.
+    auto zero_acc = [&](int buf) {
+        const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+                if (q < Q)
+#pragma unroll
+                    for (int n0 = 0; n0 < kNMax; n0 += 8)
+                        if (n0 < N) umma::st8(tbase + umma::lane_base(warp) + (uint32_t)(buf * 128 + m * 64 + q * W + n0), z);
+        umma::wait_st();
+    };
+    if (warp < 4) {
+        zero_acc(0);
+        zero_acc(1);
+    }
+    umma::fence_before();
+    __syncthreads();
+    umma::fence_after();
     // TMEM columns: accumulators [buf][mat] at (2*buf + mat) * 64 (N <= 48),
     // then kLSfc scale columns per stage: A box 0 (+0), A box 1 (+8), B tile
     // 0 (+16), B tile 1 (+24).
@@ -476,12 +660,6 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
         } else {
             // one poller per CTA (the counter's line is shared by the whole
             // grid); the other top-k warps wait on rdready
-            if (warp == 0) {
-                // a first pass of the top-k code on a stand-in row (the first E
-                // router weights; picks overwritten below) while the router
-                // rows are summed: the code is fetched now, not on the path
-                warp_topk(rp.wr, E, k, s_tidx, s_tw, nullptr, false, s_tk);
-            }
             if (lane == 0) {
                 if (warp == 0) {
                     if (!spin_geq(&hdr->router_done, (uint32_t)E, rp.wait_ns, s_abort)) {
@@ -503,10 +681,34 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
         }
         if (ok && p.mode != kLayerRouted) {
             const float *logits = reinterpret_cast<const float *>(rp.ws + L.logits);
-            for (int t = tw; t < Tc; t += kLTopkWarps)
-                warp_topk(logits + (size_t)t * E, E, k, s_tidx + t * 32, s_tw + t * 32,
-                          (rp.route_flags & kRouteBiasSelect) ? rp.bias : nullptr, (rp.route_flags & kRouteRenorm) != 0,
-                          s_tk + tw * 2 * kTkCand);
+            const float *sb = (rp.route_flags & kRouteBiasSelect) ? rp.bias : nullptr;
+            const bool rn = (rp.route_flags & kRouteRenorm) != 0;
+            if (Tc == 1) {
+                // one token: a quarter of the row per warp 0-3, merged by warp 0
+                if (warp < 4) {
+                    const int per = (E + 3) / 4;
+                    const int e0 = warp * per, e1 = min(E, e0 + per);
+                    warp_topk_part(logits, e0, e1, k, sb, s_tk + warp * kTkWords);
+                    __syncwarp();
+                    if (lane == 0)
+                        asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(tkpart)) : "memory");
+                    if (warp == 0) {
+                        int all = 1;
+                        if (lane == 0) all = mbar_wait_bounded(tkpart, 0u, hdr, rp.wait_ns) ? 1 : 0;
+                        all = __shfl_sync(0xffffffffu, all, 0);
+                        if (all) {
+                            (void)mbar_try_wait(tkpart, 0u);
+                            if (!warp_topk_merge(logits, k, s_tidx, s_tw, sb, rn, s_tk))
+                                warp_topk(logits, E, k, s_tidx, s_tw, sb, rn, s_tk + 4 * kTkWords);
+                        } else {
+                            *s_abort = 1;
+                        }
+                    }
+                }
+            } else {
+                for (int t = tw; t < Tc; t += kLTopkWarps)
+                    warp_topk(logits + (size_t)t * E, E, k, s_tidx + t * 32, s_tw + t * 32, sb, rn, s_tk + tw * kTkWords);
+            }
         }
         // the picks are in shared memory: each top-k warp counts on tkready,
         // the dispatching warp waits for all of them
@@ -603,7 +805,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
             auto issue_b = [&](int s, const Unit &x) {
                 uint8_t *st = smem + s * SB;
                 // the B scale words travel with the stage when the A scales do
-                const bool sfb = x.kind == 3 && p.sf_tma_dn && s_blob[x.u] != nullptr;
+                const bool sfb = x.kind == 3 && sf_dn && s_blob[x.u] != nullptr;
                 for (int tt = 0; tt < x.nt; ++tt) {
                     const size_t bt = x.kind == 3 ? (size_t)x.u * nkt_ff + x.kt + tt : (size_t)(x.kt + tt);
                     const uint8_t *bsrc = x.kind == 3 ? rp.ws + L.hb + bt * N * 128 : rp.ws + L.hsb + bt * N * 128;
@@ -677,7 +879,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                         scmaps = em + (x.kind == 2 ? 384 : 640);
                         blob_ok = s_blob[x.u] != nullptr;
                     }
-                    const bool sf_dma = blob_ok && ((x.kind == 2 && p.sf_tma_gu) || (x.kind == 3 && p.sf_tma_dn));
+                    const bool sf_dma = blob_ok && ((x.kind == 2 && sf_gu) || (x.kind == 3 && sf_dn));
                     // bytes: A boxes, B tiles, A scale box(es), B scale words
                     uint32_t tx = 0u;
                     const int nbox = (x.kind == 1 || x.kind == 2) ? 2 : x.nt;
@@ -935,7 +1137,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                     if (x.kind == 2 || x.kind == 3) {
                         const uint8_t *blob = s_blob[x.u];
                         const bool has = blob != nullptr;
-                        const bool tma_sc = x.kind == 2 ? p.sf_tma_gu : p.sf_tma_dn;
+                        const bool tma_sc = x.kind == 2 ? sf_gu : sf_dn;
                         const uint32_t col = tbase + lb + sf0 + (uint32_t)(s * kLSfc);
                         const int K = x.kind == 2 ? d : ff, M = x.kind == 2 ? ff : d;
                         const int nbox = x.kind == 2 ? 2 : x.nt;
@@ -1045,7 +1247,9 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                     if (seg >= 2 && !wait(&aempty[buf], (uint32_t)(((seg >> 1) + 1) & 1))) break;
                     umma::fence_after();
                     const uint32_t dcol = tbase + (uint32_t)(buf * 128);
-                    uint32_t acc = 0u;
+                    // the epilogue zeroes every accumulator after reading it (and
+                    // all of them at the start), so each MMA accumulates
+                    constexpr uint32_t acc = 1u;
                     for (int un = unit; un < seg_end; ++un, ++i) {
                         if (un != unit) x = decode(r, un);
                         const int s = i % nst;
@@ -1061,15 +1265,16 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                         const uint64_t a0 = adesc0 + soff, b0 = bdesc0 + soff;
                         const uint32_t sfc = tbase + sf0 + (uint32_t)(s * kLSfc);
                         if (x.kind == 1) {
-                            // shared gate/up: bf16, W_g -> acc 0, W_u -> acc 1
+                            // shared gate/up: bf16, W_g -> matrix 0, W_u -> matrix 1,
+                            // k-step sk into chain sk mod Q of its matrix
                             const int nks = min(4, (d - x.kt * kTileKs) / 16);
 #pragma unroll
                             for (int sk = 0; sk < 4; ++sk) {
                                 if (sk < nks) {
                                     const uint64_t bd = b0 + sk * bstep;
-                                    umma::mma_bf16(dcol, a0 + 2 * sk, bd, idesc16, acc);
-                                    umma::mma_bf16(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, idesc16, acc);
-                                    acc = 1u;
+                                    const uint32_t cq = (uint32_t)((sk % Q) * W);
+                                    umma::mma_bf16(dcol + cq, a0 + 2 * sk, bd, idesc16, acc);
+                                    umma::mma_bf16(dcol + 64 + cq, a0 + (kAtile >> 4) + 2 * sk, bd, idesc16, acc);
                                 }
                             }
                         } else if (x.kind == 2) {
@@ -1078,16 +1283,18 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                             for (int sk = 0; sk < 4; ++sk) {
                                 if (sk < nks) {
                                     const uint64_t bd = b0 + sk * bstep;
+                                    const uint32_t cq = (uint32_t)((sk % Q) * W);
                                     const uint32_t sfid = (uint32_t)(2 * (sk & 1)) << 30;
                                     const uint32_t sfb = (sfc + 16 + (sk >> 1) * 4) | sfid;
-                                    umma::mma_mxf4(dcol, a0 + 2 * sk, bd, id4[sk & 1], acc, (sfc + (sk >> 1) * 4) | sfid, sfb);
-                                    umma::mma_mxf4(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, id4[sk & 1], acc,
+                                    umma::mma_mxf4(dcol + cq, a0 + 2 * sk, bd, id4[sk & 1], acc, (sfc + (sk >> 1) * 4) | sfid, sfb);
+                                    umma::mma_mxf4(dcol + 64 + cq, a0 + (kAtile >> 4) + 2 * sk, bd, id4[sk & 1], acc,
                                                    (sfc + 8 + (sk >> 1) * 4) | sfid, sfb);
-                                    acc = 1u;
                                 }
                             }
                         } else {
-                            // down: K-tiles kt, kt + 1 (A box tt, B tile tt) into acc 0
+                            // down: K-tiles kt, kt + 1 (A box tt, B tile tt); MMA j
+                            // (= 4 tt + sk) into chain j mod 2Q (matrix slots of
+                            // both halves: the epilogue sums them all)
                             for (int tt = 0; tt < x.nt; ++tt) {
                                 const uint64_t at = a0 + (uint32_t)(tt * (kAtile >> 4));
                                 const uint64_t bt = b0 + tt * btile;
@@ -1096,11 +1303,12 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
 #pragma unroll
                                     for (int sk = 0; sk < 4; ++sk) {
                                         if (sk < nks) {
+                                            const int c = (4 * tt + sk) % (2 * Q);
+                                            const uint32_t cc = (uint32_t)((c / Q) * 64 + (c % Q) * W);
                                             const uint32_t sfid = (uint32_t)(2 * (sk & 1)) << 30;
-                                            umma::mma_mxf4(dcol, at + 2 * sk, bt + sk * bstep, id4[sk & 1], acc,
+                                            umma::mma_mxf4(dcol + cc, at + 2 * sk, bt + sk * bstep, id4[sk & 1], acc,
                                                            (sfc + 8 * tt + (sk >> 1) * 4) | sfid,
                                                            (sfc + 16 + 8 * tt + (sk >> 1) * 4) | sfid);
-                                            acc = 1u;
                                         }
                                     }
                                 } else {
@@ -1108,8 +1316,9 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
 #pragma unroll
                                     for (int sk = 0; sk < 4; ++sk) {
                                         if (sk < nks) {
-                                            umma::mma_bf16(dcol, at + 2 * sk, bt + sk * bstep, idesc16, acc);
-                                            acc = 1u;
+                                            const int c = (4 * tt + sk) % (2 * Q);
+                                            const uint32_t cc = (uint32_t)((c / Q) * 64 + (c % Q) * W);
+                                            umma::mma_bf16(dcol + cc, at + 2 * sk, bt + sk * bstep, idesc16, acc);
                                         }
                                     }
                                 }
@@ -1138,9 +1347,9 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
             // the four warps agree on going on (they share named barrier 1)
             if (r == 2 && !umma::bar_red_and(1, 128, routed_ranges(true))) break;
             const Range R = rgr(r);
+            const int NM = r == 3 ? 1 : 2;
             uint32_t *icnt = reinterpret_cast<uint32_t *>(rp.ws + L.icnt) +
                              (r == 1 ? L.umax * nrb_ff : (r == 2 ? 0 : L.umax * nrb_ff + nrbs));
-            const int NM = r == 3 ? 1 : 2;
             for (int unit = R.a; unit < R.b; ++seg) {
                 const Unit x = decode(r, unit);
                 const int item = x.item;
@@ -1156,24 +1365,37 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_kernel(const __grid_consta
                 if (lane == 0) wait(&afull[buf], (uint32_t)((seg >> 1) & 1));
                 __syncwarp();
                 umma::fence_after();
+                // matrix m's chains (R3: both matrix slots hold chains of the one
+                // output); then zero them for the MMAs of this buffer's next use
 #pragma unroll
                 for (int m = 0; m < 2; ++m) {
-                    if (m < NM) {
 #pragma unroll
-                        for (int n0 = 0; n0 < kNMax; n0 += 8) {
-                            if (n0 < N) {
-                                uint32_t v[8];
-                                umma::ld8(tbase + lb + (uint32_t)((buf * 2 + m) * 64 + n0), v);
-                                umma::wait_ld();
+                    for (int q = 0; q < 2; ++q) {
+                        if (q < Q) {
 #pragma unroll
-                                for (int jj = 0; jj < 8; ++jj) {
-                                    const int t = (n0 + jj) / kPieces;
-                                    if (t < kChunk) acc[m][t] += __uint_as_float(v[jj]);
+                            for (int n0 = 0; n0 < kNMax; n0 += 8) {
+                                if (n0 < N) {
+                                    uint32_t v[8];
+                                    umma::ld8(tbase + lb + (uint32_t)(buf * 128 + m * 64 + q * W + n0), v);
+                                    umma::wait_ld();
+#pragma unroll
+                                    for (int jj = 0; jj < 8; ++jj) {
+                                        const int t = (n0 + jj) / kPieces;
+                                        if (t < kChunk) acc[m][t] += __uint_as_float(v[jj]);
+                                    }
                                 }
                             }
                         }
                     }
                 }
+                if (r == 3) {
+#pragma unroll
+                    for (int t = 0; t < kChunk; ++t) {
+                        acc[0][t] += acc[1][t];
+                        acc[1][t] = 0.f;
+                    }
+                }
+                zero_acc(buf);
                 umma::fence_before();
                 __syncwarp();
                 if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&aempty[buf])) : "memory");
