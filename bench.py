@@ -320,6 +320,8 @@ def main():
                     help="also time one token through this many K3 MoE layers in a row (0: skip)")
     ap.add_argument("--cache-slots", type=int, nargs="*", default=[64, 128, 256],
                     help="expert-cache slot counts to simulate (the middle one also timed); none: skip")
+    ap.add_argument("--one-launch", action="store_true",
+                    help="decode passes as one cooperative launch (K3MOE_ONE_LAUNCH) instead of three")
     ap.add_argument("--no-configs", action="store_true",
                     help="measure the headline workload only (not the T=8 / prefill workloads)")
     ap.add_argument("--experts", type=int, default=None,
@@ -369,8 +371,12 @@ def main():
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
-    head = measure(cfg, W, k3, args, flush_l2, stream, world, e2e=not args.quick)
+    head = measure(cfg, W, k3, args, flush_l2, stream, world, e2e=not args.quick, one_launch=args.one_launch)
     others = {}
+    alt = None
+    if args.config == "k3_decode" and args.experts is None and not args.quick and not args.no_configs:
+        # the other decode implementation on the same workload (K3MOE_ONE_LAUNCH toggled)
+        alt = measure(cfg, W, k3, args, flush_l2, stream, world, e2e=False, one_launch=not args.one_launch)
     if args.config == "k3_decode" and args.experts is None and not args.quick and not args.no_configs:
         for name in ("k3_decode_t8", "k3_prefill_512", "k3_prefill_4096"):
             others[name] = measure(k3gen.CONFIGS[name], W, k3, args, flush_l2, stream, world, e2e=False)
@@ -416,6 +422,10 @@ def main():
         "gpu_launches": head["launches"] * args.steps,
         "clocks": clk,
     }
+    line["config"]["decode"] = "one launch (K3MOE_ONE_LAUNCH)" if args.one_launch else "three launches (default)"
+    if alt is not None:
+        line["other_decode"] = dict(summary(alt, peak),
+                                    decode="three launches (default)" if args.one_launch else "one launch (K3MOE_ONE_LAUNCH)")
     if others:
         line["configs"] = {name: summary(r, peak) for name, r in others.items()}
     if model is not None:
@@ -608,7 +618,7 @@ def kernel_bytes(cfg, U, pairs, name):
             "expert_down": down_bytes(cfg, U, pairs), "layer": alg_bytes(cfg, U)}.get(name)
 
 
-def measure(cfg, W, k3, args, flush_l2, stream, world, e2e=False):
+def measure(cfg, W, k3, args, flush_l2, stream, world, e2e=False, one_launch=False):
     """W warm-up and K timed layer calls on one workload (L2 flushed before
     each, CUDA events on the launching stream, max over ranks); for passes of
     up to 8 tokens also K calls with events between the library's kernels,
@@ -618,7 +628,7 @@ def measure(cfg, W, k3, args, flush_l2, stream, world, e2e=False):
     inp = kdev.DeviceInputs(cfg)
     T = inp.T
     dims = k3.make_dims(cfg.d, cfg.ff, cfg.E, cfg.k, cfg.ff_shared,
-                        k3.K3MOE_OUT_FP32 if cfg.out_fp32 else 0)
+                        (k3.K3MOE_OUT_FP32 if cfg.out_fp32 else 0) | (k3.K3MOE_ONE_LAUNCH if one_launch else 0))
     ws = k3.new_workspace(dims, T, host_staging=e2e)
     ybytes = 4 if cfg.out_fp32 else 2
     y = torch.empty((T, cfg.d), dtype=torch.float32 if cfg.out_fp32 else torch.int16, device="cuda")

@@ -119,6 +119,15 @@ typedef enum {
  * both). */
 #define K3MOE_RENORM_TOPK 8u
 #define K3MOE_BIAS_SELECT_ONLY 16u
+/* Decode passes (T <= 8 tokens per pass) as one cooperative launch (router,
+ * top-k, gate/up, down and combine in one kernel, the shared expert's gate/up
+ * streamed while the routing is decided) instead of the default three
+ * launches (route; gate/up; down).  Same results within the output tolerance
+ * (the partial sums are added in another order); the routing of the two may
+ * differ only where two logits tie to the last bit.  Shapes the one-launch
+ * kernel does not take (d > 8192, too many router rows per CTA) run the
+ * three launches. */
+#define K3MOE_ONE_LAUNCH 32u
 
 /*
  * Layer dimensions.  d and ff: multiples of 64, 64 <= d <= 8192,

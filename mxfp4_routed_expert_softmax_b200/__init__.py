@@ -28,6 +28,7 @@ K3MOE_NO_SHARED = 2
 K3MOE_STRICT = 4
 K3MOE_RENORM_TOPK = 8
 K3MOE_BIAS_SELECT_ONLY = 16
+K3MOE_ONE_LAUNCH = 32
 
 
 class K3moeError(RuntimeError):

@@ -115,7 +115,8 @@ int umma_stages(bool gu, int N) {
 
 k3moe_status check_dims(const k3moe_dims *dm) {
     if (!dm) return K3MOE_ERR_INVALID_ARGUMENT;
-    if (dm->flags & ~(K3MOE_OUT_FP32 | K3MOE_NO_SHARED | K3MOE_STRICT | K3MOE_RENORM_TOPK | K3MOE_BIAS_SELECT_ONLY))
+    if (dm->flags & ~(K3MOE_OUT_FP32 | K3MOE_NO_SHARED | K3MOE_STRICT | K3MOE_RENORM_TOPK | K3MOE_BIAS_SELECT_ONLY |
+                      K3MOE_ONE_LAUNCH))
         return K3MOE_ERR_INVALID_ARGUMENT;
     if (dm->d < 64 || dm->d > 8192 || dm->d % 64) return K3MOE_ERR_UNSUPPORTED_SHAPE;
     if (dm->ff < 64 || dm->ff > 3072 || dm->ff % 64) return K3MOE_ERR_UNSUPPORTED_SHAPE;
@@ -361,9 +362,9 @@ cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st, int *g
     return cudaLaunchKernelEx(&cfg, route_kernel, rp);
 }
 
-// TEMP: the one-launch decode kernel serves only the pre-norm calls until it
-// has been checked on the GPU.
-constexpr bool kUseLayerKernel = false;
+// Decode passes of this call by the one-launch kernel (K3MOE_ONE_LAUNCH);
+// the pre-norm and routing-given calls take it whatever the flag.
+inline bool one_launch(const k3moe_dims *dm) { return (dm->flags & K3MOE_ONE_LAUNCH) != 0; }
 
 // The one-launch decode pass (layer_kernel) for this shape, if it fits: the
 // pipeline stages and the routing tables in one SM's shared memory, and the
@@ -673,7 +674,7 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         EventHook none;
         EventHook &hk = hook ? *hook : none;
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
-        const int lst = (kUseLayerKernel || norm_w || layer_mode != kLayerFull) ? layer_stages(*di, dims, Tc) : 0;
+        const int lst = (one_launch(dims) || norm_w || layer_mode != kLayerFull) ? layer_stages(*di, dims, Tc) : 0;
         if (layer_mode != kLayerFull && lst == 0) return K3MOE_ERR_UNSUPPORTED_SHAPE;
         if (lst > 0) {
             // the whole pass in one launch
@@ -849,7 +850,7 @@ k3moe_status k3moe_route(const void *x, int32_t T, const float *w_router, const 
         rp.route_flags = route_flags(dims);
         rp.idx_out = idx + (size_t)c0 * dims->top_k;
         rp.w_out = weight + (size_t)c0 * dims->top_k;
-        const int lst = kUseLayerKernel ? layer_stages(*di, dims, Tc) : 0;
+        const int lst = one_launch(dims) ? layer_stages(*di, dims, Tc) : 0;
         cudaError_t e = lst > 0 ? launch_layer_route(*di, rp, lst, st, dims->ff % 512 == 0) : launch_route(*di, rp, st);
         if (e != cudaSuccess) return cuda_fail(e);
     }
@@ -1095,7 +1096,7 @@ k3moe_status k3moe_layer_cached(k3moe_cache *cache, const void *x, int32_t T, co
         rp.route_flags = route_flags(dims);
         // the routing by the kernel the layer call will use, so the experts
         // fetched are exactly the ones its dispatch takes
-        const int lst = kUseLayerKernel ? layer_stages(*di, dims, Tc) : 0;
+        const int lst = one_launch(dims) ? layer_stages(*di, dims, Tc) : 0;
         cudaError_t e = lst > 0 ? launch_layer_route(*di, rp, lst, st, dims->ff % 512 == 0) : launch_route(*di, rp, st);
         if (e != cudaSuccess) return cuda_fail(e, "router launch");
         e = cudaMemcpyAsync(idx_host + (size_t)c0 * k, reinterpret_cast<uint8_t *>(ws) + L.idx,

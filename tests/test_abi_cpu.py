@@ -81,7 +81,7 @@ A16 = 0x10000  # a fake 16-byte aligned address: never dereferenced, calls fail 
     ((7168, 1536, 896, 33, 1536, 0), 1),     # k > 32
     ((256, 128, 4, 5, 128, 0), 1),           # k > E
     ((7168, 1536, 896, 16, 100, 0), 2),      # shared width not a multiple of 64
-    ((7168, 1536, 896, 16, 1536, 32), 1),    # unknown flag
+    ((7168, 1536, 896, 16, 1536, 64), 1),    # unknown flag
     ((7168, 8192, 896, 16, 1536, 0), 2),     # down tile does not fit shared memory
 ])
 def test_layer_rejects_bad_dims(m, dims, want):
@@ -140,7 +140,7 @@ def test_product_path_has_no_oracle_reference():
                 assert "oracle" not in text.lower(), f
 
 
-@pytest.mark.parametrize("flag", ["K3MOE_STRICT", "K3MOE_RENORM_TOPK", "K3MOE_BIAS_SELECT_ONLY"])
+@pytest.mark.parametrize("flag", ["K3MOE_STRICT", "K3MOE_RENORM_TOPK", "K3MOE_BIAS_SELECT_ONLY", "K3MOE_ONE_LAUNCH"])
 def test_option_flags_are_accepted(m, flag):
     """The option flags pass validation (the call then fails only on the tiny
     workspace size, before anything is launched)."""

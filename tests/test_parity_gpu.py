@@ -274,3 +274,29 @@ def test_grouped_prefill_deterministic_and_multi_pass(orc):
     yo, problems, _, _, _, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx, tokens)
     assert not problems
     assert g1_error(y[tokens], yo).max() <= G1_TOL
+
+
+@pytest.mark.parametrize("name,T", [("tiny", 1), ("tiny", 4), ("k3_decode", 1), ("k3_decode_t8", 8), ("k3_decode", 3)])
+def test_one_launch_parity(orc, name, T):
+    """K3MOE_ONE_LAUNCH: the decode pass as one cooperative launch, against the
+    oracle on every token, bf16 = RNE(fp32), and against the three launches."""
+    cfg = k3gen.CONFIGS[name]
+    W = kdev.weights(cfg)
+    inp = kdev.DeviceInputs(cfg, T=T)
+    one = m.K3MOE_ONE_LAUNCH
+    y32, idx, w = run_layer(cfg, W, inp.x, inp.bias, T, m.K3MOE_OUT_FP32 | one, ws_tokens=min(T, 8))
+    y16, idx2, w2 = run_layer(cfg, W, inp.x, inp.bias, T, one, ws_tokens=min(T, 8))
+    assert np.array_equal(idx, idx2) and np.array_equal(w, w2)
+    r = torch.from_numpy(y32).to(torch.bfloat16).view(torch.int16).numpy()
+    assert np.array_equal(r, y16), "bf16 output is not RNE(fp32 output)"
+    tokens = list(range(T))
+    yo, problems, nd, probs, idx_use, _ = oracle_reference(orc, cfg, W, inp.x_host, inp.bias_host, idx, tokens)
+    assert not problems, problems[:5]
+    wref = np.take_along_axis(probs, idx.astype(np.int64), axis=1)
+    assert np.allclose(w, wref, rtol=1e-5, atol=1e-7)
+    err = g1_error(y32, yo)
+    assert err.max() <= G1_TOL, (err.max(), err)
+    # the three-launch pass on the same inputs: same picks, outputs within the gate
+    y3, idx3, _ = run_layer(cfg, W, inp.x, inp.bias, T, m.K3MOE_OUT_FP32, ws_tokens=min(T, 8))
+    assert np.array_equal(idx, idx3)
+    assert g1_error(y3, y32).max() <= G1_TOL
