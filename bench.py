@@ -324,6 +324,9 @@ def main():
                     help="decode passes as one cooperative launch (K3MOE_ONE_LAUNCH) instead of three")
     ap.add_argument("--no-configs", action="store_true",
                     help="measure the headline workload only (not the T=8 / prefill workloads)")
+    ap.add_argument("--route-only", action="store_true",
+                    help="profiling: time the routing alone (k3moe_route: router, softmax, top-k) on "
+                         "the workload's router; only the router and x are on the device")
     ap.add_argument("--experts", type=int, default=None,
                     help="profiling: keep only this many experts resident (same d, ff, top-k); the "
                          "routed and shared bytes per token stay those of the workload, the router shrinks")
@@ -352,6 +355,10 @@ def main():
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    if args.route_only:
+        measure_route_only(cfg, k3, args)
+        return
 
     W = kdev.weights(cfg)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -616,6 +623,40 @@ def kernel_names(n):
 def kernel_bytes(cfg, U, pairs, name):
     return {"route": route_bytes(cfg), "expert_gu": gu_bytes(cfg, U, pairs),
             "expert_down": down_bytes(cfg, U, pairs), "layer": alg_bytes(cfg, U)}.get(name)
+
+
+def measure_route_only(cfg, k3, args):
+    """Profiling mode: W warm-up and K timed k3moe_route calls (the router
+    GEMV, softmax and top-k of the workload's first T tokens), L2 flushed
+    before each, CUDA events on the launching stream; prints one JSON line
+    (not a bench line: the routing alone)."""
+    import torch
+    wr = torch.from_numpy(k3gen.router(cfg)).cuda()
+    b = k3gen.bias(cfg)
+    bias = torch.from_numpy(b).cuda() if b is not None else None
+    T = min(cfg.T, 8)
+    x = torch.from_numpy(k3gen.hidden(cfg, T=T).view(np.int16)).cuda()
+    dims = k3.make_dims(cfg.d, cfg.ff, cfg.E, cfg.k, cfg.ff_shared, 0)
+    ws = k3.new_workspace(dims, T)
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ms = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 255)
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        k3.check(k3.k3moe_route(x, T, wr, bias, dims, idx, wts, ws), "k3moe_route")
+        e.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            ms.append(a.elapsed_time(e))
+    k3.check(k3.k3moe_device_status(ws), "device status")
+    us = 1000.0 * sum(ms) / len(ms)
+    nbytes = cfg.E * cfg.d * 4 + T * cfg.d * 2
+    print(json.dumps({"mode": "route-only", "workload": workload_desc(cfg), "tokens": T, "steps": args.steps,
+                      "us_per_call": round(us, 2), "us_min": round(1000.0 * min(ms), 2),
+                      "router_gbs": round(nbytes / (us * 1e-6) / 1e9, 1)}), flush=True)
 
 
 def measure(cfg, W, k3, args, flush_l2, stream, world, e2e=False, one_launch=False):

@@ -161,13 +161,15 @@ __device__ __forceinline__ uint32_t ld_relaxed(const uint32_t *p) {
     return v;
 }
 
-// Wait until *ctr >= target: relaxed polls with a short sleep, then one
-// acquire fence (a relaxed read that sees the producers' release, followed by
-// the fence, orders everything they published before this thread's later
-// reads), so the acquire is paid once and not on every poll.  False after
+// Wait until *ctr >= target: one acquire load first (the count is often
+// there already); else relaxed polls with a short sleep, then one acquire
+// fence (a relaxed read that sees the producers' release, followed by the
+// fence, orders everything they published before this thread's later reads),
+// so the acquire is paid once and not on every poll.  False after
 // limit_ns, or at once when *abort (if given) becomes nonzero.
 __device__ __forceinline__ bool spin_geq(const uint32_t *ctr, uint32_t target, uint64_t limit_ns,
                                          const volatile int *abort = nullptr) {
+    if (ld_acquire(ctr) >= target) return true;  // already there: one acquire load, no fence
     if (ld_relaxed(ctr) < target) {
         const uint64_t t0 = globaltimer();
         do {
@@ -183,6 +185,15 @@ __device__ __forceinline__ bool spin_geq(const uint32_t *ctr, uint32_t target, u
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// 8-byte asynchronous copy global -> shared (no register staging); complete
+// after cp_async_wait_all.  Both addresses 8-byte aligned.
+__device__ __forceinline__ void cp_async8(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n cp.async.wait_all;" ::: "memory");
 }
 
 // --------------------------------------------------------------- formats --

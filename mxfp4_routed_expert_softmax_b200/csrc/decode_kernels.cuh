@@ -1,12 +1,12 @@
 // Routing of one token chunk (up to kChunk tokens): the router GEMV on its
-// fp32 weights, streamed by warps over equal slices of the weight bytes (a
-// row split between warps is summed by the last one to finish, in a fixed
-// order); one CTA waits for every router row, then runs the softmax over all
-// experts, the top-k and the dispatch (distinct experts, their tensor maps).
-// Every CTA first builds its share of the activation pieces the tensor-core
-// gate/up pass reads.  Layer structure: the tutorial page's section 2.4
-// moe_forward (route, per selected expert FFN, weighted combine); the expert
-// FFNs themselves are in umma_kernels.cuh.
+// fp32 weights, streamed by warps with plain loads over equal ranges of row
+// parts (a row's parts are summed by the last one to finish, in part order);
+// one CTA per token waits for every router row, then runs the softmax over
+// all experts and the token's top-k; CTA 0 dispatches (distinct experts, their
+// slots and blob pointers).  The same CTAs first build the activation pieces
+// the tensor-core gate/up pass reads.  Layer structure: the tutorial page's
+// section 2.4 moe_forward (route, per selected expert FFN, weighted combine);
+// the expert FFNs themselves are in umma_kernels.cuh.
 #pragma once
 
 #include "common.cuh"
@@ -28,7 +28,7 @@ struct RouteParams {
     const uint8_t *const *blobs;  // device array [E], null: no dispatch (route only)
     int32_t *idx_out;   // optional [Tc][k]
     float *w_out;       // optional [Tc][k]
-    int nstage;         // router ring stages (kRStage bytes each)
+    int nded;           // CTAs 0 .. nded-1 run no router stream (pieces, top-k, dispatch)
     uint4 tmpl[4][8];   // tensor-map templates: W_g/W_u, W_d nibble planes; their scale planes
     int scale_mask;     // which scale-plane templates exist (bit 0: W_g/W_u, bit 1: W_d)
     uint4 smap[3][8];   // shared expert tensor maps (W_g, W_u, W_d), when has_shared
@@ -43,7 +43,12 @@ constexpr int kRouteThreads = 256;
 // moving only the selection (the logits and the softmax stay unbiased).
 constexpr int kRouteRenorm = 1;
 constexpr int kRouteBiasSelect = 2;
-constexpr int kRouteTok = 4;  // tokens per pass over the rows (x kept in smem as fp32)
+constexpr int kRouteTok = 4;  // tokens per pass over the router (their x columns held in registers)
+// the router partial sums are double-buffered by pass parity: at most two passes
+static_assert(kChunk <= 2 * kRouteTok, "a chunk takes at most two router passes");
+// Dynamic shared memory of the route kernel: CTA 0's copies of the blob
+// pointer table and of the maps' blob pointers, and a placeholder row.
+__host__ __device__ inline int route_dyn_bytes(int E) { return E * (8 + 8 + 4); }
 
 // Order-preserving 32-bit key of a float (larger float -> larger key; -0 is
 // first made +0 so that equal values have equal keys) and its inverse.
@@ -81,8 +86,14 @@ __device__ __forceinline__ uint32_t block_scan_incl(uint32_t v, uint32_t *s_tot)
 // sel_bias (non-null): the selection runs on logit + sel_bias[e] while the
 // softmax stays on the logits; renorm: the k weights are divided by their
 // sum (in pick order).
-__device__ void cta_topk_row(const float *row, int E, int k, int32_t *idx_row, float *w_row, int32_t *idx_out_row,
-                             float *w_out_row, const float *sel_bias = nullptr, bool renorm = false) {
+// idx_sh (optional, shared memory): the picks again, for a dispatch by the
+// same CTA.  row_shared: row is in shared memory (else global, written by
+// other CTAs: read through L2).  Not inlined: one copy of the code serves
+// every call, so a call on placeholder data warms the instruction caches for
+// the real one.
+__device__ __noinline__ void cta_topk_row(const float *row, int E, int k, int32_t *idx_row, float *w_row,
+                                          int32_t *idx_out_row, float *w_out_row, const float *sel_bias,
+                                          bool renorm, int32_t *idx_sh, bool row_shared) {
     __shared__ uint32_t s_hist[256];
     __shared__ uint32_t s_tot[8];
     __shared__ float s_red[2][8];
@@ -97,7 +108,7 @@ __device__ void cta_topk_row(const float *row, int E, int k, int32_t *idx_row, f
     for (int i = 0; i < 4; ++i) {
         const int e = 4 * tid + i;
         ok[i] = e < E;
-        v[i] = ok[i] ? __ldcg(row + e) : -INFINITY;
+        v[i] = ok[i] ? (row_shared ? row[e] : __ldcg(row + e)) : -INFINITY;
         key[i] = ok[i] ? fkey(sel_bias ? v[i] + __ldg(sel_bias + e) : v[i]) : 0u;  // real keys are > 0
         mx = fmaxf(mx, v[i]);
     }
@@ -196,7 +207,7 @@ __device__ void cta_topk_row(const float *row, int E, int k, int32_t *idx_row, f
     }
     // the pick's softmax numerator (its own logit: the key holds it unless
     // the selection was biased)
-    const float lv = lane < k ? (sel_bias ? __ldcg(row + mi) : fkey_value(mk)) : 0.f;
+    const float lv = lane < k ? (sel_bias ? (row_shared ? row[mi] : __ldcg(row + mi)) : fkey_value(mk)) : 0.f;
     float num = lane < k ? expf(lv - m) : 0.f;
     float w = num * inv_s;
     if (renorm) {
@@ -211,23 +222,14 @@ __device__ void cta_topk_row(const float *row, int E, int k, int32_t *idx_row, f
     if (lane < k) {
         idx_row[r] = (int32_t)mi;
         w_row[r] = w;
+        if (idx_sh) idx_sh[r] = (int32_t)mi;
         if (idx_out_row) idx_out_row[r] = (int32_t)mi;
         if (w_out_row) w_out_row[r] = w;
     }
 }
-// Token t of a decode chunk: logits, picks and weights in the workspace.
-__device__ void cta_topk(const RouteParams &p, int t) {
-    const int k = p.k;
-    cta_topk_row(reinterpret_cast<const float *>(p.ws + p.L.logits) + (size_t)t * p.E, p.E, k,
-                 reinterpret_cast<int32_t *>(p.ws + p.L.idx) + t * k, reinterpret_cast<float *>(p.ws + p.L.wt) + t * k,
-                 p.idx_out ? p.idx_out + (size_t)t * k : nullptr, p.w_out ? p.w_out + (size_t)t * k : nullptr,
-                 (p.route_flags & kRouteBiasSelect) ? p.bias : nullptr, (p.route_flags & kRouteRenorm) != 0);
-}
-
-// The dispatch of a chunk whose top-k is done: distinct experts in ascending
-// id, their token masks, the slot of each (expert, token), their blob
-// pointers (checked) and ids.  Run by one whole CTA.
-__device__ void dispatch(const RouteParams &p, WsHeader *hdr) {
+// ptab, tc: the blob pointer table and the maps' blob pointers, copied to
+// shared memory by the caller.
+__device__ void dispatch(const RouteParams &p, WsHeader *hdr, const uint8_t *const *ptab, const uint8_t **tc) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Layout &L = p.L;
     const int32_t *idx = reinterpret_cast<const int32_t *>(p.ws + L.idx);
@@ -274,7 +276,7 @@ __device__ void dispatch(const RouteParams &p, WsHeader *hdr) {
     for (int w = threadIdx.x; w < nwords * 32; w += blockDim.x) {
         if ((bitmap[w >> 5] >> (w & 31)) & 1u) {
             uint32_t u = prefix[w >> 5] + __popc(bitmap[w >> 5] & ((1u << (w & 31)) - 1u));
-            const uint8_t *b = p.blobs[w];
+            const uint8_t *b = ptab[w];
             if ((reinterpret_cast<uintptr_t>(b) & 15u) != 0u || b == nullptr) {
                 set_status(hdr, kStDeviceCheck);
                 b = nullptr;
@@ -282,6 +284,11 @@ __device__ void dispatch(const RouteParams &p, WsHeader *hdr) {
             ublob[u] = b;
             ueid[u] = w;
             gmask[u] = umask[u];
+            // the expert's tensor maps, rewritten when its blob pointer changed
+            if (b != nullptr && tc[w] != b) {
+                write_expert_tmaps(p.ws, L, w, b, p.tmpl, p.scale_mask);
+                reinterpret_cast<const uint8_t **>(p.ws + L.tcache)[w] = b;
+            }
         }
     }
 }
@@ -290,9 +297,11 @@ __device__ void dispatch(const RouteParams &p, WsHeader *hdr) {
 // when its blob pointer differs from the one they were written for (kept in
 // the workspace).  Thread i of n takes experts i, i + n, ...; index E is the
 // shared expert.
-__device__ void refresh_tmaps(const RouteParams &p, int i0, int n) {
+// Indices from i0 below e_end only (default: all of them).
+__device__ void refresh_tmaps(const RouteParams &p, int i0, int n, int e_end = -1) {
     const uint8_t **cache = reinterpret_cast<const uint8_t **>(p.ws + p.L.tcache);
-    for (int e = i0; e < p.E + 1; e += n) {
+    if (e_end < 0) e_end = p.E + 1;
+    for (int e = i0; e < e_end; e += n) {
         if (e < p.E) {
             const uint8_t *b = p.blobs[e];
             if (b != cache[e] && b != nullptr && (reinterpret_cast<uintptr_t>(b) & 15u) == 0u) {
@@ -310,234 +319,136 @@ __device__ void refresh_tmaps(const RouteParams &p, int i0, int n) {
     }
 }
 
-// Warp that holds chunk c when N chunks are split evenly over W warps
-// (warp j holds [floor(jN/W), floor((j+1)N/W))).
-__device__ __forceinline__ int chunk_owner(long long c, long long N, int W) {
-    return (int)(((c + 1) * (long long)W - 1) / N);
-}
-
 // ------------------------------------------------------ router stream --
-// Router GEMV l = W_r x + b.  The fp32 router is one array of E*d floats; CTA
-// c of G owns the contiguous units [c*U/G, (c+1)*U/G) of 16 floats (U =
-// E*d/16; rows are whole units since d is a multiple of 64).  Its slice goes
-// through a ring of kRStage-byte shared-memory stages filled by bulk
-// asynchronous copies, so one thread keeps the SM's memory pipe full.  Thread
-// i of a stage takes its 16 floats (one row), the warp sums lanes of equal
-// row with a fixed shuffle tree (segmented), and after the stage's barrier
-// threads fold the warps' row sums into the CTA's row accumulators in warp
-// order, so every sum has a fixed order.  Rows cut by a CTA boundary are
-// finished by the last of their CTAs to arrive, summing the CTAs' parts in
-// CTA order.
-constexpr int kRStage = 16384;               // bytes per ring stage
-constexpr int kRFloats = kRStage / 4;        // 4096 floats: 256 units of 16
-constexpr int kRSegs = 16;                   // row segments per warp and stage (512 floats, d >= 64)
-constexpr int kRMaxRows = 72;                // rows of one CTA's slice (E/G + 2 <= 66)
-constexpr int kRFast = 8;                    // slices of at most this many rows: per-thread row sums
+// Router GEMV l = W_r x + b.  Row r of the fp32 router is summed as P = d / Ls
+// parts of Ls floats (router_part_len); part q of row r is segment s = q*E + r
+// (part-major, so consecutive segments of a warp share their x columns).  The
+// streaming warps take equal contiguous ranges of the E*P segments.  A warp
+// reads a segment with plain 16-byte loads straight from HBM (no shared-memory
+// staging: several segments' loads are in flight per lane, so the SM's load
+// path, not its bulk-copy engine, sets the rate), multiplies it with the x
+// columns it holds in registers and sums the 32 lanes with a fixed butterfly.
+// The part's sum goes to the workspace; the last of a row's P parts to arrive
+// adds the P sums in part order (q = 0 .. P-1), so every logit has one fixed
+// summation order whatever the grid.
+// Segments whose loads a lane issues together (8 x 2 KB per warp in flight
+// with one token; with four tokens the x columns take the registers of half).
+template <int NT>
+__host__ __device__ constexpr int router_batch() { return NT == 1 ? 8 : 4; }
 
-struct RouteSmem {
-    float acc[kRMaxRows][kRouteTok];
-    int seg_row[2][8][kRSegs];
-    float seg_val[2][8][kRSegs][kRouteTok];
-    int seg_n[2][8];
-};
-
-__host__ __device__ inline int route_smem_bytes(int d, int nt, int nstage) {
-    return nstage * kRStage + nt * d * 4 + (int)sizeof(RouteSmem) + nstage * 8 + 64;
-}
-
-// This CTA's router slice: units [u0, u1) of 16 floats, in stages of 256.
-__device__ __forceinline__ void router_slice(const RouteParams &p, long long &u0, long long &u1) {
-    const long long U = (long long)p.E * p.d / 16;
-    u0 = (long long)blockIdx.x * U / gridDim.x;
-    u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;
-}
-__device__ __forceinline__ void router_issue(const RouteParams &p, uint8_t *ring, uint64_t *full, long long u0,
-                                             long long u1, int j, int slot) {
-    const long long a = u0 + 256LL * j;
-    const long long e = min(u1, a + 256);
-    const uint32_t bytes = (uint32_t)((e - a) * 64);
-    mbar_arrive_expect_tx(&full[slot], bytes);
-    bulk_g2s(ring + (size_t)slot * kRStage, p.wr + a * 16, bytes, &full[slot]);
-}
-// One thread: the first stages of a pass (the ring is free), issued before
-// anything else so the weight stream starts at once.
-__device__ void router_prefetch(const RouteParams &p, uint8_t *ring, uint64_t *full, int nstage, int chunk) {
-    long long u0, u1;
-    router_slice(p, u0, u1);
-    const int nch = (int)((u1 - u0 + 255) / 256);
-    for (int j = 0; j < nch && j < nstage; ++j) router_issue(p, ring, full, u0, u1, j, (chunk + j) % nstage);
-}
-
-// Streams this CTA's router slice once for tokens t0 .. t0+nt-1 (x in xs as
-// fp32 [nt][d]; the first stages already issued by router_prefetch);
-// finishes the rows it can and counts them on router_done.  `chunk` numbers
-// the CTA's stages across passes (ring phase).  All threads.
-__device__ void stream_router(const RouteParams &p, WsHeader *hdr, uint8_t *ring, uint64_t *full, int nstage,
-                              const float *xs, RouteSmem &sm, int t0, int nt, int pass, int &chunk) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-    const int d = p.d, G = gridDim.x, c = blockIdx.x;
-    const long long U = (long long)p.E * d / 16;
-    long long u0, u1;
-    router_slice(p, u0, u1);
-    const int row_base = (int)(u0 * 16 / d);
-    const int nrows = u1 > u0 ? (int)((u1 * 16 - 1) / d) - row_base + 1 : 0;
-    const int nch = (int)((u1 - u0 + 255) / 256);
-    for (int i = tid; i < kRMaxRows * kRouteTok; i += blockDim.x) (&sm.acc[0][0])[i] = 0.f;
-    auto issue = [&](int j, int slot) { router_issue(p, ring, full, u0, u1, j, slot); };
-    // Few rows per slice (the usual case): each thread keeps its own sum per
-    // row of the slice across all stages, and the warps reduce once at the
-    // end.  Otherwise the row sums are reduced and folded stage by stage.
-    const bool fast = nrows <= kRFast;
-    float racc[kRFast][kRouteTok];
+template <int NT>
+__device__ void stream_router(const RouteParams &p, WsHeader *hdr, int t0, int nt, int pass, int wi, int nw) {
+    const int lane = threadIdx.x & 31;
+    const int d = p.d, E = p.E;
+    const int Ls = router_part_len(d), P = d / Ls;
+    const int nv = Ls >= 128 ? Ls / 128 : 1;  // float4 per lane per segment
+    const bool lact = Ls >= 128 || lane < 16;
+    const int NS = E * P;  // E*d < 2^31 floats
+    const int s0 = (int)((long long)wi * NS / nw), s1 = (int)((long long)(wi + 1) * NS / nw);
+    float *part = reinterpret_cast<float *>(p.ws + p.L.part) + (size_t)(pass & 1) * NS * kRouteTok;
+    uint32_t *cnt = reinterpret_cast<uint32_t *>(p.ws + p.L.cnt) + (size_t)(pass & 1) * E;
+    float *logits = reinterpret_cast<float *>(p.ws + p.L.logits);
+    const bool add_bias = p.bias && !(p.route_flags & kRouteBiasSelect);
+    float xr[NT][16];
+    int xq = -1;
+    // x columns q*Ls + 128 i + 4 lane .. +3 of each token (bf16 -> fp32)
+    auto load_x = [&](int q) {
 #pragma unroll
-    for (int k = 0; k < kRFast; ++k)
+        for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int t = 0; t < kRouteTok; ++t) racc[k][t] = 0.f;
-    __syncthreads();  // the accumulators are cleared
-    for (int j = 0; j < nch; ++j, ++chunk) {
-        const int slot = chunk % nstage;
-        const uint32_t par = (uint32_t)((chunk / nstage) & 1);
-        // bounded; after a timeout the CTA keeps going (its barriers stay in
-        // step) with unused values, the status word says so
-        {
-            // lane 0 polls; the others then take the completed phase themselves
-            int ok = 1;
-            if (lane == 0) ok = mbar_wait_bounded(&full[slot], par, hdr, p.wait_ns) ? 1 : 0;
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (ok && lane != 0) (void)mbar_try_wait(&full[slot], par);
-        }
-        const long long unit = u0 + 256LL * j + tid;
-        int row = -1;
-        float v[kRouteTok];
+            for (int i = 0; i < 4; ++i)
+                if (t < nt && i < nv && lact) {
+                    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p.x + (size_t)(t0 + t) * d + (size_t)q * Ls +
+                                                                          128 * i + 4 * lane));
+                    xr[t][4 * i + 0] = bf16_lo(u.x);
+                    xr[t][4 * i + 1] = bf16_hi(u.x);
+                    xr[t][4 * i + 2] = bf16_lo(u.y);
+                    xr[t][4 * i + 3] = bf16_hi(u.y);
+                }
+        xq = q;
+    };
+    if (s0 < s1) load_x(s0 / E);  // before the weight loads, so it lands first
+    for (int g0 = s0; g0 < s1; g0 += 32) {
+        // lane j owns segment g0 + j of this group: it stores the segment's sum
+        // and counts it on its row
+        const int ng = min(32, s1 - g0);
+        constexpr int kRSeg = router_batch<NT>();
+        for (int b0 = 0; b0 < ng; b0 += kRSeg) {
+            float4 w[kRSeg][4];
 #pragma unroll
-        for (int t = 0; t < kRouteTok; ++t) v[t] = 0.f;
-        if (unit < u1) {
-            const uint32_t f = (uint32_t)unit * 16u;  // E*d < 2^31 floats
-            row = (int)(f / (uint32_t)d);
-            const int col = (int)(f - (uint32_t)row * (uint32_t)d);
-            const float4 *w4 = reinterpret_cast<const float4 *>(ring + (size_t)slot * kRStage) + tid * 4;
+            for (int b = 0; b < kRSeg; ++b) {
+                if (b0 + b < ng) {
+                    const int s = g0 + b0 + b, q = s / E, r = s - q * E;
+                    const float4 *src = reinterpret_cast<const float4 *>(p.wr + (size_t)r * d + (size_t)q * Ls) + lane;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 w = w4[q];
+                    for (int i = 0; i < 4; ++i)
+                        if (i < nv && lact) w[b][i] = __ldcs(src + 32 * i);
+                }
+            }
+            // every segment's products first, then the lane sums of all of
+            // them side by side (independent shuffle chains overlap)
+            float v[kRSeg][NT];
 #pragma unroll
-                for (int t = 0; t < kRouteTok; ++t) {
-                    if (t < nt) {
-                        const float4 xv = *reinterpret_cast<const float4 *>(xs + t * d + col + 4 * q);
-                        v[t] = fmaf(w.x, xv.x, v[t]);
-                        v[t] = fmaf(w.y, xv.y, v[t]);
-                        v[t] = fmaf(w.z, xv.z, v[t]);
-                        v[t] = fmaf(w.w, xv.w, v[t]);
+            for (int b = 0; b < kRSeg; ++b) {
+#pragma unroll
+                for (int t = 0; t < NT; ++t) v[b][t] = 0.f;
+                if (b0 + b < ng) {
+                    const int q = (g0 + b0 + b) / E;
+                    if (q != xq) load_x(q);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (i < nv && lact) {
+                            const float4 wv = w[b][i];
+#pragma unroll
+                            for (int t = 0; t < NT; ++t) {
+                                v[b][t] = fmaf(wv.x, xr[t][4 * i + 0], v[b][t]);
+                                v[b][t] = fmaf(wv.y, xr[t][4 * i + 1], v[b][t]);
+                                v[b][t] = fmaf(wv.z, xr[t][4 * i + 2], v[b][t]);
+                                v[b][t] = fmaf(wv.w, xr[t][4 * i + 3], v[b][t]);
+                            }
+                        }
                     }
                 }
             }
-        }
-        if (fast) {
-            if (row >= 0) {
-                const int k = row - row_base;
 #pragma unroll
-                for (int kk = 0; kk < kRFast; ++kk)
-                    if (kk == k)
+            for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-                        for (int t = 0; t < kRouteTok; ++t) racc[kk][t] += v[t];
-            }
-            if (j + nstage < nch) {
-                __syncthreads();  // every thread is done with this stage: refill it
-                if (tid == 0) issue(j + nstage, slot);
-            }
-            continue;
-        }
-        // segmented sum over lanes of equal row (rows do not decrease along lanes)
+                for (int b = 0; b < kRSeg; ++b)
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int rn = __shfl_down_sync(0xffffffffu, row, o);
+                    for (int t = 0; t < NT; ++t) v[b][t] += __shfl_xor_sync(0xffffffffu, v[b][t], o);
 #pragma unroll
-            for (int t = 0; t < kRouteTok; ++t) {
-                const float vn = __shfl_down_sync(0xffffffffu, v[t], o);
-                if (lane + o < 32 && rn == row) v[t] += vn;
-            }
-        }
-        const int rprev = __shfl_up_sync(0xffffffffu, row, 1);
-        const bool head = row >= 0 && (lane == 0 || rprev != row);
-        const uint32_t heads = __ballot_sync(0xffffffffu, head);
-        const int b = j & 1;
-        if (head) {
-            const int k = __popc(heads & ((1u << lane) - 1u));
-            sm.seg_row[b][warp][k] = row;
+            for (int b = 0; b < kRSeg; ++b) {
+                if (b0 + b < ng && lane == b0 + b) {
+                    const int s = g0 + b0 + b, q = s / E, r = s - q * E;
+                    float *dst = part + ((size_t)r * P + q) * kRouteTok;
 #pragma unroll
-            for (int t = 0; t < kRouteTok; ++t) sm.seg_val[b][warp][k][t] = v[t];
-        }
-        if (lane == 0) sm.seg_n[b][warp] = __popc(heads);
-        __syncthreads();  // this stage is read and its row sums posted
-        if (tid == 0 && j + nstage < nch) issue(j + nstage, slot);
-        if (tid < nrows) {
-            const int r = row_base + tid;
-            for (int w = 0; w < 8; ++w)
-                for (int k = 0; k < sm.seg_n[b][w]; ++k)
-                    if (sm.seg_row[b][w][k] == r)
-#pragma unroll
-                        for (int t = 0; t < kRouteTok; ++t) sm.acc[tid][t] += sm.seg_val[b][w][k][t];
-        }
-    }
-    if (fast) {
-        // per row: the warp's sum (fixed butterfly), then the warps in order
-#pragma unroll
-        for (int k = 0; k < kRFast; ++k) {
-            if (k < nrows) {
-#pragma unroll
-                for (int t = 0; t < kRouteTok; ++t) {
-                    if (t < nt) {
-                        float v = racc[k][t];
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                        if (lane == 0) sm.seg_val[0][warp][k][t] = v;
-                    }
+                    for (int t = 0; t < NT; ++t)
+                        if (t < nt) dst[t] = v[b][t];
                 }
             }
         }
-        __syncthreads();
-        if (tid < nrows)
-            for (int w = 0; w < 8; ++w)
+        if (lane < ng) {
+            const int s = g0 + lane, q = s / E, r = s - q * E;
+            (void)q;
+            // release: this lane's part store; acquire: the other parts of the row
+            const uint32_t old = atom_add_acq_rel(&cnt[r], 1u);
+            if (old == (uint32_t)(P - 1)) {
+                float out[NT];
 #pragma unroll
-                for (int t = 0; t < kRouteTok; ++t)
-                    if (t < nt) sm.acc[tid][t] += sm.seg_val[0][w][tid][t];
-    }
-    // every stage this CTA issued has been waited for above (a stage whose
-    // wait ran out is the only copy that may not have landed)
-    __syncthreads();  // every fold is done
-    if (tid < nrows) {
-        const int r = row_base + tid;
-        const long long rs = (long long)r * d / 16, re = (long long)(r + 1) * d / 16;  // its units
-        float *logits = reinterpret_cast<float *>(p.ws + p.L.logits);
-        const float bias = (p.bias && !(p.route_flags & kRouteBiasSelect)) ? p.bias[r] : 0.f;
-        bool done = false;
-        float out[kRouteTok];
-        if (rs >= u0 && re <= u1) {
+                for (int t = 0; t < NT; ++t) out[t] = 0.f;
+                const float *src = part + (size_t)r * P * kRouteTok;
+#pragma unroll 7
+                for (int qq = 0; qq < P; ++qq)
 #pragma unroll
-            for (int t = 0; t < kRouteTok; ++t) out[t] = sm.acc[tid][t];
-            done = true;
-        } else {
-            // cut by a CTA boundary: park this CTA's part; the last to arrive
-            // sums the parts in CTA order
-            const int first = chunk_owner(rs, U, G);
-            const int nseg = chunk_owner(re - 1, U, G) - first + 1;
-            float *pp = reinterpret_cast<float *>(p.ws + p.L.part) + (((size_t)(pass & 1) * p.E + r) * kMaxSeg) * kRouteTok;
-            uint32_t *pc = reinterpret_cast<uint32_t *>(p.ws + p.L.cnt) + (size_t)(pass & 1) * p.E + r;
+                    for (int t = 0; t < NT; ++t)
+                        if (t < nt) out[t] += __ldcg(src + qq * kRouteTok + t);
+                cnt[r] = 0u;
+                const float bv = add_bias ? __ldg(p.bias + r) : 0.f;
 #pragma unroll
-            for (int t = 0; t < kRouteTok; ++t) pp[(c - first) * kRouteTok + t] = sm.acc[tid][t];
-            const uint32_t old = atom_add_acq_rel(pc, 1u);
-            if (old == (uint32_t)(nseg - 1)) {
-#pragma unroll
-                for (int t = 0; t < kRouteTok; ++t) out[t] = 0.f;
-                for (int sl = 0; sl < nseg; ++sl)
-#pragma unroll
-                    for (int t = 0; t < kRouteTok; ++t) out[t] += __ldcg(pp + sl * kRouteTok + t);
-                *pc = 0u;
-                done = true;
+                for (int t = 0; t < NT; ++t)
+                    if (t < nt) logits[(size_t)(t0 + t) * E + r] = out[t] + bv;
+                red_add_release(&hdr->router_done, 1u);  // after this lane's logit stores
             }
-        }
-        if (done) {
-            for (int t = 0; t < nt; ++t) logits[(size_t)(t0 + t) * p.E + r] = out[t] + bias;
-            red_add_release(&hdr->router_done, 1u);  // after this thread's logit stores
         }
     }
 }
@@ -549,108 +460,169 @@ __device__ bool wait_count(const uint32_t *ctr, uint32_t target, WsHeader *hdr, 
     return false;
 }
 
-// Cooperative launch (every CTA resident), one CTA per SM.  Every CTA
-// streams its slice of the router; once all rows are in, token t's top-k runs
-// on CTA t mod G (all its warps), and CTA 0, after its own tokens, waits for
-// the others' and dispatches.  Meanwhile CTAs 1.. (CTA 0 when it is alone)
-// build the gate/up pass's activation pieces and every expert's tensor maps,
-// which need no routing.
+// One token (Tc == 1): the dispatch by warp 0 right after the token's top-k
+// (its k picks are k distinct experts): expert of pick j goes to distinct
+// slot u = number of picks with a smaller id, so the slots are in ascending
+// id as the general dispatch orders them; the picked experts' tensor maps
+// are rewritten where their blob pointer changed.  picks: the k picks in shared
+// memory; ptab, tc: shared copies of the blob pointer table and of the maps'
+// blob pointers; o: the workspace's dispatch arrays.
+// Where dispatch_one writes (the workspace's dispatch arrays).
+struct DispatchOut {
+    const uint8_t **ublob;
+    int32_t *ueid;
+    uint32_t *umask;
+    int8_t *uslot;
+    uint32_t *n_unique;
+};
+__device__ __noinline__ void dispatch_one(const RouteParams &p, WsHeader *hdr, int k, const int32_t *picks,
+                                          const uint8_t *const *ptab, const uint8_t *const *tc, DispatchOut o) {
+    const int lane = threadIdx.x & 31;
+    int e = 0x7FFFFFFF;
+    if (lane < k) e = picks[lane];
+    int u = 0;
+    for (int q = 0; q < k; ++q) u += __shfl_sync(0xffffffffu, e, q) < e ? 1 : 0;
+    if (lane < k) {
+        const uint8_t *b = ptab[e];
+        if ((reinterpret_cast<uintptr_t>(b) & 15u) != 0u || b == nullptr) {
+            set_status(hdr, kStDeviceCheck);
+            b = nullptr;
+        }
+        // the expert's tensor maps, rewritten when its blob pointer changed
+        if (b != nullptr && tc[e] != b) {
+            write_expert_tmaps(p.ws, p.L, e, b, p.tmpl, p.scale_mask);
+            reinterpret_cast<const uint8_t **>(p.ws + p.L.tcache)[e] = b;
+        }
+        o.ublob[u] = b;
+        o.ueid[u] = e;
+        o.umask[u] = 1u;
+#pragma unroll
+        for (int t = 0; t < kChunk; ++t) o.uslot[(size_t)u * kChunk + t] = t == 0 ? (int8_t)lane : (int8_t)-1;
+    }
+    if (lane == 0) *o.n_unique = (uint32_t)k;
+}
+
+// Cooperative launch (every CTA resident), one CTA per SM.  CTAs 0 .. Tc-1
+// (p.nded of them) stream nothing: they run their top-k code once on
+// placeholder data (so the code is cached when the router rows arrive), wait
+// for every router row, and each runs the softmax and top-k of token t = its
+// index; CTA 0 then dispatches (at once for one token, else after the other
+// tokens' top-k), refreshing the selected experts' maps.  The other CTAs
+// stream the router (all tokens of the chunk, NT per pass) and then build the
+// gate/up pass's activation pieces (the last one also the shared expert's
+// maps).  Every CTA counts on prep_done once, after what it writes there.
+template <int NT>
 __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_constant__ RouteParams p) {
-    extern __shared__ __align__(128) uint8_t rsm[];
-    const int nstage = p.nstage;
-    const int ntmax = min(p.Tc, kRouteTok);
-    uint8_t *ring = rsm;
-    float *xs = reinterpret_cast<float *>(rsm + (size_t)nstage * kRStage);  // [ntmax][d]
-    RouteSmem &sm = *reinterpret_cast<RouteSmem *>(xs + (size_t)ntmax * p.d);
-    uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(&sm) + sizeof(RouteSmem));
     WsHeader *hdr = reinterpret_cast<WsHeader *>(p.ws + p.L.hdr);
     __shared__ int s_ok;
-    if (threadIdx.x == 0) {
-        for (int st = 0; st < nstage; ++st) mbar_init(&full[st], 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
+    __shared__ int32_t s_didx[32];
+    __shared__ float s_dw[32];
+    extern __shared__ __align__(16) uint8_t rdyn[];  // route_dyn_bytes(E): CTA 0's tables
     pdl_trigger();
-    const int npass = (p.Tc + kRouteTok - 1) / kRouteTok;
-    const int G = gridDim.x;
+    const int G = gridDim.x, nded = p.nded;
     const int warp = threadIdx.x >> 5;
-    int chunk = 0;
-    if (threadIdx.x == 0) router_prefetch(p, ring, full, nstage, 0);  // pass 0's first stages
-    // while the first router stages are in flight
-    if (p.blobs != nullptr) {
-        refresh_tmaps(p, blockIdx.x * kRouteThreads + threadIdx.x, G * kRouteThreads);
-        if (blockIdx.x == 0 && G > 1) {
-            // CTA 0 builds no x pieces: its maps are all it publishes to the
-            // gate/up pass's shared units (the other CTAs count after their pieces)
+    const int npass = (p.Tc + NT - 1) / NT;
+    if ((int)blockIdx.x >= nded) {
+        const int nw = (G - nded) * (kRouteThreads / 32);
+        const int wi = ((int)blockIdx.x - nded) * (kRouteThreads / 32) + warp;
+        for (int pass = 0; pass < npass; ++pass)
+            stream_router<NT>(p, hdr, pass * NT, min(NT, p.Tc - pass * NT), pass, wi, nw);
+        if (p.blobs != nullptr) {
+            // a share of the activation pieces (x is in L2 by now): one
+            // 32-column block per warp for most warps; the last CTA (which
+            // has no pieces at the usual sizes) the shared expert's maps
+            build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L, wi, nw, p.has_shared != 0);
+            if ((int)blockIdx.x == G - 1 && threadIdx.x == 0) refresh_tmaps(p, p.E, 1);  // index E
             __syncthreads();
-            if (threadIdx.x == 0) red_add_release(&hdr->prep_done, 1u);
-        }
-    }
-    for (int pass = 0; pass < npass; ++pass) {
-        const int t0 = pass * kRouteTok;
-        const int nt = min(kRouteTok, p.Tc - t0);
-        __syncthreads();  // the previous pass no longer reads xs or the ring
-        if (pass > 0 && threadIdx.x == 0) router_prefetch(p, ring, full, nstage, chunk);
-        // x of these tokens as fp32: 16-byte loads, several in flight per thread
-        const uint4 *xv = reinterpret_cast<const uint4 *>(p.x + (size_t)t0 * p.d);
-        const int n8 = nt * p.d / 8;
-#pragma unroll 4
-        for (int i = threadIdx.x; i < n8; i += blockDim.x) {
-            const uint4 w = __ldg(xv + i);
-            float4 *o = reinterpret_cast<float4 *>(xs + 8 * i);
-            o[0] = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
-            o[1] = make_float4(bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w));
-        }
-        __syncthreads();
-        stream_router(p, hdr, ring, full, nstage, xs, sm, t0, nt, pass, chunk);
-    }
-    // work of the gate/up pass that needs no routing (before the top-k wait
-    // on a lone CTA, after it elsewhere is not needed: other CTAs do it)
-    auto prep = [&](int first_cta) {
-        if (p.blobs == nullptr) return;
-        const int nworkers = G - first_cta;
-        const int wi = (blockIdx.x - first_cta) * (kRouteThreads / 32) + warp;
-        build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L, wi, nworkers * (kRouteThreads / 32), p.has_shared != 0);
-    };
-    if (G == 1 && p.blobs != nullptr) {
-        prep(0);
-        __syncthreads();
-        if (threadIdx.x == 0) red_add_release(&hdr->prep_done, 1u);
-    }
-    // top-k of this CTA's tokens once every router row is in
-    if ((int)blockIdx.x < p.Tc) {
-        __syncthreads();
-        if (threadIdx.x == 0) s_ok = wait_count(&hdr->router_done, (uint32_t)(p.E * npass), hdr, p.wait_ns);
-        __syncthreads();
-        if (!s_ok) return;
-        for (int t = blockIdx.x; t < p.Tc; t += G) {
-            cta_topk(p, t);
-            __syncthreads();
-        }
-        if (blockIdx.x > 0 && threadIdx.x == 0) {
-            int mine = 0;
-            for (int t = blockIdx.x; t < p.Tc; t += G) ++mine;
-            red_add_release(&hdr->topk_done, (uint32_t)mine);  // after thread 0's own result stores
-        }
-    }
-    if (blockIdx.x == 0) {
-        int mine = 0;
-        for (int t = 0; t < p.Tc; t += G) ++mine;
-        if (threadIdx.x == 0) s_ok = wait_count(&hdr->topk_done, (uint32_t)(p.Tc - mine), hdr, p.wait_ns);
-        __syncthreads();
-        if (!s_ok) return;
-        if (p.blobs != nullptr) dispatch(p, hdr);
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            hdr->router_done = 0u;
-            hdr->topk_done = 0u;
+            if (threadIdx.x == 0) red_add_release(&hdr->prep_done, 1u);  // after this CTA's pieces (and maps)
         }
         return;
     }
-    prep(1);
-    if (p.blobs != nullptr) {
+    // ---- CTAs 0 .. nded-1: top-k (they write nothing the gate/up pass's
+    // shared units read: they count on prep_done at once).  Everything the
+    // top-k and the dispatch take from the launch parameters is read here,
+    // at the start, into shared memory: after the last router row arrives
+    // no constant-bank miss sits on the path.
+    struct TopkArgs {
+        const float *row;
+        int32_t *idx_row, *idx_out;
+        float *w_row, *w_out;
+        const float *sel_bias;
+        DispatchOut out;
+        uint64_t wait_ns;
+        uint32_t rows_target;
+        int E, k, renorm, Tc, dispatch;
+    };
+    __shared__ TopkArgs s_a;
+    const int t = blockIdx.x;  // this CTA's token (nded = Tc)
+    if (threadIdx.x == 0) {
+        s_a.row = reinterpret_cast<const float *>(p.ws + p.L.logits) + (size_t)t * p.E;
+        s_a.idx_row = reinterpret_cast<int32_t *>(p.ws + p.L.idx) + t * p.k;
+        s_a.w_row = reinterpret_cast<float *>(p.ws + p.L.wt) + t * p.k;
+        s_a.idx_out = p.idx_out ? p.idx_out + (size_t)t * p.k : nullptr;
+        s_a.w_out = p.w_out ? p.w_out + (size_t)t * p.k : nullptr;
+        s_a.sel_bias = (p.route_flags & kRouteBiasSelect) ? p.bias : nullptr;
+        s_a.out = DispatchOut{reinterpret_cast<const uint8_t **>(p.ws + p.L.uniq_blob),
+                              reinterpret_cast<int32_t *>(p.ws + p.L.uniq_eid),
+                              reinterpret_cast<uint32_t *>(p.ws + p.L.uniq_mask),
+                              reinterpret_cast<int8_t *>(p.ws + p.L.uniq_slot), &hdr->n_unique};
+        s_a.wait_ns = p.wait_ns;
+        s_a.rows_target = (uint32_t)(p.E * npass);
+        s_a.E = p.E;
+        s_a.k = p.k;
+        s_a.renorm = (p.route_flags & kRouteRenorm) != 0;
+        s_a.Tc = p.Tc;
+        s_a.dispatch = p.blobs != nullptr;
+        if (p.blobs != nullptr) red_add_release(&hdr->prep_done, 1u);
+    }
+    const uint8_t **s_ptab = reinterpret_cast<const uint8_t **>(rdyn);  // [E] blob pointers
+    const uint8_t **s_tc = s_ptab + p.E;                                // [E] the maps' blob pointers
+    float *s_row = reinterpret_cast<float *>(s_tc + p.E);               // [E] placeholder row
+    for (int e = threadIdx.x; e < p.E; e += kRouteThreads) s_row[e] = 0.f;  // the placeholder row
+    if (p.blobs != nullptr && blockIdx.x == 0) {
+        // the dispatch reads these from shared memory: asynchronous copies,
+        // waited for only before the dispatch
+        const uint8_t *const *gtc = reinterpret_cast<const uint8_t *const *>(p.ws + p.L.tcache);
+        for (int e = threadIdx.x; e < p.E; e += kRouteThreads) {
+            cp_async8(&s_ptab[e], &p.blobs[e]);
+            cp_async8(&s_tc[e], &gtc[e]);
+        }
+    }
+    __syncthreads();
+    const int E = s_a.E, k = s_a.k;
+    // The top-k code runs once on placeholder data (a row of zeros in shared
+    // memory: all ties, k valid picks; results to shared scratch) while the
+    // router streams: the first run of that code on this SM waits on
+    // instruction fetches (about 10 us at the K3 shape), the real run after
+    // the last router row does not.  (A dry dispatch as well would end after
+    // the router rows: the dispatch runs cold.)
+    cta_topk_row(s_row, E, k, s_didx, s_dw, nullptr, nullptr, s_a.sel_bias, s_a.renorm != 0, nullptr, true);
+    cp_async_wait_all();  // this thread's table copies
+    __syncthreads();
+    const bool one = s_a.Tc == 1 && s_a.dispatch;
+    if (threadIdx.x == 0) s_ok = wait_count(&hdr->router_done, s_a.rows_target, hdr, s_a.wait_ns);
+    __syncthreads();
+    if (!s_ok) return;
+    cta_topk_row(s_a.row, E, k, s_a.idx_row, s_a.w_row, s_a.idx_out, s_a.w_out, s_a.sel_bias, s_a.renorm != 0,
+                 s_didx, false);
+    __syncthreads();
+    if (blockIdx.x > 0) {
+        if (threadIdx.x == 0) red_add_release(&hdr->topk_done, 1u);  // after thread 0's own result stores
+        return;
+    }
+    if (s_a.Tc > 1) {
+        // the other tokens' top-k (their CTAs count on topk_done)
+        if (threadIdx.x == 0) s_ok = wait_count(&hdr->topk_done, (uint32_t)(s_a.Tc - 1), hdr, s_a.wait_ns);
         __syncthreads();
-        if (threadIdx.x == 0) red_add_release(&hdr->prep_done, 1u);  // after this CTA's pieces and maps
+        if (!s_ok) return;
+        if (s_a.dispatch) dispatch(p, hdr, s_ptab, s_tc);
+    } else if (one && warp == 0) {
+        dispatch_one(p, hdr, k, s_didx, s_ptab, s_tc, s_a.out);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        hdr->router_done = 0u;
+        hdr->topk_done = 0u;
     }
 }
 

@@ -37,7 +37,6 @@ static __device__ __align__(256) uint8_t g_noalloc_ws[kNoAllocBytes];
 
 struct DeviceInfo {
     bool ready = false;
-    int route_dyn_max = 0;       // dynamic smem the route kernel may take beside its static arrays
     uint8_t *noalloc = nullptr;  // device address of g_noalloc_ws on this device, once set up
     int noalloc_shape[5] = {0, 0, 0, 0, 0};  // (d, ff, E, k, ff_shared) its layout was last used for
     int sms = 0;
@@ -79,13 +78,7 @@ k3moe_status device_info(DeviceInfo **out) {
         e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return cuda_fail(e);
         const int big = kSmemLimit;
-        cudaFuncAttributes fa;
-        cudaError_t r = cudaFuncGetAttributes(&fa, route_kernel);
-        if (r == cudaSuccess) {
-            di.route_dyn_max = big - (int)fa.sharedSizeBytes;
-            r = set_smem(route_kernel, di.route_dyn_max);
-        }
-        if (r == cudaSuccess) r = set_smem(umma_expert_kernel<true>, big);
+        cudaError_t r = set_smem(umma_expert_kernel<true>, big);
         if (r == cudaSuccess) r = set_smem(umma_expert_kernel<false>, big);
         if (r == cudaSuccess) r = set_smem(pf_expert_kernel<true>, big);
         if (r == cudaSuccess) r = set_smem(pf_expert_kernel<false>, big);
@@ -333,33 +326,31 @@ cudaError_t launch_umma(const DeviceInfo &di, UmmaParams up, cudaStream_t st) {
 
 
 // Router (+ top-k + dispatch + activation pieces) for one chunk.  Cooperative
-// launch: CTA 0 waits on the other CTAs' router rows, so all must be resident.
+// launch (CTA t waits on the other CTAs' router rows, so all must be
+// resident), one CTA per SM: Tc CTAs for the pieces and the top-k, the rest
+// stream the router, about eight row parts per warp at least.  grid_out: the
+// CTAs that count on prep_done (all of them; the gate/up pass waits for it).
 cudaError_t launch_route(DeviceInfo &di, RouteParams rp, cudaStream_t st, int *grid_out = nullptr) {
-    // one CTA per SM, at most one per router row and one per stage of router
-    // bytes; as many ring stages as fit beside x (12 at most)
-    const int nt = rp.Tc < kRouteTok ? rp.Tc : kRouteTok;
-    const long long bytes = (long long)rp.E * rp.d * 4;
-    long long g = (bytes + kRStage - 1) / kRStage;
-    if (g > di.sms) g = di.sms;
-    if (g > rp.E) g = rp.E;
-    if (g < 1) g = 1;
-    int nstage = 12;
-    while (nstage > 2 && route_smem_bytes(rp.d, nt, nstage) > di.route_dyn_max) --nstage;
-    if (route_smem_bytes(rp.d, nt, nstage) > di.route_dyn_max) return cudaErrorInvalidConfiguration;
-    rp.nstage = nstage;
+    if (di.sms < kChunk + 1) return cudaErrorInvalidConfiguration;
+    const long long nseg = (long long)rp.E * (rp.d / router_part_len(rp.d));
+    long long ns = (nseg + 8 * (kRouteThreads / 32) - 1) / (8 * (kRouteThreads / 32));
+    if (ns > di.sms - rp.Tc) ns = di.sms - rp.Tc;
+    if (ns < 1) ns = 1;
+    rp.nded = rp.Tc;
     rp.wait_ns = wait_limit();
-    if (grid_out) *grid_out = (int)g;
+    if (grid_out) *grid_out = (int)(rp.Tc + ns);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)g);
+    cfg.gridDim = dim3((unsigned)(rp.Tc + ns));
     cfg.blockDim = dim3(kRouteThreads);
-    cfg.dynamicSmemBytes = route_smem_bytes(rp.d, nt, nstage);
+    cfg.dynamicSmemBytes = route_dyn_bytes(rp.E);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, route_kernel, rp);
+    return rp.Tc == 1 ? cudaLaunchKernelEx(&cfg, route_kernel<1>, rp)
+                      : cudaLaunchKernelEx(&cfg, route_kernel<kRouteTok>, rp);
 }
 
 // Decode passes of this call by the one-launch kernel (K3MOE_ONE_LAUNCH);

@@ -49,6 +49,7 @@ namespace k3 {
 constexpr int kLThreads = 352;
 constexpr int kLMaxCtas = 160;        // grid cap (one CTA per SM)
 constexpr int kLRUnit = 8192;         // router floats per R0 unit at most (32 KB): whole rows
+constexpr int kRMaxRows = 72;         // router rows one CTA sums at most
 constexpr int kLSfc = 32;             // TMEM scale columns per stage
 constexpr int kLTopkWarps = 5;        // warps 0-3 and 10
 constexpr int kTkCand = 128;          // top-k candidates per warp (scratch: keys, then ids)

@@ -7,7 +7,6 @@
 namespace k3 {
 
 constexpr int kChunk = 8;   // tokens per decode pass
-constexpr int kMaxSeg = 8;  // most warps that share one router/shared row
 
 // Tensor-core path: each activation element enters the MMA as kPieces E2M1
 // values with their own per-32 E8M0 scales; B-operand row n = t*kPieces + p.
@@ -33,8 +32,8 @@ struct Layout {
     size_t uniq_eid;   // i32 [kChunk*k]    its expert id (index of its tensor maps)
     size_t uniq_mask;  // u32 [kChunk*k]    tokens (bit t) that selected it
     size_t uniq_slot;  // i8  [kChunk*k][kChunk] slot j of token t for it, -1 if none
-    size_t part;       // f32 [2][E][kMaxSeg][4] partial sums of router rows split between warps
-    size_t cnt;        // u32 [2][E] arrivals per split row (back to 0 after each row)
+    size_t part;       // f32 [2][E][P][4] partial sums of the P parts of each router row
+    size_t cnt;        // u32 [2][E] parts summed per router row (back to 0 after each row)
     size_t tmap;       // 128-byte tensor maps [E][6]: W_g, W_u, W_d nibble planes and their
                        // scale planes, of each expert; then the shared expert's W_g, W_u,
                        // W_d (bf16) at [E*6 ..]
@@ -51,6 +50,12 @@ struct Layout {
     size_t total;
     int d, ff, E, k, ffs, umax;
 };
+
+// The decode router sums a row of d floats as d / Ls parts of Ls floats
+// (Ls = 512 where d allows it; d is a multiple of 64).
+__host__ __device__ inline int router_part_len(int d) {
+    return d % 512 == 0 ? 512 : d % 256 == 0 ? 256 : d % 128 == 0 ? 128 : 64;
+}
 
 __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int ffs) {
     Layout L;
@@ -78,7 +83,7 @@ __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int f
     L.uniq_slot = o;
     o = align256(o + C * k * C);
     L.part = o;
-    o = align256(o + (size_t)2 * E * kMaxSeg * 4 * 4);
+    o = align256(o + (size_t)2 * E * (d / router_part_len(d)) * 4 * 4);
     L.cnt = o;
     o = align256(o + (size_t)2 * E * 4);
     const int umax = E < kChunk * k ? E : kChunk * k;

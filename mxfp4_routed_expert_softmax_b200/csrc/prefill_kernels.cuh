@@ -157,7 +157,8 @@ __global__ void __launch_bounds__(kRouteThreads) pf_topk_kernel(const __grid_con
                  reinterpret_cast<int32_t *>(ws + p.P.idx) + (size_t)t * k,
                  reinterpret_cast<float *>(ws + p.P.wt) + (size_t)t * k,
                  p.r.idx_out ? p.r.idx_out + (size_t)t * k : nullptr, p.r.w_out ? p.r.w_out + (size_t)t * k : nullptr,
-                 (p.r.route_flags & kRouteBiasSelect) ? p.r.bias : nullptr, (p.r.route_flags & kRouteRenorm) != 0);
+                 (p.r.route_flags & kRouteBiasSelect) ? p.r.bias : nullptr, (p.r.route_flags & kRouteRenorm) != 0,
+                 nullptr, false);
 }
 
 // --------------------------------------------------------------- dispatch --

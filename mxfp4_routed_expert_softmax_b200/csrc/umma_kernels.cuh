@@ -175,8 +175,10 @@ __device__ void write_shared_tmaps(uint8_t *ws, const Layout &L, const uint4 (&s
 // [1] W_d nibbles (d rows of ff/2 bytes), [2] W_g/W_u scales (ff rows of d/32
 // bytes), [3] W_d scales (d rows of ff/32 bytes); the scale maps are written
 // only where scale_mask says their template exists (bit 0: W_g/W_u, bit 1:
-// W_d; the reduction length a multiple of 512).  One thread.
-__device__ void write_expert_tmaps(uint8_t *ws, const Layout &L, int e, const uint8_t *blob,
+// W_d; the reduction length a multiple of 512).  One thread.  Not inlined:
+// callers run it only when an expert's blob pointer changed and keep their
+// hot code short.
+__device__ __noinline__ void write_expert_tmaps(uint8_t *ws, const Layout &L, int e, const uint8_t *blob,
                                    const uint4 (&tmpl)[4][8], int scale_mask) {
     const size_t mat = (size_t)L.d * L.ff;
     uint8_t *dst = ws + L.tmap + (size_t)e * kMapsPerExpert * 128;
@@ -306,29 +308,6 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     umma::fence_after();
     const uint32_t tbase = *tslot;
     const int Tc = p.Tc, N = act_n(Tc);
-    // accumulator chains: each matrix slot of 64 columns holds QC chains of
-    // WC columns (independent MMAs overlap in the tensor pipe; the epilogue
-    // sums them and zeroes them after reading, so every MMA accumulates)
-    const int QC = NMAT == 1 ? (N <= 16 ? 4 : (N <= 32 ? 2 : 1)) : (N <= 32 ? 2 : 1);
-    const int WC = 64 / QC;
-    auto zero_acc = [&](int buf) {
-        const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int m = 0; m < NMAT; ++m)
-            for (int q = 0; q < QC; ++q)
-#pragma unroll
-                for (int n0 = 0; n0 < kNMax; n0 += 8)
-                    if (n0 < N)
-                        umma::st8(tbase + umma::lane_base(warp) + (uint32_t)((buf * NMAT + m) * 64 + q * WC + n0), z);
-        umma::wait_st();
-    };
-    if (warp < 4) {
-        zero_acc(0);
-        zero_acc(1);
-    }
-    umma::fence_before();
-    __syncthreads();
-    umma::fence_after();
     // the routing of the chunk (written by the router kernel) -> shared memory
     auto load_meta = [&](int i0, int nthr) {
         const int U = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_unique);
@@ -748,7 +727,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 if (seg >= 2 && !wait(&aempty[buf], (uint32_t)(((seg >> 1) + 1) & 1))) break;
                 umma::fence_after();
                 const uint32_t dcol = tbase + (uint32_t)(buf * NMAT * 64);
-                constexpr uint32_t acc = 1u;  // the accumulators start at zero
+                uint32_t acc = 0u;
                 for (int un = unit; un < seg_end; x = advance(x, ++un, rg.b)) {
                     if (!wait(&full[s], ph) || !wait(&sfr[s], ph)) break;
                     umma::fence_after();
@@ -760,9 +739,9 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                         for (int sk = 0; sk < 4; ++sk) {
                             if (sk < nks) {
                                 const uint64_t bd = b0 + sk * bstep;
-                                const uint32_t cq = (uint32_t)((sk % QC) * WC);
-                                umma::mma_bf16(dcol + cq, a0 + 2 * sk, bd, idesc16, acc);
-                                if (GU) umma::mma_bf16(dcol + 64 + cq, a0 + (kAtile >> 4) + 2 * sk, bd, idesc16, acc);
+                                umma::mma_bf16(dcol, a0 + 2 * sk, bd, idesc16, acc);
+                                if (GU) umma::mma_bf16(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, idesc16, acc);
+                                acc = 1u;
                             }
                         }
                     } else {
@@ -771,14 +750,14 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                         for (int sk = 0; sk < 4; ++sk) {
                             if (sk < nks) {
                                 const uint64_t bd = b0 + sk * bstep;
-                                const uint32_t cq = (uint32_t)((sk % QC) * WC);
                                 const uint32_t sfid = (uint32_t)(2 * (sk & 1)) << 30;
                                 const uint32_t sfb = (sfc + 8 * NMAT + (sk >> 1) * 4) | sfid;
-                                umma::mma_mxf4(dcol + cq, a0 + 2 * sk, bd, id4[sk & 1], acc, (sfc + (sk >> 1) * 4) | sfid,
+                                umma::mma_mxf4(dcol, a0 + 2 * sk, bd, id4[sk & 1], acc, (sfc + (sk >> 1) * 4) | sfid,
                                                sfb);
                                 if (GU)
-                                    umma::mma_mxf4(dcol + 64 + cq, a0 + (kAtile >> 4) + 2 * sk, bd, id4[sk & 1], acc,
+                                    umma::mma_mxf4(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, id4[sk & 1], acc,
                                                    (sfc + 8 + (sk >> 1) * 4) | sfid, sfb);
+                                acc = 1u;
                             }
                         }
                     }
@@ -826,25 +805,19 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    if (q < QC) {
+                for (int n0 = 0; n0 < kNMax; n0 += 8) {
+                    if (n0 < N) {
+                        uint32_t r[8];
+                        umma::ld8(tbase + lb + (uint32_t)((buf * NMAT + m) * 64 + n0), r);
+                        umma::wait_ld();
 #pragma unroll
-                        for (int n0 = 0; n0 < kNMax; n0 += 8) {
-                            if (n0 < N) {
-                                uint32_t r[8];
-                                umma::ld8(tbase + lb + (uint32_t)((buf * NMAT + m) * 64 + q * WC + n0), r);
-                                umma::wait_ld();
-#pragma unroll
-                                for (int jj = 0; jj < 8; ++jj) {
-                                    const int t = (n0 + jj) / kPieces;
-                                    if (t < kChunk) acc[m][t] += __uint_as_float(r[jj]);
-                                }
-                            }
+                        for (int jj = 0; jj < 8; ++jj) {
+                            const int t = (n0 + jj) / kPieces;
+                            if (t < kChunk) acc[m][t] += __uint_as_float(r[jj]);
                         }
                     }
                 }
             }
-            zero_acc(buf);
             umma::fence_before();
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&aempty[buf])) : "memory");
