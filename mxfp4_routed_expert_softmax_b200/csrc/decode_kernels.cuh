@@ -29,9 +29,9 @@ struct RouteParams {
     int32_t *idx_out;   // optional [Tc][k]
     float *w_out;       // optional [Tc][k]
     int nded;           // CTAs 0 .. nded-1 run no router stream (pieces, top-k, dispatch)
-    uint4 tmpl[4][8];   // tensor-map templates: W_g/W_u, W_d nibble planes; their scale planes
+    uint4 tmpl[kTemplates][8];  // tensor-map templates (see kTemplates)
     int scale_mask;     // which scale-plane templates exist (bit 0: W_g/W_u, bit 1: W_d)
-    uint4 smap[3][8];   // shared expert tensor maps (W_g, W_u, W_d), when has_shared
+    uint4 smap[kSharedMaps][8];  // shared expert tensor maps (W_g, W_u, W_d, W_d 256-row), when has_shared
     int has_shared;     // the tensor-core kernels run a shared expert
     const uint8_t *sw[3];  // the shared expert's W_g, W_u, W_d (the key of its cached maps)
     uint64_t wait_ns;   // bound of every device wait
@@ -632,7 +632,7 @@ struct SingleParams {
     const uint8_t *blob;
     uint8_t *ws;
     Layout L;
-    uint4 tmpl[4][8];
+    uint4 tmpl[kTemplates][8];
     int scale_mask;
 };
 

@@ -183,12 +183,12 @@ cudaError_t launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
 // library does not link the driver library itself.
 struct TmapCache {
     int d = 0, ff = 0;
-    uint4 t[4][8];
+    uint4 t[kTemplates][8];
 };
 TmapCache g_tmaps[16];
 int g_ntmaps = 0;
 
-k3moe_status tmap_templates(int d, int ff, void *placeholder, uint4 (&out)[4][8]) {
+k3moe_status tmap_templates(int d, int ff, void *placeholder, uint4 (&out)[kTemplates][8]) {
     std::lock_guard<std::mutex> lock(g_mu);
     for (int i = 0; i < g_ntmaps; ++i)
         if (g_tmaps[i].d == d && g_tmaps[i].ff == ff) {
@@ -210,17 +210,19 @@ k3moe_status tmap_templates(int d, int ff, void *placeholder, uint4 (&out)[4][8]
     // [0], [1]: nibble planes, 128 rows x 128 bytes, 128-byte swizzle (the
     // MMA's K-major layout); [2], [3]: scale planes, 128 rows x 16 bytes, no
     // swizzle, only when the row of scales is a multiple of 16 bytes (the
-    // reduction length a multiple of 512), else left zero.
-    CUtensorMap m[4];
+    // reduction length a multiple of 512), else left zero; [4], [5]: W_d's
+    // nibble and scale planes again with 256-row boxes.
+    CUtensorMap m[kTemplates];
     memset(m, 0, sizeof(m));
-    for (int i = 0; i < 4; ++i) {
-        const int kdim = (i % 2 == 0) ? d : ff, rdim = (i % 2 == 0) ? ff : d;
-        const bool scale = i >= 2;
+    for (int i = 0; i < kTemplates; ++i) {
+        const bool wd = i == 1 || i == 3 || i >= 4;
+        const int kdim = wd ? ff : d, rdim = wd ? d : ff;
+        const bool scale = i == 2 || i == 3 || i == 5;
         if (scale && kdim % 512 != 0) continue;
         const cuuint64_t cols = (cuuint64_t)(scale ? kdim / 32 : kdim / 2), rows = (cuuint64_t)rdim;
         const cuuint64_t dims[2] = {cols, rows};
         const cuuint64_t strides[1] = {cols};
-        const cuuint32_t box[2] = {scale ? 16u : 128u, (cuuint32_t)kTileM};
+        const cuuint32_t box[2] = {scale ? 16u : 128u, (cuuint32_t)(i >= 4 ? 2 * kTileM : kTileM)};
         const cuuint32_t es[2] = {1, 1};
         CUresult r = encode(&m[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, placeholder, dims, strides, box, es,
                             CU_TENSOR_MAP_INTERLEAVE_NONE, scale ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
@@ -243,8 +245,9 @@ k3moe_status tmap_templates(int d, int ff, void *placeholder, uint4 (&out)[4][8]
 
 // Tensor maps of the bf16 shared expert at its real addresses (u8 elements,
 // 128 x 128-byte boxes, 128-byte swizzle): W_g, W_u (ff_s rows of 2d bytes),
-// W_d (d rows of 2 ff_s bytes).
-k3moe_status shared_tmaps(int d, int ffs, const void *wg, const void *wu, const void *wd, uint4 (&out)[3][8]) {
+// W_d (d rows of 2 ff_s bytes), and W_d again with 256-row boxes.
+k3moe_status shared_tmaps(int d, int ffs, const void *wg, const void *wu, const void *wd,
+                          uint4 (&out)[kSharedMaps][8]) {
     std::lock_guard<std::mutex> lock(g_mu);
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
@@ -258,13 +261,13 @@ k3moe_status shared_tmaps(int d, int ffs, const void *wg, const void *wu, const 
         }
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    const void *addr[3] = {wg, wu, wd};
-    CUtensorMap m[3];
-    for (int i = 0; i < 3; ++i) {
+    const void *addr[kSharedMaps] = {wg, wu, wd, wd};
+    CUtensorMap m[kSharedMaps];
+    for (int i = 0; i < kSharedMaps; ++i) {
         const cuuint64_t cols = (cuuint64_t)(i < 2 ? d : ffs) * 2, rows = (cuuint64_t)(i < 2 ? ffs : d);
         const cuuint64_t dims[2] = {cols, rows};
         const cuuint64_t strides[1] = {cols};
-        const cuuint32_t box[2] = {128, (cuuint32_t)kTileM};
+        const cuuint32_t box[2] = {128, (cuuint32_t)(i == 3 ? 2 * kTileM : kTileM)};
         const cuuint32_t es[2] = {1, 1};
         CUresult r = encode(&m[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(addr[i]), dims, strides, box,
                             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -580,10 +583,10 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
     uint8_t *xstage = wsb + base;
     uint8_t *ystage = xstage + align256((size_t)(grouped ? T : kChunk) * d * 2);
 
-    uint4 tmpl[4][8];
+    uint4 tmpl[kTemplates][8];
     s = tmap_templates(d, dims->ff, ws, tmpl);
     if (s != K3MOE_OK) return s;
-    uint4 smap[3][8];
+    uint4 smap[kSharedMaps][8];
     memset(smap, 0, sizeof(smap));
     if (ffs > 0) {
         s = shared_tmaps(d, ffs, shared_wg, shared_wu, shared_wd, smap);
@@ -865,7 +868,7 @@ k3moe_status k3moe_expert_ffn(const void *x, int32_t T, const uint8_t *blob,
     uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
     const int d = dims->d;
     const bool out32 = (dims->flags & K3MOE_OUT_FP32) != 0;
-    uint4 tmpl[4][8];
+    uint4 tmpl[kTemplates][8];
     s = tmap_templates(d, dims->ff, ws, tmpl);
     if (s != K3MOE_OK) return s;
     for (int c0 = 0; c0 < T; c0 += kChunk) {

@@ -57,6 +57,13 @@ __host__ __device__ inline int router_part_len(int d) {
     return d % 512 == 0 ? 512 : d % 256 == 0 ? 256 : d % 128 == 0 ? 128 : 64;
 }
 
+// Tensor maps in the workspace: per expert W_g, W_u, W_d nibble planes and
+// their scale planes (128-row boxes), then W_d's nibble and scale planes again
+// with 256-row boxes (the decode down pass); after all experts the shared
+// expert's W_g, W_u, W_d (128-row boxes) and W_d (256-row boxes).
+constexpr int kMapsPerExpert = 8;
+constexpr int kSharedMaps = 4;
+
 __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int ffs) {
     Layout L;
     L.d = d;
@@ -90,7 +97,7 @@ __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int f
     const int nkt_d = ceil_div(d, kTileK), nkt_ff = ceil_div(ff, kTileK);
     L.umax = umax;
     L.tmap = o;
-    o = align256(o + ((size_t)E * 6 + 3) * 128);
+    o = align256(o + ((size_t)E * kMapsPerExpert + kSharedMaps) * 128);
     L.tcache = o;
     o = align256(o + ((size_t)E + 3) * 8);
     L.xb = o;

@@ -41,10 +41,11 @@
 namespace k3 {
 
 constexpr int kUThreads = 352;
-// Tensor maps per expert in the workspace: W_g, W_u, W_d nibble planes, then
-// (used when the reduction lengths are multiples of 512) their scale planes.
-constexpr int kMapsPerExpert = 6;
-constexpr int kAtile = kTileM * 128;  // one A box: 128 rows x 128 bytes (16 KB)
+constexpr int kAtile = kTileM * 128;  // 128 rows x 128 bytes (16 KB) of an A operand
+// Host-encoded tensor-map templates: [0] W_g/W_u nibbles, [1] W_d nibbles,
+// [2] W_g/W_u scales, [3] W_d scales (128-row boxes), [4] W_d nibbles, [5]
+// W_d scales (256-row boxes).
+constexpr int kTemplates = 6;
 
 // ---------------------------------------------------------------- pieces --
 // One 32-element activation block (element = this lane's v) of token t ->
@@ -161,10 +162,10 @@ __device__ void build_x_pieces(const uint16_t *x, int Tc, int d, uint8_t *ws, co
 
 // The shared expert's three tensor maps (encoded by the host with their real
 // addresses) into the workspace, where the tensor-core kernels read them.
-__device__ void write_shared_tmaps(uint8_t *ws, const Layout &L, const uint4 (&smap)[3][8]) {
+__device__ void write_shared_tmaps(uint8_t *ws, const Layout &L, const uint4 (&smap)[kSharedMaps][8]) {
     uint4 *o = reinterpret_cast<uint4 *>(ws + L.tmap + (size_t)L.E * kMapsPerExpert * 128);
 #pragma unroll
-    for (int m = 0; m < 3; ++m)
+    for (int m = 0; m < kSharedMaps; ++m)
 #pragma unroll
         for (int j = 0; j < 8; ++j) o[m * 8 + j] = smap[m][j];
     umma::tmap_release();
@@ -179,16 +180,17 @@ __device__ void write_shared_tmaps(uint8_t *ws, const Layout &L, const uint4 (&s
 // callers run it only when an expert's blob pointer changed and keep their
 // hot code short.
 __device__ __noinline__ void write_expert_tmaps(uint8_t *ws, const Layout &L, int e, const uint8_t *blob,
-                                   const uint4 (&tmpl)[4][8], int scale_mask) {
+                                   const uint4 (&tmpl)[kTemplates][8], int scale_mask) {
     const size_t mat = (size_t)L.d * L.ff;
     uint8_t *dst = ws + L.tmap + (size_t)e * kMapsPerExpert * 128;
     const uint8_t *addr[kMapsPerExpert] = {blob,           blob + mat / 2 + mat / 32, blob + mat + mat / 16,
-                                           blob + mat / 2, blob + mat + mat / 32,     blob + mat + mat / 16 + mat / 2};
-    const int which[kMapsPerExpert] = {0, 0, 1, 2, 2, 3};
+                                           blob + mat / 2, blob + mat + mat / 32,     blob + mat + mat / 16 + mat / 2,
+                                           blob + mat + mat / 16, blob + mat + mat / 16 + mat / 2};
+    const int which[kMapsPerExpert] = {0, 0, 1, 2, 2, 3, 4, 5};
 #pragma unroll
     for (int m = 0; m < kMapsPerExpert; ++m) {
         if (which[m] == 2 && !(scale_mask & 1)) continue;
-        if (which[m] == 3 && !(scale_mask & 2)) continue;
+        if ((which[m] == 3 || which[m] == 5) && !(scale_mask & 2)) continue;
         const uint4 *src = tmpl[which[m]];
         uint4 *o = reinterpret_cast<uint4 *>(dst + m * 128);
 #pragma unroll
@@ -223,14 +225,14 @@ struct UmmaParams {
 // x 128 bytes), the A scale boxes (128 rows x 16 bytes per matrix: the scales
 // of this K-tile and its neighbour) and the B scale words (2 x kSfRow words),
 // rounded up to 1024 bytes.
-__host__ __device__ inline int umma_sfa_off(bool gu, int N) { return (gu ? 2 : 1) * kAtile + N * 128; }
-__host__ __device__ inline int umma_sfb_off(bool gu, int N) { return umma_sfa_off(gu, N) + (gu ? 2 : 1) * 2048; }
+__host__ __device__ inline int umma_sfa_off(bool, int N) { return 2 * kAtile + N * 128; }
+__host__ __device__ inline int umma_sfb_off(bool gu, int N) { return umma_sfa_off(gu, N) + 2 * 2048; }
 __host__ __device__ inline int umma_stage_bytes(bool gu, int N) {
     return (umma_sfb_off(gu, N) + 2 * kSfRow * 4 + 1023) & ~1023;
 }
 // TMEM scale columns of one stage, every group aligned: A scales 8 per matrix
 // (2 groups x 4 row blocks), then B scales (group g at +4g, up to 2 columns).
-__host__ __device__ inline int umma_sf_cols(bool gu) { return gu ? 32 : 16; }
+__host__ __device__ inline int umma_sf_cols(bool) { return 32; }
 // Per-call metadata copied into shared memory by every CTA: blob pointer,
 // expert id and per-token routing weight (0 where the token did not select
 // it) of each distinct expert.  Global loads issued while the weight stream
@@ -266,8 +268,11 @@ template <bool GU>
 __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    constexpr int NMAT = GU ? 2 : 1;
-    constexpr int SFC = GU ? 32 : 16;  // TMEM scale columns per stage (8-aligned)
+    // Two 128-row A operands per stage: W_g and W_u (gate/up), or the two
+    // halves of one 256-row box of W_d (down: one copy per 32 KB of weights)
+    constexpr int NMAT = 2;
+    constexpr int RB = GU ? kTileM : 2 * kTileM;  // weight rows per item
+    constexpr int SFC = 32;                       // TMEM scale columns per stage (8-aligned)
     const int nst = p.nst, SB = p.sb;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + nst * SB);  // stage bytes landed (TMA)
     uint64_t *sfr = full + nst;                                        // stage scales in TMEM (4 warps)
@@ -301,7 +306,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         fence_mbar_init();
         *s_abort = 0;
     }
-    constexpr uint32_t kCols = GU ? 512u : 256u;
+    constexpr uint32_t kCols = 512u;
     if (warp == 0) umma::tmem_alloc(tslot, kCols);
     umma::fence_before();
     __syncthreads();
@@ -352,7 +357,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     const int M = GU ? p.ff : p.d;   // routed weight rows
     const int Ks = GU ? p.d : p.ffs; // shared reduction length
     const int nkt = ceil_div(K, kTileK);
-    const int nrb = ceil_div(M, kTileM);
+    const int nrb = ceil_div(M, RB);
     const int nkts = p.ffs > 0 ? ceil_div(Ks, kTileKs) : 0;
     const int nrbs = (GU && p.ffs > 0) ? ceil_div(p.ffs, kTileM) : 0;
     const int S = GU ? nrbs * nkts : 0;               // shared units (gate/up: the first range)
@@ -406,7 +411,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     const uint32_t idesc4 = umma::idesc_mxf4(N), idesc16 = umma::idesc_bf16(N);
     // TMEM columns: accumulators [buf][mat] at (buf*NMAT + mat)*64 (N <= 64), then
     // the scale columns of each stage from sf0
-    const uint32_t sf0 = GU ? 256u : 128u;
+    const uint32_t sf0 = 256u;
 
     // Bounded wait that gives up at once after any role has given up, so a
     // failure ends the kernel in bounded time.
@@ -511,12 +516,12 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 const uint8_t *scmaps = nullptr;  // the A scale planes' maps (TMA scale path)
                 const uint8_t *sfbsrc = nullptr;  // the B scale words of this K-tile
                 if (x.shared) {
-                    maps = smaps + (GU ? 0 : 256);
+                    maps = smaps + (GU ? 0 : 384);
                     bsrc = (GU ? p.ws + L.xbf : p.ws + L.hsb) + (size_t)x.kt * N * 128;
                 } else {
                     const uint8_t *em = p.ws + L.tmap + (size_t)ueid[x.u] * kMapsPerExpert * 128;
-                    maps = em + (GU ? 0 : 256);
-                    scmaps = em + (GU ? 384 : 640);
+                    maps = em + (GU ? 0 : 768);
+                    scmaps = em + (GU ? 384 : 896);
                     bsrc = GU ? p.ws + L.xb + (size_t)x.kt * N * 128
                               : p.ws + L.hb + ((size_t)x.u * nkt + x.kt) * N * 128;
                     sfbsrc = GU ? p.ws + L.xsf + (size_t)x.kt * 2 * kSfRow * 4
@@ -535,13 +540,13 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     }
                     mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * kAtile + N * 128 +
                                                                (sf_dma ? NMAT * 2048 + 2 * kSfRow * 4 : 0)));
-                    umma::tma_load_2d(st, maps, x.kt * 128, x.rb * kTileM, &full[s]);
-                    if (GU) umma::tma_load_2d(st + kAtile, maps + 128, x.kt * 128, x.rb * kTileM, &full[s]);
+                    umma::tma_load_2d(st, maps, x.kt * 128, x.rb * RB, &full[s]);
+                    if (GU) umma::tma_load_2d(st + kAtile, maps + 128, x.kt * 128, x.rb * RB, &full[s]);
                     if (sf_dma) {
                         // 16 scale bytes per row: this K-tile's 8 and its neighbour's
                         uint8_t *sfa = st + umma_sfa_off(GU, N);
-                        umma::tma_load_2d(sfa, scmaps, (x.kt >> 1) * 16, x.rb * kTileM, &full[s]);
-                        if (GU) umma::tma_load_2d(sfa + 2048, scmaps + 128, (x.kt >> 1) * 16, x.rb * kTileM, &full[s]);
+                        umma::tma_load_2d(sfa, scmaps, (x.kt >> 1) * 16, x.rb * RB, &full[s]);
+                        if (GU) umma::tma_load_2d(sfa + 2048, scmaps + 128, (x.kt >> 1) * 16, x.rb * RB, &full[s]);
                         bulk_g2s(st + umma_sfb_off(GU, N), sfbsrc, (uint32_t)(2 * kSfRow * 4), &full[s]);
                     }
                 } else {
@@ -645,7 +650,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                     plane = GU ? (m == 0 ? blob + mat / 2 : blob + mat + mat / 32) : blob + mat + mat / 16 + mat / 2;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const int row = x.rb * kTileM + 32 * j + lane;
+                    const int row = x.rb * RB + (GU ? 0 : m * kTileM) + 32 * j + lane;
                     uint2 v = make_uint2(0u, 0u);
                     if (plane != nullptr && row < M) v = load_sf8(plane + (size_t)row * (K / 32) + x.kt * 8, nks);
                     nanb |= e8m0_nan8(v.x, v.y);
@@ -740,7 +745,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                             if (sk < nks) {
                                 const uint64_t bd = b0 + sk * bstep;
                                 umma::mma_bf16(dcol, a0 + 2 * sk, bd, idesc16, acc);
-                                if (GU) umma::mma_bf16(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, idesc16, acc);
+                                umma::mma_bf16(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, idesc16, acc);
                                 acc = 1u;
                             }
                         }
@@ -754,9 +759,8 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                                 const uint32_t sfb = (sfc + 8 * NMAT + (sk >> 1) * 4) | sfid;
                                 umma::mma_mxf4(dcol, a0 + 2 * sk, bd, id4[sk & 1], acc, (sfc + (sk >> 1) * 4) | sfid,
                                                sfb);
-                                if (GU)
-                                    umma::mma_mxf4(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, id4[sk & 1], acc,
-                                                   (sfc + 8 + (sk >> 1) * 4) | sfid, sfb);
+                                umma::mma_mxf4(dcol + 64, a0 + (kAtile >> 4) + 2 * sk, bd, id4[sk & 1], acc,
+                                               (sfc + 8 + (sk >> 1) * 4) | sfid, sfb);
                                 acc = 1u;
                             }
                         }
@@ -899,16 +903,20 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                         }
                     }
                 } else {
-                    const int row = item * kTileM + rowl;
-                    if (row < p.d) {
 #pragma unroll
-                        for (int t = 0; t < kChunk; ++t) {
-                            if (t < Tc) {
-                                const float y = acc[0][t];
-                                if (p.out_fp32)
-                                    reinterpret_cast<float *>(p.y)[(size_t)t * p.d + row] = y;
-                                else
-                                    reinterpret_cast<__nv_bfloat16 *>(p.y)[(size_t)t * p.d + row] = __float2bfloat16_rn(y);
+                    for (int m = 0; m < NMAT; ++m) {
+                        const int row = item * RB + m * kTileM + rowl;
+                        if (row < p.d) {
+#pragma unroll
+                            for (int t = 0; t < kChunk; ++t) {
+                                if (t < Tc) {
+                                    const float y = acc[m][t];
+                                    if (p.out_fp32)
+                                        reinterpret_cast<float *>(p.y)[(size_t)t * p.d + row] = y;
+                                    else
+                                        reinterpret_cast<__nv_bfloat16 *>(p.y)[(size_t)t * p.d + row] =
+                                            __float2bfloat16_rn(y);
+                                }
                             }
                         }
                     }
