@@ -31,7 +31,9 @@ struct WsHeader {
                            // by the end of the call)
     uint32_t gu_done;      // gate/up items whose activations are written (layer kernel)
     uint32_t exit_cnt;     // CTAs of the layer kernel that have finished (the last resets)
-    uint32_t pad[57];
+    uint32_t disp_cnt;     // 1 once the chunk's dispatch is written (released for the down pass)
+    uint32_t disp_seen;    // down-pass CTAs that have read the dispatch (the last resets both)
+    uint32_t pad[55];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 

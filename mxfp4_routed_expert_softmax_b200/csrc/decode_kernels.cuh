@@ -621,6 +621,9 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
     }
     __syncthreads();
     if (threadIdx.x == 0) {
+        // the down pass reads the dispatch (and the selected experts' maps)
+        // before the gate/up pass completes: publish it
+        if (s_a.dispatch) red_add_release(&hdr->disp_cnt, 1u);
         hdr->router_done = 0u;
         hdr->topk_done = 0u;
     }
@@ -661,6 +664,8 @@ __global__ void single_expert_setup_kernel(const __grid_constant__ SingleParams 
             reinterpret_cast<int8_t *>(p.ws + p.L.uniq_slot)[t] = t < p.Tc ? 0 : -1;
             reinterpret_cast<float *>(p.ws + p.L.wt)[t * p.L.k] = 1.0f;
         }
+        __syncthreads();
+        if (threadIdx.x == 0) red_add_release(&hdr->disp_cnt, 1u);  // the dispatch is written
     }
     build_x_pieces(p.x, p.Tc, p.d, p.ws, p.L, blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5),
                    gridDim.x * (blockDim.x >> 5), false);

@@ -716,6 +716,8 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         up.y = yc;
         up.route_ctas = route_ctas;
         up.strict = (dims->flags & K3MOE_STRICT) != 0;
+        static_assert(sizeof(up.smap_d) == sizeof(smap[3]), "one tensor map");
+        memcpy(up.smap_d, smap[3], sizeof(up.smap_d));
         e = launch_umma<true>(*di, up, st);
         if (e != cudaSuccess) return cuda_fail(e, "gate/up launch");
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);

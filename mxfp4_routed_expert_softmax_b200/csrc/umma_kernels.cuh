@@ -218,6 +218,10 @@ struct UmmaParams {
     uint64_t wait_ns;  // bound of every device wait
     int strict;        // flag E8M0 NaN bytes (0xFF) among the weight scales read
     int inject;        // failure-path tests: 1 = never signal "routing loaded"
+    // down only: the shared expert's W_d tensor map (256-row boxes), encoded by
+    // the host with its real address (read from the launch parameters, so the
+    // pass can stream it before the gate/up pass completes)
+    alignas(64) uint4 smap_d[8];
 };
 
 // One pipeline stage for MMA width N: the A boxes (16 KB per matrix, first,
@@ -265,7 +269,7 @@ __device__ __forceinline__ uint2 load_sf8(const uint8_t *p, int nks) {
 // routing weights (folded into the routed pieces) and the shared expert are
 // combined by the tensor core itself.
 template <bool GU>
-__global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p) {
+__global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(const __grid_constant__ UmmaParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     // Two 128-row A operands per stage: W_g and W_u (gate/up), or the two
@@ -325,23 +329,42 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
             s_blob[i] = gb[i];
             s_eid[i] = ge[i];
         }
-        for (int i = i0; i < U * kChunk; i += nthr) {
-            const int u = i / kChunk, t = i - u * kChunk;
-            float w = 0.f;
-            if (t < Tc && ((gm[u] >> t) & 1u)) w = gw[t * p.k + gs[u * kChunk + t]];
-            s_wu[i] = w;
+        // pairs (expert u, token t < Tc) only (the epilogue reads no others);
+        // the mask and the slot are loaded side by side, then the weight
+        for (int j = i0; j < U * Tc; j += nthr) {
+            const int u = j / Tc, t = j - u * Tc;
+            const uint32_t m = gm[u];
+            const int sl = gs[u * kChunk + t];
+            s_wu[u * kChunk + t] = ((m >> t) & 1u) ? gw[t * p.k + sl] : 0.f;
         }
         return U;
     };
     if constexpr (!GU) {
-        pdl_wait();
+        // The routing comes from the router kernel's dispatch, published by a
+        // release on disp_cnt: read it without waiting for the gate/up pass,
+        // so the producer can start the weight stream at once.  Everything the
+        // gate/up pass writes (h pieces and scales) is read after griddepcontrol
+        // .wait: by the producer after its first weight copies, by every other
+        // thread here.
         pdl_trigger();
-        const int U0 = load_meta(threadIdx.x, kUThreads);
-        if (threadIdx.x == 0) {
-            *s_U = U0;
-            hdr->prep_done = 0u;  // every gate/up CTA has read it (the gate/up grid is complete)
+        if (threadIdx.x == 0 && !spin_geq(&hdr->disp_cnt, 1u, p.wait_ns)) {
+            set_status(hdr, kStTimeout);
+            *s_abort = 1;
         }
         __syncthreads();
+        const int U0 = load_meta(threadIdx.x, kUThreads);
+        if (threadIdx.x == 0) *s_U = U0;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            // the last CTA to have read the dispatch resets the two counters
+            // (the next router kernel starts after this grid completes)
+            const uint32_t old = atom_add_acq_rel(&hdr->disp_seen, 1u);
+            if (old == gridDim.x - 1) {
+                hdr->disp_seen = 0u;
+                hdr->disp_cnt = 0u;
+            }
+        }
+        if (!(warp == 8 && lane == 0)) pdl_wait();
     } else {
         pdl_trigger();
         if (warp == 10) {
@@ -371,11 +394,11 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     struct Range {
         int base, n, G, a, b;
     };
-    auto make_range = [&](int base, int n) {
+    auto make_range = [&](int base, int n, int ctas) {
         Range r;
         r.base = base;
         r.n = n;
-        r.G = min((int)gridDim.x, max(n, 1));
+        r.G = min(ctas, max(n, 1));
         r.a = cta < r.G && n > 0 ? base + (int)(((long long)cta * n) / r.G) : base;
         r.b = cta < r.G && n > 0 ? base + (int)(((long long)(cta + 1) * n) / r.G) : base;
         return r;
@@ -387,8 +410,13 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
     // gate/up: [shared units | routed units]; down: [all units | nothing]
     // (two scalars, not an array: an array indexed by a loop counter would
     // live in local memory)
-    Range rng0 = GU ? make_range(0, S) : make_range(0, nrb * upi);
-    Range rng1 = make_range(0, 0);
+    // The gate/up shared range leaves out the last CTA: CTAs start in index
+    // order as the router kernel's CTAs leave their SMs, and the last one
+    // waits for the router's top-k CTA; it starts its share with the routed
+    // range, which every CTA begins at the same time.
+    const int G = gridDim.x;
+    Range rng0 = GU ? make_range(0, S, G > 1 ? G - 1 : 1) : make_range(0, nrb * upi, G);
+    Range rng1 = make_range(0, 0, G);
     auto rng = [&](int ri) { return ri == 0 ? rng0 : rng1; };
     // gate/up, before the routed range: wait for the routing (lane 0 of the
     // calling warp waits, the warp follows), then size the routed range
@@ -401,7 +429,7 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
         if (warp_wide) ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) return false;
         U = *s_U;
-        rng1 = make_range(S, U * nrb * nkt);
+        rng1 = make_range(S, U * nrb * nkt, G);
         return true;
     };
     const size_t mat = (size_t)p.d * p.ff;
@@ -503,6 +531,34 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 }
                 asm volatile("fence.proxy.async.global;" ::: "memory");  // before the bulk copies read x
             }
+            // The B operand (and its scale words) of a unit: activation pieces
+            // written by the previous kernel of the layer.
+            auto b_src = [&](const Unit &x, const uint8_t *&bsrc, const uint8_t *&sfbsrc) {
+                if (x.shared) {
+                    bsrc = (GU ? p.ws + L.xbf : p.ws + L.hsb) + (size_t)x.kt * N * 128;
+                    sfbsrc = nullptr;
+                } else {
+                    bsrc = GU ? p.ws + L.xb + (size_t)x.kt * N * 128
+                              : p.ws + L.hb + ((size_t)x.u * nkt + x.kt) * N * 128;
+                    sfbsrc = GU ? p.ws + L.xsf + (size_t)x.kt * 2 * kSfRow * 4
+                                : p.ws + L.hsf + ((size_t)x.u * nkt + x.kt) * 2 * kSfRow * 4;
+                }
+            };
+            auto sf_dma_of = [&](const Unit &x) {
+                return p.sf_tma && !x.shared && ublob[x.u] != nullptr;
+            };
+            // B copies of stage s (after the A copies and the stage's expect_tx)
+            auto issue_b = [&](const Unit &x, int s) {
+                uint8_t *st = smem + s * SB;
+                const uint8_t *bsrc, *sfbsrc;
+                b_src(x, bsrc, sfbsrc);
+                if (sf_dma_of(x)) bulk_g2s(st + umma_sfb_off(GU, N), sfbsrc, (uint32_t)(2 * kSfRow * 4), &full[s]);
+                bulk_g2s(st + NMAT * kAtile, bsrc, (uint32_t)(N * 128), &full[s]);
+            };
+            // down: the first two stages' weight copies go out before the wait
+            // for the gate/up pass (weights need nothing from it), their B copies
+            // after (more stages in flight there slow that pass's last writes)
+            const int npre = GU ? 0 : min(min(nst, 2), rng0.b - rng0.a);
             for (int ri = 0; ri < 2 && !*s_abort; ++ri) {
             if (ri == 1 && (!GU || !routed_range(false))) break;
             const Range rg = rng(ri);
@@ -512,25 +568,24 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                 uint8_t *st = smem + s * SB;
                 const uint8_t *blob = x.shared ? nullptr : ublob[x.u];
                 const uint8_t *maps = nullptr;
-                const uint8_t *bsrc;
                 const uint8_t *scmaps = nullptr;  // the A scale planes' maps (TMA scale path)
-                const uint8_t *sfbsrc = nullptr;  // the B scale words of this K-tile
+                bool ws_map = true;               // the map lives in the workspace (acquire it)
                 if (x.shared) {
-                    maps = smaps + (GU ? 0 : 384);
-                    bsrc = (GU ? p.ws + L.xbf : p.ws + L.hsb) + (size_t)x.kt * N * 128;
+                    if (GU) {
+                        maps = smaps;
+                    } else {
+                        maps = reinterpret_cast<const uint8_t *>(p.smap_d);
+                        ws_map = false;
+                    }
                 } else {
                     const uint8_t *em = p.ws + L.tmap + (size_t)ueid[x.u] * kMapsPerExpert * 128;
                     maps = em + (GU ? 0 : 768);
                     scmaps = em + (GU ? 384 : 896);
-                    bsrc = GU ? p.ws + L.xb + (size_t)x.kt * N * 128
-                              : p.ws + L.hb + ((size_t)x.u * nkt + x.kt) * N * 128;
-                    sfbsrc = GU ? p.ws + L.xsf + (size_t)x.kt * 2 * kSfRow * 4
-                                : p.ws + L.hsf + ((size_t)x.u * nkt + x.kt) * 2 * kSfRow * 4;
                 }
-                const bool sf_dma = p.sf_tma && !x.shared && blob != nullptr;
+                const bool sf_dma = sf_dma_of(x);
                 if (x.shared || blob != nullptr) {
                     if (x.u != last_u) {
-                        umma::tmap_acquire(maps);
+                        if (ws_map) umma::tmap_acquire(maps);
                         if (GU) umma::tmap_acquire(maps + 128);
                         if (sf_dma) {
                             umma::tmap_acquire(scmaps);
@@ -547,17 +602,29 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(UmmaParams p)
                         uint8_t *sfa = st + umma_sfa_off(GU, N);
                         umma::tma_load_2d(sfa, scmaps, (x.kt >> 1) * 16, x.rb * RB, &full[s]);
                         if (GU) umma::tma_load_2d(sfa + 2048, scmaps + 128, (x.kt >> 1) * 16, x.rb * RB, &full[s]);
-                        bulk_g2s(st + umma_sfb_off(GU, N), sfbsrc, (uint32_t)(2 * kSfRow * 4), &full[s]);
                     }
                 } else {
                     mbar_arrive_expect_tx(&full[s], (uint32_t)(N * 128));
                 }
-                bulk_g2s(st + NMAT * kAtile, bsrc, (uint32_t)(N * 128), &full[s]);
+                if (it >= npre) issue_b(x, s);
+                if (it + 1 == npre || (npre > 0 && it + 1 < npre && unit + 1 == rg.b)) {
+                    // the pre-issued stages: now wait for the gate/up pass and
+                    // send their B copies
+                    pdl_wait();
+                    hdr->prep_done = 0u;  // every gate/up CTA has read it (that grid is complete)
+                    asm volatile("fence.proxy.async.global;" ::: "memory");  // before the bulk copies read h
+                    Unit y = decode(rg.a);
+                    for (int q = 0; q <= it; ++q, y = advance(y, rg.a + q, rg.b)) issue_b(y, q);
+                }
                 if (++s == nst) {
                     s = 0;
                     ph ^= 1u;
                 }
             }
+            }
+            if (!GU && npre == 0) {
+                pdl_wait();
+                hdr->prep_done = 0u;
             }
             if (*s_abort) {
                 // a wait gave up somewhere: wait (bounded) for the last copy
