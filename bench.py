@@ -448,13 +448,18 @@ def main():
 def measure_model(cfg, W, k3, args, flush_l2, stream, world, n_layers):
     """One decode token through n_layers K3 MoE layers in a row (the steps of
     a pre-norm block: RMSNorm, the layer, the residual add; k3moe_layer_residual
-    with the residual stream updated in place), every layer with its own router,
+    with the residual stream updated in place, one launch per layer), every
+    layer with its own router,
     shared expert and norm weights and its own permutation of the resident
     experts, captured in a CUDA graph.  L2 is flushed before each token, not
-    between layers: consecutive layers stream different weights."""
+    between layers: consecutive layers stream different weights.  The layers
+    share one workspace, so its tensor maps (cached per expert id) change with
+    every layer: the one-launch decode kernel (K3MOE_ONE_LAUNCH) rewrites them
+    in its set-up, off the routing path, where the three-launch path rewrites
+    the selected experts' maps at dispatch, on it."""
     import torch
     E, d = cfg.E, cfg.d
-    dims = k3.make_dims(cfg.d, cfg.ff, cfg.E, cfg.k, cfg.ff_shared, 0)
+    dims = k3.make_dims(cfg.d, cfg.ff, cfg.E, cfg.k, cfg.ff_shared, k3.K3MOE_ONE_LAUNCH)
     ws = k3.new_workspace(dims, 1)
     layers = []
     for l in range(n_layers):
@@ -511,7 +516,7 @@ def measure_model(cfg, W, k3, args, flush_l2, stream, world, n_layers):
            "value": round(world * 1000.0 / ms, 2), "unit": "tokens/s (all layers)",
            "us_per_layer": round(1000.0 * ms / n_layers, 2), "hbm_gbs": round(gbs, 1),
            "hbm_frac": round(gbs / peak, 4), "cuda_graph": graph is not None,
-           "gpu_launches_per_token": n_layers}
+           "gpu_launches_per_token": n_layers, "decode": "one launch (K3MOE_ONE_LAUNCH)"}
     if graph is None:
         out["cuda_graph_error"] = capture_error
     del graph, layers

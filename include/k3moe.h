@@ -208,13 +208,14 @@ k3moe_status k3moe_layer(const void *x, int32_t T, const float *w_router, const 
  *   h_out  = h + layer(x)                                      rounded once
  * h: bf16 [T][d] (the residual stream); norm_w: bf16 [d], 16-byte aligned;
  * eps >= 0; h_out: [T][d] bf16 (or fp32 with K3MOE_OUT_FP32), and may be h
- * itself (updated in place).  The normalisation runs in fp32 inside the
- * kernels that read x (1/rms as 1/sqrtf of the fp32 mean of squares, each
- * element (h * r) * w rounded to bf16).  Other arguments as for k3moe_layer
- * (no routing copies).  Up to 8 tokens per pass this needs the one-launch
- * decode kernel's shape limits (K3MOE_ERR_UNSUPPORTED_SHAPE otherwise); with
- * a workspace sized for more tokens the grouped path normalises each pass
- * first and adds h in its final sum.
+ * itself (updated in place).  The normalisation runs in fp32 (1/rms as
+ * 1/sqrtf of the fp32 mean of squares, each element (h * r) * w rounded to
+ * bf16): up to 8 tokens per pass a norm launch writes x into the workspace
+ * before the decode launches and the down pass adds h before its rounding
+ * (with K3MOE_ONE_LAUNCH both are fused into the one-launch kernel, within its
+ * shape limits); with a workspace sized for more tokens the grouped path
+ * normalises each pass first and adds h in its final sum.  Other arguments as
+ * for k3moe_layer (no routing copies).
  */
 k3moe_status k3moe_layer_residual(const void *h, int32_t T, const void *norm_w, float eps,
                                   const float *w_router, const float *bias,

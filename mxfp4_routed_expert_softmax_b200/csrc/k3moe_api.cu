@@ -628,7 +628,6 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         return K3MOE_OK;
     }
 
-    if (norm_w && layer_stages(*di, dims, T < kChunk ? T : kChunk) == 0) return K3MOE_ERR_UNSUPPORTED_SHAPE;
     for (int c0 = 0; c0 < T; c0 += kChunk) {
         const int Tc = (T - c0) < kChunk ? (T - c0) : kChunk;
         const uint16_t *xc;
@@ -668,7 +667,7 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         EventHook none;
         EventHook &hk = hook ? *hook : none;
         if ((e = hk.record(st)) != cudaSuccess) return cuda_fail(e);
-        const int lst = (one_launch(dims) || norm_w || layer_mode != kLayerFull) ? layer_stages(*di, dims, Tc) : 0;
+        const int lst = (one_launch(dims) || layer_mode != kLayerFull) ? layer_stages(*di, dims, Tc) : 0;
         if (layer_mode != kLayerFull && lst == 0) return K3MOE_ERR_UNSUPPORTED_SHAPE;
         if (lst > 0) {
             // the whole pass in one launch
@@ -699,6 +698,14 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
             continue;
         }
         hk.kernels = 3;
+        if (norm_w) {
+            // pre-norm: the chunk's normalised input into the workspace (the
+            // residual stream xc stays for the residual add at the end)
+            const PfNormParams np{xc, norm_w, eps, Tc, d, reinterpret_cast<uint16_t *>(wsb + L.xn)};
+            e = launch(pf_rmsnorm_kernel, dim3(ceil_div(Tc, 8)), dim3(256), 0, st, false, np);
+            if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
+            rp.x = reinterpret_cast<const uint16_t *>(wsb + L.xn);
+        }
         int route_ctas = 0;
         e = launch_route(*di, rp, st, &route_ctas);
         if (e != cudaSuccess) return cuda_fail(e, "router launch");
@@ -714,6 +721,7 @@ k3moe_status layer_impl(const void *x, int32_t T, const float *w_router, const f
         up.L = L;
         up.out_fp32 = out32;
         up.y = yc;
+        up.resid = norm_w ? xc : nullptr;
         up.route_ctas = route_ctas;
         up.strict = (dims->flags & K3MOE_STRICT) != 0;
         static_assert(sizeof(up.smap_d) == sizeof(smap[3]), "one tensor map");

@@ -34,6 +34,7 @@ struct Layout {
     size_t uniq_slot;  // i8  [kChunk*k][kChunk] slot j of token t for it, -1 if none
     size_t part;       // f32 [2][E][P][4] partial sums of the P parts of each router row
     size_t cnt;        // u32 [2][E] parts summed per router row (back to 0 after each row)
+    size_t xn;         // bf16 [kChunk][d] the normalised input of pre-norm calls
     size_t tmap;       // 128-byte tensor maps [E][6]: W_g, W_u, W_d nibble planes and their
                        // scale planes, of each expert; then the shared expert's W_g, W_u,
                        // W_d (bf16) at [E*6 ..]
@@ -93,6 +94,8 @@ __host__ __device__ inline Layout make_layout(int d, int ff, int E, int k, int f
     o = align256(o + (size_t)2 * E * (d / router_part_len(d)) * 4 * 4);
     L.cnt = o;
     o = align256(o + (size_t)2 * E * 4);
+    L.xn = o;
+    o = align256(o + C * d * 2);
     const int umax = E < kChunk * k ? E : kChunk * k;
     const int nkt_d = ceil_div(d, kTileK), nkt_ff = ceil_div(ff, kTileK);
     L.umax = umax;

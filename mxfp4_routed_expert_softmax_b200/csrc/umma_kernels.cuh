@@ -212,6 +212,7 @@ struct UmmaParams {
     // down only
     int out_fp32;     // y in fp32 (else bf16, rounded once)
     void *y;          // [Tc][d] of this chunk
+    const uint16_t *resid;  // bf16 [Tc][d] added before the rounding (pre-norm calls), or null
     // gate/up: router-kernel CTAs that announce their x pieces and tensor maps
     // in the header's prep_done (0: nothing to wait for)
     int route_ctas;
@@ -977,7 +978,8 @@ __global__ void __launch_bounds__(kUThreads, 1) umma_expert_kernel(const __grid_
 #pragma unroll
                             for (int t = 0; t < kChunk; ++t) {
                                 if (t < Tc) {
-                                    const float y = acc[m][t];
+                                    float y = acc[m][t];
+                                    if (p.resid) y += __uint_as_float((uint32_t)p.resid[(size_t)t * p.d + row] << 16);
                                     if (p.out_fp32)
                                         reinterpret_cast<float *>(p.y)[(size_t)t * p.d + row] = y;
                                     else

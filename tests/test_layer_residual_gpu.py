@@ -1,5 +1,6 @@
 """k3moe_layer_residual: RMSNorm of the residual stream before the layer and
-the residual add after it, fused into the kernels, against the oracle's
+the residual add after it (a norm launch and the down pass's epilogue, or fused
+into the one-launch kernel), against the oracle's
 statement of the block: h_out = h + layer(RNE_bf16(RMSNorm(h))).  Tokens whose
 top-k is a near tie under the oracle's logits (relative k / k+1 gap <= 1e-5)
 are left out, since the kernel's fp32 normalisation may round an element of
@@ -50,16 +51,19 @@ def oracle_block(orc, cfg, W, h, bias, g, tokens):
     return orc.residual_add(h[tokens], y), np.array(decisive)
 
 
-@pytest.mark.parametrize("cfg,T,ws_tokens", [
-    (k3gen.CONFIGS["tiny"], 4, 4), (SMALL, 8, 8), (SMALL, 13, 8),
-    (k3gen.CONFIGS["k3_decode"], 1, 1), (k3gen.CONFIGS["k3_decode_t8"], 8, 8),
-    (k3gen.CONFIGS["tiny"], 64, 64), (SMALL, 40, 40)])
-def test_layer_residual_matches_oracle(orc, cfg, T, ws_tokens):
+# one_launch: the decode passes as one cooperative launch (K3MOE_ONE_LAUNCH)
+# instead of the default norm + router + gate/up + down launches
+@pytest.mark.parametrize("cfg,T,ws_tokens,one_launch", [
+    (k3gen.CONFIGS["tiny"], 4, 4, False), (SMALL, 8, 8, False), (SMALL, 13, 8, False),
+    (k3gen.CONFIGS["k3_decode"], 1, 1, False), (k3gen.CONFIGS["k3_decode_t8"], 8, 8, False),
+    (k3gen.CONFIGS["tiny"], 64, 64, False), (SMALL, 40, 40, False),
+    (SMALL, 13, 8, True), (k3gen.CONFIGS["k3_decode"], 1, 1, True), (k3gen.CONFIGS["k3_decode_t8"], 8, 8, True)])
+def test_layer_residual_matches_oracle(orc, cfg, T, ws_tokens, one_launch):
     W = kdev.weights(cfg)
     inp = kdev.DeviceInputs(cfg, T=T)
     g = k3gen.norm_weights(cfg)
     gd = torch.from_numpy(g.view(np.int16)).cuda()
-    dims = dims_of(cfg, m.K3MOE_OUT_FP32)
+    dims = dims_of(cfg, m.K3MOE_OUT_FP32 | (m.K3MOE_ONE_LAUNCH if one_launch else 0))
     ws = m.new_workspace(dims, ws_tokens)
     out = torch.empty((T, cfg.d), dtype=torch.float32, device="cuda")
     m.check(m.k3moe_layer_residual(inp.x, T, gd, EPS, W.w_router, inp.bias, W.blob_ptrs, *W.shared, dims,
@@ -74,13 +78,14 @@ def test_layer_residual_matches_oracle(orc, cfg, T, ws_tokens):
     assert err.max() <= G1_TOL, (err.max(), err)
 
 
-@pytest.mark.parametrize("cfg,T", [(k3gen.CONFIGS["k3_decode_t8"], 8), (SMALL, 40)])
-def test_layer_residual_in_place(cfg, T):
+@pytest.mark.parametrize("cfg,T,one_launch", [(k3gen.CONFIGS["k3_decode_t8"], 8, False), (SMALL, 40, False),
+                                               (k3gen.CONFIGS["k3_decode"], 1, True)])
+def test_layer_residual_in_place(cfg, T, one_launch):
     """h_out may be h: the same bf16 bytes as a separate output buffer."""
     W = kdev.weights(cfg)
     inp = kdev.DeviceInputs(cfg, T=T)
     gd = torch.from_numpy(k3gen.norm_weights(cfg).view(np.int16)).cuda()
-    dims = dims_of(cfg, 0)
+    dims = dims_of(cfg, m.K3MOE_ONE_LAUNCH if one_launch else 0)
     ws = m.new_workspace(dims, T)
     out = torch.empty((T, cfg.d), dtype=torch.int16, device="cuda")
     m.check(m.k3moe_layer_residual(inp.x, T, gd, EPS, W.w_router, inp.bias, W.blob_ptrs, *W.shared, dims,
