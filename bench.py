@@ -212,11 +212,32 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def cpu_oracle_time(cfg, seconds=10.0):
+def omp_threads(n=None):
+    """The OpenMP thread count the oracle's parallel regions use (the process's
+    libgomp, which the oracle links); with n, set it first."""
+    import ctypes
+    gomp = ctypes.CDLL("libgomp.so.1")
+    if n is not None:
+        gomp.omp_set_num_threads(int(n))
+    return int(gomp.omp_get_max_threads())
+
+
+def cpu_oracle_time(cfg, seconds=10.0, threads=None):
     """Time the fp64 oracle (as it stands) on whole tokens of the workload
-    until ~`seconds` of work; -> (tokens/s, threads, n_tokens)."""
+    until ~`seconds` of work (at least one token), on `threads` OpenMP threads
+    (None: as configured); -> (tokens/s, threads used, n_tokens, seconds)."""
     import oracle
     orc = oracle.oracle()
+    before = omp_threads()
+    if threads is not None:
+        omp_threads(threads)
+    try:
+        return _cpu_oracle_time(orc, cfg, seconds)
+    finally:
+        omp_threads(before)
+
+
+def _cpu_oracle_time(orc, cfg, seconds):
     # tokens beyond the workload's own T are further draws of the same
     # distribution (stream 0), so a small-T workload still gives a sample of
     # ~`seconds` of oracle work
@@ -225,7 +246,7 @@ def cpu_oracle_time(cfg, seconds=10.0):
     b = k3gen.bias(cfg)
     sh = k3gen.shared(cfg) if cfg.ff_shared else None
     cache = {}
-    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    threads = omp_threads()
     done = 0
     t_total = 0.0
     while t_total < seconds and done < x.shape[0]:
@@ -279,7 +300,7 @@ def run_reference(args, cfg, rank, world):
     w = k3gen.router(cfg)
     b = k3gen.bias(cfg)
     sh = k3gen.shared(cfg) if cfg.ff_shared else None
-    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    threads = omp_threads()
     cache = {}
     t_total = 0.0
     for i in range(n):
@@ -404,8 +425,11 @@ def main():
         tok_s, threads, n, t = cpu_oracle_time(cfg, seconds=10.0)
         cpu = {"value": tok_s, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"{n} token(s) of the workload ({t:.1f} s), fp64 scalar C oracle, "
-                         f"OpenMP over output rows",
+                         f"OpenMP over output rows ({threads} threads: the process's OpenMP setting)",
                "cpu_model": cpu_model()}
+        tok_1, _, n1, t1 = cpu_oracle_time(cfg, seconds=5.0, threads=1)
+        cpu["single_thread"] = {"value": tok_1, "unit": UNIT, "cores": 1,
+                                "sample": f"{n1} token(s) of the workload ({t1:.1f} s) on one OpenMP thread"}
         for name, r in others.items():
             tok_s, threads, n, t = cpu_oracle_time(k3gen.CONFIGS[name], seconds=4.0)
             r["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "cores": threads, "kind": "oracle",

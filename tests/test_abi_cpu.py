@@ -68,6 +68,13 @@ def test_workspace_grows_with_the_grouped_prefill_region(m):
     assert m.k3moe_workspace_size(d, 8192) == m.k3moe_workspace_size(d, 100000)
 
 
+def test_k3_decode_scratch_fits_the_built_in_buffer(m):
+    """k3moe_layer_noalloc serves shapes whose decode scratch fits its 16 MiB
+    buffer: the K3 shape must (with and without the shared expert)."""
+    for ffs in (1536, 0):
+        assert 0 < m.k3moe_workspace_size(m.make_dims(7168, 1536, 896, 16, ffs), 8) <= 16 << 20
+
+
 BIG = 1 << 30
 A16 = 0x10000  # a fake 16-byte aligned address: never dereferenced, calls fail validation first
 
