@@ -72,7 +72,7 @@ def test_layer_residual_matches_oracle(orc, cfg, T, ws_tokens, one_launch):
     m.check(m.k3moe_device_status(ws), "device status")
     tokens = sample_tokens(T, 16)
     ref, decisive = oracle_block(orc, cfg, W, inp.x_host, inp.bias_host, g, tokens)
-    assert decisive.sum() >= len(tokens) - 1, "too many near ties to judge"
+    assert decisive.sum() >= len(tokens) - 1, "too many near ties to compare"
     got = out.cpu().numpy()[tokens]
     err = g1_error(got[decisive], ref[decisive])
     assert err.max() <= G1_TOL, (err.max(), err)
