@@ -22,10 +22,12 @@ int main(int argc, char **argv) {
     const Layout L = make_layout(d, ff, E, k, ffs);
     printf("{\"decode\": {");
     const size_t dv[] = {L.hdr, L.logits, L.idx, L.wt, L.uniq_blob, L.uniq_eid, L.uniq_mask, L.uniq_slot, L.part,
-                         L.cnt, L.tmap, L.tcache, L.xb, L.xsf, L.hb, L.hsf, L.xbf, L.hsb, L.spart, L.icnt, L.total};
+                         L.cnt, L.xn, L.tmap, L.tcache, L.xb, L.xsf, L.hb, L.hsf, L.xbf, L.hsb, L.spart, L.icnt,
+                         L.total};
     const char *dn[] = {"hdr", "logits", "idx", "wt", "uniq_blob", "uniq_eid", "uniq_mask", "uniq_slot", "part",
-                        "cnt", "tmap", "tcache", "xb", "xsf", "hb", "hsf", "xbf", "hsb", "spart", "icnt", "total"};
-    for (int i = 0; i < 21; ++i) printf("%s\"%s\": %zu", i ? ", " : "", dn[i], dv[i]);
+                        "cnt", "xn", "tmap", "tcache", "xb", "xsf", "hb", "hsf", "xbf", "hsb", "spart", "icnt", "total"};
+    for (int i = 0; i < 22; ++i) printf("%s\"%s\": %zu", i ? ", " : "", dn[i], dv[i]);
+    printf(", \"router_part_len\": %d", router_part_len(d));
     printf("}");
     if (Tp > 0) {
         const PLayout P = make_playout(L.total, d, ff, E, k, ffs, Tp);
@@ -67,7 +69,8 @@ SHAPES = [(7168, 1536, 896, 16, 1536), (256, 128, 32, 4, 128), (512, 256, 64, 8,
 @pytest.mark.parametrize("Tp", [0, 9, 512, 8192])
 def test_regions_are_aligned_ordered_and_disjoint(driver, shape, Tp):
     lay = layout(driver, shape, Tp)
-    dec = lay["decode"]
+    dec = dict(lay["decode"])
+    ls = dec.pop("router_part_len")
     starts = [v for k, v in dec.items() if k != "total"]
     assert starts == sorted(starts) and len(set(starts)) == len(starts)
     assert all(v % 256 == 0 for v in dec.values())
@@ -83,6 +86,24 @@ def test_regions_are_aligned_ordered_and_disjoint(driver, shape, Tp):
         assert pf["total"] - pf["o"] >= Tp * (k + 1) * d * 4
         # a group per 32 pairs, plus one partial group per expert at most
         assert pf["ngr"] >= Tp * k // 32 and pf["ngs"] == (-(-Tp // 32) if ffs else 0)
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_decode_regions_hold_their_contents(driver, shape):
+    """The regions whose size depends on the shape: the router's part sums
+    [2][E][d/Ls][4] fp32 (Ls = 512 where d allows it), the normalised input
+    [8][d] bf16, and 8 tensor maps per expert plus 4 for the shared expert."""
+    d, ff, E, k, ffs = shape
+    dec = dict(layout(driver, shape, 0)["decode"])
+    ls = dec.pop("router_part_len")
+    assert ls in (512, 256, 128, 64) and d % ls == 0
+    assert ls == max(x for x in (512, 256, 128, 64) if d % x == 0)
+    names = [n for n in dec if n != "total"] + ["total"]
+    size = {n: dec[names[i + 1]] - dec[n] for i, n in enumerate(names[:-1])}
+    assert size["part"] >= 2 * E * (d // ls) * 4 * 4
+    assert size["cnt"] >= 2 * E * 4
+    assert size["xn"] >= 8 * d * 2
+    assert size["tmap"] >= (E * 8 + 4) * 128
 
 
 @pytest.mark.parametrize("shape", SHAPES)
