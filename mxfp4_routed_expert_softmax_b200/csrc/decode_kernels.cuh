@@ -3,8 +3,8 @@
 // parts (a row's parts are summed by the last one to finish, in part order);
 // one CTA per token waits for every router row, then runs the softmax over
 // all experts and the token's top-k; CTA 0 dispatches (distinct experts, their
-// slots and blob pointers).  The same CTAs first build the activation pieces
-// the tensor-core gate/up pass reads.  Layer structure: the tutorial page's
+// slots and blob pointers).  The streaming CTAs then build the activation
+// pieces the tensor-core gate/up pass reads.  Layer structure: the tutorial page's
 // section 2.4 moe_forward (route, per selected expert FFN, weighted combine);
 // the expert FFNs themselves are in umma_kernels.cuh.
 #pragma once
