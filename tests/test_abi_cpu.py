@@ -131,6 +131,26 @@ def test_route_and_expert_ffn_reject(m):
                                        A16, A16 * 16, BIG, None) == 1
 
 
+def test_layer_residual_rejects(m):
+    """The pre-norm entry checks its norm weights and eps, then everything
+    k3moe_layer checks, before any launch."""
+    d = m.make_dims(256, 128, 32, 4, 128)
+    ws = A16 * 16
+
+    def call(h=A16, g=A16, eps=1e-6, wsb=BIG, dims=d):
+        return m.lib.k3moe_layer_residual(h, 4, g, eps, A16, None, A16, A16, A16, A16, ctypes.byref(dims), A16,
+                                          ws, wsb, None)
+
+    assert call(g=None) == 1
+    assert call(g=A16 + 8) == 1
+    assert call(eps=-1.0) == 1
+    assert call(eps=float("nan")) == 1
+    assert call(eps=float("inf")) == 1
+    assert call(h=None) == 1
+    assert call(wsb=16) == 3
+    assert call(dims=m.make_dims(100, 128, 32, 4, 128)) == 2
+
+
 def test_status_strings(m):
     for s in range(7):
         assert m.k3moe_status_string(s) not in ("", "unknown status")
